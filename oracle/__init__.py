@@ -1,0 +1,213 @@
+"""fp64 CPU oracle for the block-diffusion bidirectional Mamba-2 scan.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py`` may import this package; the product path
+(``bidirectional_mamba_state_b200``) never does, and this package never imports
+the product.  The arithmetic lives in ``bdscan_oracle.c`` (plain sequential
+recurrence in double precision, see that file's header for the equations it
+follows); this module only marshals arrays through ctypes.
+
+Inputs are dictionaries with keys ``x, dt, B, C, A, D`` and optionally ``z``
+(torch tensors or numpy arrays, any dtype, any device).  They are widened
+exactly to float64 on the host before the call, so the oracle sees the same
+rounded values the device consumed.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "bdscan_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libbdscan_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+class _Shape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in
+                ("batch", "seqlen", "nheads", "headdim", "dstate", "ngroups", "block_len")]
+
+
+_dp = ctypes.POINTER(ctypes.c_double)
+
+
+class _Dir(ctypes.Structure):
+    _fields_ = [("x", _dp), ("dt", _dp), ("Bm", _dp), ("Cm", _dp), ("z", _dp),
+                ("A", _dp), ("D", _dp)]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle shared library with gcc (-O2, OpenMP).  Returns its path."""
+    if force or not os.path.exists(_LIB_PATH) or (
+            os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+               "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _open(path: str):
+    lib = ctypes.CDLL(path)
+    for name in ("oracle_prefix", "oracle_block_step", "oracle_allblock"):
+        getattr(lib, name).restype = ctypes.c_int
+    lib.oracle_max_threads.restype = ctypes.c_int
+    lib.oracle_set_threads.argtypes = [ctypes.c_int]
+    return lib
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            _lib = _open(_LIB_PATH)
+    return _lib
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def set_threads(n: int) -> None:
+    _load().oracle_set_threads(int(n))
+
+
+def _f64(t) -> np.ndarray:
+    """Exact widening of a torch tensor / numpy array to a C-contiguous float64 array."""
+    if t is None:
+        return None
+    if hasattr(t, "detach"):  # torch tensor
+        t = t.detach().to("cpu")
+        import torch
+        t = t.to(torch.float64).contiguous().numpy()
+    return np.ascontiguousarray(np.asarray(t, dtype=np.float64))
+
+
+def _ptr(a):
+    return a.ctypes.data_as(_dp) if a is not None else None
+
+
+class _Marshal:
+    """Keeps the float64 copies alive for the duration of one oracle call."""
+
+    def __init__(self):
+        self.keep = []
+
+    def arr(self, t):
+        a = _f64(t)
+        if a is not None:
+            self.keep.append(a)
+        return a
+
+    def dir(self, d):
+        if d is None:
+            return None
+        fields = {}
+        for key, cname in (("x", "x"), ("dt", "dt"), ("B", "Bm"), ("C", "Cm"), ("z", "z"),
+                           ("A", "A"), ("D", "D")):
+            fields[cname] = _ptr(self.arr(d.get(key)))
+        return ctypes.pointer(_Dir(**fields))
+
+
+def _shape(s: dict) -> _Shape:
+    return _Shape(*(int(s[k]) for k in
+                    ("batch", "seqlen", "nheads", "headdim", "dstate", "ngroups", "block_len")))
+
+
+def _check(rc: int, name: str):
+    if rc != 0:
+        raise ValueError(f"{name}: oracle returned {rc}")
+
+
+def prefix(shape: dict, fwd: dict, rev: dict | None = None, h0=None,
+           want_states: bool = True, want_final: bool = True, lib=None):
+    """Forward scan of the clean stream from h0 (eq. (10) boundary states), plus a
+    block-local reverse scan of every block when ``rev`` is given (eq. (12)),
+    summed (eq. (13)).  Returns (y, states or None, final or None) as float64."""
+    lib = lib or _load()
+    B, L, H, P, N, T = (int(shape[k]) for k in
+                        ("batch", "seqlen", "nheads", "headdim", "dstate", "block_len"))
+    K = L // T
+    m = _Marshal()
+    y = np.zeros((B, L, H, P))
+    st = np.zeros((B, K, H, P, N)) if want_states else None
+    fin = np.zeros((B, H, P, N)) if want_final else None
+    rc = lib.oracle_prefix(ctypes.byref(_shape(shape)), m.dir(fwd), m.dir(rev),
+                           _ptr(m.arr(h0)), _ptr(y), _ptr(st), _ptr(fin))
+    _check(rc, "oracle_prefix")
+    return y, st, fin
+
+
+def block_step(shape: dict, fwd: dict, rev: dict | None, state_in, want_state_out: bool = False,
+               lib=None):
+    """One denoising step on a single block from the cached state (eq. (11)-(13)).
+    ``shape['seqlen']`` must equal ``shape['block_len']``.  Returns (y, state_out or None)."""
+    lib = lib or _load()
+    B, L, H, P, N = (int(shape[k]) for k in ("batch", "seqlen", "nheads", "headdim", "dstate"))
+    m = _Marshal()
+    y = np.zeros((B, L, H, P))
+    so = np.zeros((B, H, P, N)) if want_state_out else None
+    rc = lib.oracle_block_step(ctypes.byref(_shape(shape)), m.dir(fwd), m.dir(rev),
+                               _ptr(m.arr(state_in)), _ptr(y), _ptr(so))
+    _check(rc, "oracle_block_step")
+    return y, so
+
+
+def allblock(shape: dict, clean_fwd: dict, clean_rev: dict | None, noisy_fwd: dict,
+             noisy_rev: dict | None, h0=None, want_clean: bool = True, lib=None):
+    """All-block pass (eq. (14)): clean stream as in ``prefix``; every noisy block k
+    continues from the clean boundary state before it.  Returns
+    (y_clean or None, y_noisy, states)."""
+    lib = lib or _load()
+    B, L, H, P, N, T = (int(shape[k]) for k in
+                        ("batch", "seqlen", "nheads", "headdim", "dstate", "block_len"))
+    K = L // T
+    m = _Marshal()
+    yc = np.zeros((B, L, H, P)) if want_clean else None
+    yn = np.zeros((B, L, H, P))
+    st = np.zeros((B, K, H, P, N))
+    rc = lib.oracle_allblock(ctypes.byref(_shape(shape)), m.dir(clean_fwd), m.dir(clean_rev),
+                             m.dir(noisy_fwd), m.dir(noisy_rev), _ptr(m.arr(h0)),
+                             _ptr(yc), _ptr(yn), _ptr(st))
+    _check(rc, "oracle_allblock")
+    return yc, yn, st
+
+
+class Variant:
+    """The same API bound to another build of the oracle source (used by the
+    tests that plant a mistake in a copy of the oracle and check that the pins
+    catch it)."""
+
+    def __init__(self, lib_path: str):
+        self.lib = _open(lib_path)
+
+    def prefix(self, *a, **k):
+        return prefix(*a, lib=self.lib, **k)
+
+    def block_step(self, *a, **k):
+        return block_step(*a, lib=self.lib, **k)
+
+    def allblock(self, *a, **k):
+        return allblock(*a, lib=self.lib, **k)
+
+
+def compile_variant(src_text: str, out_path: str) -> str:
+    """Compile an edited copy of the oracle source to ``out_path``."""
+    src = out_path + ".c"
+    with open(src, "w") as f:
+        f.write(src_text)
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-fno-fast-math",
+                    "-ffp-contract=off", src, "-o", out_path, "-lm"], check=True)
+    return out_path
+
+
+def source_text() -> str:
+    with open(_SRC) as f:
+        return f.read()
