@@ -1,0 +1,249 @@
+"""Python binding of libbdscan (ctypes; argument marshalling only).
+
+The functions named ``bdscan_*`` mirror the C ABI in ``include/bdscan.h`` one to
+one and take raw pointers / ctypes structs.  ``prefix``, ``block_step`` and
+``allblock`` are the torch-facing conveniences: they check devices, dtypes and
+contiguity, allocate the outputs and the workspace with torch, and call the C
+ABI on the current torch CUDA stream.  Every step of the scan runs in the
+library's CUDA kernels; there is no CPU or PyTorch fallback, and a missing
+library is an error.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import threading
+
+import torch
+
+from .workload import Shape
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbdscan.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "bdscan.h")
+
+BDSCAN_BF16, BDSCAN_FP32 = 0, 1
+BDSCAN_OP_PREFIX, BDSCAN_OP_BLOCK_STEP, BDSCAN_OP_ALLBLOCK = 0, 1, 2
+STATUS = {0: "BDSCAN_OK", -1: "BDSCAN_ERR_INVALID_ARG", -2: "BDSCAN_ERR_UNSUPPORTED_SHAPE",
+          -3: "BDSCAN_ERR_MISALIGNED", -4: "BDSCAN_ERR_WORKSPACE", -5: "BDSCAN_ERR_CUDA",
+          -6: "BDSCAN_ERR_TIMEOUT"}
+
+
+class bdscan_shape_t(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("batch", "seqlen", "nheads", "headdim", "dstate",
+                                               "ngroups", "block_len", "chunk_len")] + \
+               [("in_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32)]
+
+
+class bdscan_dir_t(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("dt", ctypes.c_void_p), ("B", ctypes.c_void_p),
+                ("C", ctypes.c_void_p), ("z", ctypes.c_void_p), ("A", ctypes.c_void_p),
+                ("D", ctypes.c_void_p)]
+
+
+class BdscanError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)} ({msg})")
+        self.status = status
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libbdscan.so (built in-tree by ``bidirectional_mamba_state_b200.build``)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"libbdscan.so is not built ({LIB_PATH}); run "
+                                   "`python -m bidirectional_mamba_state_b200.build` or "
+                                   "`__graft_entry__.build()`")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, sz = ctypes.c_void_p, ctypes.c_size_t
+            sp, dp = ctypes.POINTER(bdscan_shape_t), ctypes.POINTER(bdscan_dir_t)
+            L.bdscan_prefix.argtypes = [sp, dp, dp, vp, vp, vp, vp, vp, sz, vp]
+            L.bdscan_block_step.argtypes = [sp, dp, dp, vp, vp, vp, vp, sz, vp]
+            L.bdscan_allblock.argtypes = [sp, dp, dp, dp, dp, vp, vp, vp, vp, vp, sz, vp]
+            for fn in ("bdscan_prefix", "bdscan_block_step", "bdscan_allblock",
+                       "bdscan_check_status", "bdscan_version"):
+                getattr(L, fn).restype = ctypes.c_int
+            L.bdscan_workspace_size.argtypes = [sp, ctypes.c_int]
+            L.bdscan_workspace_size.restype = ctypes.c_size_t
+            L.bdscan_check_status.argtypes = [vp, vp]
+            L.bdscan_status_string.argtypes = [ctypes.c_int]
+            L.bdscan_status_string.restype = ctypes.c_char_p
+            _lib = L
+    return _lib
+
+
+def header_symbols() -> list[str]:
+    """Names of the functions declared in include/bdscan.h."""
+    with open(HEADER) as f:
+        text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    return sorted(set(re.findall(r"\b(bdscan_\w+)\s*\(", text)))
+
+
+# ----------------------------------------------------------------------------- raw C ABI
+def bdscan_prefix(shape, fwd, rev, h0, y, block_states, final_state, ws, ws_bytes, stream) -> int:
+    return lib().bdscan_prefix(shape, fwd, rev, h0, y, block_states, final_state, ws, ws_bytes, stream)
+
+
+def bdscan_block_step(shape, fwd, rev, state_in, y, state_out, ws, ws_bytes, stream) -> int:
+    return lib().bdscan_block_step(shape, fwd, rev, state_in, y, state_out, ws, ws_bytes, stream)
+
+
+def bdscan_allblock(shape, cf, cr, nf, nr, h0, y_clean, y_noisy, block_states, ws, ws_bytes,
+                    stream) -> int:
+    return lib().bdscan_allblock(shape, cf, cr, nf, nr, h0, y_clean, y_noisy, block_states, ws,
+                                 ws_bytes, stream)
+
+
+def bdscan_workspace_size(shape, op: int) -> int:
+    return int(lib().bdscan_workspace_size(shape, op))
+
+
+def bdscan_check_status(ws, stream) -> int:
+    return int(lib().bdscan_check_status(ws, stream))
+
+
+def bdscan_status_string(status: int) -> str:
+    return lib().bdscan_status_string(int(status)).decode()
+
+
+def bdscan_version() -> int:
+    return int(lib().bdscan_version())
+
+
+# ----------------------------------------------------------------------------- torch-facing
+_DT = {"bf16": (torch.bfloat16, BDSCAN_BF16), "fp32": (torch.float32, BDSCAN_FP32)}
+
+
+def c_shape(s: Shape) -> bdscan_shape_t:
+    return bdscan_shape_t(s.batch, s.seqlen, s.nheads, s.headdim, s.dstate, s.ngroups, s.block_len,
+                          s.chunk_len, _DT[s.in_dtype][1], _DT[s.out_dtype][1])
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _check_tensor(name, t, shape, dtype, device):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def c_dir(s: Shape, d: dict | None, device) -> bdscan_dir_t | None:
+    if d is None:
+        return None
+    tin = _DT[s.in_dtype][0]
+    B, L, H, P, N, G = s.batch, s.seqlen, s.nheads, s.headdim, s.dstate, s.ngroups
+    _check_tensor("x", d["x"], (B, L, H, P), tin, device)
+    _check_tensor("dt", d["dt"], (B, L, H), tin, device)
+    _check_tensor("B", d["B"], (B, L, G, N), tin, device)
+    _check_tensor("C", d["C"], (B, L, G, N), tin, device)
+    if d.get("z") is not None:
+        _check_tensor("z", d["z"], (B, L, H, P), tin, device)
+    _check_tensor("A", d["A"], (H,), torch.float32, device)
+    _check_tensor("D", d["D"], (H,), torch.float32, device)
+    return bdscan_dir_t(_ptr(d["x"]), _ptr(d["dt"]), _ptr(d["B"]), _ptr(d["C"]), _ptr(d.get("z")),
+                        _ptr(d["A"]), _ptr(d["D"]))
+
+
+def _ref(x):
+    return ctypes.byref(x) if x is not None else None
+
+
+def _stream(device, stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return s.cuda_stream
+
+
+def workspace(s: Shape, op: int, device) -> torch.Tensor:
+    n = bdscan_workspace_size(ctypes.byref(c_shape(s)), op)
+    if n == 0:
+        raise BdscanError("bdscan_workspace_size", -2, "invalid shape or op")
+    return torch.empty(((n + 255) // 256) * 256, dtype=torch.uint8, device=device)
+
+
+def _raise(fn, rc):
+    if rc != 0:
+        raise BdscanError(fn, rc, bdscan_status_string(rc))
+
+
+def _out(s: Shape, device):
+    return torch.empty((s.batch, s.seqlen, s.nheads, s.headdim), device=device,
+                       dtype=_DT[s.out_dtype][0])
+
+
+def _state(s: Shape, device, K=None):
+    if K is None:
+        return torch.empty((s.batch, s.nheads, s.headdim, s.dstate), device=device, dtype=torch.float32)
+    return torch.empty((s.batch, K, s.nheads, s.headdim, s.dstate), device=device, dtype=torch.float32)
+
+
+def prefix(s: Shape, fwd: dict, rev: dict | None = None, h0=None, want_states: bool = True,
+           want_final: bool = True, y=None, states=None, final=None, ws=None, stream=None):
+    """Clean-prefix scan (prefill / commit).  Returns (y, block_states or None,
+    final_state or None)."""
+    dev = fwd["x"].device
+    cs, cf, cr = c_shape(s), c_dir(s, fwd, dev), c_dir(s, rev, dev)
+    if h0 is not None:
+        _check_tensor("h0", h0, (s.batch, s.nheads, s.headdim, s.dstate), torch.float32, dev)
+    y = _out(s, dev) if y is None else y
+    states = (_state(s, dev, s.nblocks) if want_states else None) if states is None else states
+    final = (_state(s, dev) if want_final else None) if final is None else final
+    ws = workspace(s, BDSCAN_OP_PREFIX, dev) if ws is None else ws
+    rc = bdscan_prefix(ctypes.byref(cs), ctypes.byref(cf), _ref(cr), _ptr(h0), _ptr(y), _ptr(states),
+                       _ptr(final), _ptr(ws), ws.numel(), _stream(dev, stream))
+    _raise("bdscan_prefix", rc)
+    return y, states, final
+
+
+def block_step(s: Shape, fwd: dict, rev: dict | None, state_in, state_out=None, y=None, ws=None,
+               stream=None):
+    """One denoising step of the active block from the cached state.  ``state_out``:
+    None (no commit), a tensor (commit into it; may be ``state_in``) or True
+    (allocate).  Returns (y, state_out or None)."""
+    dev = fwd["x"].device
+    cs, cf, cr = c_shape(s), c_dir(s, fwd, dev), c_dir(s, rev, dev)
+    _check_tensor("state_in", state_in, (s.batch, s.nheads, s.headdim, s.dstate), torch.float32, dev)
+    if state_out is True:
+        state_out = _state(s, dev)
+    y = _out(s, dev) if y is None else y
+    ws = workspace(s, BDSCAN_OP_BLOCK_STEP, dev) if ws is None else ws
+    rc = bdscan_block_step(ctypes.byref(cs), ctypes.byref(cf), _ref(cr), _ptr(state_in), _ptr(y),
+                           _ptr(state_out), _ptr(ws), ws.numel(), _stream(dev, stream))
+    _raise("bdscan_block_step", rc)
+    return y, state_out
+
+
+def allblock(s: Shape, clean_fwd: dict, clean_rev: dict | None, noisy_fwd: dict,
+             noisy_rev: dict | None, h0=None, want_clean: bool = True, y_clean=None, y_noisy=None,
+             states=None, ws=None, stream=None):
+    """All-block training pass.  Returns (y_clean or None, y_noisy, block_states)."""
+    dev = clean_fwd["x"].device
+    cs = c_shape(s)
+    cf, cr = c_dir(s, clean_fwd, dev), c_dir(s, clean_rev, dev)
+    nf, nr = c_dir(s, noisy_fwd, dev), c_dir(s, noisy_rev, dev)
+    if h0 is not None:
+        _check_tensor("h0", h0, (s.batch, s.nheads, s.headdim, s.dstate), torch.float32, dev)
+    y_clean = (_out(s, dev) if want_clean else None) if y_clean is None else y_clean
+    y_noisy = _out(s, dev) if y_noisy is None else y_noisy
+    states = _state(s, dev, s.nblocks) if states is None else states
+    ws = workspace(s, BDSCAN_OP_ALLBLOCK, dev) if ws is None else ws
+    rc = bdscan_allblock(ctypes.byref(cs), ctypes.byref(cf), _ref(cr), ctypes.byref(nf), _ref(nr),
+                         _ptr(h0), _ptr(y_clean), _ptr(y_noisy), _ptr(states), _ptr(ws), ws.numel(),
+                         _stream(dev, stream))
+    _raise("bdscan_allblock", rc)
+    return y_clean, y_noisy, states

@@ -1,0 +1,295 @@
+// api.cu -- the C ABI of libbdscan: argument validation, workspace sizing,
+// dispatch to the kernels, status reporting.  See include/bdscan.h.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <utility>
+#include <vector>
+
+#include "bdscan.h"
+#include "bdscan_internal.h"
+
+using bdscan::DirArgs;
+using bdscan::Mode;
+using bdscan::ScanArgs;
+
+namespace {
+
+constexpr size_t kStatusBytes = 256;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Range {
+  uintptr_t lo, hi;  // [lo, hi)
+};
+
+Range range_of(const void *p, size_t bytes) {
+  uintptr_t lo = reinterpret_cast<uintptr_t>(p);
+  return {lo, lo + bytes};
+}
+
+bool overlaps(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi && a.hi > a.lo && b.hi > b.lo; }
+
+int check_shape(const bdscan_shape_t *s) {
+  if (!s) return BDSCAN_ERR_INVALID_ARG;
+  if (s->batch < 0 || s->seqlen < 0 || s->nheads < 1 || s->headdim < 1 || s->dstate < 1 ||
+      s->ngroups < 1 || s->block_len < 1 || s->chunk_len < 1)
+    return BDSCAN_ERR_INVALID_ARG;
+  if ((s->in_dtype != BDSCAN_BF16 && s->in_dtype != BDSCAN_FP32) ||
+      (s->out_dtype != BDSCAN_BF16 && s->out_dtype != BDSCAN_FP32))
+    return BDSCAN_ERR_INVALID_ARG;
+  if (s->nheads % s->ngroups) return BDSCAN_ERR_UNSUPPORTED_SHAPE;
+  if (s->seqlen % s->block_len) return BDSCAN_ERR_UNSUPPORTED_SHAPE;
+  if (s->chunk_len % s->block_len) return BDSCAN_ERR_UNSUPPORTED_SHAPE;
+  if (!(s->block_len <= 32 || (s->block_len % 32 == 0 && s->block_len <= 256)))
+    return BDSCAN_ERR_UNSUPPORTED_SHAPE;
+  if (!(s->headdim == 16 || s->headdim == 32 || s->headdim == 64 || s->headdim == 128))
+    return BDSCAN_ERR_UNSUPPORTED_SHAPE;
+  if (s->dstate > 256) return BDSCAN_ERR_UNSUPPORTED_SHAPE;
+  // 32-bit grid limits of the kernels
+  if (s->batch * s->nheads * (s->headdim / 16) > (int64_t)INT32_MAX) return BDSCAN_ERR_UNSUPPORTED_SHAPE;
+  return BDSCAN_OK;
+}
+
+struct Sizes {
+  size_t x, dt, bc, y, state, states, ad;
+};
+
+Sizes sizes_of(const bdscan_shape_t *s) {
+  const size_t in = s->in_dtype == BDSCAN_BF16 ? 2 : 4, out = s->out_dtype == BDSCAN_BF16 ? 2 : 4;
+  const size_t B = (size_t)s->batch, L = (size_t)s->seqlen, H = (size_t)s->nheads,
+               P = (size_t)s->headdim, N = (size_t)s->dstate, G = (size_t)s->ngroups,
+               K = (size_t)(s->seqlen / s->block_len);
+  Sizes z;
+  z.x = B * L * H * P * in;
+  z.dt = B * L * H * in;
+  z.bc = B * L * G * N * in;
+  z.y = B * L * H * P * out;
+  z.state = B * H * P * N * 4;
+  z.states = B * K * H * P * N * 4;
+  z.ad = H * 4;
+  return z;
+}
+
+// Validates one direction; appends its input ranges to `ins`.
+int check_dir(const bdscan_dir_t *d, const Sizes &z, std::vector<Range> &ins) {
+  // A pointer to a zero-byte tensor may be NULL (empty batch or sequence).
+  if (!d || !d->A || !d->D) return BDSCAN_ERR_INVALID_ARG;
+  if (z.x && (!d->x || !d->dt || !d->B || !d->C)) return BDSCAN_ERR_INVALID_ARG;
+  const void *ptrs[] = {d->x, d->dt, d->B, d->C, d->z, d->A, d->D};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return BDSCAN_ERR_MISALIGNED;
+  ins.push_back(range_of(d->x, z.x));
+  ins.push_back(range_of(d->dt, z.dt));
+  ins.push_back(range_of(d->B, z.bc));
+  ins.push_back(range_of(d->C, z.bc));
+  if (d->z) ins.push_back(range_of(d->z, z.x));
+  ins.push_back(range_of(d->A, z.ad));
+  ins.push_back(range_of(d->D, z.ad));
+  return BDSCAN_OK;
+}
+
+DirArgs to_args(const bdscan_dir_t *d) {
+  DirArgs a{};
+  if (d) {
+    a.x = d->x; a.dt = d->dt; a.B = d->B; a.C = d->C; a.z = d->z; a.A = d->A; a.D = d->D;
+  }
+  return a;
+}
+
+ScanArgs base_args(const bdscan_shape_t *s) {
+  ScanArgs a{};
+  a.Bsz = s->batch; a.L = s->seqlen; a.H = s->nheads; a.P = s->headdim; a.N = s->dstate;
+  a.G = s->ngroups; a.T = s->block_len; a.Q = s->chunk_len;
+  a.in_bf16 = s->in_dtype == BDSCAN_BF16;
+  a.out_bf16 = s->out_dtype == BDSCAN_BF16;
+  return a;
+}
+
+int check_outputs(const std::vector<Range> &ins, const std::vector<Range> &outs) {
+  for (size_t i = 0; i < outs.size(); ++i) {
+    for (const Range &r : ins)
+      if (overlaps(outs[i], r)) return BDSCAN_ERR_INVALID_ARG;
+    for (size_t j = i + 1; j < outs.size(); ++j)
+      if (overlaps(outs[i], outs[j])) return BDSCAN_ERR_INVALID_ARG;
+  }
+  return BDSCAN_OK;
+}
+
+int check_ws(void *ws, size_t ws_bytes, size_t need) {
+  if (!ws || ws_bytes < need) return BDSCAN_ERR_WORKSPACE;
+  if (!aligned16(ws)) return BDSCAN_ERR_MISALIGNED;
+  return BDSCAN_OK;
+}
+
+int launch(ScanArgs &a, cudaStream_t stream) {
+  a.status = reinterpret_cast<int *>(a.ws);
+  if (cudaMemsetAsync(a.ws, 0, sizeof(int), stream) != cudaSuccess) return BDSCAN_ERR_CUDA;
+  if (a.Bsz == 0) return BDSCAN_OK;
+  if (a.L == 0) {
+    // Nothing to scan: the final state is the initial one.
+    if (a.final_state) {
+      const size_t bytes = (size_t)(a.Bsz * a.H * a.P * a.N) * sizeof(float);
+      cudaError_t e = a.h0 ? cudaMemcpyAsync(a.final_state, a.h0, bytes, cudaMemcpyDeviceToDevice, stream)
+                           : cudaMemsetAsync(a.final_state, 0, bytes, stream);
+      if (e != cudaSuccess) return BDSCAN_ERR_CUDA;
+    }
+    return BDSCAN_OK;
+  }
+  cudaError_t e = bdscan::launch_seq(a, stream);
+  return e == cudaSuccess ? BDSCAN_OK : BDSCAN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t bdscan_workspace_size(const bdscan_shape_t *shape, int op) {
+  if (check_shape(shape) != BDSCAN_OK) return 0;
+  if (op != BDSCAN_OP_PREFIX && op != BDSCAN_OP_BLOCK_STEP && op != BDSCAN_OP_ALLBLOCK) return 0;
+  return kStatusBytes;
+}
+
+int bdscan_prefix(const bdscan_shape_t *shape, const bdscan_dir_t *fwd, const bdscan_dir_t *rev,
+                  const float *h0, void *y, float *block_states, float *final_state, void *ws,
+                  size_t ws_bytes, void *cuda_stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  const Sizes z = sizes_of(shape);
+  std::vector<Range> ins, outs;
+  if ((rc = check_dir(fwd, z, ins))) return rc;
+  if (rev && (rc = check_dir(rev, z, ins))) return rc;
+  if (!y && z.y) return BDSCAN_ERR_INVALID_ARG;
+  const void *ptrs[] = {h0, y, block_states, final_state};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return BDSCAN_ERR_MISALIGNED;
+  if (h0) ins.push_back(range_of(h0, z.state));
+  outs.push_back(range_of(y, z.y));
+  if (block_states) outs.push_back(range_of(block_states, z.states));
+  if (final_state) outs.push_back(range_of(final_state, z.state));
+  if ((rc = check_outputs(ins, outs))) return rc;
+  if ((rc = check_ws(ws, ws_bytes, bdscan_workspace_size(shape, BDSCAN_OP_PREFIX)))) return rc;
+  ScanArgs a = base_args(shape);
+  a.mode = Mode::Prefix;
+  a.cf = to_args(fwd);
+  a.cr = to_args(rev);
+  a.has_cr = rev != nullptr;
+  a.h0 = h0;
+  a.y_clean = y;
+  a.states = block_states;
+  a.final_state = final_state;
+  a.ws = ws;
+  a.ws_bytes = ws_bytes;
+  return launch(a, static_cast<cudaStream_t>(cuda_stream));
+}
+
+int bdscan_block_step(const bdscan_shape_t *shape, const bdscan_dir_t *fwd,
+                      const bdscan_dir_t *rev, const float *state_in, void *y, float *state_out,
+                      void *ws, size_t ws_bytes, void *cuda_stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (shape->seqlen != shape->block_len) return BDSCAN_ERR_UNSUPPORTED_SHAPE;
+  const Sizes z = sizes_of(shape);
+  std::vector<Range> ins, outs;
+  if ((rc = check_dir(fwd, z, ins))) return rc;
+  if (rev && (rc = check_dir(rev, z, ins))) return rc;
+  if ((!y && z.y) || (!state_in && z.state)) return BDSCAN_ERR_INVALID_ARG;
+  const void *ptrs[] = {state_in, y, state_out};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return BDSCAN_ERR_MISALIGNED;
+  // state_out may be exactly state_in (in-place commit) but must not partially
+  // overlap it; an in-place state must not alias any other input.
+  const Range rin = range_of(state_in, z.state);
+  if (state_out == state_in) {
+    for (const Range &r : ins)
+      if (overlaps(rin, r)) return BDSCAN_ERR_INVALID_ARG;
+  }
+  ins.push_back(rin);
+  outs.push_back(range_of(y, z.y));
+  if (state_out && state_out != state_in) outs.push_back(range_of(state_out, z.state));
+  if ((rc = check_outputs(ins, outs))) return rc;
+  if ((rc = check_ws(ws, ws_bytes, bdscan_workspace_size(shape, BDSCAN_OP_BLOCK_STEP)))) return rc;
+  ScanArgs a = base_args(shape);
+  a.mode = Mode::Step;
+  a.cf = to_args(fwd);
+  a.cr = to_args(rev);
+  a.has_cr = rev != nullptr;
+  a.h0 = state_in;
+  a.y_clean = y;
+  a.final_state = state_out;
+  a.ws = ws;
+  a.ws_bytes = ws_bytes;
+  return launch(a, static_cast<cudaStream_t>(cuda_stream));
+}
+
+int bdscan_allblock(const bdscan_shape_t *shape, const bdscan_dir_t *clean_fwd,
+                    const bdscan_dir_t *clean_rev, const bdscan_dir_t *noisy_fwd,
+                    const bdscan_dir_t *noisy_rev, const float *h0, void *y_clean, void *y_noisy,
+                    float *block_states, void *ws, size_t ws_bytes, void *cuda_stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  const Sizes z = sizes_of(shape);
+  std::vector<Range> ins, outs;
+  if ((rc = check_dir(clean_fwd, z, ins))) return rc;
+  if (clean_rev && (rc = check_dir(clean_rev, z, ins))) return rc;
+  if ((rc = check_dir(noisy_fwd, z, ins))) return rc;
+  if (noisy_rev && (rc = check_dir(noisy_rev, z, ins))) return rc;
+  if ((!y_noisy && z.y) || (!block_states && z.states)) return BDSCAN_ERR_INVALID_ARG;
+  const void *ptrs[] = {h0, y_clean, y_noisy, block_states};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return BDSCAN_ERR_MISALIGNED;
+  if (h0) ins.push_back(range_of(h0, z.state));
+  if (y_clean) outs.push_back(range_of(y_clean, z.y));
+  outs.push_back(range_of(y_noisy, z.y));
+  outs.push_back(range_of(block_states, z.states));
+  if ((rc = check_outputs(ins, outs))) return rc;
+  if ((rc = check_ws(ws, ws_bytes, bdscan_workspace_size(shape, BDSCAN_OP_ALLBLOCK)))) return rc;
+  ScanArgs a = base_args(shape);
+  a.mode = Mode::AllBlock;
+  a.cf = to_args(clean_fwd);
+  a.cr = to_args(clean_rev);
+  a.nf = to_args(noisy_fwd);
+  a.nr = to_args(noisy_rev);
+  a.has_cr = clean_rev != nullptr;
+  a.has_nr = noisy_rev != nullptr;
+  a.h0 = h0;
+  a.y_clean = y_clean;
+  a.y_noisy = y_noisy;
+  a.states = block_states;
+  a.ws = ws;
+  a.ws_bytes = ws_bytes;
+  return launch(a, static_cast<cudaStream_t>(cuda_stream));
+}
+
+int bdscan_check_status(const void *ws, void *cuda_stream) {
+  if (!ws) return BDSCAN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  int host = 0;
+  if (cudaMemcpyAsync(&host, ws, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return BDSCAN_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return BDSCAN_ERR_CUDA;
+  if (host != 0) {
+    if (cudaMemsetAsync(const_cast<void *>(ws), 0, sizeof(int), st) != cudaSuccess)
+      return BDSCAN_ERR_CUDA;
+  }
+  return host;
+}
+
+const char *bdscan_status_string(int status) {
+  switch (status) {
+    case BDSCAN_OK: return "ok";
+    case BDSCAN_ERR_INVALID_ARG: return "invalid argument (null pointer, bad enum or overlapping buffers)";
+    case BDSCAN_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case BDSCAN_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case BDSCAN_ERR_WORKSPACE: return "workspace missing or too small";
+    case BDSCAN_ERR_CUDA: return "CUDA launch or runtime error";
+    case BDSCAN_ERR_TIMEOUT: return "bounded device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int bdscan_version(void) { return 100; }
+
+}  // extern "C"

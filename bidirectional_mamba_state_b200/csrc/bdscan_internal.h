@@ -1,0 +1,37 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace bdscan {
+
+enum class Mode : int { Prefix = 0, Step = 1, AllBlock = 2 };
+
+struct DirArgs {
+  const void *x, *dt, *B, *C, *z;  // z == nullptr: no gate
+  const float *A, *D;
+};
+
+// One fully validated call.  Step is expressed as a prefix over a single block
+// (h0 = state_in, final_state = state_out).
+struct ScanArgs {
+  int64_t Bsz, L, H, P, N, G, T, Q;
+  bool in_bf16, out_bf16;
+  Mode mode;
+  DirArgs cf, cr, nf, nr;  // clean fwd/rev, noisy fwd/rev (noisy: AllBlock only)
+  bool has_cr, has_nr;
+  const float *h0;         // nullptr = zeros
+  void *y_clean;           // may be nullptr (AllBlock)
+  void *y_noisy;           // AllBlock only
+  float *states;           // [B][K][H][P][N] or nullptr
+  float *final_state;      // [B][H][P][N] or nullptr
+  void *ws;                // workspace (>= 256 B); first word: device status
+  size_t ws_bytes;
+  int *status;             // == ws
+};
+
+// Generic path: direct sequential recurrence on CUDA cores (any supported
+// shape, fp32 or bf16 inputs, gated or not).
+cudaError_t launch_seq(const ScanArgs &a, cudaStream_t stream);
+
+}  // namespace bdscan

@@ -1,0 +1,149 @@
+/*
+ * bdscan.h -- C ABI of libbdscan, the cache-aligned bidirectional Mamba-2 scan
+ * of a block-diffusion (BDLM Mamba-H style) denoiser, for NVIDIA B200 (sm_100a).
+ *
+ * The operation (per batch row b and head h, with group g = h / (H / G)):
+ *
+ *   a_t = exp(dt_t * A_h)
+ *   h_t = a_t * h_{t-1} + dt_t * x_t B_t^T               state h_t is P x N, fp32
+ *   y_t = (h_t C_t + D_h * x_t) [* silu(z_t) if z is given]
+ *
+ * ("Training Hybrid Block Diffusion Language Models with Partial
+ * Bidirectionality", eq. (1), Mamba-2 form with a scalar decay per head.)
+ * The sequence is cut into blocks of T = block_len tokens.  The forward
+ * direction runs over the whole sequence and leaves one boundary state per
+ * block (eq. (10)); the reverse direction runs right to left inside each block
+ * only, from a zero state, with its own parameters (eq. (12)); the two outputs
+ * are summed (eq. (13); "Breaking the Bottleneck with DiffuApriel",
+ * section 3.2, eq. (6)).
+ *
+ * Layouts: every tensor is dense row-major, innermost dimension last.
+ *   x, z, y    [B][L][H][P]     in_dtype (x, z) / out_dtype (y)
+ *   dt         [B][L][H]        in_dtype; already positive (softplus applied)
+ *   B, C       [B][L][G][N]     in_dtype
+ *   A, D       [H]              fp32
+ *   state      [B][H][P][N]     fp32 (h0, state_in, state_out, final_state)
+ *   block_states [B][K][H][P][N] fp32, K = L / T; block_states[b][k] is the
+ *              forward state after token (k+1)*T - 1 (end of block k).
+ *
+ * Ownership: the caller owns every buffer, including the workspace; the
+ * library allocates no device memory and keeps no global mutable state, so
+ * calls are reentrant.  All device pointers must be device-accessible memory
+ * of the current device.  Every call is asynchronous on `cuda_stream` (a
+ * cudaStream_t; NULL = the legacy default stream).
+ *
+ * Errors: every entry point validates its arguments synchronously, before any
+ * launch, and returns a BDSCAN_* status; nothing aborts the process.  A launch
+ * failure returns BDSCAN_ERR_CUDA.  Numeric problems (NaN/Inf inputs) are not
+ * trapped; they propagate to the outputs of the same (b, h) only.
+ */
+#ifndef BDSCAN_H
+#define BDSCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* element types (bdscan_shape_t.in_dtype / out_dtype) */
+#define BDSCAN_BF16 0
+#define BDSCAN_FP32 1
+
+/* status codes */
+#define BDSCAN_OK 0
+#define BDSCAN_ERR_INVALID_ARG (-1)       /* null pointer, bad enum, negative size, aliasing */
+#define BDSCAN_ERR_UNSUPPORTED_SHAPE (-2) /* shape outside the supported set (see below) */
+#define BDSCAN_ERR_MISALIGNED (-3)        /* a pointer is not 16-byte aligned */
+#define BDSCAN_ERR_WORKSPACE (-4)         /* ws NULL or ws_bytes < bdscan_workspace_size() */
+#define BDSCAN_ERR_CUDA (-5)              /* a kernel launch or CUDA runtime call failed */
+#define BDSCAN_ERR_TIMEOUT (-6)           /* a bounded device-side wait ran out (check_status) */
+
+/* operations (bdscan_workspace_size) */
+#define BDSCAN_OP_PREFIX 0
+#define BDSCAN_OP_BLOCK_STEP 1
+#define BDSCAN_OP_ALLBLOCK 2
+
+/* Problem shape.  Supported: batch >= 0, seqlen >= 0, seqlen % block_len == 0,
+ * 1 <= block_len <= 32 or block_len % 32 == 0 (<= 256), chunk_len % block_len
+ * == 0 (chunk_len is the tile of tokens a kernel stages at once; it changes
+ * no result beyond rounding order), nheads % ngroups == 0, headdim in
+ * {16, 32, 64, 128}, 1 <= dstate <= 256. */
+typedef struct {
+    int64_t batch, seqlen, nheads, headdim, dstate, ngroups, block_len, chunk_len;
+    int32_t in_dtype;  /* BDSCAN_BF16 | BDSCAN_FP32: x, dt, B, C, z */
+    int32_t out_dtype; /* BDSCAN_FP32 | BDSCAN_BF16: y */
+} bdscan_shape_t;
+
+/* One scan direction's inputs (device pointers).  z may be NULL (no gate).
+ * A direction may alias another (tied weights). */
+typedef struct {
+    const void *x, *dt, *B, *C, *z;
+    const float *A, *D;
+} bdscan_dir_t;
+
+/* bdscan_prefix -- clean-prefix scan, for prefill and for committing blocks.
+ * Source: eq. (10) (boundary states) and the commit described after eq. (6)
+ * ("after the block is finalized, a clean forward pass ... appends") of the
+ * first page; eq. (12)-(13) for the optional block-local reverse.
+ *   fwd          forward direction (required)
+ *   rev          reverse direction, applied inside every block; NULL = none
+ *   h0           [B][H][P][N] initial state; NULL = zeros
+ *   y            [B][L][H][P] output (out_dtype), y = y_fwd + y_rev
+ *   block_states [B][K][H][P][N] or NULL: forward state at the end of each block
+ *   final_state  [B][H][P][N] or NULL: forward state after token L-1
+ *                (== h0, or zeros, when L == 0)
+ *   ws, ws_bytes workspace of at least bdscan_workspace_size(shape, PREFIX)
+ *                bytes (16-byte aligned); its contents need no initialisation
+ * y must not overlap any input; block_states / final_state must not overlap
+ * h0 or any input. */
+int bdscan_prefix(const bdscan_shape_t *shape, const bdscan_dir_t *fwd, const bdscan_dir_t *rev,
+                  const float *h0, void *y, float *block_states, float *final_state, void *ws,
+                  size_t ws_bytes, void *cuda_stream);
+
+/* bdscan_block_step -- one denoising step of the active block from the cached
+ * forward state: forward continuation (eq. (11)), block-local reverse
+ * (eq. (12)), sum (eq. (13)).  shape->seqlen must equal shape->block_len.
+ *   state_in   [B][H][P][N] cached state (read only; never modified unless it
+ *              is also passed as state_out)
+ *   y          [B][T][H][P] output
+ *   state_out  [B][H][P][N] or NULL: forward state after the block (commit);
+ *              may be equal to state_in (in-place commit), must not partially
+ *              overlap it. */
+int bdscan_block_step(const bdscan_shape_t *shape, const bdscan_dir_t *fwd,
+                      const bdscan_dir_t *rev, const float *state_in, void *y, float *state_out,
+                      void *ws, size_t ws_bytes, void *cuda_stream);
+
+/* bdscan_allblock -- all-block training pass (eq. (14) and the all-block
+ * objective after eq. (5)): the clean stream is scanned as by bdscan_prefix
+ * (with clean_rev inside each block) and emits every boundary state; every
+ * noisy block k is scanned forward from the clean boundary state before it
+ * (h0 for k = 0) plus its own block-local reverse.
+ *   y_clean      [B][L][H][P] or NULL
+ *   y_noisy      [B][L][H][P] (required)
+ *   block_states [B][K][H][P][N] (required) */
+int bdscan_allblock(const bdscan_shape_t *shape, const bdscan_dir_t *clean_fwd,
+                    const bdscan_dir_t *clean_rev, const bdscan_dir_t *noisy_fwd,
+                    const bdscan_dir_t *noisy_rev, const float *h0, void *y_clean, void *y_noisy,
+                    float *block_states, void *ws, size_t ws_bytes, void *cuda_stream);
+
+/* Workspace bytes an operation needs for this shape (>= 256: the first 256
+ * bytes hold the device status word).  Returns 0 for an invalid shape/op. */
+size_t bdscan_workspace_size(const bdscan_shape_t *shape, int op);
+
+/* Reads the device status word in ws after the work queued on cuda_stream
+ * completes (synchronises that stream), clears it, and returns it
+ * (BDSCAN_OK or BDSCAN_ERR_TIMEOUT).  Returns BDSCAN_ERR_CUDA if the copy fails. */
+int bdscan_check_status(const void *ws, void *cuda_stream);
+
+/* Static description of a status code. */
+const char *bdscan_status_string(int status);
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int bdscan_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BDSCAN_H */

@@ -1,0 +1,156 @@
+"""CPU tests of the C-ABI library: it loads without a GPU, exports every symbol
+the header declares, sizes workspaces, and rejects bad arguments with the
+documented status codes before any launch (validation is host-side)."""
+import ctypes
+
+import pytest
+
+from bidirectional_mamba_state_b200 import bdscan as bd
+from bidirectional_mamba_state_b200.workload import Shape, WORKLOADS
+
+
+def test_exports_every_header_symbol():
+    names = bd.header_symbols()
+    assert {"bdscan_prefix", "bdscan_block_step", "bdscan_allblock", "bdscan_workspace_size",
+            "bdscan_check_status", "bdscan_status_string"} <= set(names)
+    L = bd.lib()
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, f"libbdscan.so lacks {missing}"
+
+
+def test_status_strings_and_version():
+    for code in bd.STATUS:
+        assert bd.bdscan_status_string(code)
+    assert bd.bdscan_status_string(12345) == "unknown status"
+    assert bd.bdscan_version() >= 100
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_workspace_size_valid(name):
+    s = bd.c_shape(WORKLOADS[name])
+    for op in (bd.BDSCAN_OP_PREFIX, bd.BDSCAN_OP_ALLBLOCK):
+        assert bd.bdscan_workspace_size(ctypes.byref(s), op) >= 256
+    if WORKLOADS[name].seqlen == WORKLOADS[name].block_len:
+        assert bd.bdscan_workspace_size(ctypes.byref(s), bd.BDSCAN_OP_BLOCK_STEP) >= 256
+
+
+BAD_SHAPES = [
+    (dict(seqlen=100), -2),        # not a multiple of block_len
+    (dict(chunk_len=40), -2),      # chunk not a multiple of block
+    (dict(nheads=5), -2),          # H % G != 0 (G = 2 below)
+    (dict(headdim=48), -2),
+    (dict(dstate=512), -2),
+    (dict(block_len=48, seqlen=96, chunk_len=96), -2),
+    (dict(batch=-1), -1),
+    (dict(nheads=0), -1),
+    (dict(in_dtype="fp16"), None),  # not representable: checked below via raw enum
+]
+
+
+def _base(**kw):
+    d = dict(batch=2, seqlen=64, nheads=4, headdim=16, dstate=32, ngroups=2, block_len=16,
+             chunk_len=32, in_dtype="bf16", out_dtype="fp32")
+    d.update(kw)
+    return d
+
+
+@pytest.mark.parametrize("kw,code", BAD_SHAPES[:-1])
+def test_bad_shape_rejected(kw, code):
+    s = bd.c_shape(Shape(**_base(**kw)))
+    assert bd.bdscan_workspace_size(ctypes.byref(s), bd.BDSCAN_OP_PREFIX) == 0
+    fwd = _fake_dir(0x10000)
+    rc = bd.bdscan_prefix(ctypes.byref(s), ctypes.byref(fwd), None, None, 0x900000, None, None,
+                          0xA00000, 1 << 20, None)
+    assert rc == code
+
+
+def test_bad_dtype_enum():
+    s = bd.c_shape(Shape(**_base()))
+    s.in_dtype = 7
+    fwd = _fake_dir(0x10000)
+    rc = bd.bdscan_prefix(ctypes.byref(s), ctypes.byref(fwd), None, None, 0x900000, None, None,
+                          0xA00000, 1 << 20, None)
+    assert rc == -1
+
+
+def _fake_dir(base, step=0x100000):
+    # Distinct, 16-byte aligned, non-overlapping fake device addresses.  They are
+    # never dereferenced: every call below fails validation before any launch.
+    p = [base + i * step for i in range(7)]
+    return bd.bdscan_dir_t(p[0], p[1], p[2], p[3], None, p[4], p[5])
+
+
+def _prefix(shape_kw=None, fwd=None, rev=None, h0=None, y=0x90000000, states=None, final=None,
+            ws=0xA0000000, ws_bytes=1 << 20):
+    s = bd.c_shape(Shape(**_base(**(shape_kw or {}))))
+    fwd = _fake_dir(0x10000000) if fwd is None else fwd
+    return bd.bdscan_prefix(ctypes.byref(s), ctypes.byref(fwd) if fwd != "null" else None,
+                            ctypes.byref(rev) if rev is not None else None, h0, y, states, final,
+                            ws, ws_bytes, None)
+
+
+def test_null_pointers_rejected():
+    assert _prefix(fwd="null") == -1
+    assert _prefix(y=None) == -1
+    d = _fake_dir(0x10000000)
+    d.x = None
+    assert _prefix(fwd=d) == -1
+    d = _fake_dir(0x10000000)
+    d.A = None
+    assert _prefix(fwd=d) == -1
+
+
+def test_misaligned_rejected():
+    d = _fake_dir(0x10000000)
+    d.B = d.B + 4
+    assert _prefix(fwd=d) == -3
+    assert _prefix(y=0x90000008) == -3
+    assert _prefix(ws=0xA0000004) == -3
+
+
+def test_workspace_checked():
+    assert _prefix(ws=None) == -4
+    assert _prefix(ws_bytes=16) == -4
+
+
+def test_output_aliasing_rejected():
+    d = _fake_dir(0x10000000)
+    assert _prefix(fwd=d, y=d.x) == -1           # y over x
+    assert _prefix(fwd=d, y=d.x + 0x100) == -1   # partial overlap
+    assert _prefix(states=0x90000000) == -1      # states over y
+
+
+def test_block_step_requires_single_block():
+    s = bd.c_shape(Shape(**_base()))  # seqlen 64 != block_len 16
+    fwd = _fake_dir(0x10000000)
+    rc = bd.bdscan_block_step(ctypes.byref(s), ctypes.byref(fwd), None, 0x80000000, 0x90000000, None,
+                              0xA0000000, 1 << 20, None)
+    assert rc == -2
+
+
+def test_block_step_state_aliasing():
+    s = bd.c_shape(Shape(**_base(seqlen=16)))
+    fwd = _fake_dir(0x10000000)
+    # partial overlap of state_out with state_in is rejected
+    rc = bd.bdscan_block_step(ctypes.byref(s), ctypes.byref(fwd), None, 0x80000000, 0x90000000,
+                              0x80000100, 0xA0000000, 1 << 20, None)
+    assert rc == -1
+    # y over state_in is rejected
+    rc = bd.bdscan_block_step(ctypes.byref(s), ctypes.byref(fwd), None, 0x80000000, 0x80000000,
+                              None, 0xA0000000, 1 << 20, None)
+    assert rc == -1
+    # null state_in is rejected
+    rc = bd.bdscan_block_step(ctypes.byref(s), ctypes.byref(fwd), None, None, 0x90000000, None,
+                              0xA0000000, 1 << 20, None)
+    assert rc == -1
+
+
+def test_allblock_requires_outputs():
+    s = bd.c_shape(Shape(**_base()))
+    cf, nf = _fake_dir(0x10000000), _fake_dir(0x20000000)
+    rc = bd.bdscan_allblock(ctypes.byref(s), ctypes.byref(cf), None, ctypes.byref(nf), None, None,
+                            None, None, 0x90000000, 0xA0000000, 1 << 20, None)
+    assert rc == -1   # y_noisy missing
+    rc = bd.bdscan_allblock(ctypes.byref(s), ctypes.byref(cf), None, None, None, None,
+                            None, 0x90000000, 0x98000000, 0xA0000000, 1 << 20, None)
+    assert rc == -1   # noisy_fwd missing

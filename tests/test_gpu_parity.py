@@ -1,0 +1,234 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle on the
+same seeded inputs, plus the invariants that must hold bit-exactly on the
+device (boundary-state independence, state_in untouched, determinism)."""
+import pytest
+import torch
+
+import oracle
+from bidirectional_mamba_state_b200 import bdscan as bd
+from bidirectional_mamba_state_b200 import workload as W
+from parity import check_states, check_y, heads
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _shape(**kw):
+    d = dict(batch=2, seqlen=160, nheads=6, headdim=64, dstate=128, ngroups=2, block_len=32,
+             chunk_len=64, in_dtype="bf16", out_dtype="fp32")
+    d.update(kw)
+    return W.Shape(**d)
+
+
+# shapes spanning several tiles, ragged tails and the degenerate cases
+SMALL = {
+    "tiny_fp32": W.WORKLOADS["tiny"],
+    "bf16_multi": _shape(),
+    "bf16_p16_n48_t16": _shape(headdim=16, dstate=48, block_len=16, chunk_len=16, seqlen=80),
+    "fp32_p32_n16_t8": _shape(headdim=32, dstate=16, block_len=8, chunk_len=8, seqlen=40,
+                              in_dtype="fp32", nheads=4),
+    "bf16_t64_p128_n256": _shape(headdim=128, dstate=256, block_len=64, chunk_len=64, seqlen=128,
+                                 nheads=2, ngroups=1, batch=1),
+    "bf16_out_bf16": _shape(out_dtype="bf16"),
+    "g1_h8": _shape(ngroups=1, nheads=8, batch=1, seqlen=96),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+@pytest.mark.parametrize("with_h0", [False, True])
+def test_prefix_parity(name, with_h0):
+    s = SMALL[name]
+    f, r = W.make_streams(s, 1, streams=(W.CLEAN_FWD, W.CLEAN_REV), device=DEV)
+    h0 = W.make_state(s, 1, device=DEV) if with_h0 else None
+    y, st, fin = bd.prefix(s, f, r, h0=h0)
+    ry, rst, rfin = oracle.prefix(s.as_dict(), f, r, h0=h0)
+    check_y(y, ry, bf16_out=s.out_dtype == "bf16")
+    check_states(st, rst)
+    check_states(fin, rfin, "final")
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_allblock_parity(name):
+    s = SMALL[name]
+    cf, cr, nf, nr = W.make_streams(s, 2, device=DEV)
+    h0 = W.make_state(s, 2, device=DEV)
+    yc, yn, st = bd.allblock(s, cf, cr, nf, nr, h0=h0)
+    ryc, ryn, rst = oracle.allblock(s.as_dict(), cf, cr, nf, nr, h0=h0)
+    check_y(yc, ryc, bf16_out=s.out_dtype == "bf16", what="y_clean")
+    check_y(yn, ryn, bf16_out=s.out_dtype == "bf16", what="y_noisy")
+    check_states(st, rst)
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+@pytest.mark.parametrize("commit", ["none", "new", "inplace"])
+def test_block_step_parity(name, commit):
+    s = SMALL[name].with_(seqlen=SMALL[name].block_len, chunk_len=SMALL[name].block_len)
+    f, r = W.make_streams(s, 3, streams=(W.CLEAN_FWD, W.CLEAN_REV), device=DEV)
+    state = W.make_state(s, 3, device=DEV, scale=2.0)
+    keep = state.clone()
+    ry, rso = oracle.block_step(s.as_dict(), f, r, keep, want_state_out=True)
+    out = {"none": None, "new": True, "inplace": state}[commit]
+    y, so = bd.block_step(s, f, r, state, state_out=out)
+    torch.cuda.synchronize()
+    check_y(y, ry, bf16_out=s.out_dtype == "bf16")
+    if commit == "none":
+        assert torch.equal(state, keep), "state_in modified by a non-committing step"
+    else:
+        check_states(so, rso, "state_out")
+
+
+def test_no_reverse_and_gated():
+    s = _shape()
+    f = W.make_dir(s, 4, 0, W.CLEAN_FWD, DEV, gated=True)
+    r = W.make_dir(s, 4, 0, W.CLEAN_REV, DEV, gated=True)
+    for rev in (None, r):
+        y, st, fin = bd.prefix(s, f, rev)
+        ry, rst, rfin = oracle.prefix(s.as_dict(), f, rev)
+        check_y(y, ry)
+        check_states(st, rst)
+
+
+def test_cache_independent_of_active_block_bitwise():
+    """Boundary states do not depend on the noisy stream or the reverse
+    direction (bit-exact), and a perturbation of clean x at token j leaves
+    states[k] for k < j // T bit-identical."""
+    s = _shape(batch=1)
+    cf, cr, nf, nr = W.make_streams(s, 5, device=DEV)
+    _, _, st = bd.allblock(s, cf, cr, nf, nr)
+    nf2, nr2, cr2 = (W.make_dir(s, 77, 0, k, DEV) for k in (W.NOISY_FWD, W.NOISY_REV, W.CLEAN_REV))
+    _, _, st2 = bd.allblock(s, cf, cr2, nf2, nr2)
+    assert torch.equal(st, st2)
+    j = 70
+    cf3 = {k: v.clone() for k, v in cf.items()}
+    cf3["x"][0, j] += 1.0
+    _, _, st3 = bd.allblock(s, cf3, cr, nf, nr)
+    kb = j // s.block_len
+    assert torch.equal(st3[:, :kb], st[:, :kb])
+    assert not torch.equal(st3[:, kb], st[:, kb])
+
+
+def test_deterministic_bitwise():
+    s = _shape()
+    cf, cr, nf, nr = W.make_streams(s, 6, device=DEV)
+    a = bd.allblock(s, cf, cr, nf, nr)
+    b = bd.allblock(s, cf, cr, nf, nr)
+    for u, v in zip(a, b):
+        assert torch.equal(u, v)
+
+
+def test_empty_inputs():
+    for kw in (dict(batch=0), dict(seqlen=0)):
+        s = _shape(**kw)
+        f = W.make_dir(s, 7, 0, W.CLEAN_FWD, DEV)
+        h0 = torch.randn((s.batch, s.nheads, s.headdim, s.dstate), device=DEV)
+        y, st, fin = bd.prefix(s, f, None, h0=h0)
+        torch.cuda.synchronize()
+        assert y.numel() == 0 or s.batch == 0
+        if s.seqlen == 0:
+            assert torch.equal(fin, h0)
+
+
+def test_noisy_equals_clean_on_device():
+    s = _shape(batch=1)
+    cf, cr, _, _ = W.make_streams(s, 8, device=DEV)
+    yc, yn, _ = bd.allblock(s, cf, cr, cf, cr)
+    torch.testing.assert_close(yn, yc, rtol=1e-5, atol=1e-5)
+
+
+def test_status_word_clear_after_call():
+    s = _shape(batch=1)
+    cf, cr, nf, nr = W.make_streams(s, 9, device=DEV)
+    ws = bd.workspace(s, bd.BDSCAN_OP_ALLBLOCK, DEV)
+    bd.allblock(s, cf, cr, nf, nr, ws=ws)
+    assert bd.bdscan_check_status(ws.data_ptr(), torch.cuda.current_stream().cuda_stream) == 0
+
+
+# ---------------------------------------------------------------- the five workloads
+def test_workload_tiny():
+    s = W.WORKLOADS["tiny"]
+    cf, cr, nf, nr = W.make_streams(s, W.SEEDS["tiny"], device=DEV)
+    yc, yn, st = bd.allblock(s, cf, cr, nf, nr)
+    ryc, ryn, rst = oracle.allblock(s.as_dict(), cf, cr, nf, nr)
+    check_y(yc, ryc)
+    check_y(yn, ryn)
+    check_states(st, rst)
+
+
+def test_workload_87m_allblock_full():
+    """87M all-block layer at full size (B16 x 1024, 24 heads), every output."""
+    s = W.WORKLOADS["87m_allblock"]
+    cf, cr, nf, nr = W.make_streams(s, W.SEEDS["87m_allblock"], device=DEV)
+    yc, yn, st = bd.allblock(s, cf, cr, nf, nr)
+    ryc, ryn, rst = oracle.allblock(s.as_dict(), cf, cr, nf, nr)
+    check_y(yc, ryc, what="y_clean")
+    check_y(yn, ryn, what="y_noisy")
+    check_states(st, rst)
+
+
+def test_workload_350m_allblock_sampled_heads():
+    """350M all-block layer (B4 x 8192, 32 heads) on the device at full size;
+    the oracle recomputes 3 heads of 2 batch rows (every block)."""
+    s = W.WORKLOADS["350m_allblock"]
+    cf, cr, nf, nr = W.make_streams(s, W.SEEDS["350m_allblock"], device=DEV)
+    yc, yn, st = bd.allblock(s, cf, cr, nf, nr)
+    hs = [0, 13, 31]
+    bs = [0, 3]
+    sub = s.with_(batch=len(bs), nheads=len(hs))
+    pick = lambda d: {k: (v[bs] if k not in ("A", "D") else v) for k, v in heads(d, hs).items()}
+    ryc, ryn, rst = oracle.allblock(sub.as_dict(), pick(cf), pick(cr), pick(nf), pick(nr))
+    check_y(yc[bs][:, :, hs], ryc, what="y_clean")
+    check_y(yn[bs][:, :, hs], ryn, what="y_noisy")
+    check_states(st[bs][:, :, hs], rst)
+
+
+@pytest.mark.parametrize("L", [8192, 32768])
+def test_workload_700m_prefill_then_steps(L):
+    """700M inference: prefill of L tokens (final state only) on the device over
+    all 48 heads, then two denoising steps and a commit; the oracle follows 4
+    heads through prefill, steps and commit."""
+    s = W.WORKLOADS["700m_prefill_8k"].with_(seqlen=L)
+    f, r = W.make_streams(s, W.SEEDS["700m_prefill_8k"], streams=(W.CLEAN_FWD, W.CLEAN_REV), device=DEV)
+    y, _, fin = bd.prefix(s, f, r, want_states=False)
+    hs = [0, 7, 30, 47]
+    sub = s.with_(nheads=len(hs))
+    ry, _, rfin = oracle.prefix(sub.as_dict(), heads(f, hs), heads(r, hs), want_states=False)
+    check_y(y[:, :, hs], ry)
+    check_states(fin[:, hs], rfin, "prefill final")
+    st = W.WORKLOADS["700m_step"]
+    for step in range(2):
+        af, ar = W.make_streams(st, 100 + step, streams=(W.CLEAN_FWD, W.CLEAN_REV), device=DEV)
+        yb, _ = bd.block_step(st, af, ar, fin)
+        ryb, _ = oracle.block_step(st.with_(nheads=len(hs)).as_dict(), heads(af, hs), heads(ar, hs),
+                                   rfin)
+        check_y(yb[:, :, hs], ryb, what=f"step {step}")
+    yb, so = bd.block_step(st, af, ar, fin, state_out=True)
+    _, rso = oracle.block_step(st.with_(nheads=len(hs)).as_dict(), heads(af, hs), heads(ar, hs), rfin,
+                               want_state_out=True)
+    check_states(so[:, hs], rso, "commit")
+
+
+def test_workload_3b_256k_prefill_and_batch64_step():
+    """3B: 262,144-token prefill on the device (all 80 heads, final state only),
+    oracle on 2 heads; then a batch-64 step (all heads on the device, oracle on
+    4 sequences x 4 heads)."""
+    s = W.WORKLOADS["3b_prefill_256k"]
+    f, r = W.make_streams(s, W.SEEDS["3b_prefill_256k"], streams=(W.CLEAN_FWD, W.CLEAN_REV), device=DEV)
+    y, _, fin = bd.prefix(s, f, r, want_states=False)
+    hs = [0, 79]
+    ry, _, rfin = oracle.prefix(s.with_(nheads=2).as_dict(), heads(f, hs), heads(r, hs),
+                                want_states=False)
+    check_y(y[:, -4096:, hs], ry[:, -4096:], what="last 4096 tokens")
+    check_y(y[:, :, hs], ry)
+    check_states(fin[:, hs], rfin, "final")
+    del y, f, r
+    st = W.WORKLOADS["3b_step_b64"]
+    af, ar = W.make_streams(st, 4, streams=(W.CLEAN_FWD, W.CLEAN_REV), device=DEV)
+    state = W.make_state(st, 4, device=DEV, scale=1.0)
+    yb, so = bd.block_step(st, af, ar, state, state_out=True)
+    bs, hs = [0, 21, 42, 63], [1, 40, 41, 78]
+    pick = lambda d: {k: (v[bs] if k not in ("A", "D") else v) for k, v in heads(d, hs).items()}
+    sub = st.with_(batch=4, nheads=4)
+    ryb, rso = oracle.block_step(sub.as_dict(), pick(af), pick(ar), state[bs][:, hs], want_state_out=True)
+    check_y(yb[bs][:, :, hs], ryb)
+    check_states(so[bs][:, hs], rso, "commit")
