@@ -1,0 +1,420 @@
+#!/usr/bin/env python
+"""Benchmark of libbdscan on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-extra]
+
+A step is one bdscan_allblock call on the 87M-scale all-block training layer
+(batch 16 x 1024 tokens in 32-token blocks, 24 heads x headdim 64, d_state 128,
+one B/C group, bf16 inputs, fp32 state and outputs): the clean forward scan
+with every boundary state, the block-local reverse of both streams, and every
+noisy block continued from the clean boundary state before it - all rows of
+the hot path.  Inputs are seeded synthetic tensors resident in HBM; they are
+larger than L2 (126 MB), so no flush is needed between steps.
+
+Prints one JSON line (rank 0).  For N > 1 (torchrun), every rank runs an
+independent replica on its own GPU (the scan has no cross-GPU exchange);
+timing is the max over ranks of CUDA-event time, and `value` counts the
+tokens of all ranks.  `--impl reference` times the fp64 CPU oracle instead
+(rank 0 only, a bounded sample per step).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from bidirectional_mamba_state_b200 import bdscan as bd  # noqa: E402
+from bidirectional_mamba_state_b200 import roofline as RL  # noqa: E402
+from bidirectional_mamba_state_b200 import workload as W  # noqa: E402
+
+METRIC = "bidir block-scan tokens/s & denoise-step µs; % of HBM / tensor-core roofline"
+WORKLOAD = "87m_allblock"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        p["source"] = "measured"
+        return p
+    except (OSError, ValueError):
+        p = dict(FALLBACK_PEAKS)
+        p["source"] = "fallback"
+        return p
+
+
+# ----------------------------------------------------------------------------- clocks
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+            0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+            0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML (what nvidia-smi
+    reads) every `period` seconds on a background thread."""
+
+    def __init__(self, device_index: int, period: float = 0.01):
+        self.period, self.samples, self.ok = period, [], False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = int(vis.split(",")[device_index]) if vis else device_index
+            self.nv, self.h = pynvml, pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.err = repr(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self) -> dict:
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.err}
+        mask = 0
+        for _, r in self.samples:
+            mask |= r
+        reasons = [n for b, n in _REASONS.items() if mask & b and n != "gpu_idle"]
+        mhz = [m for m, _ in self.samples]
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(mhz)}
+
+
+# ----------------------------------------------------------------------------- distributed
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int, dev) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- workload
+def make_inputs(s: W.Shape, dev):
+    seed = W.SEEDS[WORKLOAD]
+    return W.make_streams(s, seed, device=dev)
+
+
+def cpu_baseline(s: W.Shape, target_s: float = 12.0) -> dict:
+    """The fp64 oracle, as it stands, on the host's cores over a bounded sample
+    of the same workload (a subset of the batch rows, all heads, full length)."""
+    sys.path.insert(0, ROOT)
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    oracle.set_threads(cores)
+    one = s.with_(batch=1)
+    streams = W.make_streams(one, W.SEEDS[WORKLOAD], device="cpu")
+    t0 = time.perf_counter()
+    oracle.allblock(one.as_dict(), *streams)
+    t1 = time.perf_counter() - t0
+    nb = max(1, min(s.batch, int(round(target_s / max(t1, 1e-3)))))
+    sub = s.with_(batch=nb)
+    streams = W.make_streams(sub, W.SEEDS[WORKLOAD], device="cpu")
+    t0 = time.perf_counter()
+    oracle.allblock(sub.as_dict(), *streams)
+    dt = time.perf_counter() - t0
+    return {"value": nb * s.seqlen / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"allblock on {nb} of {s.batch} batch rows x {s.seqlen} tokens x "
+                      f"{s.nheads} heads (fp64, OpenMP over batch x head), {dt:.1f} s"}
+
+
+def run_ours(args):
+    rank, world, local = dist_init()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    s = W.WORKLOADS[WORKLOAD]
+    cf, cr, nf, nr = make_inputs(s, dev)
+    ws = bd.workspace(s, bd.BDSCAN_OP_ALLBLOCK, dev)
+    K = s.nblocks
+    yc = torch.empty((s.batch, s.seqlen, s.nheads, s.headdim), device=dev, dtype=torch.float32)
+    yn = torch.empty_like(yc)
+    st = torch.empty((s.batch, K, s.nheads, s.headdim, s.dstate), device=dev, dtype=torch.float32)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        bd.allblock(s, cf, cr, nf, nr, y_clean=yc, y_noisy=yn, states=st, ws=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    launches_per_step = bd.kernel_launches(s, bd.BDSCAN_OP_ALLBLOCK)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+    ms = e0.elapsed_time(e1)
+    ms = max_over_ranks(ms, world, dev)
+    ms_step = ms / args.steps
+    tokens = s.batch * s.seqlen * world
+    value = tokens / (ms_step * 1e-3)
+
+    pk = peaks()
+    bytes_step = RL.allblock_bytes(s)
+    achieved = bytes_step / (ms_step * 1e-3) / 1e9
+    flops = RL.allblock_flops(s)
+    result = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16-in/fp32-state", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "op": "bdscan_allblock", "batch": s.batch,
+                   "seqlen": s.seqlen, "nheads": s.nheads, "headdim": s.headdim,
+                   "dstate": s.dstate, "ngroups": s.ngroups, "block_len": s.block_len,
+                   "chunk_len": s.chunk_len, "in_dtype": s.in_dtype, "out_dtype": s.out_dtype,
+                   "l2": "inputs larger than L2 (no flush)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                     "algorithmic_bytes_per_launch": bytes_step,
+                     "peak_source": f"{pk['source']} hbm_gbs",
+                     "tensor_tflops": flops / (ms_step * 1e-3) / 1e12,
+                     "tensor_frac_of_bf16": flops / (ms_step * 1e-3) / 1e12 / pk["bf16_tflops"]},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0:
+        result["e2e"] = run_e2e(s, dev, cf, cr, nf, nr, ws, min(args.steps, 10), world)
+    else:
+        run_e2e(s, dev, cf, cr, nf, nr, ws, min(args.steps, 10), world)
+    if rank == 0 and world == 1 and not args.no_extra:
+        result["extra"] = run_extra(dev, pk)
+    if rank == 0 and world == 1 and not args.no_cpu:
+        result["cpu_baseline"] = cpu_baseline(s)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(s, dev, cf, cr, nf, nr, ws, steps, world):
+    """Same step through the public API from pinned host buffers: every step
+    copies that step's inputs host->device, runs allblock, and copies all of its
+    outputs (y_clean, y_noisy, boundary states) device->host."""
+    host = [{k: v.to("cpu").pin_memory() for k, v in d.items()} for d in (cf, cr, nf, nr)]
+    devb = [{k: torch.empty_like(v) for k, v in d.items()} for d in (cf, cr, nf, nr)]
+    K = s.nblocks
+    yc = torch.empty((s.batch, s.seqlen, s.nheads, s.headdim), device=dev, dtype=torch.float32)
+    yn = torch.empty_like(yc)
+    st = torch.empty((s.batch, K, s.nheads, s.headdim, s.dstate), device=dev, dtype=torch.float32)
+    hyc, hyn = torch.empty(yc.shape, pin_memory=True), torch.empty(yn.shape, pin_memory=True)
+    hst = torch.empty(st.shape, pin_memory=True)
+    stream = torch.cuda.current_stream(dev)
+    h2d = sum(v.numel() * v.element_size() for d in host for v in d.values())
+    d2h = sum(t.numel() * t.element_size() for t in (hyc, hyn, hst))
+
+    def step():
+        for hd, dd in zip(host, devb):
+            for k in hd:
+                dd[k].copy_(hd[k], non_blocking=True)
+        bd.allblock(s, *devb, y_clean=yc, y_noisy=yn, states=st, ws=ws, stream=stream)
+        hyc.copy_(yc, non_blocking=True)
+        hyn.copy_(yn, non_blocking=True)
+        hst.copy_(st, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    return {"value": s.batch * s.seqlen * world / (ms * 1e-3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
+            "steps": steps}
+
+
+def _time(fn, dev, reps, warm=3):
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    return e0.elapsed_time(e1) / reps
+
+
+def run_extra(dev, pk) -> dict:
+    """Secondary lines: the denoising step (block_step) over a layer stack captured
+    in one CUDA graph, and prefill of the 700M layer.  Median of 20 graph
+    replays after 5 warm-ups (the pages' own methodology)."""
+    out = {}
+    try:
+        out["block_step_700m_b1_24layers"] = _step_stack(W.WORKLOADS["700m_step"], 24, dev, pk)
+        out["block_step_3b_b1_40layers"] = _step_stack(W.WORKLOADS["3b_step_b1"], 40, dev, pk)
+        out["block_step_3b_b64_40layers"] = _step_stack(W.WORKLOADS["3b_step_b64"], 40, dev, pk)
+        out["prefill_700m_8k_per_layer"] = _prefill(W.WORKLOADS["700m_prefill_8k"], dev, pk)
+    except Exception as e:  # report, never hide
+        out["error"] = repr(e)
+    return out
+
+
+def _step_stack(s: W.Shape, layers: int, dev, pk) -> dict:
+    seed = W.SEEDS["700m_step" if s.nheads == 48 else "3b_step_b1"]
+    ins = [W.make_streams(s, seed, layer, device=dev, streams=(W.CLEAN_FWD, W.CLEAN_REV))
+           for layer in range(layers)]
+    states = [W.make_state(s, seed, layer, device=dev) for layer in range(layers)]
+    ys = [torch.empty((s.batch, s.seqlen, s.nheads, s.headdim), device=dev) for _ in range(layers)]
+    wss = [bd.workspace(s, bd.BDSCAN_OP_BLOCK_STEP, dev) for _ in range(layers)]
+    g_stream = torch.cuda.Stream(dev)
+
+    def stack():
+        for l in range(layers):
+            bd.block_step(s, ins[l][0], ins[l][1], states[l], y=ys[l], ws=wss[l],
+                          stream=torch.cuda.current_stream(dev))
+
+    with torch.cuda.stream(g_stream):
+        stack()
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=g_stream):
+        stack()
+    torch.cuda.synchronize(dev)
+    times = []
+    for _ in range(5):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    for _ in range(20):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        graph.replay()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    b = RL.block_step_bytes(s) * layers
+    del graph
+    return {"us_per_step": ms * 1e3, "tokens_per_s": s.batch * s.seqlen / (ms * 1e-3),
+            "algorithmic_bytes": b, "hbm_frac": b / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+            "layers": layers, "batch": s.batch, "graph": True}
+
+
+def _prefill(s: W.Shape, dev, pk) -> dict:
+    f, r = W.make_streams(s, W.SEEDS["700m_prefill_8k"], device=dev, streams=(W.CLEAN_FWD, W.CLEAN_REV))
+    y = torch.empty((s.batch, s.seqlen, s.nheads, s.headdim), device=dev)
+    fin = torch.empty((s.batch, s.nheads, s.headdim, s.dstate), device=dev)
+    ws = bd.workspace(s, bd.BDSCAN_OP_PREFIX, dev)
+    ms = _time(lambda: bd.prefix(s, f, r, want_states=False, y=y, final=fin, ws=ws), dev, 20, 5)
+    b = RL.prefix_bytes(s, block_states=False)
+    return {"us_per_layer": ms * 1e3, "tokens_per_s": s.batch * s.seqlen / (ms * 1e-3),
+            "algorithmic_bytes": b, "hbm_frac": b / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+
+
+def run_reference(args):
+    """The fp64 CPU oracle as the reference arm: rank 0 only, each step the
+    oracle's allblock on a bounded sample (one batch row, all heads, full
+    length) of the same workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    s = W.WORKLOADS[WORKLOAD]
+    cores = len(os.sched_getaffinity(0))
+    oracle.set_threads(cores)
+    one = s.with_(batch=1)
+    streams = W.make_streams(one, W.SEEDS[WORKLOAD], device="cpu")
+    for _ in range(args.warmup):
+        oracle.allblock(one.as_dict(), *streams)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.allblock(one.as_dict(), *streams)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = one.batch * one.seqlen / dt
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "op": "oracle allblock", "sample_batch": 1,
+                       "batch": s.batch, "seqlen": s.seqlen, "nheads": s.nheads},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"1 of {s.batch} batch rows per step, all heads, full length"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -72,6 +72,8 @@ def lib() -> ctypes.CDLL:
                 getattr(L, fn).restype = ctypes.c_int
             L.bdscan_workspace_size.argtypes = [sp, ctypes.c_int]
             L.bdscan_workspace_size.restype = ctypes.c_size_t
+            L.bdscan_kernel_launches.argtypes = [sp, ctypes.c_int]
+            L.bdscan_kernel_launches.restype = ctypes.c_int
             L.bdscan_check_status.argtypes = [vp, vp]
             L.bdscan_status_string.argtypes = [ctypes.c_int]
             L.bdscan_status_string.restype = ctypes.c_char_p
@@ -103,6 +105,10 @@ def bdscan_allblock(shape, cf, cr, nf, nr, h0, y_clean, y_noisy, block_states, w
 
 def bdscan_workspace_size(shape, op: int) -> int:
     return int(lib().bdscan_workspace_size(shape, op))
+
+
+def bdscan_kernel_launches(shape, op: int) -> int:
+    return int(lib().bdscan_kernel_launches(shape, op))
 
 
 def bdscan_check_status(ws, stream) -> int:
@@ -174,6 +180,11 @@ def workspace(s: Shape, op: int, device) -> torch.Tensor:
     if n == 0:
         raise BdscanError("bdscan_workspace_size", -2, "invalid shape or op")
     return torch.empty(((n + 255) // 256) * 256, dtype=torch.uint8, device=device)
+
+
+def kernel_launches(s: Shape, op: int) -> int:
+    """Kernels one call of ``op`` launches for shape ``s``."""
+    return bdscan_kernel_launches(ctypes.byref(c_shape(s)), op)
 
 
 def _raise(fn, rc):

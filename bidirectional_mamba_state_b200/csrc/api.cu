@@ -152,6 +152,14 @@ size_t bdscan_workspace_size(const bdscan_shape_t *shape, int op) {
   return kStatusBytes;
 }
 
+int bdscan_kernel_launches(const bdscan_shape_t *shape, int op) {
+  if (check_shape(shape) != BDSCAN_OK) return -1;
+  if (op != BDSCAN_OP_PREFIX && op != BDSCAN_OP_BLOCK_STEP && op != BDSCAN_OP_ALLBLOCK) return -1;
+  if (op == BDSCAN_OP_BLOCK_STEP && shape->seqlen != shape->block_len) return -1;
+  if (shape->batch == 0 || shape->seqlen == 0) return 0;
+  return 1;
+}
+
 int bdscan_prefix(const bdscan_shape_t *shape, const bdscan_dir_t *fwd, const bdscan_dir_t *rev,
                   const float *h0, void *y, float *block_states, float *final_state, void *ws,
                   size_t ws_bytes, void *cuda_stream) {

@@ -1,0 +1,65 @@
+"""Algorithmic byte and flop counts of the three operations (the roofline model).
+
+Bytes count every input read once, every output written once and every
+boundary state written once; a re-read of anything is not counted (it is the
+kernel's cost, not the algorithm's).  Flops are those of the chunked form
+with block-sized chunks (the form the tensor-core kernel computes):
+  per (b, h, block) of T tokens:  S = (w o X)^T B  -> 2 T P N    (clean forward)
+                                  Y_off = C h^T      -> 2 T N P    (per forward stream)
+                                  Y_diag = M X       -> 2 T T P    (per direction)
+  per (b, g, block):              C B^T              -> 2 T T N    (per direction)
+This is the memory-bound throughput model of "Breaking the Bottleneck with
+DiffuApriel", section 4.2 (T_max ~ M_p / bytes per token), applied per call.
+"""
+from __future__ import annotations
+
+from .workload import Shape
+
+
+def _elt(dtype: str) -> int:
+    return 2 if dtype == "bf16" else 4
+
+
+def dir_bytes(s: Shape) -> int:
+    e = _elt(s.in_dtype)
+    return e * s.batch * s.seqlen * (s.nheads * s.headdim + s.nheads + 2 * s.ngroups * s.dstate) \
+        + 8 * s.nheads
+
+
+def y_bytes(s: Shape) -> int:
+    return _elt(s.out_dtype) * s.batch * s.seqlen * s.nheads * s.headdim
+
+
+def state_bytes(s: Shape) -> int:
+    return 4 * s.batch * s.nheads * s.headdim * s.dstate
+
+
+def allblock_bytes(s: Shape, with_clean_y: bool = True, with_rev: bool = True) -> int:
+    ndir = 4 if with_rev else 2
+    return ndir * dir_bytes(s) + (2 if with_clean_y else 1) * y_bytes(s) + \
+        s.nblocks * state_bytes(s)
+
+
+def prefix_bytes(s: Shape, with_rev: bool = True, block_states: bool = True,
+                 final_state: bool = True, with_h0: bool = False) -> int:
+    return (2 if with_rev else 1) * dir_bytes(s) + y_bytes(s) + \
+        (s.nblocks * state_bytes(s) if block_states else 0) + \
+        (state_bytes(s) if final_state else 0) + (state_bytes(s) if with_h0 else 0)
+
+
+def block_step_bytes(s: Shape, with_rev: bool = True, commit: bool = False) -> int:
+    return (2 if with_rev else 1) * dir_bytes(s) + y_bytes(s) + state_bytes(s) * (2 if commit else 1)
+
+
+def allblock_flops(s: Shape) -> int:
+    B, H, P, N, G, T, K = s.batch, s.nheads, s.headdim, s.dstate, s.ngroups, s.block_len, s.nblocks
+    per_bhk = 2 * T * P * N + 2 * (2 * T * N * P) + 4 * (2 * T * T * P)
+    per_bgk = 4 * (2 * T * T * N)
+    return B * K * (H * per_bhk + G * per_bgk)
+
+
+def prefix_flops(s: Shape, with_rev: bool = True) -> int:
+    B, H, P, N, G, T, K = s.batch, s.nheads, s.headdim, s.dstate, s.ngroups, s.block_len, s.nblocks
+    nd = 2 if with_rev else 1
+    per_bhk = 2 * T * P * N + 2 * T * N * P + nd * 2 * T * T * P
+    return B * K * (H * per_bhk + G * nd * 2 * T * T * N)

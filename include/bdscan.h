@@ -132,6 +132,11 @@ int bdscan_allblock(const bdscan_shape_t *shape, const bdscan_dir_t *clean_fwd,
  * bytes hold the device status word).  Returns 0 for an invalid shape/op. */
 size_t bdscan_workspace_size(const bdscan_shape_t *shape, int op);
 
+/* Number of kernels one call of `op` launches for this shape (0 for an empty
+ * problem, -1 for an invalid shape/op).  Lets a caller size CUDA graphs and
+ * count launches; it does not launch anything. */
+int bdscan_kernel_launches(const bdscan_shape_t *shape, int op);
+
 /* Reads the device status word in ws after the work queued on cuda_stream
  * completes (synchronises that stream), clears it, and returns it
  * (BDSCAN_OK or BDSCAN_ERR_TIMEOUT).  Returns BDSCAN_ERR_CUDA if the copy fails. */
