@@ -138,7 +138,7 @@ int launch(ScanArgs &a, cudaStream_t stream) {
     }
     return BDSCAN_OK;
   }
-  cudaError_t e = bdscan::launch_seq(a, stream);
+  cudaError_t e = bdscan::tc_supported(a) ? bdscan::launch_tc(a, stream) : bdscan::launch_seq(a, stream);
   return e == cudaSuccess ? BDSCAN_OK : BDSCAN_ERR_CUDA;
 }
 

@@ -34,4 +34,8 @@ struct ScanArgs {
 // shape, fp32 or bf16 inputs, gated or not).
 cudaError_t launch_seq(const ScanArgs &a, cudaStream_t stream);
 
+// Tensor-core path (sm_100a): bf16 inputs, P = 64, N = 128, T = 32, no gate.
+bool tc_supported(const ScanArgs &a);
+cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream);
+
 }  // namespace bdscan

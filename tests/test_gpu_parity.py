@@ -1,6 +1,8 @@
 """GPU parity: the CUDA path through the C ABI against the fp64 oracle on the
 same seeded inputs, plus the invariants that must hold bit-exactly on the
 device (boundary-state independence, state_in untouched, determinism)."""
+import os
+
 import pytest
 import torch
 
@@ -232,3 +234,46 @@ def test_workload_3b_256k_prefill_and_batch64_step():
     ryb, rso = oracle.block_step(sub.as_dict(), pick(af), pick(ar), state[bs][:, hs], want_state_out=True)
     check_y(yb[bs][:, :, hs], ryb)
     check_states(so[bs][:, hs], rso, "commit")
+
+
+# ---------------------------------------------------------------- both device paths
+def _with_env(name, value, fn):
+    old = os.environ.get(name)
+    os.environ[name] = value
+    try:
+        return fn()
+    finally:
+        if old is None:
+            del os.environ[name]
+        else:
+            os.environ[name] = old
+
+
+def test_tensor_core_path_matches_generic_path():
+    """The tcgen05 kernel and the CUDA-core kernel agree on the same inputs
+    (both are also checked against the oracle above)."""
+    s = _shape(batch=3, seqlen=256, nheads=4, ngroups=2)
+    cf, cr, nf, nr = W.make_streams(s, 10, device=DEV)
+    h0 = W.make_state(s, 10, device=DEV)
+    tc = bd.allblock(s, cf, cr, nf, nr, h0=h0)
+    gen = _with_env("BDSCAN_FORCE_GENERIC", "1", lambda: bd.allblock(s, cf, cr, nf, nr, h0=h0))
+    torch.testing.assert_close(tc[0], gen[0], rtol=0, atol=2e-3)
+    torch.testing.assert_close(tc[1], gen[1], rtol=0, atol=2e-3)
+    torch.testing.assert_close(tc[2], gen[2], rtol=1e-4, atol=1e-5)
+
+
+def test_bounded_wait_timeout_reports_status():
+    """With the wait limit forced to zero every bounded wait gives up at once:
+    the kernel reports BDSCAN_ERR_TIMEOUT through the workspace status word and
+    returns; the context stays usable and the next call is correct."""
+    s = _shape(batch=1, seqlen=128)
+    cf, cr, nf, nr = W.make_streams(s, 11, device=DEV)
+    ws = bd.workspace(s, bd.BDSCAN_OP_ALLBLOCK, DEV)
+    stream = torch.cuda.current_stream().cuda_stream
+    _with_env("BDSCAN_WAIT_TIMEOUT_NS", "0", lambda: bd.allblock(s, cf, cr, nf, nr, ws=ws))
+    assert bd.bdscan_check_status(ws.data_ptr(), stream) == -6
+    yc, yn, st = bd.allblock(s, cf, cr, nf, nr, ws=ws)
+    assert bd.bdscan_check_status(ws.data_ptr(), stream) == 0
+    ryc, ryn, rst = oracle.allblock(s.as_dict(), cf, cr, nf, nr)
+    check_y(yn, ryn)
+    check_states(st, rst)
