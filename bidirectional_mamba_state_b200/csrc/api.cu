@@ -149,6 +149,10 @@ extern "C" {
 size_t bdscan_workspace_size(const bdscan_shape_t *shape, int op) {
   if (check_shape(shape) != BDSCAN_OK) return 0;
   if (op != BDSCAN_OP_PREFIX && op != BDSCAN_OP_BLOCK_STEP && op != BDSCAN_OP_ALLBLOCK) return 0;
+  // The tensor-core path keeps C B^T of every (direction, batch, block, group)
+  // in the workspace; shapes it cannot take need only the status word.
+  if (bdscan::tc_shape_ok(shape->headdim, shape->dstate, shape->block_len, shape->in_dtype == BDSCAN_BF16))
+    return bdscan::kWsHeader + bdscan::tc_workspace_bytes(shape->batch, shape->seqlen, shape->ngroups);
   return kStatusBytes;
 }
 
@@ -157,6 +161,9 @@ int bdscan_kernel_launches(const bdscan_shape_t *shape, int op) {
   if (op != BDSCAN_OP_PREFIX && op != BDSCAN_OP_BLOCK_STEP && op != BDSCAN_OP_ALLBLOCK) return -1;
   if (op == BDSCAN_OP_BLOCK_STEP && shape->seqlen != shape->block_len) return -1;
   if (shape->batch == 0 || shape->seqlen == 0) return 0;
+  // tensor-core path: C B^T pre-pass + scan; generic path: one kernel
+  if (bdscan::tc_shape_ok(shape->headdim, shape->dstate, shape->block_len, shape->in_dtype == BDSCAN_BF16))
+    return 2;
   return 1;
 }
 
