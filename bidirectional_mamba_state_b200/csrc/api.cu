@@ -4,6 +4,8 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <utility>
 #include <vector>
@@ -139,7 +141,12 @@ int launch(ScanArgs &a, cudaStream_t stream) {
     return BDSCAN_OK;
   }
   cudaError_t e = bdscan::tc_supported(a) ? bdscan::launch_tc(a, stream) : bdscan::launch_seq(a, stream);
-  return e == cudaSuccess ? BDSCAN_OK : BDSCAN_ERR_CUDA;
+  if (e != cudaSuccess) {
+    const char *v = std::getenv("BDSCAN_VERBOSE");
+    if (v && v[0] == '1') std::fprintf(stderr, "libbdscan: launch failed: %s\n", cudaGetErrorString(e));
+    return BDSCAN_ERR_CUDA;
+  }
+  return BDSCAN_OK;
 }
 
 }  // namespace

@@ -24,15 +24,19 @@
 // Two kernels:
 //   bd_cb_kernel  C B^T of every (direction, batch, block, group) -- shared by
 //                 all heads of a group -- with one M=128 tcgen05 MMA chain per
-//                 four blocks, into the workspace (fp32, 4 KB per block).
+//                 four blocks, into the workspace (bf16, 2 KB per block; the
+//                 masked-decay matrix built from it is rounded to bf16 anyway).
 //   bd_tc_kernel  one CTA per (b, h) walks its blocks in order with the fp32
 //                 state on chip.  Warp roles (448 threads, one CTA per SM):
-//     warp 0      TMA producer: x, B, C and C B^T tiles of block k, 2 stages
+//     warp 0      TMA producers: lane 0 B, C and C B^T tiles (2 stages),
+//                 lane 1 x tiles (3 slots, running further ahead)
 //     warp 1      TMEM allocator and single-thread tcgen05.mma issuer
 //     warps 2-5   operands: decays, (w o X) (bf16 hi + lo), masked-decay M
-//     warps 6-9   state chain: h_k = exp(cum_31) h_{k-1} + S, boundary-state
-//                 stores, h operand (bf16 hi + lo) for the next block
-//     warps 10-13 epilogue: y = exp(cum) Y_off + Y_diag + D x, stores
+//     warps 6-9   state chain: thread n keeps column n of the fp32 state,
+//                 h_k = exp(cum_31) h_{k-1} + S; boundary-state stores (one
+//                 128-byte line per warp instruction); h operand (bf16 hi + lo)
+//     warps 10-13 epilogue: thread (p, stream) forms y[t][p] = exp(cum_t) Y_off
+//                 + Y_diag + D x for the block's 32 tokens and stores them
 //   S, Y, the h operand and M are double-buffered, so the only serial
 //   dependency between blocks is the state recurrence itself.
 // Every wait is bounded; on a timeout the CTA raises BDSCAN_ERR_TIMEOUT in the
@@ -79,10 +83,15 @@ struct CbParams {
   CUtensorMap tc[4];
   int slot[4];  // blockIdx.z -> stacking slot
   int Bsz, K, G;
-  float *cb;    // [4][B][K][G][32 s][32 t]
+  __nv_bfloat16 *cb;  // [4][B][K][G][32 s][32 t]
   int *status;
   unsigned long long timeout_ns;
 };
+
+__device__ __forceinline__ uint32_t pack2(uint32_t lo_bits, uint32_t hi_bits) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(lo_bits), __uint_as_float(hi_bits));
+  return *reinterpret_cast<uint32_t *>(&v);
+}
 
 __global__ void __launch_bounds__(kCbThreads) bd_cb_kernel(const __grid_constant__ CbParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -146,11 +155,11 @@ __global__ void __launch_bounds__(kCbThreads) bd_cb_kernel(const __grid_constant
     tmem_ld_wait();
     if (warp < nvalid) {
       const int64_t idx = ((static_cast<int64_t>(slot) * p.Bsz + b) * p.K + k0 + warp) * p.G + g;
-      float4 *dst = reinterpret_cast<float4 *>(p.cb + idx * 1024 + lane * 32);
+      uint4 *dst = reinterpret_cast<uint4 *>(p.cb + idx * 1024 + lane * 32);
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                             __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+      for (int i = 0; i < 4; ++i)
+        dst[i] = make_uint4(pack2(r[8 * i], r[8 * i + 1]), pack2(r[8 * i + 2], r[8 * i + 3]),
+                            pack2(r[8 * i + 4], r[8 * i + 5]), pack2(r[8 * i + 6], r[8 * i + 7]));
     }
   } else if (lane == 0) {
     atomicCAS(p.status, 0, kStatusTimeout);
@@ -168,37 +177,43 @@ __global__ void __launch_bounds__(kCbThreads) bd_cb_kernel(const __grid_constant
 constexpr int kThreads = 448;
 
 // shared memory map (bytes from a 1024-aligned base)
-constexpr uint32_t kOffX = 0;                 // 4 slots x [32 t][64 p] bf16, SW128
-constexpr uint32_t kOffBcf = 4 * kTile;       // clean-forward B: [32 s][n 0..63], [32 s][n 64..127]
-constexpr uint32_t kOffClo = 6 * kTile;       // [C_cf; C_nf] rows x n 0..63
-constexpr uint32_t kOffChi = 8 * kTile;       // [C_cf; C_nf] rows x n 64..127
-constexpr uint32_t kOffCB = 10 * kTile;       // 4 slots x [32 s][32 t] fp32, SW128
-constexpr uint32_t kStage = 14 * kTile;       // 56 KB per stage
-constexpr uint32_t kOffXw = 2 * kStage;       // hi [32 t][64 p], lo [32 t][64 p] (bf16, SW128)
-constexpr uint32_t kOffH = kOffXw + 2 * kTile;  // 2 buffers x {hi, lo} x {n 0..63, n 64..127} x [64 p][128 B]
-constexpr uint32_t kHBuf = 8 * kTile;           // per buffer: hi at +0, lo at +4 tiles; n-half at +2 tiles
+//   operand ring (2 stages, released by the MMA warp and the operand warps):
+constexpr uint32_t kOffBcf = 0;               // clean-forward B: [32 s][n 0..63], [32 s][n 64..127] (SW128)
+constexpr uint32_t kOffClo = 2 * kTile;       // [C_cf; C_nf] rows x n 0..63 (SW128)
+constexpr uint32_t kOffChi = 4 * kTile;       // [C_cf; C_nf] rows x n 64..127
+constexpr uint32_t kOffCB = 6 * kTile;        // 4 slots x [32 s][32 t] bf16 (SW64), 2 KB each
+constexpr uint32_t kStage = 8 * kTile;        // 32 KB per stage
+//   x ring (3 slots, also read by the epilogue for the D x terms):
+constexpr int kXSlots = 3;
+constexpr uint32_t kOffX = 2 * kStage;        // slot r: 4 dirs x [32 t][64 p] bf16 (SW128)
+constexpr uint32_t kXSlot = 4 * kTile;
+constexpr uint32_t kOffXw = kOffX + kXSlots * kXSlot;  // hi [32 t][64 p], lo [32 t][64 p] (SW128)
+constexpr uint32_t kOffH = kOffXw + 2 * kTile;  // 2 buffers x {hi, lo} x [128 n][64 p] bf16 (SW128)
+constexpr uint32_t kHBuf = 8 * kTile;           // per buffer: hi at +0, lo at +4 tiles
 constexpr uint32_t kOffMh = kOffH + 2 * kHBuf;  // 2 buffers x {fwd, rev} x [64 t][64 s] interleaved
 constexpr uint32_t kMhBuf = 4 * kTile;
-constexpr uint32_t kOffCum = kOffMh + 2 * kMhBuf;  // [2][4][32] f32, log2 units
-constexpr uint32_t kOffDt = kOffCum + 1024;        // [2][4][32] f32
-constexpr uint32_t kOffBar = kOffDt + 1024;
-constexpr int kNumBars = 24;
+constexpr uint32_t kOffCum = kOffMh + 2 * kMhBuf;  // [4 blocks][4 dirs][32] f32: cumulative decay (log2)
+constexpr uint32_t kOffDt = kOffCum + 2048;        // [4][4][32] f32: dt
+constexpr uint32_t kOffEc = kOffDt + 2048;         // [4][2 fwd dirs][32] f32: exp(cum_t)
+constexpr uint32_t kOffBar = kOffEc + 1024;
+constexpr int kNumBars = 32;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
-// masked-decay operand: [64 t][64 s] (block diagonal: first/second direction
-// of the pair), interleaved MN-major (t contiguous): t-groups 128 B apart,
+// masked-decay operand: [64 t][64 s] block diagonal (first/second direction of
+// the pair), interleaved MN-major (t contiguous): t-groups 128 B apart,
 // s-groups 1024 B apart.
 constexpr uint32_t kMhSbo = 128, kMhLbo = 1024;
 
 enum : int {
-  bFull0 = 0, bFull1, bEmpty0, bEmpty1, bAux0, bAux1, bXwFull, bSFull0, bSFull1, bSEmpty0, bSEmpty1,
-  bMhFull0, bMhFull1, bHFull0, bHFull1, bYFull0, bYFull1, bYEmpty0, bYEmpty1, bDrain
+  bFull0 = 0, bFull1, bEmpty0, bEmpty1, bXFull0, bXFull1, bXFull2, bXEmpty0, bXEmpty1, bXEmpty2,
+  bAux0, bAux1, bXwFull, bSFull0, bSFull1, bSEmpty0, bSEmpty1, bMhFull0, bMhFull1, bHFull0, bHFull1,
+  bYFull0, bYFull1, bYEmpty0, bYEmpty1, bDrain, bCount
 };
 
-// TMEM columns: S[2] (M=64 x 128), Y[2] = {Y_off (M=64 x 64), Y_diag (M=64 x 64)}
-constexpr uint32_t kColS0 = 0, kColY0 = 256;
+// TMEM columns: S^T[2] (M=128 x 64), Y^T[2] = {Y_off^T (M=64 x 64), Y_diag^T (M=64 x 64)}
+constexpr uint32_t kColS0 = 0, kColY0 = 128;
 constexpr uint32_t kTmemCols = 512;
 
 struct TcParams {
@@ -231,6 +246,26 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo_f(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi_f(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
+// Element i of a 4-entry kernel-parameter array without dynamic indexing (which
+// would copy the array to local memory).
+template <class T>
+__device__ __forceinline__ T pick4(const T (&a)[4], int i) {
+  return i == 0 ? a[0] : i == 1 ? a[1] : i == 2 ? a[2] : a[3];
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint16_t lds_u16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void sts_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
@@ -239,6 +274,12 @@ __device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t &a, uint32_
                                              uint32_t &d) {
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                : "=r"(a), "=r"(b), "=r"(c), "=r"(d)
+               : "r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ void ld_shared_v4f(uint32_t addr, float (&v)[4]) {
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3])
                : "r"(addr)
                : "memory");
 }
@@ -262,10 +303,11 @@ struct Ctl {
   unsigned long long timeout_ns;
 };
 
-__device__ __noinline__ void raise_timeout(const Ctl &c) {
-  *c.abort = 1;
-  atomicCAS(c.status, 0, kStatusTimeout);
+__device__ __noinline__ void raise_timeout_p(volatile int *abort, int *status) {
+  *abort = 1;
+  atomicCAS(status, 0, kStatusTimeout);
 }
+__device__ __forceinline__ void raise_timeout(const Ctl &c) { raise_timeout_p(c.abort, c.status); }
 
 __device__ __forceinline__ bool wait1(const Ctl &c, int bar, uint32_t parity) {
   if (mbar_wait(&c.bar[bar], parity, c.timeout_ns, c.abort)) return true;
@@ -289,16 +331,18 @@ __device__ __forceinline__ void arrive_lane0(const Ctl &c, int bar) {
 
 // parity of the completion of a double-buffered barrier that block k uses
 __device__ __forceinline__ uint32_t par2(int k) { return (static_cast<uint32_t>(k) >> 1) & 1u; }
+// x ring: slot and parity of block k
+__device__ __forceinline__ int xslot(int k) { return k % kXSlots; }
+__device__ __forceinline__ uint32_t parx(int k) { return static_cast<uint32_t>(k / kXSlots) & 1u; }
 
-// ---------------------------------------------------------------- producer
-__device__ void producer(const TcParams &p, const Ctl &c, uint8_t *sm, int b, int h, int g) {
-  uint32_t bytes = 2 * kTile + (p.allblock ? 4 : 2) * kTile;
-  for (int i = 0; i < 4; ++i)
-    if (p.active[i]) bytes += 2 * kTile;
+// ---------------------------------------------------------------- producers
+// lane 0 of warp 0: B/C/C B^T ring; lane 1: x ring (runs further ahead).
+__device__ void producer_rest(const TcParams &p, const Ctl &c, uint8_t *sm, int b, int g) {
+  const uint32_t bytes = (2 + (p.allblock ? 4 : 2)) * kTile + (p.active[0] + p.active[1] + p.active[2] + p.active[3]) * 2048;
   tma_prefetch_desc(&p.tbcf);
   tma_prefetch_desc(&p.tccf);
   tma_prefetch_desc(&p.tcb);
-  int last_k[2] = {-1, -1};
+  int last0 = -1, last1 = -1;
   for (int k = 0; k < p.K; ++k) {
     const int s = k & 1;
     if (!wait1(c, bEmpty0 + s, par2(k) ^ 1)) break;
@@ -306,12 +350,6 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint8_t *sm, int b, in
     mbar_arrive_expect_tx(full, bytes);
     uint8_t *st = sm + s * kStage;
     const int t0 = k * kT;
-    for (int i = 0; i < 4; ++i) {
-      if (!p.active[i]) continue;
-      tma_load_4d(st + kOffX + i * kTile, &p.tx[i], full, 0, h, t0, b);
-      const int idx = ((i * p.Bsz + b) * p.K + k) * p.G + g;
-      tma_load_3d(st + kOffCB + i * kTile, &p.tcb, full, 0, 0, idx);
-    }
     tma_load_4d(st + kOffBcf, &p.tbcf, full, 0, g, t0, b);
     tma_load_4d(st + kOffBcf + kTile, &p.tbcf, full, 64, g, t0, b);
     tma_load_4d(st + kOffClo, &p.tccf, full, 0, g, t0, b);
@@ -320,37 +358,69 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint8_t *sm, int b, in
       tma_load_4d(st + kOffClo + kTile, &p.tcnf, full, 0, g, t0, b);
       tma_load_4d(st + kOffChi + kTile, &p.tcnf, full, 64, g, t0, b);
     }
-    last_k[s] = k;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (!p.active[i]) continue;
+      const int idx = ((i * p.Bsz + b) * p.K + k) * p.G + g;
+      tma_load_3d(st + kOffCB + i * 2048, &p.tcb, full, 0, 0, idx);
+    }
+    if (s) last1 = k; else last0 = k;
   }
   // no copy into this CTA's shared memory may still be in flight at exit
-  for (int s = 0; s < 2; ++s)
-    if (last_k[s] >= 0) (void)mbar_wait(&c.bar[bFull0 + s], par2(last_k[s]), p.drain_ns, nullptr);
+  if (last0 >= 0) (void)mbar_wait(&c.bar[bFull0], par2(last0), p.drain_ns, nullptr);
+  if (last1 >= 0) (void)mbar_wait(&c.bar[bFull1], par2(last1), p.drain_ns, nullptr);
+}
+
+__device__ void producer_x(const TcParams &p, const Ctl &c, uint8_t *sm, int b, int h) {
+  const uint32_t bytes = (p.active[0] + p.active[1] + p.active[2] + p.active[3]) * kTile;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    if (p.active[i]) tma_prefetch_desc(&p.tx[i]);
+  int last[kXSlots] = {-1, -1, -1};
+  for (int k = 0; k < p.K; ++k) {
+    const int r = xslot(k);
+    if (!wait1(c, bXEmpty0 + r, parx(k) ^ 1)) break;
+    uint64_t *full = &c.bar[bXFull0 + r];
+    mbar_arrive_expect_tx(full, bytes);
+    uint8_t *xs = sm + kOffX + r * kXSlot;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (p.active[i]) tma_load_4d(xs + i * kTile, &p.tx[i], full, 0, h, k * kT, b);
+#pragma unroll
+    for (int j = 0; j < kXSlots; ++j)
+      if (j == r) last[j] = k;
+  }
+#pragma unroll
+  for (int j = 0; j < kXSlots; ++j)
+    if (last[j] >= 0) (void)mbar_wait(&c.bar[bXFull0 + j], parx(last[j]), p.drain_ns, nullptr);
 }
 
 // ---------------------------------------------------------------- MMA issuer
 __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
-  const uint32_t id_s = idesc_bf16(64, 128, 1, 1);  // S[p][n] = (w o X)^T B
-  const uint32_t id_yo = idesc_bf16(64, 64, 0, 0);  // Y_off[t][p] = C h^T
-  const uint32_t id_yd = idesc_bf16(64, 64, 1, 1);  // Y_diag[t][p] = M X
+  const uint32_t id_s = idesc_bf16(128, 64, 1, 1);  // S^T[n][p] = B^T (w o X)
+  const uint32_t id_yo = idesc_bf16(64, 64, 1, 0);  // Y_off^T[p][t] = h C^T
+  const uint32_t id_yd = idesc_bf16(64, 64, 1, 1);  // Y_diag^T[p][t] = X^T M^T
   const bool any_rev = p.active[kCR] || p.active[kNR];
   for (int k = 0; k < p.K; ++k) {
-    const int s = k & 1, i2 = k & 1;
+    const int s = k & 1, i2 = k & 1, r = xslot(k);
     const uint32_t st = base + s * kStage;
+    const uint32_t xs = base + kOffX + r * kXSlot;
     if (!wait1(c, bFull0 + s, par2(k))) break;
-    // ---- S(k) = (w o X)^T B_cf: A MN-major (p), B MN-major (n; halves 4 KB apart)
+    // ---- S^T(k) = B_cf^T (w o X): A MN-major (n; halves 4 KB apart), B MN-major (p)
     if (!wait1(c, bXwFull, k & 1)) break;
     if (k >= 2 && !wait1(c, bSEmpty0 + i2, par2(k - 2))) break;
     tc_fence_after();
-    const uint32_t colS = kColS0 + 128 * i2;
+    const uint32_t colS = kColS0 + 64 * i2;
     for (int ks = 0; ks < 2; ++ks) {
-      const uint64_t ah = sdesc(base + kOffXw + ks * 2048, 0, 1024, kLayoutSw128);
-      const uint64_t al = sdesc(base + kOffXw + kTile + ks * 2048, 0, 1024, kLayoutSw128);
-      const uint64_t bb = sdesc(st + kOffBcf + ks * 2048, kTile, 1024, kLayoutSw128);
-      umma_bf16(tmem + colS, ah, bb, id_s, ks > 0);
-      umma_bf16(tmem + colS, al, bb, id_s, 1);
+      const uint64_t a = sdesc(st + kOffBcf + ks * 2048, kTile, 1024, kLayoutSw128);
+      const uint64_t bh = sdesc(base + kOffXw + ks * 2048, 0, 1024, kLayoutSw128);
+      const uint64_t bl = sdesc(base + kOffXw + kTile + ks * 2048, 0, 1024, kLayoutSw128);
+      umma_bf16(tmem + colS, a, bh, id_s, ks > 0);
+      umma_bf16(tmem + colS, a, bl, id_s, 1);
     }
     umma_commit(&c.bar[bSFull0 + i2]);
-    // ---- Y(k): Y_off = [C_cf; C_nf] h_{k-1}^T, Y_diag = M_fwd X_fwd + M_rev X_rev
+    // ---- Y^T(k): Y_off^T = h_{k-1} [C_cf; C_nf]^T, Y_diag^T = X_fwd^T M_fwd^T + X_rev^T M_rev^T
+    if (!wait1(c, bXFull0 + r, parx(k))) break;
     if (!wait1(c, bMhFull0 + i2, par2(k))) break;
     if (!wait1(c, bHFull0 + ((k + 1) & 1), par2(k))) break;  // h_{k-1} lives in buffer (k-1) & 1
     if (k >= 2 && !wait1(c, bYEmpty0 + i2, par2(k - 2))) break;
@@ -358,28 +428,28 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
     const uint32_t colY = kColY0 + 128 * i2;
     const uint32_t hb = base + kOffH + ((k + 1) & 1) * kHBuf;
     for (int ks = 0; ks < 8; ++ks) {
-      const uint32_t koff = (ks < 4 ? 0 : 2 * kTile) + (ks & 3) * 32;
-      const uint64_t a = sdesc(st + (ks < 4 ? kOffClo : kOffChi) + (ks & 3) * 32, 16, 1024, kLayoutSw128);
-      const uint64_t bh = sdesc(hb + koff, 16, 1024, kLayoutSw128);
-      const uint64_t bl = sdesc(hb + 4 * kTile + koff, 16, 1024, kLayoutSw128);
-      umma_bf16(tmem + colY, a, bh, id_yo, ks > 0);
-      umma_bf16(tmem + colY, a, bl, id_yo, 1);
+      const uint64_t ah = sdesc(hb + ks * 2048, 0, 1024, kLayoutSw128);
+      const uint64_t al = sdesc(hb + 4 * kTile + ks * 2048, 0, 1024, kLayoutSw128);
+      const uint64_t bc = sdesc(st + (ks < 4 ? kOffClo : kOffChi) + (ks & 3) * 32, 16, 1024, kLayoutSw128);
+      umma_bf16(tmem + colY, ah, bc, id_yo, ks > 0);
+      umma_bf16(tmem + colY, al, bc, id_yo, 1);
     }
     const uint32_t mb = base + kOffMh + i2 * kMhBuf;
     for (int ks = 0; ks < 4; ++ks) {
-      const uint64_t a = sdesc(mb + ks * 2048, kMhLbo, kMhSbo, kLayoutNone);
-      const uint64_t bb = sdesc(st + kOffX + ks * 2048, 0, 1024, kLayoutSw128);
-      umma_bf16(tmem + colY + 64, a, bb, id_yd, ks > 0);
+      const uint64_t a = sdesc(xs + ks * 2048, 0, 1024, kLayoutSw128);
+      const uint64_t m = sdesc(mb + ks * 2048, kMhLbo, kMhSbo, kLayoutNone);
+      umma_bf16(tmem + colY + 64, a, m, id_yd, ks > 0);
     }
     if (any_rev) {
       for (int ks = 0; ks < 4; ++ks) {
-        const uint64_t a = sdesc(mb + 2 * kTile + ks * 2048, kMhLbo, kMhSbo, kLayoutNone);
-        const uint64_t bb = sdesc(st + kOffX + 2 * kTile + ks * 2048, 0, 1024, kLayoutSw128);
-        umma_bf16(tmem + colY + 64, a, bb, id_yd, 1);
+        const uint64_t a = sdesc(xs + 2 * kTile + ks * 2048, 0, 1024, kLayoutSw128);
+        const uint64_t m = sdesc(mb + 2 * kTile + ks * 2048, kMhLbo, kMhSbo, kLayoutNone);
+        umma_bf16(tmem + colY + 64, a, m, id_yd, 1);
       }
     }
     umma_commit(&c.bar[bYFull0 + i2]);
     umma_commit(&c.bar[bEmpty0 + s]);
+    umma_commit(&c.bar[bXEmpty0 + r]);
   }
   umma_commit(&c.bar[bDrain]);
   (void)mbar_wait(&c.bar[bDrain], 0, p.drain_ns, nullptr);
@@ -387,17 +457,16 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
 
 // ---------------------------------------------------------------- operand group
 // warps 2..5; q = warp & 3 is the direction slot whose decays and M it builds.
-__device__ void operand_group(const TcParams &p, const Ctl &c, uint8_t *sm, uint32_t base, int b, int h) {
+__device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base, int b, int h) {
   const int lane = threadIdx.x & 31;
   const int q = (threadIdx.x >> 5) & 3;
   const int gt = threadIdx.x - 64;  // 0..127
-  const bool act = p.active[q] != 0;
+  const bool act = pick4(p.active, q) != 0;
   const bool rev = q >= 2;
-  float *cum = reinterpret_cast<float *>(sm + kOffCum);
-  float *dts = reinterpret_cast<float *>(sm + kOffDt);
+  const uint32_t cum = base + kOffCum, dts = base + kOffDt, ecum = base + kOffEc;
   const int64_t H = p.H, L = p.L;
-  const float A2 = act ? p.A[q][h] * kLog2e : 0.f;
-  const __nv_bfloat16 *dtp = p.dt[q];
+  const float A2 = act ? pick4(p.A, q)[h] * kLog2e : 0.f;
+  const __nv_bfloat16 *dtp = pick4(p.dt, q);
   auto load_dt = [&](int k) -> float {
     if (!act || k >= p.K) return 0.f;
     return __bfloat162float(dtp[(static_cast<int64_t>(b) * L + k * kT + lane) * H + h]);
@@ -407,12 +476,14 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint8_t *sm, uint
   const uint32_t mset = rev ? 2 * kTile : 0;
   const uint32_t d0 = (q & 1) ? 32 : 0;
   for (int k = 0; k < p.K; ++k) {
-    const int s = k & 1, i2 = k & 1;
+    const int s = k & 1, i2 = k & 1, c4 = k & 3;
+    const uint32_t xs = base + kOffX + xslot(k) * kXSlot;
     const float dt_cur = dt_next;
     dt_next = load_dt(k + 1);
-    if (!waitw(c, bFull0 + s, par2(k))) break;
+    // ---- decays of this warp's direction (log2 units): prefix sum (forward)
+    //      or suffix sum (reverse) over the block
+    float v = dt_cur * A2;
     if (act) {
-      float v = dt_cur * A2;
       if (!rev) {
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -426,58 +497,66 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint8_t *sm, uint
           if (lane + o < 32) v += u;
         }
       }
-      cum[(s * 4 + q) * 32 + lane] = v;
-      dts[(s * 4 + q) * 32 + lane] = dt_cur;
+      sts_f32(cum + ((c4 * 4 + q) * 32 + lane) * 4, v);
+      sts_f32(dts + ((c4 * 4 + q) * 32 + lane) * 4, dt_cur);
+      if (!rev) sts_f32(ecum + ((c4 * 2 + q) * 32 + lane) * 4, exp2f(v));
     }
     arrive_lane0(c, bAux0 + s);
     if (!waitw(c, bAux0 + s, par2(k))) break;
     // ---- (w o X) of the clean forward direction, bf16 hi + lo
-    if (k >= 1 && !waitw(c, bSFull0 + ((k + 1) & 1), par2(k - 1))) break;
+    if (k >= 1 && !waitw(c, bSFull0 + ((k + 1) & 1), par2(k - 1))) break;  // S(k-1) read Xw
+    if (!waitw(c, bXFull0 + xslot(k), parx(k))) break;
     {
-      const float *cf = cum + (s * 4 + kCF) * 32;
-      const float *df = dts + (s * 4 + kCF) * 32;
-      const float c31 = cf[31];
+      const uint32_t cf = cum + (c4 * 4 + kCF) * 128, df = dts + (c4 * 4 + kCF) * 128;
+      const float c31 = lds_f32(cf + 31 * 4);
 #pragma unroll
       for (int rep = 0; rep < 2; ++rep) {
         const int i = gt + 128 * rep;
         const int t = i >> 3, ch = i & 7;
         const uint32_t off = sw128_chunk(t, ch);
         uint32_t r0, r1, r2, r3;
-        ld_shared_v4(base + s * kStage + kOffX + off, r0, r1, r2, r3);
-        const float w = df[t] * exp2f(c31 - cf[t]);
-        float v[8] = {bf16_lo_f(r0) * w, bf16_hi_f(r0) * w, bf16_lo_f(r1) * w, bf16_hi_f(r1) * w,
-                      bf16_lo_f(r2) * w, bf16_hi_f(r2) * w, bf16_lo_f(r3) * w, bf16_hi_f(r3) * w};
-        store_split8(base + kOffXw + off, base + kOffXw + kTile + off, v);
+        ld_shared_v4(xs + off, r0, r1, r2, r3);
+        const float w = lds_f32(df + t * 4) * exp2f(c31 - lds_f32(cf + t * 4));
+        float vv[8] = {bf16_lo_f(r0) * w, bf16_hi_f(r0) * w, bf16_lo_f(r1) * w, bf16_hi_f(r1) * w,
+                       bf16_lo_f(r2) * w, bf16_hi_f(r2) * w, bf16_lo_f(r3) * w, bf16_hi_f(r3) * w};
+        store_split8(base + kOffXw + off, base + kOffXw + kTile + off, vv);
       }
       fence_proxy_async_smem();
       arrive_lane0(c, bXwFull);
     }
     // ---- masked-decay matrix, row s = lane of M^T for this direction
-    if (k >= 2 && !waitw(c, bYFull0 + i2, par2(k - 2))) break;
+    if (!waitw(c, bFull0 + s, par2(k))) break;
+    if (k >= 2 && !waitw(c, bYFull0 + i2, par2(k - 2))) break;  // Y(k-2) read this M buffer
     if (act) {
-      const uint32_t cbrow = base + s * kStage + kOffCB + q * kTile + lane * 128;
+      const uint32_t cbrow = base + s * kStage + kOffCB + q * 2048;
       float cbv[32];
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
+      for (int ch = 0; ch < 4; ++ch) {
         uint32_t r0, r1, r2, r3;
-        ld_shared_v4(cbrow + ((ch ^ (lane & 7)) << 4), r0, r1, r2, r3);
-        cbv[4 * ch] = __uint_as_float(r0);
-        cbv[4 * ch + 1] = __uint_as_float(r1);
-        cbv[4 * ch + 2] = __uint_as_float(r2);
-        cbv[4 * ch + 3] = __uint_as_float(r3);
+        ld_shared_v4(cbrow + sw64_chunk(lane, ch), r0, r1, r2, r3);
+        cbv[8 * ch] = bf16_lo_f(r0);
+        cbv[8 * ch + 1] = bf16_hi_f(r0);
+        cbv[8 * ch + 2] = bf16_lo_f(r1);
+        cbv[8 * ch + 3] = bf16_hi_f(r1);
+        cbv[8 * ch + 4] = bf16_lo_f(r2);
+        cbv[8 * ch + 5] = bf16_hi_f(r2);
+        cbv[8 * ch + 6] = bf16_lo_f(r3);
+        cbv[8 * ch + 7] = bf16_hi_f(r3);
       }
-      const float *cq = cum + (s * 4 + q) * 32;
-      const float cs = cq[lane];
-      const float ds = dts[(s * 4 + q) * 32 + lane];
+      const uint32_t cq = cum + (c4 * 4 + q) * 128;
+      const float cs = v, ds = dt_cur;
       const uint32_t mrow = base + kOffMh + i2 * kMhBuf + mset;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
+        float cj[8];
+        ld_shared_v4f(cq + 32 * j, *reinterpret_cast<float(*)[4]>(&cj[0]));
+        ld_shared_v4f(cq + 32 * j + 16, *reinterpret_cast<float(*)[4]>(&cj[4]));
         float m[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int t = 8 * j + i;
           const bool valid = rev ? (t <= lane) : (t >= lane);
-          const float e = exp2f(cq[t] - cs);
+          const float e = exp2f(cj[i] - cs);
           m[i] = valid ? cbv[t] * ds * e : 0.f;
         }
         st_shared_v4(mrow + inter_mn_off(d0 + 8 * j, d0 + lane, kMhSbo, kMhLbo), pack_bf16x2(m[0], m[1]),
@@ -487,40 +566,31 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint8_t *sm, uint
     fence_proxy_async_smem();
     arrive_lane0(c, bMhFull0 + i2);
     arrive_lane0(c, bEmpty0 + s);
+    arrive_lane0(c, bXEmpty0 + xslot(k));
   }
 }
 
 // ---------------------------------------------------------------- state group
-// warps 6..9: thread owns h[p][n0 .. n0+63], p = 16 q + (lane & 15), n0 = 64 (lane >> 4).
-__device__ void state_group(const TcParams &p, const Ctl &c, uint8_t *sm, uint32_t base, uint32_t tmem,
-                            int b, int h) {
+// warps 6..9: thread owns column n = 32 q + lane of the state, h^T[n][0..63].
+__device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem, int b, int h) {
   const int lane = threadIdx.x & 31;
   const int q = (threadIdx.x >> 5) & 3;
-  const int prow = 16 * q + (lane & 15);
-  const int half = lane >> 4;
-  const int n0 = 64 * half;
-  const float *cum = reinterpret_cast<const float *>(sm + kOffCum);
+  const int n = 32 * q + lane;
+  const uint32_t cum = base + kOffCum;
   const int64_t H = p.H;
   const int64_t PN = kP * kN;
-  float hreg[64];
+  float hreg[kP];
   {
-    const float *src = p.h0 ? p.h0 + (static_cast<int64_t>(b) * H + h) * PN + prow * kN + n0 : nullptr;
+    const float *src = p.h0 ? p.h0 + (static_cast<int64_t>(b) * H + h) * PN + n : nullptr;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float4 v = src ? reinterpret_cast<const float4 *>(src)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-      hreg[4 * i] = v.x;
-      hreg[4 * i + 1] = v.y;
-      hreg[4 * i + 2] = v.z;
-      hreg[4 * i + 3] = v.w;
-    }
+    for (int pp = 0; pp < kP; ++pp) hreg[pp] = src ? src[pp * kN] : 0.f;
   }
-  // h operand of Y_off (K-major, SW128): buffer hbuf holds {hi: n 0..63, n 64..127;
-  // lo: n 0..63, n 64..127}, each [64 p rows][128 B].
+  // h operand of Y_off^T (A, MN-major): buffer hbuf, {hi, lo} x [128 n rows][64 p] (SW128)
   auto write_h = [&](int hbuf) {
-    const uint32_t hb = base + kOffH + hbuf * kHBuf + half * 2 * kTile;
+    const uint32_t hb = base + kOffH + hbuf * kHBuf;
 #pragma unroll
     for (int cc = 0; cc < 8; ++cc) {
-      const uint32_t off = sw128_chunk(prow, cc);
+      const uint32_t off = sw128_chunk(n, cc);
       store_split8(hb + off, hb + 4 * kTile + off, hreg + 8 * cc);
     }
     fence_proxy_async_smem();
@@ -528,69 +598,62 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint8_t *sm, uint32
   };
   write_h(1);  // h_{-1} lives in buffer 1
   for (int k = 0; k < p.K; ++k) {
-    const int s = k & 1, i2 = k & 1;
-    if (!waitw(c, bAux0 + s, par2(k))) break;
-    const float atot = exp2f(cum[(s * 4 + kCF) * 32 + 31]);
+    const int i2 = k & 1, c4 = k & 3;
+    if (!waitw(c, bAux0 + (k & 1), par2(k))) break;
+    const float atot = exp2f(lds_f32(cum + ((c4 * 4 + kCF) * 32 + 31) * 4));
     if (!waitw(c, bSFull0 + i2, par2(k))) break;
     tc_fence_after();
     {
       uint32_t sv[32];
-      const uint32_t ta = tmem_addr(tmem, 32 * q, kColS0 + 128 * i2);
-      tmem_ld_16x32bx2_x32<64>(ta, sv);
+      const uint32_t ta = tmem_addr(tmem, 32 * q, kColS0 + 64 * i2);
+      tmem_ld_32x32b_x32(ta, sv);
       tmem_ld_wait();
 #pragma unroll
       for (int i = 0; i < 32; ++i) hreg[i] = fmaf(atot, hreg[i], __uint_as_float(sv[i]));
-      tmem_ld_16x32bx2_x32<64>(ta + 32, sv);
+      tmem_ld_32x32b_x32(ta + 32, sv);
       tmem_ld_wait();
 #pragma unroll
       for (int i = 0; i < 32; ++i) hreg[32 + i] = fmaf(atot, hreg[32 + i], __uint_as_float(sv[i]));
     }
     tc_fence_before();
     arrive_lane0(c, bSEmpty0 + i2);
-    arrive_lane0(c, bEmpty0 + s);
-    if (p.states) {
-      float4 *dst = reinterpret_cast<float4 *>(p.states + ((static_cast<int64_t>(b) * p.K + k) * H + h) * PN +
-                                               prow * kN + n0);
-#pragma unroll
-      for (int i = 0; i < 16; ++i)
-        dst[i] = make_float4(hreg[4 * i], hreg[4 * i + 1], hreg[4 * i + 2], hreg[4 * i + 3]);
-    }
     // buffer k & 1 held h_{k-2}; Y(k-1) has read it once y_full(k-1) completes
     if (k >= 1 && !waitw(c, bYFull0 + ((k + 1) & 1), par2(k - 1))) break;
     write_h(k & 1);
+    if (p.states) {  // each warp instruction stores one contiguous 128-byte row segment
+      float *dst = p.states + ((static_cast<int64_t>(b) * p.K + k) * H + h) * PN + n;
+#pragma unroll
+      for (int pp = 0; pp < kP; ++pp) dst[pp * kN] = hreg[pp];
+    }
   }
   if (p.final_state && !*c.abort) {
-    float4 *dst =
-        reinterpret_cast<float4 *>(p.final_state + (static_cast<int64_t>(b) * H + h) * PN + prow * kN + n0);
+    float *dst = p.final_state + (static_cast<int64_t>(b) * H + h) * PN + n;
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
-      dst[i] = make_float4(hreg[4 * i], hreg[4 * i + 1], hreg[4 * i + 2], hreg[4 * i + 3]);
+    for (int pp = 0; pp < kP; ++pp) dst[pp * kN] = hreg[pp];
   }
 }
 
 // ---------------------------------------------------------------- epilogue
-// warps 10..13: accumulator row r = 16 q + (lane & 15) is token t = r & 31 of the
-// clean (r < 32) or noisy (r >= 32) stream; columns p0 .. p0+31, p0 = 32 (lane >> 4).
-__device__ void epilogue_group(const TcParams &p, const Ctl &c, uint8_t *sm, uint32_t base, uint32_t tmem,
-                               int b, int h) {
+// warps 10..13: thread owns column p = 16 q + (lane & 15) of the clean
+// (lane < 16) or noisy (lane >= 16) stream's outputs y[t][p], t = 0..31.
+__device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem, int b, int h) {
   const int lane = threadIdx.x & 31;
   const int q = (threadIdx.x >> 5) & 3;
-  const int row = 16 * q + (lane & 15);
-  const int t = row & 31;
-  const bool noisy = row >= 32;
-  const int p0 = 32 * (lane >> 4);
-  const float *cum = reinterpret_cast<const float *>(sm + kOffCum);
+  const int pcol = 16 * q + (lane & 15);
+  const bool noisy = lane >= 16;
   const int fs = noisy ? kNF : kCF, rs = noisy ? kNR : kCR;
   void *yout = noisy ? p.y_noisy : p.y_clean;
   const bool mine = (noisy ? p.allblock != 0 : true) && yout != nullptr;
-  const bool has_rev = p.active[rs] != 0;
-  const float Df = p.active[fs] ? p.D[fs][h] : 0.f;
-  const float Dr = has_rev ? p.D[rs][h] : 0.f;
+  const bool has_rev = pick4(p.active, rs) != 0;
+  const float Df = pick4(p.active, fs) ? pick4(p.D, fs)[h] : 0.f;
+  const float Dr = has_rev ? pick4(p.D, rs)[h] : 0.f;
+  const uint32_t ecum = base + kOffEc;
   const int64_t H = p.H, L = p.L;
   for (int k = 0; k < p.K; ++k) {
-    const int s = k & 1, i2 = k & 1;
-    if (!waitw(c, bFull0 + s, par2(k))) break;
-    if (!waitw(c, bAux0 + s, par2(k))) break;
+    const int i2 = k & 1, c4 = k & 3;
+    const uint32_t xs = base + kOffX + xslot(k) * kXSlot;
+    if (!waitw(c, bAux0 + (k & 1), par2(k))) break;
+    if (!waitw(c, bXFull0 + xslot(k), parx(k))) break;
     if (!waitw(c, bYFull0 + i2, par2(k))) break;
     tc_fence_after();
     uint32_t yo[32], yd[32];
@@ -601,43 +664,35 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint8_t *sm, uin
     tc_fence_before();
     arrive_lane0(c, bYEmpty0 + i2);
     if (mine) {
-      const float e = exp2f(cum[(s * 4 + fs) * 32 + t]);
-      const uint32_t xf = base + s * kStage + kOffX + fs * kTile;
-      const uint32_t xr = base + s * kStage + kOffX + rs * kTile;
-      float y[32];
+      const uint32_t eq = ecum + (c4 * 2 + fs) * 128;
+      const uint32_t xf = xs + fs * kTile, xr = xs + rs * kTile;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const uint32_t ch = (p0 >> 3) + cc;
-        uint32_t f[4], r[4] = {0, 0, 0, 0};
-        ld_shared_v4(xf + sw128_chunk(t, ch), f[0], f[1], f[2], f[3]);
-        if (has_rev) ld_shared_v4(xr + sw128_chunk(t, ch), r[0], r[1], r[2], r[3]);
+      for (int j = 0; j < 8; ++j) {
+        float e4[4];
+        ld_shared_v4f(eq + 16 * j, e4);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int j = 8 * cc + 2 * i;
-          float v0 = fmaf(e, __uint_as_float(yo[j]), __uint_as_float(yd[j]));
-          float v1 = fmaf(e, __uint_as_float(yo[j + 1]), __uint_as_float(yd[j + 1]));
-          v0 = fmaf(Df, bf16_lo_f(f[i]), v0);
-          v1 = fmaf(Df, bf16_hi_f(f[i]), v1);
-          v0 = fmaf(Dr, bf16_lo_f(r[i]), v0);
-          v1 = fmaf(Dr, bf16_hi_f(r[i]), v1);
-          y[j] = v0;
-          y[j + 1] = v1;
+          const int t = 4 * j + i;
+          const uint32_t xo = sw128_off(t, pcol);
+          float y = fmaf(e4[i], __uint_as_float(yo[t]), __uint_as_float(yd[t]));
+          y = fmaf(Df, __uint_as_float(static_cast<uint32_t>(lds_u16(xf + xo)) << 16), y);
+          if (has_rev) y = fmaf(Dr, __uint_as_float(static_cast<uint32_t>(lds_u16(xr + xo)) << 16), y);
+          yo[t] = __float_as_uint(y);
         }
       }
-      const int64_t yi = ((static_cast<int64_t>(b) * L + k * kT + t) * H + h) * kP + p0;
+      const int64_t yi = ((static_cast<int64_t>(b) * L + k * kT) * H + h) * kP + pcol;
+      const int64_t tstride = H * kP;
       if (p.out_bf16) {
-        uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(yout) + yi);
+        __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(yout) + yi;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          dst[i] = make_uint4(pack_bf16x2(y[8 * i], y[8 * i + 1]), pack_bf16x2(y[8 * i + 2], y[8 * i + 3]),
-                              pack_bf16x2(y[8 * i + 4], y[8 * i + 5]), pack_bf16x2(y[8 * i + 6], y[8 * i + 7]));
+        for (int t = 0; t < 32; ++t) dst[t * tstride] = __float2bfloat16_rn(__uint_as_float(yo[t]));
       } else {
-        float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(yout) + yi);
+        float *dst = reinterpret_cast<float *>(yout) + yi;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) dst[i] = make_float4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
+        for (int t = 0; t < 32; ++t) dst[t * tstride] = __uint_as_float(yo[t]);
       }
     }
-    arrive_lane0(c, bEmpty0 + s);
+    arrive_lane0(c, bXEmpty0 + xslot(k));
   }
 }
 
@@ -655,21 +710,32 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(sm + kOffMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kOffMisc + 4);
   if (threadIdx.x == 0) {
-    const uint32_t counts[bDrain + 1] = {1, 1, 13, 13, 4, 4, 4, 1, 1, 4, 4, 4, 4, 4, 4, 1, 1, 4, 4, 1};
-    for (int i = 0; i <= bDrain; ++i) mbar_init(&bars[i], counts[i]);
+    // arrival counts: full = producer; empty = MMA commit + 4 operand warps;
+    // x empty = MMA commit + 4 operand warps + 4 epilogue warps; the rest as named
+    for (int i = 0; i < bCount; ++i) {
+      uint32_t cnt = 4;
+      if (i == bFull0 || i == bFull1 || i == bXFull0 || i == bXFull1 || i == bXFull2 || i == bSFull0 ||
+          i == bSFull1 || i == bYFull0 || i == bYFull1 || i == bDrain)
+        cnt = 1;
+      else if (i == bEmpty0 || i == bEmpty1)
+        cnt = 5;
+      else if (i == bXEmpty0 || i == bXEmpty1 || i == bXEmpty2)
+        cnt = 9;
+      mbar_init(&bars[i], cnt);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  // Tiles that are never loaded are read by MMAs next to zero operands: clear
-  // them (and both masked-decay buffers, whose off-diagonal blocks stay zero) so
-  // that no uninitialised NaN/Inf bit pattern can reach an output.
+  // x tiles of inactive directions are read next to zero operands by the MMAs:
+  // clear them (and the masked-decay buffers, whose off-diagonal blocks stay
+  // zero) so that no uninitialised NaN/Inf bit pattern can reach an output.
   {
     const uint4 zero = make_uint4(0, 0, 0, 0);
     for (int i = 0; i < 4; ++i) {
       if (p.active[i]) continue;
-      for (int s = 0; s < 2; ++s)
+      for (int r = 0; r < kXSlots; ++r)
         for (uint32_t o = threadIdx.x * 16; o < kTile; o += kThreads * 16)
-          *reinterpret_cast<uint4 *>(sm + s * kStage + kOffX + i * kTile + o) = zero;
+          *reinterpret_cast<uint4 *>(sm + kOffX + r * kXSlot + i * kTile + o) = zero;
     }
     if (!p.allblock)
       for (int s = 0; s < 2; ++s)
@@ -692,15 +758,17 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
   Ctl c{bars, abort_flag, p.status, p.timeout_ns};
 
   if (warp == 0) {
-    if ((threadIdx.x & 31) == 0) producer(p, c, sm, b, h, g);
+    const int lane = threadIdx.x & 31;
+    if (lane == 0) producer_rest(p, c, sm, b, g);
+    else if (lane == 1) producer_x(p, c, sm, b, h);
   } else if (warp == 1) {
     if ((threadIdx.x & 31) == 0) mma_issuer(p, c, base, tmem);
   } else if (warp < 6) {
-    operand_group(p, c, sm, base, b, h);
+    operand_group(p, c, base, b, h);
   } else if (warp < 10) {
-    state_group(p, c, sm, base, tmem, b, h);
+    state_group(p, c, base, tmem, b, h);
   } else {
-    epilogue_group(p, c, sm, base, tmem, b, h);
+    epilogue_group(p, c, base, tmem, b, h);
   }
   tc_fence_before();
   __syncthreads();
@@ -738,16 +806,16 @@ bool make_map_bf16(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, ui
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// fp32 C B^T tiles [n][32][32], box (32, 32, 1), 128-byte swizzle.
+// bf16 C B^T tiles [n][32][32], box (32, 32, 1), 64-byte swizzle.
 bool make_map_cb(CUtensorMap *m, const void *ptr, uint64_t ntiles) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {32, 32, ntiles};
-  cuuint64_t strides[2] = {32 * 4, 32 * 32 * 4};
+  cuuint64_t strides[2] = {32 * 2, 32 * 32 * 2};
   cuuint32_t box[3] = {32, 32, 1};
   cuuint32_t es[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void *>(ptr), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -779,7 +847,7 @@ bool tc_shape_ok(int64_t P, int64_t N, int64_t T, bool in_bf16) {
 }
 
 size_t tc_workspace_bytes(int64_t Bsz, int64_t L, int64_t G) {
-  return static_cast<size_t>(4) * Bsz * (L / kT) * G * kTile;
+  return static_cast<size_t>(4) * Bsz * (L / kT) * G * 2048;  // bf16 [32][32] per (dir, b, block, g)
 }
 
 bool tc_supported(const ScanArgs &a) {
@@ -800,7 +868,7 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
   const bool all = a.mode == Mode::AllBlock;
   const DirArgs *ds[4] = {&a.cf, all ? &a.nf : nullptr, a.has_cr ? &a.cr : nullptr,
                           (all && a.has_nr) ? &a.nr : nullptr};
-  float *cbws = reinterpret_cast<float *>(static_cast<uint8_t *>(a.ws) + kWsHeader);
+  __nv_bfloat16 *cbws = reinterpret_cast<__nv_bfloat16 *>(static_cast<uint8_t *>(a.ws) + kWsHeader);
   const unsigned long long timeout = env_ns("BDSCAN_WAIT_TIMEOUT_NS", 2000000000ull);
   const int K = static_cast<int>(a.L / kT);
 

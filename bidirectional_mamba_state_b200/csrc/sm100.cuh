@@ -52,6 +52,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that lets the hardware suspend the thread for up to `hint_ns`
+// while the phase is incomplete, so waiting warps do not take issue slots
+// from working ones.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, "
+      "p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity.  Gives up (returns false)
 // once `timeout_ns` has passed without the phase completing, or as soon as
 // `*abort` (if given) is set by another thread of the CTA; never spins forever.
@@ -59,12 +73,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
                                           const volatile int *abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t deadline = globaltimer_ns() + timeout_ns;
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 15u) == 0) {
-      if (abort && *abort) return false;
-      if (globaltimer_ns() > deadline) return false;
-    }
+  const uint32_t hint = timeout_ns < 20000 ? static_cast<uint32_t>(timeout_ns) : 20000u;
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, hint)) return true;
+    if (abort && *abort) return false;
+    if (globaltimer_ns() > deadline) return false;
   }
 }
 
@@ -220,6 +233,13 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar) {
 // and the SW128 UMMA descriptors read (tile base 1024-byte aligned).
 __host__ __device__ __forceinline__ uint32_t sw128_off(uint32_t row, uint32_t col) {
   return row * 128u + ((((col >> 3) ^ (row & 7u)) & 7u) << 4) + ((col & 7u) << 1);
+}
+
+// Byte offset of 16-byte chunk `chunk` (0..3) of row `row` of a tile with
+// 64-byte rows in the 64-byte-swizzled layout TMA SWIZZLE_64B writes (tile
+// base 512-byte aligned).
+__host__ __device__ __forceinline__ uint32_t sw64_chunk(uint32_t row, uint32_t chunk) {
+  return row * 64u + (((chunk ^ (row >> 1)) & 3u) << 4);
 }
 
 // Byte offset of 16-byte chunk `chunk` (elements 8*chunk .. 8*chunk+7) of row `row`.
