@@ -28,17 +28,18 @@
 //                 masked-decay matrix built from it is rounded to bf16 anyway).
 //   bd_tc_kernel  one CTA per (b, h) walks its blocks in order with the fp32
 //                 state on chip.  Warp roles (448 threads, one CTA per SM):
-//     warp 0      TMA producers: lane 0 B, C and C B^T tiles (2 stages),
-//                 lane 1 x tiles (3 slots, running further ahead)
+//     warp 0      TMA producer: x, B, C and C B^T tiles of block k into a
+//                 3-slot ring (two blocks of lookahead)
 //     warp 1      TMEM allocator and single-thread tcgen05.mma issuer
 //     warps 2-5   operands: decays, (w o X) (bf16 hi + lo), masked-decay M
 //     warps 6-9   state chain: thread n keeps column n of the fp32 state,
 //                 h_k = exp(cum_31) h_{k-1} + S; boundary-state stores (one
 //                 128-byte line per warp instruction); h operand (bf16 hi + lo)
 //     warps 10-13 epilogue: thread (p, stream) forms y[t][p] = exp(cum_t) Y_off
-//                 + Y_diag + D x for the block's 32 tokens and stores them
-//   S, Y, the h operand and M are double-buffered, so the only serial
-//   dependency between blocks is the state recurrence itself.
+//                 + Y_diag for the block's 32 tokens and stores them; the D x
+//                 terms are small tensor-core products against D I_16 (bf16
+//                 hi + lo) accumulated into Y_diag
+//   S, Y and M are double-buffered; the h operand is single-buffered.
 // Every wait is bounded; on a timeout the CTA raises BDSCAN_ERR_TIMEOUT in the
 // workspace status word, drains its own copies and MMAs, frees TMEM and exits.
 //
@@ -177,29 +178,31 @@ __global__ void __launch_bounds__(kCbThreads) bd_cb_kernel(const __grid_constant
 constexpr int kThreads = 448;
 
 // shared memory map (bytes from a 1024-aligned base)
-//   operand ring (2 stages, released by the MMA warp and the operand warps):
-constexpr uint32_t kOffBcf = 0;               // clean-forward B: [32 s][n 0..63], [32 s][n 64..127] (SW128)
-constexpr uint32_t kOffClo = 2 * kTile;       // [C_cf; C_nf] rows x n 0..63 (SW128)
-constexpr uint32_t kOffChi = 4 * kTile;       // [C_cf; C_nf] rows x n 64..127
-constexpr uint32_t kOffCB = 6 * kTile;        // 4 slots x [32 s][32 t] bf16 (SW64), 2 KB each
-constexpr uint32_t kStage = 8 * kTile;        // 32 KB per stage
-//   x ring (3 slots, also read by the epilogue for the D x terms):
-constexpr int kXSlots = 3;
-constexpr uint32_t kOffX = 2 * kStage;        // slot r: 4 dirs x [32 t][64 p] bf16 (SW128)
-constexpr uint32_t kXSlot = 4 * kTile;
-constexpr uint32_t kOffXw = kOffX + kXSlots * kXSlot;  // hi [32 t][64 p], lo [32 t][64 p] (SW128)
-constexpr uint32_t kOffH = kOffXw + 2 * kTile;  // 2 buffers x {hi, lo} x [128 n][64 p] bf16 (SW128)
-constexpr uint32_t kHBuf = 8 * kTile;           // per buffer: hi at +0, lo at +4 tiles
-constexpr uint32_t kOffMh = kOffH + 2 * kHBuf;  // 2 buffers x {fwd, rev} x [64 t][64 s] interleaved
+//   TMA ring, 3 slots (two blocks of lookahead); slot r holds block k = r mod 3:
+constexpr int kSlots = 3;
+constexpr uint32_t kOffX = 0;                 // 4 dirs x [32 t][64 p] bf16 (SW128)
+constexpr uint32_t kOffBcf = 4 * kTile;       // clean-forward B: [32 s][n 0..63], [32 s][n 64..127] (SW128)
+constexpr uint32_t kOffClo = 6 * kTile;       // [C_cf; C_nf] rows x n 0..63 (SW128)
+constexpr uint32_t kOffChi = 8 * kTile;       // [C_cf; C_nf] rows x n 64..127
+constexpr uint32_t kOffCB = 10 * kTile;       // 4 dirs x [32 s][32 t] bf16 (SW64), 2 KB each
+constexpr uint32_t kSlot = 12 * kTile;        // 48 KB per slot
+constexpr uint32_t kOffXw = kSlots * kSlot;   // hi [32 t][64 p], lo [32 t][64 p] (bf16, SW128)
+constexpr uint32_t kOffH = kOffXw + 2 * kTile;  // {hi, lo} x [128 n][64 p] bf16 (SW128)
+constexpr uint32_t kOffMh = kOffH + 8 * kTile;  // 2 buffers x {fwd, rev} x [64 t][64 s] interleaved
 constexpr uint32_t kMhBuf = 4 * kTile;
-constexpr uint32_t kOffCum = kOffMh + 2 * kMhBuf;  // [4 blocks][4 dirs][32] f32: cumulative decay (log2)
-constexpr uint32_t kOffDt = kOffCum + 2048;        // [4][4][32] f32: dt
-constexpr uint32_t kOffEc = kOffDt + 2048;         // [4][2 fwd dirs][32] f32: exp(cum_t)
+constexpr uint32_t kOffDg = kOffMh + 2 * kMhBuf;  // 4 dirs x {hi, lo} x D I_16 (bf16, 512 B each)
+constexpr uint32_t kOffCum = kOffDg + 4096;       // [4 blocks][4 dirs][32] f32: cumulative decay (log2)
+constexpr uint32_t kOffDt = kOffCum + 2048;       // [4][4][32] f32: dt
+constexpr uint32_t kOffEc = kOffDt + 2048;        // [4][2 fwd dirs][32] f32: exp(cum_t)
 constexpr uint32_t kOffBar = kOffEc + 1024;
 constexpr int kNumBars = 32;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+// D I_16 operand (B of the D x MMAs): [16 t][16 s] interleaved K-major, 8x8 core
+// matrices, t-groups 128 B apart, s-groups 256 B apart.
+constexpr uint32_t kDgSbo = 128, kDgLbo = 256;
 
 // masked-decay operand: [64 t][64 s] block diagonal (first/second direction of
 // the pair), interleaved MN-major (t contiguous): t-groups 128 B apart,
@@ -207,9 +210,8 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 constexpr uint32_t kMhSbo = 128, kMhLbo = 1024;
 
 enum : int {
-  bFull0 = 0, bFull1, bEmpty0, bEmpty1, bXFull0, bXFull1, bXFull2, bXEmpty0, bXEmpty1, bXEmpty2,
-  bAux0, bAux1, bXwFull, bSFull0, bSFull1, bSEmpty0, bSEmpty1, bMhFull0, bMhFull1, bHFull0, bHFull1,
-  bYFull0, bYFull1, bYEmpty0, bYEmpty1, bDrain, bCount
+  bFull0 = 0, bFull1, bFull2, bEmpty0, bEmpty1, bEmpty2, bAux0, bAux1, bXwFull, bSFull0, bSFull1,
+  bSEmpty0, bSEmpty1, bMhFull0, bMhFull1, bHFull, bYFull0, bYFull1, bYEmpty0, bYEmpty1, bDrain, bCount
 };
 
 // TMEM columns: S^T[2] (M=128 x 64), Y^T[2] = {Y_off^T (M=64 x 64), Y_diag^T (M=64 x 64)}
@@ -256,11 +258,6 @@ __device__ __forceinline__ T pick4(const T (&a)[4], int i) {
 __device__ __forceinline__ float lds_f32(uint32_t addr) {
   float v;
   asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
-}
-__device__ __forceinline__ uint16_t lds_u16(uint32_t addr) {
-  uint16_t v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr) : "memory");
   return v;
 }
 __device__ __forceinline__ void sts_f32(uint32_t addr, float v) {
@@ -331,25 +328,36 @@ __device__ __forceinline__ void arrive_lane0(const Ctl &c, int bar) {
 
 // parity of the completion of a double-buffered barrier that block k uses
 __device__ __forceinline__ uint32_t par2(int k) { return (static_cast<uint32_t>(k) >> 1) & 1u; }
-// x ring: slot and parity of block k
-__device__ __forceinline__ int xslot(int k) { return k % kXSlots; }
-__device__ __forceinline__ uint32_t parx(int k) { return static_cast<uint32_t>(k / kXSlots) & 1u; }
+// TMA ring: slot and parity of block k
+__device__ __forceinline__ int rslot(int k) { return k % kSlots; }
+__device__ __forceinline__ uint32_t parr(int k) { return static_cast<uint32_t>(k / kSlots) & 1u; }
 
-// ---------------------------------------------------------------- producers
-// lane 0 of warp 0: B/C/C B^T ring; lane 1: x ring (runs further ahead).
-__device__ void producer_rest(const TcParams &p, const Ctl &c, uint8_t *sm, int b, int g) {
-  const uint32_t bytes = (2 + (p.allblock ? 4 : 2)) * kTile + (p.active[0] + p.active[1] + p.active[2] + p.active[3]) * 2048;
+// ---------------------------------------------------------------- producer
+__device__ void producer(const TcParams &p, const Ctl &c, uint8_t *sm, int b, int h, int g) {
+  const int nact = p.active[0] + p.active[1] + p.active[2] + p.active[3];
+  const uint32_t bytes = nact * (kTile + 2048) + (2 + (p.allblock ? 4 : 2)) * kTile;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    if (p.active[i]) tma_prefetch_desc(&p.tx[i]);
   tma_prefetch_desc(&p.tbcf);
   tma_prefetch_desc(&p.tccf);
+  if (p.allblock) tma_prefetch_desc(&p.tcnf);
   tma_prefetch_desc(&p.tcb);
-  int last0 = -1, last1 = -1;
+  int last[kSlots] = {-1, -1, -1};
   for (int k = 0; k < p.K; ++k) {
-    const int s = k & 1;
-    if (!wait1(c, bEmpty0 + s, par2(k) ^ 1)) break;
-    uint64_t *full = &c.bar[bFull0 + s];
+    const int r = rslot(k);
+    if (!wait1(c, bEmpty0 + r, parr(k) ^ 1)) break;
+    uint64_t *full = &c.bar[bFull0 + r];
     mbar_arrive_expect_tx(full, bytes);
-    uint8_t *st = sm + s * kStage;
+    uint8_t *st = sm + r * kSlot;
     const int t0 = k * kT;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (!p.active[i]) continue;
+      tma_load_4d(st + kOffX + i * kTile, &p.tx[i], full, 0, h, t0, b);
+      const int idx = ((i * p.Bsz + b) * p.K + k) * p.G + g;
+      tma_load_3d(st + kOffCB + i * 2048, &p.tcb, full, 0, 0, idx);
+    }
     tma_load_4d(st + kOffBcf, &p.tbcf, full, 0, g, t0, b);
     tma_load_4d(st + kOffBcf + kTile, &p.tbcf, full, 64, g, t0, b);
     tma_load_4d(st + kOffClo, &p.tccf, full, 0, g, t0, b);
@@ -359,40 +367,13 @@ __device__ void producer_rest(const TcParams &p, const Ctl &c, uint8_t *sm, int 
       tma_load_4d(st + kOffChi + kTile, &p.tcnf, full, 64, g, t0, b);
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (!p.active[i]) continue;
-      const int idx = ((i * p.Bsz + b) * p.K + k) * p.G + g;
-      tma_load_3d(st + kOffCB + i * 2048, &p.tcb, full, 0, 0, idx);
-    }
-    if (s) last1 = k; else last0 = k;
-  }
-  // no copy into this CTA's shared memory may still be in flight at exit
-  if (last0 >= 0) (void)mbar_wait(&c.bar[bFull0], par2(last0), p.drain_ns, nullptr);
-  if (last1 >= 0) (void)mbar_wait(&c.bar[bFull1], par2(last1), p.drain_ns, nullptr);
-}
-
-__device__ void producer_x(const TcParams &p, const Ctl &c, uint8_t *sm, int b, int h) {
-  const uint32_t bytes = (p.active[0] + p.active[1] + p.active[2] + p.active[3]) * kTile;
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    if (p.active[i]) tma_prefetch_desc(&p.tx[i]);
-  int last[kXSlots] = {-1, -1, -1};
-  for (int k = 0; k < p.K; ++k) {
-    const int r = xslot(k);
-    if (!wait1(c, bXEmpty0 + r, parx(k) ^ 1)) break;
-    uint64_t *full = &c.bar[bXFull0 + r];
-    mbar_arrive_expect_tx(full, bytes);
-    uint8_t *xs = sm + kOffX + r * kXSlot;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (p.active[i]) tma_load_4d(xs + i * kTile, &p.tx[i], full, 0, h, k * kT, b);
-#pragma unroll
-    for (int j = 0; j < kXSlots; ++j)
+    for (int j = 0; j < kSlots; ++j)
       if (j == r) last[j] = k;
   }
+  // no copy into this CTA's shared memory may still be in flight at exit
 #pragma unroll
-  for (int j = 0; j < kXSlots; ++j)
-    if (last[j] >= 0) (void)mbar_wait(&c.bar[bXFull0 + j], parx(last[j]), p.drain_ns, nullptr);
+  for (int j = 0; j < kSlots; ++j)
+    if (last[j] >= 0) (void)mbar_wait(&c.bar[bFull0 + j], parr(last[j]), p.drain_ns, nullptr);
 }
 
 // ---------------------------------------------------------------- MMA issuer
@@ -400,12 +381,12 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
   const uint32_t id_s = idesc_bf16(128, 64, 1, 1);  // S^T[n][p] = B^T (w o X)
   const uint32_t id_yo = idesc_bf16(64, 64, 1, 0);  // Y_off^T[p][t] = h C^T
   const uint32_t id_yd = idesc_bf16(64, 64, 1, 1);  // Y_diag^T[p][t] = X^T M^T
+  const uint32_t id_dx = idesc_bf16(64, 16, 1, 0);  // (D x)^T[p][t] = X^T (D I_16)
   const bool any_rev = p.active[kCR] || p.active[kNR];
   for (int k = 0; k < p.K; ++k) {
-    const int s = k & 1, i2 = k & 1, r = xslot(k);
-    const uint32_t st = base + s * kStage;
-    const uint32_t xs = base + kOffX + r * kXSlot;
-    if (!wait1(c, bFull0 + s, par2(k))) break;
+    const int r = rslot(k), i2 = k & 1;
+    const uint32_t st = base + r * kSlot;
+    if (!wait1(c, bFull0 + r, parr(k))) break;
     // ---- S^T(k) = B_cf^T (w o X): A MN-major (n; halves 4 KB apart), B MN-major (p)
     if (!wait1(c, bXwFull, k & 1)) break;
     if (k >= 2 && !wait1(c, bSEmpty0 + i2, par2(k - 2))) break;
@@ -419,14 +400,14 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
       umma_bf16(tmem + colS, a, bl, id_s, 1);
     }
     umma_commit(&c.bar[bSFull0 + i2]);
-    // ---- Y^T(k): Y_off^T = h_{k-1} [C_cf; C_nf]^T, Y_diag^T = X_fwd^T M_fwd^T + X_rev^T M_rev^T
-    if (!wait1(c, bXFull0 + r, parx(k))) break;
+    // ---- Y^T(k): Y_off^T = h_{k-1} [C_cf; C_nf]^T;
+    //      Y_diag^T = X_fwd^T M_fwd^T + X_rev^T M_rev^T + X^T (D I) for every direction
     if (!wait1(c, bMhFull0 + i2, par2(k))) break;
-    if (!wait1(c, bHFull0 + ((k + 1) & 1), par2(k))) break;  // h_{k-1} lives in buffer (k-1) & 1
+    if (!wait1(c, bHFull, k & 1)) break;  // h_{k-1}
     if (k >= 2 && !wait1(c, bYEmpty0 + i2, par2(k - 2))) break;
     tc_fence_after();
     const uint32_t colY = kColY0 + 128 * i2;
-    const uint32_t hb = base + kOffH + ((k + 1) & 1) * kHBuf;
+    const uint32_t hb = base + kOffH;
     for (int ks = 0; ks < 8; ++ks) {
       const uint64_t ah = sdesc(hb + ks * 2048, 0, 1024, kLayoutSw128);
       const uint64_t al = sdesc(hb + 4 * kTile + ks * 2048, 0, 1024, kLayoutSw128);
@@ -436,20 +417,31 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
     }
     const uint32_t mb = base + kOffMh + i2 * kMhBuf;
     for (int ks = 0; ks < 4; ++ks) {
-      const uint64_t a = sdesc(xs + ks * 2048, 0, 1024, kLayoutSw128);
+      const uint64_t a = sdesc(st + kOffX + ks * 2048, 0, 1024, kLayoutSw128);
       const uint64_t m = sdesc(mb + ks * 2048, kMhLbo, kMhSbo, kLayoutNone);
       umma_bf16(tmem + colY + 64, a, m, id_yd, ks > 0);
     }
     if (any_rev) {
       for (int ks = 0; ks < 4; ++ks) {
-        const uint64_t a = sdesc(xs + 2 * kTile + ks * 2048, 0, 1024, kLayoutSw128);
+        const uint64_t a = sdesc(st + kOffX + 2 * kTile + ks * 2048, 0, 1024, kLayoutSw128);
         const uint64_t m = sdesc(mb + 2 * kTile + ks * 2048, kMhLbo, kMhSbo, kLayoutNone);
         umma_bf16(tmem + colY + 64, a, m, id_yd, 1);
       }
     }
+    // D x of every direction: 16-token diagonal blocks against D I_16 (hi + lo)
+    for (int i = 0; i < 4; ++i) {
+      if (!p.active[i]) continue;
+      const uint32_t col = colY + 64 + ((i & 1) ? 32 : 0);
+      for (int ks = 0; ks < 2; ++ks) {
+        const uint64_t a = sdesc(st + kOffX + i * kTile + ks * 2048, 0, 1024, kLayoutSw128);
+        const uint64_t dh = sdesc(base + kOffDg + (2 * i) * 512, kDgLbo, kDgSbo, kLayoutNone);
+        const uint64_t dl = sdesc(base + kOffDg + (2 * i + 1) * 512, kDgLbo, kDgSbo, kLayoutNone);
+        umma_bf16(tmem + col + 16 * ks, a, dh, id_dx, 1);
+        umma_bf16(tmem + col + 16 * ks, a, dl, id_dx, 1);
+      }
+    }
     umma_commit(&c.bar[bYFull0 + i2]);
-    umma_commit(&c.bar[bEmpty0 + s]);
-    umma_commit(&c.bar[bXEmpty0 + r]);
+    umma_commit(&c.bar[bEmpty0 + r]);
   }
   umma_commit(&c.bar[bDrain]);
   (void)mbar_wait(&c.bar[bDrain], 0, p.drain_ns, nullptr);
@@ -477,7 +469,7 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base, in
   const uint32_t d0 = (q & 1) ? 32 : 0;
   for (int k = 0; k < p.K; ++k) {
     const int s = k & 1, i2 = k & 1, c4 = k & 3;
-    const uint32_t xs = base + kOffX + xslot(k) * kXSlot;
+    const uint32_t st = base + rslot(k) * kSlot;
     const float dt_cur = dt_next;
     dt_next = load_dt(k + 1);
     // ---- decays of this warp's direction (log2 units): prefix sum (forward)
@@ -499,13 +491,13 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base, in
       }
       sts_f32(cum + ((c4 * 4 + q) * 32 + lane) * 4, v);
       sts_f32(dts + ((c4 * 4 + q) * 32 + lane) * 4, dt_cur);
-      if (!rev) sts_f32(ecum + ((c4 * 2 + q) * 32 + lane) * 4, exp2f(v));
+      if (!rev) sts_f32(ecum + ((c4 * 2 + q) * 32 + lane) * 4, ex2_approx(v));
     }
     arrive_lane0(c, bAux0 + s);
     if (!waitw(c, bAux0 + s, par2(k))) break;
     // ---- (w o X) of the clean forward direction, bf16 hi + lo
     if (k >= 1 && !waitw(c, bSFull0 + ((k + 1) & 1), par2(k - 1))) break;  // S(k-1) read Xw
-    if (!waitw(c, bXFull0 + xslot(k), parx(k))) break;
+    if (!waitw(c, bFull0 + rslot(k), parr(k))) break;
     {
       const uint32_t cf = cum + (c4 * 4 + kCF) * 128, df = dts + (c4 * 4 + kCF) * 128;
       const float c31 = lds_f32(cf + 31 * 4);
@@ -515,8 +507,8 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base, in
         const int t = i >> 3, ch = i & 7;
         const uint32_t off = sw128_chunk(t, ch);
         uint32_t r0, r1, r2, r3;
-        ld_shared_v4(xs + off, r0, r1, r2, r3);
-        const float w = lds_f32(df + t * 4) * exp2f(c31 - lds_f32(cf + t * 4));
+        ld_shared_v4(st + kOffX + off, r0, r1, r2, r3);
+        const float w = lds_f32(df + t * 4) * ex2_approx(c31 - lds_f32(cf + t * 4));
         float vv[8] = {bf16_lo_f(r0) * w, bf16_hi_f(r0) * w, bf16_lo_f(r1) * w, bf16_hi_f(r1) * w,
                        bf16_lo_f(r2) * w, bf16_hi_f(r2) * w, bf16_lo_f(r3) * w, bf16_hi_f(r3) * w};
         store_split8(base + kOffXw + off, base + kOffXw + kTile + off, vv);
@@ -525,10 +517,9 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base, in
       arrive_lane0(c, bXwFull);
     }
     // ---- masked-decay matrix, row s = lane of M^T for this direction
-    if (!waitw(c, bFull0 + s, par2(k))) break;
     if (k >= 2 && !waitw(c, bYFull0 + i2, par2(k - 2))) break;  // Y(k-2) read this M buffer
     if (act) {
-      const uint32_t cbrow = base + s * kStage + kOffCB + q * 2048;
+      const uint32_t cbrow = st + kOffCB + q * 2048;
       float cbv[32];
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
@@ -556,7 +547,7 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base, in
         for (int i = 0; i < 8; ++i) {
           const int t = 8 * j + i;
           const bool valid = rev ? (t <= lane) : (t >= lane);
-          const float e = exp2f(cj[i] - cs);
+          const float e = ex2_approx(cj[i] - cs);
           m[i] = valid ? cbv[t] * ds * e : 0.f;
         }
         st_shared_v4(mrow + inter_mn_off(d0 + 8 * j, d0 + lane, kMhSbo, kMhLbo), pack_bf16x2(m[0], m[1]),
@@ -565,8 +556,7 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base, in
     }
     fence_proxy_async_smem();
     arrive_lane0(c, bMhFull0 + i2);
-    arrive_lane0(c, bEmpty0 + s);
-    arrive_lane0(c, bXEmpty0 + xslot(k));
+    arrive_lane0(c, bEmpty0 + rslot(k));
   }
 }
 
@@ -585,22 +575,22 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
 #pragma unroll
     for (int pp = 0; pp < kP; ++pp) hreg[pp] = src ? src[pp * kN] : 0.f;
   }
-  // h operand of Y_off^T (A, MN-major): buffer hbuf, {hi, lo} x [128 n rows][64 p] (SW128)
-  auto write_h = [&](int hbuf) {
-    const uint32_t hb = base + kOffH + hbuf * kHBuf;
+  // h operand of Y_off^T (A, MN-major): {hi, lo} x [128 n rows][64 p] (SW128)
+  auto write_h = [&]() {
+    const uint32_t hb = base + kOffH;
 #pragma unroll
     for (int cc = 0; cc < 8; ++cc) {
       const uint32_t off = sw128_chunk(n, cc);
       store_split8(hb + off, hb + 4 * kTile + off, hreg + 8 * cc);
     }
     fence_proxy_async_smem();
-    arrive_lane0(c, bHFull0 + hbuf);
+    arrive_lane0(c, bHFull);
   };
-  write_h(1);  // h_{-1} lives in buffer 1
+  write_h();  // h_{-1}
   for (int k = 0; k < p.K; ++k) {
     const int i2 = k & 1, c4 = k & 3;
     if (!waitw(c, bAux0 + (k & 1), par2(k))) break;
-    const float atot = exp2f(lds_f32(cum + ((c4 * 4 + kCF) * 32 + 31) * 4));
+    const float atot = ex2_approx(lds_f32(cum + ((c4 * 4 + kCF) * 32 + 31) * 4));
     if (!waitw(c, bSFull0 + i2, par2(k))) break;
     tc_fence_after();
     {
@@ -617,9 +607,9 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
     }
     tc_fence_before();
     arrive_lane0(c, bSEmpty0 + i2);
-    // buffer k & 1 held h_{k-2}; Y(k-1) has read it once y_full(k-1) completes
-    if (k >= 1 && !waitw(c, bYFull0 + ((k + 1) & 1), par2(k - 1))) break;
-    write_h(k & 1);
+    // Y(k) reads h_{k-1} from the operand buffer; h_k replaces it afterwards
+    if (!waitw(c, bYFull0 + i2, par2(k))) break;
+    write_h();
     if (p.states) {  // each warp instruction stores one contiguous 128-byte row segment
       float *dst = p.states + ((static_cast<int64_t>(b) * p.K + k) * H + h) * PN + n;
 #pragma unroll
@@ -635,25 +625,21 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
 
 // ---------------------------------------------------------------- epilogue
 // warps 10..13: thread owns column p = 16 q + (lane & 15) of the clean
-// (lane < 16) or noisy (lane >= 16) stream's outputs y[t][p], t = 0..31.
+// (lane < 16) or noisy (lane >= 16) stream's outputs y[t][p], t = 0..31:
+// y = exp(cum_t) Y_off + Y_diag (Y_diag already holds both directions' D x).
 __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem, int b, int h) {
   const int lane = threadIdx.x & 31;
   const int q = (threadIdx.x >> 5) & 3;
   const int pcol = 16 * q + (lane & 15);
   const bool noisy = lane >= 16;
-  const int fs = noisy ? kNF : kCF, rs = noisy ? kNR : kCR;
+  const int fs = noisy ? kNF : kCF;
   void *yout = noisy ? p.y_noisy : p.y_clean;
   const bool mine = (noisy ? p.allblock != 0 : true) && yout != nullptr;
-  const bool has_rev = pick4(p.active, rs) != 0;
-  const float Df = pick4(p.active, fs) ? pick4(p.D, fs)[h] : 0.f;
-  const float Dr = has_rev ? pick4(p.D, rs)[h] : 0.f;
   const uint32_t ecum = base + kOffEc;
   const int64_t H = p.H, L = p.L;
   for (int k = 0; k < p.K; ++k) {
     const int i2 = k & 1, c4 = k & 3;
-    const uint32_t xs = base + kOffX + xslot(k) * kXSlot;
     if (!waitw(c, bAux0 + (k & 1), par2(k))) break;
-    if (!waitw(c, bXFull0 + xslot(k), parx(k))) break;
     if (!waitw(c, bYFull0 + i2, par2(k))) break;
     tc_fence_after();
     uint32_t yo[32], yd[32];
@@ -665,20 +651,13 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
     arrive_lane0(c, bYEmpty0 + i2);
     if (mine) {
       const uint32_t eq = ecum + (c4 * 2 + fs) * 128;
-      const uint32_t xf = xs + fs * kTile, xr = xs + rs * kTile;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         float e4[4];
         ld_shared_v4f(eq + 16 * j, e4);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int t = 4 * j + i;
-          const uint32_t xo = sw128_off(t, pcol);
-          float y = fmaf(e4[i], __uint_as_float(yo[t]), __uint_as_float(yd[t]));
-          y = fmaf(Df, __uint_as_float(static_cast<uint32_t>(lds_u16(xf + xo)) << 16), y);
-          if (has_rev) y = fmaf(Dr, __uint_as_float(static_cast<uint32_t>(lds_u16(xr + xo)) << 16), y);
-          yo[t] = __float_as_uint(y);
-        }
+        for (int i = 0; i < 4; ++i)
+          yo[4 * j + i] = __float_as_uint(fmaf(e4[i], __uint_as_float(yo[4 * j + i]), __uint_as_float(yd[4 * j + i])));
       }
       const int64_t yi = ((static_cast<int64_t>(b) * L + k * kT) * H + h) * kP + pcol;
       const int64_t tstride = H * kP;
@@ -692,7 +671,6 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
         for (int t = 0; t < 32; ++t) dst[t * tstride] = __uint_as_float(yo[t]);
       }
     }
-    arrive_lane0(c, bXEmpty0 + xslot(k));
   }
 }
 
@@ -710,17 +688,15 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(sm + kOffMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kOffMisc + 4);
   if (threadIdx.x == 0) {
-    // arrival counts: full = producer; empty = MMA commit + 4 operand warps;
-    // x empty = MMA commit + 4 operand warps + 4 epilogue warps; the rest as named
+    // arrival counts: full = producer (plus TMA bytes); empty = MMA commit + 4
+    // operand warps; commits of the MMA warp count 1; the rest 4 warps each
     for (int i = 0; i < bCount; ++i) {
       uint32_t cnt = 4;
-      if (i == bFull0 || i == bFull1 || i == bXFull0 || i == bXFull1 || i == bXFull2 || i == bSFull0 ||
-          i == bSFull1 || i == bYFull0 || i == bYFull1 || i == bDrain)
+      if (i == bFull0 || i == bFull1 || i == bFull2 || i == bSFull0 || i == bSFull1 || i == bYFull0 ||
+          i == bYFull1 || i == bDrain)
         cnt = 1;
-      else if (i == bEmpty0 || i == bEmpty1)
+      else if (i == bEmpty0 || i == bEmpty1 || i == bEmpty2)
         cnt = 5;
-      else if (i == bXEmpty0 || i == bXEmpty1 || i == bXEmpty2)
-        cnt = 9;
       mbar_init(&bars[i], cnt);
     }
     *abort_flag = 0;
@@ -729,22 +705,35 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
   // x tiles of inactive directions are read next to zero operands by the MMAs:
   // clear them (and the masked-decay buffers, whose off-diagonal blocks stay
   // zero) so that no uninitialised NaN/Inf bit pattern can reach an output.
+  // Build the D I_16 operands (bf16 hi + lo of each direction's D).
   {
     const uint4 zero = make_uint4(0, 0, 0, 0);
     for (int i = 0; i < 4; ++i) {
       if (p.active[i]) continue;
-      for (int r = 0; r < kXSlots; ++r)
+      for (int r = 0; r < kSlots; ++r)
         for (uint32_t o = threadIdx.x * 16; o < kTile; o += kThreads * 16)
-          *reinterpret_cast<uint4 *>(sm + kOffX + r * kXSlot + i * kTile + o) = zero;
+          *reinterpret_cast<uint4 *>(sm + r * kSlot + kOffX + i * kTile + o) = zero;
     }
     if (!p.allblock)
-      for (int s = 0; s < 2; ++s)
+      for (int r = 0; r < kSlots; ++r)
         for (uint32_t o = threadIdx.x * 16; o < kTile; o += kThreads * 16) {
-          *reinterpret_cast<uint4 *>(sm + s * kStage + kOffClo + kTile + o) = zero;
-          *reinterpret_cast<uint4 *>(sm + s * kStage + kOffChi + kTile + o) = zero;
+          *reinterpret_cast<uint4 *>(sm + r * kSlot + kOffClo + kTile + o) = zero;
+          *reinterpret_cast<uint4 *>(sm + r * kSlot + kOffChi + kTile + o) = zero;
         }
-    for (uint32_t o = threadIdx.x * 16; o < 2 * kMhBuf; o += kThreads * 16)
-      *reinterpret_cast<uint4 *>(sm + kOffMh + o) = zero;
+    for (uint32_t o = threadIdx.x * 16; o < 2 * kMhBuf + 4096; o += kThreads * 16)
+      *reinterpret_cast<uint4 *>(sm + kOffMh + o) = zero;  // M buffers and D I_16 tiles
+    __syncthreads();
+    if (threadIdx.x < 4 * 16) {
+      const int i = threadIdx.x >> 4, d = threadIdx.x & 15;
+      if (p.active[i]) {
+        const float Dv = pick4(p.D, i)[h];
+        const __nv_bfloat16 dh = __float2bfloat16_rn(Dv);
+        const __nv_bfloat16 dl = __float2bfloat16_rn(Dv - __bfloat162float(dh));
+        const uint32_t off = (d >> 3) * kDgSbo + (d >> 3) * kDgLbo + (d & 7) * 16 + (d & 7) * 2;
+        *reinterpret_cast<__nv_bfloat16 *>(sm + kOffDg + (2 * i) * 512 + off) = dh;
+        *reinterpret_cast<__nv_bfloat16 *>(sm + kOffDg + (2 * i + 1) * 512 + off) = dl;
+      }
+    }
     fence_proxy_async_smem();
   }
   if (warp == 1) {
@@ -758,9 +747,7 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
   Ctl c{bars, abort_flag, p.status, p.timeout_ns};
 
   if (warp == 0) {
-    const int lane = threadIdx.x & 31;
-    if (lane == 0) producer_rest(p, c, sm, b, g);
-    else if (lane == 1) producer_x(p, c, sm, b, h);
+    if ((threadIdx.x & 31) == 0) producer(p, c, sm, b, h, g);
   } else if (warp == 1) {
     if ((threadIdx.x & 31) == 0) mma_issuer(p, c, base, tmem);
   } else if (warp < 6) {
