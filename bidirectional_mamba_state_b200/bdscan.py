@@ -27,7 +27,7 @@ BDSCAN_BF16, BDSCAN_FP32 = 0, 1
 BDSCAN_OP_PREFIX, BDSCAN_OP_BLOCK_STEP, BDSCAN_OP_ALLBLOCK = 0, 1, 2
 STATUS = {0: "BDSCAN_OK", -1: "BDSCAN_ERR_INVALID_ARG", -2: "BDSCAN_ERR_UNSUPPORTED_SHAPE",
           -3: "BDSCAN_ERR_MISALIGNED", -4: "BDSCAN_ERR_WORKSPACE", -5: "BDSCAN_ERR_CUDA",
-          -6: "BDSCAN_ERR_TIMEOUT"}
+          -6: "BDSCAN_ERR_TIMEOUT", -7: "BDSCAN_ERR_SCRATCH_LIMIT"}
 
 
 class bdscan_shape_t(ctypes.Structure):
@@ -74,6 +74,10 @@ def lib() -> ctypes.CDLL:
             L.bdscan_workspace_size.restype = ctypes.c_size_t
             L.bdscan_kernel_launches.argtypes = [sp, ctypes.c_int]
             L.bdscan_kernel_launches.restype = ctypes.c_int
+            L.bdscan_block_step_noalloc.argtypes = [sp, dp, dp, vp, vp, vp, vp]
+            L.bdscan_block_step_noalloc.restype = ctypes.c_int
+            L.bdscan_noalloc_scratch.argtypes = []
+            L.bdscan_noalloc_scratch.restype = ctypes.c_void_p
             L.bdscan_check_status.argtypes = [vp, vp]
             L.bdscan_status_string.argtypes = [ctypes.c_int]
             L.bdscan_status_string.restype = ctypes.c_char_p
@@ -101,6 +105,14 @@ def bdscan_allblock(shape, cf, cr, nf, nr, h0, y_clean, y_noisy, block_states, w
                     stream) -> int:
     return lib().bdscan_allblock(shape, cf, cr, nf, nr, h0, y_clean, y_noisy, block_states, ws,
                                  ws_bytes, stream)
+
+
+def bdscan_block_step_noalloc(shape, fwd, rev, state_in, y, state_out, stream) -> int:
+    return lib().bdscan_block_step_noalloc(shape, fwd, rev, state_in, y, state_out, stream)
+
+
+def bdscan_noalloc_scratch() -> int | None:
+    return lib().bdscan_noalloc_scratch()
 
 
 def bdscan_workspace_size(shape, op: int) -> int:

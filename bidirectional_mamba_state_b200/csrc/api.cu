@@ -7,6 +7,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <utility>
 #include <vector>
 
@@ -308,10 +309,64 @@ const char *bdscan_status_string(int status) {
     case BDSCAN_ERR_WORKSPACE: return "workspace missing or too small";
     case BDSCAN_ERR_CUDA: return "CUDA launch or runtime error";
     case BDSCAN_ERR_TIMEOUT: return "bounded device-side wait timed out";
+    case BDSCAN_ERR_SCRATCH_LIMIT:
+      return "shape needs more scratch than the no-alloc entry point's built-in buffer holds";
     default: return "unknown status";
   }
 }
 
 int bdscan_version(void) { return 100; }
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- no-alloc step
+// Scratch of bdscan_block_step_noalloc: a static device buffer (every GPU that
+// loads the library holds it until exit).  Host code must not pass the symbol
+// itself to a kernel -- on the host it is only a stand-in -- but the device
+// address that cudaGetSymbolAddress returns for the current device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[BDSCAN_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch buffer on the current device, looked up once per
+// device (with that device current); nullptr if the lookup fails.
+void *noalloc_scratch_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+void *bdscan_noalloc_scratch(void) { return noalloc_scratch_ptr(); }
+
+int bdscan_block_step_noalloc(const bdscan_shape_t *shape, const bdscan_dir_t *fwd,
+                              const bdscan_dir_t *rev, const float *state_in, void *y,
+                              float *state_out, void *cuda_stream) {
+  const size_t need = bdscan_workspace_size(shape, BDSCAN_OP_BLOCK_STEP);
+  if (need == 0) {
+    const int rc = check_shape(shape);
+    return rc ? rc : BDSCAN_ERR_INVALID_ARG;
+  }
+  if (need > BDSCAN_NOALLOC_SCRATCH_BYTES) return BDSCAN_ERR_SCRATCH_LIMIT;
+  void *ws = noalloc_scratch_ptr();
+  if (!ws) return BDSCAN_ERR_CUDA;
+  // The call clears the status word itself; the C B^T tiles are fully rewritten
+  // before they are read, so nothing else needs to start at zero.
+  return bdscan_block_step(shape, fwd, rev, state_in, y, state_out, ws, BDSCAN_NOALLOC_SCRATCH_BYTES,
+                           cuda_stream);
+}
 
 }  // extern "C"

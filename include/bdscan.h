@@ -59,6 +59,7 @@ extern "C" {
 #define BDSCAN_ERR_WORKSPACE (-4)         /* ws NULL or ws_bytes < bdscan_workspace_size() */
 #define BDSCAN_ERR_CUDA (-5)              /* a kernel launch or CUDA runtime call failed */
 #define BDSCAN_ERR_TIMEOUT (-6)           /* a bounded device-side wait ran out (check_status) */
+#define BDSCAN_ERR_SCRATCH_LIMIT (-7)     /* shape needs more than the built-in no-alloc scratch */
 
 /* operations (bdscan_workspace_size) */
 #define BDSCAN_OP_PREFIX 0
@@ -144,6 +145,35 @@ int bdscan_check_status(const void *ws, void *cuda_stream);
 
 /* Static description of a status code. */
 const char *bdscan_status_string(int status);
+
+/* bdscan_block_step_noalloc -- the denoising step of bdscan_block_step for
+ * callers that cannot allocate device memory: code that runs under a fixed
+ * memory plan that has already handed out all device memory (an inference
+ * server or graph executor with a static arena), or code that runs while a
+ * stream is being captured, where cudaMalloc is not allowed.  The pages have
+ * no counterpart; this is a deployment convenience.
+ *
+ * Same arguments, results and errors as bdscan_block_step, minus the
+ * workspace: the scratch it needs (the status word and the tensor-core path's
+ * C B^T tiles) lives in a static device buffer of BDSCAN_NOALLOC_SCRATCH_BYTES
+ * inside the library, which every GPU that loads the library holds until the
+ * process exits.  It calls no cudaMalloc or cudaFree.
+ *   - Shapes whose workspace (bdscan_workspace_size(shape, BLOCK_STEP)) exceeds
+ *     BDSCAN_NOALLOC_SCRATCH_BYTES are rejected with BDSCAN_ERR_SCRATCH_LIMIT
+ *     (for the tensor-core shapes: batch * ngroups <= 512).
+ *   - The first call on a device looks up the buffer's device address on that
+ *     device (the device current at the call); make that first call before any
+ *     stream capture begins.
+ *   - All calls share the one buffer: calls that may overlap on the GPU (other
+ *     streams, other host threads) race on it; serialise them on one stream.
+ *   - bdscan_check_status() reads its status word through
+ *     bdscan_noalloc_scratch(), which returns the buffer's device address on
+ *     the current device (NULL if the lookup fails). */
+#define BDSCAN_NOALLOC_SCRATCH_BYTES ((size_t)(4u << 20) + 1024u)
+int bdscan_block_step_noalloc(const bdscan_shape_t *shape, const bdscan_dir_t *fwd,
+                              const bdscan_dir_t *rev, const float *state_in, void *y,
+                              float *state_out, void *cuda_stream);
+void *bdscan_noalloc_scratch(void);
 
 /* Library version (major * 10000 + minor * 100 + patch). */
 int bdscan_version(void);
