@@ -160,7 +160,8 @@ size_t bdscan_workspace_size(const bdscan_shape_t *shape, int op) {
   // The tensor-core path keeps C B^T of every (direction, batch, block, group)
   // in the workspace; shapes it cannot take need only the status word.
   if (bdscan::tc_shape_ok(shape->headdim, shape->dstate, shape->block_len, shape->in_dtype == BDSCAN_BF16))
-    return bdscan::kWsHeader + bdscan::tc_workspace_bytes(shape->batch, shape->seqlen, shape->ngroups);
+    return bdscan::kWsHeader +
+           bdscan::tc_workspace_bytes(shape->batch, shape->seqlen, shape->ngroups, shape->nheads);
   return kStatusBytes;
 }
 
@@ -169,9 +170,10 @@ int bdscan_kernel_launches(const bdscan_shape_t *shape, int op) {
   if (op != BDSCAN_OP_PREFIX && op != BDSCAN_OP_BLOCK_STEP && op != BDSCAN_OP_ALLBLOCK) return -1;
   if (op == BDSCAN_OP_BLOCK_STEP && shape->seqlen != shape->block_len) return -1;
   if (shape->batch == 0 || shape->seqlen == 0) return 0;
-  // tensor-core path: C B^T pre-pass + scan; generic path: one kernel
+  // tensor-core path: C B^T pre-pass + scan, plus an aggregate pass and a
+  // segment combine when sequences are cut into segments; generic path: one kernel
   if (bdscan::tc_shape_ok(shape->headdim, shape->dstate, shape->block_len, shape->in_dtype == BDSCAN_BF16))
-    return 2;
+    return bdscan::tc_plan_segments(shape->batch, shape->nheads, shape->seqlen / shape->block_len) > 1 ? 4 : 2;
   return 1;
 }
 

@@ -229,8 +229,13 @@ struct TcParams {
   const float *D[4];
   int active[4];
   int Bsz, L, H, G, K;
+  int nseg, seg_blocks;  // each (b, h) sequence is walked as nseg segments of seg_blocks blocks
+  int agg;               // aggregate pass: forward state of each segment from zero, nothing else
   int allblock;
   int out_bf16;
+  const float *seg_init;  // [B][H][nseg][P][N] initial state of every segment (nseg > 1)
+  float *seg_local;       // [B][H][nseg][P][N] aggregate pass: end state from a zero start
+  float *seg_decay;       // [B][H][nseg] aggregate pass: total decay (log2 units)
   const float *h0;
   float *states;
   float *final_state;
@@ -333,9 +338,9 @@ __device__ __forceinline__ int rslot(int k) { return k % kSlots; }
 __device__ __forceinline__ uint32_t parr(int k) { return static_cast<uint32_t>(k / kSlots) & 1u; }
 
 // ---------------------------------------------------------------- producer
-__device__ void producer(const TcParams &p, const Ctl &c, uint8_t *sm, int b, int h, int g) {
+__device__ void producer(const TcParams &p, const Ctl &c, uint8_t *sm, int b, int h, int g, int k0, int nk) {
   const int nact = p.active[0] + p.active[1] + p.active[2] + p.active[3];
-  const uint32_t bytes = nact * (kTile + 2048) + (2 + (p.allblock ? 4 : 2)) * kTile;
+  const uint32_t bytes = p.agg ? 3 * kTile : nact * (kTile + 2048) + (2 + (p.allblock ? 4 : 2)) * kTile;
 #pragma unroll
   for (int i = 0; i < 4; ++i)
     if (p.active[i]) tma_prefetch_desc(&p.tx[i]);
@@ -344,9 +349,10 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint8_t *sm, int b, in
   if (p.allblock) tma_prefetch_desc(&p.tcnf);
   tma_prefetch_desc(&p.tcb);
   int last[kSlots] = {-1, -1, -1};
-  for (int k = 0; k < p.K; ++k) {
-    const int r = rslot(k);
-    if (!wait1(c, bEmpty0 + r, parr(k) ^ 1)) break;
+  for (int kk = 0; kk < nk; ++kk) {
+    const int k = k0 + kk;  // global block index
+    const int r = rslot(kk);
+    if (!wait1(c, bEmpty0 + r, parr(kk) ^ 1)) break;
     uint64_t *full = &c.bar[bFull0 + r];
     mbar_arrive_expect_tx(full, bytes);
     uint8_t *st = sm + r * kSlot;
@@ -355,11 +361,18 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint8_t *sm, int b, in
     for (int i = 0; i < 4; ++i) {
       if (!p.active[i]) continue;
       tma_load_4d(st + kOffX + i * kTile, &p.tx[i], full, 0, h, t0, b);
+      if (p.agg) continue;
       const int idx = ((i * p.Bsz + b) * p.K + k) * p.G + g;
       tma_load_3d(st + kOffCB + i * 2048, &p.tcb, full, 0, 0, idx);
     }
     tma_load_4d(st + kOffBcf, &p.tbcf, full, 0, g, t0, b);
     tma_load_4d(st + kOffBcf + kTile, &p.tbcf, full, 64, g, t0, b);
+    if (p.agg) {
+#pragma unroll
+      for (int j = 0; j < kSlots; ++j)
+        if (j == r) last[j] = kk;
+      continue;
+    }
     tma_load_4d(st + kOffClo, &p.tccf, full, 0, g, t0, b);
     tma_load_4d(st + kOffChi, &p.tccf, full, 64, g, t0, b);
     if (p.allblock) {
@@ -368,7 +381,7 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint8_t *sm, int b, in
     }
 #pragma unroll
     for (int j = 0; j < kSlots; ++j)
-      if (j == r) last[j] = k;
+      if (j == r) last[j] = kk;
   }
   // no copy into this CTA's shared memory may still be in flight at exit
 #pragma unroll
@@ -377,19 +390,19 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint8_t *sm, int b, in
 }
 
 // ---------------------------------------------------------------- MMA issuer
-__device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
+__device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem, int nk) {
   const uint32_t id_s = idesc_bf16(128, 64, 1, 1);  // S^T[n][p] = B^T (w o X)
   const uint32_t id_yo = idesc_bf16(64, 64, 1, 0);  // Y_off^T[p][t] = h C^T
   const uint32_t id_yd = idesc_bf16(64, 64, 1, 1);  // Y_diag^T[p][t] = X^T M^T
   const uint32_t id_dx = idesc_bf16(64, 16, 1, 0);  // (D x)^T[p][t] = X^T (D I_16)
   const bool any_rev = p.active[kCR] || p.active[kNR];
-  for (int k = 0; k < p.K; ++k) {
-    const int r = rslot(k), i2 = k & 1;
+  for (int kk = 0; kk < nk; ++kk) {
+    const int r = rslot(kk), i2 = kk & 1;
     const uint32_t st = base + r * kSlot;
-    if (!wait1(c, bFull0 + r, parr(k))) break;
+    if (!wait1(c, bFull0 + r, parr(kk))) break;
     // ---- S^T(k) = B_cf^T (w o X): A MN-major (n; halves 4 KB apart), B MN-major (p)
-    if (!wait1(c, bXwFull, k & 1)) break;
-    if (k >= 2 && !wait1(c, bSEmpty0 + i2, par2(k - 2))) break;
+    if (!wait1(c, bXwFull, kk & 1)) break;
+    if (kk >= 2 && !wait1(c, bSEmpty0 + i2, par2(kk - 2))) break;
     tc_fence_after();
     const uint32_t colS = kColS0 + 64 * i2;
     for (int ks = 0; ks < 2; ++ks) {
@@ -400,11 +413,15 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
       umma_bf16(tmem + colS, a, bl, id_s, 1);
     }
     umma_commit(&c.bar[bSFull0 + i2]);
+    if (p.agg) {  // aggregate pass: the forward state is all it needs
+      umma_commit(&c.bar[bEmpty0 + r]);
+      continue;
+    }
     // ---- Y^T(k): Y_off^T = h_{k-1} [C_cf; C_nf]^T;
     //      Y_diag^T = X_fwd^T M_fwd^T + X_rev^T M_rev^T + X^T (D I) for every direction
-    if (!wait1(c, bMhFull0 + i2, par2(k))) break;
-    if (!wait1(c, bHFull, k & 1)) break;  // h_{k-1}
-    if (k >= 2 && !wait1(c, bYEmpty0 + i2, par2(k - 2))) break;
+    if (!wait1(c, bMhFull0 + i2, par2(kk))) break;
+    if (!wait1(c, bHFull, kk & 1)) break;  // h_{k-1}
+    if (kk >= 2 && !wait1(c, bYEmpty0 + i2, par2(kk - 2))) break;
     tc_fence_after();
     const uint32_t colY = kColY0 + 128 * i2;
     const uint32_t hb = base + kOffH;
@@ -449,7 +466,7 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
 
 // ---------------------------------------------------------------- operand group
 // warps 2..5; q = warp & 3 is the direction slot whose decays and M it builds.
-__device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base, int b, int h) {
+__device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base, int b, int h, int k0, int nk) {
   const int lane = threadIdx.x & 31;
   const int q = (threadIdx.x >> 5) & 3;
   const int gt = threadIdx.x - 64;  // 0..127
@@ -459,19 +476,19 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base, in
   const int64_t H = p.H, L = p.L;
   const float A2 = act ? pick4(p.A, q)[h] * kLog2e : 0.f;
   const __nv_bfloat16 *dtp = pick4(p.dt, q);
-  auto load_dt = [&](int k) -> float {
-    if (!act || k >= p.K) return 0.f;
-    return __bfloat162float(dtp[(static_cast<int64_t>(b) * L + k * kT + lane) * H + h]);
+  auto load_dt = [&](int kk) -> float {  // dt of local block kk of this segment
+    if (!act || kk >= nk) return 0.f;
+    return __bfloat162float(dtp[(static_cast<int64_t>(b) * L + (k0 + kk) * kT + lane) * H + h]);
   };
   float dt_next = load_dt(0);
   // position of this direction's block in the stacked [64 t][64 s] operand
   const uint32_t mset = rev ? 2 * kTile : 0;
   const uint32_t d0 = (q & 1) ? 32 : 0;
-  for (int k = 0; k < p.K; ++k) {
-    const int s = k & 1, i2 = k & 1, c4 = k & 3;
-    const uint32_t st = base + rslot(k) * kSlot;
+  for (int kk = 0; kk < nk; ++kk) {
+    const int s = kk & 1, i2 = kk & 1, c4 = kk & 3;
+    const uint32_t st = base + rslot(kk) * kSlot;
     const float dt_cur = dt_next;
-    dt_next = load_dt(k + 1);
+    dt_next = load_dt(kk + 1);
     // ---- decays of this warp's direction (log2 units): prefix sum (forward)
     //      or suffix sum (reverse) over the block
     float v = dt_cur * A2;
@@ -494,10 +511,10 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base, in
       if (!rev) sts_f32(ecum + ((c4 * 2 + q) * 32 + lane) * 4, ex2_approx(v));
     }
     arrive_lane0(c, bAux0 + s);
-    if (!waitw(c, bAux0 + s, par2(k))) break;
+    if (!waitw(c, bAux0 + s, par2(kk))) break;
     // ---- (w o X) of the clean forward direction, bf16 hi + lo
-    if (k >= 1 && !waitw(c, bSFull0 + ((k + 1) & 1), par2(k - 1))) break;  // S(k-1) read Xw
-    if (!waitw(c, bFull0 + rslot(k), parr(k))) break;
+    if (kk >= 1 && !waitw(c, bSFull0 + ((kk + 1) & 1), par2(kk - 1))) break;  // S(k-1) read Xw
+    if (!waitw(c, bFull0 + rslot(kk), parr(kk))) break;
     {
       const uint32_t cf = cum + (c4 * 4 + kCF) * 128, df = dts + (c4 * 4 + kCF) * 128;
       const float c31 = lds_f32(cf + 31 * 4);
@@ -517,8 +534,8 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base, in
       arrive_lane0(c, bXwFull);
     }
     // ---- masked-decay matrix, row s = lane of M^T for this direction
-    if (k >= 2 && !waitw(c, bYFull0 + i2, par2(k - 2))) break;  // Y(k-2) read this M buffer
-    if (act) {
+    if (!p.agg && kk >= 2 && !waitw(c, bYFull0 + i2, par2(kk - 2))) break;  // Y(k-2) read this M buffer
+    if (act && !p.agg) {
       const uint32_t cbrow = st + kOffCB + q * 2048;
       float cbv[32];
 #pragma unroll
@@ -556,13 +573,14 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base, in
     }
     fence_proxy_async_smem();
     arrive_lane0(c, bMhFull0 + i2);
-    arrive_lane0(c, bEmpty0 + rslot(k));
+    arrive_lane0(c, bEmpty0 + rslot(kk));
   }
 }
 
 // ---------------------------------------------------------------- state group
 // warps 6..9: thread owns column n = 32 q + lane of the state, h^T[n][0..63].
-__device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem, int b, int h) {
+__device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem, int b, int h,
+                            int seg, int k0, int nk) {
   const int lane = threadIdx.x & 31;
   const int q = (threadIdx.x >> 5) & 3;
   const int n = 32 * q + lane;
@@ -571,7 +589,13 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
   const int64_t PN = kP * kN;
   float hreg[kP];
   {
-    const float *src = p.h0 ? p.h0 + (static_cast<int64_t>(b) * H + h) * PN + n : nullptr;
+    // initial state of this segment: h0 (first segment), the chained state the
+    // aggregate and combine passes left in the workspace (later segments), or
+    // zero (aggregate pass)
+    const int64_t bhs = (static_cast<int64_t>(b) * H + h) * p.nseg + seg;
+    const float *src = p.agg ? nullptr
+                       : seg == 0 ? (p.h0 ? p.h0 + (static_cast<int64_t>(b) * H + h) * PN + n : nullptr)
+                                  : p.seg_init + bhs * PN + n;
 #pragma unroll
     for (int pp = 0; pp < kP; ++pp) hreg[pp] = src ? src[pp * kN] : 0.f;
   }
@@ -586,12 +610,16 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
     fence_proxy_async_smem();
     arrive_lane0(c, bHFull);
   };
-  write_h();  // h_{-1}
-  for (int k = 0; k < p.K; ++k) {
-    const int i2 = k & 1, c4 = k & 3;
-    if (!waitw(c, bAux0 + (k & 1), par2(k))) break;
-    const float atot = ex2_approx(lds_f32(cum + ((c4 * 4 + kCF) * 32 + 31) * 4));
-    if (!waitw(c, bSFull0 + i2, par2(k))) break;
+  if (!p.agg) write_h();  // h_{-1}
+  float decay_log2 = 0.f;  // total decay over the segment (aggregate pass)
+  for (int kk = 0; kk < nk; ++kk) {
+    const int k = k0 + kk;  // global block index
+    const int i2 = kk & 1, c4 = kk & 3;
+    if (!waitw(c, bAux0 + (kk & 1), par2(kk))) break;
+    const float c31 = lds_f32(cum + ((c4 * 4 + kCF) * 32 + 31) * 4);
+    const float atot = ex2_approx(c31);
+    decay_log2 += c31;
+    if (!waitw(c, bSFull0 + i2, par2(kk))) break;
     tc_fence_after();
     {
       uint32_t sv[32];
@@ -607,8 +635,9 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
     }
     tc_fence_before();
     arrive_lane0(c, bSEmpty0 + i2);
+    if (p.agg) continue;
     // Y(k) reads h_{k-1} from the operand buffer; h_k replaces it afterwards
-    if (!waitw(c, bYFull0 + i2, par2(k))) break;
+    if (!waitw(c, bYFull0 + i2, par2(kk))) break;
     write_h();
     if (p.states) {  // each warp instruction stores one contiguous 128-byte row segment
       float *dst = p.states + ((static_cast<int64_t>(b) * p.K + k) * H + h) * PN + n;
@@ -616,7 +645,14 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
       for (int pp = 0; pp < kP; ++pp) dst[pp * kN] = hreg[pp];
     }
   }
-  if (p.final_state && !*c.abort) {
+  if (*c.abort) return;
+  if (p.agg) {
+    const int64_t bhs = (static_cast<int64_t>(b) * H + h) * p.nseg + seg;
+    float *dst = p.seg_local + bhs * PN + n;
+#pragma unroll
+    for (int pp = 0; pp < kP; ++pp) dst[pp * kN] = hreg[pp];
+    if (n == 0) p.seg_decay[bhs] = decay_log2;
+  } else if (p.final_state && k0 + nk == p.K) {
     float *dst = p.final_state + (static_cast<int64_t>(b) * H + h) * PN + n;
 #pragma unroll
     for (int pp = 0; pp < kP; ++pp) dst[pp * kN] = hreg[pp];
@@ -627,7 +663,8 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
 // warps 10..13: thread owns column p = 16 q + (lane & 15) of the clean
 // (lane < 16) or noisy (lane >= 16) stream's outputs y[t][p], t = 0..31:
 // y = exp(cum_t) Y_off + Y_diag (Y_diag already holds both directions' D x).
-__device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem, int b, int h) {
+__device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem, int b, int h,
+                               int k0, int nk) {
   const int lane = threadIdx.x & 31;
   const int q = (threadIdx.x >> 5) & 3;
   const int pcol = 16 * q + (lane & 15);
@@ -637,10 +674,12 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
   const bool mine = (noisy ? p.allblock != 0 : true) && yout != nullptr;
   const uint32_t ecum = base + kOffEc;
   const int64_t H = p.H, L = p.L;
-  for (int k = 0; k < p.K; ++k) {
-    const int i2 = k & 1, c4 = k & 3;
-    if (!waitw(c, bAux0 + (k & 1), par2(k))) break;
-    if (!waitw(c, bYFull0 + i2, par2(k))) break;
+  if (p.agg) return;
+  for (int kk = 0; kk < nk; ++kk) {
+    const int k = k0 + kk;  // global block index
+    const int i2 = kk & 1, c4 = kk & 3;
+    if (!waitw(c, bAux0 + (kk & 1), par2(kk))) break;
+    if (!waitw(c, bYFull0 + i2, par2(kk))) break;
     tc_fence_after();
     uint32_t yo[32], yd[32];
     const uint32_t ta = tmem_addr(tmem, 32 * q, kColY0 + 128 * i2);
@@ -680,9 +719,13 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t *sm = smem_raw + (base - raw);
   const int warp = threadIdx.x >> 5;
-  const int bh = blockIdx.x;
+  // CTA -> (batch row b, head h, segment seg of seg_blocks blocks)
+  const int seg = blockIdx.x % p.nseg;
+  const int bh = blockIdx.x / p.nseg;
   const int b = bh / p.H, h = bh % p.H;
   const int g = h / (p.H / p.G);
+  const int k0 = seg * p.seg_blocks;
+  const int nk = min(p.K - k0, p.seg_blocks);
 
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kOffBar);
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(sm + kOffMisc);
@@ -706,7 +749,7 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
   // clear them (and the masked-decay buffers, whose off-diagonal blocks stay
   // zero) so that no uninitialised NaN/Inf bit pattern can reach an output.
   // Build the D I_16 operands (bf16 hi + lo of each direction's D).
-  {
+  if (!p.agg) {
     const uint4 zero = make_uint4(0, 0, 0, 0);
     for (int i = 0; i < 4; ++i) {
       if (p.active[i]) continue;
@@ -747,15 +790,15 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
   Ctl c{bars, abort_flag, p.status, p.timeout_ns};
 
   if (warp == 0) {
-    if ((threadIdx.x & 31) == 0) producer(p, c, sm, b, h, g);
+    if ((threadIdx.x & 31) == 0) producer(p, c, sm, b, h, g, k0, nk);
   } else if (warp == 1) {
-    if ((threadIdx.x & 31) == 0) mma_issuer(p, c, base, tmem);
+    if ((threadIdx.x & 31) == 0) mma_issuer(p, c, base, tmem, nk);
   } else if (warp < 6) {
-    operand_group(p, c, base, b, h);
+    operand_group(p, c, base, b, h, k0, nk);
   } else if (warp < 10) {
-    state_group(p, c, base, tmem, b, h);
+    state_group(p, c, base, tmem, b, h, seg, k0, nk);
   } else {
-    epilogue_group(p, c, base, tmem, b, h);
+    epilogue_group(p, c, base, tmem, b, h, k0, nk);
   }
   tc_fence_before();
   __syncthreads();
@@ -763,6 +806,24 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
   if (warp == 1) {
     __syncwarp();
     tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ segment combine
+// Chains the segments of every (b, h) sequence: H_0 = h0 (or 0) and
+// H_{j+1} = exp(decay_j) H_j + local_j, where local_j is segment j's end state
+// from a zero start and decay_j its total decay (the aggregate pass leaves
+// both).  One thread per state element.
+__global__ void __launch_bounds__(256) bd_seg_combine_kernel(const float *h0, const float *local,
+                                                             const float *decay, float *init, int nseg) {
+  const int64_t PN = kP * kN;
+  const int64_t bh = blockIdx.x;
+  const int64_t e = static_cast<int64_t>(blockIdx.y) * 256 + threadIdx.x;
+  float hc = h0 ? h0[bh * PN + e] : 0.f;
+  for (int j = 0; j < nseg; ++j) {
+    const int64_t bj = bh * nseg + j;
+    init[bj * PN + e] = hc;
+    hc = fmaf(ex2_approx(decay[bj]), hc, local[bj * PN + e]);
   }
 }
 
@@ -833,8 +894,34 @@ bool tc_shape_ok(int64_t P, int64_t N, int64_t T, bool in_bf16) {
   return in_bf16 && P == kP && N == kN && T == kT;
 }
 
-size_t tc_workspace_bytes(int64_t Bsz, int64_t L, int64_t G) {
-  return static_cast<size_t>(4) * Bsz * (L / kT) * G * 2048;  // bf16 [32][32] per (dir, b, block, g)
+// Number of segments each (b, h) sequence is cut into: enough CTAs to fill the
+// machine several times over when there are few sequences (long prefill at
+// batch 1), at least 4 blocks per segment; one segment otherwise.
+int tc_plan_segments(int64_t Bsz, int64_t H, int64_t K) {
+  constexpr int64_t kSms = 148;
+  const int64_t chains = Bsz * H;
+  if (K < 8 || chains >= 2 * kSms) return 1;
+  int64_t nseg = (4 * kSms + chains - 1) / chains;
+  if (nseg > K / 4) nseg = K / 4;
+  if (nseg < 1) nseg = 1;
+  const int64_t seg_blocks = (K + nseg - 1) / nseg;
+  return static_cast<int>((K + seg_blocks - 1) / seg_blocks);
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// C B^T tiles (bf16 [32][32] per direction, b, block, group), then for a
+// segmented plan the segments' local end states, their initial states and
+// their decays.
+size_t tc_workspace_bytes(int64_t Bsz, int64_t L, int64_t G, int64_t H) {
+  const int64_t K = L / kT;
+  size_t bytes = align256(static_cast<size_t>(4) * Bsz * K * G * 2048);
+  const int nseg = tc_plan_segments(Bsz, H, K);
+  if (nseg > 1) {
+    const size_t states = static_cast<size_t>(Bsz) * H * nseg * kP * kN * sizeof(float);
+    bytes += 2 * align256(states) + align256(static_cast<size_t>(Bsz) * H * nseg * sizeof(float));
+  }
+  return bytes;
 }
 
 bool tc_supported(const ScanArgs &a) {
@@ -845,7 +932,7 @@ bool tc_supported(const ScanArgs &a) {
     if (d->z) return false;
   if (a.Bsz * a.H > 0x7fffffffLL || a.L > 0x7fffffffLL || 4 * a.Bsz * (a.L / kT) * a.G > 0x7fffffffLL)
     return false;
-  if (a.ws_bytes < kWsHeader + tc_workspace_bytes(a.Bsz, a.L, a.G)) return false;
+  if (a.ws_bytes < kWsHeader + tc_workspace_bytes(a.Bsz, a.L, a.G, a.H)) return false;
   const char *force = std::getenv("BDSCAN_FORCE_GENERIC");
   if (force && force[0] == '1') return false;
   return device_is_sm100();
@@ -904,6 +991,9 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
   p.H = static_cast<int>(a.H);
   p.G = static_cast<int>(a.G);
   p.K = K;
+  const int nseg = tc_plan_segments(a.Bsz, a.H, K);
+  p.nseg = nseg;
+  p.seg_blocks = (K + nseg - 1) / nseg;
   p.allblock = all ? 1 : 0;
   p.out_bf16 = a.out_bf16 ? 1 : 0;
   p.h0 = a.h0;
@@ -917,7 +1007,33 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
   e = cudaFuncSetAttribute(bd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
-  bd_tc_kernel<<<static_cast<unsigned>(a.Bsz * a.H), kThreads, kSmemBytes, stream>>>(p);
+  const unsigned grid = static_cast<unsigned>(a.Bsz * a.H * nseg);
+  if (nseg > 1) {
+    // aggregate pass (clean forward state of every segment from zero), then
+    // the chain of segment states
+    uint8_t *wsb = static_cast<uint8_t *>(a.ws) + kWsHeader;
+    const size_t cb_bytes = align256(static_cast<size_t>(4) * a.Bsz * K * a.G * 2048);
+    const size_t st_bytes = align256(static_cast<size_t>(a.Bsz) * a.H * nseg * kP * kN * sizeof(float));
+    float *seg_local = reinterpret_cast<float *>(wsb + cb_bytes);
+    float *seg_init = reinterpret_cast<float *>(wsb + cb_bytes + st_bytes);
+    float *seg_decay = reinterpret_cast<float *>(wsb + cb_bytes + 2 * st_bytes);
+    TcParams q = p;
+    q.agg = 1;
+    q.allblock = 0;
+    for (int i = 1; i < 4; ++i) q.active[i] = 0;
+    q.states = nullptr;
+    q.final_state = nullptr;
+    q.y_clean = q.y_noisy = nullptr;
+    q.seg_local = seg_local;
+    q.seg_decay = seg_decay;
+    bd_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(q);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    bd_seg_combine_kernel<<<dim3(static_cast<unsigned>(a.Bsz * a.H), (kP * kN) / 256), 256, 0, stream>>>(
+        a.h0, seg_local, seg_decay, seg_init, nseg);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    p.seg_init = seg_init;
+  }
+  bd_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(p);
   return cudaGetLastError();
 }
 

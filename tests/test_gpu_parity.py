@@ -34,6 +34,9 @@ SMALL = {
                                  nheads=2, ngroups=1, batch=1),
     "bf16_out_bf16": _shape(out_dtype="bf16"),
     "g1_h8": _shape(ngroups=1, nheads=8, batch=1, seqlen=96),
+    # few sequences, many blocks: the tensor-core path cuts each sequence into
+    # segments (aggregate pass + segment combine + main pass)
+    "bf16_segmented": _shape(batch=1, nheads=2, ngroups=1, seqlen=1280),
 }
 
 
