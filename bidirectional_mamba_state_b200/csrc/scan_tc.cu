@@ -26,8 +26,10 @@
 //                 all heads of a group -- with one M=128 tcgen05 MMA chain per
 //                 four blocks, into the workspace (bf16, 2 KB per block; the
 //                 masked-decay matrix built from it is rounded to bf16 anyway).
-//   bd_tc_kernel  one CTA per (b, h) walks its blocks in order with the fp32
-//                 state on chip.  Warp roles (448 threads, one CTA per SM):
+//   bd_tc_kernel  persistent, one CTA per SM: each CTA walks its share of the
+//                 work items -- (b, h) sequences, or segments of them -- block
+//                 by block with the fp32 state on chip, the pipeline running
+//                 on across item boundaries.  Warp roles (448 threads):
 //     warp 0      TMA producer: x, B, C and C B^T tiles of block k into a
 //                 3-slot ring (two blocks of lookahead)
 //     warp 1      TMEM allocator and single-thread tcgen05.mma issuer
@@ -39,7 +41,7 @@
 //                 + Y_diag for the block's 32 tokens and stores them; the D x
 //                 terms are small tensor-core products against D I_16 (bf16
 //                 hi + lo) accumulated into Y_diag
-//   S, Y and M are double-buffered; the h operand is single-buffered.
+//   S, Y, M and D I_16 are double-buffered; the h operand is single-buffered.
 // Every wait is bounded; on a timeout the CTA raises BDSCAN_ERR_TIMEOUT in the
 // workspace status word, drains its own copies and MMAs, frees TMEM and exits.
 //
@@ -67,7 +69,9 @@ using namespace sm100;
 
 constexpr int kT = 32, kP = 64, kN = 128;
 // stacking slots of the four directions
+// (the MMAs and the masked-decay buffers rely on: stream = slot & 1, reverse = slot >= 2)
 constexpr int kCF = 0, kNF = 1, kCR = 2, kNR = 3;
+static_assert(kCR == (kCF | 2) && kNR == (kNF | 2), "direction slots");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kStatusTimeout = -6;
 
@@ -188,10 +192,11 @@ constexpr uint32_t kOffCB = 10 * kTile;       // 4 dirs x [32 s][32 t] bf16 (SW6
 constexpr uint32_t kSlot = 12 * kTile;        // 48 KB per slot
 constexpr uint32_t kOffXw = kSlots * kSlot;   // hi [32 t][64 p], lo [32 t][64 p] (bf16, SW128)
 constexpr uint32_t kOffH = kOffXw + 2 * kTile;  // {hi, lo} x [128 n][64 p] bf16 (SW128)
-constexpr uint32_t kOffMh = kOffH + 8 * kTile;  // 2 buffers x {fwd, rev} x [64 t][64 s] interleaved
-constexpr uint32_t kMhBuf = 4 * kTile;
-constexpr uint32_t kOffDg = kOffMh + 2 * kMhBuf;  // 4 dirs x {hi, lo} x D I_16 (bf16, 512 B each)
-constexpr uint32_t kOffCum = kOffDg + 4096;       // [4 blocks][4 dirs][32] f32: cumulative decay (log2)
+constexpr uint32_t kOffMh = kOffH + 8 * kTile;  // 2 buffers x 4 dirs x [32 t][32 s] interleaved
+constexpr uint32_t kMhBuf = 4 * 2048;
+constexpr uint32_t kOffDg = kOffMh + 2 * kMhBuf;  // 2 items x 4 dirs x {hi, lo} x D I_16 (bf16, 512 B each)
+constexpr uint32_t kDgBuf = 4096;
+constexpr uint32_t kOffCum = kOffDg + 2 * kDgBuf;  // [4 blocks][4 dirs][32] f32: cumulative decay (log2)
 constexpr uint32_t kOffDt = kOffCum + 2048;       // [4][4][32] f32: dt
 constexpr uint32_t kOffEc = kOffDt + 2048;        // [4][2 fwd dirs][32] f32: exp(cum_t)
 constexpr uint32_t kOffBar = kOffEc + 1024;
@@ -204,14 +209,13 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 // matrices, t-groups 128 B apart, s-groups 256 B apart.
 constexpr uint32_t kDgSbo = 128, kDgLbo = 256;
 
-// masked-decay operand: [64 t][64 s] block diagonal (first/second direction of
-// the pair), interleaved MN-major (t contiguous): t-groups 128 B apart,
-// s-groups 1024 B apart.
-constexpr uint32_t kMhSbo = 128, kMhLbo = 1024;
+// masked-decay operand of one direction: [32 t][32 s], interleaved MN-major
+// (t contiguous): t-groups 128 B apart, s-groups 512 B apart.
+constexpr uint32_t kMhSbo = 128, kMhLbo = 512;
 
 enum : int {
-  bFull0 = 0, bFull1, bFull2, bEmpty0, bEmpty1, bEmpty2, bAux0, bAux1, bXwFull, bSFull0, bSFull1,
-  bSEmpty0, bSEmpty1, bMhFull0, bMhFull1, bHFull, bYFull0, bYFull1, bYEmpty0, bYEmpty1, bDrain, bCount
+  bFull0 = 0, bFull1, bFull2, bEmpty0, bEmpty1, bEmpty2, bAux0, bAux1, bAux2, bAux3, bXwFull, bSFull0, bSFull1,
+  bSEmpty0, bSEmpty1, bMhFull0, bMhFull1, bHFull, bHCons, bYFull0, bYFull1, bYEmpty0, bYEmpty1, bDrain, bCount
 };
 
 // TMEM columns: S^T[2] (M=128 x 64), Y^T[2] = {Y_off^T (M=64 x 64), Y_diag^T (M=64 x 64)}
@@ -230,6 +234,7 @@ struct TcParams {
   int active[4];
   int Bsz, L, H, G, K;
   int nseg, seg_blocks;  // each (b, h) sequence is walked as nseg segments of seg_blocks blocks
+  int items;             // Bsz * H * nseg work items, spread round-robin over the CTAs
   int agg;               // aggregate pass: forward state of each segment from zero, nothing else
   int allblock;
   int out_bf16;
@@ -267,6 +272,9 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
 }
 __device__ __forceinline__ void sts_f32(uint32_t addr, float v) {
   asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void sts_u16(uint32_t addr, unsigned short v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
@@ -337,8 +345,33 @@ __device__ __forceinline__ uint32_t par2(int k) { return (static_cast<uint32_t>(
 __device__ __forceinline__ int rslot(int k) { return k % kSlots; }
 __device__ __forceinline__ uint32_t parr(int k) { return static_cast<uint32_t>(k / kSlots) & 1u; }
 
+// ---------------------------------------------------------------- work items
+// A work item is one (batch row b, head h, segment seg) sequence of nk blocks
+// starting at block k0.  CTA c walks items c, c + gridDim.x, ... and every
+// role runs the same sequence of steps j = 0, 1, ... (one block of one item
+// each); ring slots, double buffers and barrier phases follow j, so the
+// pipeline runs on across item boundaries.
+struct Item {
+  int b, h, g, seg, k0, nk;
+};
+
+__device__ __forceinline__ Item item_at(const TcParams &p, int it) {
+  Item r;
+  r.seg = it % p.nseg;
+  const int bh = it / p.nseg;
+  r.b = bh / p.H;
+  r.h = bh % p.H;
+  r.g = r.h / (p.H / p.G);
+  r.k0 = r.seg * p.seg_blocks;
+  r.nk = min(p.K - r.k0, p.seg_blocks);
+  return r;
+}
+
+// 4-deep barrier ring of the per-block decay tables (phase of step j)
+__device__ __forceinline__ uint32_t par4(int j) { return (static_cast<uint32_t>(j) >> 2) & 1u; }
+
 // ---------------------------------------------------------------- producer
-__device__ void producer(const TcParams &p, const Ctl &c, uint8_t *sm, int b, int h, int g, int k0, int nk) {
+__device__ void producer(const TcParams &p, const Ctl &c, uint8_t *sm) {
   const int nact = p.active[0] + p.active[1] + p.active[2] + p.active[3];
   const uint32_t bytes = p.agg ? 3 * kTile : nact * (kTile + 2048) + (2 + (p.allblock ? 4 : 2)) * kTile;
 #pragma unroll
@@ -349,124 +382,145 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint8_t *sm, int b, in
   if (p.allblock) tma_prefetch_desc(&p.tcnf);
   tma_prefetch_desc(&p.tcb);
   int last[kSlots] = {-1, -1, -1};
-  for (int kk = 0; kk < nk; ++kk) {
-    const int k = k0 + kk;  // global block index
-    const int r = rslot(kk);
-    if (!wait1(c, bEmpty0 + r, parr(kk) ^ 1)) break;
-    uint64_t *full = &c.bar[bFull0 + r];
-    mbar_arrive_expect_tx(full, bytes);
-    uint8_t *st = sm + r * kSlot;
-    const int t0 = k * kT;
+  int j = 0;
+  bool ok = true;
+  for (int it = blockIdx.x; ok && it < p.items; it += gridDim.x) {
+    const Item I = item_at(p, it);
+    for (int kk = 0; kk < I.nk; ++kk, ++j) {
+      const int k = I.k0 + kk;  // block index in the sequence
+      const int r = rslot(j);
+      if (!wait1(c, bEmpty0 + r, parr(j) ^ 1)) {
+        ok = false;
+        break;
+      }
+      uint64_t *full = &c.bar[bFull0 + r];
+      mbar_arrive_expect_tx(full, bytes);
+      uint8_t *st = sm + r * kSlot;
+      const int t0 = k * kT;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (!p.active[i]) continue;
-      tma_load_4d(st + kOffX + i * kTile, &p.tx[i], full, 0, h, t0, b);
-      if (p.agg) continue;
-      const int idx = ((i * p.Bsz + b) * p.K + k) * p.G + g;
-      tma_load_3d(st + kOffCB + i * 2048, &p.tcb, full, 0, 0, idx);
-    }
-    tma_load_4d(st + kOffBcf, &p.tbcf, full, 0, g, t0, b);
-    tma_load_4d(st + kOffBcf + kTile, &p.tbcf, full, 64, g, t0, b);
-    if (p.agg) {
+      for (int i = 0; i < 4; ++i) {
+        if (!p.active[i]) continue;
+        tma_load_4d(st + kOffX + i * kTile, &p.tx[i], full, 0, I.h, t0, I.b);
+        if (p.agg) continue;
+        const int idx = ((i * p.Bsz + I.b) * p.K + k) * p.G + I.g;
+        tma_load_3d(st + kOffCB + i * 2048, &p.tcb, full, 0, 0, idx);
+      }
+      tma_load_4d(st + kOffBcf, &p.tbcf, full, 0, I.g, t0, I.b);
+      tma_load_4d(st + kOffBcf + kTile, &p.tbcf, full, 64, I.g, t0, I.b);
+      if (!p.agg) {
+        tma_load_4d(st + kOffClo, &p.tccf, full, 0, I.g, t0, I.b);
+        tma_load_4d(st + kOffChi, &p.tccf, full, 64, I.g, t0, I.b);
+        if (p.allblock) {
+          tma_load_4d(st + kOffClo + kTile, &p.tcnf, full, 0, I.g, t0, I.b);
+          tma_load_4d(st + kOffChi + kTile, &p.tcnf, full, 64, I.g, t0, I.b);
+        }
+      }
 #pragma unroll
-      for (int j = 0; j < kSlots; ++j)
-        if (j == r) last[j] = kk;
-      continue;
+      for (int s = 0; s < kSlots; ++s)
+        if (s == r) last[s] = j;
     }
-    tma_load_4d(st + kOffClo, &p.tccf, full, 0, g, t0, b);
-    tma_load_4d(st + kOffChi, &p.tccf, full, 64, g, t0, b);
-    if (p.allblock) {
-      tma_load_4d(st + kOffClo + kTile, &p.tcnf, full, 0, g, t0, b);
-      tma_load_4d(st + kOffChi + kTile, &p.tcnf, full, 64, g, t0, b);
-    }
-#pragma unroll
-    for (int j = 0; j < kSlots; ++j)
-      if (j == r) last[j] = kk;
   }
   // no copy into this CTA's shared memory may still be in flight at exit
 #pragma unroll
-  for (int j = 0; j < kSlots; ++j)
-    if (last[j] >= 0) (void)mbar_wait(&c.bar[bFull0 + j], parr(last[j]), p.drain_ns, nullptr);
+  for (int s = 0; s < kSlots; ++s)
+    if (last[s] >= 0) (void)mbar_wait(&c.bar[bFull0 + s], parr(last[s]), p.drain_ns, nullptr);
 }
 
 // ---------------------------------------------------------------- MMA issuer
-__device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem, int nk) {
+// Issue order per step: S; Y_off (then commit "h consumed" so the state group
+// may overwrite the h operand at once); Y_diag and the D x products.
+// Descriptors are built once; per step only their start addresses move.
+__device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
   const uint32_t id_s = idesc_bf16(128, 64, 1, 1);  // S^T[n][p] = B^T (w o X)
   const uint32_t id_yo = idesc_bf16(64, 64, 1, 0);  // Y_off^T[p][t] = h C^T
-  const uint32_t id_yd = idesc_bf16(64, 64, 1, 1);  // Y_diag^T[p][t] = X^T M^T
+  const uint32_t id_yd = idesc_bf16(64, 32, 1, 1);  // Y_diag^T[p][t] = X^T M^T, one stream
   const uint32_t id_dx = idesc_bf16(64, 16, 1, 0);  // (D x)^T[p][t] = X^T (D I_16)
-  const bool any_rev = p.active[kCR] || p.active[kNR];
-  for (int kk = 0; kk < nk; ++kk) {
-    const int r = rslot(kk), i2 = kk & 1;
-    const uint32_t st = base + r * kSlot;
-    if (!wait1(c, bFull0 + r, parr(kk))) break;
-    // ---- S^T(k) = B_cf^T (w o X): A MN-major (n; halves 4 KB apart), B MN-major (p)
-    if (!wait1(c, bXwFull, kk & 1)) break;
-    if (kk >= 2 && !wait1(c, bSEmpty0 + i2, par2(kk - 2))) break;
-    tc_fence_after();
-    const uint32_t colS = kColS0 + 64 * i2;
-    for (int ks = 0; ks < 2; ++ks) {
-      const uint64_t a = sdesc(st + kOffBcf + ks * 2048, kTile, 1024, kLayoutSw128);
-      const uint64_t bh = sdesc(base + kOffXw + ks * 2048, 0, 1024, kLayoutSw128);
-      const uint64_t bl = sdesc(base + kOffXw + kTile + ks * 2048, 0, 1024, kLayoutSw128);
-      umma_bf16(tmem + colS, a, bh, id_s, ks > 0);
-      umma_bf16(tmem + colS, a, bl, id_s, 1);
-    }
-    umma_commit(&c.bar[bSFull0 + i2]);
-    if (p.agg) {  // aggregate pass: the forward state is all it needs
-      umma_commit(&c.bar[bEmpty0 + r]);
-      continue;
-    }
-    // ---- Y^T(k): Y_off^T = h_{k-1} [C_cf; C_nf]^T;
-    //      Y_diag^T = X_fwd^T M_fwd^T + X_rev^T M_rev^T + X^T (D I) for every direction
-    if (!wait1(c, bMhFull0 + i2, par2(kk))) break;
-    if (!wait1(c, bHFull, kk & 1)) break;  // h_{k-1}
-    if (kk >= 2 && !wait1(c, bYEmpty0 + i2, par2(kk - 2))) break;
-    tc_fence_after();
-    const uint32_t colY = kColY0 + 128 * i2;
-    const uint32_t hb = base + kOffH;
-    for (int ks = 0; ks < 8; ++ks) {
-      const uint64_t ah = sdesc(hb + ks * 2048, 0, 1024, kLayoutSw128);
-      const uint64_t al = sdesc(hb + 4 * kTile + ks * 2048, 0, 1024, kLayoutSw128);
-      const uint64_t bc = sdesc(st + (ks < 4 ? kOffClo : kOffChi) + (ks & 3) * 32, 16, 1024, kLayoutSw128);
-      umma_bf16(tmem + colY, ah, bc, id_yo, ks > 0);
-      umma_bf16(tmem + colY, al, bc, id_yo, 1);
-    }
-    const uint32_t mb = base + kOffMh + i2 * kMhBuf;
-    for (int ks = 0; ks < 4; ++ks) {
-      const uint64_t a = sdesc(st + kOffX + ks * 2048, 0, 1024, kLayoutSw128);
-      const uint64_t m = sdesc(mb + ks * 2048, kMhLbo, kMhSbo, kLayoutNone);
-      umma_bf16(tmem + colY + 64, a, m, id_yd, ks > 0);
-    }
-    if (any_rev) {
-      for (int ks = 0; ks < 4; ++ks) {
-        const uint64_t a = sdesc(st + kOffX + 2 * kTile + ks * 2048, 0, 1024, kLayoutSw128);
-        const uint64_t m = sdesc(mb + 2 * kTile + ks * 2048, kMhLbo, kMhSbo, kLayoutNone);
-        umma_bf16(tmem + colY + 64, a, m, id_yd, 1);
-      }
-    }
-    // D x of every direction: 16-token diagonal blocks against D I_16 (hi + lo)
-    for (int i = 0; i < 4; ++i) {
-      if (!p.active[i]) continue;
-      const uint32_t col = colY + 64 + ((i & 1) ? 32 : 0);
+  // descriptor of each operand at its first tile; moving an operand by b bytes adds b >> 4
+  const uint64_t dBcf = sdesc(base + kOffBcf, kTile, 1024, kLayoutSw128);
+  const uint64_t dXw = sdesc(base + kOffXw, 0, 1024, kLayoutSw128);
+  const uint64_t dH = sdesc(base + kOffH, 0, 1024, kLayoutSw128);
+  const uint64_t dC = sdesc(base + kOffClo, 16, 1024, kLayoutSw128);
+  const uint64_t dX = sdesc(base + kOffX, 0, 1024, kLayoutSw128);
+  const uint64_t dM = sdesc(base + kOffMh, kMhLbo, kMhSbo, kLayoutNone);
+  const uint64_t dDg = sdesc(base + kOffDg, kDgLbo, kDgSbo, kLayoutNone);
+#define BD_OFF(bytes) (static_cast<uint64_t>((bytes) >> 4))
+  int j = 0, m = 0;
+  bool ok = true;
+  for (int it = blockIdx.x; ok && it < p.items; it += gridDim.x, ++m) {
+    const int nk = item_at(p, it).nk;
+    const uint64_t go = BD_OFF(static_cast<uint32_t>(m & 1) * kDgBuf);  // this item's D I_16 operands
+    for (int kk = 0; kk < nk; ++kk, ++j) {
+      ok = false;
+      const int r = rslot(j), i2 = j & 1;
+      const uint64_t so = BD_OFF(static_cast<uint32_t>(r) * kSlot);  // this step's ring slot
+      if (!wait1(c, bFull0 + r, parr(j))) break;
+      // ---- S^T = B_cf^T (w o X): A MN-major (n; halves 4 KB apart), B MN-major (p)
+      if (!wait1(c, bXwFull, j & 1)) break;
+      if (j >= 2 && !wait1(c, bSEmpty0 + i2, par2(j - 2))) break;
+      tc_fence_after();
+      const uint32_t colS = tmem + kColS0 + 64 * i2;
+#pragma unroll
       for (int ks = 0; ks < 2; ++ks) {
-        const uint64_t a = sdesc(st + kOffX + i * kTile + ks * 2048, 0, 1024, kLayoutSw128);
-        const uint64_t dh = sdesc(base + kOffDg + (2 * i) * 512, kDgLbo, kDgSbo, kLayoutNone);
-        const uint64_t dl = sdesc(base + kOffDg + (2 * i + 1) * 512, kDgLbo, kDgSbo, kLayoutNone);
-        umma_bf16(tmem + col + 16 * ks, a, dh, id_dx, 1);
-        umma_bf16(tmem + col + 16 * ks, a, dl, id_dx, 1);
+        umma_bf16(colS, dBcf + so + BD_OFF(ks * 2048), dXw + BD_OFF(ks * 2048), id_s, ks > 0);
+        umma_bf16(colS, dBcf + so + BD_OFF(ks * 2048), dXw + BD_OFF(kTile + ks * 2048), id_s, 1);
       }
+      umma_commit(&c.bar[bSFull0 + i2]);
+      if (p.agg) {  // aggregate pass: the forward state is all it needs
+        umma_commit(&c.bar[bEmpty0 + r]);
+        ok = true;
+        continue;
+      }
+      // ---- Y_off^T = h [C_cf; C_nf]^T, h = the state before this block
+      if (!wait1(c, bHFull, j & 1)) break;
+      if (j >= 2 && !wait1(c, bYEmpty0 + i2, par2(j - 2))) break;
+      tc_fence_after();
+      const uint32_t colY = tmem + kColY0 + 128 * i2;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint64_t bc = dC + so + BD_OFF((ks < 4 ? 0 : 2 * kTile) + (ks & 3) * 32);
+        umma_bf16(colY, dH + BD_OFF(ks * 2048), bc, id_yo, ks > 0);
+        umma_bf16(colY, dH + BD_OFF(4 * kTile + ks * 2048), bc, id_yo, 1);
+      }
+      umma_commit(&c.bar[bHCons]);  // the h operand may now be overwritten
+      // ---- Y_diag^T of each stream = X_fwd^T M_fwd^T + X_rev^T M_rev^T, then
+      //      X^T (D I) of every direction
+      if (!wait1(c, bMhFull0 + i2, par2(j))) break;
+      tc_fence_after();
+      const uint64_t mo = BD_OFF(static_cast<uint32_t>(i2) * kMhBuf);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {  // the forward direction of a stream (i < 2) is always active
+        if (!p.active[i]) continue;
+        const uint32_t col = colY + 64 + ((i & 1) ? 32 : 0);
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+          umma_bf16(col, dX + so + BD_OFF(i * kTile + ks * 2048), dM + mo + BD_OFF(i * 2048 + ks * 1024), id_yd,
+                    (i >= 2 || ks > 0) ? 1u : 0u);
+      }
+      // D x of every direction: 16-token diagonal blocks against D I_16 (hi + lo)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (!p.active[i]) continue;
+        const uint32_t col = colY + 64 + ((i & 1) ? 32 : 0);
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+          const uint64_t a = dX + so + BD_OFF(i * kTile + ks * 2048);
+          umma_bf16(col + 16 * ks, a, dDg + go + BD_OFF((2 * i) * 512), id_dx, 1);
+          umma_bf16(col + 16 * ks, a, dDg + go + BD_OFF((2 * i + 1) * 512), id_dx, 1);
+        }
+      }
+      umma_commit(&c.bar[bYFull0 + i2]);
+      umma_commit(&c.bar[bEmpty0 + r]);
+      ok = true;
     }
-    umma_commit(&c.bar[bYFull0 + i2]);
-    umma_commit(&c.bar[bEmpty0 + r]);
   }
+#undef BD_OFF
   umma_commit(&c.bar[bDrain]);
   (void)mbar_wait(&c.bar[bDrain], 0, p.drain_ns, nullptr);
 }
 
 // ---------------------------------------------------------------- operand group
 // warps 2..5; q = warp & 3 is the direction slot whose decays and M it builds.
-__device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base, int b, int h, int k0, int nk) {
+__device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
   const int lane = threadIdx.x & 31;
   const int q = (threadIdx.x >> 5) & 3;
   const int gt = threadIdx.x - 64;  // 0..127
@@ -474,113 +528,146 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base, in
   const bool rev = q >= 2;
   const uint32_t cum = base + kOffCum, dts = base + kOffDt, ecum = base + kOffEc;
   const int64_t H = p.H, L = p.L;
-  const float A2 = act ? pick4(p.A, q)[h] * kLog2e : 0.f;
+  const float *Ap = pick4(p.A, q);
   const __nv_bfloat16 *dtp = pick4(p.dt, q);
-  auto load_dt = [&](int kk) -> float {  // dt of local block kk of this segment
-    if (!act || kk >= nk) return 0.f;
-    return __bfloat162float(dtp[(static_cast<int64_t>(b) * L + (k0 + kk) * kT + lane) * H + h]);
+  auto load_dt = [&](const Item &I, int kk) -> float {  // dt of block kk of item I
+    if (!act) return 0.f;
+    return __bfloat162float(dtp[(static_cast<int64_t>(I.b) * L + (I.k0 + kk) * kT + lane) * H + I.h]);
   };
-  float dt_next = load_dt(0);
-  // position of this direction's block in the stacked [64 t][64 s] operand
-  const uint32_t mset = rev ? 2 * kTile : 0;
-  const uint32_t d0 = (q & 1) ? 32 : 0;
-  for (int kk = 0; kk < nk; ++kk) {
-    const int s = kk & 1, i2 = kk & 1, c4 = kk & 3;
-    const uint32_t st = base + rslot(kk) * kSlot;
-    const float dt_cur = dt_next;
-    dt_next = load_dt(kk + 1);
-    // ---- decays of this warp's direction (log2 units): prefix sum (forward)
-    //      or suffix sum (reverse) over the block
-    float v = dt_cur * A2;
-    if (act) {
-      if (!rev) {
+  int j = 0, m = 0;
+  bool ok = true;
+  int it = blockIdx.x;
+  if (it >= p.items) return;
+  Item I = item_at(p, it);
+  float dt_next = load_dt(I, 0);
+  for (; ok && it < p.items; ++m) {
+    const float A2 = act ? Ap[I.h] * kLog2e : 0.f;
+    const int it_next = it + gridDim.x;
+    const Item In = it_next < p.items ? item_at(p, it_next) : I;
+    for (int kk = 0; kk < I.nk; ++kk, ++j) {
+      ok = false;
+      const int i2 = j & 1, c4 = j & 3;
+      const uint32_t st = base + rslot(j) * kSlot;
+      const float dt_cur = dt_next;
+      if (kk + 1 < I.nk)
+        dt_next = load_dt(I, kk + 1);
+      else if (it_next < p.items)
+        dt_next = load_dt(In, 0);
+      // ---- decays of this warp's direction (log2 units): prefix sum (forward)
+      //      or suffix sum (reverse) over the block
+      float v = dt_cur * A2;
+      if (act) {
+        if (!rev) {
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const float u = __shfl_up_sync(0xffffffffu, v, o);
-          if (lane >= o) v += u;
-        }
-      } else {
+          for (int o = 1; o < 32; o <<= 1) {
+            const float u = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += u;
+          }
+        } else {
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const float u = __shfl_down_sync(0xffffffffu, v, o);
-          if (lane + o < 32) v += u;
+          for (int o = 1; o < 32; o <<= 1) {
+            const float u = __shfl_down_sync(0xffffffffu, v, o);
+            if (lane + o < 32) v += u;
+          }
         }
+        sts_f32(cum + ((c4 * 4 + q) * 32 + lane) * 4, v);
+        sts_f32(dts + ((c4 * 4 + q) * 32 + lane) * 4, dt_cur);
+        if (!rev) sts_f32(ecum + ((c4 * 2 + q) * 32 + lane) * 4, ex2_approx(v));
       }
-      sts_f32(cum + ((c4 * 4 + q) * 32 + lane) * 4, v);
-      sts_f32(dts + ((c4 * 4 + q) * 32 + lane) * 4, dt_cur);
-      if (!rev) sts_f32(ecum + ((c4 * 2 + q) * 32 + lane) * 4, ex2_approx(v));
-    }
-    arrive_lane0(c, bAux0 + s);
-    if (!waitw(c, bAux0 + s, par2(kk))) break;
-    // ---- (w o X) of the clean forward direction, bf16 hi + lo
-    if (kk >= 1 && !waitw(c, bSFull0 + ((kk + 1) & 1), par2(kk - 1))) break;  // S(k-1) read Xw
-    if (!waitw(c, bFull0 + rslot(kk), parr(kk))) break;
-    {
-      const uint32_t cf = cum + (c4 * 4 + kCF) * 128, df = dts + (c4 * 4 + kCF) * 128;
-      const float c31 = lds_f32(cf + 31 * 4);
+      arrive_lane0(c, bAux0 + c4);
+      if (!waitw(c, bAux0 + c4, par4(j))) break;
+      // ---- (w o X) of the clean forward direction, bf16 hi + lo
+      if (j >= 1 && !waitw(c, bSFull0 + ((j + 1) & 1), par2(j - 1))) break;  // S(j-1) read Xw
+      if (!waitw(c, bFull0 + rslot(j), parr(j))) break;
+      {
+        const uint32_t cf = cum + (c4 * 4 + kCF) * 128, df = dts + (c4 * 4 + kCF) * 128;
+        const float c31 = lds_f32(cf + 31 * 4);
 #pragma unroll
-      for (int rep = 0; rep < 2; ++rep) {
-        const int i = gt + 128 * rep;
-        const int t = i >> 3, ch = i & 7;
-        const uint32_t off = sw128_chunk(t, ch);
-        uint32_t r0, r1, r2, r3;
-        ld_shared_v4(st + kOffX + off, r0, r1, r2, r3);
-        const float w = lds_f32(df + t * 4) * ex2_approx(c31 - lds_f32(cf + t * 4));
-        float vv[8] = {bf16_lo_f(r0) * w, bf16_hi_f(r0) * w, bf16_lo_f(r1) * w, bf16_hi_f(r1) * w,
-                       bf16_lo_f(r2) * w, bf16_hi_f(r2) * w, bf16_lo_f(r3) * w, bf16_hi_f(r3) * w};
-        store_split8(base + kOffXw + off, base + kOffXw + kTile + off, vv);
+        for (int rep = 0; rep < 2; ++rep) {
+          const int i = gt + 128 * rep;
+          const int t = i >> 3, ch = i & 7;
+          const uint32_t off = sw128_chunk(t, ch);
+          uint32_t r0, r1, r2, r3;
+          ld_shared_v4(st + kOffX + off, r0, r1, r2, r3);
+          const float w = lds_f32(df + t * 4) * ex2_approx(c31 - lds_f32(cf + t * 4));
+          float vv[8] = {bf16_lo_f(r0) * w, bf16_hi_f(r0) * w, bf16_lo_f(r1) * w, bf16_hi_f(r1) * w,
+                         bf16_lo_f(r2) * w, bf16_hi_f(r2) * w, bf16_lo_f(r3) * w, bf16_hi_f(r3) * w};
+          store_split8(base + kOffXw + off, base + kOffXw + kTile + off, vv);
+        }
+        fence_proxy_async_smem();
+        arrive_lane0(c, bXwFull);
+      }
+      if (!p.agg) {
+        // the epilogue of step j-2 has released its Y buffer: the MMAs that
+        // read this M buffer (and, at an item's first step, the D I_16 buffer
+        // of two items back) are complete, and the epilogue has read its
+        // decay tables
+        if (j >= 2 && !waitw(c, bYEmpty0 + i2, par2(j - 2))) break;
+        if (kk == 0 && gt < 64) {
+          // D I_16 operands of this item: bf16 hi + lo of each direction's D
+          // on the diagonal (the rest of the buffer stays zero)
+          const int i = gt >> 4, d = gt & 15;
+          if (pick4(p.active, i)) {
+            const float Dv = pick4(p.D, i)[I.h];
+            const __nv_bfloat16 dh = __float2bfloat16_rn(Dv);
+            const __nv_bfloat16 dl = __float2bfloat16_rn(Dv - __bfloat162float(dh));
+            const uint32_t off = (m & 1) * kDgBuf + (d >> 3) * kDgSbo + (d >> 3) * kDgLbo + (d & 7) * 16 + (d & 7) * 2;
+            sts_u16(base + kOffDg + (2 * i) * 512 + off, __bfloat16_as_ushort(dh));
+            sts_u16(base + kOffDg + (2 * i + 1) * 512 + off, __bfloat16_as_ushort(dl));
+          }
+        }
+        // ---- masked-decay matrix, row s = lane of M^T for this direction
+        if (act) {
+          const uint32_t cbrow = st + kOffCB + q * 2048;
+          float cbv[32];
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t r0, r1, r2, r3;
+            ld_shared_v4(cbrow + sw64_chunk(lane, ch), r0, r1, r2, r3);
+            cbv[8 * ch] = bf16_lo_f(r0);
+            cbv[8 * ch + 1] = bf16_hi_f(r0);
+            cbv[8 * ch + 2] = bf16_lo_f(r1);
+            cbv[8 * ch + 3] = bf16_hi_f(r1);
+            cbv[8 * ch + 4] = bf16_lo_f(r2);
+            cbv[8 * ch + 5] = bf16_hi_f(r2);
+            cbv[8 * ch + 6] = bf16_lo_f(r3);
+            cbv[8 * ch + 7] = bf16_hi_f(r3);
+          }
+          const uint32_t cq = cum + (c4 * 4 + q) * 128;
+          const float cs = v, ds = dt_cur;
+          const uint32_t mrow = base + kOffMh + i2 * kMhBuf + q * 2048;
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            float cj[8];
+            ld_shared_v4f(cq + 32 * jj, *reinterpret_cast<float(*)[4]>(&cj[0]));
+            ld_shared_v4f(cq + 32 * jj + 16, *reinterpret_cast<float(*)[4]>(&cj[4]));
+            float mv[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int t = 8 * jj + i;
+              const bool valid = rev ? (t <= lane) : (t >= lane);
+              const float e = ex2_approx(cj[i] - cs);
+              mv[i] = valid ? cbv[t] * ds * e : 0.f;
+            }
+            st_shared_v4(mrow + inter_mn_off(8 * jj, lane, kMhSbo, kMhLbo), pack_bf16x2(mv[0], mv[1]),
+                         pack_bf16x2(mv[2], mv[3]), pack_bf16x2(mv[4], mv[5]), pack_bf16x2(mv[6], mv[7]));
+          }
+        }
       }
       fence_proxy_async_smem();
-      arrive_lane0(c, bXwFull);
+      arrive_lane0(c, bMhFull0 + i2);
+      arrive_lane0(c, bEmpty0 + rslot(j));
+      ok = true;
     }
-    // ---- masked-decay matrix, row s = lane of M^T for this direction
-    if (!p.agg && kk >= 2 && !waitw(c, bYFull0 + i2, par2(kk - 2))) break;  // Y(k-2) read this M buffer
-    if (act && !p.agg) {
-      const uint32_t cbrow = st + kOffCB + q * 2048;
-      float cbv[32];
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t r0, r1, r2, r3;
-        ld_shared_v4(cbrow + sw64_chunk(lane, ch), r0, r1, r2, r3);
-        cbv[8 * ch] = bf16_lo_f(r0);
-        cbv[8 * ch + 1] = bf16_hi_f(r0);
-        cbv[8 * ch + 2] = bf16_lo_f(r1);
-        cbv[8 * ch + 3] = bf16_hi_f(r1);
-        cbv[8 * ch + 4] = bf16_lo_f(r2);
-        cbv[8 * ch + 5] = bf16_hi_f(r2);
-        cbv[8 * ch + 6] = bf16_lo_f(r3);
-        cbv[8 * ch + 7] = bf16_hi_f(r3);
-      }
-      const uint32_t cq = cum + (c4 * 4 + q) * 128;
-      const float cs = v, ds = dt_cur;
-      const uint32_t mrow = base + kOffMh + i2 * kMhBuf + mset;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float cj[8];
-        ld_shared_v4f(cq + 32 * j, *reinterpret_cast<float(*)[4]>(&cj[0]));
-        ld_shared_v4f(cq + 32 * j + 16, *reinterpret_cast<float(*)[4]>(&cj[4]));
-        float m[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int t = 8 * j + i;
-          const bool valid = rev ? (t <= lane) : (t >= lane);
-          const float e = ex2_approx(cj[i] - cs);
-          m[i] = valid ? cbv[t] * ds * e : 0.f;
-        }
-        st_shared_v4(mrow + inter_mn_off(d0 + 8 * j, d0 + lane, kMhSbo, kMhLbo), pack_bf16x2(m[0], m[1]),
-                     pack_bf16x2(m[2], m[3]), pack_bf16x2(m[4], m[5]), pack_bf16x2(m[6], m[7]));
-      }
-    }
-    fence_proxy_async_smem();
-    arrive_lane0(c, bMhFull0 + i2);
-    arrive_lane0(c, bEmpty0 + rslot(kk));
+    it = it_next;
+    I = In;
   }
 }
 
 // ---------------------------------------------------------------- state group
 // warps 6..9: thread owns column n = 32 q + lane of the state, h^T[n][0..63].
-__device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem, int b, int h,
-                            int seg, int k0, int nk) {
+// A failed (timed-out) wait ends the group at once: nothing else is stored.
+__device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
   const int lane = threadIdx.x & 31;
   const int q = (threadIdx.x >> 5) & 3;
   const int n = 32 * q + lane;
@@ -588,17 +675,6 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
   const int64_t H = p.H;
   const int64_t PN = kP * kN;
   float hreg[kP];
-  {
-    // initial state of this segment: h0 (first segment), the chained state the
-    // aggregate and combine passes left in the workspace (later segments), or
-    // zero (aggregate pass)
-    const int64_t bhs = (static_cast<int64_t>(b) * H + h) * p.nseg + seg;
-    const float *src = p.agg ? nullptr
-                       : seg == 0 ? (p.h0 ? p.h0 + (static_cast<int64_t>(b) * H + h) * PN + n : nullptr)
-                                  : p.seg_init + bhs * PN + n;
-#pragma unroll
-    for (int pp = 0; pp < kP; ++pp) hreg[pp] = src ? src[pp * kN] : 0.f;
-  }
   // h operand of Y_off^T (A, MN-major): {hi, lo} x [128 n rows][64 p] (SW128)
   auto write_h = [&]() {
     const uint32_t hb = base + kOffH;
@@ -610,52 +686,81 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
     fence_proxy_async_smem();
     arrive_lane0(c, bHFull);
   };
-  if (!p.agg) write_h();  // h_{-1}
-  float decay_log2 = 0.f;  // total decay over the segment (aggregate pass)
-  for (int kk = 0; kk < nk; ++kk) {
-    const int k = k0 + kk;  // global block index
-    const int i2 = kk & 1, c4 = kk & 3;
-    if (!waitw(c, bAux0 + (kk & 1), par2(kk))) break;
-    const float c31 = lds_f32(cum + ((c4 * 4 + kCF) * 32 + 31) * 4);
-    const float atot = ex2_approx(c31);
-    decay_log2 += c31;
-    if (!waitw(c, bSFull0 + i2, par2(kk))) break;
-    tc_fence_after();
+  int j = 0;
+  for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
+    int nk;
+    float *sdst;  // boundary states of this item's blocks, [B][K][H][P][N]
     {
-      uint32_t sv[32];
-      const uint32_t ta = tmem_addr(tmem, 32 * q, kColS0 + 64 * i2);
-      tmem_ld_32x32b_x32(ta, sv);
-      tmem_ld_wait();
+      const Item I = item_at(p, it);
+      nk = I.nk;
+      const int64_t bh = static_cast<int64_t>(I.b) * H + I.h;
+      sdst = p.states ? p.states + ((static_cast<int64_t>(I.b) * p.K + I.k0) * H + I.h) * PN + n : nullptr;
+      // initial state of this item: h0 (first segment), the chained state the
+      // aggregate and combine passes left in the workspace (later segments),
+      // or zero (aggregate pass)
+      const float *src = p.agg ? nullptr
+                         : I.seg == 0 ? (p.h0 ? p.h0 + bh * PN + n : nullptr)
+                                      : p.seg_init + (bh * p.nseg + I.seg) * PN + n;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) hreg[i] = fmaf(atot, hreg[i], __uint_as_float(sv[i]));
-      tmem_ld_32x32b_x32(ta + 32, sv);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) hreg[32 + i] = fmaf(atot, hreg[32 + i], __uint_as_float(sv[i]));
+      for (int pp = 0; pp < kP; ++pp) hreg[pp] = src ? src[pp * kN] : 0.f;
     }
-    tc_fence_before();
-    arrive_lane0(c, bSEmpty0 + i2);
-    if (p.agg) continue;
-    // Y(k) reads h_{k-1} from the operand buffer; h_k replaces it afterwards
-    if (!waitw(c, bYFull0 + i2, par2(kk))) break;
-    write_h();
-    if (p.states) {  // each warp instruction stores one contiguous 128-byte row segment
-      float *dst = p.states + ((static_cast<int64_t>(b) * p.K + k) * H + h) * PN + n;
+    if (!p.agg) {
+      // Y_off of the previous step (another item's last block) has read the
+      // h operand; this item's initial state replaces it
+      if (j >= 1 && !waitw(c, bHCons, (j - 1) & 1)) return;
+      write_h();
+    }
+    float decay_log2 = 0.f;  // total decay over the item (aggregate pass)
+    for (int kk = 0; kk < nk; ++kk, ++j) {
+      const int i2 = j & 1, c4 = j & 3;
+      if (!waitw(c, bAux0 + c4, par4(j))) return;
+      const float c31 = lds_f32(cum + ((c4 * 4 + kCF) * 32 + 31) * 4);
+      const float atot = ex2_approx(c31);
+      decay_log2 += c31;
+      if (!waitw(c, bSFull0 + i2, par2(j))) return;
+      tc_fence_after();
+      {
+        const uint32_t ta = tmem_addr(tmem, 32 * q, kColS0 + 64 * i2);
+#pragma unroll
+        for (int cq = 0; cq < 4; ++cq) {
+          uint32_t sv[16];
+          tmem_ld_32x32b_x16(ta + 16 * cq, sv);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) hreg[16 * cq + i] = fmaf(atot, hreg[16 * cq + i], __uint_as_float(sv[i]));
+        }
+      }
+      tc_fence_before();
+      arrive_lane0(c, bSEmpty0 + i2);
+      if (!p.agg) {
+        if (kk + 1 < nk) {
+          // Y_off of this step reads the state before the block from the
+          // operand buffer; the state after it replaces it for the next step
+          if (!waitw(c, bHCons, j & 1)) return;
+          write_h();
+        }
+        if (sdst) {  // each warp instruction stores one contiguous 128-byte row segment
+#pragma unroll
+          for (int pp = 0; pp < kP; ++pp) sdst[pp * kN] = hreg[pp];
+          sdst += H * PN;
+        }
+      }
+    }
+    if (*c.abort) return;
+    // (item coordinates recomputed rather than kept live through the block loop)
+    const Item E = item_at(p, it);
+    const int64_t ebh = static_cast<int64_t>(E.b) * H + E.h;
+    if (p.agg) {
+      const int64_t ebhs = ebh * p.nseg + E.seg;
+      float *dst = p.seg_local + ebhs * PN + n;
+#pragma unroll
+      for (int pp = 0; pp < kP; ++pp) dst[pp * kN] = hreg[pp];
+      if (n == 0) p.seg_decay[ebhs] = decay_log2;
+    } else if (p.final_state && E.k0 + E.nk == p.K) {
+      float *dst = p.final_state + ebh * PN + n;
 #pragma unroll
       for (int pp = 0; pp < kP; ++pp) dst[pp * kN] = hreg[pp];
     }
-  }
-  if (*c.abort) return;
-  if (p.agg) {
-    const int64_t bhs = (static_cast<int64_t>(b) * H + h) * p.nseg + seg;
-    float *dst = p.seg_local + bhs * PN + n;
-#pragma unroll
-    for (int pp = 0; pp < kP; ++pp) dst[pp * kN] = hreg[pp];
-    if (n == 0) p.seg_decay[bhs] = decay_log2;
-  } else if (p.final_state && k0 + nk == p.K) {
-    float *dst = p.final_state + (static_cast<int64_t>(b) * H + h) * PN + n;
-#pragma unroll
-    for (int pp = 0; pp < kP; ++pp) dst[pp * kN] = hreg[pp];
   }
 }
 
@@ -663,8 +768,7 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
 // warps 10..13: thread owns column p = 16 q + (lane & 15) of the clean
 // (lane < 16) or noisy (lane >= 16) stream's outputs y[t][p], t = 0..31:
 // y = exp(cum_t) Y_off + Y_diag (Y_diag already holds both directions' D x).
-__device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem, int b, int h,
-                               int k0, int nk) {
+__device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
   const int lane = threadIdx.x & 31;
   const int q = (threadIdx.x >> 5) & 3;
   const int pcol = 16 * q + (lane & 15);
@@ -675,40 +779,49 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
   const uint32_t ecum = base + kOffEc;
   const int64_t H = p.H, L = p.L;
   if (p.agg) return;
-  for (int kk = 0; kk < nk; ++kk) {
-    const int k = k0 + kk;  // global block index
-    const int i2 = kk & 1, c4 = kk & 3;
-    if (!waitw(c, bAux0 + (kk & 1), par2(kk))) break;
-    if (!waitw(c, bYFull0 + i2, par2(kk))) break;
-    tc_fence_after();
-    uint32_t yo[32], yd[32];
-    const uint32_t ta = tmem_addr(tmem, 32 * q, kColY0 + 128 * i2);
-    tmem_ld_16x32bx2_x32<32>(ta, yo);
-    tmem_ld_16x32bx2_x32<32>(ta + 64, yd);
-    tmem_ld_wait();
-    tc_fence_before();
-    arrive_lane0(c, bYEmpty0 + i2);
-    if (mine) {
+  int j = 0;
+  bool ok = true;
+  for (int it = blockIdx.x; ok && it < p.items; it += gridDim.x) {
+    const Item I = item_at(p, it);
+    for (int kk = 0; kk < I.nk; ++kk, ++j) {
+      ok = false;
+      const int k = I.k0 + kk;  // block index in the sequence
+      const int i2 = j & 1, c4 = j & 3;
+      if (!waitw(c, bAux0 + c4, par4(j))) break;
+      if (!waitw(c, bYFull0 + i2, par2(j))) break;
+      tc_fence_after();
+      uint32_t yo[32], yd[32];
+      const uint32_t ta = tmem_addr(tmem, 32 * q, kColY0 + 128 * i2);
+      tmem_ld_16x32bx2_x32<32>(ta, yo);
+      tmem_ld_16x32bx2_x32<32>(ta + 64, yd);
+      tmem_ld_wait();
       const uint32_t eq = ecum + (c4 * 2 + fs) * 128;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int jj = 0; jj < 8; ++jj) {
         float e4[4];
-        ld_shared_v4f(eq + 16 * j, e4);
+        ld_shared_v4f(eq + 16 * jj, e4);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          yo[4 * j + i] = __float_as_uint(fmaf(e4[i], __uint_as_float(yo[4 * j + i]), __uint_as_float(yd[4 * j + i])));
+          yo[4 * jj + i] =
+              __float_as_uint(fmaf(e4[i], __uint_as_float(yo[4 * jj + i]), __uint_as_float(yd[4 * jj + i])));
       }
-      const int64_t yi = ((static_cast<int64_t>(b) * L + k * kT) * H + h) * kP + pcol;
-      const int64_t tstride = H * kP;
-      if (p.out_bf16) {
-        __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(yout) + yi;
+      // the Y buffer and this step's decay tables may be reused from here on
+      tc_fence_before();
+      arrive_lane0(c, bYEmpty0 + i2);
+      if (mine) {
+        const int64_t yi = ((static_cast<int64_t>(I.b) * L + k * kT) * H + I.h) * kP + pcol;
+        const int64_t tstride = H * kP;
+        if (p.out_bf16) {
+          __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(yout) + yi;
 #pragma unroll
-        for (int t = 0; t < 32; ++t) dst[t * tstride] = __float2bfloat16_rn(__uint_as_float(yo[t]));
-      } else {
-        float *dst = reinterpret_cast<float *>(yout) + yi;
+          for (int t = 0; t < 32; ++t) dst[t * tstride] = __float2bfloat16_rn(__uint_as_float(yo[t]));
+        } else {
+          float *dst = reinterpret_cast<float *>(yout) + yi;
 #pragma unroll
-        for (int t = 0; t < 32; ++t) dst[t * tstride] = __uint_as_float(yo[t]);
+          for (int t = 0; t < 32; ++t) dst[t * tstride] = __uint_as_float(yo[t]);
+        }
       }
+      ok = true;
     }
   }
 }
@@ -719,13 +832,6 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t *sm = smem_raw + (base - raw);
   const int warp = threadIdx.x >> 5;
-  // CTA -> (batch row b, head h, segment seg of seg_blocks blocks)
-  const int seg = blockIdx.x % p.nseg;
-  const int bh = blockIdx.x / p.nseg;
-  const int b = bh / p.H, h = bh % p.H;
-  const int g = h / (p.H / p.G);
-  const int k0 = seg * p.seg_blocks;
-  const int nk = min(p.K - k0, p.seg_blocks);
 
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kOffBar);
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(sm + kOffMisc);
@@ -736,7 +842,7 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
     for (int i = 0; i < bCount; ++i) {
       uint32_t cnt = 4;
       if (i == bFull0 || i == bFull1 || i == bFull2 || i == bSFull0 || i == bSFull1 || i == bYFull0 ||
-          i == bYFull1 || i == bDrain)
+          i == bYFull1 || i == bHCons || i == bDrain)
         cnt = 1;
       else if (i == bEmpty0 || i == bEmpty1 || i == bEmpty2)
         cnt = 5;
@@ -745,38 +851,19 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
     *abort_flag = 0;
     fence_mbar_init();
   }
-  // x tiles of inactive directions are read next to zero operands by the MMAs:
-  // clear them (and the masked-decay buffers, whose off-diagonal blocks stay
-  // zero) so that no uninitialised NaN/Inf bit pattern can reach an output.
-  // Build the D I_16 operands (bf16 hi + lo of each direction's D).
+  // Without a noisy stream, Y_off still reads the noisy half of the stacked C
+  // operand: clear it so that no uninitialised NaN/Inf bit pattern is ever
+  // multiplied.  Clear the D I_16 buffers (only their diagonals are written).
   if (!p.agg) {
     const uint4 zero = make_uint4(0, 0, 0, 0);
-    for (int i = 0; i < 4; ++i) {
-      if (p.active[i]) continue;
-      for (int r = 0; r < kSlots; ++r)
-        for (uint32_t o = threadIdx.x * 16; o < kTile; o += kThreads * 16)
-          *reinterpret_cast<uint4 *>(sm + r * kSlot + kOffX + i * kTile + o) = zero;
-    }
     if (!p.allblock)
       for (int r = 0; r < kSlots; ++r)
         for (uint32_t o = threadIdx.x * 16; o < kTile; o += kThreads * 16) {
           *reinterpret_cast<uint4 *>(sm + r * kSlot + kOffClo + kTile + o) = zero;
           *reinterpret_cast<uint4 *>(sm + r * kSlot + kOffChi + kTile + o) = zero;
         }
-    for (uint32_t o = threadIdx.x * 16; o < 2 * kMhBuf + 4096; o += kThreads * 16)
-      *reinterpret_cast<uint4 *>(sm + kOffMh + o) = zero;  // M buffers and D I_16 tiles
-    __syncthreads();
-    if (threadIdx.x < 4 * 16) {
-      const int i = threadIdx.x >> 4, d = threadIdx.x & 15;
-      if (p.active[i]) {
-        const float Dv = pick4(p.D, i)[h];
-        const __nv_bfloat16 dh = __float2bfloat16_rn(Dv);
-        const __nv_bfloat16 dl = __float2bfloat16_rn(Dv - __bfloat162float(dh));
-        const uint32_t off = (d >> 3) * kDgSbo + (d >> 3) * kDgLbo + (d & 7) * 16 + (d & 7) * 2;
-        *reinterpret_cast<__nv_bfloat16 *>(sm + kOffDg + (2 * i) * 512 + off) = dh;
-        *reinterpret_cast<__nv_bfloat16 *>(sm + kOffDg + (2 * i + 1) * 512 + off) = dl;
-      }
-    }
+    for (uint32_t o = threadIdx.x * 16; o < 2 * kDgBuf; o += kThreads * 16)
+      *reinterpret_cast<uint4 *>(sm + kOffDg + o) = zero;
     fence_proxy_async_smem();
   }
   if (warp == 1) {
@@ -790,15 +877,15 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
   Ctl c{bars, abort_flag, p.status, p.timeout_ns};
 
   if (warp == 0) {
-    if ((threadIdx.x & 31) == 0) producer(p, c, sm, b, h, g, k0, nk);
+    if ((threadIdx.x & 31) == 0) producer(p, c, sm);
   } else if (warp == 1) {
-    if ((threadIdx.x & 31) == 0) mma_issuer(p, c, base, tmem, nk);
+    if ((threadIdx.x & 31) == 0) mma_issuer(p, c, base, tmem);
   } else if (warp < 6) {
-    operand_group(p, c, base, b, h, k0, nk);
+    operand_group(p, c, base);
   } else if (warp < 10) {
-    state_group(p, c, base, tmem, b, h, seg, k0, nk);
+    state_group(p, c, base, tmem);
   } else {
-    epilogue_group(p, c, base, tmem, b, h, k0, nk);
+    epilogue_group(p, c, base, tmem);
   }
   tc_fence_before();
   __syncthreads();
@@ -994,6 +1081,7 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
   const int nseg = tc_plan_segments(a.Bsz, a.H, K);
   p.nseg = nseg;
   p.seg_blocks = (K + nseg - 1) / nseg;
+  p.items = static_cast<int>(a.Bsz * a.H * nseg);
   p.allblock = all ? 1 : 0;
   p.out_bf16 = a.out_bf16 ? 1 : 0;
   p.h0 = a.h0;
@@ -1007,7 +1095,12 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
   e = cudaFuncSetAttribute(bd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
-  const unsigned grid = static_cast<unsigned>(a.Bsz * a.H * nseg);
+  // persistent CTAs, one per SM, each walking its share of the work items
+  int dev = 0, nsm = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  const unsigned grid = static_cast<unsigned>(p.items < nsm ? p.items : nsm);
   if (nseg > 1) {
     // aggregate pass (clean forward state of every segment from zero), then
     // the chain of segment states
