@@ -89,6 +89,7 @@ struct CbParams {
   int slot[4];  // blockIdx.z -> stacking slot
   int Bsz, K, G;
   __nv_bfloat16 *cb;  // [4][B][K][G][32 s][32 t]
+  int *item_counters;  // the scan passes' work-item counters, zeroed here
   int *status;
   unsigned long long timeout_ns;
 };
@@ -111,6 +112,7 @@ __global__ void __launch_bounds__(kCbThreads) bd_cb_kernel(const __grid_constant
   const int b = blockIdx.y / p.G, g = blockIdx.y % p.G;
   const int k0 = 4 * blockIdx.x;
   const int nvalid = min(4, p.K - k0);
+  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x < 2) p.item_counters[threadIdx.x] = 0;
   if (threadIdx.x == 0) {
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
@@ -200,9 +202,11 @@ constexpr uint32_t kOffCum = kOffDg + 2 * kDgBuf;  // [4 blocks][4 dirs][32] f32
 constexpr uint32_t kOffDt = kOffCum + 2048;       // [4][4][32] f32: dt
 constexpr uint32_t kOffEc = kOffDt + 2048;        // [4][2 fwd dirs][32] f32: exp(cum_t)
 constexpr uint32_t kOffBar = kOffEc + 1024;
-constexpr int kNumBars = 32;
-constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
-constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;
+constexpr int kNumBars = 48;
+constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // TMEM base, abort flag
+constexpr int kItemRing = 16;
+constexpr uint32_t kOffItemQ = kOffMisc + 64;             // int[kItemRing]: published work items
+constexpr uint32_t kSmemBytes = kOffItemQ + 4 * kItemRing + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 // D I_16 operand (B of the D x MMAs): [16 t][16 s] interleaved K-major, 8x8 core
@@ -215,7 +219,8 @@ constexpr uint32_t kMhSbo = 128, kMhLbo = 512;
 
 enum : int {
   bFull0 = 0, bFull1, bFull2, bEmpty0, bEmpty1, bEmpty2, bAux0, bAux1, bAux2, bAux3, bXwFull, bSFull0, bSFull1,
-  bSEmpty0, bSEmpty1, bMhFull0, bMhFull1, bHFull, bHCons, bYFull0, bYFull1, bYEmpty0, bYEmpty1, bDrain, bCount
+  bSEmpty0, bSEmpty1, bMhFull0, bMhFull1, bHFull, bHCons, bYFull0, bYFull1, bYEmpty0, bYEmpty1, bDrain,
+  bItem0, bCount = bItem0 + kItemRing
 };
 
 // TMEM columns: S^T[2] (M=128 x 64), Y^T[2] = {Y_off^T (M=64 x 64), Y_diag^T (M=64 x 64)}
@@ -234,8 +239,11 @@ struct TcParams {
   int active[4];
   int Bsz, L, H, G, K;
   int nseg, seg_blocks;  // each (b, h) sequence is walked as nseg segments of seg_blocks blocks
-  int items;             // Bsz * H * nseg work items, spread round-robin over the CTAs
+  int items;             // Bsz * H * nseg work items, handed out one at a time
+  int *item_counter;     // next unclaimed work item (zeroed by the C B^T kernel)
   int agg;               // aggregate pass: forward state of each segment from zero, nothing else
+  int need_s;            // the state after a block is used (outputs, next block, aggregate); if not
+                         // (one-block items, no state outputs), S, w o X and the state update are skipped
   int allblock;
   int out_bf16;
   const float *seg_init;  // [B][H][nseg][P][N] initial state of every segment (nseg > 1)
@@ -306,28 +314,44 @@ __device__ __forceinline__ void store_split8(uint32_t addr_hi, uint32_t addr_lo,
   st_shared_v4(addr_lo, lo[0], lo[1], lo[2], lo[3]);
 }
 
+// The CTA's barrier array and control block, by shared-memory address (one
+// register each).  Control block: +0 TMEM base, +4 abort flag, +8 wait limit
+// (ns, u64), +16 status word pointer (u64).
 struct Ctl {
-  uint64_t *bar;
-  volatile int *abort;
-  int *status;
-  unsigned long long timeout_ns;
+  uint32_t bar;   // barrier 0
+  uint32_t misc;  // control block
 };
+__device__ __forceinline__ uint32_t bar_at(const Ctl &c, int i) { return c.bar + 8u * static_cast<uint32_t>(i); }
 
-__device__ __noinline__ void raise_timeout_p(volatile int *abort, int *status) {
-  *abort = 1;
-  atomicCAS(status, 0, kStatusTimeout);
+__device__ __forceinline__ uint64_t lds_u64(uint32_t addr) {
+  uint64_t v;
+  asm volatile("ld.shared.u64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
+  return v;
 }
-__device__ __forceinline__ void raise_timeout(const Ctl &c) { raise_timeout_p(c.abort, c.status); }
+
+__device__ __noinline__ void raise_timeout_s(uint32_t misc) {
+  asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(misc + 4), "r"(1u) : "memory");
+  atomicCAS(reinterpret_cast<int *>(lds_u64(misc + 16)), 0, kStatusTimeout);
+}
+__device__ __forceinline__ void raise_timeout(const Ctl &c) { raise_timeout_s(c.misc); }
+__device__ __forceinline__ bool aborted(const Ctl &c) { return ld_volatile_shared_u32(c.misc + 4) != 0; }
+
+// Bounded wait (the limit is read only once the first test fails).
+__device__ __forceinline__ bool bwait(const Ctl &c, int bar, uint32_t parity) {
+  const uint32_t b = bar_at(c, bar);
+  if (mbar_try_wait_s(b, parity)) return true;
+  return mbar_wait_s(b, parity, lds_u64(c.misc + 8), c.misc + 4);
+}
 
 __device__ __forceinline__ bool wait1(const Ctl &c, int bar, uint32_t parity) {
-  if (mbar_wait(&c.bar[bar], parity, c.timeout_ns, c.abort)) return true;
+  if (bwait(c, bar, parity)) return true;
   raise_timeout(c);
   return false;
 }
 
 // Whole-warp bounded wait with a warp-uniform outcome.
 __device__ __forceinline__ bool waitw(const Ctl &c, int bar, uint32_t parity) {
-  bool ok = mbar_wait(&c.bar[bar], parity, c.timeout_ns, c.abort);
+  bool ok = bwait(c, bar, parity);
   ok = __all_sync(0xffffffffu, ok);
   if (!ok && (threadIdx.x & 31) == 0) raise_timeout(c);
   __syncwarp();
@@ -336,7 +360,7 @@ __device__ __forceinline__ bool waitw(const Ctl &c, int bar, uint32_t parity) {
 
 __device__ __forceinline__ void arrive_lane0(const Ctl &c, int bar) {
   __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(&c.bar[bar]);
+  if ((threadIdx.x & 31) == 0) mbar_arrive_s(bar_at(c, bar));
 }
 
 // parity of the completion of a double-buffered barrier that block k uses
@@ -347,9 +371,12 @@ __device__ __forceinline__ uint32_t parr(int k) { return static_cast<uint32_t>(k
 
 // ---------------------------------------------------------------- work items
 // A work item is one (batch row b, head h, segment seg) sequence of nk blocks
-// starting at block k0.  CTA c walks items c, c + gridDim.x, ... and every
-// role runs the same sequence of steps j = 0, 1, ... (one block of one item
-// each); ring slots, double buffers and barrier phases follow j, so the
+// starting at block k0.  The CTAs claim items one at a time from a global
+// counter (SMs that run faster take more), in order, so that the items in
+// flight share their B, C tiles in L2.  The producer claims them, one item
+// ahead of its own progress, and publishes them in a ring in shared memory;
+// every role runs the same sequence of steps j = 0, 1, ... (one block of one
+// item each); ring slots, double buffers and barrier phases follow j, so the
 // pipeline runs on across item boundaries.
 struct Item {
   int b, h, g, seg, k0, nk;
@@ -370,8 +397,40 @@ __device__ __forceinline__ Item item_at(const TcParams &p, int it) {
 // 4-deep barrier ring of the per-block decay tables (phase of step j)
 __device__ __forceinline__ uint32_t par4(int j) { return (static_cast<uint32_t>(j) >> 2) & 1u; }
 
+__device__ __forceinline__ int lds_s32(uint32_t addr) {
+  int v;
+  asm volatile("ld.shared.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void sts_s32(uint32_t addr, int v) {
+  asm volatile("st.shared.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// Claim the next work item (-1: none left).
+__device__ __forceinline__ int claim_item(const TcParams &p) {
+  const int it = atomicAdd(p.item_counter, 1);
+  return it < p.items ? it : -1;
+}
+// Publish item `it` as this CTA's m-th (the barrier arrival releases the write).
+__device__ __forceinline__ void publish_item(const Ctl &c, uint32_t base, int m, int it) {
+  const int e = m & (kItemRing - 1);
+  sts_s32(base + kOffItemQ + 4 * e, it);
+  mbar_arrive_s(bar_at(c, bItem0 + e));
+}
+// This CTA's m-th item: >= 0, -1 (no more) or -2 (the wait timed out).
+__device__ __forceinline__ int item_one(const Ctl &c, uint32_t base, int m) {
+  const int e = m & (kItemRing - 1);
+  if (!wait1(c, bItem0 + e, static_cast<uint32_t>(m / kItemRing) & 1u)) return -2;
+  return lds_s32(base + kOffItemQ + 4 * e);
+}
+__device__ __forceinline__ int item_warp(const Ctl &c, uint32_t base, int m) {
+  const int e = m & (kItemRing - 1);
+  if (!waitw(c, bItem0 + e, static_cast<uint32_t>(m / kItemRing) & 1u)) return -2;
+  return lds_s32(base + kOffItemQ + 4 * e);
+}
+
 // ---------------------------------------------------------------- producer
-__device__ void producer(const TcParams &p, const Ctl &c, uint8_t *sm) {
+__device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
   const int nact = p.active[0] + p.active[1] + p.active[2] + p.active[3];
   const uint32_t bytes = p.agg ? 3 * kTile : nact * (kTile + 2048) + (2 + (p.allblock ? 4 : 2)) * kTile;
 #pragma unroll
@@ -384,8 +443,15 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint8_t *sm) {
   int last[kSlots] = {-1, -1, -1};
   int j = 0;
   bool ok = true;
-  for (int it = blockIdx.x; ok && it < p.items; it += gridDim.x) {
-    const Item I = item_at(p, it);
+  // items m and m + 1 are published when item m starts
+  int cur = claim_item(p), nxt = -1;
+  publish_item(c, base, 0, cur);
+  if (cur >= 0) {
+    nxt = claim_item(p);
+    publish_item(c, base, 1, nxt);
+  }
+  for (int m = 0; ok && cur >= 0; ++m) {
+    const Item I = item_at(p, cur);
     for (int kk = 0; kk < I.nk; ++kk, ++j) {
       const int k = I.k0 + kk;  // block index in the sequence
       const int r = rslot(j);
@@ -393,37 +459,42 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint8_t *sm) {
         ok = false;
         break;
       }
-      uint64_t *full = &c.bar[bFull0 + r];
-      mbar_arrive_expect_tx(full, bytes);
-      uint8_t *st = sm + r * kSlot;
+      const uint32_t full = bar_at(c, bFull0 + r);
+      mbar_arrive_expect_tx_s(full, bytes);
+      const uint32_t st = base + r * kSlot;
       const int t0 = k * kT;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         if (!p.active[i]) continue;
-        tma_load_4d(st + kOffX + i * kTile, &p.tx[i], full, 0, I.h, t0, I.b);
+        tma_load_4d_s(st + kOffX + i * kTile, &p.tx[i], full, 0, I.h, t0, I.b);
         if (p.agg) continue;
         const int idx = ((i * p.Bsz + I.b) * p.K + k) * p.G + I.g;
-        tma_load_3d(st + kOffCB + i * 2048, &p.tcb, full, 0, 0, idx);
+        tma_load_3d_s(st + kOffCB + i * 2048, &p.tcb, full, 0, 0, idx);
       }
-      tma_load_4d(st + kOffBcf, &p.tbcf, full, 0, I.g, t0, I.b);
-      tma_load_4d(st + kOffBcf + kTile, &p.tbcf, full, 64, I.g, t0, I.b);
+      tma_load_4d_s(st + kOffBcf, &p.tbcf, full, 0, I.g, t0, I.b);
+      tma_load_4d_s(st + kOffBcf + kTile, &p.tbcf, full, 64, I.g, t0, I.b);
       if (!p.agg) {
-        tma_load_4d(st + kOffClo, &p.tccf, full, 0, I.g, t0, I.b);
-        tma_load_4d(st + kOffChi, &p.tccf, full, 64, I.g, t0, I.b);
+        tma_load_4d_s(st + kOffClo, &p.tccf, full, 0, I.g, t0, I.b);
+        tma_load_4d_s(st + kOffChi, &p.tccf, full, 64, I.g, t0, I.b);
         if (p.allblock) {
-          tma_load_4d(st + kOffClo + kTile, &p.tcnf, full, 0, I.g, t0, I.b);
-          tma_load_4d(st + kOffChi + kTile, &p.tcnf, full, 64, I.g, t0, I.b);
+          tma_load_4d_s(st + kOffClo + kTile, &p.tcnf, full, 0, I.g, t0, I.b);
+          tma_load_4d_s(st + kOffChi + kTile, &p.tcnf, full, 64, I.g, t0, I.b);
         }
       }
 #pragma unroll
       for (int s = 0; s < kSlots; ++s)
         if (s == r) last[s] = j;
     }
+    cur = nxt;
+    if (ok && cur >= 0) {
+      nxt = claim_item(p);
+      publish_item(c, base, m + 2, nxt);
+    }
   }
   // no copy into this CTA's shared memory may still be in flight at exit
 #pragma unroll
   for (int s = 0; s < kSlots; ++s)
-    if (last[s] >= 0) (void)mbar_wait(&c.bar[bFull0 + s], parr(last[s]), p.drain_ns, nullptr);
+    if (last[s] >= 0) (void)mbar_wait_s(bar_at(c, bFull0 + s), parr(last[s]), p.drain_ns, 0);
 }
 
 // ---------------------------------------------------------------- MMA issuer
@@ -444,9 +515,11 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
   const uint64_t dM = sdesc(base + kOffMh, kMhLbo, kMhSbo, kLayoutNone);
   const uint64_t dDg = sdesc(base + kOffDg, kDgLbo, kDgSbo, kLayoutNone);
 #define BD_OFF(bytes) (static_cast<uint64_t>((bytes) >> 4))
-  int j = 0, m = 0;
+  int j = 0;
   bool ok = true;
-  for (int it = blockIdx.x; ok && it < p.items; it += gridDim.x, ++m) {
+  for (int m = 0; ok; ++m) {
+    const int it = item_one(c, base, m);
+    if (it < 0) break;
     const int nk = item_at(p, it).nk;
     const uint64_t go = BD_OFF(static_cast<uint32_t>(m & 1) * kDgBuf);  // this item's D I_16 operands
     for (int kk = 0; kk < nk; ++kk, ++j) {
@@ -455,18 +528,20 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
       const uint64_t so = BD_OFF(static_cast<uint32_t>(r) * kSlot);  // this step's ring slot
       if (!wait1(c, bFull0 + r, parr(j))) break;
       // ---- S^T = B_cf^T (w o X): A MN-major (n; halves 4 KB apart), B MN-major (p)
-      if (!wait1(c, bXwFull, j & 1)) break;
-      if (j >= 2 && !wait1(c, bSEmpty0 + i2, par2(j - 2))) break;
-      tc_fence_after();
-      const uint32_t colS = tmem + kColS0 + 64 * i2;
+      if (p.need_s) {
+        if (!wait1(c, bXwFull, j & 1)) break;
+        if (j >= 2 && !wait1(c, bSEmpty0 + i2, par2(j - 2))) break;
+        tc_fence_after();
+        const uint32_t colS = tmem + kColS0 + 64 * i2;
 #pragma unroll
-      for (int ks = 0; ks < 2; ++ks) {
-        umma_bf16(colS, dBcf + so + BD_OFF(ks * 2048), dXw + BD_OFF(ks * 2048), id_s, ks > 0);
-        umma_bf16(colS, dBcf + so + BD_OFF(ks * 2048), dXw + BD_OFF(kTile + ks * 2048), id_s, 1);
+        for (int ks = 0; ks < 2; ++ks) {
+          umma_bf16(colS, dBcf + so + BD_OFF(ks * 2048), dXw + BD_OFF(ks * 2048), id_s, ks > 0);
+          umma_bf16(colS, dBcf + so + BD_OFF(ks * 2048), dXw + BD_OFF(kTile + ks * 2048), id_s, 1);
+        }
+        umma_commit_s(bar_at(c, bSFull0 + i2));
       }
-      umma_commit(&c.bar[bSFull0 + i2]);
       if (p.agg) {  // aggregate pass: the forward state is all it needs
-        umma_commit(&c.bar[bEmpty0 + r]);
+        umma_commit_s(bar_at(c, bEmpty0 + r));
         ok = true;
         continue;
       }
@@ -481,7 +556,7 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
         umma_bf16(colY, dH + BD_OFF(ks * 2048), bc, id_yo, ks > 0);
         umma_bf16(colY, dH + BD_OFF(4 * kTile + ks * 2048), bc, id_yo, 1);
       }
-      umma_commit(&c.bar[bHCons]);  // the h operand may now be overwritten
+      umma_commit_s(bar_at(c, bHCons));  // the h operand may now be overwritten
       // ---- Y_diag^T of each stream = X_fwd^T M_fwd^T + X_rev^T M_rev^T, then
       //      X^T (D I) of every direction
       if (!wait1(c, bMhFull0 + i2, par2(j))) break;
@@ -508,14 +583,14 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
           umma_bf16(col + 16 * ks, a, dDg + go + BD_OFF((2 * i + 1) * 512), id_dx, 1);
         }
       }
-      umma_commit(&c.bar[bYFull0 + i2]);
-      umma_commit(&c.bar[bEmpty0 + r]);
+      umma_commit_s(bar_at(c, bYFull0 + i2));
+      umma_commit_s(bar_at(c, bEmpty0 + r));
       ok = true;
     }
   }
 #undef BD_OFF
-  umma_commit(&c.bar[bDrain]);
-  (void)mbar_wait(&c.bar[bDrain], 0, p.drain_ns, nullptr);
+  umma_commit_s(bar_at(c, bDrain));
+  (void)mbar_wait_s(bar_at(c, bDrain), 0, p.drain_ns, 0);
 }
 
 // ---------------------------------------------------------------- operand group
@@ -534,25 +609,30 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
     if (!act) return 0.f;
     return __bfloat162float(dtp[(static_cast<int64_t>(I.b) * L + (I.k0 + kk) * kT + lane) * H + I.h]);
   };
-  int j = 0, m = 0;
-  bool ok = true;
-  int it = blockIdx.x;
-  if (it >= p.items) return;
+  // A failed (timed-out) wait ends the group at once.
+  int j = 0;
+  int it = item_warp(c, base, 0);
+  if (it < 0) return;
   Item I = item_at(p, it);
   float dt_next = load_dt(I, 0);
-  for (; ok && it < p.items; ++m) {
+  for (int m = 0;; ++m) {
     const float A2 = act ? Ap[I.h] * kLog2e : 0.f;
-    const int it_next = it + gridDim.x;
-    const Item In = it_next < p.items ? item_at(p, it_next) : I;
+    int it_next = -1;
+    Item In = I;
     for (int kk = 0; kk < I.nk; ++kk, ++j) {
-      ok = false;
       const int i2 = j & 1, c4 = j & 3;
       const uint32_t st = base + rslot(j) * kSlot;
       const float dt_cur = dt_next;
-      if (kk + 1 < I.nk)
+      if (kk + 1 < I.nk) {
         dt_next = load_dt(I, kk + 1);
-      else if (it_next < p.items)
-        dt_next = load_dt(In, 0);
+      } else {  // the next item's first block
+        it_next = item_warp(c, base, m + 1);
+        if (it_next == -2) return;
+        if (it_next >= 0) {
+          In = item_at(p, it_next);
+          dt_next = load_dt(In, 0);
+        }
+      }
       // ---- decays of this warp's direction (log2 units): prefix sum (forward)
       //      or suffix sum (reverse) over the block
       float v = dt_cur * A2;
@@ -575,11 +655,11 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
         if (!rev) sts_f32(ecum + ((c4 * 2 + q) * 32 + lane) * 4, ex2_approx(v));
       }
       arrive_lane0(c, bAux0 + c4);
-      if (!waitw(c, bAux0 + c4, par4(j))) break;
+      if (!waitw(c, bAux0 + c4, par4(j))) return;
       // ---- (w o X) of the clean forward direction, bf16 hi + lo
-      if (j >= 1 && !waitw(c, bSFull0 + ((j + 1) & 1), par2(j - 1))) break;  // S(j-1) read Xw
-      if (!waitw(c, bFull0 + rslot(j), parr(j))) break;
-      {
+      if (p.need_s && j >= 1 && !waitw(c, bSFull0 + ((j + 1) & 1), par2(j - 1))) return;  // S(j-1) read Xw
+      if (!waitw(c, bFull0 + rslot(j), parr(j))) return;
+      if (p.need_s) {
         const uint32_t cf = cum + (c4 * 4 + kCF) * 128, df = dts + (c4 * 4 + kCF) * 128;
         const float c31 = lds_f32(cf + 31 * 4);
 #pragma unroll
@@ -602,7 +682,7 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
         // read this M buffer (and, at an item's first step, the D I_16 buffer
         // of two items back) are complete, and the epilogue has read its
         // decay tables
-        if (j >= 2 && !waitw(c, bYEmpty0 + i2, par2(j - 2))) break;
+        if (j >= 2 && !waitw(c, bYEmpty0 + i2, par2(j - 2))) return;
         if (kk == 0 && gt < 64) {
           // D I_16 operands of this item: bf16 hi + lo of each direction's D
           // on the diagonal (the rest of the buffer stays zero)
@@ -657,9 +737,8 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
       fence_proxy_async_smem();
       arrive_lane0(c, bMhFull0 + i2);
       arrive_lane0(c, bEmpty0 + rslot(j));
-      ok = true;
     }
-    it = it_next;
+    if (it_next < 0) return;
     I = In;
   }
 }
@@ -677,17 +756,23 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
   float hreg[kP];
   // h operand of Y_off^T (A, MN-major): {hi, lo} x [128 n rows][64 p] (SW128)
   auto write_h = [&]() {
-    const uint32_t hb = base + kOffH;
+    // (row address made opaque so that the eight chunk addresses are formed
+    // here rather than held in registers across the block loop)
+    uint32_t row = base + kOffH + 128u * static_cast<uint32_t>(n);
+    asm volatile("" : "+r"(row));
+    const uint32_t sw = (row >> 7) & 7u;
 #pragma unroll
     for (int cc = 0; cc < 8; ++cc) {
-      const uint32_t off = sw128_chunk(n, cc);
-      store_split8(hb + off, hb + 4 * kTile + off, hreg + 8 * cc);
+      const uint32_t a = row + ((static_cast<uint32_t>(cc) ^ sw) << 4);
+      store_split8(a, a + 4 * kTile, hreg + 8 * cc);
     }
     fence_proxy_async_smem();
     arrive_lane0(c, bHFull);
   };
   int j = 0;
-  for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
+  for (int m = 0;; ++m) {
+    const int it = item_warp(c, base, m);
+    if (it < 0) return;
     int nk;
     float *sdst;  // boundary states of this item's blocks, [B][K][H][P][N]
     {
@@ -709,6 +794,10 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
       // h operand; this item's initial state replaces it
       if (j >= 1 && !waitw(c, bHCons, (j - 1) & 1)) return;
       write_h();
+    }
+    if (!p.need_s) {  // one block, the state after it unused
+      j += nk;
+      continue;
     }
     float decay_log2 = 0.f;  // total decay over the item (aggregate pass)
     for (int kk = 0; kk < nk; ++kk, ++j) {
@@ -746,9 +835,10 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
         }
       }
     }
-    if (*c.abort) return;
-    // (item coordinates recomputed rather than kept live through the block loop)
-    const Item E = item_at(p, it);
+    if (aborted(c)) return;
+    // (item re-read from the ring -- its entry is not reused before every role
+    // has moved on -- rather than kept live through the block loop)
+    const Item E = item_at(p, lds_s32(base + kOffItemQ + 4 * (m & (kItemRing - 1))));
     const int64_t ebh = static_cast<int64_t>(E.b) * H + E.h;
     if (p.agg) {
       const int64_t ebhs = ebh * p.nseg + E.seg;
@@ -779,16 +869,17 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
   const uint32_t ecum = base + kOffEc;
   const int64_t H = p.H, L = p.L;
   if (p.agg) return;
+  // A failed (timed-out) wait ends the group at once.
   int j = 0;
-  bool ok = true;
-  for (int it = blockIdx.x; ok && it < p.items; it += gridDim.x) {
+  for (int m = 0;; ++m) {
+    const int it = item_warp(c, base, m);
+    if (it < 0) return;
     const Item I = item_at(p, it);
     for (int kk = 0; kk < I.nk; ++kk, ++j) {
-      ok = false;
       const int k = I.k0 + kk;  // block index in the sequence
       const int i2 = j & 1, c4 = j & 3;
-      if (!waitw(c, bAux0 + c4, par4(j))) break;
-      if (!waitw(c, bYFull0 + i2, par2(j))) break;
+      if (!waitw(c, bAux0 + c4, par4(j))) return;
+      if (!waitw(c, bYFull0 + i2, par2(j))) return;
       tc_fence_after();
       uint32_t yo[32], yd[32];
       const uint32_t ta = tmem_addr(tmem, 32 * q, kColY0 + 128 * i2);
@@ -821,7 +912,6 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
           for (int t = 0; t < 32; ++t) dst[t * tstride] = __uint_as_float(yo[t]);
         }
       }
-      ok = true;
     }
   }
 }
@@ -842,13 +932,15 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
     for (int i = 0; i < bCount; ++i) {
       uint32_t cnt = 4;
       if (i == bFull0 || i == bFull1 || i == bFull2 || i == bSFull0 || i == bSFull1 || i == bYFull0 ||
-          i == bYFull1 || i == bHCons || i == bDrain)
+          i == bYFull1 || i == bHCons || i == bDrain || i >= bItem0)
         cnt = 1;
       else if (i == bEmpty0 || i == bEmpty1 || i == bEmpty2)
         cnt = 5;
       mbar_init(&bars[i], cnt);
     }
     *abort_flag = 0;
+    *reinterpret_cast<unsigned long long *>(sm + kOffMisc + 8) = p.timeout_ns;
+    *reinterpret_cast<int **>(sm + kOffMisc + 16) = p.status;
     fence_mbar_init();
   }
   // Without a noisy stream, Y_off still reads the noisy half of the stacked C
@@ -874,10 +966,10 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  Ctl c{bars, abort_flag, p.status, p.timeout_ns};
+  Ctl c{smem_u32(bars), base + kOffMisc};
 
   if (warp == 0) {
-    if ((threadIdx.x & 31) == 0) producer(p, c, sm);
+    if ((threadIdx.x & 31) == 0) producer(p, c, base);
   } else if (warp == 1) {
     if ((threadIdx.x & 31) == 0) mma_issuer(p, c, base, tmem);
   } else if (warp < 6) {
@@ -915,6 +1007,8 @@ __global__ void __launch_bounds__(256) bd_seg_combine_kernel(const float *h0, co
 }
 
 // ------------------------------------------------------------------ host side
+constexpr size_t kCounterOffset = 256;  // bytes into the workspace header
+static_assert(kCounterOffset + 2 * sizeof(int) <= kWsHeader, "workspace header");
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -1048,6 +1142,10 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
   cp.K = K;
   cp.G = static_cast<int>(a.G);
   cp.cb = cbws;
+  // work-item counters of the aggregate [0] and main [1] scan passes, in the
+  // workspace header next to the status word
+  int *counters = reinterpret_cast<int *>(static_cast<uint8_t *>(a.ws) + kCounterOffset);
+  cp.item_counters = counters;
   cp.status = a.status;
   cp.timeout_ns = timeout;
   cudaError_t e = cudaFuncSetAttribute(bd_cb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1082,7 +1180,9 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
   p.nseg = nseg;
   p.seg_blocks = (K + nseg - 1) / nseg;
   p.items = static_cast<int>(a.Bsz * a.H * nseg);
+  p.item_counter = counters + 1;
   p.allblock = all ? 1 : 0;
+  p.need_s = (a.states || a.final_state || p.seg_blocks > 1 || nseg > 1) ? 1 : 0;
   p.out_bf16 = a.out_bf16 ? 1 : 0;
   p.h0 = a.h0;
   p.states = a.states;
@@ -1112,12 +1212,14 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
     float *seg_decay = reinterpret_cast<float *>(wsb + cb_bytes + 2 * st_bytes);
     TcParams q = p;
     q.agg = 1;
+    q.need_s = 1;
     q.allblock = 0;
     for (int i = 1; i < 4; ++i) q.active[i] = 0;
     q.states = nullptr;
     q.final_state = nullptr;
     q.y_clean = q.y_noisy = nullptr;
     q.seg_local = seg_local;
+    q.item_counter = counters;
     q.seg_decay = seg_decay;
     bd_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(q);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
