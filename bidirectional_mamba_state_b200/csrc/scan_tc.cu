@@ -113,6 +113,9 @@ __global__ void __launch_bounds__(kCbThreads) bd_cb_kernel(const __grid_constant
   const int k0 = 4 * blockIdx.x;
   const int nvalid = min(4, p.K - k0);
   if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x < 2) p.item_counters[threadIdx.x] = 0;
+  // the scan kernel that follows may start its prologue on free SMs now (it
+  // waits for this grid's completion before reading anything written here)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (threadIdx.x == 0) {
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
@@ -205,8 +208,8 @@ constexpr uint32_t kOffBar = kOffEc + 1024;
 constexpr int kNumBars = 48;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // TMEM base, abort flag
 constexpr int kItemRing = 16;
-constexpr uint32_t kOffItemQ = kOffMisc + 64;             // int[kItemRing]: published work items
-constexpr uint32_t kSmemBytes = kOffItemQ + 4 * kItemRing + 1024;
+constexpr uint32_t kOffItemQ = kOffMisc + 64;             // int4[kItemRing]: published work items
+constexpr uint32_t kSmemBytes = kOffItemQ + 16 * kItemRing + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 // D I_16 operand (B of the D x MMAs): [16 t][16 s] interleaved K-major, 8x8 core
@@ -336,11 +339,16 @@ __device__ __noinline__ void raise_timeout_s(uint32_t misc) {
 __device__ __forceinline__ void raise_timeout(const Ctl &c) { raise_timeout_s(c.misc); }
 __device__ __forceinline__ bool aborted(const Ctl &c) { return ld_volatile_shared_u32(c.misc + 4) != 0; }
 
-// Bounded wait (the limit is read only once the first test fails).
+// Bounded wait.  The first test is inline; the sleeping retry loop with its
+// time limit and abort check is out of line, so that the many wait sites do
+// not each carry it through the instruction cache.
+__device__ __noinline__ bool bwait_slow(uint32_t b, uint32_t parity, uint32_t misc) {
+  return mbar_wait_s(b, parity, lds_u64(misc + 8), misc + 4);
+}
 __device__ __forceinline__ bool bwait(const Ctl &c, int bar, uint32_t parity) {
   const uint32_t b = bar_at(c, bar);
   if (mbar_try_wait_s(b, parity)) return true;
-  return mbar_wait_s(b, parity, lds_u64(c.misc + 8), c.misc + 4);
+  return bwait_slow(b, parity, c.misc);
 }
 
 __device__ __forceinline__ bool wait1(const Ctl &c, int bar, uint32_t parity) {
@@ -382,6 +390,17 @@ struct Item {
   int b, h, g, seg, k0, nk;
 };
 
+__device__ __forceinline__ Item item_unpack(const TcParams &p, int b, int h, int g, int seg) {
+  Item r;
+  r.b = b;
+  r.h = h;
+  r.g = g;
+  r.seg = seg;
+  r.k0 = seg * p.seg_blocks;
+  r.nk = min(p.K - r.k0, p.seg_blocks);
+  return r;
+}
+
 __device__ __forceinline__ Item item_at(const TcParams &p, int it) {
   Item r;
   r.seg = it % p.nseg;
@@ -397,11 +416,6 @@ __device__ __forceinline__ Item item_at(const TcParams &p, int it) {
 // 4-deep barrier ring of the per-block decay tables (phase of step j)
 __device__ __forceinline__ uint32_t par4(int j) { return (static_cast<uint32_t>(j) >> 2) & 1u; }
 
-__device__ __forceinline__ int lds_s32(uint32_t addr) {
-  int v;
-  asm volatile("ld.shared.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return v;
-}
 __device__ __forceinline__ void sts_s32(uint32_t addr, int v) {
   asm volatile("st.shared.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
@@ -411,22 +425,37 @@ __device__ __forceinline__ int claim_item(const TcParams &p) {
   const int it = atomicAdd(p.item_counter, 1);
   return it < p.items ? it : -1;
 }
-// Publish item `it` as this CTA's m-th (the barrier arrival releases the write).
-__device__ __forceinline__ void publish_item(const Ctl &c, uint32_t base, int m, int it) {
+// Publish item `it` (-1: none) as this CTA's m-th, as its coordinates
+// {b, h, g, seg} (the barrier arrival releases the write).
+__device__ __forceinline__ void publish_item(const TcParams &p, const Ctl &c, uint32_t base, int m, int it) {
   const int e = m & (kItemRing - 1);
-  sts_s32(base + kOffItemQ + 4 * e, it);
+  const uint32_t a = base + kOffItemQ + 16 * e;
+  if (it >= 0) {
+    const Item I = item_at(p, it);
+    asm volatile("st.shared.v4.s32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(I.b), "r"(I.h), "r"(I.g), "r"(I.seg)
+                 : "memory");
+  } else {
+    sts_s32(a, -1);
+  }
   mbar_arrive_s(bar_at(c, bItem0 + e));
 }
-// This CTA's m-th item: >= 0, -1 (no more) or -2 (the wait timed out).
-__device__ __forceinline__ int item_one(const Ctl &c, uint32_t base, int m) {
-  const int e = m & (kItemRing - 1);
-  if (!wait1(c, bItem0 + e, static_cast<uint32_t>(m / kItemRing) & 1u)) return -2;
-  return lds_s32(base + kOffItemQ + 4 * e);
+// Ring entry m (already published) as an item; false: none.
+__device__ __forceinline__ bool item_read(const TcParams &p, uint32_t base, int m, Item &I) {
+  const uint32_t a = base + kOffItemQ + 16 * (m & (kItemRing - 1));
+  int b, h, g, seg;
+  asm volatile("ld.shared.v4.s32 {%0, %1, %2, %3}, [%4];" : "=r"(b), "=r"(h), "=r"(g), "=r"(seg) : "r"(a) : "memory");
+  if (b < 0) return false;
+  I = item_unpack(p, b, h, g, seg);
+  return true;
 }
-__device__ __forceinline__ int item_warp(const Ctl &c, uint32_t base, int m) {
-  const int e = m & (kItemRing - 1);
-  if (!waitw(c, bItem0 + e, static_cast<uint32_t>(m / kItemRing) & 1u)) return -2;
-  return lds_s32(base + kOffItemQ + 4 * e);
+// This CTA's m-th item: 1 (in I), 0 (no more) or -1 (the wait timed out).
+__device__ __forceinline__ int item_one(const TcParams &p, const Ctl &c, uint32_t base, int m, Item &I) {
+  if (!wait1(c, bItem0 + (m & (kItemRing - 1)), static_cast<uint32_t>(m / kItemRing) & 1u)) return -1;
+  return item_read(p, base, m, I) ? 1 : 0;
+}
+__device__ __forceinline__ int item_warp(const TcParams &p, const Ctl &c, uint32_t base, int m, Item &I) {
+  if (!waitw(c, bItem0 + (m & (kItemRing - 1)), static_cast<uint32_t>(m / kItemRing) & 1u)) return -1;
+  return item_read(p, base, m, I) ? 1 : 0;
 }
 
 // ---------------------------------------------------------------- producer
@@ -443,12 +472,14 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
   int last[kSlots] = {-1, -1, -1};
   int j = 0;
   bool ok = true;
-  // items m and m + 1 are published when item m starts
+  // items m and m + 1 are published when item m starts (nothing after a -1);
+  // claiming further ahead would hold items back from CTAs that run dry at
+  // the end of the pass
   int cur = claim_item(p), nxt = -1;
-  publish_item(c, base, 0, cur);
+  publish_item(p, c, base, 0, cur);
   if (cur >= 0) {
     nxt = claim_item(p);
-    publish_item(c, base, 1, nxt);
+    publish_item(p, c, base, 1, nxt);
   }
   for (int m = 0; ok && cur >= 0; ++m) {
     const Item I = item_at(p, cur);
@@ -486,9 +517,10 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
         if (s == r) last[s] = j;
     }
     cur = nxt;
+    nxt = -1;
     if (ok && cur >= 0) {
       nxt = claim_item(p);
-      publish_item(c, base, m + 2, nxt);
+      publish_item(p, c, base, m + 2, nxt);
     }
   }
   // no copy into this CTA's shared memory may still be in flight at exit
@@ -518,9 +550,9 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
   int j = 0;
   bool ok = true;
   for (int m = 0; ok; ++m) {
-    const int it = item_one(c, base, m);
-    if (it < 0) break;
-    const int nk = item_at(p, it).nk;
+    Item I;
+    if (item_one(p, c, base, m, I) <= 0) break;
+    const int nk = I.nk;
     const uint64_t go = BD_OFF(static_cast<uint32_t>(m & 1) * kDgBuf);  // this item's D I_16 operands
     for (int kk = 0; kk < nk; ++kk, ++j) {
       ok = false;
@@ -550,7 +582,7 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
       if (j >= 2 && !wait1(c, bYEmpty0 + i2, par2(j - 2))) break;
       tc_fence_after();
       const uint32_t colY = tmem + kColY0 + 128 * i2;
-#pragma unroll
+#pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
         const uint64_t bc = dC + so + BD_OFF((ks < 4 ? 0 : 2 * kTile) + (ks & 3) * 32);
         umma_bf16(colY, dH + BD_OFF(ks * 2048), bc, id_yo, ks > 0);
@@ -605,33 +637,62 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
   const int64_t H = p.H, L = p.L;
   const float *Ap = pick4(p.A, q);
   const __nv_bfloat16 *dtp = pick4(p.dt, q);
-  auto load_dt = [&](const Item &I, int kk) -> float {  // dt of block kk of item I
-    if (!act) return 0.f;
-    return __bfloat162float(dtp[(static_cast<int64_t>(I.b) * L + (I.k0 + kk) * kT + lane) * H + I.h]);
-  };
+  // D of direction gt >> 4 (threads that build the D I_16 operands)
+  const float *Dp = gt < 64 ? pick4(p.D, gt >> 4) : nullptr;
+  const bool dact = gt < 64 && pick4(p.active, gt >> 4) != 0;
   // A failed (timed-out) wait ends the group at once.
+  Item I;
+  if (item_warp(p, c, base, 0, I) <= 0) return;
+  // Global loads two steps ahead (their latency is microseconds under the
+  // kernel's own traffic): a cursor walks the steps, through the items the
+  // producer publishes, and fills a two-deep register queue with dt of this
+  // lane's token, A (log2 units) and D of the step's head.
+  int cm = 0, ckk = 0;
+  bool cv = true;  // the cursor is on an item
+  Item CI = I;
+  float qdt[2], qa[2], qd[2];
+  auto cursor_load = [&](int e) {
+    qdt[e] = 0.f;
+    qa[e] = 0.f;
+    qd[e] = 0.f;
+    if (!cv) return;
+    if (act) {
+      qdt[e] = __bfloat162float(dtp[(static_cast<int64_t>(CI.b) * L + (CI.k0 + ckk) * kT + lane) * H + CI.h]);
+      qa[e] = Ap[CI.h] * kLog2e;
+    }
+    if (dact) qd[e] = Dp[CI.h];
+  };
+  auto cursor_next = [&]() -> bool {  // false: a wait timed out
+    if (!cv) return true;
+    if (++ckk < CI.nk) return true;
+    ++cm;
+    ckk = 0;
+    const int r = item_warp(p, c, base, cm, CI);
+    if (r < 0) return false;
+    cv = r > 0;
+    return true;
+  };
+  cursor_load(0);
+  if (!cursor_next()) return;
+  cursor_load(1);
+  if (!cursor_next()) return;
   int j = 0;
-  int it = item_warp(c, base, 0);
-  if (it < 0) return;
-  Item I = item_at(p, it);
-  float dt_next = load_dt(I, 0);
   for (int m = 0;; ++m) {
-    const float A2 = act ? Ap[I.h] * kLog2e : 0.f;
-    int it_next = -1;
+    bool has_next = false;
     Item In = I;
     for (int kk = 0; kk < I.nk; ++kk, ++j) {
       const int i2 = j & 1, c4 = j & 3;
       const uint32_t st = base + rslot(j) * kSlot;
-      const float dt_cur = dt_next;
-      if (kk + 1 < I.nk) {
-        dt_next = load_dt(I, kk + 1);
-      } else {  // the next item's first block
-        it_next = item_warp(c, base, m + 1);
-        if (it_next == -2) return;
-        if (it_next >= 0) {
-          In = item_at(p, it_next);
-          dt_next = load_dt(In, 0);
-        }
+      const float dt_cur = qdt[0], A2 = qa[0], Dv = qd[0];
+      qdt[0] = qdt[1];
+      qa[0] = qa[1];
+      qd[0] = qd[1];
+      cursor_load(1);
+      if (!cursor_next()) return;
+      if (kk + 1 == I.nk) {  // the next item
+        const int r = item_warp(p, c, base, m + 1, In);
+        if (r < 0) return;
+        has_next = r > 0;
       }
       // ---- decays of this warp's direction (log2 units): prefix sum (forward)
       //      or suffix sum (reverse) over the block
@@ -687,8 +748,7 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
           // D I_16 operands of this item: bf16 hi + lo of each direction's D
           // on the diagonal (the rest of the buffer stays zero)
           const int i = gt >> 4, d = gt & 15;
-          if (pick4(p.active, i)) {
-            const float Dv = pick4(p.D, i)[I.h];
+          if (dact) {
             const __nv_bfloat16 dh = __float2bfloat16_rn(Dv);
             const __nv_bfloat16 dl = __float2bfloat16_rn(Dv - __bfloat162float(dh));
             const uint32_t off = (m & 1) * kDgBuf + (d >> 3) * kDgSbo + (d >> 3) * kDgLbo + (d & 7) * 16 + (d & 7) * 2;
@@ -699,25 +759,14 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
         // ---- masked-decay matrix, row s = lane of M^T for this direction
         if (act) {
           const uint32_t cbrow = st + kOffCB + q * 2048;
-          float cbv[32];
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            uint32_t r0, r1, r2, r3;
-            ld_shared_v4(cbrow + sw64_chunk(lane, ch), r0, r1, r2, r3);
-            cbv[8 * ch] = bf16_lo_f(r0);
-            cbv[8 * ch + 1] = bf16_hi_f(r0);
-            cbv[8 * ch + 2] = bf16_lo_f(r1);
-            cbv[8 * ch + 3] = bf16_hi_f(r1);
-            cbv[8 * ch + 4] = bf16_lo_f(r2);
-            cbv[8 * ch + 5] = bf16_hi_f(r2);
-            cbv[8 * ch + 6] = bf16_lo_f(r3);
-            cbv[8 * ch + 7] = bf16_hi_f(r3);
-          }
           const uint32_t cq = cum + (c4 * 4 + q) * 128;
           const float cs = v, ds = dt_cur;
           const uint32_t mrow = base + kOffMh + i2 * kMhBuf + q * 2048;
-#pragma unroll
+          // (not unrolled: a compact loop keeps the instruction cache footprint down)
+#pragma unroll 1
           for (int jj = 0; jj < 4; ++jj) {
+            uint32_t r[4];
+            ld_shared_v4(cbrow + sw64_chunk(lane, jj), r[0], r[1], r[2], r[3]);  // C B^T[s = lane][8 jj ..]
             float cj[8];
             ld_shared_v4f(cq + 32 * jj, *reinterpret_cast<float(*)[4]>(&cj[0]));
             ld_shared_v4f(cq + 32 * jj + 16, *reinterpret_cast<float(*)[4]>(&cj[4]));
@@ -727,7 +776,8 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
               const int t = 8 * jj + i;
               const bool valid = rev ? (t <= lane) : (t >= lane);
               const float e = ex2_approx(cj[i] - cs);
-              mv[i] = valid ? cbv[t] * ds * e : 0.f;
+              const float cb = (i & 1) ? bf16_hi_f(r[i >> 1]) : bf16_lo_f(r[i >> 1]);
+              mv[i] = valid ? cb * ds * e : 0.f;
             }
             st_shared_v4(mrow + inter_mn_off(8 * jj, lane, kMhSbo, kMhLbo), pack_bf16x2(mv[0], mv[1]),
                          pack_bf16x2(mv[2], mv[3]), pack_bf16x2(mv[4], mv[5]), pack_bf16x2(mv[6], mv[7]));
@@ -738,12 +788,78 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
       arrive_lane0(c, bMhFull0 + i2);
       arrive_lane0(c, bEmpty0 + rslot(j));
     }
-    if (it_next < 0) return;
+    if (!has_next) return;
     I = In;
   }
 }
 
 // ---------------------------------------------------------------- state group
+// One-block items whose state after the block is not used (no S chain): the
+// group only turns each item's initial state into the h operand of Y_off.
+// The fp32 state of item m + 1 is loaded while item m is converted, staged in
+// TMEM (the unused S accumulator columns, two buffers of 64 columns: lane n,
+// column p), so that the load latency overlaps the pipeline instead of
+// adding to every item.
+__device__ void state_group_staged(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
+  const int lane = threadIdx.x & 31;
+  const int q = (threadIdx.x >> 5) & 3;
+  const int n = 32 * q + lane;
+  const int64_t H = p.H;
+  const int64_t PN = kP * kN;
+  float hreg[kP];
+  auto load_h = [&](const Item &I) {
+    const float *src = p.h0 ? p.h0 + (static_cast<int64_t>(I.b) * H + I.h) * PN + n : nullptr;
+#pragma unroll
+    for (int pp = 0; pp < kP; ++pp) hreg[pp] = src ? src[pp * kN] : 0.f;
+  };
+  auto stage = [&](int e) {  // hreg -> TMEM buffer e
+    const uint32_t ta = tmem_addr(tmem, 32 * q, kColS0 + 64 * e);
+#pragma unroll
+    for (int cq = 0; cq < 4; ++cq) {
+      uint32_t r[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(hreg[16 * cq + i]);
+      tmem_st_32x32b_x16(ta + 16 * cq, r);
+    }
+    tmem_st_wait();
+  };
+  Item I;
+  if (item_warp(p, c, base, 0, I) <= 0) return;
+  load_h(I);
+  stage(0);
+  for (int m = 0;; ++m) {
+    const int rn = item_warp(p, c, base, m + 1, I);
+    if (rn < 0) return;
+    if (rn > 0) load_h(I);  // in flight while item m is converted
+    // Y_off of the previous item has read the h operand
+    if (m >= 1 && !waitw(c, bHCons, (m - 1) & 1)) return;
+    {
+      uint32_t row = base + kOffH + 128u * static_cast<uint32_t>(n);
+      asm volatile("" : "+r"(row));
+      const uint32_t sw = (row >> 7) & 7u;
+      const uint32_t ta = tmem_addr(tmem, 32 * q, kColS0 + 64 * (m & 1));
+#pragma unroll
+      for (int cq = 0; cq < 4; ++cq) {
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(ta + 16 * cq, r);
+        tmem_ld_wait();
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const uint32_t a = row + ((static_cast<uint32_t>(2 * cq + h2) ^ sw) << 4);
+          store_split8(a, a + 4 * kTile, v + 8 * h2);
+        }
+      }
+    }
+    fence_proxy_async_smem();
+    arrive_lane0(c, bHFull);
+    if (rn == 0) return;
+    stage((m + 1) & 1);
+  }
+}
+
 // warps 6..9: thread owns column n = 32 q + lane of the state, h^T[n][0..63].
 // A failed (timed-out) wait ends the group at once: nothing else is stored.
 __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
@@ -751,6 +867,10 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
   const int q = (threadIdx.x >> 5) & 3;
   const int n = 32 * q + lane;
   const uint32_t cum = base + kOffCum;
+  if (!p.need_s) {
+    state_group_staged(p, c, base, tmem);
+    return;
+  }
   const int64_t H = p.H;
   const int64_t PN = kP * kN;
   float hreg[kP];
@@ -769,14 +889,18 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
     fence_proxy_async_smem();
     arrive_lane0(c, bHFull);
   };
+  // Each item: load its initial state, then per block kk: write the h
+  // operand of the state entering the block, store the state after block
+  // kk - 1, and advance the state with S of block kk; a last pass (kk == nk)
+  // stores the state after the item's last block (boundary, final or segment
+  // state).  Each store sequence and the operand write appear once in code.
   int j = 0;
   for (int m = 0;; ++m) {
-    const int it = item_warp(c, base, m);
-    if (it < 0) return;
     int nk;
     float *sdst;  // boundary states of this item's blocks, [B][K][H][P][N]
     {
-      const Item I = item_at(p, it);
+      Item I;
+      if (item_warp(p, c, base, m, I) <= 0) return;
       nk = I.nk;
       const int64_t bh = static_cast<int64_t>(I.b) * H + I.h;
       sdst = p.states ? p.states + ((static_cast<int64_t>(I.b) * p.K + I.k0) * H + I.h) * PN + n : nullptr;
@@ -789,18 +913,41 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
 #pragma unroll
       for (int pp = 0; pp < kP; ++pp) hreg[pp] = src ? src[pp * kN] : 0.f;
     }
-    if (!p.agg) {
-      // Y_off of the previous step (another item's last block) has read the
-      // h operand; this item's initial state replaces it
-      if (j >= 1 && !waitw(c, bHCons, (j - 1) & 1)) return;
-      write_h();
-    }
-    if (!p.need_s) {  // one block, the state after it unused
-      j += nk;
-      continue;
-    }
     float decay_log2 = 0.f;  // total decay over the item (aggregate pass)
-    for (int kk = 0; kk < nk; ++kk, ++j) {
+    for (int kk = 0;; ++kk) {
+      if (kk < nk && !p.agg) {
+        // Y_off of the previous step has read the h operand; the state
+        // entering this block replaces it
+        if (j >= 1 && !waitw(c, bHCons, (j - 1) & 1)) return;
+        write_h();
+      }
+      if (kk >= 1) {
+#pragma unroll 1
+        for (int d = 0; d < 2; ++d) {
+          float *dst = sdst;
+          if (d == 1) {  // after the item's last block: final or segment state
+            dst = nullptr;
+            if (kk == nk && !aborted(c)) {
+              Item E;  // (re-read from the ring: its entry is not reused before every role moved on)
+              (void)item_read(p, base, m, E);
+              const int64_t ebh = static_cast<int64_t>(E.b) * H + E.h;
+              if (p.agg) {
+                const int64_t ebhs = ebh * p.nseg + E.seg;
+                dst = p.seg_local + ebhs * PN + n;
+                if (n == 0) p.seg_decay[ebhs] = decay_log2;
+              } else if (p.final_state && E.k0 + E.nk == p.K) {
+                dst = p.final_state + ebh * PN + n;
+              }
+            }
+          }
+          if (dst) {  // each warp instruction stores one contiguous 128-byte row segment
+#pragma unroll
+            for (int pp = 0; pp < kP; ++pp) dst[pp * kN] = hreg[pp];
+          }
+        }
+        if (sdst) sdst += static_cast<int64_t>(p.H) * PN;
+      }
+      if (kk == nk) break;
       const int i2 = j & 1, c4 = j & 3;
       if (!waitw(c, bAux0 + c4, par4(j))) return;
       const float c31 = lds_f32(cum + ((c4 * 4 + kCF) * 32 + 31) * 4);
@@ -821,35 +968,7 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
       }
       tc_fence_before();
       arrive_lane0(c, bSEmpty0 + i2);
-      if (!p.agg) {
-        if (kk + 1 < nk) {
-          // Y_off of this step reads the state before the block from the
-          // operand buffer; the state after it replaces it for the next step
-          if (!waitw(c, bHCons, j & 1)) return;
-          write_h();
-        }
-        if (sdst) {  // each warp instruction stores one contiguous 128-byte row segment
-#pragma unroll
-          for (int pp = 0; pp < kP; ++pp) sdst[pp * kN] = hreg[pp];
-          sdst += H * PN;
-        }
-      }
-    }
-    if (aborted(c)) return;
-    // (item re-read from the ring -- its entry is not reused before every role
-    // has moved on -- rather than kept live through the block loop)
-    const Item E = item_at(p, lds_s32(base + kOffItemQ + 4 * (m & (kItemRing - 1))));
-    const int64_t ebh = static_cast<int64_t>(E.b) * H + E.h;
-    if (p.agg) {
-      const int64_t ebhs = ebh * p.nseg + E.seg;
-      float *dst = p.seg_local + ebhs * PN + n;
-#pragma unroll
-      for (int pp = 0; pp < kP; ++pp) dst[pp * kN] = hreg[pp];
-      if (n == 0) p.seg_decay[ebhs] = decay_log2;
-    } else if (p.final_state && E.k0 + E.nk == p.K) {
-      float *dst = p.final_state + ebh * PN + n;
-#pragma unroll
-      for (int pp = 0; pp < kP; ++pp) dst[pp * kN] = hreg[pp];
+      ++j;
     }
   }
 }
@@ -872,9 +991,8 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
   // A failed (timed-out) wait ends the group at once.
   int j = 0;
   for (int m = 0;; ++m) {
-    const int it = item_warp(c, base, m);
-    if (it < 0) return;
-    const Item I = item_at(p, it);
+    Item I;
+    if (item_warp(p, c, base, m, I) <= 0) return;
     for (int kk = 0; kk < I.nk; ++kk, ++j) {
       const int k = I.k0 + kk;  // block index in the sequence
       const int i2 = j & 1, c4 = j & 3;
@@ -967,6 +1085,10 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   Ctl c{smem_u32(bars), base + kOffMisc};
+  // Launched as a programmatic dependent of the previous kernel on the stream:
+  // the prologue above overlaps its tail; nothing it wrote (C B^T tiles, work
+  // counters, segment states) is read before it has completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == 0) {
     if ((threadIdx.x & 31) == 0) producer(p, c, base);
@@ -1046,6 +1168,24 @@ bool make_map_cb(CUtensorMap *m, const void *ptr, uint64_t ntiles) {
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The scan kernel as a programmatic dependent launch (its prologue may overlap
+// the previous kernel in the stream; it waits for that kernel before reading).
+cudaError_t launch_scan(unsigned grid, cudaStream_t stream, const TcParams &p) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, bd_tc_kernel, p);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 bool device_is_sm100() {
@@ -1221,15 +1361,13 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
     q.seg_local = seg_local;
     q.item_counter = counters;
     q.seg_decay = seg_decay;
-    bd_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(q);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_scan(grid, stream, q)) != cudaSuccess) return e;
     bd_seg_combine_kernel<<<dim3(static_cast<unsigned>(a.Bsz * a.H), (kP * kN) / 256), 256, 0, stream>>>(
         a.h0, seg_local, seg_decay, seg_init, nseg);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     p.seg_init = seg_init;
   }
-  bd_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(p);
-  return cudaGetLastError();
+  return launch_scan(grid, stream, p);
 }
 
 }  // namespace bdscan
