@@ -40,7 +40,9 @@
 //     warps 10-13 epilogue: thread (p, stream) forms y[t][p] = exp(cum_t) Y_off
 //                 + Y_diag for the block's 32 tokens and stores them; the D x
 //                 terms are small tensor-core products against D I_16 (bf16
-//                 hi + lo) accumulated into Y_diag
+//                 hi + lo) accumulated into Y_diag.  Two blocks ahead, the
+//                 same warps build the masked-decay matrices M and the D I_16
+//                 operands.
 //   S, Y, M and D I_16 are double-buffered; the h operand is single-buffered.
 // Every wait is bounded; on a timeout the CTA raises BDSCAN_ERR_TIMEOUT in the
 // workspace status word, drains its own copies and MMAs, frees TMEM and exits.
@@ -201,10 +203,15 @@ constexpr uint32_t kOffMh = kOffH + 8 * kTile;  // 2 buffers x 4 dirs x [32 t][3
 constexpr uint32_t kMhBuf = 4 * 2048;
 constexpr uint32_t kOffDg = kOffMh + 2 * kMhBuf;  // 2 items x 4 dirs x {hi, lo} x D I_16 (bf16, 512 B each)
 constexpr uint32_t kDgBuf = 4096;
-constexpr uint32_t kOffCum = kOffDg + 2 * kDgBuf;  // [4 blocks][4 dirs][32] f32: cumulative decay (log2)
-constexpr uint32_t kOffDt = kOffCum + 2048;       // [4][4][32] f32: dt
-constexpr uint32_t kOffEc = kOffDt + 2048;        // [4][2 fwd dirs][32] f32: exp(cum_t)
-constexpr uint32_t kOffBar = kOffEc + 1024;
+// per-step tables, a ring of kTab steps (slot j mod kTab)
+constexpr int kTab = 8;
+constexpr uint32_t kOffCum = kOffDg + 2 * kDgBuf;    // [kTab][4 dirs][32] f32: cumulative decay (log2)
+constexpr uint32_t kOffDt = kOffCum + kTab * 512;    // [kTab][4][32] f32: dt
+constexpr uint32_t kOffEc = kOffDt + kTab * 512;     // [kTab][2 fwd dirs][32] f32: exp(cum_t)
+constexpr uint32_t kOffDtab = kOffEc + kTab * 256;   // [kTab][4] f32: D of the step's head
+constexpr uint32_t kOffFtab = kOffDtab + kTab * 16;  // [kTab] s32: 1 + item parity at an item's first step,
+                                                     // 0 at its other steps, -1 past the CTA's last step
+constexpr uint32_t kOffBar = kOffFtab + 128;
 constexpr int kNumBars = 48;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // TMEM base, abort flag
 constexpr int kItemRing = 16;
@@ -221,10 +228,11 @@ constexpr uint32_t kDgSbo = 128, kDgLbo = 256;
 constexpr uint32_t kMhSbo = 128, kMhLbo = 512;
 
 enum : int {
-  bFull0 = 0, bFull1, bFull2, bEmpty0, bEmpty1, bEmpty2, bAux0, bAux1, bAux2, bAux3, bXwFull, bSFull0, bSFull1,
+  bFull0 = 0, bFull1, bFull2, bEmpty0, bEmpty1, bEmpty2, bAux0, bAux7 = bAux0 + kTab - 1, bXwFull, bSFull0, bSFull1,
   bSEmpty0, bSEmpty1, bMhFull0, bMhFull1, bHFull, bHCons, bYFull0, bYFull1, bYEmpty0, bYEmpty1, bDrain,
   bItem0, bCount = bItem0 + kItemRing
 };
+static_assert(bCount <= kNumBars, "barrier array");
 
 // TMEM columns: S^T[2] (M=128 x 64), Y^T[2] = {Y_off^T (M=64 x 64), Y_diag^T (M=64 x 64)}
 constexpr uint32_t kColS0 = 0, kColY0 = 128;
@@ -413,9 +421,14 @@ __device__ __forceinline__ Item item_at(const TcParams &p, int it) {
   return r;
 }
 
-// 4-deep barrier ring of the per-block decay tables (phase of step j)
-__device__ __forceinline__ uint32_t par4(int j) { return (static_cast<uint32_t>(j) >> 2) & 1u; }
+// barrier ring of the per-step tables: phase parity of step j
+__device__ __forceinline__ uint32_t part(int j) { return (static_cast<uint32_t>(j) / kTab) & 1u; }
 
+__device__ __forceinline__ int lds_s32(uint32_t addr) {
+  int v;
+  asm volatile("ld.shared.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
 __device__ __forceinline__ void sts_s32(uint32_t addr, int v) {
   asm volatile("st.shared.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
@@ -626,20 +639,23 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
 }
 
 // ---------------------------------------------------------------- operand group
-// warps 2..5; q = warp & 3 is the direction slot whose decays and M it builds.
+// warps 2..5; q = warp & 3 is the direction slot whose decays it computes.
+// Per step: the per-step tables (cumulative decays, dt, exp(cum) of the
+// forward directions, D of the step's head, item-start flag) and w o X.
+// The masked-decay matrices are built by the epilogue warps.
 __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
   const int lane = threadIdx.x & 31;
   const int q = (threadIdx.x >> 5) & 3;
   const int gt = threadIdx.x - 64;  // 0..127
   const bool act = pick4(p.active, q) != 0;
-  const bool rev = q >= 2;
   const uint32_t cum = base + kOffCum, dts = base + kOffDt, ecum = base + kOffEc;
   const int64_t H = p.H, L = p.L;
+  const bool rev = q >= 2;
   const float *Ap = pick4(p.A, q);
   const __nv_bfloat16 *dtp = pick4(p.dt, q);
-  // D of direction gt >> 4 (threads that build the D I_16 operands)
+  // D of direction gt >> 4 (one writer per direction into the D table)
   const float *Dp = gt < 64 ? pick4(p.D, gt >> 4) : nullptr;
-  const bool dact = gt < 64 && pick4(p.active, gt >> 4) != 0;
+  const bool dact = gt < 64 && (gt & 15) == 0 && pick4(p.active, gt >> 4) != 0;
   // A failed (timed-out) wait ends the group at once.
   Item I;
   if (item_warp(p, c, base, 0, I) <= 0) return;
@@ -681,7 +697,7 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
     bool has_next = false;
     Item In = I;
     for (int kk = 0; kk < I.nk; ++kk, ++j) {
-      const int i2 = j & 1, c4 = j & 3;
+      const int ct = j % kTab;
       const uint32_t st = base + rslot(j) * kSlot;
       const float dt_cur = qdt[0], A2 = qa[0], Dv = qd[0];
       qdt[0] = qdt[1];
@@ -694,34 +710,30 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
         if (r < 0) return;
         has_next = r > 0;
       }
-      // ---- decays of this warp's direction (log2 units): prefix sum (forward)
-      //      or suffix sum (reverse) over the block
-      float v = dt_cur * A2;
+      // ---- decays of this warp's direction (log2 units): prefix sum over
+      //      the block; the reverse direction's suffix sum is total - prefix + own
+      const float v0 = dt_cur * A2;
       if (act) {
-        if (!rev) {
+        float v = v0;
 #pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const float u = __shfl_up_sync(0xffffffffu, v, o);
-            if (lane >= o) v += u;
-          }
-        } else {
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const float u = __shfl_down_sync(0xffffffffu, v, o);
-            if (lane + o < 32) v += u;
-          }
+        for (int o = 1; o < 32; o <<= 1) {
+          const float u = __shfl_up_sync(0xffffffffu, v, o);
+          if (lane >= o) v += u;
         }
-        sts_f32(cum + ((c4 * 4 + q) * 32 + lane) * 4, v);
-        sts_f32(dts + ((c4 * 4 + q) * 32 + lane) * 4, dt_cur);
-        if (!rev) sts_f32(ecum + ((c4 * 2 + q) * 32 + lane) * 4, ex2_approx(v));
+        if (rev) v = __shfl_sync(0xffffffffu, v, 31) - v + v0;
+        sts_f32(cum + ((ct * 4 + q) * 32 + lane) * 4, v);
+        sts_f32(dts + ((ct * 4 + q) * 32 + lane) * 4, dt_cur);
+        if (!rev) sts_f32(ecum + ((ct * 2 + q) * 32 + lane) * 4, ex2_approx(v));
       }
-      arrive_lane0(c, bAux0 + c4);
-      if (!waitw(c, bAux0 + c4, par4(j))) return;
-      // ---- (w o X) of the clean forward direction, bf16 hi + lo
-      if (p.need_s && j >= 1 && !waitw(c, bSFull0 + ((j + 1) & 1), par2(j - 1))) return;  // S(j-1) read Xw
+      if (dact) sts_f32(base + kOffDtab + (ct * 4 + (gt >> 4)) * 4, Dv);
+      if (gt == 0) sts_s32(base + kOffFtab + ct * 4, kk == 0 ? 1 + (m & 1) : 0);
+      arrive_lane0(c, bAux0 + ct);
+      if (!waitw(c, bAux0 + ct, part(j))) return;
       if (!waitw(c, bFull0 + rslot(j), parr(j))) return;
+      // ---- (w o X) of the clean forward direction, bf16 hi + lo
       if (p.need_s) {
-        const uint32_t cf = cum + (c4 * 4 + kCF) * 128, df = dts + (c4 * 4 + kCF) * 128;
+        if (j >= 1 && !waitw(c, bSFull0 + ((j + 1) & 1), par2(j - 1))) return;  // S(j-1) read Xw
+        const uint32_t cf = cum + (ct * 4 + kCF) * 128, df = dts + (ct * 4 + kCF) * 128;
         const float c31 = lds_f32(cf + 31 * 4);
 #pragma unroll
         for (int rep = 0; rep < 2; ++rep) {
@@ -738,59 +750,15 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
         fence_proxy_async_smem();
         arrive_lane0(c, bXwFull);
       }
-      if (!p.agg) {
-        // the epilogue of step j-2 has released its Y buffer: the MMAs that
-        // read this M buffer (and, at an item's first step, the D I_16 buffer
-        // of two items back) are complete, and the epilogue has read its
-        // decay tables
-        if (j >= 2 && !waitw(c, bYEmpty0 + i2, par2(j - 2))) return;
-        if (kk == 0 && gt < 64) {
-          // D I_16 operands of this item: bf16 hi + lo of each direction's D
-          // on the diagonal (the rest of the buffer stays zero)
-          const int i = gt >> 4, d = gt & 15;
-          if (dact) {
-            const __nv_bfloat16 dh = __float2bfloat16_rn(Dv);
-            const __nv_bfloat16 dl = __float2bfloat16_rn(Dv - __bfloat162float(dh));
-            const uint32_t off = (m & 1) * kDgBuf + (d >> 3) * kDgSbo + (d >> 3) * kDgLbo + (d & 7) * 16 + (d & 7) * 2;
-            sts_u16(base + kOffDg + (2 * i) * 512 + off, __bfloat16_as_ushort(dh));
-            sts_u16(base + kOffDg + (2 * i + 1) * 512 + off, __bfloat16_as_ushort(dl));
-          }
-        }
-        // ---- masked-decay matrix, row s = lane of M^T for this direction
-        if (act) {
-          const uint32_t cbrow = st + kOffCB + q * 2048;
-          const uint32_t cq = cum + (c4 * 4 + q) * 128;
-          const float cs = v, ds = dt_cur;
-          const uint32_t mrow = base + kOffMh + i2 * kMhBuf + q * 2048;
-          // (not unrolled: a compact loop keeps the instruction cache footprint down)
-#pragma unroll 1
-          for (int jj = 0; jj < 4; ++jj) {
-            uint32_t r[4];
-            ld_shared_v4(cbrow + sw64_chunk(lane, jj), r[0], r[1], r[2], r[3]);  // C B^T[s = lane][8 jj ..]
-            float cj[8];
-            ld_shared_v4f(cq + 32 * jj, *reinterpret_cast<float(*)[4]>(&cj[0]));
-            ld_shared_v4f(cq + 32 * jj + 16, *reinterpret_cast<float(*)[4]>(&cj[4]));
-            float mv[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const int t = 8 * jj + i;
-              const bool valid = rev ? (t <= lane) : (t >= lane);
-              const float e = ex2_approx(cj[i] - cs);
-              const float cb = (i & 1) ? bf16_hi_f(r[i >> 1]) : bf16_lo_f(r[i >> 1]);
-              mv[i] = valid ? cb * ds * e : 0.f;
-            }
-            st_shared_v4(mrow + inter_mn_off(8 * jj, lane, kMhSbo, kMhLbo), pack_bf16x2(mv[0], mv[1]),
-                         pack_bf16x2(mv[2], mv[3]), pack_bf16x2(mv[4], mv[5]), pack_bf16x2(mv[6], mv[7]));
-          }
-        }
-      }
-      fence_proxy_async_smem();
-      arrive_lane0(c, bMhFull0 + i2);
       arrive_lane0(c, bEmpty0 + rslot(j));
     }
-    if (!has_next) return;
+    if (!has_next) break;
     I = In;
   }
+  // past the last step: tell the epilogue's look-ahead that there is no more
+  const int ct = j % kTab;
+  if (gt == 0) sts_s32(base + kOffFtab + ct * 4, -1);
+  arrive_lane0(c, bAux0 + ct);
 }
 
 // ---------------------------------------------------------------- state group
@@ -948,9 +916,9 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
         if (sdst) sdst += static_cast<int64_t>(p.H) * PN;
       }
       if (kk == nk) break;
-      const int i2 = j & 1, c4 = j & 3;
-      if (!waitw(c, bAux0 + c4, par4(j))) return;
-      const float c31 = lds_f32(cum + ((c4 * 4 + kCF) * 32 + 31) * 4);
+      const int i2 = j & 1, ct = j % kTab;
+      if (!waitw(c, bAux0 + ct, part(j))) return;
+      const float c31 = lds_f32(cum + ((ct * 4 + kCF) * 32 + 31) * 4);
       const float atot = ex2_approx(c31);
       decay_log2 += c31;
       if (!waitw(c, bSFull0 + i2, par2(j))) return;
@@ -977,9 +945,13 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
 // warps 10..13: thread owns column p = 16 q + (lane & 15) of the clean
 // (lane < 16) or noisy (lane >= 16) stream's outputs y[t][p], t = 0..31:
 // y = exp(cum_t) Y_off + Y_diag (Y_diag already holds both directions' D x).
+// After the outputs of step j the group builds, two steps ahead, the
+// masked-decay matrices of step j + 2 (warp q: direction slot q, row s = lane
+// of M^T) and, at an item's first step, the D I_16 operands of the item.
 __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
   const int lane = threadIdx.x & 31;
   const int q = (threadIdx.x >> 5) & 3;
+  const int gq = threadIdx.x - 320;  // 0..127
   const int pcol = 16 * q + (lane & 15);
   const bool noisy = lane >= 16;
   const int fs = noisy ? kNF : kCF;
@@ -988,15 +960,78 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
   const uint32_t ecum = base + kOffEc;
   const int64_t H = p.H, L = p.L;
   if (p.agg) return;
+  const bool act = pick4(p.active, q) != 0;
+  const bool rev = q >= 2;
+  int mla = 0;        // next step whose masked-decay matrices this group builds
+  bool mend = false;  // past the CTA's last step
   // A failed (timed-out) wait ends the group at once.
+  auto build_m = [&]() -> bool {
+    if (mend) return true;
+    const int jm = mla;
+    const int ct = jm % kTab;
+    if (!waitw(c, bAux0 + ct, part(jm))) return false;
+    const int f = lds_s32(base + kOffFtab + ct * 4);
+    if (f < 0) {
+      mend = true;
+      return true;
+    }
+    if (!waitw(c, bFull0 + rslot(jm), parr(jm))) return false;  // C B^T tiles
+    if (act) {
+      const uint32_t cbrow = base + rslot(jm) * kSlot + kOffCB + q * 2048;
+      const uint32_t cq = base + kOffCum + (ct * 4 + q) * 128;
+      const float cs = lds_f32(cq + lane * 4);
+      const float ds = lds_f32(base + kOffDt + (ct * 4 + q) * 128 + lane * 4);
+      const uint32_t mrow = base + kOffMh + (jm & 1) * kMhBuf + q * 2048;
+      // (not unrolled: a compact loop keeps the instruction cache footprint down)
+#pragma unroll 1
+      for (int jj = 0; jj < 4; ++jj) {
+        uint32_t r[4];
+        ld_shared_v4(cbrow + sw64_chunk(lane, jj), r[0], r[1], r[2], r[3]);  // C B^T[s = lane][8 jj ..]
+        float cj[8];
+        ld_shared_v4f(cq + 32 * jj, *reinterpret_cast<float(*)[4]>(&cj[0]));
+        ld_shared_v4f(cq + 32 * jj + 16, *reinterpret_cast<float(*)[4]>(&cj[4]));
+        float mv[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int t = 8 * jj + i;
+          const bool valid = rev ? (t <= lane) : (t >= lane);
+          const float e = ex2_approx(cj[i] - cs);
+          const float cb = (i & 1) ? bf16_hi_f(r[i >> 1]) : bf16_lo_f(r[i >> 1]);
+          mv[i] = valid ? cb * ds * e : 0.f;
+        }
+        st_shared_v4(mrow + inter_mn_off(8 * jj, lane, kMhSbo, kMhLbo), pack_bf16x2(mv[0], mv[1]),
+                     pack_bf16x2(mv[2], mv[3]), pack_bf16x2(mv[4], mv[5]), pack_bf16x2(mv[6], mv[7]));
+      }
+    }
+    if (f > 0 && gq < 64) {
+      // D I_16 operands of the item that starts here: bf16 hi + lo of each
+      // direction's D on the diagonal (the rest of the buffer stays zero).
+      // The MMAs of two items back, the buffer's last readers, are complete.
+      const int i = gq >> 4, d = gq & 15;
+      if (pick4(p.active, i)) {
+        const float Dv = lds_f32(base + kOffDtab + (ct * 4 + i) * 4);
+        const __nv_bfloat16 dh = __float2bfloat16_rn(Dv);
+        const __nv_bfloat16 dl = __float2bfloat16_rn(Dv - __bfloat162float(dh));
+        const uint32_t off =
+            static_cast<uint32_t>(f - 1) * kDgBuf + (d >> 3) * kDgSbo + (d >> 3) * kDgLbo + (d & 7) * 16 + (d & 7) * 2;
+        sts_u16(base + kOffDg + (2 * i) * 512 + off, __bfloat16_as_ushort(dh));
+        sts_u16(base + kOffDg + (2 * i + 1) * 512 + off, __bfloat16_as_ushort(dl));
+      }
+    }
+    fence_proxy_async_smem();
+    arrive_lane0(c, bMhFull0 + (jm & 1));
+    ++mla;
+    return true;
+  };
+  if (!build_m() || !build_m()) return;  // steps 0 and 1
   int j = 0;
   for (int m = 0;; ++m) {
     Item I;
     if (item_warp(p, c, base, m, I) <= 0) return;
     for (int kk = 0; kk < I.nk; ++kk, ++j) {
       const int k = I.k0 + kk;  // block index in the sequence
-      const int i2 = j & 1, c4 = j & 3;
-      if (!waitw(c, bAux0 + c4, par4(j))) return;
+      const int i2 = j & 1, ct = j % kTab;
+      if (!waitw(c, bAux0 + ct, part(j))) return;
       if (!waitw(c, bYFull0 + i2, par2(j))) return;
       tc_fence_after();
       uint32_t yo[32], yd[32];
@@ -1004,7 +1039,7 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
       tmem_ld_16x32bx2_x32<32>(ta, yo);
       tmem_ld_16x32bx2_x32<32>(ta + 64, yd);
       tmem_ld_wait();
-      const uint32_t eq = ecum + (c4 * 2 + fs) * 128;
+      const uint32_t eq = ecum + (ct * 2 + fs) * 128;
 #pragma unroll
       for (int jj = 0; jj < 8; ++jj) {
         float e4[4];
@@ -1014,7 +1049,7 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
           yo[4 * jj + i] =
               __float_as_uint(fmaf(e4[i], __uint_as_float(yo[4 * jj + i]), __uint_as_float(yd[4 * jj + i])));
       }
-      // the Y buffer and this step's decay tables may be reused from here on
+      // the Y buffer may be reused from here on
       tc_fence_before();
       arrive_lane0(c, bYEmpty0 + i2);
       if (mine) {
@@ -1030,6 +1065,7 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
           for (int t = 0; t < 32; ++t) dst[t * tstride] = __uint_as_float(yo[t]);
         }
       }
+      if (!build_m()) return;  // step j + 2
     }
   }
 }
