@@ -41,6 +41,10 @@ class _Dir(ctypes.Structure):
                 ("A", _dp), ("D", _dp)]
 
 
+class _Grad(ctypes.Structure):
+    _fields_ = [("dx", _dp), ("ddt", _dp), ("dB", _dp), ("dC", _dp), ("dA", _dp), ("dD", _dp)]
+
+
 def build(force: bool = False) -> str:
     """Compile the oracle shared library with gcc (-O2, OpenMP).  Returns its path."""
     if force or not os.path.exists(_LIB_PATH) or (
@@ -55,7 +59,7 @@ def build(force: bool = False) -> str:
 
 def _open(path: str):
     lib = ctypes.CDLL(path)
-    for name in ("oracle_prefix", "oracle_block_step", "oracle_allblock"):
+    for name in ("oracle_prefix", "oracle_block_step", "oracle_allblock", "oracle_allblock_backward"):
         getattr(lib, name).restype = ctypes.c_int
     lib.oracle_max_threads.restype = ctypes.c_int
     lib.oracle_set_threads.argtypes = [ctypes.c_int]
@@ -180,6 +184,42 @@ def allblock(shape: dict, clean_fwd: dict, clean_rev: dict | None, noisy_fwd: di
     return yc, yn, st
 
 
+GRAD_KEYS = ("x", "dt", "B", "C", "A", "D")
+
+
+def allblock_backward(shape: dict, clean_fwd: dict, clean_rev: dict | None, noisy_fwd: dict,
+                      noisy_rev: dict | None, h0=None, dy_clean=None, dy_noisy=None, dstates=None,
+                      lib=None):
+    """Gradients of a loss L(y_clean, y_noisy, states) through the all-block pass
+    (ungated), given dL/dy_clean (or None), dL/dy_noisy and dL/dstates (or None).
+    Returns (grads, dh0): grads[i] (i = 0 clean fwd, 1 clean rev, 2 noisy fwd,
+    3 noisy rev; None for an absent direction) is a dict with keys
+    x, dt, B, C, A, D holding float64 arrays shaped like the inputs."""
+    lib = lib or _load()
+    B, L, H, P, N, G = (int(shape[k]) for k in
+                        ("batch", "seqlen", "nheads", "headdim", "dstate", "ngroups"))
+    m = _Marshal()
+    dirs = [clean_fwd, clean_rev, noisy_fwd, noisy_rev]
+    grads, structs = [], []
+    for d in dirs:
+        if d is None:
+            grads.append(None)
+            structs.append(None)
+            continue
+        g = {"x": np.zeros((B, L, H, P)), "dt": np.zeros((B, L, H)), "B": np.zeros((B, L, G, N)),
+             "C": np.zeros((B, L, G, N)), "A": np.zeros((H,)), "D": np.zeros((H,))}
+        grads.append(g)
+        structs.append(ctypes.pointer(_Grad(dx=_ptr(g["x"]), ddt=_ptr(g["dt"]), dB=_ptr(g["B"]),
+                                            dC=_ptr(g["C"]), dA=_ptr(g["A"]), dD=_ptr(g["D"]))))
+    dh0 = np.zeros((B, H, P, N))
+    rc = lib.oracle_allblock_backward(ctypes.byref(_shape(shape)), m.dir(clean_fwd), m.dir(clean_rev),
+                                      m.dir(noisy_fwd), m.dir(noisy_rev), _ptr(m.arr(h0)),
+                                      _ptr(m.arr(dy_clean)), _ptr(m.arr(dy_noisy)), _ptr(m.arr(dstates)),
+                                      structs[0], structs[1], structs[2], structs[3], _ptr(dh0))
+    _check(rc, "oracle_allblock_backward")
+    return grads, dh0
+
+
 class Variant:
     """The same API bound to another build of the oracle source (used by the
     tests that plant a mistake in a copy of the oracle and check that the pins
@@ -196,6 +236,9 @@ class Variant:
 
     def allblock(self, *a, **k):
         return allblock(*a, lib=self.lib, **k)
+
+    def allblock_backward(self, *a, **k):
+        return allblock_backward(*a, lib=self.lib, **k)
 
 
 def compile_variant(src_text: str, out_path: str) -> str:

@@ -247,6 +247,233 @@ int oracle_allblock(const oracle_shape_t *s, const oracle_dir_t *cf, const oracl
     return failed ? ORACLE_ENOMEM : ORACLE_OK;
 }
 
+/* ------------------------------------------------------------------ backward
+ *
+ * Reverse-mode derivative of oracle_allblock (ungated), for the training pass
+ * that the all-block objective implies: gradients of a loss
+ * L(y_clean, y_noisy, states) reach every input, and through the boundary
+ * states the noisy blocks' losses reach the clean prefix scan ("Training
+ * Hybrid Block Diffusion Language Models with Partial Bidirectionality",
+ * all-block paragraph after eq. (5) and eq. (14)).
+ *
+ * Plain adjoint of the recurrence of eq. (1), token by token in reverse
+ * processing order, with the forward states of each pass recomputed and
+ * stored (no chunking).  For a token t with a_t = exp(dt_t A):
+ *     G        <- G + dy_t C_t^T                 (dL/dh_t, P x N)
+ *     dC_t     += dy_t^T h_t          dx_t += D dy_t + dt_t G B_t
+ *     dB_t     += dt_t G^T x_t        dD   += dy_t . x_t
+ *     ddt_t    += sum G o (A a_t h_prev + x_t B_t^T)
+ *     dA       += sum G o (dt_t a_t h_prev)
+ *     G        <- a_t G                          (dL/dh_prev)
+ * dB and dC of a group sum over its heads; dA and dD sum over batch and
+ * tokens.  Sums are taken in a fixed order (per (b, h) partials, then a
+ * serial reduction), so the result does not depend on the thread count. */
+typedef struct {
+    double *dx, *ddt, *dB, *dC, *dA, *dD; /* any may be NULL (not wanted) */
+} oracle_grad_t;
+
+typedef struct {
+    double *dx, *ddt; /* [L][P], [L] of this (b, h) */
+    double *dB, *dC;  /* [L][N] of this (b, h) (group sums taken later) */
+    double dA, dD;
+} bwd_acc_t;
+
+/* Backward through the pass that processed tokens order[0..n-1] (in that
+ * order) from the state h_start.  G holds dL/d(state after the last processed
+ * token) on entry and dL/dh_start on return.  dstate_at(i) (may be NULL)
+ * adds the incoming gradient on the state after processed token i.
+ * hist: scratch of n * P * N doubles. */
+static void pass_backward(const oracle_shape_t *s, const oracle_dir_t *d, int64_t b, int64_t h,
+                          const int64_t *order, int64_t n, const double *h_start, const double *dy,
+                          const double *const *dstate_at, double *G, double *hist, bwd_acc_t *acc) {
+    const int64_t L = s->seqlen, H = s->nheads, P = s->headdim, N = s->dstate, Gn = s->ngroups;
+    const int64_t g = h / (H / Gn), PN = P * N;
+    /* forward recompute */
+    for (int64_t i = 0; i < n; ++i) {
+        const int64_t t = order[i];
+        const double dt = d->dt[(b * L + t) * H + h];
+        const double a = exp(dt * d->A[h]);
+        const double *x = d->x + ((b * L + t) * H + h) * P;
+        const double *Bt = d->Bm + ((b * L + t) * Gn + g) * N;
+        const double *prev = i ? hist + (i - 1) * PN : h_start;
+        double *cur = hist + i * PN;
+        for (int64_t p = 0; p < P; ++p)
+            for (int64_t q = 0; q < N; ++q)
+                cur[p * N + q] = a * (prev ? prev[p * N + q] : 0.0) + dt * x[p] * Bt[q];
+    }
+    /* adjoint, reverse processing order */
+    for (int64_t i = n - 1; i >= 0; --i) {
+        const int64_t t = order[i];
+        const double dt = d->dt[(b * L + t) * H + h];
+        const double A = d->A[h];
+        const double a = exp(dt * A);
+        const double *x = d->x + ((b * L + t) * H + h) * P;
+        const double *Bt = d->Bm + ((b * L + t) * Gn + g) * N;
+        const double *Ct = d->Cm + ((b * L + t) * Gn + g) * N;
+        const double *dyt = dy ? dy + ((b * L + t) * H + h) * P : NULL;
+        const double *ht = hist + i * PN;
+        const double *prev = i ? hist + (i - 1) * PN : h_start;
+        if (dstate_at && dstate_at[i])
+            for (int64_t e = 0; e < PN; ++e) G[e] += dstate_at[i][e];
+        if (dyt)
+            for (int64_t p = 0; p < P; ++p)
+                for (int64_t q = 0; q < N; ++q) G[p * N + q] += dyt[p] * Ct[q];
+        double ddt = 0.0, dA = 0.0;
+        for (int64_t p = 0; p < P; ++p) {
+            double gb = 0.0;
+            for (int64_t q = 0; q < N; ++q) {
+                const double Gv = G[p * N + q];
+                const double hp = prev ? prev[p * N + q] : 0.0;
+                gb += Gv * Bt[q];
+                ddt += Gv * (A * a * hp + x[p] * Bt[q]);
+                dA += Gv * dt * a * hp;
+            }
+            acc->dx[t * P + p] += dt * gb + (dyt ? d->D[h] * dyt[p] : 0.0);
+        }
+        for (int64_t q = 0; q < N; ++q) {
+            double sb = 0.0, sc = 0.0;
+            for (int64_t p = 0; p < P; ++p) {
+                sb += G[p * N + q] * x[p];
+                if (dyt) sc += dyt[p] * ht[p * N + q];
+            }
+            acc->dB[t * N + q] += dt * sb;
+            acc->dC[t * N + q] += sc;
+        }
+        if (dyt)
+            for (int64_t p = 0; p < P; ++p) acc->dD += dyt[p] * x[p];
+        acc->ddt[t] += ddt;
+        acc->dA += dA;
+        for (int64_t e = 0; e < PN; ++e) G[e] *= a;
+    }
+}
+
+int oracle_allblock_backward(const oracle_shape_t *s, const oracle_dir_t *cf, const oracle_dir_t *cr,
+                             const oracle_dir_t *nf, const oracle_dir_t *nr, const double *h0,
+                             const double *dy_clean, const double *dy_noisy, const double *dstates,
+                             oracle_grad_t *gcf, oracle_grad_t *gcr, oracle_grad_t *gnf, oracle_grad_t *gnr,
+                             double *dh0) {
+    int rc = check_shape(s);
+    if (rc || (rc = check_dir(cf)) || (rc = check_dir(nf))) return rc;
+    if (cr && (rc = check_dir(cr))) return rc;
+    if (nr && (rc = check_dir(nr))) return rc;
+    if (cf->z || nf->z || (cr && cr->z) || (nr && nr->z)) return ORACLE_EINVAL; /* ungated only */
+    if (!gcf || !gnf || (cr && !gcr) || (nr && !gnr)) return ORACLE_EINVAL;
+    const int64_t B = s->batch, L = s->seqlen, H = s->nheads, P = s->headdim, N = s->dstate;
+    const int64_t Gn = s->ngroups, T = s->block_len, K = L / T, PN = P * N;
+    const oracle_dir_t *dirs[4] = {cf, cr, nf, nr};
+    oracle_grad_t *grads[4] = {gcf, gcr, gnf, gnr};
+    /* forward states of the clean stream (the checkpoints of the pass) */
+    double *states = (double *)malloc(sizeof(double) * (B * K * H * PN > 0 ? B * K * H * PN : 1));
+    double *ytmp = (double *)malloc(sizeof(double) * (B * L * H * P > 0 ? B * L * H * P : 1));
+    /* per (direction, b, h) partials */
+    const size_t nbh = (size_t)(B * H);
+    bwd_acc_t *acc = (bwd_acc_t *)calloc(4 * (nbh ? nbh : 1), sizeof(bwd_acc_t));
+    double *pool = (double *)calloc(4 * (nbh ? nbh : 1) * (size_t)(L * P + L + 2 * L * N), sizeof(double));
+    if (!states || !ytmp || !acc || !pool) {
+        free(states); free(ytmp); free(acc); free(pool);
+        return ORACLE_ENOMEM;
+    }
+    for (size_t i = 0; i < 4 * nbh; ++i) {
+        double *base = pool + i * (size_t)(L * P + L + 2 * L * N);
+        acc[i].dx = base;
+        acc[i].ddt = base + L * P;
+        acc[i].dB = base + L * P + L;
+        acc[i].dC = base + L * P + L + L * N;
+    }
+    rc = oracle_allblock(s, cf, cr, nf, nr, h0, NULL, ytmp, states);
+    free(ytmp);
+    if (rc) { free(states); free(acc); free(pool); return rc; }
+    int failed = 0;
+#pragma omp parallel
+    {
+        double *G = (double *)malloc(sizeof(double) * PN);
+        double *hist = (double *)malloc(sizeof(double) * (L > 0 ? L : 1) * PN);
+        int64_t *order = (int64_t *)malloc(sizeof(int64_t) * (L > 0 ? L : 1));
+        const double **dat = (const double **)calloc(L > 0 ? L : 1, sizeof(double *));
+        double *dsn = (double *)malloc(sizeof(double) * (K > 0 ? K : 1) * PN); /* dL/d states[k] from noisy block k+1 */
+        if (!G || !hist || !order || !dat || !dsn) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t bh = 0; bh < B * H; ++bh) {
+                const int64_t b = bh / H, h = bh % H;
+                memset(dsn, 0, sizeof(double) * K * PN);
+                double *dh0_bh = dh0 ? dh0 + (b * H + h) * PN : NULL;
+                if (dh0_bh) memset(dh0_bh, 0, sizeof(double) * PN);
+                /* noisy blocks: forward from the clean boundary state before it */
+                for (int64_t k = 0; k < K; ++k) {
+                    const double *hs0 = k ? states + ((b * K + k - 1) * H + h) * PN
+                                          : (h0 ? h0 + (b * H + h) * PN : NULL);
+                    for (int64_t i = 0; i < T; ++i) order[i] = k * T + i;
+                    memset(G, 0, sizeof(double) * PN);
+                    pass_backward(s, nf, b, h, order, T, hs0, dy_noisy, NULL, G, hist, &acc[2 * nbh + bh]);
+                    if (k) {
+                        for (int64_t e = 0; e < PN; ++e) dsn[(k - 1) * PN + e] += G[e];
+                    } else if (dh0_bh) {
+                        for (int64_t e = 0; e < PN; ++e) dh0_bh[e] += G[e];
+                    }
+                    if (nr) {
+                        for (int64_t i = 0; i < T; ++i) order[i] = (k + 1) * T - 1 - i;
+                        memset(G, 0, sizeof(double) * PN);
+                        pass_backward(s, nr, b, h, order, T, NULL, dy_noisy, NULL, G, hist, &acc[3 * nbh + bh]);
+                    }
+                    if (cr) {
+                        for (int64_t i = 0; i < T; ++i) order[i] = (k + 1) * T - 1 - i;
+                        memset(G, 0, sizeof(double) * PN);
+                        pass_backward(s, cr, b, h, order, T, NULL, dy_clean, NULL, G, hist, &acc[1 * nbh + bh]);
+                    }
+                }
+                /* clean forward over the whole sequence; incoming gradients on
+                 * states[k] (given, and from noisy block k + 1) after token (k+1)T-1 */
+                if (dstates)
+                    for (int64_t k = 0; k < K; ++k)
+                        for (int64_t e = 0; e < PN; ++e)
+                            dsn[k * PN + e] += dstates[((b * K + k) * H + h) * PN + e];
+                for (int64_t i = 0; i < L; ++i) {
+                    order[i] = i;
+                    dat[i] = ((i + 1) % T == 0) ? dsn + (i / T) * PN : NULL;
+                }
+                memset(G, 0, sizeof(double) * PN);
+                pass_backward(s, cf, b, h, order, L, h0 ? h0 + (b * H + h) * PN : NULL, dy_clean, dat, G,
+                              hist, &acc[0 * nbh + bh]);
+                if (dh0_bh)
+                    for (int64_t e = 0; e < PN; ++e) dh0_bh[e] += G[e];
+            }
+        }
+        free(G); free(hist); free(order); free((void *)dat); free(dsn);
+    }
+    if (!failed) {
+        /* fixed-order reductions */
+        for (int di = 0; di < 4; ++di) {
+            if (!dirs[di]) continue;
+            oracle_grad_t *gr = grads[di];
+            if (gr->dB) memset(gr->dB, 0, sizeof(double) * B * L * Gn * N);
+            if (gr->dC) memset(gr->dC, 0, sizeof(double) * B * L * Gn * N);
+            if (gr->dA) memset(gr->dA, 0, sizeof(double) * H);
+            if (gr->dD) memset(gr->dD, 0, sizeof(double) * H);
+            for (int64_t b = 0; b < B; ++b)
+                for (int64_t h = 0; h < H; ++h) {
+                    const bwd_acc_t *a = &acc[di * nbh + b * H + h];
+                    const int64_t g = h / (H / Gn);
+                    for (int64_t t = 0; t < L; ++t) {
+                        if (gr->dx)
+                            memcpy(gr->dx + ((b * L + t) * H + h) * P, a->dx + t * P, sizeof(double) * P);
+                        if (gr->ddt) gr->ddt[(b * L + t) * H + h] = a->ddt[t];
+                        for (int64_t q = 0; q < N; ++q) {
+                            if (gr->dB) gr->dB[((b * L + t) * Gn + g) * N + q] += a->dB[t * N + q];
+                            if (gr->dC) gr->dC[((b * L + t) * Gn + g) * N + q] += a->dC[t * N + q];
+                        }
+                    }
+                    if (gr->dA) gr->dA[h] += a->dA;
+                    if (gr->dD) gr->dD[h] += a->dD;
+                }
+        }
+    }
+    free(states); free(acc); free(pool);
+    return failed ? ORACLE_ENOMEM : ORACLE_OK;
+}
+
 int oracle_max_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();
