@@ -292,7 +292,7 @@ static void pass_backward(const oracle_shape_t *s, const oracle_dir_t *d, int64_
     for (int64_t i = 0; i < n; ++i) {
         const int64_t t = order[i];
         const double dt = d->dt[(b * L + t) * H + h];
-        const double a = exp(dt * d->A[h]);
+        const double a = exp(d->A[h] * dt); /* (same decay as the forward pass) */
         const double *x = d->x + ((b * L + t) * H + h) * P;
         const double *Bt = d->Bm + ((b * L + t) * Gn + g) * N;
         const double *prev = i ? hist + (i - 1) * PN : h_start;
