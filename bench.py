@@ -333,6 +333,7 @@ def run_extra(dev, pk) -> dict:
         out["block_step_3b_b1_40layers"] = _step_stack(W.WORKLOADS["3b_step_b1"], 40, dev, pk)
         out["block_step_3b_b64_40layers"] = _step_stack(W.WORKLOADS["3b_step_b64"], 40, dev, pk)
         out["prefill_700m_8k_per_layer"] = _prefill(W.WORKLOADS["700m_prefill_8k"], dev, pk)
+        out["allblock_backward_87m"] = _backward(W.WORKLOADS["87m_allblock"], dev, pk)
     except Exception as e:  # report, never hide
         out["error"] = repr(e)
     return out
@@ -376,6 +377,22 @@ def _step_stack(s: W.Shape, layers: int, dev, pk) -> dict:
     return {"us_per_step": ms * 1e3, "tokens_per_s": s.batch * s.seqlen / (ms * 1e-3),
             "algorithmic_bytes": b, "hbm_frac": b / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
             "layers": layers, "batch": s.batch, "graph": True}
+
+
+def _backward(s: W.Shape, dev, pk) -> dict:
+    """Backward of the all-block layer (gradients of every input of the four
+    directions and of h0), from the forward's boundary states."""
+    cf, cr, nf, nr = W.make_streams(s, W.SEEDS[WORKLOAD], device=dev)
+    _, yn, st = bd.allblock(s, cf, cr, nf, nr)
+    g = torch.Generator(device=dev).manual_seed(7)
+    dyn = torch.randn(yn.shape, generator=g, device=dev)
+    dyc = torch.randn(yn.shape, generator=g, device=dev)
+    ws = bd.workspace(s, bd.BDSCAN_OP_ALLBLOCK_BACKWARD, dev)
+    grads, dh0 = bd.allblock_backward(s, cf, cr, nf, nr, st, dyn, dy_clean=dyc, ws=ws)
+    ms = _time(lambda: bd.allblock_backward(s, cf, cr, nf, nr, st, dyn, dy_clean=dyc, grads=grads, ws=ws),
+               dev, 5)
+    return {"us_per_call": ms * 1e3, "tokens_per_s": s.batch * s.seqlen / (ms * 1e-3),
+            "kernel": "generic CUDA-core backward (per-block adjoint in shared memory)"}
 
 
 def _prefill(s: W.Shape, dev, pk) -> dict:

@@ -24,7 +24,7 @@ LIB_PATH = os.path.join(_PKG, "libbdscan.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "bdscan.h")
 
 BDSCAN_BF16, BDSCAN_FP32 = 0, 1
-BDSCAN_OP_PREFIX, BDSCAN_OP_BLOCK_STEP, BDSCAN_OP_ALLBLOCK = 0, 1, 2
+BDSCAN_OP_PREFIX, BDSCAN_OP_BLOCK_STEP, BDSCAN_OP_ALLBLOCK, BDSCAN_OP_ALLBLOCK_BACKWARD = 0, 1, 2, 3
 STATUS = {0: "BDSCAN_OK", -1: "BDSCAN_ERR_INVALID_ARG", -2: "BDSCAN_ERR_UNSUPPORTED_SHAPE",
           -3: "BDSCAN_ERR_MISALIGNED", -4: "BDSCAN_ERR_WORKSPACE", -5: "BDSCAN_ERR_CUDA",
           -6: "BDSCAN_ERR_TIMEOUT", -7: "BDSCAN_ERR_SCRATCH_LIMIT"}
@@ -40,6 +40,10 @@ class bdscan_dir_t(ctypes.Structure):
     _fields_ = [("x", ctypes.c_void_p), ("dt", ctypes.c_void_p), ("B", ctypes.c_void_p),
                 ("C", ctypes.c_void_p), ("z", ctypes.c_void_p), ("A", ctypes.c_void_p),
                 ("D", ctypes.c_void_p)]
+
+
+class bdscan_grad_t(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("dx", "ddt", "dB", "dC", "dA", "dD")]
 
 
 class BdscanError(RuntimeError):
@@ -67,7 +71,10 @@ def lib() -> ctypes.CDLL:
             L.bdscan_prefix.argtypes = [sp, dp, dp, vp, vp, vp, vp, vp, sz, vp]
             L.bdscan_block_step.argtypes = [sp, dp, dp, vp, vp, vp, vp, sz, vp]
             L.bdscan_allblock.argtypes = [sp, dp, dp, dp, dp, vp, vp, vp, vp, vp, sz, vp]
-            for fn in ("bdscan_prefix", "bdscan_block_step", "bdscan_allblock",
+            gp = ctypes.POINTER(bdscan_grad_t)
+            L.bdscan_allblock_backward.argtypes = [sp, dp, dp, dp, dp, vp, vp, vp, vp, vp, gp, gp, gp, gp,
+                                                   vp, vp, sz, vp]
+            for fn in ("bdscan_prefix", "bdscan_block_step", "bdscan_allblock", "bdscan_allblock_backward",
                        "bdscan_check_status", "bdscan_version"):
                 getattr(L, fn).restype = ctypes.c_int
             L.bdscan_workspace_size.argtypes = [sp, ctypes.c_int]
@@ -105,6 +112,12 @@ def bdscan_allblock(shape, cf, cr, nf, nr, h0, y_clean, y_noisy, block_states, w
                     stream) -> int:
     return lib().bdscan_allblock(shape, cf, cr, nf, nr, h0, y_clean, y_noisy, block_states, ws,
                                  ws_bytes, stream)
+
+
+def bdscan_allblock_backward(shape, cf, cr, nf, nr, h0, block_states, dy_clean, dy_noisy, dstates,
+                             g_cf, g_cr, g_nf, g_nr, dh0, ws, ws_bytes, stream) -> int:
+    return lib().bdscan_allblock_backward(shape, cf, cr, nf, nr, h0, block_states, dy_clean, dy_noisy,
+                                          dstates, g_cf, g_cr, g_nf, g_nr, dh0, ws, ws_bytes, stream)
 
 
 def bdscan_block_step_noalloc(shape, fwd, rev, state_in, y, state_out, stream) -> int:
@@ -270,3 +283,44 @@ def allblock(s: Shape, clean_fwd: dict, clean_rev: dict | None, noisy_fwd: dict,
                          _stream(dev, stream))
     _raise("bdscan_allblock", rc)
     return y_clean, y_noisy, states
+
+
+GRAD_KEYS = ("x", "dt", "B", "C", "A", "D")
+
+
+def allblock_backward(s: Shape, clean_fwd: dict, clean_rev: dict | None, noisy_fwd: dict,
+                      noisy_rev: dict | None, states, dy_noisy, dy_clean=None, dstates=None, h0=None,
+                      want_dh0: bool = True, grads=None, ws=None, stream=None):
+    """Backward of the all-block pass.  ``states`` is the forward call's block
+    states; ``dy_*`` have the output dtype.  Returns (grads, dh0): grads[i]
+    (i = clean fwd, clean rev, noisy fwd, noisy rev; None if absent) is a dict
+    of fp32 tensors keyed like the inputs (x, dt, B, C, A, D)."""
+    dev = clean_fwd["x"].device
+    cs = c_shape(s)
+    dirs = [clean_fwd, clean_rev, noisy_fwd, noisy_rev]
+    cd = [c_dir(s, d, dev) for d in dirs]
+    B, L, H, P, N, G, K = s.batch, s.seqlen, s.nheads, s.headdim, s.dstate, s.ngroups, s.nblocks
+    tout = _DT[s.out_dtype][0]
+    _check_tensor("states", states, (B, K, H, P, N), torch.float32, dev)
+    _check_tensor("dy_noisy", dy_noisy, (B, L, H, P), tout, dev)
+    if dy_clean is not None:
+        _check_tensor("dy_clean", dy_clean, (B, L, H, P), tout, dev)
+    if dstates is not None:
+        _check_tensor("dstates", dstates, (B, K, H, P, N), torch.float32, dev)
+    if h0 is not None:
+        _check_tensor("h0", h0, (B, H, P, N), torch.float32, dev)
+    if grads is None:
+        f = dict(device=dev, dtype=torch.float32)
+        grads = [None if d is None else
+                 {"x": torch.empty((B, L, H, P), **f), "dt": torch.empty((B, L, H), **f),
+                  "B": torch.empty((B, L, G, N), **f), "C": torch.empty((B, L, G, N), **f),
+                  "A": torch.empty((H,), **f), "D": torch.empty((H,), **f)} for d in dirs]
+    cg = [None if g is None else bdscan_grad_t(*(_ptr(g[k]) for k in GRAD_KEYS)) for g in grads]
+    dh0 = _state(s, dev) if want_dh0 else None
+    ws = workspace(s, BDSCAN_OP_ALLBLOCK_BACKWARD, dev) if ws is None else ws
+    rc = bdscan_allblock_backward(ctypes.byref(cs), _ref(cd[0]), _ref(cd[1]), _ref(cd[2]), _ref(cd[3]),
+                                  _ptr(h0), _ptr(states), _ptr(dy_clean), _ptr(dy_noisy), _ptr(dstates),
+                                  _ref(cg[0]), _ref(cg[1]), _ref(cg[2]), _ref(cg[3]), _ptr(dh0), _ptr(ws),
+                                  ws.numel(), _stream(dev, stream))
+    _raise("bdscan_allblock_backward", rc)
+    return grads, dh0

@@ -156,6 +156,8 @@ extern "C" {
 
 size_t bdscan_workspace_size(const bdscan_shape_t *shape, int op) {
   if (check_shape(shape) != BDSCAN_OK) return 0;
+  if (op == BDSCAN_OP_ALLBLOCK_BACKWARD)
+    return bdscan::kWsHeader + bdscan::bwd_workspace_bytes(shape->batch, shape->seqlen, shape->nheads, shape->dstate);
   if (op != BDSCAN_OP_PREFIX && op != BDSCAN_OP_BLOCK_STEP && op != BDSCAN_OP_ALLBLOCK) return 0;
   // The tensor-core path keeps C B^T of every (direction, batch, block, group)
   // in the workspace; shapes it cannot take need only the status word.
@@ -167,6 +169,12 @@ size_t bdscan_workspace_size(const bdscan_shape_t *shape, int op) {
 
 int bdscan_kernel_launches(const bdscan_shape_t *shape, int op) {
   if (check_shape(shape) != BDSCAN_OK) return -1;
+  if (op == BDSCAN_OP_ALLBLOCK_BACKWARD) {
+    // backward kernel + a dB/dC and a dA/dD reduction per present direction
+    // (2 or 4 directions; counted here for all four)
+    if (shape->batch == 0 || shape->seqlen == 0) return 0;
+    return 1 + 2 * 4;
+  }
   if (op != BDSCAN_OP_PREFIX && op != BDSCAN_OP_BLOCK_STEP && op != BDSCAN_OP_ALLBLOCK) return -1;
   if (op == BDSCAN_OP_BLOCK_STEP && shape->seqlen != shape->block_len) return -1;
   if (shape->batch == 0 || shape->seqlen == 0) return 0;
@@ -286,6 +294,92 @@ int bdscan_allblock(const bdscan_shape_t *shape, const bdscan_dir_t *clean_fwd,
   a.ws = ws;
   a.ws_bytes = ws_bytes;
   return launch(a, static_cast<cudaStream_t>(cuda_stream));
+}
+
+int bdscan_allblock_backward(const bdscan_shape_t *shape, const bdscan_dir_t *clean_fwd,
+                             const bdscan_dir_t *clean_rev, const bdscan_dir_t *noisy_fwd,
+                             const bdscan_dir_t *noisy_rev, const float *h0, const float *block_states,
+                             const void *dy_clean, const void *dy_noisy, const float *dstates,
+                             const bdscan_grad_t *g_clean_fwd, const bdscan_grad_t *g_clean_rev,
+                             const bdscan_grad_t *g_noisy_fwd, const bdscan_grad_t *g_noisy_rev,
+                             float *dh0, void *ws, size_t ws_bytes, void *cuda_stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  const Sizes z = sizes_of(shape);
+  if (bdscan::bwd_smem_bytes(shape->headdim, shape->dstate, shape->block_len) > 227u * 1024u)
+    return BDSCAN_ERR_UNSUPPORTED_SHAPE;
+  const bdscan_dir_t *dirs[4] = {clean_fwd, clean_rev, noisy_fwd, noisy_rev};
+  const bdscan_grad_t *grads[4] = {g_clean_fwd, g_clean_rev, g_noisy_fwd, g_noisy_rev};
+  if (!clean_fwd || !noisy_fwd) return BDSCAN_ERR_INVALID_ARG;
+  std::vector<Range> ins, outs;
+  const size_t f32 = 4, B = (size_t)shape->batch, L = (size_t)shape->seqlen, H = (size_t)shape->nheads,
+               P = (size_t)shape->headdim, N = (size_t)shape->dstate, G = (size_t)shape->ngroups;
+  for (int i = 0; i < 4; ++i) {
+    if (!dirs[i]) continue;
+    if ((rc = check_dir(dirs[i], z, ins))) return rc;
+    if (dirs[i]->z) return BDSCAN_ERR_UNSUPPORTED_SHAPE;  // gated backward is not provided
+    const bdscan_grad_t *g = grads[i];
+    if (!g || (z.x && (!g->dx || !g->ddt || !g->dB || !g->dC)) || !g->dA || !g->dD) return BDSCAN_ERR_INVALID_ARG;
+    const void *gp[] = {g->dx, g->ddt, g->dB, g->dC, g->dA, g->dD};
+    for (const void *q : gp)
+      if (q && !aligned16(q)) return BDSCAN_ERR_MISALIGNED;
+    outs.push_back(range_of(g->dx, B * L * H * P * f32));
+    outs.push_back(range_of(g->ddt, B * L * H * f32));
+    outs.push_back(range_of(g->dB, B * L * G * N * f32));
+    outs.push_back(range_of(g->dC, B * L * G * N * f32));
+    outs.push_back(range_of(g->dA, H * f32));
+    outs.push_back(range_of(g->dD, H * f32));
+  }
+  if ((!block_states && z.states) || (!dy_noisy && z.y)) return BDSCAN_ERR_INVALID_ARG;
+  const void *ptrs[] = {h0, block_states, dy_clean, dy_noisy, dstates, dh0};
+  for (const void *q : ptrs)
+    if (q && !aligned16(q)) return BDSCAN_ERR_MISALIGNED;
+  if (h0) ins.push_back(range_of(h0, z.state));
+  ins.push_back(range_of(block_states, z.states));
+  if (dy_clean) ins.push_back(range_of(dy_clean, z.y));
+  ins.push_back(range_of(dy_noisy, z.y));
+  if (dstates) ins.push_back(range_of(dstates, z.states));
+  if (dh0) outs.push_back(range_of(dh0, z.state));
+  if ((rc = check_outputs(ins, outs))) return rc;
+  if ((rc = check_ws(ws, ws_bytes, bdscan_workspace_size(shape, BDSCAN_OP_ALLBLOCK_BACKWARD)))) return rc;
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  if (cudaMemsetAsync(ws, 0, sizeof(int), stream) != cudaSuccess) return BDSCAN_ERR_CUDA;
+  if (shape->batch == 0) return BDSCAN_OK;
+  if (shape->seqlen == 0) {
+    // nothing scanned: all gradients are zero, dh0 = dstates has no blocks
+    for (int i = 0; i < 4; ++i)
+      if (dirs[i] && (cudaMemsetAsync(grads[i]->dA, 0, H * f32, stream) != cudaSuccess ||
+                      cudaMemsetAsync(grads[i]->dD, 0, H * f32, stream) != cudaSuccess))
+        return BDSCAN_ERR_CUDA;
+    if (dh0 && cudaMemsetAsync(dh0, 0, z.state, stream) != cudaSuccess) return BDSCAN_ERR_CUDA;
+    return BDSCAN_OK;
+  }
+  bdscan::BwdArgs a{};
+  a.Bsz = shape->batch; a.L = shape->seqlen; a.H = shape->nheads; a.P = shape->headdim;
+  a.N = shape->dstate; a.G = shape->ngroups; a.T = shape->block_len;
+  a.in_bf16 = shape->in_dtype == BDSCAN_BF16;
+  a.dy_bf16 = shape->out_dtype == BDSCAN_BF16;
+  for (int i = 0; i < 4; ++i) {
+    a.dir[i] = to_args(dirs[i]);
+    if (dirs[i]) {
+      const bdscan_grad_t *g = grads[i];
+      a.grad[i] = bdscan::GradArgs{g->dx, g->ddt, g->dB, g->dC, g->dA, g->dD};
+    }
+  }
+  a.h0 = h0;
+  a.states = block_states;
+  a.dstates = dstates;
+  a.dy_clean = dy_clean;
+  a.dy_noisy = dy_noisy;
+  a.dh0 = dh0;
+  a.ws = static_cast<uint8_t *>(ws) + bdscan::kWsHeader;
+  cudaError_t e = bdscan::launch_bwd(a, stream);
+  if (e != cudaSuccess) {
+    const char *v = std::getenv("BDSCAN_VERBOSE");
+    if (v && v[0] == '1') std::fprintf(stderr, "libbdscan: launch failed: %s\n", cudaGetErrorString(e));
+    return BDSCAN_ERR_CUDA;
+  }
+  return BDSCAN_OK;
 }
 
 int bdscan_check_status(const void *ws, void *cuda_stream) {

@@ -45,4 +45,23 @@ int tc_plan_segments(int64_t Bsz, int64_t H, int64_t K);
 bool tc_supported(const ScanArgs &a);
 cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream);
 
+// Backward of the all-block pass (generic kernel, any accepted ungated shape
+// whose block fits the shared-memory plan).
+struct GradArgs {
+  float *dx, *ddt, *dB, *dC, *dA, *dD;
+};
+struct BwdArgs {
+  int64_t Bsz, L, H, P, N, G, T;
+  bool in_bf16, dy_bf16;
+  DirArgs dir[4];   // clean fwd, clean rev, noisy fwd, noisy rev (x == nullptr: absent)
+  GradArgs grad[4];
+  const float *h0, *states, *dstates;
+  const void *dy_clean, *dy_noisy;
+  float *dh0;
+  void *ws;         // partial sums (bwd_workspace_bytes)
+};
+size_t bwd_smem_bytes(int64_t P, int64_t N, int64_t T);
+size_t bwd_workspace_bytes(int64_t Bsz, int64_t L, int64_t H, int64_t N);
+cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream);
+
 }  // namespace bdscan

@@ -1,0 +1,421 @@
+// scan_bwd.cu -- backward pass of the all-block scan: gradients of a loss
+// L(y_clean, y_noisy, states) with respect to every input of every direction
+// and the initial state.  Through the boundary states the noisy blocks'
+// losses reach the clean prefix scan ("Training Hybrid Block Diffusion
+// Language Models with Partial Bidirectionality", all-block paragraph after
+// eq. (5), eq. (14)).
+//
+// Per 32-token block, in the processing order i = 0..T-1 of one direction
+// (forward: tokens of the block left to right; reverse: right to left), with
+// cum_i = sum_{v <= i} dt_v A, Lam_i = exp(cum_i), W_iu = exp(cum_i - cum_u)
+// (u <= i), the block maps its start state h_s and inputs to
+//   y_i = Lam_i h_s C_i + sum_{u <= i} W_iu dt_u (C_i . B_u) x_u + D x_i
+//   h_e = Lam_{T-1} h_s + sum_u W_{T-1,u} dt_u x_u B_u^T
+// (eq. (1) unrolled over the block).  Given dy_i and dh_e = dL/dh_e:
+//   dx_u = D dy_u + dt_u sum_{i>=u} W_iu (C_i.B_u) dy_i + dt_u W_{T-1,u} dh_e B_u
+//   dC_i = Lam_i dy_i^T h_s + sum_{u<=i} W_iu dt_u (dy_i.x_u) B_u
+//   dB_u = dt_u sum_{i>=u} W_iu (dy_i.x_u) C_i + dt_u W_{T-1,u} x_u^T dh_e
+//   dh_s = Lam_{T-1} dh_e + sum_i Lam_i dy_i C_i^T
+//   dL/dcum_i = Lam_i dy_i.(h_s C_i) + sum_{u<=i} W_iu dt_u (C_i.B_u)(dy_i.x_u)
+//             - sum_{i'>=i} W_i'i dt_i (C_i'.B_i)(dy_i'.x_i)
+//             + [i = T-1] <dh_e, h_e> - dt_i W_{T-1,i} x_i.(dh_e B_i)
+//   ddt_v = (explicit dt_v terms) + A sum_{i>=v} dL/dcum_i,
+//   dA   += sum_v dt_v sum_{i>=v} dL/dcum_i,   dD += sum_i dy_i . x_i.
+// The clean forward stream chains the blocks: dh_e of block k is dL/dstates[k]
+// (given) plus dh_s of clean block k+1 plus dh_s of noisy block k+1 (which
+// starts from states[k]); dh_s of clean block 0 and of noisy block 0 is dh0.
+//
+// One CTA of 256 threads per (b, h) walks the blocks from last to first; all
+// block quantities live in shared memory, fp32 arithmetic on CUDA cores.  dB
+// and dC of a group and dA, dD of a head are sums over heads / batch rows:
+// each CTA writes its own partials to the workspace and a second kernel sums
+// them in a fixed order, so the result is deterministic.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "bdscan_internal.h"
+
+namespace bdscan {
+namespace {
+
+constexpr int kBwdThreads = 256;
+
+struct BwdDir {
+  const void *x, *dt, *B, *C;
+  const float *A, *D;
+  float *dx, *ddt;   // [B][L][H][P], [B][L][H]
+  float *pB, *pC;    // partials [B][L][H][N]
+  float *pA, *pD;    // partials [B][H]
+};
+
+struct BwdParams {
+  BwdDir dir[4];     // clean fwd, clean rev, noisy fwd, noisy rev
+  int active[4];
+  int Bsz, L, H, P, N, G, T, K;
+  int in_bf16, dy_bf16;
+  const float *h0;       // [B][H][P][N] or null
+  const float *states;   // [B][K][H][P][N] (forward output)
+  const void *dy_clean;  // [B][L][H][P] or null
+  const void *dy_noisy;  // [B][L][H][P]
+  const float *dstates;  // [B][K][H][P][N] or null
+  float *dh0;            // [B][H][P][N] or null
+};
+
+__device__ __forceinline__ float ldv(const void *p, int64_t i, int bf16) {
+  return bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i])
+              : reinterpret_cast<const float *>(p)[i];
+}
+
+struct BwdSmem {
+  float *x, *dy, *Bm, *Cm;  // [T][P], [T][P], [T][N], [T][N]
+  float *dt, *cum, *lam;    // [T]
+  float *S, *expl, *red;    // [T], [T], [kBwdThreads]
+  float *CB, *YX, *W;       // [T][T]
+  float *hsC, *dhB;         // [T][P]
+  float *dyh, *xdh;         // [T][N]
+  float *hs, *carry;        // [P][N]
+};
+
+__device__ float block_sum(float v, float *red) {
+  red[threadIdx.x] = v;
+  __syncthreads();
+  for (int s = kBwdThreads / 2; s > 0; s >>= 1) {
+    if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
+    __syncthreads();
+  }
+  const float r = red[0];
+  __syncthreads();
+  return r;
+}
+
+// One block of one direction.  kind: 0 clean fwd (h_s, dh_e = carry, h_e =
+// states[k]; carry <- dh_s), 2 noisy fwd (h_s, no dh_e; carry += dh_s),
+// 1 / 3 reverse (zero start, no dh_e).  Accumulates this CTA's dA, dD.
+__device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b, int h, int k, float &accA,
+                          float &accD) {
+  const BwdDir &d = p.dir[kind];
+  const int T = p.T, P = p.P, N = p.N, H = p.H, L = p.L, G = p.G, K = p.K;
+  const int g = h / (H / G);
+  const int tid = threadIdx.x;
+  const bool rev = kind == 1 || kind == 3;
+  const bool has_hs = !rev && (k > 0 || p.h0 != nullptr);
+  const bool has_dhe = kind == 0;
+  const void *dy = (kind < 2) ? p.dy_clean : p.dy_noisy;
+  const float A = d.A[h], Dh = d.D[h];
+  const int64_t PN = static_cast<int64_t>(P) * N;
+  auto tok = [&](int i) { return k * T + (rev ? T - 1 - i : i); };
+
+  // ---- inputs of the block in processing order
+  for (int e = tid; e < T * P; e += kBwdThreads) {
+    const int i = e / P, pp = e % P;
+    const int64_t xi = ((static_cast<int64_t>(b) * L + tok(i)) * H + h) * P + pp;
+    s.x[e] = ldv(d.x, xi, p.in_bf16);
+    s.dy[e] = dy ? ldv(dy, xi, p.dy_bf16) : 0.f;
+  }
+  for (int e = tid; e < T * N; e += kBwdThreads) {
+    const int i = e / N, n = e % N;
+    const int64_t bi = ((static_cast<int64_t>(b) * L + tok(i)) * G + g) * N + n;
+    s.Bm[e] = ldv(d.B, bi, p.in_bf16);
+    s.Cm[e] = ldv(d.C, bi, p.in_bf16);
+  }
+  for (int i = tid; i < T; i += kBwdThreads)
+    s.dt[i] = ldv(d.dt, (static_cast<int64_t>(b) * L + tok(i)) * H + h, p.in_bf16);
+  if (has_hs) {
+    const float *src = k > 0 ? p.states + ((static_cast<int64_t>(b) * K + (k - 1)) * H + h) * PN
+                             : p.h0 + (static_cast<int64_t>(b) * H + h) * PN;
+    for (int64_t e = tid; e < PN; e += kBwdThreads) s.hs[e] = src[e];
+  }
+  __syncthreads();
+  if (tid == 0) {
+    float c = 0.f;
+    for (int i = 0; i < T; ++i) {
+      c += s.dt[i] * A;
+      s.cum[i] = c;
+      s.lam[i] = expf(c);
+    }
+  }
+  __syncthreads();
+
+  // ---- T x T quantities
+  for (int e = tid; e < T * T; e += kBwdThreads) {
+    const int i = e / T, u = e % T;
+    float cb = 0.f, yx = 0.f;
+    for (int n = 0; n < N; ++n) cb += s.Cm[i * N + n] * s.Bm[u * N + n];
+    for (int q = 0; q < P; ++q) yx += s.dy[i * P + q] * s.x[u * P + q];
+    s.CB[e] = cb;
+    s.YX[e] = yx;
+    s.W[e] = u <= i ? expf(s.cum[i] - s.cum[u]) : 0.f;
+  }
+  // ---- products with the start state and the end-state gradient
+  if (has_hs) {
+    for (int e = tid; e < T * P; e += kBwdThreads) {
+      const int i = e / P, q = e % P;
+      float a = 0.f;
+      for (int n = 0; n < N; ++n) a += s.hs[q * N + n] * s.Cm[i * N + n];
+      s.hsC[e] = a;
+    }
+    for (int e = tid; e < T * N; e += kBwdThreads) {
+      const int i = e / N, n = e % N;
+      float a = 0.f;
+      for (int q = 0; q < P; ++q) a += s.dy[i * P + q] * s.hs[q * N + n];
+      s.dyh[e] = a;
+    }
+  }
+  float he_dot = 0.f;
+  if (has_dhe) {
+    for (int e = tid; e < T * P; e += kBwdThreads) {
+      const int u = e / P, q = e % P;
+      float a = 0.f;
+      for (int n = 0; n < N; ++n) a += s.carry[q * N + n] * s.Bm[u * N + n];
+      s.dhB[e] = a;
+    }
+    for (int e = tid; e < T * N; e += kBwdThreads) {
+      const int u = e / N, n = e % N;
+      float a = 0.f;
+      for (int q = 0; q < P; ++q) a += s.x[u * P + q] * s.carry[q * N + n];
+      s.xdh[e] = a;
+    }
+    const float *he = p.states + ((static_cast<int64_t>(b) * K + k) * H + h) * PN;
+    float part = 0.f;
+    for (int64_t e = tid; e < PN; e += kBwdThreads) part += s.carry[e] * he[e];
+    he_dot = block_sum(part, s.red);
+  }
+  __syncthreads();
+  const float lame = s.lam[T - 1];
+
+  // ---- token gradients
+  for (int e = tid; e < T * P; e += kBwdThreads) {
+    const int u = e / P, q = e % P;
+    float a = 0.f;
+    for (int i = u; i < T; ++i) a += s.W[i * T + u] * s.CB[i * T + u] * s.dy[i * P + q];
+    float v = Dh * s.dy[e] + s.dt[u] * a;
+    if (has_dhe) v += s.dt[u] * (lame / s.lam[u]) * s.dhB[e];
+    d.dx[((static_cast<int64_t>(b) * L + tok(u)) * H + h) * P + q] = v;
+  }
+  for (int e = tid; e < T * N; e += kBwdThreads) {
+    const int i = e / N, n = e % N;
+    float c = has_hs ? s.lam[i] * s.dyh[e] : 0.f;
+    for (int u = 0; u <= i; ++u) c += s.W[i * T + u] * s.dt[u] * s.YX[i * T + u] * s.Bm[u * N + n];
+    // (i as u of the dB formula)
+    float bb = 0.f;
+    for (int i2 = i; i2 < T; ++i2) bb += s.W[i2 * T + i] * s.YX[i2 * T + i] * s.Cm[i2 * N + n];
+    bb *= s.dt[i];
+    if (has_dhe) bb += s.dt[i] * (lame / s.lam[i]) * s.xdh[e];
+    const int64_t o = ((static_cast<int64_t>(b) * L + tok(i)) * H + h) * N + n;
+    d.pC[o] = c;
+    d.pB[o] = bb;
+  }
+  for (int i = tid; i < T; i += kBwdThreads) {
+    float sa = 0.f;
+    if (has_hs)
+      for (int q = 0; q < P; ++q) sa += s.dy[i * P + q] * s.hsC[i * P + q];
+    sa *= s.lam[i];
+    float num = 0.f, den = 0.f, ex = 0.f;
+    for (int u = 0; u <= i; ++u) num += s.W[i * T + u] * s.dt[u] * s.CB[i * T + u] * s.YX[i * T + u];
+    for (int i2 = i; i2 < T; ++i2) {
+      const float m = s.W[i2 * T + i] * s.CB[i2 * T + i] * s.YX[i2 * T + i];
+      den += m;
+      ex += m;
+    }
+    float Si = sa + num - s.dt[i] * den;
+    if (has_dhe) {
+      float xd = 0.f;
+      for (int q = 0; q < P; ++q) xd += s.x[i * P + q] * s.dhB[i * P + q];
+      const float r = lame / s.lam[i];
+      Si -= s.dt[i] * r * xd;
+      ex += r * xd;
+      if (i == T - 1) Si += he_dot;
+    }
+    s.S[i] = Si;
+    s.expl[i] = ex;
+  }
+  __syncthreads();
+  float pa = 0.f, pd = 0.f;
+  if (tid == 0) {
+    float suffix = 0.f;
+    for (int v = T - 1; v >= 0; --v) {
+      suffix += s.S[v];
+      d.ddt[(static_cast<int64_t>(b) * L + tok(v)) * H + h] = s.expl[v] + A * suffix;
+      pa += s.dt[v] * suffix;
+    }
+  }
+  for (int e = tid; e < T * P; e += kBwdThreads) pd += s.dy[e] * s.x[e];
+  pd = block_sum(pd, s.red);
+  if (tid == 0) {
+    accA += pa;
+    accD += pd;
+  }
+  // ---- gradient of the start state
+  if (!rev) {
+    for (int64_t e = tid; e < PN; e += kBwdThreads) {
+      const int q = static_cast<int>(e / N), n = static_cast<int>(e % N);
+      float a = 0.f;
+      for (int i = 0; i < T; ++i) a += s.lam[i] * s.dy[i * P + q] * s.Cm[i * N + n];
+      s.carry[e] = (kind == 0 ? lame * s.carry[e] : s.carry[e]) + a;
+    }
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kBwdThreads) bd_bwd_kernel(const __grid_constant__ BwdParams p) {
+  extern __shared__ float sm[];
+  const int T = p.T, P = p.P, N = p.N, K = p.K, H = p.H;
+  const int64_t PN = static_cast<int64_t>(P) * N;
+  BwdSmem s;
+  float *q = sm;
+  s.x = q; q += T * P;
+  s.dy = q; q += T * P;
+  s.Bm = q; q += T * N;
+  s.Cm = q; q += T * N;
+  s.dt = q; q += T;
+  s.cum = q; q += T;
+  s.lam = q; q += T;
+  s.S = q; q += T;
+  s.expl = q; q += T;
+  s.red = q; q += kBwdThreads;
+  s.CB = q; q += T * T;
+  s.YX = q; q += T * T;
+  s.W = q; q += T * T;
+  s.hsC = q; q += T * P;
+  s.dhB = q; q += T * P;
+  s.dyh = q; q += T * N;
+  s.xdh = q; q += T * N;
+  s.hs = q; q += PN;
+  s.carry = q;
+  const int b = blockIdx.x / H, h = blockIdx.x % H;
+  // carry = dL/dstates[K-1] (given part)
+  for (int64_t e = threadIdx.x; e < PN; e += kBwdThreads)
+    s.carry[e] = p.dstates ? p.dstates[((static_cast<int64_t>(b) * K + (K - 1)) * H + h) * PN + e] : 0.f;
+  __syncthreads();
+  float accA[4] = {0.f, 0.f, 0.f, 0.f}, accD[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int k = K - 1; k >= 0; --k) {
+    bwd_block(p, s, 0, b, h, k, accA[0], accD[0]);
+    bwd_block(p, s, 2, b, h, k, accA[2], accD[2]);
+    if (p.active[1]) bwd_block(p, s, 1, b, h, k, accA[1], accD[1]);
+    if (p.active[3]) bwd_block(p, s, 3, b, h, k, accA[3], accD[3]);
+    if (k > 0 && p.dstates) {
+      for (int64_t e = threadIdx.x; e < PN; e += kBwdThreads)
+        s.carry[e] += p.dstates[((static_cast<int64_t>(b) * K + (k - 1)) * H + h) * PN + e];
+      __syncthreads();
+    }
+  }
+  if (p.dh0)
+    for (int64_t e = threadIdx.x; e < PN; e += kBwdThreads)
+      p.dh0[(static_cast<int64_t>(b) * H + h) * PN + e] = s.carry[e];
+  if (threadIdx.x == 0)
+    for (int di = 0; di < 4; ++di)
+      if (p.active[di]) {
+        p.dir[di].pA[static_cast<int64_t>(b) * H + h] = accA[di];
+        p.dir[di].pD[static_cast<int64_t>(b) * H + h] = accD[di];
+      }
+}
+
+// Fixed-order sums of the partials: dB, dC over the heads of a group, dA, dD
+// over the batch rows.
+__global__ void bd_bwd_reduce_kernel(const float *pB, const float *pC, float *dB, float *dC, int64_t rows,
+                                     int H, int G, int N) {
+  const int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // over rows * G * N
+  if (e >= rows * G * N) return;
+  const int n = static_cast<int>(e % N);
+  const int g = static_cast<int>((e / N) % G);
+  const int64_t r = e / (static_cast<int64_t>(N) * G);  // (b, t)
+  const int hpg = H / G;
+  float sb = 0.f, sc = 0.f;
+  for (int j = 0; j < hpg; ++j) {
+    const int64_t o = (r * H + g * hpg + j) * N + n;
+    sb += pB[o];
+    sc += pC[o];
+  }
+  dB[e] = sb;
+  dC[e] = sc;
+}
+
+__global__ void bd_bwd_reduce_head_kernel(const float *pA, const float *pD, float *dA, float *dD, int Bsz,
+                                          int H) {
+  const int h = blockIdx.x * blockDim.x + threadIdx.x;
+  if (h >= H) return;
+  float sa = 0.f, sd = 0.f;
+  for (int b = 0; b < Bsz; ++b) {
+    sa += pA[static_cast<int64_t>(b) * H + h];
+    sd += pD[static_cast<int64_t>(b) * H + h];
+  }
+  dA[h] = sa;
+  dD[h] = sd;
+}
+
+}  // namespace
+
+size_t bwd_smem_bytes(int64_t P, int64_t N, int64_t T) {
+  const int64_t floats = 2 * T * P + 2 * T * N + 5 * T + kBwdThreads + 3 * T * T + 2 * T * P + 2 * T * N + 2 * P * N;
+  return static_cast<size_t>(floats) * sizeof(float);
+}
+
+size_t bwd_workspace_bytes(int64_t Bsz, int64_t L, int64_t H, int64_t N) {
+  // per direction: dB, dC partials [B][L][H][N] and dA, dD partials [B][H]
+  const size_t per = (2 * static_cast<size_t>(Bsz) * L * H * N + 2 * static_cast<size_t>(Bsz) * H) * sizeof(float);
+  return 4 * ((per + 255) & ~static_cast<size_t>(255));
+}
+
+cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream) {
+  BwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  const int64_t per_floats = 2 * a.Bsz * a.L * a.H * a.N + 2 * a.Bsz * a.H;
+  const size_t per = ((static_cast<size_t>(per_floats) * sizeof(float)) + 255) & ~static_cast<size_t>(255);
+  for (int i = 0; i < 4; ++i) {
+    p.active[i] = a.dir[i].x != nullptr;
+    if (!p.active[i]) continue;
+    BwdDir &d = p.dir[i];
+    d.x = a.dir[i].x;
+    d.dt = a.dir[i].dt;
+    d.B = a.dir[i].B;
+    d.C = a.dir[i].C;
+    d.A = a.dir[i].A;
+    d.D = a.dir[i].D;
+    d.dx = a.grad[i].dx;
+    d.ddt = a.grad[i].ddt;
+    float *base = reinterpret_cast<float *>(static_cast<uint8_t *>(a.ws) + i * per);
+    d.pB = base;
+    d.pC = base + a.Bsz * a.L * a.H * a.N;
+    d.pA = base + 2 * a.Bsz * a.L * a.H * a.N;
+    d.pD = d.pA + a.Bsz * a.H;
+  }
+  p.Bsz = static_cast<int>(a.Bsz);
+  p.L = static_cast<int>(a.L);
+  p.H = static_cast<int>(a.H);
+  p.P = static_cast<int>(a.P);
+  p.N = static_cast<int>(a.N);
+  p.G = static_cast<int>(a.G);
+  p.T = static_cast<int>(a.T);
+  p.K = static_cast<int>(a.L / a.T);
+  p.in_bf16 = a.in_bf16 ? 1 : 0;
+  p.dy_bf16 = a.dy_bf16 ? 1 : 0;
+  p.h0 = a.h0;
+  p.states = a.states;
+  p.dy_clean = a.dy_clean;
+  p.dy_noisy = a.dy_noisy;
+  p.dstates = a.dstates;
+  p.dh0 = a.dh0;
+  const size_t smem = bwd_smem_bytes(a.P, a.N, a.T);
+  cudaError_t e = cudaFuncSetAttribute(bd_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  bd_bwd_kernel<<<static_cast<unsigned>(a.Bsz * a.H), kBwdThreads, smem, stream>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int64_t rows = a.Bsz * a.L;
+  const int64_t cnt = rows * a.G * a.N;
+  for (int i = 0; i < 4; ++i) {
+    if (!p.active[i]) continue;
+    const BwdDir &d = p.dir[i];
+    bd_bwd_reduce_kernel<<<static_cast<unsigned>((cnt + 255) / 256), 256, 0, stream>>>(
+        d.pB, d.pC, a.grad[i].dB, a.grad[i].dC, rows, p.H, p.G, p.N);
+    bd_bwd_reduce_head_kernel<<<static_cast<unsigned>((a.H + 127) / 128), 128, 0, stream>>>(
+        d.pA, d.pD, a.grad[i].dA, a.grad[i].dD, p.Bsz, p.H);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace bdscan

@@ -548,7 +548,8 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
 // Descriptors are built once; per step only their start addresses move.
 __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
   const uint32_t id_s = idesc_bf16(128, 64, 1, 1);  // S^T[n][p] = B^T (w o X)
-  const uint32_t id_yo = idesc_bf16(64, 64, 1, 0);  // Y_off^T[p][t] = h C^T
+  // Y_off^T[p][t] = h C^T over the stacked [C_cf; C_nf] rows (only C_cf without a noisy stream)
+  const uint32_t id_yo = p.allblock ? idesc_bf16(64, 64, 1, 0) : idesc_bf16(64, 32, 1, 0);
   const uint32_t id_yd = idesc_bf16(64, 32, 1, 1);  // Y_diag^T[p][t] = X^T M^T, one stream
   const uint32_t id_dx = idesc_bf16(64, 16, 1, 0);  // (D x)^T[p][t] = X^T (D I_16)
   // descriptor of each operand at its first tile; moving an operand by b bytes adds b >> 4
@@ -1097,17 +1098,9 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
     *reinterpret_cast<int **>(sm + kOffMisc + 16) = p.status;
     fence_mbar_init();
   }
-  // Without a noisy stream, Y_off still reads the noisy half of the stacked C
-  // operand: clear it so that no uninitialised NaN/Inf bit pattern is ever
-  // multiplied.  Clear the D I_16 buffers (only their diagonals are written).
+  // Clear the D I_16 buffers (only their diagonals are written).
   if (!p.agg) {
     const uint4 zero = make_uint4(0, 0, 0, 0);
-    if (!p.allblock)
-      for (int r = 0; r < kSlots; ++r)
-        for (uint32_t o = threadIdx.x * 16; o < kTile; o += kThreads * 16) {
-          *reinterpret_cast<uint4 *>(sm + r * kSlot + kOffClo + kTile + o) = zero;
-          *reinterpret_cast<uint4 *>(sm + r * kSlot + kOffChi + kTile + o) = zero;
-        }
     for (uint32_t o = threadIdx.x * 16; o < 2 * kDgBuf; o += kThreads * 16)
       *reinterpret_cast<uint4 *>(sm + kOffDg + o) = zero;
     fence_proxy_async_smem();

@@ -65,6 +65,7 @@ extern "C" {
 #define BDSCAN_OP_PREFIX 0
 #define BDSCAN_OP_BLOCK_STEP 1
 #define BDSCAN_OP_ALLBLOCK 2
+#define BDSCAN_OP_ALLBLOCK_BACKWARD 3
 
 /* Problem shape.  Supported: batch >= 0, seqlen >= 0, seqlen % block_len == 0,
  * 1 <= block_len <= 32 or block_len % 32 == 0 (<= 256), chunk_len % block_len
@@ -128,6 +129,44 @@ int bdscan_allblock(const bdscan_shape_t *shape, const bdscan_dir_t *clean_fwd,
                     const bdscan_dir_t *clean_rev, const bdscan_dir_t *noisy_fwd,
                     const bdscan_dir_t *noisy_rev, const float *h0, void *y_clean, void *y_noisy,
                     float *block_states, void *ws, size_t ws_bytes, void *cuda_stream);
+
+/* Gradients of one direction (fp32, overwritten): dx [B][L][H][P],
+ * ddt [B][L][H], dB and dC [B][L][G][N] (summed over the heads of a group),
+ * dA and dD [H] (summed over batch rows and tokens). */
+typedef struct {
+    float *dx, *ddt, *dB, *dC, *dA, *dD;
+} bdscan_grad_t;
+
+/* bdscan_allblock_backward -- reverse-mode derivative of bdscan_allblock for
+ * training: given dL/dy_clean, dL/dy_noisy and dL/dstates of a loss
+ * L(y_clean, y_noisy, block_states), the gradients of every input.  The
+ * all-block objective makes the noisy blocks' losses reach the clean prefix
+ * scan through the boundary states ("Training Hybrid Block Diffusion Language
+ * Models with Partial Bidirectionality", all-block paragraph after eq. (5),
+ * eq. (14)); the derivative itself is that of eq. (1) over eqs. (10)-(13).
+ *   directions    as for bdscan_allblock (ungated only: a direction with z
+ *                 gives BDSCAN_ERR_UNSUPPORTED_SHAPE)
+ *   h0            [B][H][P][N] or NULL (zeros), as in the forward call
+ *   block_states  [B][K][H][P][N]: the forward call's output (required)
+ *   dy_clean      [B][L][H][P] of out_dtype, or NULL (no loss on y_clean)
+ *   dy_noisy      [B][L][H][P] of out_dtype (required)
+ *   dstates       [B][K][H][P][N] fp32 or NULL (no loss on the states)
+ *   g_*           gradient outputs per direction (required for the present
+ *                 directions; pointers of the absent ones are ignored)
+ *   dh0           [B][H][P][N] or NULL
+ *   ws, ws_bytes  at least bdscan_workspace_size(shape, ALLBLOCK_BACKWARD)
+ *                 bytes (per-head / per-row partial sums, reduced in a fixed
+ *                 order: the result is deterministic)
+ * Shapes: as for the forward; additionally the per-block shared-memory plan
+ * (P, N, block_len) must fit one CTA (P = 64, N = 128, block_len = 32 does).
+ * Gradients must not overlap any input or each other. */
+int bdscan_allblock_backward(const bdscan_shape_t *shape, const bdscan_dir_t *clean_fwd,
+                             const bdscan_dir_t *clean_rev, const bdscan_dir_t *noisy_fwd,
+                             const bdscan_dir_t *noisy_rev, const float *h0, const float *block_states,
+                             const void *dy_clean, const void *dy_noisy, const float *dstates,
+                             const bdscan_grad_t *g_clean_fwd, const bdscan_grad_t *g_clean_rev,
+                             const bdscan_grad_t *g_noisy_fwd, const bdscan_grad_t *g_noisy_rev,
+                             float *dh0, void *ws, size_t ws_bytes, void *cuda_stream);
 
 /* Workspace bytes an operation needs for this shape (>= 256: the first 256
  * bytes hold the device status word).  Returns 0 for an invalid shape/op. */

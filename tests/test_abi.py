@@ -154,3 +154,42 @@ def test_allblock_requires_outputs():
     rc = bd.bdscan_allblock(ctypes.byref(s), ctypes.byref(cf), None, None, None, None,
                             None, 0x90000000, 0x98000000, 0xA0000000, 1 << 20, None)
     assert rc == -1   # noisy_fwd missing
+
+
+def _fake_grad(base, step=0x100000):
+    p = [base + i * step for i in range(6)]
+    return bd.bdscan_grad_t(*p)
+
+
+def _backward(s_kw=None, gated=False, states=0x70000000, dyn=0x71000000, g_cf=None, g_nf=None,
+              ws=0xA0000000, ws_bytes=None):
+    s = bd.c_shape(Shape(**_base(**(s_kw or {}))))
+    cf, nf = _fake_dir(0x10000000), _fake_dir(0x20000000)
+    if gated:
+        cf.z = 0x30000000
+    g_cf = _fake_grad(0x40000000) if g_cf is None else g_cf
+    g_nf = _fake_grad(0x50000000) if g_nf is None else g_nf
+    if ws_bytes is None:
+        ws_bytes = bd.bdscan_workspace_size(ctypes.byref(s), bd.BDSCAN_OP_ALLBLOCK_BACKWARD)
+    return bd.bdscan_allblock_backward(ctypes.byref(s), ctypes.byref(cf), None, ctypes.byref(nf), None, None,
+                                       states, None, dyn, None, ctypes.byref(g_cf), None,
+                                       ctypes.byref(g_nf) if g_nf != "null" else None, None, None, ws,
+                                       ws_bytes, None)
+
+
+def test_backward_validation():
+    s = bd.c_shape(Shape(**_base()))
+    assert bd.bdscan_workspace_size(ctypes.byref(s), bd.BDSCAN_OP_ALLBLOCK_BACKWARD) > 1024
+    assert _backward(gated=True) == -2            # the backward is ungated only
+    assert _backward(states=None) == -1           # forward states required
+    assert _backward(dyn=None) == -1              # dy_noisy required
+    assert _backward(g_nf="null") == -1           # gradients of a present direction required
+    g = _fake_grad(0x40000000)
+    g.dx = g.dx + 4
+    assert _backward(g_cf=g) == -3                # misaligned gradient
+    g = _fake_grad(0x40000000)
+    g.dx = 0x10000000                             # gradient over an input
+    assert _backward(g_cf=g) == -1
+    assert _backward(ws_bytes=64) == -4           # workspace too small
+    # a block whose shared-memory plan does not fit one CTA
+    assert _backward(s_kw=dict(headdim=128, dstate=256, block_len=64, chunk_len=64, seqlen=128)) == -2
