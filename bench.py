@@ -391,8 +391,17 @@ def _backward(s: W.Shape, dev, pk) -> dict:
     grads, dh0 = bd.allblock_backward(s, cf, cr, nf, nr, st, dyn, dy_clean=dyc, ws=ws)
     ms = _time(lambda: bd.allblock_backward(s, cf, cr, nf, nr, st, dyn, dy_clean=dyc, grads=grads, ws=ws),
                dev, 5)
+    flops = RL.allblock_backward_flops(s)
+    bytes_ = RL.allblock_backward_bytes(s)
+    # fp32 CUDA-core peak: 148 SMs x 128 FMA lanes x 2 flops x the max SM clock
+    alu_peak = 148 * 128 * 2 * pk["sm_max_mhz"] * 1e6 / 1e12
+    tf = flops / (ms * 1e-3) / 1e12
     return {"us_per_call": ms * 1e3, "tokens_per_s": s.batch * s.seqlen / (ms * 1e-3),
-            "kernel": "generic CUDA-core backward (per-block adjoint in shared memory)"}
+            "kernel": "generic CUDA-core backward (per-block adjoint in shared memory)",
+            "roofline": {"bound": "alu", "achieved": tf, "peak": alu_peak, "unit": "TFLOP/s",
+                         "frac": tf / alu_peak, "algorithmic_flops": flops,
+                         "algorithmic_bytes": bytes_,
+                         "hbm_frac": bytes_ / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}}
 
 
 def _prefill(s: W.Shape, dev, pk) -> dict:

@@ -71,6 +71,8 @@ __device__ __forceinline__ float ldv(const void *p, int64_t i, int bf16) {
 
 struct BwdSmem {
   float *x, *dy, *Bm, *Cm;  // [T][P], [T][P], [T][N], [T][N]
+  float *xt, *Bt, *Ct;      // transposed copies [P][T], [N][T], [N][T] (conflict-free
+                            // shared-memory reads when the lanes run over tokens)
   float *dt, *cum, *lam;    // [T]
   float *S, *expl, *red;    // [T], [T], [kBwdThreads]
   float *CB, *YX, *W;       // [T][T]
@@ -121,6 +123,16 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
     s.Bm[e] = ldv(d.B, bi, p.in_bf16);
     s.Cm[e] = ldv(d.C, bi, p.in_bf16);
   }
+  for (int e = tid; e < T * P; e += kBwdThreads) {
+    const int pp = e / T, i = e % T;
+    s.xt[e] = ldv(d.x, ((static_cast<int64_t>(b) * L + tok(i)) * H + h) * P + pp, p.in_bf16);
+  }
+  for (int e = tid; e < T * N; e += kBwdThreads) {
+    const int n = e / T, i = e % T;
+    const int64_t bi = ((static_cast<int64_t>(b) * L + tok(i)) * G + g) * N + n;
+    s.Bt[e] = ldv(d.B, bi, p.in_bf16);
+    s.Ct[e] = ldv(d.C, bi, p.in_bf16);
+  }
   for (int i = tid; i < T; i += kBwdThreads)
     s.dt[i] = ldv(d.dt, (static_cast<int64_t>(b) * L + tok(i)) * H + h, p.in_bf16);
   if (has_hs) {
@@ -143,8 +155,8 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
   for (int e = tid; e < T * T; e += kBwdThreads) {
     const int i = e / T, u = e % T;
     float cb = 0.f, yx = 0.f;
-    for (int n = 0; n < N; ++n) cb += s.Cm[i * N + n] * s.Bm[u * N + n];
-    for (int q = 0; q < P; ++q) yx += s.dy[i * P + q] * s.x[u * P + q];
+    for (int n = 0; n < N; ++n) cb += s.Cm[i * N + n] * s.Bt[n * T + u];
+    for (int q = 0; q < P; ++q) yx += s.dy[i * P + q] * s.xt[q * T + u];
     s.CB[e] = cb;
     s.YX[e] = yx;
     s.W[e] = u <= i ? expf(s.cum[i] - s.cum[u]) : 0.f;
@@ -152,10 +164,10 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
   // ---- products with the start state and the end-state gradient
   if (has_hs) {
     for (int e = tid; e < T * P; e += kBwdThreads) {
-      const int i = e / P, q = e % P;
+      const int q = e / T, i = e % T;
       float a = 0.f;
-      for (int n = 0; n < N; ++n) a += s.hs[q * N + n] * s.Cm[i * N + n];
-      s.hsC[e] = a;
+      for (int n = 0; n < N; ++n) a += s.hs[q * N + n] * s.Ct[n * T + i];
+      s.hsC[i * P + q] = a;
     }
     for (int e = tid; e < T * N; e += kBwdThreads) {
       const int i = e / N, n = e % N;
@@ -167,10 +179,10 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
   float he_dot = 0.f;
   if (has_dhe) {
     for (int e = tid; e < T * P; e += kBwdThreads) {
-      const int u = e / P, q = e % P;
+      const int q = e / T, u = e % T;
       float a = 0.f;
-      for (int n = 0; n < N; ++n) a += s.carry[q * N + n] * s.Bm[u * N + n];
-      s.dhB[e] = a;
+      for (int n = 0; n < N; ++n) a += s.carry[q * N + n] * s.Bt[n * T + u];
+      s.dhB[u * P + q] = a;
     }
     for (int e = tid; e < T * N; e += kBwdThreads) {
       const int u = e / N, n = e % N;
@@ -270,6 +282,9 @@ __global__ void __launch_bounds__(kBwdThreads) bd_bwd_kernel(const __grid_consta
   s.dy = q; q += T * P;
   s.Bm = q; q += T * N;
   s.Cm = q; q += T * N;
+  s.xt = q; q += T * P;
+  s.Bt = q; q += T * N;
+  s.Ct = q; q += T * N;
   s.dt = q; q += T;
   s.cum = q; q += T;
   s.lam = q; q += T;
@@ -349,7 +364,7 @@ __global__ void bd_bwd_reduce_head_kernel(const float *pA, const float *pD, floa
 }  // namespace
 
 size_t bwd_smem_bytes(int64_t P, int64_t N, int64_t T) {
-  const int64_t floats = 2 * T * P + 2 * T * N + 5 * T + kBwdThreads + 3 * T * T + 2 * T * P + 2 * T * N + 2 * P * N;
+  const int64_t floats = 3 * T * P + 4 * T * N + 5 * T + kBwdThreads + 3 * T * T + 2 * T * P + 2 * T * N + 2 * P * N;
   return static_cast<size_t>(floats) * sizeof(float);
 }
 

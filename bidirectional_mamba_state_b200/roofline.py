@@ -63,3 +63,25 @@ def prefix_flops(s: Shape, with_rev: bool = True) -> int:
     nd = 2 if with_rev else 1
     per_bhk = 2 * T * P * N + 2 * T * N * P + nd * 2 * T * T * P
     return B * K * (H * per_bhk + G * nd * 2 * T * T * N)
+
+
+def allblock_backward_bytes(s: Shape, with_dy_clean: bool = True, with_dstates: bool = False) -> int:
+    """Inputs of the four directions, dy (output dtype), the forward's boundary
+    states, (dstates), and fp32 gradients of every input plus dh0."""
+    B, L, H, P, N, G = s.batch, s.seqlen, s.nheads, s.headdim, s.dstate, s.ngroups
+    grads = 4 * (4 * B * L * H * P + 4 * B * L * H + 2 * 4 * B * L * G * N + 8 * H)
+    return 4 * dir_bytes(s) + (2 if with_dy_clean else 1) * y_bytes(s) + \
+        s.nblocks * state_bytes(s) * (2 if with_dstates else 1) + grads + state_bytes(s)
+
+
+def allblock_backward_flops(s: Shape) -> int:
+    """Flops of the per-block closed-form derivative (per (b, h, block)):
+    Gram matrices C B^T and dy x^T of every direction, the products with the
+    start state (forward directions) and with the end-state gradient (clean
+    forward), the intra-block sums for dx, dB, dC and the start-state gradient."""
+    B, H, P, N, T, K = s.batch, s.nheads, s.headdim, s.dstate, s.block_len, s.nblocks
+    gram = 2 * T * T * (N + P)              # C B^T and dy x^T
+    intra = 2 * T * T * (P + 2 * N) // 2    # dx, dC, dB sums over the causal triangle
+    tpn = 2 * T * P * N
+    per = (gram + intra + 5 * tpn) + (gram + intra + 3 * tpn) + 2 * (gram + intra)
+    return B * H * K * per
