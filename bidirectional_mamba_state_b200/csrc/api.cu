@@ -306,7 +306,10 @@ int bdscan_allblock_backward(const bdscan_shape_t *shape, const bdscan_dir_t *cl
   int rc = check_shape(shape);
   if (rc) return rc;
   const Sizes z = sizes_of(shape);
-  if (bdscan::bwd_smem_bytes(shape->headdim, shape->dstate, shape->block_len) > 227u * 1024u)
+  // the backward's shared-memory plan: 16-byte rows (block_len and d_state
+  // multiples of 4) that fit one CTA
+  if (shape->block_len % 4 || shape->dstate % 4 ||
+      bdscan::bwd_smem_bytes(shape->headdim, shape->dstate, shape->block_len) > 227u * 1024u)
     return BDSCAN_ERR_UNSUPPORTED_SHAPE;
   const bdscan_dir_t *dirs[4] = {clean_fwd, clean_rev, noisy_fwd, noisy_rev};
   const bdscan_grad_t *grads[4] = {g_clean_fwd, g_clean_rev, g_noisy_fwd, g_noisy_rev};

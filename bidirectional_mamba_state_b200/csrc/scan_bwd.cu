@@ -26,7 +26,9 @@
 // starts from states[k]); dh_s of clean block 0 and of noisy block 0 is dh0.
 //
 // One CTA of 256 threads per (b, h) walks the blocks from last to first; all
-// block quantities live in shared memory, fp32 arithmetic on CUDA cores.  dB
+// block quantities live in shared memory (with transposed copies where the
+// threads run over tokens), the products are register-tiled (4 x 4 per
+// thread), fp32 arithmetic on CUDA cores.  dB
 // and dC of a group and dA, dD of a head are sums over heads / batch rows:
 // each CTA writes its own partials to the workspace and a second kernel sums
 // them in a fixed order, so the result is deterministic.
@@ -70,14 +72,14 @@ __device__ __forceinline__ float ldv(const void *p, int64_t i, int bf16) {
 }
 
 struct BwdSmem {
-  float *x, *dy, *Bm, *Cm;  // [T][P], [T][P], [T][N], [T][N]
-  float *xt, *Bt, *Ct;      // transposed copies [P][T], [N][T], [N][T] (conflict-free
-                            // shared-memory reads when the lanes run over tokens)
-  float *dt, *cum, *lam;    // [T]
+  float *x, *dy, *Bm, *Cm;  // row-major [T][P], [T][P], [T][N], [T][N]
+  float *xt, *dyt;          // transposed [P][T]
+  float *Bt, *Ct;           // transposed [N][T]
+  float *dt, *cum, *lam, *r;  // [T]; r_u = Lam_{T-1} / Lam_u
   float *S, *expl, *red;    // [T], [T], [kBwdThreads]
-  float *CB, *YX, *W;       // [T][T]
-  float *hsC, *dhB;         // [T][P]
-  float *dyh, *xdh;         // [T][N]
+  float *WCB, *YX, *G2;     // [T][T]: W o (C B^T), dy x^T, W o (dy x^T)
+  float *Q;                 // [T][T + 1]: W o (C B^T) o (dy x^T), padded rows
+  float *hsCt, *dhBt;       // [P][T]: (h_s C^T)^T, (dh_e B^T)^T
   float *hs, *carry;        // [P][N]
 };
 
@@ -91,6 +93,57 @@ __device__ float block_sum(float v, float *red) {
   const float r = red[0];
   __syncthreads();
   return r;
+}
+
+// Register-tiled product over shared-memory operands: for every 4 x 4 output
+// tile (m0.., n0..) of an M x Nn result,
+//   acc[i][j] = sum_k a1(m0+i, k) B1[k][n0+j]  (+ sum_k a2(m0+i, k) B2[k][n0+j])
+// with a(m, k) = A[m am + k ak] (times ks1[k], resp. ms2[m], when given) and
+// B rows contiguous in n (16-byte loads).  A threads of a warp share m0, so A
+// loads are broadcasts.  epi(m0, n0, acc) consumes the tile.
+template <class Epi>
+__device__ __forceinline__ void sgemm(int M, int Nn, int K1, const float *A1, int am1, int ak1, const float *ks1,
+                                      const float *B1, int ldb1, int K2, const float *A2, int am2, int ak2,
+                                      const float *ms2, const float *B2, int ldb2, Epi epi) {
+  const int nt = Nn >> 2;
+  const int tiles = (M >> 2) * nt;
+  for (int t = threadIdx.x; t < tiles; t += kBwdThreads) {
+    const int m0 = (t / nt) << 2, n0 = (t % nt) << 2;
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    for (int k = 0; k < K1; ++k) {
+      const float4 bv = *reinterpret_cast<const float4 *>(B1 + k * ldb1 + n0);
+      const float sk = ks1 ? ks1[k] : 1.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float a = A1[(m0 + i) * am1 + k * ak1] * sk;
+        acc[i][0] = fmaf(a, bv.x, acc[i][0]);
+        acc[i][1] = fmaf(a, bv.y, acc[i][1]);
+        acc[i][2] = fmaf(a, bv.z, acc[i][2]);
+        acc[i][3] = fmaf(a, bv.w, acc[i][3]);
+      }
+    }
+    if (A2) {
+      float sm2[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) sm2[i] = ms2 ? ms2[m0 + i] : 1.f;
+      for (int k = 0; k < K2; ++k) {
+        const float4 bv = *reinterpret_cast<const float4 *>(B2 + k * ldb2 + n0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float a = A2[(m0 + i) * am2 + k * ak2] * sm2[i];
+          acc[i][0] = fmaf(a, bv.x, acc[i][0]);
+          acc[i][1] = fmaf(a, bv.y, acc[i][1]);
+          acc[i][2] = fmaf(a, bv.z, acc[i][2]);
+          acc[i][3] = fmaf(a, bv.w, acc[i][3]);
+        }
+      }
+    }
+    epi(m0, n0, acc);
+  }
 }
 
 // One block of one direction.  kind: 0 clean fwd (h_s, dh_e = carry, h_e =
@@ -109,8 +162,9 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
   const float A = d.A[h], Dh = d.D[h];
   const int64_t PN = static_cast<int64_t>(P) * N;
   auto tok = [&](int i) { return k * T + (rev ? T - 1 - i : i); };
+  const float *nul = nullptr;
 
-  // ---- inputs of the block in processing order
+  // ---- inputs of the block in processing order (row-major and transposed copies)
   for (int e = tid; e < T * P; e += kBwdThreads) {
     const int i = e / P, pp = e % P;
     const int64_t xi = ((static_cast<int64_t>(b) * L + tok(i)) * H + h) * P + pp;
@@ -123,16 +177,6 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
     s.Bm[e] = ldv(d.B, bi, p.in_bf16);
     s.Cm[e] = ldv(d.C, bi, p.in_bf16);
   }
-  for (int e = tid; e < T * P; e += kBwdThreads) {
-    const int pp = e / T, i = e % T;
-    s.xt[e] = ldv(d.x, ((static_cast<int64_t>(b) * L + tok(i)) * H + h) * P + pp, p.in_bf16);
-  }
-  for (int e = tid; e < T * N; e += kBwdThreads) {
-    const int n = e / T, i = e % T;
-    const int64_t bi = ((static_cast<int64_t>(b) * L + tok(i)) * G + g) * N + n;
-    s.Bt[e] = ldv(d.B, bi, p.in_bf16);
-    s.Ct[e] = ldv(d.C, bi, p.in_bf16);
-  }
   for (int i = tid; i < T; i += kBwdThreads)
     s.dt[i] = ldv(d.dt, (static_cast<int64_t>(b) * L + tok(i)) * H + h, p.in_bf16);
   if (has_hs) {
@@ -141,6 +185,16 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
     for (int64_t e = tid; e < PN; e += kBwdThreads) s.hs[e] = src[e];
   }
   __syncthreads();
+  for (int e = tid; e < T * P; e += kBwdThreads) {
+    const int pp = e / T, i = e % T;
+    s.xt[e] = s.x[i * P + pp];
+    s.dyt[e] = s.dy[i * P + pp];
+  }
+  for (int e = tid; e < T * N; e += kBwdThreads) {
+    const int n = e / T, i = e % T;
+    s.Bt[e] = s.Bm[i * N + n];
+    s.Ct[e] = s.Cm[i * N + n];
+  }
   if (tid == 0) {
     float c = 0.f;
     for (int i = 0; i < T; ++i) {
@@ -148,97 +202,101 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
       s.cum[i] = c;
       s.lam[i] = expf(c);
     }
+    for (int i = 0; i < T; ++i) s.r[i] = expf(c - s.cum[i]);
   }
   __syncthreads();
 
-  // ---- T x T quantities
-  for (int e = tid; e < T * T; e += kBwdThreads) {
-    const int i = e / T, u = e % T;
-    float cb = 0.f, yx = 0.f;
-    for (int n = 0; n < N; ++n) cb += s.Cm[i * N + n] * s.Bt[n * T + u];
-    for (int q = 0; q < P; ++q) yx += s.dy[i * P + q] * s.xt[q * T + u];
-    s.CB[e] = cb;
-    s.YX[e] = yx;
-    s.W[e] = u <= i ? expf(s.cum[i] - s.cum[u]) : 0.f;
-  }
+  // ---- Gram matrices: C B^T and dy x^T
+  sgemm(T, T, N, s.Cm, N, 1, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+        [&](int m0, int n0, float (&acc)[4][4]) {
+          for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4 *>(s.WCB + (m0 + i) * T + n0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+        });
+  sgemm(T, T, P, s.dy, P, 1, nul, s.xt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+        [&](int m0, int n0, float (&acc)[4][4]) {
+          for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4 *>(s.YX + (m0 + i) * T + n0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+        });
   // ---- products with the start state and the end-state gradient
-  if (has_hs) {
-    for (int e = tid; e < T * P; e += kBwdThreads) {
-      const int q = e / T, i = e % T;
-      float a = 0.f;
-      for (int n = 0; n < N; ++n) a += s.hs[q * N + n] * s.Ct[n * T + i];
-      s.hsC[i * P + q] = a;
-    }
-    for (int e = tid; e < T * N; e += kBwdThreads) {
-      const int i = e / N, n = e % N;
-      float a = 0.f;
-      for (int q = 0; q < P; ++q) a += s.dy[i * P + q] * s.hs[q * N + n];
-      s.dyh[e] = a;
-    }
-  }
+  if (has_hs)
+    sgemm(P, T, N, s.hs, N, 1, nul, s.Ct, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+          [&](int m0, int n0, float (&acc)[4][4]) {
+            for (int i = 0; i < 4; ++i)
+              *reinterpret_cast<float4 *>(s.hsCt + (m0 + i) * T + n0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+          });
+  if (has_dhe)
+    sgemm(P, T, N, s.carry, N, 1, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+          [&](int m0, int n0, float (&acc)[4][4]) {
+            for (int i = 0; i < 4; ++i)
+              *reinterpret_cast<float4 *>(s.dhBt + (m0 + i) * T + n0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+          });
   float he_dot = 0.f;
   if (has_dhe) {
-    for (int e = tid; e < T * P; e += kBwdThreads) {
-      const int q = e / T, u = e % T;
-      float a = 0.f;
-      for (int n = 0; n < N; ++n) a += s.carry[q * N + n] * s.Bt[n * T + u];
-      s.dhB[u * P + q] = a;
-    }
-    for (int e = tid; e < T * N; e += kBwdThreads) {
-      const int u = e / N, n = e % N;
-      float a = 0.f;
-      for (int q = 0; q < P; ++q) a += s.x[u * P + q] * s.carry[q * N + n];
-      s.xdh[e] = a;
-    }
     const float *he = p.states + ((static_cast<int64_t>(b) * K + k) * H + h) * PN;
     float part = 0.f;
     for (int64_t e = tid; e < PN; e += kBwdThreads) part += s.carry[e] * he[e];
     he_dot = block_sum(part, s.red);
   }
   __syncthreads();
+  // ---- decay-weighted matrices (W_iu = exp(cum_i - cum_u), u <= i)
+  for (int e = tid; e < T * T; e += kBwdThreads) {
+    const int i = e / T, u = e % T;
+    const float w = u <= i ? expf(s.cum[i] - s.cum[u]) : 0.f;
+    const float cb = s.WCB[e], yx = s.YX[e];
+    s.WCB[e] = w * cb;
+    s.G2[e] = w * yx;
+    s.Q[i * (T + 1) + u] = w * cb * yx;
+  }
+  __syncthreads();
   const float lame = s.lam[T - 1];
 
   // ---- token gradients
-  for (int e = tid; e < T * P; e += kBwdThreads) {
-    const int u = e / P, q = e % P;
-    float a = 0.f;
-    for (int i = u; i < T; ++i) a += s.W[i * T + u] * s.CB[i * T + u] * s.dy[i * P + q];
-    float v = Dh * s.dy[e] + s.dt[u] * a;
-    if (has_dhe) v += s.dt[u] * (lame / s.lam[u]) * s.dhB[e];
-    d.dx[((static_cast<int64_t>(b) * L + tok(u)) * H + h) * P + q] = v;
-  }
-  for (int e = tid; e < T * N; e += kBwdThreads) {
-    const int i = e / N, n = e % N;
-    float c = has_hs ? s.lam[i] * s.dyh[e] : 0.f;
-    for (int u = 0; u <= i; ++u) c += s.W[i * T + u] * s.dt[u] * s.YX[i * T + u] * s.Bm[u * N + n];
-    // (i as u of the dB formula)
-    float bb = 0.f;
-    for (int i2 = i; i2 < T; ++i2) bb += s.W[i2 * T + i] * s.YX[i2 * T + i] * s.Cm[i2 * N + n];
-    bb *= s.dt[i];
-    if (has_dhe) bb += s.dt[i] * (lame / s.lam[i]) * s.xdh[e];
-    const int64_t o = ((static_cast<int64_t>(b) * L + tok(i)) * H + h) * N + n;
-    d.pC[o] = c;
-    d.pB[o] = bb;
-  }
+  // dx_u = D dy_u + dt_u sum_i WCB[i][u] dy_i (+ dt_u r_u dh_e B_u)
+  sgemm(T, P, T, s.WCB, 1, T, nul, s.dy, P, 0, nullptr, 0, 0, nul, nullptr, 0,
+        [&](int m0, int n0, float (&acc)[4][4]) {
+          for (int i = 0; i < 4; ++i) {
+            const int u = m0 + i;
+            float v[4];
+            for (int j = 0; j < 4; ++j) {
+              v[j] = Dh * s.dy[u * P + n0 + j] + s.dt[u] * acc[i][j];
+              if (has_dhe) v[j] += s.dt[u] * s.r[u] * s.dhBt[(n0 + j) * T + u];
+            }
+            *reinterpret_cast<float4 *>(d.dx + ((static_cast<int64_t>(b) * L + tok(u)) * H + h) * P + n0) =
+                make_float4(v[0], v[1], v[2], v[3]);
+          }
+        });
+  // dC_i = sum_u G2[i][u] dt_u B_u (+ Lam_i dy_i^T h_s)
+  sgemm(T, N, T, s.G2, T, 1, s.dt, s.Bm, N, has_hs ? P : 0, has_hs ? s.dy : nullptr, P, 1, s.lam, s.hs, N,
+        [&](int m0, int n0, float (&acc)[4][4]) {
+          for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4 *>(d.pC + ((static_cast<int64_t>(b) * L + tok(m0 + i)) * H + h) * N + n0) =
+                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+        });
+  // dB_u = dt_u (sum_i G2[i][u] C_i (+ r_u x_u^T dh_e))
+  sgemm(T, N, T, s.G2, 1, T, nul, s.Cm, N, has_dhe ? P : 0, has_dhe ? s.x : nullptr, P, 1, s.r, s.carry, N,
+        [&](int m0, int n0, float (&acc)[4][4]) {
+          for (int i = 0; i < 4; ++i) {
+            const float du = s.dt[m0 + i];
+            *reinterpret_cast<float4 *>(d.pB + ((static_cast<int64_t>(b) * L + tok(m0 + i)) * H + h) * N + n0) =
+                make_float4(du * acc[i][0], du * acc[i][1], du * acc[i][2], du * acc[i][3]);
+          }
+        });
+  // dL/dcum and the explicit dt terms
   for (int i = tid; i < T; i += kBwdThreads) {
     float sa = 0.f;
     if (has_hs)
-      for (int q = 0; q < P; ++q) sa += s.dy[i * P + q] * s.hsC[i * P + q];
+      for (int q = 0; q < P; ++q) sa += s.dyt[q * T + i] * s.hsCt[q * T + i];
     sa *= s.lam[i];
-    float num = 0.f, den = 0.f, ex = 0.f;
-    for (int u = 0; u <= i; ++u) num += s.W[i * T + u] * s.dt[u] * s.CB[i * T + u] * s.YX[i * T + u];
-    for (int i2 = i; i2 < T; ++i2) {
-      const float m = s.W[i2 * T + i] * s.CB[i2 * T + i] * s.YX[i2 * T + i];
-      den += m;
-      ex += m;
-    }
+    float num = 0.f, den = 0.f;
+    for (int u = 0; u <= i; ++u) num += s.Q[i * (T + 1) + u] * s.dt[u];
+    for (int i2 = i; i2 < T; ++i2) den += s.Q[i2 * (T + 1) + i];
     float Si = sa + num - s.dt[i] * den;
+    float ex = den;
     if (has_dhe) {
       float xd = 0.f;
-      for (int q = 0; q < P; ++q) xd += s.x[i * P + q] * s.dhB[i * P + q];
-      const float r = lame / s.lam[i];
-      Si -= s.dt[i] * r * xd;
-      ex += r * xd;
+      for (int q = 0; q < P; ++q) xd += s.xt[q * T + i] * s.dhBt[q * T + i];
+      Si -= s.dt[i] * s.r[i] * xd;
+      ex += s.r[i] * xd;
       if (i == T - 1) Si += he_dot;
     }
     s.S[i] = Si;
@@ -260,15 +318,20 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
     accA += pa;
     accD += pd;
   }
-  // ---- gradient of the start state
-  if (!rev) {
-    for (int64_t e = tid; e < PN; e += kBwdThreads) {
-      const int q = static_cast<int>(e / N), n = static_cast<int>(e % N);
-      float a = 0.f;
-      for (int i = 0; i < T; ++i) a += s.lam[i] * s.dy[i * P + q] * s.Cm[i * N + n];
-      s.carry[e] = (kind == 0 ? lame * s.carry[e] : s.carry[e]) + a;
-    }
-  }
+  // ---- gradient of the start state: dh_s = Lam_e dh_e + sum_i Lam_i dy_i C_i^T
+  if (!rev)
+    sgemm(P, N, T, s.dy, 1, P, s.lam, s.Cm, N, 0, nullptr, 0, 0, nul, nullptr, 0,
+          [&](int m0, int n0, float (&acc)[4][4]) {
+            for (int i = 0; i < 4; ++i) {
+              float4 *cp = reinterpret_cast<float4 *>(s.carry + (m0 + i) * N + n0);
+              float4 c = *cp;
+              if (kind == 0) {
+                c.x *= lame; c.y *= lame; c.z *= lame; c.w *= lame;
+              }
+              c.x += acc[i][0]; c.y += acc[i][1]; c.z += acc[i][2]; c.w += acc[i][3];
+              *cp = c;
+            }
+          });
   __syncthreads();
 }
 
@@ -283,21 +346,22 @@ __global__ void __launch_bounds__(kBwdThreads) bd_bwd_kernel(const __grid_consta
   s.Bm = q; q += T * N;
   s.Cm = q; q += T * N;
   s.xt = q; q += T * P;
+  s.dyt = q; q += T * P;
   s.Bt = q; q += T * N;
   s.Ct = q; q += T * N;
   s.dt = q; q += T;
   s.cum = q; q += T;
   s.lam = q; q += T;
+  s.r = q; q += T;
   s.S = q; q += T;
   s.expl = q; q += T;
   s.red = q; q += kBwdThreads;
-  s.CB = q; q += T * T;
+  s.WCB = q; q += T * T;
   s.YX = q; q += T * T;
-  s.W = q; q += T * T;
-  s.hsC = q; q += T * P;
-  s.dhB = q; q += T * P;
-  s.dyh = q; q += T * N;
-  s.xdh = q; q += T * N;
+  s.G2 = q; q += T * T;
+  s.Q = q; q += T * (T + 1);  // (a multiple of 4 floats: the buffers after it stay 16-byte aligned)
+  s.hsCt = q; q += P * T;
+  s.dhBt = q; q += P * T;
   s.hs = q; q += PN;
   s.carry = q;
   const int b = blockIdx.x / H, h = blockIdx.x % H;
@@ -364,7 +428,8 @@ __global__ void bd_bwd_reduce_head_kernel(const float *pA, const float *pD, floa
 }  // namespace
 
 size_t bwd_smem_bytes(int64_t P, int64_t N, int64_t T) {
-  const int64_t floats = 3 * T * P + 4 * T * N + 5 * T + kBwdThreads + 3 * T * T + 2 * T * P + 2 * T * N + 2 * P * N;
+  const int64_t floats = 4 * T * P + 4 * T * N + 6 * T + kBwdThreads + 3 * T * T + T * (T + 1) + 2 * P * T +
+                         2 * P * N;
   return static_cast<size_t>(floats) * sizeof(float);
 }
 

@@ -157,8 +157,9 @@ typedef struct {
  *   ws, ws_bytes  at least bdscan_workspace_size(shape, ALLBLOCK_BACKWARD)
  *                 bytes (per-head / per-row partial sums, reduced in a fixed
  *                 order: the result is deterministic)
- * Shapes: as for the forward; additionally the per-block shared-memory plan
- * (P, N, block_len) must fit one CTA (P = 64, N = 128, block_len = 32 does).
+ * Shapes: as for the forward; additionally block_len and dstate must be
+ * multiples of 4 and the per-block shared-memory plan (P, N, block_len) must
+ * fit one CTA (P = 64, N = 128, block_len = 32 does).
  * Gradients must not overlap any input or each other. */
 int bdscan_allblock_backward(const bdscan_shape_t *shape, const bdscan_dir_t *clean_fwd,
                              const bdscan_dir_t *clean_rev, const bdscan_dir_t *noisy_fwd,
