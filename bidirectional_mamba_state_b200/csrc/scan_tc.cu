@@ -29,15 +29,18 @@
 //   bd_tc_kernel  persistent, one CTA per SM: each CTA walks its share of the
 //                 work items -- (b, h) sequences, or segments of them -- block
 //                 by block with the fp32 state on chip, the pipeline running
-//                 on across item boundaries.  Warp roles (448 threads):
+//                 on across item boundaries.  Warp roles (512 threads; warp w
+//                 runs on SM sub-partition w mod 4):
 //     warp 0      TMA producer: x, B, C and C B^T tiles of block k into a
 //                 3-slot ring (two blocks of lookahead)
 //     warp 1      TMEM allocator and single-thread tcgen05.mma issuer
-//     warps 2-5   operands: decays, (w o X) (bf16 hi + lo), masked-decay M
-//     warps 6-9   state chain: thread n keeps column n of the fp32 state,
+//     warps 2,3,6,7  operands: per-step decay tables, (w o X) (bf16 hi + lo)
+//     warps 4,5   idle (they keep the operand warps off the MMA issuer's
+//                 sub-partition)
+//     warps 8-11  state chain: thread n keeps column n of the fp32 state,
 //                 h_k = exp(cum_31) h_{k-1} + S; boundary-state stores (one
 //                 128-byte line per warp instruction); h operand (bf16 hi + lo)
-//     warps 10-13 epilogue: thread (p, stream) forms y[t][p] = exp(cum_t) Y_off
+//     warps 12-15 epilogue: thread (p, stream) forms y[t][p] = exp(cum_t) Y_off
 //                 + Y_diag for the block's 32 tokens and stores them; the D x
 //                 terms are small tensor-core products against D I_16 (bf16
 //                 hi + lo) accumulated into Y_diag.  Two blocks ahead, the
@@ -186,7 +189,7 @@ __global__ void __launch_bounds__(kCbThreads) bd_cb_kernel(const __grid_constant
 }
 
 // ------------------------------------------------------------------ main kernel
-constexpr int kThreads = 448;
+constexpr int kThreads = 512;
 
 // shared memory map (bytes from a 1024-aligned base)
 //   TMA ring, 3 slots (two blocks of lookahead); slot r holds block k = r mod 3:
@@ -433,8 +436,17 @@ __device__ __forceinline__ void sts_s32(uint32_t addr, int v) {
   asm volatile("st.shared.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
-// Claim the next work item (-1: none left).
-__device__ __forceinline__ int claim_item(const TcParams &p) {
+__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Claim the next work item (-1: none left).  With no more items than CTAs,
+// CTA c takes item c and nothing else (no counter, no wait for the pre-pass);
+// otherwise items come from the global counter the pre-pass zeroed.
+__device__ __forceinline__ int claim_item(const TcParams &p, int nth, bool &waited) {
+  if (p.items <= static_cast<int>(gridDim.x)) return nth == 0 ? static_cast<int>(blockIdx.x) : -1;
+  if (!waited) {
+    wait_prior_grid();
+    waited = true;
+  }
   const int it = atomicAdd(p.item_counter, 1);
   return it < p.items ? it : -1;
 }
@@ -488,10 +500,12 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
   // items m and m + 1 are published when item m starts (nothing after a -1);
   // claiming further ahead would hold items back from CTAs that run dry at
   // the end of the pass
-  int cur = claim_item(p), nxt = -1;
+  bool waited = false;  // past the wait for the preceding grid
+  int nclaim = 0;
+  int cur = claim_item(p, nclaim++, waited), nxt = -1;
   publish_item(p, c, base, 0, cur);
   if (cur >= 0) {
-    nxt = claim_item(p);
+    nxt = claim_item(p, nclaim++, waited);
     publish_item(p, c, base, 1, nxt);
   }
   for (int m = 0; ok && cur >= 0; ++m) {
@@ -508,13 +522,8 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
       const uint32_t st = base + r * kSlot;
       const int t0 = k * kT;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (!p.active[i]) continue;
-        tma_load_4d_s(st + kOffX + i * kTile, &p.tx[i], full, 0, I.h, t0, I.b);
-        if (p.agg) continue;
-        const int idx = ((i * p.Bsz + I.b) * p.K + k) * p.G + I.g;
-        tma_load_3d_s(st + kOffCB + i * 2048, &p.tcb, full, 0, 0, idx);
-      }
+      for (int i = 0; i < 4; ++i)
+        if (p.active[i]) tma_load_4d_s(st + kOffX + i * kTile, &p.tx[i], full, 0, I.h, t0, I.b);
       tma_load_4d_s(st + kOffBcf, &p.tbcf, full, 0, I.g, t0, I.b);
       tma_load_4d_s(st + kOffBcf + kTile, &p.tbcf, full, 64, I.g, t0, I.b);
       if (!p.agg) {
@@ -524,6 +533,17 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
           tma_load_4d_s(st + kOffClo + kTile, &p.tcnf, full, 0, I.g, t0, I.b);
           tma_load_4d_s(st + kOffChi + kTile, &p.tcnf, full, 64, I.g, t0, I.b);
         }
+        // C B^T tiles: written by the pre-pass this kernel may overlap
+        if (!waited) {
+          wait_prior_grid();
+          waited = true;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (!p.active[i]) continue;
+          const int idx = ((i * p.Bsz + I.b) * p.K + k) * p.G + I.g;
+          tma_load_3d_s(st + kOffCB + i * 2048, &p.tcb, full, 0, 0, idx);
+        }
       }
 #pragma unroll
       for (int s = 0; s < kSlots; ++s)
@@ -532,7 +552,7 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
     cur = nxt;
     nxt = -1;
     if (ok && cur >= 0) {
-      nxt = claim_item(p);
+      nxt = claim_item(p, nclaim++, waited);
       publish_item(p, c, base, m + 2, nxt);
     }
   }
@@ -640,14 +660,15 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
 }
 
 // ---------------------------------------------------------------- operand group
-// warps 2..5; q = warp & 3 is the direction slot whose decays it computes.
+// warps 2, 3, 6, 7 (direction slots q = 0..3, whose decays each computes).
 // Per step: the per-step tables (cumulative decays, dt, exp(cum) of the
 // forward directions, D of the step's head, item-start flag) and w o X.
 // The masked-decay matrices are built by the epilogue warps.
 __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
   const int lane = threadIdx.x & 31;
-  const int q = (threadIdx.x >> 5) & 3;
-  const int gt = threadIdx.x - 64;  // 0..127
+  const int wq = threadIdx.x >> 5;
+  const int q = wq < 4 ? wq - 2 : wq - 4;
+  const int gt = q * 32 + (threadIdx.x & 31);  // 0..127
   const bool act = pick4(p.active, q) != 0;
   const uint32_t cum = base + kOffCum, dts = base + kOffDt, ecum = base + kOffEc;
   const int64_t H = p.H, L = p.L;
@@ -829,7 +850,7 @@ __device__ void state_group_staged(const TcParams &p, const Ctl &c, uint32_t bas
   }
 }
 
-// warps 6..9: thread owns column n = 32 q + lane of the state, h^T[n][0..63].
+// warps 8..11: thread owns column n = 32 q + lane of the state, h^T[n][0..63].
 // A failed (timed-out) wait ends the group at once: nothing else is stored.
 __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
   const int lane = threadIdx.x & 31;
@@ -879,6 +900,7 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
       const float *src = p.agg ? nullptr
                          : I.seg == 0 ? (p.h0 ? p.h0 + bh * PN + n : nullptr)
                                       : p.seg_init + (bh * p.nseg + I.seg) * PN + n;
+      if (src && I.seg > 0) wait_prior_grid();  // segment states: written by the combine kernel
 #pragma unroll
       for (int pp = 0; pp < kP; ++pp) hreg[pp] = src ? src[pp * kN] : 0.f;
     }
@@ -943,7 +965,7 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
 }
 
 // ---------------------------------------------------------------- epilogue
-// warps 10..13: thread owns column p = 16 q + (lane & 15) of the clean
+// warps 12..15: thread owns column p = 16 q + (lane & 15) of the clean
 // (lane < 16) or noisy (lane >= 16) stream's outputs y[t][p], t = 0..31:
 // y = exp(cum_t) Y_off + Y_diag (Y_diag already holds both directions' D x).
 // After the outputs of step j the group builds, two steps ahead, the
@@ -952,7 +974,7 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
 __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
   const int lane = threadIdx.x & 31;
   const int q = (threadIdx.x >> 5) & 3;
-  const int gq = threadIdx.x - 320;  // 0..127
+  const int gq = threadIdx.x - 384;  // 0..127
   const int pcol = 16 * q + (lane & 15);
   const bool noisy = lane >= 16;
   const int fs = noisy ? kNF : kCF;
@@ -1114,18 +1136,21 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   Ctl c{smem_u32(bars), base + kOffMisc};
-  // Launched as a programmatic dependent of the previous kernel on the stream:
-  // the prologue above overlaps its tail; nothing it wrote (C B^T tiles, work
-  // counters, segment states) is read before it has completed.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // Launched as a programmatic dependent of the previous kernel on the stream
+  // (the C B^T pre-pass, or the segment combine): the threads that read what it
+  // wrote -- the producer (work counter, C B^T tiles) and the state warps
+  // (segment initial states) -- wait for its completion (griddepcontrol.wait)
+  // just before those reads; everything else overlaps its tail.
 
   if (warp == 0) {
     if ((threadIdx.x & 31) == 0) producer(p, c, base);
   } else if (warp == 1) {
     if ((threadIdx.x & 31) == 0) mma_issuer(p, c, base, tmem);
-  } else if (warp < 6) {
+  } else if (warp == 2 || warp == 3 || warp == 6 || warp == 7) {
     operand_group(p, c, base);
-  } else if (warp < 10) {
+  } else if (warp == 4 || warp == 5) {
+    // idle: keeps the operand warps off the MMA issuer's SM sub-partition
+  } else if (warp < 12) {
     state_group(p, c, base, tmem);
   } else {
     epilogue_group(p, c, base, tmem);
