@@ -45,6 +45,15 @@ class _Grad(ctypes.Structure):
     _fields_ = [("dx", _dp), ("ddt", _dp), ("dB", _dp), ("dC", _dp), ("dA", _dp), ("dD", _dp)]
 
 
+class _ConvShape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in
+                ("batch", "seqlen", "channels", "width", "block_len", "silu")]
+
+
+class _ConvDir(ctypes.Structure):
+    _fields_ = [("u", _dp), ("w", _dp), ("bias", _dp), ("v", _dp)]
+
+
 def build(force: bool = False) -> str:
     """Compile the oracle shared library with gcc (-O2, OpenMP).  Returns its path."""
     if force or not os.path.exists(_LIB_PATH) or (
@@ -59,7 +68,8 @@ def build(force: bool = False) -> str:
 
 def _open(path: str):
     lib = ctypes.CDLL(path)
-    for name in ("oracle_prefix", "oracle_block_step", "oracle_allblock", "oracle_allblock_backward"):
+    for name in ("oracle_prefix", "oracle_block_step", "oracle_allblock", "oracle_allblock_backward",
+                 "oracle_conv_prefix", "oracle_conv_allblock"):
         getattr(lib, name).restype = ctypes.c_int
     lib.oracle_max_threads.restype = ctypes.c_int
     lib.oracle_set_threads.argtypes = [ctypes.c_int]
@@ -220,6 +230,86 @@ def allblock_backward(shape: dict, clean_fwd: dict, clean_rev: dict | None, nois
     return grads, dh0
 
 
+# ---- short convolution in front of the scan --------------------------------
+#
+# A direction's convolution inputs are a dict with keys x [B][L][H][P],
+# B and C [B][L][G][N] (pre-convolution), weight [H*P + 2*G*N][width] and
+# optionally bias [H*P + 2*G*N].  The channels are packed x | B | C into flat
+# rows for the C code and unpacked again; outputs are dicts with keys x, B, C.
+
+
+def _pack_rows(shape: dict, d: dict) -> np.ndarray:
+    B, L = int(shape["batch"]), int(shape["seqlen"])
+    parts = []
+    for k in ("x", "B", "C"):
+        a = _f64(d[k])
+        parts.append(a.reshape(B, L, int(np.prod(a.shape[2:]))))
+    return np.ascontiguousarray(np.concatenate(parts, axis=2))
+
+
+def _unpack_rows(shape: dict, v: np.ndarray) -> dict:
+    B, L, H, P, N, G = (int(shape[k]) for k in
+                        ("batch", "seqlen", "nheads", "headdim", "dstate", "ngroups"))
+    hp, gn = H * P, G * N
+    return {"x": v[:, :, :hp].reshape(B, L, H, P), "B": v[:, :, hp:hp + gn].reshape(B, L, G, N),
+            "C": v[:, :, hp + gn:].reshape(B, L, G, N)}
+
+
+def _conv_shape(shape: dict, width: int, silu: bool) -> _ConvShape:
+    H, P, N, G = (int(shape[k]) for k in ("nheads", "headdim", "dstate", "ngroups"))
+    return _ConvShape(int(shape["batch"]), int(shape["seqlen"]), H * P + 2 * G * N, int(width),
+                      int(shape["block_len"]), 1 if silu else 0)
+
+
+class _ConvMarshal(_Marshal):
+    def __init__(self, shape: dict):
+        super().__init__()
+        self.shape = shape
+        self.outs = []
+
+    def conv(self, d):
+        if d is None:
+            self.outs.append(None)
+            return None
+        u = _pack_rows(self.shape, d)
+        v = np.zeros_like(u)
+        self.keep += [u, v]
+        self.outs.append(v)
+        w = self.arr(d["weight"])
+        bias = self.arr(d.get("bias"))
+        return ctypes.pointer(_ConvDir(u=_ptr(u), w=_ptr(w), bias=_ptr(bias), v=_ptr(v)))
+
+
+def conv_prefix(shape: dict, width: int, silu: bool, fwd: dict, rev: dict | None = None,
+                state_in=None, want_state_out: bool = False, lib=None):
+    """Short convolution of one sequence: causal for ``fwd`` from ``state_in``
+    ([B][width-1][H*P + 2*G*N], None = zeros), anti-causal inside each block for
+    ``rev``.  Returns (fwd outputs, rev outputs or None, state_out or None)."""
+    lib = lib or _load()
+    m = _ConvMarshal(shape)
+    cs = _conv_shape(shape, width, silu)
+    pf, pr = m.conv(fwd), m.conv(rev)
+    so = np.zeros((int(shape["batch"]), int(width) - 1, cs.channels)) if want_state_out else None
+    rc = lib.oracle_conv_prefix(ctypes.byref(cs), pf, pr, _ptr(m.arr(state_in)), _ptr(so))
+    _check(rc, "oracle_conv_prefix")
+    vf, vr = m.outs
+    return (_unpack_rows(shape, vf), None if vr is None else _unpack_rows(shape, vr), so)
+
+
+def conv_allblock(shape: dict, width: int, silu: bool, clean_fwd: dict, clean_rev: dict | None,
+                  noisy_fwd: dict, noisy_rev: dict | None, state_in=None, lib=None):
+    """Short convolution of the all-block pass: the clean stream as in
+    ``conv_prefix``; every noisy block's forward convolution reads the clean rows
+    before it.  Returns a list of four output dicts (None for absent directions)."""
+    lib = lib or _load()
+    m = _ConvMarshal(shape)
+    cs = _conv_shape(shape, width, silu)
+    ptrs = [m.conv(d) for d in (clean_fwd, clean_rev, noisy_fwd, noisy_rev)]
+    rc = lib.oracle_conv_allblock(ctypes.byref(cs), *ptrs, _ptr(m.arr(state_in)))
+    _check(rc, "oracle_conv_allblock")
+    return [None if v is None else _unpack_rows(shape, v) for v in m.outs]
+
+
 class Variant:
     """The same API bound to another build of the oracle source (used by the
     tests that plant a mistake in a copy of the oracle and check that the pins
@@ -239,6 +329,12 @@ class Variant:
 
     def allblock_backward(self, *a, **k):
         return allblock_backward(*a, lib=self.lib, **k)
+
+    def conv_prefix(self, *a, **k):
+        return conv_prefix(*a, lib=self.lib, **k)
+
+    def conv_allblock(self, *a, **k):
+        return conv_allblock(*a, lib=self.lib, **k)
 
 
 def compile_variant(src_text: str, out_path: str) -> str:

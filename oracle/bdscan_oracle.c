@@ -29,6 +29,11 @@
  *   the clean stream's boundary state before it (h0 for block 0) and gets its
  *   own block-local reverse scan.
  *
+ *   The short convolution (+SiLU) in front of the scan, causal for the
+ *   forward direction and anti-causal inside the block for the reverse one,
+ *   with the conv state of the cache (see the section before
+ *   oracle_max_threads for its definition and citations).
+ *
  * Layouts (row-major, innermost last):
  *   x, z, y  [B][L][H][P]    dt [B][L][H]    Bm, Cm [B][L][G][N]
  *   A, D     [H]             state [B][H][P][N]   states [B][K][H][P][N]
@@ -472,6 +477,132 @@ int oracle_allblock_backward(const oracle_shape_t *s, const oracle_dir_t *cf, co
     }
     free(states); free(acc); free(pool);
     return failed ? ORACLE_ENOMEM : ORACLE_OK;
+}
+
+/* ---- Short convolution in front of the scan ---------------------------------
+ *
+ * In a Mamba-2 layer every x, B and C channel goes through a depthwise
+ * convolution of `width` taps over time, then a SiLU, before the scan.  A Mamba
+ * layer's cache holds this convolution's state (the last width-1 input rows)
+ * beside the scan state ("Training Hybrid Block Diffusion Language Models with
+ * Partial Bidirectionality", the paragraph after eq. (14)).  The reverse
+ * direction's convolution is anti-causal ("Breaking the Bottleneck with
+ * DiffuApriel", section 3.2, after eq. (5)) and, like the reverse scan, stays
+ * inside its block (first page, eq. (12)).
+ *
+ * Rows are flat: u[b][t][c] with c < channels (the caller packs x | B | C).
+ * The conv state is [b][width-1][channels], oldest row first.
+ *   causal:       v[t] = act(bias + sum_{j < W} w[j] * u[t - (W-1) + j])
+ *   anti-causal:  v[t] = act(bias + sum_{j < W} w[j] * u[t + (W-1) - j]),
+ *                 u taken as 0 past the end of t's block
+ * act is silu when asked for, else the identity. */
+typedef struct {
+    int64_t batch, seqlen, channels, width, block_len;
+    int64_t silu;
+} oracle_conv_shape_t;
+
+typedef struct {
+    const double *u;    /* [B][L][channels] pre-convolution rows */
+    const double *w;    /* [channels][width] taps */
+    const double *bias; /* [channels] or NULL (zeros) */
+    double *v;          /* [B][L][channels] output */
+} oracle_conv_dir_t;
+
+/* Pre-convolution value of channel c at token tp of batch row b as a causal
+ * convolution sees it: the direction's own rows from token own_from on, the
+ * rows of `halo` (another stream, same layout) between token 0 and own_from,
+ * the conv state before token 0, and zeros before the state (or without one). */
+static double conv_input(const oracle_conv_shape_t *s, const double *own, int64_t own_from,
+                         const double *halo, const double *state, int64_t b, int64_t tp, int64_t c) {
+    const int64_t L = s->seqlen, Cx = s->channels, W = s->width;
+    if (tp >= own_from) return own[(b * L + tp) * Cx + c];
+    if (tp >= 0) return halo[(b * L + tp) * Cx + c];
+    if (state && tp >= -(W - 1)) return state[(b * (W - 1) + (W - 1 + tp)) * Cx + c];
+    return 0.0;
+}
+
+static double conv_act(const oracle_conv_shape_t *s, const oracle_conv_dir_t *d, int64_t c, double acc) {
+    const double v = acc + (d->bias ? d->bias[c] : 0.0);
+    return s->silu ? silu(v) : v;
+}
+
+/* Causal convolution of one direction.  halo == NULL: over the whole stream;
+ * otherwise every block continues from `halo`'s rows before it. */
+static void conv_causal(const oracle_conv_shape_t *s, const oracle_conv_dir_t *d, const double *halo,
+                        const double *state) {
+    const int64_t L = s->seqlen, Cx = s->channels, W = s->width, T = s->block_len;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < s->batch; ++b)
+        for (int64_t t = 0; t < L; ++t) {
+            const int64_t own_from = halo ? (t / T) * T : 0;
+            for (int64_t c = 0; c < Cx; ++c) {
+                double acc = 0.0;
+                for (int64_t j = 0; j < W; ++j)
+                    acc += d->w[c * W + j] * conv_input(s, d->u, own_from, halo, state, b, t - (W - 1) + j, c);
+                d->v[(b * L + t) * Cx + c] = conv_act(s, d, c, acc);
+            }
+        }
+}
+
+/* Anti-causal convolution confined to each block, from zeros past its end. */
+static void conv_anticausal(const oracle_conv_shape_t *s, const oracle_conv_dir_t *d) {
+    const int64_t L = s->seqlen, Cx = s->channels, W = s->width, T = s->block_len;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < s->batch; ++b)
+        for (int64_t t = 0; t < L; ++t) {
+            const int64_t block_end = (t / T + 1) * T;
+            for (int64_t c = 0; c < Cx; ++c) {
+                double acc = 0.0;
+                for (int64_t j = 0; j < W; ++j) {
+                    const int64_t tp = t + (W - 1) - j;
+                    acc += d->w[c * W + j] * (tp < block_end ? d->u[(b * L + tp) * Cx + c] : 0.0);
+                }
+                d->v[(b * L + t) * Cx + c] = conv_act(s, d, c, acc);
+            }
+        }
+}
+
+static int conv_check(const oracle_conv_shape_t *s, const oracle_conv_dir_t *d) {
+    if (!s || s->batch < 0 || s->seqlen < 0 || s->channels < 1 || s->width < 1 || s->block_len < 1 ||
+        s->seqlen % s->block_len)
+        return ORACLE_EINVAL;
+    if (d && (!d->u || !d->w || !d->v)) return ORACLE_EINVAL;
+    return ORACLE_OK;
+}
+
+/* Convolution of one sequence (prefill, commit or a denoising step): the
+ * forward direction causal from state_in (NULL: zeros), the reverse one
+ * anti-causal inside each block; state_out (or NULL) receives the last W-1
+ * rows of the forward stream, state_in's rows included when L < W-1. */
+int oracle_conv_prefix(const oracle_conv_shape_t *s, const oracle_conv_dir_t *fwd,
+                       const oracle_conv_dir_t *rev, const double *state_in, double *state_out) {
+    if (conv_check(s, fwd) || !fwd || conv_check(s, rev)) return ORACLE_EINVAL;
+    conv_causal(s, fwd, NULL, state_in);
+    if (rev) conv_anticausal(s, rev);
+    if (state_out) {
+        const int64_t W = s->width, Cx = s->channels;
+        for (int64_t b = 0; b < s->batch; ++b)
+            for (int64_t r = 0; r < W - 1; ++r)
+                for (int64_t c = 0; c < Cx; ++c)
+                    state_out[(b * (W - 1) + r) * Cx + c] =
+                        conv_input(s, fwd->u, 0, NULL, state_in, b, s->seqlen - (W - 1) + r, c);
+    }
+    return ORACLE_OK;
+}
+
+/* Convolution of the all-block pass: the clean stream as by oracle_conv_prefix;
+ * noisy block k's forward convolution reads the clean rows before the block
+ * (state_in before token 0), the noisy reverse stays inside the block. */
+int oracle_conv_allblock(const oracle_conv_shape_t *s, const oracle_conv_dir_t *cf,
+                         const oracle_conv_dir_t *cr, const oracle_conv_dir_t *nf,
+                         const oracle_conv_dir_t *nr, const double *state_in) {
+    if (conv_check(s, cf) || !cf || conv_check(s, cr) || conv_check(s, nf) || !nf || conv_check(s, nr))
+        return ORACLE_EINVAL;
+    conv_causal(s, cf, NULL, state_in);
+    if (cr) conv_anticausal(s, cr);
+    conv_causal(s, nf, cf->u, state_in);
+    if (nr) conv_anticausal(s, nr);
+    return ORACLE_OK;
 }
 
 int oracle_max_threads(void) {
