@@ -95,30 +95,31 @@ __device__ float block_sum(float v, float *red) {
   return r;
 }
 
-// Register-tiled product over shared-memory operands: for every 4 x 4 output
-// tile (m0.., n0..) of an M x Nn result,
+// Register-tiled product over shared-memory operands: for every TM x 4 output
+// tile (m0.., n0..) of an M x Nn result (TM chosen per product so that the
+// 256 threads have a tile each),
 //   acc[i][j] = sum_k a1(m0+i, k) B1[k][n0+j]  (+ sum_k a2(m0+i, k) B2[k][n0+j])
 // with a(m, k) = A[m am + k ak] (times ks1[k], resp. ms2[m], when given) and
 // B rows contiguous in n (16-byte loads).  A threads of a warp share m0, so A
 // loads are broadcasts.  epi(m0, n0, acc) consumes the tile.
-template <class Epi>
+template <int TM, class Epi>
 __device__ __forceinline__ void sgemm(int M, int Nn, int K1, const float *A1, int am1, int ak1, const float *ks1,
                                       const float *B1, int ldb1, int K2, const float *A2, int am2, int ak2,
                                       const float *ms2, const float *B2, int ldb2, Epi epi) {
   const int nt = Nn >> 2;
-  const int tiles = (M >> 2) * nt;
+  const int tiles = (M / TM) * nt;
   for (int t = threadIdx.x; t < tiles; t += kBwdThreads) {
-    const int m0 = (t / nt) << 2, n0 = (t % nt) << 2;
-    float acc[4][4];
+    const int m0 = (t / nt) * TM, n0 = (t % nt) << 2;
+    float acc[TM][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < TM; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
     for (int k = 0; k < K1; ++k) {
       const float4 bv = *reinterpret_cast<const float4 *>(B1 + k * ldb1 + n0);
       const float sk = ks1 ? ks1[k] : 1.f;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < TM; ++i) {
         const float a = A1[(m0 + i) * am1 + k * ak1] * sk;
         acc[i][0] = fmaf(a, bv.x, acc[i][0]);
         acc[i][1] = fmaf(a, bv.y, acc[i][1]);
@@ -127,13 +128,13 @@ __device__ __forceinline__ void sgemm(int M, int Nn, int K1, const float *A1, in
       }
     }
     if (A2) {
-      float sm2[4];
+      float sm2[TM];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) sm2[i] = ms2 ? ms2[m0 + i] : 1.f;
+      for (int i = 0; i < TM; ++i) sm2[i] = ms2 ? ms2[m0 + i] : 1.f;
       for (int k = 0; k < K2; ++k) {
         const float4 bv = *reinterpret_cast<const float4 *>(B2 + k * ldb2 + n0);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < TM; ++i) {
           const float a = A2[(m0 + i) * am2 + k * ak2] * sm2[i];
           acc[i][0] = fmaf(a, bv.x, acc[i][0]);
           acc[i][1] = fmaf(a, bv.y, acc[i][1]);
@@ -207,27 +208,31 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
   __syncthreads();
 
   // ---- Gram matrices: C B^T and dy x^T
-  sgemm(T, T, N, s.Cm, N, 1, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
-        [&](int m0, int n0, float (&acc)[4][4]) {
-          for (int i = 0; i < 4; ++i)
+  sgemm<1>(T, T, N, s.Cm, N, 1, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+        [&](int m0, int n0, auto &acc) {
+          constexpr int R = sizeof(acc) / sizeof(acc[0]);
+          for (int i = 0; i < R; ++i)
             *reinterpret_cast<float4 *>(s.WCB + (m0 + i) * T + n0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
         });
-  sgemm(T, T, P, s.dy, P, 1, nul, s.xt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
-        [&](int m0, int n0, float (&acc)[4][4]) {
-          for (int i = 0; i < 4; ++i)
+  sgemm<1>(T, T, P, s.dy, P, 1, nul, s.xt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+        [&](int m0, int n0, auto &acc) {
+          constexpr int R = sizeof(acc) / sizeof(acc[0]);
+          for (int i = 0; i < R; ++i)
             *reinterpret_cast<float4 *>(s.YX + (m0 + i) * T + n0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
         });
   // ---- products with the start state and the end-state gradient
   if (has_hs)
-    sgemm(P, T, N, s.hs, N, 1, nul, s.Ct, T, 0, nullptr, 0, 0, nul, nullptr, 0,
-          [&](int m0, int n0, float (&acc)[4][4]) {
-            for (int i = 0; i < 4; ++i)
+    sgemm<2>(P, T, N, s.hs, N, 1, nul, s.Ct, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+          [&](int m0, int n0, auto &acc) {
+          constexpr int R = sizeof(acc) / sizeof(acc[0]);
+            for (int i = 0; i < R; ++i)
               *reinterpret_cast<float4 *>(s.hsCt + (m0 + i) * T + n0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
           });
   if (has_dhe)
-    sgemm(P, T, N, s.carry, N, 1, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
-          [&](int m0, int n0, float (&acc)[4][4]) {
-            for (int i = 0; i < 4; ++i)
+    sgemm<2>(P, T, N, s.carry, N, 1, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+          [&](int m0, int n0, auto &acc) {
+          constexpr int R = sizeof(acc) / sizeof(acc[0]);
+            for (int i = 0; i < R; ++i)
               *reinterpret_cast<float4 *>(s.dhBt + (m0 + i) * T + n0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
           });
   float he_dot = 0.f;
@@ -252,9 +257,10 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
 
   // ---- token gradients
   // dx_u = D dy_u + dt_u sum_i WCB[i][u] dy_i (+ dt_u r_u dh_e B_u)
-  sgemm(T, P, T, s.WCB, 1, T, nul, s.dy, P, 0, nullptr, 0, 0, nul, nullptr, 0,
-        [&](int m0, int n0, float (&acc)[4][4]) {
-          for (int i = 0; i < 4; ++i) {
+  sgemm<2>(T, P, T, s.WCB, 1, T, nul, s.dy, P, 0, nullptr, 0, 0, nul, nullptr, 0,
+        [&](int m0, int n0, auto &acc) {
+          constexpr int R = sizeof(acc) / sizeof(acc[0]);
+          for (int i = 0; i < R; ++i) {
             const int u = m0 + i;
             float v[4];
             for (int j = 0; j < 4; ++j) {
@@ -266,16 +272,18 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
           }
         });
   // dC_i = sum_u G2[i][u] dt_u B_u (+ Lam_i dy_i^T h_s)
-  sgemm(T, N, T, s.G2, T, 1, s.dt, s.Bm, N, has_hs ? P : 0, has_hs ? s.dy : nullptr, P, 1, s.lam, s.hs, N,
-        [&](int m0, int n0, float (&acc)[4][4]) {
-          for (int i = 0; i < 4; ++i)
+  sgemm<4>(T, N, T, s.G2, T, 1, s.dt, s.Bm, N, has_hs ? P : 0, has_hs ? s.dy : nullptr, P, 1, s.lam, s.hs, N,
+        [&](int m0, int n0, auto &acc) {
+          constexpr int R = sizeof(acc) / sizeof(acc[0]);
+          for (int i = 0; i < R; ++i)
             *reinterpret_cast<float4 *>(d.pC + ((static_cast<int64_t>(b) * L + tok(m0 + i)) * H + h) * N + n0) =
                 make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
         });
   // dB_u = dt_u (sum_i G2[i][u] C_i (+ r_u x_u^T dh_e))
-  sgemm(T, N, T, s.G2, 1, T, nul, s.Cm, N, has_dhe ? P : 0, has_dhe ? s.x : nullptr, P, 1, s.r, s.carry, N,
-        [&](int m0, int n0, float (&acc)[4][4]) {
-          for (int i = 0; i < 4; ++i) {
+  sgemm<4>(T, N, T, s.G2, 1, T, nul, s.Cm, N, has_dhe ? P : 0, has_dhe ? s.x : nullptr, P, 1, s.r, s.carry, N,
+        [&](int m0, int n0, auto &acc) {
+          constexpr int R = sizeof(acc) / sizeof(acc[0]);
+          for (int i = 0; i < R; ++i) {
             const float du = s.dt[m0 + i];
             *reinterpret_cast<float4 *>(d.pB + ((static_cast<int64_t>(b) * L + tok(m0 + i)) * H + h) * N + n0) =
                 make_float4(du * acc[i][0], du * acc[i][1], du * acc[i][2], du * acc[i][3]);
@@ -320,9 +328,10 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
   }
   // ---- gradient of the start state: dh_s = Lam_e dh_e + sum_i Lam_i dy_i C_i^T
   if (!rev)
-    sgemm(P, N, T, s.dy, 1, P, s.lam, s.Cm, N, 0, nullptr, 0, 0, nul, nullptr, 0,
-          [&](int m0, int n0, float (&acc)[4][4]) {
-            for (int i = 0; i < 4; ++i) {
+    sgemm<4>(P, N, T, s.dy, 1, P, s.lam, s.Cm, N, 0, nullptr, 0, 0, nul, nullptr, 0,
+          [&](int m0, int n0, auto &acc) {
+          constexpr int R = sizeof(acc) / sizeof(acc[0]);
+            for (int i = 0; i < R; ++i) {
               float4 *cp = reinterpret_cast<float4 *>(s.carry + (m0 + i) * N + n0);
               float4 c = *cp;
               if (kind == 0) {

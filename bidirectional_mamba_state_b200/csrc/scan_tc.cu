@@ -573,25 +573,25 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
   const uint32_t id_yd = idesc_bf16(64, 32, 1, 1);  // Y_diag^T[p][t] = X^T M^T, one stream
   const uint32_t id_dx = idesc_bf16(64, 16, 1, 0);  // (D x)^T[p][t] = X^T (D I_16)
   // descriptor of each operand at its first tile; moving an operand by b bytes adds b >> 4
-  const uint64_t dBcf = sdesc(base + kOffBcf, kTile, 1024, kLayoutSw128);
-  const uint64_t dXw = sdesc(base + kOffXw, 0, 1024, kLayoutSw128);
-  const uint64_t dH = sdesc(base + kOffH, 0, 1024, kLayoutSw128);
-  const uint64_t dC = sdesc(base + kOffClo, 16, 1024, kLayoutSw128);
-  const uint64_t dX = sdesc(base + kOffX, 0, 1024, kLayoutSw128);
-  const uint64_t dM = sdesc(base + kOffMh, kMhLbo, kMhSbo, kLayoutNone);
-  const uint64_t dDg = sdesc(base + kOffDg, kDgLbo, kDgSbo, kLayoutNone);
-#define BD_OFF(bytes) (static_cast<uint64_t>((bytes) >> 4))
+  const D64 dBcf = split64(sdesc(base + kOffBcf, kTile, 1024, kLayoutSw128));
+  const D64 dXw = split64(sdesc(base + kOffXw, 0, 1024, kLayoutSw128));
+  const D64 dH = split64(sdesc(base + kOffH, 0, 1024, kLayoutSw128));
+  const D64 dC = split64(sdesc(base + kOffClo, 16, 1024, kLayoutSw128));
+  const D64 dX = split64(sdesc(base + kOffX, 0, 1024, kLayoutSw128));
+  const D64 dM = split64(sdesc(base + kOffMh, kMhLbo, kMhSbo, kLayoutNone));
+  const D64 dDg = split64(sdesc(base + kOffDg, kDgLbo, kDgSbo, kLayoutNone));
+#define BD_OFF(bytes) (static_cast<uint32_t>((bytes) >> 4))
   int j = 0;
   bool ok = true;
   for (int m = 0; ok; ++m) {
     Item I;
     if (item_one(p, c, base, m, I) <= 0) break;
     const int nk = I.nk;
-    const uint64_t go = BD_OFF(static_cast<uint32_t>(m & 1) * kDgBuf);  // this item's D I_16 operands
+    const uint32_t go = BD_OFF(static_cast<uint32_t>(m & 1) * kDgBuf);  // this item's D I_16 operands
     for (int kk = 0; kk < nk; ++kk, ++j) {
       ok = false;
       const int r = rslot(j), i2 = j & 1;
-      const uint64_t so = BD_OFF(static_cast<uint32_t>(r) * kSlot);  // this step's ring slot
+      const uint32_t so = BD_OFF(static_cast<uint32_t>(r) * kSlot);  // this step's ring slot
       if (!wait1(c, bFull0 + r, parr(j))) break;
       // ---- S^T = B_cf^T (w o X): A MN-major (n; halves 4 KB apart), B MN-major (p)
       if (p.need_s) {
@@ -618,7 +618,7 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
       const uint32_t colY = tmem + kColY0 + 128 * i2;
 #pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t bc = dC + so + BD_OFF((ks < 4 ? 0 : 2 * kTile) + (ks & 3) * 32);
+        const D64 bc = dC + so + BD_OFF((ks < 4 ? 0 : 2 * kTile) + (ks & 3) * 32);
         umma_bf16(colY, dH + BD_OFF(ks * 2048), bc, id_yo, ks > 0);
         umma_bf16(colY, dH + BD_OFF(4 * kTile + ks * 2048), bc, id_yo, 1);
       }
@@ -627,7 +627,7 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
       //      X^T (D I) of every direction
       if (!wait1(c, bMhFull0 + i2, par2(j))) break;
       tc_fence_after();
-      const uint64_t mo = BD_OFF(static_cast<uint32_t>(i2) * kMhBuf);
+      const uint32_t mo = BD_OFF(static_cast<uint32_t>(i2) * kMhBuf);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {  // the forward direction of a stream (i < 2) is always active
         if (!p.active[i]) continue;
@@ -644,7 +644,7 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
         const uint32_t col = colY + 64 + ((i & 1) ? 32 : 0);
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks) {
-          const uint64_t a = dX + so + BD_OFF(i * kTile + ks * 2048);
+          const D64 a = dX + so + BD_OFF(i * kTile + ks * 2048);
           umma_bf16(col + 16 * ks, a, dDg + go + BD_OFF((2 * i) * 512), id_dx, 1);
           umma_bf16(col + 16 * ks, a, dDg + go + BD_OFF((2 * i + 1) * 512), id_dx, 1);
         }

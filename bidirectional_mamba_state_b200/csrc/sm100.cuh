@@ -335,6 +335,25 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t 
       : "memory");
 }
 
+// A shared-memory descriptor held as two 32-bit words.  Offsets move only the
+// low word: its start-address field (address >> 4, 14 bits) covers all of
+// shared memory, so adding an offset that keeps the address inside shared
+// memory never carries into the next field.  Saves the 64-bit adds in the
+// single-thread MMA issue loop.
+struct D64 {
+  uint32_t lo, hi;
+};
+__device__ __forceinline__ D64 split64(uint64_t d) { return D64{static_cast<uint32_t>(d), static_cast<uint32_t>(d >> 32)}; }
+__device__ __forceinline__ D64 operator+(D64 d, uint32_t off) { return D64{d.lo + off, d.hi}; }
+// umma_bf16 on split descriptors.
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, D64 a, D64 b, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\tmov.b64 da, {%1, %2};\n\tmov.b64 db, {%3, %4};\n\t"
+      "setp.ne.b32 p, %6, 0;\n\ttcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}" ::"r"(d_tmem),
+      "r"(a.lo), "r"(a.hi), "r"(b.lo), "r"(b.hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive on `bar` once every tcgen05.mma issued so far by this thread completes.
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
