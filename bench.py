@@ -355,22 +355,37 @@ def run_extra(dev, pk) -> dict:
         out["block_step_3b_b64_40layers"] = _step_stack(W.WORKLOADS["3b_step_b64"], 40, dev, pk)
         out["prefill_700m_8k_per_layer"] = _prefill(W.WORKLOADS["700m_prefill_8k"], dev, pk)
         out["allblock_backward_87m"] = _backward(W.WORKLOADS["87m_allblock"], dev, pk)
+        out["conv_allblock_87m"] = _conv_allblock(W.WORKLOADS["87m_allblock"], 4, dev, pk)
+        out["conv_block_step_700m_b1_24layers"] = _step_stack(W.WORKLOADS["700m_step"], 24, dev, pk,
+                                                              conv_width=4)
     except Exception as e:  # report, never hide
         out["error"] = repr(e)
     return out
 
 
-def _step_stack(s: W.Shape, layers: int, dev, pk) -> dict:
+def _step_stack(s: W.Shape, layers: int, dev, pk, conv_width: int = 0) -> dict:
+    """With ``conv_width``, every layer first runs the short convolution of both
+    directions from its cached conv state (writing the scan's x, B, C), then the
+    scan step: the selective-scan core of a Mamba layer's denoising step."""
     seed = W.SEEDS["700m_step" if s.nheads == 48 else "3b_step_b1"]
     ins = [W.make_streams(s, seed, layer, device=dev, streams=(W.CLEAN_FWD, W.CLEAN_REV))
            for layer in range(layers)]
     states = [W.make_state(s, seed, layer, device=dev) for layer in range(layers)]
     ys = [torch.empty((s.batch, s.seqlen, s.nheads, s.headdim), device=dev) for _ in range(layers)]
     wss = [bd.workspace(s, bd.BDSCAN_OP_BLOCK_STEP, dev) for _ in range(layers)]
+    if conv_width:
+        convs = [[W.make_conv_dir(s, conv_width, seed, layer, st, device=dev) for st in (W.CLEAN_FWD, W.CLEAN_REV)]
+                 for layer in range(layers)]
+        cstates = [W.make_conv_state(s, conv_width, seed, layer, device=dev) for layer in range(layers)]
+        # the convolution writes straight into the scan's x, B, C
+        couts = [[{k: ins[l][i][k] for k in bd.CONV_KEYS} for i in range(2)] for l in range(layers)]
     g_stream = torch.cuda.Stream(dev)
 
     def stack():
         for l in range(layers):
+            if conv_width:
+                bd.conv_prefix(s, conv_width, True, convs[l][0], convs[l][1], cstates[l],
+                               out_fwd=couts[l][0], out_rev=couts[l][1], stream=torch.cuda.current_stream(dev))
             bd.block_step(s, ins[l][0], ins[l][1], states[l], y=ys[l], ws=wss[l],
                           stream=torch.cuda.current_stream(dev))
 
@@ -394,10 +409,29 @@ def _step_stack(s: W.Shape, layers: int, dev, pk) -> dict:
         times.append(e0.elapsed_time(e1))
     ms = statistics.median(times)
     b = RL.block_step_bytes(s) * layers
+    if conv_width:
+        b += RL.conv_bytes(s, conv_width, 2, state_in=True) * layers
     del graph
-    return {"us_per_step": ms * 1e3, "tokens_per_s": s.batch * s.seqlen / (ms * 1e-3),
-            "algorithmic_bytes": b, "hbm_frac": b / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
-            "layers": layers, "batch": s.batch, "graph": True}
+    out = {"us_per_step": ms * 1e3, "tokens_per_s": s.batch * s.seqlen / (ms * 1e-3),
+           "algorithmic_bytes": b, "hbm_frac": b / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+           "layers": layers, "batch": s.batch, "graph": True}
+    if conv_width:
+        out["conv_width"] = conv_width
+    return out
+
+
+def _conv_allblock(s: W.Shape, width: int, dev, pk) -> dict:
+    """Short convolution (+SiLU) of the all-block layer's four directions, the
+    noisy blocks continuing from the clean rows before them."""
+    dirs = [W.make_conv_dir(s, width, W.SEEDS[WORKLOAD], stream=i, device=dev) for i in range(4)]
+    outs = bd.conv_allblock(s, width, True, *dirs)
+    ms = _time(lambda: bd.conv_allblock(s, width, True, *dirs, outs=outs), dev, 20)
+    b = RL.conv_bytes(s, width, 4)
+    achieved = b / (ms * 1e-3) / 1e9
+    return {"us_per_call": ms * 1e3, "tokens_per_s": s.batch * s.seqlen / (ms * 1e-3), "width": width,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / pk["hbm_gbs"], "algorithmic_bytes": b,
+                         "algorithmic_flops": RL.conv_flops(s, width, 4)}}
 
 
 def _backward(s: W.Shape, dev, pk) -> dict:

@@ -25,6 +25,7 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "bdscan.h")
 
 BDSCAN_BF16, BDSCAN_FP32 = 0, 1
 BDSCAN_OP_PREFIX, BDSCAN_OP_BLOCK_STEP, BDSCAN_OP_ALLBLOCK, BDSCAN_OP_ALLBLOCK_BACKWARD = 0, 1, 2, 3
+BDSCAN_OP_CONV_PREFIX, BDSCAN_OP_CONV_ALLBLOCK = 4, 5
 STATUS = {0: "BDSCAN_OK", -1: "BDSCAN_ERR_INVALID_ARG", -2: "BDSCAN_ERR_UNSUPPORTED_SHAPE",
           -3: "BDSCAN_ERR_MISALIGNED", -4: "BDSCAN_ERR_WORKSPACE", -5: "BDSCAN_ERR_CUDA",
           -6: "BDSCAN_ERR_TIMEOUT", -7: "BDSCAN_ERR_SCRATCH_LIMIT"}
@@ -44,6 +45,10 @@ class bdscan_dir_t(ctypes.Structure):
 
 class bdscan_grad_t(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("dx", "ddt", "dB", "dC", "dA", "dD")]
+
+
+class bdscan_conv_t(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("x", "B", "C", "weight", "bias", "x_out", "B_out", "C_out")]
 
 
 class BdscanError(RuntimeError):
@@ -74,8 +79,11 @@ def lib() -> ctypes.CDLL:
             gp = ctypes.POINTER(bdscan_grad_t)
             L.bdscan_allblock_backward.argtypes = [sp, dp, dp, dp, dp, vp, vp, vp, vp, vp, gp, gp, gp, gp,
                                                    vp, vp, sz, vp]
+            cp, ci = ctypes.POINTER(bdscan_conv_t), ctypes.c_int
+            L.bdscan_conv_prefix.argtypes = [sp, ci, ci, cp, cp, vp, vp, vp]
+            L.bdscan_conv_allblock.argtypes = [sp, ci, ci, cp, cp, cp, cp, vp, vp]
             for fn in ("bdscan_prefix", "bdscan_block_step", "bdscan_allblock", "bdscan_allblock_backward",
-                       "bdscan_check_status", "bdscan_version"):
+                       "bdscan_conv_prefix", "bdscan_conv_allblock", "bdscan_check_status", "bdscan_version"):
                 getattr(L, fn).restype = ctypes.c_int
             L.bdscan_workspace_size.argtypes = [sp, ctypes.c_int]
             L.bdscan_workspace_size.restype = ctypes.c_size_t
@@ -118,6 +126,14 @@ def bdscan_allblock_backward(shape, cf, cr, nf, nr, h0, block_states, dy_clean, 
                              g_cf, g_cr, g_nf, g_nr, dh0, ws, ws_bytes, stream) -> int:
     return lib().bdscan_allblock_backward(shape, cf, cr, nf, nr, h0, block_states, dy_clean, dy_noisy,
                                           dstates, g_cf, g_cr, g_nf, g_nr, dh0, ws, ws_bytes, stream)
+
+
+def bdscan_conv_prefix(shape, width, silu, fwd, rev, conv_state_in, conv_state_out, stream) -> int:
+    return lib().bdscan_conv_prefix(shape, width, silu, fwd, rev, conv_state_in, conv_state_out, stream)
+
+
+def bdscan_conv_allblock(shape, width, silu, cf, cr, nf, nr, conv_state_in, stream) -> int:
+    return lib().bdscan_conv_allblock(shape, width, silu, cf, cr, nf, nr, conv_state_in, stream)
 
 
 def bdscan_block_step_noalloc(shape, fwd, rev, state_in, y, state_out, stream) -> int:
@@ -324,3 +340,78 @@ def allblock_backward(s: Shape, clean_fwd: dict, clean_rev: dict | None, noisy_f
                                   ws.numel(), _stream(dev, stream))
     _raise("bdscan_allblock_backward", rc)
     return grads, dh0
+
+
+# ----------------------------------------------------------------------------- short convolution
+CONV_KEYS = ("x", "B", "C")
+
+
+def conv_channels(s: Shape) -> int:
+    """Channels of the convolution: x's H*P, then B's and C's G*N each."""
+    return s.nheads * s.headdim + 2 * s.ngroups * s.dstate
+
+
+def c_conv(s: Shape, d: dict | None, width: int, device, out: dict | None = None):
+    """ctypes struct of one convolution direction.  ``d`` holds the pre-convolution
+    x, B, C (in_dtype), weight [Cx][width] and optionally bias [Cx] (fp32);
+    ``out`` the output tensors (allocated when None).  Returns (struct, out)."""
+    if d is None:
+        return None, None
+    tin = _DT[s.in_dtype][0]
+    B, L, H, P, N, G = s.batch, s.seqlen, s.nheads, s.headdim, s.dstate, s.ngroups
+    shapes = {"x": (B, L, H, P), "B": (B, L, G, N), "C": (B, L, G, N)}
+    for k in CONV_KEYS:
+        _check_tensor(k, d[k], shapes[k], tin, device)
+    cx = conv_channels(s)
+    _check_tensor("weight", d["weight"], (cx, width), torch.float32, device)
+    if d.get("bias") is not None:
+        _check_tensor("bias", d["bias"], (cx,), torch.float32, device)
+    if out is None:
+        out = {k: torch.empty(shapes[k], dtype=tin, device=device) for k in CONV_KEYS}
+    st = bdscan_conv_t(_ptr(d["x"]), _ptr(d["B"]), _ptr(d["C"]), _ptr(d["weight"]), _ptr(d.get("bias")),
+                       _ptr(out["x"]), _ptr(out["B"]), _ptr(out["C"]))
+    return st, out
+
+
+def _check_conv_state(name, t, s: Shape, width: int, device):
+    if t is not None:
+        _check_tensor(name, t, (s.batch, width - 1, conv_channels(s)), _DT[s.in_dtype][0], device)
+
+
+def conv_prefix(s: Shape, width: int, silu: bool, fwd: dict, rev: dict | None = None, state_in=None,
+                state_out=None, out_fwd=None, out_rev=None, stream=None):
+    """Short convolution (+SiLU) of one sequence: causal for ``fwd`` from
+    ``state_in`` ([B][width-1][Cx], None = zeros), anti-causal inside each
+    block for ``rev``.  ``state_out``: None, a tensor (may be ``state_in`` when
+    seqlen <= 32) or True (allocate).  Returns (fwd outputs, rev outputs or
+    None, state_out or None); outputs are dicts keyed x, B, C."""
+    dev = fwd["x"].device
+    cs = c_shape(s)
+    cf, out_fwd = c_conv(s, fwd, width, dev, out_fwd)
+    cr, out_rev = c_conv(s, rev, width, dev, out_rev)
+    _check_conv_state("state_in", state_in, s, width, dev)
+    if state_out is True:
+        state_out = torch.empty((s.batch, width - 1, conv_channels(s)), dtype=_DT[s.in_dtype][0], device=dev)
+    _check_conv_state("state_out", state_out, s, width, dev)
+    rc = bdscan_conv_prefix(ctypes.byref(cs), int(width), 1 if silu else 0, ctypes.byref(cf), _ref(cr),
+                            _ptr(state_in), _ptr(state_out), _stream(dev, stream))
+    _raise("bdscan_conv_prefix", rc)
+    return out_fwd, out_rev, state_out
+
+
+def conv_allblock(s: Shape, width: int, silu: bool, clean_fwd: dict, clean_rev: dict | None,
+                  noisy_fwd: dict, noisy_rev: dict | None, state_in=None, outs=None, stream=None):
+    """Short convolution of the all-block pass: the clean stream as in
+    ``conv_prefix``; every noisy block's forward convolution reads the clean
+    rows before it.  Returns four output dicts (None for absent directions)."""
+    dev = clean_fwd["x"].device
+    cs = c_shape(s)
+    dirs = [clean_fwd, clean_rev, noisy_fwd, noisy_rev]
+    outs = outs or [None] * 4
+    built = [c_conv(s, d, width, dev, o) for d, o in zip(dirs, outs)]
+    _check_conv_state("state_in", state_in, s, width, dev)
+    cd = [b[0] for b in built]
+    rc = bdscan_conv_allblock(ctypes.byref(cs), int(width), 1 if silu else 0, _ref(cd[0]), _ref(cd[1]),
+                              _ref(cd[2]), _ref(cd[3]), _ptr(state_in), _stream(dev, stream))
+    _raise("bdscan_conv_allblock", rc)
+    return [b[1] for b in built]

@@ -169,6 +169,8 @@ size_t bdscan_workspace_size(const bdscan_shape_t *shape, int op) {
 
 int bdscan_kernel_launches(const bdscan_shape_t *shape, int op) {
   if (check_shape(shape) != BDSCAN_OK) return -1;
+  if (op == BDSCAN_OP_CONV_PREFIX || op == BDSCAN_OP_CONV_ALLBLOCK)
+    return (shape->batch == 0 || shape->seqlen == 0) ? 0 : 1;
   if (op == BDSCAN_OP_ALLBLOCK_BACKWARD) {
     // backward kernel + a dB/dC and a dA/dD reduction per present direction
     // (2 or 4 directions; counted here for all four)
@@ -466,6 +468,154 @@ int bdscan_block_step_noalloc(const bdscan_shape_t *shape, const bdscan_dir_t *f
   // before they are read, so nothing else needs to start at zero.
   return bdscan_block_step(shape, fwd, rev, state_in, y, state_out, ws, BDSCAN_NOALLOC_SCRATCH_BYTES,
                            cuda_stream);
+}
+
+}  // extern "C"
+
+// ---- short convolution in front of the scan --------------------------------
+namespace {
+
+struct ConvSizes {
+  size_t x, bc, w, bias, state;
+  int64_t Cx;
+};
+
+ConvSizes conv_sizes(const bdscan_shape_t *s, int width) {
+  const size_t in = s->in_dtype == BDSCAN_BF16 ? 2 : 4;
+  const size_t B = (size_t)s->batch, L = (size_t)s->seqlen, H = (size_t)s->nheads,
+               P = (size_t)s->headdim, N = (size_t)s->dstate, G = (size_t)s->ngroups;
+  ConvSizes z;
+  z.Cx = (int64_t)(H * P + 2 * G * N);
+  z.x = B * L * H * P * in;
+  z.bc = B * L * G * N * in;
+  z.w = (size_t)z.Cx * (size_t)width * 4;
+  z.bias = (size_t)z.Cx * 4;
+  z.state = B * (size_t)(width - 1) * (size_t)z.Cx * in;
+  return z;
+}
+
+int check_conv_shape(const bdscan_shape_t *shape, int width) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (width < 1 || width > 4) return BDSCAN_ERR_UNSUPPORTED_SHAPE;
+  // B and C rows must be whole 4-channel vectors
+  if ((shape->ngroups * shape->dstate) % 4) return BDSCAN_ERR_UNSUPPORTED_SHAPE;
+  return BDSCAN_OK;
+}
+
+// Validates one direction of the convolution; appends its ranges.
+int check_conv_dir(const bdscan_conv_t *d, const ConvSizes &z, std::vector<Range> &ins,
+                   std::vector<Range> &outs) {
+  if (!d || !d->weight) return BDSCAN_ERR_INVALID_ARG;
+  if (z.x && (!d->x || !d->B || !d->C || !d->x_out || !d->B_out || !d->C_out)) return BDSCAN_ERR_INVALID_ARG;
+  const void *ptrs[] = {d->x, d->B, d->C, d->weight, d->bias, d->x_out, d->B_out, d->C_out};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return BDSCAN_ERR_MISALIGNED;
+  ins.push_back(range_of(d->x, z.x));
+  ins.push_back(range_of(d->B, z.bc));
+  ins.push_back(range_of(d->C, z.bc));
+  ins.push_back(range_of(d->weight, z.w));
+  if (d->bias) ins.push_back(range_of(d->bias, z.bias));
+  outs.push_back(range_of(d->x_out, z.x));
+  outs.push_back(range_of(d->B_out, z.bc));
+  outs.push_back(range_of(d->C_out, z.bc));
+  return BDSCAN_OK;
+}
+
+bdscan::ConvDirArgs to_conv_args(const bdscan_conv_t *d) {
+  bdscan::ConvDirArgs a{};
+  if (d) {
+    a.x = d->x; a.B = d->B; a.C = d->C; a.weight = d->weight; a.bias = d->bias;
+    a.x_out = d->x_out; a.B_out = d->B_out; a.C_out = d->C_out;
+  }
+  return a;
+}
+
+bdscan::ConvArgs conv_base(const bdscan_shape_t *s, int width, int silu) {
+  bdscan::ConvArgs a{};
+  a.Bsz = s->batch; a.L = s->seqlen; a.H = s->nheads; a.P = s->headdim; a.N = s->dstate;
+  a.G = s->ngroups; a.T = s->block_len; a.W = width;
+  a.in_bf16 = s->in_dtype == BDSCAN_BF16;
+  a.silu = silu != 0;
+  return a;
+}
+
+int conv_launch(const bdscan::ConvArgs &a, const ConvSizes &z, cudaStream_t stream) {
+  if (a.Bsz == 0) return BDSCAN_OK;
+  if (a.L == 0) {
+    // nothing to convolve: the new conv state is the old one (or zeros)
+    if (a.state_out && a.state_out != a.state_in && z.state) {
+      cudaError_t e = a.state_in ? cudaMemcpyAsync(a.state_out, a.state_in, z.state, cudaMemcpyDeviceToDevice, stream)
+                                 : cudaMemsetAsync(a.state_out, 0, z.state, stream);
+      if (e != cudaSuccess) return BDSCAN_ERR_CUDA;
+    }
+    return BDSCAN_OK;
+  }
+  cudaError_t e = bdscan::launch_conv(a, stream);
+  if (e != cudaSuccess) {
+    const char *v = std::getenv("BDSCAN_VERBOSE");
+    if (v && v[0] == '1') std::fprintf(stderr, "libbdscan: conv launch failed: %s\n", cudaGetErrorString(e));
+    return BDSCAN_ERR_CUDA;
+  }
+  return BDSCAN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int bdscan_conv_prefix(const bdscan_shape_t *shape, int width, int silu, const bdscan_conv_t *fwd,
+                       const bdscan_conv_t *rev, const void *conv_state_in, void *conv_state_out,
+                       void *cuda_stream) {
+  int rc = check_conv_shape(shape, width);
+  if (rc) return rc;
+  const ConvSizes z = conv_sizes(shape, width);
+  std::vector<Range> ins, outs;
+  if ((rc = check_conv_dir(fwd, z, ins, outs))) return rc;
+  if (rev && (rc = check_conv_dir(rev, z, ins, outs))) return rc;
+  if ((conv_state_in && !aligned16(conv_state_in)) || (conv_state_out && !aligned16(conv_state_out)))
+    return BDSCAN_ERR_MISALIGNED;
+  const Range rin = range_of(conv_state_in, z.state);
+  if (conv_state_out && conv_state_out == conv_state_in) {
+    // in place: each thread reads its state rows before it writes them, which
+    // needs the whole sequence in one tile
+    if (shape->seqlen > 32) return BDSCAN_ERR_INVALID_ARG;
+    for (const Range &r : ins)
+      if (overlaps(rin, r)) return BDSCAN_ERR_INVALID_ARG;
+  }
+  if (conv_state_in) ins.push_back(rin);
+  if (conv_state_out && conv_state_out != conv_state_in) outs.push_back(range_of(conv_state_out, z.state));
+  if ((rc = check_outputs(ins, outs))) return rc;
+  bdscan::ConvArgs a = conv_base(shape, width, silu);
+  a.dir[0] = to_conv_args(fwd);
+  a.dir[1] = to_conv_args(rev);
+  a.state_in = conv_state_in;
+  a.state_out = conv_state_out;
+  return conv_launch(a, z, static_cast<cudaStream_t>(cuda_stream));
+}
+
+int bdscan_conv_allblock(const bdscan_shape_t *shape, int width, int silu,
+                         const bdscan_conv_t *clean_fwd, const bdscan_conv_t *clean_rev,
+                         const bdscan_conv_t *noisy_fwd, const bdscan_conv_t *noisy_rev,
+                         const void *conv_state_in, void *cuda_stream) {
+  int rc = check_conv_shape(shape, width);
+  if (rc) return rc;
+  const ConvSizes z = conv_sizes(shape, width);
+  std::vector<Range> ins, outs;
+  if ((rc = check_conv_dir(clean_fwd, z, ins, outs))) return rc;
+  if (clean_rev && (rc = check_conv_dir(clean_rev, z, ins, outs))) return rc;
+  if ((rc = check_conv_dir(noisy_fwd, z, ins, outs))) return rc;
+  if (noisy_rev && (rc = check_conv_dir(noisy_rev, z, ins, outs))) return rc;
+  if (conv_state_in && !aligned16(conv_state_in)) return BDSCAN_ERR_MISALIGNED;
+  if (conv_state_in) ins.push_back(range_of(conv_state_in, z.state));
+  if ((rc = check_outputs(ins, outs))) return rc;
+  bdscan::ConvArgs a = conv_base(shape, width, silu);
+  a.dir[0] = to_conv_args(clean_fwd);
+  a.dir[1] = to_conv_args(clean_rev);
+  a.dir[2] = to_conv_args(noisy_fwd);
+  a.dir[3] = to_conv_args(noisy_rev);
+  a.state_in = conv_state_in;
+  return conv_launch(a, z, static_cast<cudaStream_t>(cuda_stream));
 }
 
 }  // extern "C"

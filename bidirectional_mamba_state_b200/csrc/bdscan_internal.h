@@ -64,4 +64,21 @@ size_t bwd_smem_bytes(int64_t P, int64_t N, int64_t T);
 size_t bwd_workspace_bytes(int64_t Bsz, int64_t L, int64_t H, int64_t N);
 cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream);
 
+// Short convolution (+SiLU) in front of the scan.
+struct ConvDirArgs {
+  const void *x, *B, *C;         // pre-convolution inputs (x == nullptr: absent direction)
+  const float *weight, *bias;    // [Cx][W], [Cx] or nullptr
+  void *x_out, *B_out, *C_out;
+};
+struct ConvArgs {
+  int64_t Bsz, L, H, P, N, G, T;
+  int W;
+  bool in_bf16, silu;
+  ConvDirArgs dir[4];  // clean (or prefix) fwd, its rev, noisy fwd, noisy rev
+  const void *state_in;  // [B][W-1][Cx] or nullptr
+  void *state_out;       // [B][W-1][Cx] or nullptr (dir[0]'s last rows)
+};
+int conv_tile(const ConvArgs &a);
+cudaError_t launch_conv(const ConvArgs &a, cudaStream_t stream);
+
 }  // namespace bdscan

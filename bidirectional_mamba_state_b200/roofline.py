@@ -85,3 +85,30 @@ def allblock_backward_flops(s: Shape) -> int:
     tpn = 2 * T * P * N
     per = (gram + intra + 5 * tpn) + (gram + intra + 3 * tpn) + 2 * (gram + intra)
     return B * H * K * per
+
+
+def conv_channels(s: Shape) -> int:
+    return s.nheads * s.headdim + 2 * s.ngroups * s.dstate
+
+
+def conv_dir_bytes(s: Shape, width: int) -> int:
+    """One direction of the short convolution: pre-convolution rows read once,
+    outputs written once (input dtype), taps and bias (fp32)."""
+    cx = conv_channels(s)
+    return 2 * _elt(s.in_dtype) * s.batch * s.seqlen * cx + 4 * cx * (width + 1)
+
+
+def conv_state_bytes(s: Shape, width: int) -> int:
+    return _elt(s.in_dtype) * s.batch * (width - 1) * conv_channels(s)
+
+
+def conv_bytes(s: Shape, width: int, ndir: int, state_in: bool = False, state_out: bool = False) -> int:
+    """A convolution call over ``ndir`` directions (halo rows a tile shares
+    with its neighbour, or a noisy block with the clean stream, are re-reads
+    and not counted)."""
+    return ndir * conv_dir_bytes(s, width) + conv_state_bytes(s, width) * (int(state_in) + int(state_out))
+
+
+def conv_flops(s: Shape, width: int, ndir: int) -> int:
+    """2 flops per tap per output (SiLU not counted)."""
+    return ndir * 2 * width * s.batch * s.seqlen * conv_channels(s)

@@ -10,6 +10,10 @@ Value distributions (the workloads' stated recipe):
   u ~ N(-3, 0.5);  A_h = -exp(U(0, ln 16)) (fp32);  D_h ~ N(0, 1) (fp32);
   z ~ N(0, 1) (gated runs only).  The reverse direction and the noisy stream
   are independent draws.
+Short convolution in front of the scan: pre-convolution x, B, C ~ N(0, 1)
+  (the input projection's unit-scale outputs); taps and bias ~ U(-1/sqrt(W),
+  1/sqrt(W)) (the usual initialisation bound of a depthwise filter of W taps,
+  fan-in W); conv state ~ N(0, 1) rounded to the input dtype.
 """
 from __future__ import annotations
 
@@ -20,7 +24,8 @@ import torch
 
 # stream ids
 CLEAN_FWD, CLEAN_REV, NOISY_FWD, NOISY_REV = 0, 1, 2, 3
-_TENSOR_IDS = {"x": 0, "dt": 1, "B": 2, "C": 3, "z": 4, "A": 5, "D": 6, "h0": 7}
+_TENSOR_IDS = {"x": 0, "dt": 1, "B": 2, "C": 3, "z": 4, "A": 5, "D": 6, "h0": 7,
+               "conv_x": 8, "conv_B": 9, "conv_C": 10, "conv_w": 11, "conv_b": 12, "conv_state": 13}
 
 
 @dataclass(frozen=True)
@@ -130,3 +135,32 @@ def sub_batch_block(d: dict, t0: int, t1: int) -> dict:
         else:
             out[k] = v[:, t0:t1].contiguous()
     return out
+
+
+def make_conv_dir(shape: Shape, width: int = 4, seed: int = 0, layer: int = 0, stream: int = CLEAN_FWD,
+                  device="cpu", bias: bool = True) -> dict:
+    """Draw one direction's short-convolution inputs: pre-convolution x, B, C
+    (input dtype), weight [H*P + 2*G*N][width] and bias (fp32)."""
+    Bsz, L, H, P, N, G = (shape.batch, shape.seqlen, shape.nheads, shape.headdim,
+                          shape.dstate, shape.ngroups)
+    dev = torch.device(device)
+    dt_in = _dtype(shape.in_dtype)
+    cx = H * P + 2 * G * N
+    d = {"x": _normal((Bsz, L, H, P), 0.0, 1.0, _gen(seed, layer, stream, "conv_x", dev), dev).to(dt_in),
+         "B": _normal((Bsz, L, G, N), 0.0, 1.0, _gen(seed, layer, stream, "conv_B", dev), dev).to(dt_in),
+         "C": _normal((Bsz, L, G, N), 0.0, 1.0, _gen(seed, layer, stream, "conv_C", dev), dev).to(dt_in)}
+    bound = 1.0 / math.sqrt(width)
+    gw = _gen(seed, layer, stream, "conv_w", dev)
+    d["weight"] = (torch.rand((cx, width), generator=gw, device=dev, dtype=torch.float32) * 2 - 1) * bound
+    if bias:
+        gb = _gen(seed, layer, stream, "conv_b", dev)
+        d["bias"] = (torch.rand((cx,), generator=gb, device=dev, dtype=torch.float32) * 2 - 1) * bound
+    return d
+
+
+def make_conv_state(shape: Shape, width: int = 4, seed: int = 0, layer: int = 0, device="cpu") -> torch.Tensor:
+    """A random conv state [B, width-1, H*P + 2*G*N] in the input dtype."""
+    dev = torch.device(device)
+    cx = shape.nheads * shape.headdim + 2 * shape.ngroups * shape.dstate
+    g = _gen(seed, layer, 9, "conv_state", dev)
+    return _normal((shape.batch, width - 1, cx), 0.0, 1.0, g, dev).to(_dtype(shape.in_dtype))

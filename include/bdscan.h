@@ -66,6 +66,8 @@ extern "C" {
 #define BDSCAN_OP_BLOCK_STEP 1
 #define BDSCAN_OP_ALLBLOCK 2
 #define BDSCAN_OP_ALLBLOCK_BACKWARD 3
+#define BDSCAN_OP_CONV_PREFIX 4   /* no workspace (bdscan_workspace_size returns 0) */
+#define BDSCAN_OP_CONV_ALLBLOCK 5 /* no workspace */
 
 /* Problem shape.  Supported: batch >= 0, seqlen >= 0, seqlen % block_len == 0,
  * 1 <= block_len <= 32 or block_len % 32 == 0 (<= 256), chunk_len % block_len
@@ -168,6 +170,70 @@ int bdscan_allblock_backward(const bdscan_shape_t *shape, const bdscan_dir_t *cl
                              const bdscan_grad_t *g_clean_fwd, const bdscan_grad_t *g_clean_rev,
                              const bdscan_grad_t *g_noisy_fwd, const bdscan_grad_t *g_noisy_rev,
                              float *dh0, void *ws, size_t ws_bytes, void *cuda_stream);
+
+/* ---- Short convolution in front of the scan ---------------------------------
+ *
+ * In a Mamba-2 layer the scan's x, B and C are not the input projection's
+ * outputs themselves: each of their channels first goes through a short
+ * depthwise convolution over time and a SiLU.  The layer's cache for the
+ * block-diffusion decoder therefore keeps, beside the scan state, the
+ * convolution's state: the last width-1 pre-convolution rows of the forward
+ * stream ("Training Hybrid Block Diffusion Language Models with Partial
+ * Bidirectionality", the paragraph after eq. (14) on the cache object of a
+ * Mamba layer).  The forward direction's convolution is causal; the reverse
+ * direction's is anti-causal ("Breaking the Bottleneck with DiffuApriel",
+ * section 3.2, after eq. (5)) and, like its scan, confined to the block.
+ *
+ * Per channel c of one direction, with u the pre-convolution input, v the
+ * output, W = width, w[c][0..W-1] the taps and s(v) = v / (1 + exp(-v)):
+ *   forward:  v_t = s(bias[c] + sum_j w[c][j] * u_{t-(W-1)+j})
+ *             where u_{t'} for t' < 0 is row W-1+t' of the conv state (zeros
+ *             when no state is given); tokens earlier than the state are 0.
+ *   reverse:  v_t = s(bias[c] + sum_j w[c][j] * u_{t+(W-1)-j})
+ *             where u_{t'} = 0 for t' past the end of t's block: the forward
+ *             rule applied to the block read right to left, from zeros.
+ * (s is skipped when `silu` is 0.)
+ *
+ * Channels: the x channels (h, p) in order, then B's (g, n), then C's (g, n):
+ * Cx = H*P + 2*G*N channels.  dt and z are not convolved.
+ * Layouts: inputs and outputs have the layouts of bdscan_dir_t's x, B, C and
+ * the element type in_dtype; weight [Cx][W] fp32; bias [Cx] fp32 or NULL;
+ * conv state [B][W-1][Cx] in_dtype (rows oldest first; row W-2 is the token
+ * just before the sequence).
+ * Supported: 1 <= width <= 4 (else BDSCAN_ERR_UNSUPPORTED_SHAPE), G*N a
+ * multiple of 4, every pointer 16-byte aligned.  Each output is computed in
+ * fp32 (taps applied oldest row first, bias first) from the rounded inputs and
+ * rounded once to in_dtype.  The calls take no workspace; one kernel launch. */
+typedef struct {
+    const void *x, *B, *C;  /* pre-convolution inputs */
+    const float *weight;    /* [Cx][width] */
+    const float *bias;      /* [Cx] or NULL (zeros) */
+    void *x_out, *B_out, *C_out;
+} bdscan_conv_t;
+
+/* bdscan_conv_prefix -- the convolution of one sequence (prefill, commit, or
+ * one denoising step of the active block with shape->seqlen == block_len).
+ *   fwd             forward direction (required)
+ *   rev             reverse direction (anti-causal inside each block) or NULL
+ *   conv_state_in   [B][W-1][Cx] or NULL (zeros): rows before token 0
+ *   conv_state_out  [B][W-1][Cx] or NULL: the last W-1 rows of the forward
+ *                   stream (conv_state_in followed by fwd's inputs); may
+ *                   equal conv_state_in only when seqlen <= 32
+ * Outputs must not overlap any input or each other (except the in-place
+ * state above). */
+int bdscan_conv_prefix(const bdscan_shape_t *shape, int width, int silu, const bdscan_conv_t *fwd,
+                       const bdscan_conv_t *rev, const void *conv_state_in, void *conv_state_out,
+                       void *cuda_stream);
+
+/* bdscan_conv_allblock -- the convolution of the all-block training pass: the
+ * clean stream as by bdscan_conv_prefix; each noisy block k's forward
+ * convolution continues from the clean stream's rows before the block (the
+ * conv state at the end of block k-1; conv_state_in for k = 0), the noisy
+ * reverse stays inside the block.  clean_rev / noisy_rev may be NULL. */
+int bdscan_conv_allblock(const bdscan_shape_t *shape, int width, int silu,
+                         const bdscan_conv_t *clean_fwd, const bdscan_conv_t *clean_rev,
+                         const bdscan_conv_t *noisy_fwd, const bdscan_conv_t *noisy_rev,
+                         const void *conv_state_in, void *cuda_stream);
 
 /* Workspace bytes an operation needs for this shape (>= 256: the first 256
  * bytes hold the device status word).  Returns 0 for an invalid shape/op. */

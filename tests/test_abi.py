@@ -193,3 +193,43 @@ def test_backward_validation():
     assert _backward(ws_bytes=64) == -4           # workspace too small
     # a block whose shared-memory plan does not fit one CTA
     assert _backward(s_kw=dict(headdim=128, dstate=256, block_len=64, chunk_len=64, seqlen=128)) == -2
+
+
+def _fake_conv(base, step=0x100000):
+    p = [base + i * step for i in range(8)]
+    return bd.bdscan_conv_t(*p)
+
+
+def _conv(s_kw=None, width=4, fwd=None, rev=None, st_in=None, st_out=None):
+    s = bd.c_shape(Shape(**_base(**(s_kw or {}))))
+    fwd = _fake_conv(0x10000000) if fwd is None else fwd
+    return bd.bdscan_conv_prefix(ctypes.byref(s), width, 1, ctypes.byref(fwd) if fwd != "null" else None,
+                                 ctypes.byref(rev) if rev is not None else None, st_in, st_out, None)
+
+
+def test_conv_validation():
+    s = bd.c_shape(Shape(**_base()))
+    for op in (bd.BDSCAN_OP_CONV_PREFIX, bd.BDSCAN_OP_CONV_ALLBLOCK):
+        assert bd.bdscan_workspace_size(ctypes.byref(s), op) == 0      # no workspace
+        assert bd.bdscan_kernel_launches(ctypes.byref(s), op) == 1
+    assert _conv(width=0) == -2 and _conv(width=5) == -2                # 1 <= width <= 4
+    assert _conv(s_kw=dict(dstate=2, ngroups=1, nheads=4)) == -2        # G*N not a multiple of 4
+    assert _conv(fwd="null") == -1
+    d = _fake_conv(0x10000000)
+    d.weight = None
+    assert _conv(fwd=d) == -1                                           # taps required
+    d = _fake_conv(0x10000000)
+    d.C_out = d.C_out + 8
+    assert _conv(fwd=d) == -3                                           # misaligned output
+    d = _fake_conv(0x10000000)
+    d.x_out = d.x                                                       # output over an input
+    assert _conv(fwd=d) == -1
+    assert _conv(st_in=0x80000000, st_out=0x80000100) == -1            # partial state overlap
+    assert _conv(st_in=0x80000000, st_out=0x80000000) == -1            # in place needs seqlen <= 32
+    assert _conv(st_in=0x80000004) == -3                                # misaligned state
+    r = _fake_conv(0x20000000)
+    r.x_out = _fake_conv(0x10000000).x_out                              # two directions write one buffer
+    assert _conv(rev=r) == -1
+    cf, nf = _fake_conv(0x10000000), _fake_conv(0x20000000)
+    rc = bd.bdscan_conv_allblock(ctypes.byref(s), 4, 1, ctypes.byref(cf), None, None, None, None, None)
+    assert rc == -1                                                     # noisy_fwd required
