@@ -14,8 +14,8 @@
 // threads take consecutive vectors of the same token row, so each warp load or
 // store is 256 or 512 contiguous bytes.  The taps of the thread's channels, the bias
 // and the last W-1 rows stay in registers while the thread walks its tile
-// (forward: oldest to newest; reverse: newest to oldest), loading
-// kConvBatchBytes of rows ahead of their use.
+// (forward: oldest to newest; reverse: newest to oldest) in batches of 64
+// bytes of rows whose loads are all issued before their first use.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -27,7 +27,6 @@ namespace bdscan {
 namespace {
 
 constexpr int kConvThreads = 256;
-constexpr int kConvBatchBytes = 64;  // input bytes a thread loads ahead of their use
 
 struct ConvJob {
   const void *u[3];     // x, B, C inputs of this direction
@@ -102,13 +101,84 @@ __device__ __forceinline__ float act(float v, int silu) {
   return silu ? __fdividef(v, 1.0f + __expf(-v)) : v;
 }
 
+// NB consecutive rows (already loaded) of a causal convolution, written to
+// pd[0], pd[step], ...: the window (rows before the batch, oldest first) is
+// extended by the batch and its last W-1 rows kept.
+template <class Vt, int NB>
+__device__ __forceinline__ void load_rows(typename Vt::Raw (&raw)[NB], const typename Vt::Raw *ps, int64_t step) {
+#pragma unroll
+  for (int k = 0; k < NB; ++k) raw[k] = __ldg(ps + k * step);
+}
+
+template <class Vt, int W, int NB>
+__device__ __forceinline__ void rows_fwd(const typename Vt::Raw (&raw)[NB], typename Vt::Raw *pd, int64_t step,
+                                         const float (&w)[W][Vt::V], const float (&bias)[Vt::V],
+                                         float (&win)[W > 1 ? W - 1 : 1][Vt::V], int silu) {
+  constexpr int V = Vt::V;
+  float uu[W - 1 + NB][V];
+#pragma unroll
+  for (int m = 0; m < W - 1; ++m)
+#pragma unroll
+    for (int c = 0; c < V; ++c) uu[m][c] = win[m][c];
+#pragma unroll
+  for (int k = 0; k < NB; ++k) Vt::unpack(raw[k], uu[W - 1 + k]);
+#pragma unroll
+  for (int k = 0; k < NB; ++k) {
+    float o[V];
+#pragma unroll
+    for (int c = 0; c < V; ++c) {
+      float acc = bias[c];
+#pragma unroll
+      for (int j = 0; j < W; ++j) acc = fmaf(w[j][c], uu[k + j][c], acc);
+      o[c] = act(acc, silu);
+    }
+    pd[k * step] = Vt::pack(o);
+  }
+#pragma unroll
+  for (int m = 0; m < W - 1; ++m)
+#pragma unroll
+    for (int c = 0; c < V; ++c) win[m][c] = uu[NB + m][c];
+}
+
+// NB consecutive rows (already loaded, ascending) of an anti-causal
+// convolution, the window holding the W-1 rows above the batch (nearest first).
+template <class Vt, int W, int NB>
+__device__ __forceinline__ void rows_rev(const typename Vt::Raw (&raw)[NB], typename Vt::Raw *pd, int64_t step,
+                                         const float (&w)[W][Vt::V], const float (&bias)[Vt::V],
+                                         float (&win)[W > 1 ? W - 1 : 1][Vt::V], int silu) {
+  constexpr int V = Vt::V;
+  float uu[NB + W - 1][V];  // ascending tokens: the batch, then the window
+#pragma unroll
+  for (int k = 0; k < NB; ++k) Vt::unpack(raw[k], uu[k]);
+#pragma unroll
+  for (int m = 0; m < W - 1; ++m)
+#pragma unroll
+    for (int c = 0; c < V; ++c) uu[NB + m][c] = win[m][c];
+#pragma unroll
+  for (int k = 0; k < NB; ++k) {
+    float o[V];
+#pragma unroll
+    for (int c = 0; c < V; ++c) {
+      float acc = bias[c];
+#pragma unroll
+      for (int j = 0; j < W; ++j) acc = fmaf(w[j][c], uu[k + W - 1 - j][c], acc);
+      o[c] = act(acc, silu);
+    }
+    pd[k * step] = Vt::pack(o);
+  }
+#pragma unroll
+  for (int m = 0; m < W - 1; ++m)
+#pragma unroll
+    for (int c = 0; c < V; ++c) win[m][c] = uu[m][c];
+}
+
 template <typename E, int W>
 __global__ void __launch_bounds__(kConvThreads, 2) bd_conv_kernel(const __grid_constant__ ConvParams p) {
   using Vt = Vec<E>;
   using Raw = typename Vt::Raw;
   constexpr int V = Vt::V;
-  constexpr int kConvBatch = kConvBatchBytes / static_cast<int>(sizeof(Raw));
   constexpr int WH = W > 1 ? W - 1 : 1;  // window rows (at least one, unused when W == 1)
+  constexpr int NBM = sizeof(Raw) == 8 ? 8 : 4;  // rows per batch: 64 bytes of loads in flight
   const ConvJob &J = p.job[blockIdx.y];
   const int64_t item = static_cast<int64_t>(blockIdx.x) * kConvThreads + threadIdx.x;
   if (item >= static_cast<int64_t>(p.Bsz) * J.tiles * p.nvec) return;
@@ -161,6 +231,7 @@ __global__ void __launch_bounds__(kConvThreads, 2) bd_conv_kernel(const __grid_c
   const int64_t t0 = static_cast<int64_t>(tile) * J.tile;
   const Raw zero = Vt::zero();
   float win[WH][V];
+  const int64_t step = rowv;  // one token row, in vectors
 
   if (J.mode != 2) {
     // ---- causal: window = rows t-(W-1) .. t-1, oldest first
@@ -178,33 +249,35 @@ __global__ void __launch_bounds__(kConvThreads, 2) bd_conv_kernel(const __grid_c
         r = st_in[st_at(static_cast<int>(W - 1 + tp))];
       Vt::unpack(r, win[i]);
     }
-    for (int64_t tb = t0; tb < t1; tb += kConvBatch) {
-      Raw raw[kConvBatch];
+    const Raw *ps = src + at(t0);
+    Raw *pd = dst + at(t0);
+    int64_t n = t1 - t0;
+    if (n >= NBM) {
+      // the next batch's loads are in flight while this batch is computed
+      Raw cur[NBM];
+      load_rows<Vt, NBM>(cur, ps, step);
+      for (;;) {
+        n -= NBM;
+        ps += NBM * step;
+        Raw nxt[NBM];
+        if (n >= NBM) load_rows<Vt, NBM>(nxt, ps, step);
+        rows_fwd<Vt, W, NBM>(cur, pd, step, w, bias, win, p.silu);
+        pd += NBM * step;
+        if (n < NBM) break;
 #pragma unroll
-      for (int k = 0; k < kConvBatch; ++k) raw[k] = tb + k < t1 ? __ldg(src + at(tb + k)) : zero;
-#pragma unroll
-      for (int k = 0; k < kConvBatch; ++k) {
-        if (tb + k < t1) {
-          float u[V], o[V];
-          Vt::unpack(raw[k], u);
-#pragma unroll
-          for (int c = 0; c < V; ++c) {
-            float acc = bias[c];
-#pragma unroll
-            for (int j = 0; j < W - 1; ++j) acc = fmaf(w[j][c], win[j][c], acc);
-            o[c] = act(fmaf(w[W - 1][c], u[c], acc), p.silu);
-          }
-          dst[at(tb + k)] = Vt::pack(o);
-#pragma unroll
-          for (int j = 0; j + 1 < W - 1; ++j)
-#pragma unroll
-            for (int c = 0; c < V; ++c) win[j][c] = win[j + 1][c];
-          if (W > 1) {
-#pragma unroll
-            for (int c = 0; c < V; ++c) win[WH - 1][c] = u[c];
-          }
-        }
+        for (int k = 0; k < NBM; ++k) cur[k] = nxt[k];
       }
+    }
+    if (NBM > 4 && n >= 4) {
+      Raw r4[4];
+      load_rows<Vt, 4>(r4, ps, step);
+      rows_fwd<Vt, W, 4>(r4, pd, step, w, bias, win, p.silu);
+      n -= 4; ps += 4 * step; pd += 4 * step;
+    }
+    for (; n > 0; --n, ps += step, pd += step) {
+      Raw r1[1];
+      load_rows<Vt, 1>(r1, ps, step);
+      rows_fwd<Vt, W, 1>(r1, pd, step, w, bias, win, p.silu);
     }
     // the window now holds the stream's last W-1 rows (exact copies of inputs
     // or of state rows, so packing them back is lossless)
@@ -221,33 +294,37 @@ __global__ void __launch_bounds__(kConvThreads, 2) bd_conv_kernel(const __grid_c
       const int64_t tp = t1 + i;
       Vt::unpack(tp < bend ? __ldg(src + at(tp)) : zero, win[i]);
     }
-    for (int64_t tb = t1 - 1; tb >= t0; tb -= kConvBatch) {
-      Raw raw[kConvBatch];
+    // walk down from the tile's end: each batch covers the NB rows below ps
+    const Raw *ps = src + at(t1);
+    Raw *pd = dst + at(t1);
+    int64_t n = t1 - t0;
+    if (n >= NBM) {
+      Raw cur[NBM];
+      ps -= NBM * step;
+      load_rows<Vt, NBM>(cur, ps, step);
+      for (;;) {
+        n -= NBM;
+        Raw nxt[NBM];
+        if (n >= NBM) load_rows<Vt, NBM>(nxt, ps - NBM * step, step);
+        pd -= NBM * step;
+        rows_rev<Vt, W, NBM>(cur, pd, step, w, bias, win, p.silu);
+        if (n < NBM) break;
+        ps -= NBM * step;
 #pragma unroll
-      for (int k = 0; k < kConvBatch; ++k) raw[k] = tb - k >= t0 ? __ldg(src + at(tb - k)) : zero;
-#pragma unroll
-      for (int k = 0; k < kConvBatch; ++k) {
-        if (tb - k >= t0) {
-          float u[V], o[V];
-          Vt::unpack(raw[k], u);
-#pragma unroll
-          for (int c = 0; c < V; ++c) {
-            float acc = bias[c];
-#pragma unroll
-            for (int j = 0; j < W - 1; ++j) acc = fmaf(w[j][c], win[W - 2 - j][c], acc);
-            o[c] = act(fmaf(w[W - 1][c], u[c], acc), p.silu);
-          }
-          dst[at(tb - k)] = Vt::pack(o);
-#pragma unroll
-          for (int j = W - 2; j >= 1; --j)
-#pragma unroll
-            for (int c = 0; c < V; ++c) win[j][c] = win[j - 1][c];
-          if (W > 1) {
-#pragma unroll
-            for (int c = 0; c < V; ++c) win[0][c] = u[c];
-          }
-        }
+        for (int k = 0; k < NBM; ++k) cur[k] = nxt[k];
       }
+    }
+    if (NBM > 4 && n >= 4) {
+      Raw r4[4];
+      ps -= 4 * step; pd -= 4 * step; n -= 4;
+      load_rows<Vt, 4>(r4, ps, step);
+      rows_rev<Vt, W, 4>(r4, pd, step, w, bias, win, p.silu);
+    }
+    for (; n > 0; --n) {
+      Raw r1[1];
+      ps -= step; pd -= step;
+      load_rows<Vt, 1>(r1, ps, step);
+      rows_rev<Vt, W, 1>(r1, pd, step, w, bias, win, p.silu);
     }
   }
 }
