@@ -344,23 +344,39 @@ def _time(fn, dev, reps, warm=3):
     return e0.elapsed_time(e1) / reps
 
 
-def run_extra(dev, pk) -> dict:
+EXTRA = {
+    "block_step_700m_b1_24layers": lambda dev, pk: _step_stack(W.WORKLOADS["700m_step"], 24, dev, pk),
+    "block_step_3b_b1_40layers": lambda dev, pk: _step_stack(W.WORKLOADS["3b_step_b1"], 40, dev, pk),
+    "block_step_3b_b64_40layers": lambda dev, pk: _step_stack(W.WORKLOADS["3b_step_b64"], 40, dev, pk),
+    "prefill_700m_8k_per_layer": lambda dev, pk: _prefill(W.WORKLOADS["700m_prefill_8k"], dev, pk),
+    "allblock_backward_87m": lambda dev, pk: _backward(W.WORKLOADS["87m_allblock"], dev, pk),
+    "conv_allblock_87m": lambda dev, pk: _conv_allblock(W.WORKLOADS["87m_allblock"], 4, dev, pk),
+    "conv_block_step_700m_b1_24layers": lambda dev, pk: _step_stack(W.WORKLOADS["700m_step"], 24, dev, pk,
+                                                                    conv_width=4),
+}
+
+
+def run_extra(dev, pk, only=None) -> dict:
     """Secondary lines: the denoising step (block_step) over a layer stack captured
-    in one CUDA graph, and prefill of the 700M layer.  Median of 20 graph
-    replays after 5 warm-ups (the pages' own methodology)."""
+    in one CUDA graph, prefill of the 700M layer, the all-block backward and the
+    short convolution.  Median of 20 graph replays after 5 warm-ups (the pages'
+    own methodology) for the stacks; CUDA-event means for the rest."""
     out = {}
     try:
-        out["block_step_700m_b1_24layers"] = _step_stack(W.WORKLOADS["700m_step"], 24, dev, pk)
-        out["block_step_3b_b1_40layers"] = _step_stack(W.WORKLOADS["3b_step_b1"], 40, dev, pk)
-        out["block_step_3b_b64_40layers"] = _step_stack(W.WORKLOADS["3b_step_b64"], 40, dev, pk)
-        out["prefill_700m_8k_per_layer"] = _prefill(W.WORKLOADS["700m_prefill_8k"], dev, pk)
-        out["allblock_backward_87m"] = _backward(W.WORKLOADS["87m_allblock"], dev, pk)
-        out["conv_allblock_87m"] = _conv_allblock(W.WORKLOADS["87m_allblock"], 4, dev, pk)
-        out["conv_block_step_700m_b1_24layers"] = _step_stack(W.WORKLOADS["700m_step"], 24, dev, pk,
-                                                              conv_width=4)
+        for name, fn in EXTRA.items():
+            if only is None or name == only:
+                out[name] = fn(dev, pk)
     except Exception as e:  # report, never hide
         out["error"] = repr(e)
     return out
+
+
+def run_only(args):
+    """One secondary line alone (``--only NAME``): prints {"extra": {NAME: ...}}.
+    Used to profile one operation under ncu without the rest of the bench."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    print(json.dumps({"extra": run_extra(dev, peaks(), only=args.only)}), flush=True)
 
 
 def _step_stack(s: W.Shape, layers: int, dev, pk, conv_width: int = 0) -> dict:
@@ -511,10 +527,13 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--only", choices=sorted(EXTRA), help="run one secondary line alone")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.only:
+        run_only(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
