@@ -69,7 +69,7 @@ def build(force: bool = False) -> str:
 def _open(path: str):
     lib = ctypes.CDLL(path)
     for name in ("oracle_prefix", "oracle_block_step", "oracle_allblock", "oracle_allblock_backward",
-                 "oracle_conv_prefix", "oracle_conv_allblock"):
+                 "oracle_conv_prefix", "oracle_conv_allblock", "oracle_gated_rmsnorm"):
         getattr(lib, name).restype = ctypes.c_int
     lib.oracle_max_threads.restype = ctypes.c_int
     lib.oracle_set_threads.argtypes = [ctypes.c_int]
@@ -310,6 +310,27 @@ def conv_allblock(shape: dict, width: int, silu: bool, clean_fwd: dict, clean_re
     return [None if v is None else _unpack_rows(shape, v) for v in m.outs]
 
 
+def gated_rmsnorm(y, z=None, weight=None, groups: int = 1, eps: float = 1e-5, lib=None):
+    """Gated RMSNorm of token rows: y (and z) [..., H, P] or [..., C]; the last
+    two dimensions (or the last) are the channels.  Returns float64 of y's shape:
+    per row and group of C / groups channels, v * w / sqrt(mean(v^2) + eps) with
+    v = y * silu(z) (v = y without z)."""
+    lib = lib or _load()
+    ya = _f64(y)
+    shape = ya.shape
+    C = int(np.asarray(_f64(weight)).size)
+    rows = int(ya.size // C) if C else 0
+    m = _Marshal()
+    yk = m.arr(ya.reshape(rows, C))
+    zk = m.arr(None if z is None else _f64(z).reshape(rows, C))
+    wk = m.arr(weight)
+    out = np.zeros((rows, C))
+    rc = lib.oracle_gated_rmsnorm(ctypes.c_int64(rows), ctypes.c_int64(C), ctypes.c_int64(int(groups)),
+                                  ctypes.c_double(float(eps)), _ptr(yk), _ptr(zk), _ptr(wk), _ptr(out))
+    _check(rc, "oracle_gated_rmsnorm")
+    return out.reshape(shape)
+
+
 class Variant:
     """The same API bound to another build of the oracle source (used by the
     tests that plant a mistake in a copy of the oracle and check that the pins
@@ -335,6 +356,9 @@ class Variant:
 
     def conv_allblock(self, *a, **k):
         return conv_allblock(*a, lib=self.lib, **k)
+
+    def gated_rmsnorm(self, *a, **k):
+        return gated_rmsnorm(*a, lib=self.lib, **k)
 
 
 def compile_variant(src_text: str, out_path: str) -> str:

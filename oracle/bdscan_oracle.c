@@ -34,6 +34,8 @@
  *   with the conv state of the cache (see the section before
  *   oracle_max_threads for its definition and citations).
  *
+ *   The gated RMSNorm of the summed output (same place).
+ *
  * Layouts (row-major, innermost last):
  *   x, z, y  [B][L][H][P]    dt [B][L][H]    Bm, Cm [B][L][G][N]
  *   A, D     [H]             state [B][H][P][N]   states [B][K][H][P][N]
@@ -602,6 +604,38 @@ int oracle_conv_allblock(const oracle_conv_shape_t *s, const oracle_conv_dir_t *
     if (cr) conv_anticausal(s, cr);
     conv_causal(s, nf, cf->u, state_in);
     if (nr) conv_anticausal(s, nr);
+    return ORACLE_OK;
+}
+
+/* ---- Gated RMSNorm after the directional sum ----------------------------------
+ *
+ * "Breaking the Bottleneck with DiffuApriel", section 3.2 (after eq. (6)): the
+ * summed hidden sequence y = y_fwd + y_rev is normalised before the layer's
+ * projection.  Read as the Mamba-2 layer's gated RMSNorm with the gate applied
+ * before the norm: per token row, v_c = y_c * silu(z_c) (v = y without z); the
+ * channels are cut into `groups` consecutive groups of gs = C / groups; per
+ * group, r = 1 / sqrt(mean_{c in group} v_c^2 + eps); out_c = v_c * r * w_c.
+ * Rows: y, z, out [rows][C] (C = H * P), w [C]. */
+int oracle_gated_rmsnorm(int64_t rows, int64_t channels, int64_t groups, double eps, const double *y,
+                         const double *z, const double *w, double *out) {
+    if (rows < 0 || channels < 1 || groups < 1 || channels % groups || !w || !out || (rows && !y))
+        return ORACLE_EINVAL;
+    const int64_t gs = channels / groups;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t g = 0; g < groups; ++g) {
+            double ss = 0.0;
+            for (int64_t c = g * gs; c < (g + 1) * gs; ++c) {
+                const double v = y[r * channels + c] * (z ? silu(z[r * channels + c]) : 1.0);
+                ss += v * v;
+            }
+            const double rstd = 1.0 / sqrt(ss / (double)gs + eps);
+            for (int64_t c = g * gs; c < (g + 1) * gs; ++c) {
+                const double v = y[r * channels + c] * (z ? silu(z[r * channels + c]) : 1.0);
+                out[r * channels + c] = v * rstd * w[c];
+            }
+        }
+    }
     return ORACLE_OK;
 }
 
