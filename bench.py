@@ -353,6 +353,9 @@ EXTRA = {
     "conv_allblock_87m": lambda dev, pk: _conv_allblock(W.WORKLOADS["87m_allblock"], 4, dev, pk),
     "conv_block_step_700m_b1_24layers": lambda dev, pk: _step_stack(W.WORKLOADS["700m_step"], 24, dev, pk,
                                                                     conv_width=4),
+    "gated_rmsnorm_87m": lambda dev, pk: _norm(W.WORKLOADS["87m_allblock"], dev, pk),
+    "conv_block_step_norm_700m_b1_24layers": lambda dev, pk: _step_stack(W.WORKLOADS["700m_step"], 24, dev,
+                                                                         pk, conv_width=4, norm=True),
 }
 
 
@@ -379,10 +382,11 @@ def run_only(args):
     print(json.dumps({"extra": run_extra(dev, peaks(), only=args.only)}), flush=True)
 
 
-def _step_stack(s: W.Shape, layers: int, dev, pk, conv_width: int = 0) -> dict:
+def _step_stack(s: W.Shape, layers: int, dev, pk, conv_width: int = 0, norm: bool = False) -> dict:
     """With ``conv_width``, every layer first runs the short convolution of both
     directions from its cached conv state (writing the scan's x, B, C), then the
-    scan step: the selective-scan core of a Mamba layer's denoising step."""
+    scan step; with ``norm``, the gated RMSNorm of the summed output follows
+    (bf16): the selective-scan core of a Mamba layer's denoising step."""
     seed = W.SEEDS["700m_step" if s.nheads == 48 else "3b_step_b1"]
     ins = [W.make_streams(s, seed, layer, device=dev, streams=(W.CLEAN_FWD, W.CLEAN_REV))
            for layer in range(layers)]
@@ -395,6 +399,11 @@ def _step_stack(s: W.Shape, layers: int, dev, pk, conv_width: int = 0) -> dict:
         cstates = [W.make_conv_state(s, conv_width, seed, layer, device=dev) for layer in range(layers)]
         # the convolution writes straight into the scan's x, B, C
         couts = [[{k: ins[l][i][k] for k in bd.CONV_KEYS} for i in range(2)] for l in range(layers)]
+    if norm:
+        gz = torch.Generator(device=dev).manual_seed(11)
+        zs = [torch.randn(ys[0].shape, generator=gz, device=dev).to(torch.bfloat16) for _ in range(layers)]
+        nws = [torch.ones(s.nheads * s.headdim, device=dev) for _ in range(layers)]
+        nouts = [torch.empty(ys[0].shape, dtype=torch.bfloat16, device=dev) for _ in range(layers)]
     g_stream = torch.cuda.Stream(dev)
 
     def stack():
@@ -404,6 +413,9 @@ def _step_stack(s: W.Shape, layers: int, dev, pk, conv_width: int = 0) -> dict:
                                out_fwd=couts[l][0], out_rev=couts[l][1], stream=torch.cuda.current_stream(dev))
             bd.block_step(s, ins[l][0], ins[l][1], states[l], y=ys[l], ws=wss[l],
                           stream=torch.cuda.current_stream(dev))
+            if norm:
+                bd.gated_rmsnorm(s, ys[l], zs[l], nws[l], 1, 1e-5, out=nouts[l],
+                                 stream=torch.cuda.current_stream(dev))
 
     with torch.cuda.stream(g_stream):
         stack()
@@ -427,13 +439,34 @@ def _step_stack(s: W.Shape, layers: int, dev, pk, conv_width: int = 0) -> dict:
     b = RL.block_step_bytes(s) * layers
     if conv_width:
         b += RL.conv_bytes(s, conv_width, 2, state_in=True) * layers
+    if norm:
+        b += RL.norm_bytes(s, gated=True) * layers
     del graph
     out = {"us_per_step": ms * 1e3, "tokens_per_s": s.batch * s.seqlen / (ms * 1e-3),
            "algorithmic_bytes": b, "hbm_frac": b / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
            "layers": layers, "batch": s.batch, "graph": True}
     if conv_width:
         out["conv_width"] = conv_width
+    if norm:
+        out["gated_rmsnorm"] = True
     return out
+
+
+def _norm(s: W.Shape, dev, pk) -> dict:
+    """Gated RMSNorm (one group over all H*P channels, bf16 result) of the 87M
+    all-block layer's fp32 noisy output with a bf16 gate."""
+    cf, cr, nf, nr = W.make_streams(s, W.SEEDS[WORKLOAD], device=dev)
+    _, yn, _ = bd.allblock(s, cf, cr, nf, nr, want_clean=False)
+    g = torch.Generator(device=dev).manual_seed(9)
+    z = torch.randn(yn.shape, generator=g, device=dev).to(torch.bfloat16)
+    w = torch.ones(s.nheads * s.headdim, device=dev)
+    out = bd.gated_rmsnorm(s, yn, z, w, 1, 1e-5)
+    ms = _time(lambda: bd.gated_rmsnorm(s, yn, z, w, 1, 1e-5, out=out), dev, 20)
+    b = RL.norm_bytes(s, gated=True)
+    achieved = b / (ms * 1e-3) / 1e9
+    return {"us_per_call": ms * 1e3, "tokens_per_s": s.batch * s.seqlen / (ms * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / pk["hbm_gbs"], "algorithmic_bytes": b}}
 
 
 def _conv_allblock(s: W.Shape, width: int, dev, pk) -> dict:

@@ -25,7 +25,7 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "bdscan.h")
 
 BDSCAN_BF16, BDSCAN_FP32 = 0, 1
 BDSCAN_OP_PREFIX, BDSCAN_OP_BLOCK_STEP, BDSCAN_OP_ALLBLOCK, BDSCAN_OP_ALLBLOCK_BACKWARD = 0, 1, 2, 3
-BDSCAN_OP_CONV_PREFIX, BDSCAN_OP_CONV_ALLBLOCK = 4, 5
+BDSCAN_OP_CONV_PREFIX, BDSCAN_OP_CONV_ALLBLOCK, BDSCAN_OP_GATED_RMSNORM = 4, 5, 6
 STATUS = {0: "BDSCAN_OK", -1: "BDSCAN_ERR_INVALID_ARG", -2: "BDSCAN_ERR_UNSUPPORTED_SHAPE",
           -3: "BDSCAN_ERR_MISALIGNED", -4: "BDSCAN_ERR_WORKSPACE", -5: "BDSCAN_ERR_CUDA",
           -6: "BDSCAN_ERR_TIMEOUT", -7: "BDSCAN_ERR_SCRATCH_LIMIT"}
@@ -82,8 +82,10 @@ def lib() -> ctypes.CDLL:
             cp, ci = ctypes.POINTER(bdscan_conv_t), ctypes.c_int
             L.bdscan_conv_prefix.argtypes = [sp, ci, ci, cp, cp, vp, vp, vp]
             L.bdscan_conv_allblock.argtypes = [sp, ci, ci, cp, cp, cp, cp, vp, vp]
+            L.bdscan_gated_rmsnorm.argtypes = [sp, vp, vp, vp, ctypes.c_int64, ctypes.c_float, vp, vp]
             for fn in ("bdscan_prefix", "bdscan_block_step", "bdscan_allblock", "bdscan_allblock_backward",
-                       "bdscan_conv_prefix", "bdscan_conv_allblock", "bdscan_check_status", "bdscan_version"):
+                       "bdscan_conv_prefix", "bdscan_conv_allblock", "bdscan_gated_rmsnorm",
+                       "bdscan_check_status", "bdscan_version"):
                 getattr(L, fn).restype = ctypes.c_int
             L.bdscan_workspace_size.argtypes = [sp, ctypes.c_int]
             L.bdscan_workspace_size.restype = ctypes.c_size_t
@@ -134,6 +136,10 @@ def bdscan_conv_prefix(shape, width, silu, fwd, rev, conv_state_in, conv_state_o
 
 def bdscan_conv_allblock(shape, width, silu, cf, cr, nf, nr, conv_state_in, stream) -> int:
     return lib().bdscan_conv_allblock(shape, width, silu, cf, cr, nf, nr, conv_state_in, stream)
+
+
+def bdscan_gated_rmsnorm(shape, y, z, weight, groups, eps, out, stream) -> int:
+    return lib().bdscan_gated_rmsnorm(shape, y, z, weight, groups, eps, out, stream)
 
 
 def bdscan_block_step_noalloc(shape, fwd, rev, state_in, y, state_out, stream) -> int:
@@ -415,3 +421,25 @@ def conv_allblock(s: Shape, width: int, silu: bool, clean_fwd: dict, clean_rev: 
                               _ref(cd[2]), _ref(cd[3]), _ptr(state_in), _stream(dev, stream))
     _raise("bdscan_conv_allblock", rc)
     return [b[1] for b in built]
+
+
+# ----------------------------------------------------------------------------- gated RMSNorm
+def gated_rmsnorm(s: Shape, y, z=None, weight=None, groups: int = 1, eps: float = 1e-5, out=None,
+                  stream=None):
+    """Gated RMSNorm of a scan output ``y`` [B, L, H, P] (out_dtype): per token row
+    and group of H*P/groups channels, v * weight / sqrt(mean(v^2) + eps) with
+    v = y * silu(z) (z in_dtype, optional); bf16 result (``out`` may be ``y``
+    when y is bf16)."""
+    dev = y.device
+    B, L, H, P = s.batch, s.seqlen, s.nheads, s.headdim
+    _check_tensor("y", y, (B, L, H, P), _DT[s.out_dtype][0], dev)
+    if z is not None:
+        _check_tensor("z", z, (B, L, H, P), _DT[s.in_dtype][0], dev)
+    _check_tensor("weight", weight, (H * P,), torch.float32, dev)
+    if out is None:
+        out = torch.empty((B, L, H, P), dtype=torch.bfloat16, device=dev)
+    _check_tensor("out", out, (B, L, H, P), torch.bfloat16, dev)
+    rc = bdscan_gated_rmsnorm(ctypes.byref(c_shape(s)), _ptr(y), _ptr(z), _ptr(weight), int(groups),
+                              float(eps), _ptr(out), _stream(dev, stream))
+    _raise("bdscan_gated_rmsnorm", rc)
+    return out

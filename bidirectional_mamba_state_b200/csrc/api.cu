@@ -169,6 +169,7 @@ size_t bdscan_workspace_size(const bdscan_shape_t *shape, int op) {
 
 int bdscan_kernel_launches(const bdscan_shape_t *shape, int op) {
   if (check_shape(shape) != BDSCAN_OK) return -1;
+  if (op == BDSCAN_OP_GATED_RMSNORM) return (shape->batch == 0 || shape->seqlen == 0) ? 0 : 1;
   if (op == BDSCAN_OP_CONV_PREFIX || op == BDSCAN_OP_CONV_ALLBLOCK)
     return (shape->batch == 0 || shape->seqlen == 0) ? 0 : 1;
   if (op == BDSCAN_OP_ALLBLOCK_BACKWARD) {
@@ -616,6 +617,48 @@ int bdscan_conv_allblock(const bdscan_shape_t *shape, int width, int silu,
   a.dir[3] = to_conv_args(noisy_rev);
   a.state_in = conv_state_in;
   return conv_launch(a, z, static_cast<cudaStream_t>(cuda_stream));
+}
+
+}  // extern "C"
+
+// ---- gated RMSNorm of the summed output ----------------------------------------
+extern "C" {
+
+int bdscan_gated_rmsnorm(const bdscan_shape_t *shape, const void *y, const void *z, const float *weight,
+                         int64_t groups, float eps, void *out, void *cuda_stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  const int64_t C = shape->nheads * shape->headdim;
+  if (groups < 1 || !(eps >= 0.0f) || eps > 3.0e38f) return BDSCAN_ERR_INVALID_ARG;
+  if (C % groups || (C / groups) % 4 || bdscan::norm_smem_bytes(C, groups) > 227u * 1024u)
+    return BDSCAN_ERR_UNSUPPORTED_SHAPE;
+  const size_t rows = (size_t)shape->batch * (size_t)shape->seqlen;
+  if (rows > (size_t)INT32_MAX) return BDSCAN_ERR_UNSUPPORTED_SHAPE;  // one CTA per row
+  const size_t ysz = rows * (size_t)C * (shape->out_dtype == BDSCAN_BF16 ? 2 : 4);
+  const size_t zsz = rows * (size_t)C * (shape->in_dtype == BDSCAN_BF16 ? 2 : 4);
+  const size_t osz = rows * (size_t)C * 2;
+  if (!weight || (rows && (!y || !out))) return BDSCAN_ERR_INVALID_ARG;
+  const void *ptrs[] = {y, z, weight, out};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return BDSCAN_ERR_MISALIGNED;
+  const Range ro = range_of(out, osz);
+  // in place (out == y) only when y is bf16: each row is read whole before it is written
+  const bool in_place = out == y && shape->out_dtype == BDSCAN_BF16;
+  if (!in_place && overlaps(ro, range_of(y, ysz))) return BDSCAN_ERR_INVALID_ARG;
+  if (z && overlaps(ro, range_of(z, zsz))) return BDSCAN_ERR_INVALID_ARG;
+  if (overlaps(ro, range_of(weight, (size_t)C * 4))) return BDSCAN_ERR_INVALID_ARG;
+  bdscan::NormArgs a{};
+  a.Bsz = shape->batch; a.L = shape->seqlen; a.C = C; a.groups = groups; a.eps = eps;
+  a.y = y; a.z = z; a.weight = weight; a.out = out;
+  a.y_bf16 = shape->out_dtype == BDSCAN_BF16;
+  a.z_bf16 = shape->in_dtype == BDSCAN_BF16;
+  cudaError_t e = bdscan::launch_norm(a, static_cast<cudaStream_t>(cuda_stream));
+  if (e != cudaSuccess) {
+    const char *v = std::getenv("BDSCAN_VERBOSE");
+    if (v && v[0] == '1') std::fprintf(stderr, "libbdscan: norm launch failed: %s\n", cudaGetErrorString(e));
+    return BDSCAN_ERR_CUDA;
+  }
+  return BDSCAN_OK;
 }
 
 }  // extern "C"

@@ -81,4 +81,16 @@ struct ConvArgs {
 int conv_tile(const ConvArgs &a);
 cudaError_t launch_conv(const ConvArgs &a, cudaStream_t stream);
 
+// Gated RMSNorm of the summed output, bf16 result.
+struct NormArgs {
+  int64_t Bsz, L, C, groups;  // rows = Bsz * L, C = H * P channels per row
+  float eps;
+  const void *y, *z;          // y: out_dtype, z: in_dtype or nullptr
+  const float *weight;        // [C]
+  void *out;                  // bf16 [rows][C]
+  bool y_bf16, z_bf16;
+};
+size_t norm_smem_bytes(int64_t C, int64_t groups);
+cudaError_t launch_norm(const NormArgs &a, cudaStream_t stream);
+
 }  // namespace bdscan

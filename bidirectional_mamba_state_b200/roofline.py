@@ -112,3 +112,10 @@ def conv_bytes(s: Shape, width: int, ndir: int, state_in: bool = False, state_ou
 def conv_flops(s: Shape, width: int, ndir: int) -> int:
     """2 flops per tap per output (SiLU not counted)."""
     return ndir * 2 * width * s.batch * s.seqlen * conv_channels(s)
+
+
+def norm_bytes(s: Shape, gated: bool = True) -> int:
+    """Gated RMSNorm of one scan output: y (out dtype) and z (input dtype) read
+    once, the bf16 result written once, the fp32 weights."""
+    n = s.batch * s.seqlen * s.nheads * s.headdim
+    return n * (_elt(s.out_dtype) + (_elt(s.in_dtype) if gated else 0) + 2) + 4 * s.nheads * s.headdim

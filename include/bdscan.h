@@ -68,6 +68,7 @@ extern "C" {
 #define BDSCAN_OP_ALLBLOCK_BACKWARD 3
 #define BDSCAN_OP_CONV_PREFIX 4   /* no workspace (bdscan_workspace_size returns 0) */
 #define BDSCAN_OP_CONV_ALLBLOCK 5 /* no workspace */
+#define BDSCAN_OP_GATED_RMSNORM 6 /* no workspace */
 
 /* Problem shape.  Supported: batch >= 0, seqlen >= 0, seqlen % block_len == 0,
  * 1 <= block_len <= 32 or block_len % 32 == 0 (<= 256), chunk_len % block_len
@@ -234,6 +235,26 @@ int bdscan_conv_allblock(const bdscan_shape_t *shape, int width, int silu,
                          const bdscan_conv_t *clean_fwd, const bdscan_conv_t *clean_rev,
                          const bdscan_conv_t *noisy_fwd, const bdscan_conv_t *noisy_rev,
                          const void *conv_state_in, void *cuda_stream);
+
+/* bdscan_gated_rmsnorm -- the normalisation of the summed output before the
+ * layer's projection ("Breaking the Bottleneck with DiffuApriel", section 3.2
+ * after eq. (6)), read as the Mamba-2 layer's gated RMSNorm with the gate
+ * before the norm, written in bf16.  Per token row (b, t), with C = H*P
+ * channels cut into `groups` groups of gs = C / groups consecutive channels:
+ *   v_c   = y_c * silu(z_c)            (v = y when z is NULL)
+ *   out_c = v_c * weight_c / sqrt(mean_{c' in group(c)} v_c'^2 + eps)
+ *   y       [B][L][H][P] of shape->out_dtype (a scan call's output)
+ *   z       [B][L][H][P] of shape->in_dtype, or NULL
+ *   weight  [H*P] fp32
+ *   groups  >= 1, C % groups == 0, gs % 4 == 0 (else UNSUPPORTED_SHAPE); the
+ *           row (4*C + C + 4*groups bytes) must fit one CTA's shared memory
+ *   eps     >= 0 and finite
+ *   out     [B][L][H][P] bf16; may be y itself when y is bf16 (in place),
+ *           must not overlap y otherwise, nor z or weight
+ * Computed in fp32 (sums of squares in a fixed order: deterministic), rounded
+ * once to bf16.  One kernel launch; no workspace. */
+int bdscan_gated_rmsnorm(const bdscan_shape_t *shape, const void *y, const void *z, const float *weight,
+                         int64_t groups, float eps, void *out, void *cuda_stream);
 
 /* Workspace bytes an operation needs for this shape (>= 256: the first 256
  * bytes hold the device status word).  Returns 0 for an invalid shape/op. */

@@ -233,3 +233,23 @@ def test_conv_validation():
     cf, nf = _fake_conv(0x10000000), _fake_conv(0x20000000)
     rc = bd.bdscan_conv_allblock(ctypes.byref(s), 4, 1, ctypes.byref(cf), None, None, None, None, None)
     assert rc == -1                                                     # noisy_fwd required
+
+
+def test_gated_rmsnorm_validation():
+    s = bd.c_shape(Shape(**_base()))   # H*P = 64 channels, fp32 y (out_dtype), bf16 z
+    assert bd.bdscan_workspace_size(ctypes.byref(s), bd.BDSCAN_OP_GATED_RMSNORM) == 0
+    assert bd.bdscan_kernel_launches(ctypes.byref(s), bd.BDSCAN_OP_GATED_RMSNORM) == 1
+    y, z, w, out = 0x10000000, 0x20000000, 0x30000000, 0x40000000
+
+    def call(y=y, z=z, w=w, groups=1, eps=1e-5, out=out, shape=s):
+        return bd.bdscan_gated_rmsnorm(ctypes.byref(shape), y, z, w, groups, eps, out, None)
+
+    assert call(groups=0) == -1
+    assert call(eps=-1.0) == -1 and call(eps=float("nan")) == -1
+    assert call(groups=3) == -2            # 64 % 3 != 0
+    assert call(groups=32) == -2           # groups of 2 channels: not whole 4-channel vectors
+    assert call(w=None) == -1 and call(out=None) == -1 and call(y=None) == -1
+    assert call(out=out + 8) == -3         # misaligned
+    assert call(out=y) == -1               # in place needs a bf16 y
+    assert call(out=y + 0x40) == -1       # partial overlap with y
+    assert call(out=z) == -1 and call(out=w) == -1
