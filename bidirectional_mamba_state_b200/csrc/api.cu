@@ -129,7 +129,11 @@ int check_ws(void *ws, size_t ws_bytes, size_t need) {
 
 int launch(ScanArgs &a, cudaStream_t stream) {
   a.status = reinterpret_cast<int *>(a.ws);
-  if (cudaMemsetAsync(a.ws, 0, sizeof(int), stream) != cudaSuccess) return BDSCAN_ERR_CUDA;
+  // The tensor-core path clears the status word in its first kernel (a
+  // memset here would stand between that kernel and the one before it and
+  // stop their launches from overlapping); every other path clears it here.
+  const bool tc = a.Bsz > 0 && a.L > 0 && bdscan::tc_supported(a);
+  if (!tc && cudaMemsetAsync(a.ws, 0, sizeof(int), stream) != cudaSuccess) return BDSCAN_ERR_CUDA;
   if (a.Bsz == 0) return BDSCAN_OK;
   if (a.L == 0) {
     // Nothing to scan: the final state is the initial one.
@@ -141,7 +145,7 @@ int launch(ScanArgs &a, cudaStream_t stream) {
     }
     return BDSCAN_OK;
   }
-  cudaError_t e = bdscan::tc_supported(a) ? bdscan::launch_tc(a, stream) : bdscan::launch_seq(a, stream);
+  cudaError_t e = tc ? bdscan::launch_tc(a, stream) : bdscan::launch_seq(a, stream);
   if (e != cudaSuccess) {
     const char *v = std::getenv("BDSCAN_VERBOSE");
     if (v && v[0] == '1') std::fprintf(stderr, "libbdscan: launch failed: %s\n", cudaGetErrorString(e));

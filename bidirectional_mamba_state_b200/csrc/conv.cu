@@ -20,6 +20,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstring>
 
 #include "bdscan_internal.h"
 
@@ -179,6 +180,11 @@ __global__ void __launch_bounds__(kConvThreads, 2) bd_conv_kernel(const __grid_c
   constexpr int V = Vt::V;
   constexpr int WH = W > 1 ? W - 1 : 1;  // window rows (at least one, unused when W == 1)
   constexpr int NBM = sizeof(Raw) == 8 ? 8 : 4;  // rows per batch: 64 bytes of loads in flight
+  // Launched as a programmatic dependent of the kernel before it on the stream:
+  // wait for that kernel before touching memory, then let the next one (e.g.
+  // the scan's pre-pass, which waits for us in turn) be scheduled.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const ConvJob &J = p.job[blockIdx.y];
   const int64_t item = static_cast<int64_t>(blockIdx.x) * kConvThreads + threadIdx.x;
   if (item >= static_cast<int64_t>(p.Bsz) * J.tiles * p.nvec) return;
@@ -329,15 +335,32 @@ __global__ void __launch_bounds__(kConvThreads, 2) bd_conv_kernel(const __grid_c
   }
 }
 
+// Programmatic dependent launch: the CTAs may be scheduled while the previous
+// kernel on the stream finishes (they wait for it in the kernel).
+template <typename E, int W>
+cudaError_t launch_pdl(const ConvParams &p, dim3 grid, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kConvThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, bd_conv_kernel<E, W>, p);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 template <typename E>
 cudaError_t launch_typed(const ConvParams &p, int W, dim3 grid, cudaStream_t stream) {
   switch (W) {
-    case 1: bd_conv_kernel<E, 1><<<grid, kConvThreads, 0, stream>>>(p); break;
-    case 2: bd_conv_kernel<E, 2><<<grid, kConvThreads, 0, stream>>>(p); break;
-    case 3: bd_conv_kernel<E, 3><<<grid, kConvThreads, 0, stream>>>(p); break;
-    default: bd_conv_kernel<E, 4><<<grid, kConvThreads, 0, stream>>>(p); break;
+    case 1: return launch_pdl<E, 1>(p, grid, stream);
+    case 2: return launch_pdl<E, 2>(p, grid, stream);
+    case 3: return launch_pdl<E, 3>(p, grid, stream);
+    default: return launch_pdl<E, 4>(p, grid, stream);
   }
-  return cudaGetLastError();
 }
 
 // Largest power of two <= want that divides T (a tile never straddles a block).

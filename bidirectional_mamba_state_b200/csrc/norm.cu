@@ -17,6 +17,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstring>
 
 #include "bdscan_internal.h"
 
@@ -55,6 +56,10 @@ __global__ void __launch_bounds__(kNormThreads) bd_norm_kernel(const __grid_cons
   float4 *vrow = smem4;                                           // v of the row, [nv]
   float *part = reinterpret_cast<float *>(smem4 + p.nv);          // sum of squares per vector, [nv]
   float *rstd = part + p.nv;                                      // per group, [groups]
+  // programmatic dependent of the kernel before it (the scan that wrote y):
+  // wait for it, then let the next kernel be scheduled
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t row = blockIdx.x;
   const TY *y = static_cast<const TY *>(p.y) + row * p.C;
   const TZ *z = p.z ? static_cast<const TZ *>(p.z) + row * p.C : nullptr;
@@ -99,8 +104,20 @@ cudaError_t launch_typed(const NormParams &p, int64_t rows, size_t smem, cudaStr
   cudaError_t e = cudaFuncSetAttribute(bd_norm_kernel<TY, TZ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  bd_norm_kernel<TY, TZ><<<static_cast<unsigned>(rows), kNormThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  // programmatic dependent launch (see the kernel's first lines)
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(static_cast<unsigned>(rows));
+  cfg.blockDim = dim3(kNormThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, bd_norm_kernel<TY, TZ>, p);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace

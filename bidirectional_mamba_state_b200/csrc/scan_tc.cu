@@ -117,9 +117,17 @@ __global__ void __launch_bounds__(kCbThreads) bd_cb_kernel(const __grid_constant
   const int b = blockIdx.y / p.G, g = blockIdx.y % p.G;
   const int k0 = 4 * blockIdx.x;
   const int nvalid = min(4, p.K - k0);
-  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x < 2) p.item_counters[threadIdx.x] = 0;
-  // the scan kernel that follows may start its prologue on free SMs now (it
-  // waits for this grid's completion before reading anything written here)
+  // Launched as a programmatic dependent of whatever kernel precedes it on the
+  // stream (e.g. the short convolution that writes B and C): wait for it before
+  // touching memory, then clear the status word and the work counters.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) {
+    if (threadIdx.x < 2) p.item_counters[threadIdx.x] = 0;
+    if (threadIdx.x == 2) *p.status = 0;
+  }
+  // The scan kernel that follows may start now: it reads x, B and C before
+  // its own wait, which is safe because every CTA of this grid triggers only
+  // after the wait above, i.e. after all earlier kernels have completed.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (threadIdx.x == 0) {
     mbar_init(&bars[0], 1);
@@ -1103,6 +1111,9 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kOffBar);
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(sm + kOffMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kOffMisc + 4);
+  // the next kernel on the stream may be scheduled now; it waits for this
+  // grid's completion before it reads anything (its CTAs take SMs as ours exit)
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (threadIdx.x == 0) {
     // arrival counts: full = producer (plus TMA bytes); empty = MMA commit + 4
     // operand warps; commits of the MMA warp count 1; the rest 4 warps each
@@ -1346,8 +1357,23 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
                                        static_cast<int>(kCbSmem));
   if (e != cudaSuccess) return e;
   dim3 cgrid((K + 3) / 4, static_cast<unsigned>(a.Bsz * a.G), nz);
-  bd_cb_kernel<<<cgrid, kCbThreads, kCbSmem, stream>>>(cp);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  {
+    // programmatic dependent launch: its CTAs may be scheduled while the
+    // previous kernel finishes; they wait for it before touching memory
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = cgrid;
+    cfg.blockDim = dim3(kCbThreads);
+    cfg.dynamicSmemBytes = kCbSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if ((e = cudaLaunchKernelEx(&cfg, bd_cb_kernel, cp)) != cudaSuccess) return e;
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
 
   // ---- the scan
   TcParams p;
