@@ -49,6 +49,7 @@ def _check(out, ref, what):
     (dict(), 1, False, 1e-5),
     (dict(), 4, True, 1e-6),                                   # four groups of 384 channels
     (dict(), 24, True, 1e-5),                                  # one group per head
+    (dict(), 48, True, 1e-5),                                  # 48 groups of 32: the shared-memory path
     (dict(nheads=48), 1, True, 1e-5),                          # 700M widths
     (dict(nheads=80, batch=1, seqlen=32), 2, True, 1e-5),      # 3B widths, one block
     (dict(out_dtype="bf16"), 1, True, 1e-5),                   # bf16 scan output
