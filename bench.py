@@ -275,7 +275,7 @@ def run_ours(args):
         "clocks": clk.summary(),
     }
     if rank == 0:
-        result["e2e"] = run_e2e(s, dev, cf, cr, nf, nr, ws, min(args.steps, 10), world)
+        result["e2e"] = run_e2e(s, dev, cf, cr, nf, nr, ws, min(args.steps, 10), world, ref_y_noisy=yn)
     else:
         run_e2e(s, dev, cf, cr, nf, nr, ws, min(args.steps, 10), world)
     if rank == 0 and world == 1 and not args.no_extra:
@@ -290,10 +290,13 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_e2e(s, dev, cf, cr, nf, nr, ws, steps, world):
+def run_e2e(s, dev, cf, cr, nf, nr, ws, steps, world, ref_y_noisy=None):
     """Same step through the public API from pinned host buffers: every step
     copies that step's inputs host->device, runs allblock, and copies all of its
-    outputs (y_clean, y_noisy, boundary states) device->host."""
+    outputs (y_clean, y_noisy, boundary states) device->host.  The batch is
+    processed in chunks of rows (rows are independent sequences) so that the
+    copy-in of one chunk, the scan of the previous one and the copy-out of the
+    one before overlap on three streams; steps do not overlap each other."""
     host = [{k: v.to("cpu").pin_memory() for k, v in d.items()} for d in (cf, cr, nf, nr)]
     devb = [{k: torch.empty_like(v) for k, v in d.items()} for d in (cf, cr, nf, nr)]
     K = s.nblocks
@@ -302,33 +305,67 @@ def run_e2e(s, dev, cf, cr, nf, nr, ws, steps, world):
     st = torch.empty((s.batch, K, s.nheads, s.headdim, s.dstate), device=dev, dtype=torch.float32)
     hyc, hyn = torch.empty(yc.shape, pin_memory=True), torch.empty(yn.shape, pin_memory=True)
     hst = torch.empty(st.shape, pin_memory=True)
-    stream = torch.cuda.current_stream(dev)
+    comp = torch.cuda.current_stream(dev)
+    cin, cout = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     h2d = sum(v.numel() * v.element_size() for d in host for v in d.values())
     d2h = sum(t.numel() * t.element_size() for t in (hyc, hyn, hst))
+    rows = max(1, s.batch // 8)
+    chunks = [(b0, min(s.batch, b0 + rows)) for b0 in range(0, s.batch, rows)]
+    subs = {n: s.with_(batch=n) for n in {b1 - b0 for b0, b1 in chunks}}
+    wss = {n: bd.workspace(sub, bd.BDSCAN_OP_ALLBLOCK, dev) for n, sub in subs.items()}
+
+    def rows_of(d, b0, b1):
+        return {k: (v if k in ("A", "D") else v[b0:b1]) for k, v in d.items()}
 
     def step():
-        for hd, dd in zip(host, devb):
-            for k in hd:
-                dd[k].copy_(hd[k], non_blocking=True)
-        bd.allblock(s, *devb, y_clean=yc, y_noisy=yn, states=st, ws=ws, stream=stream)
-        hyc.copy_(yc, non_blocking=True)
-        hyn.copy_(yn, non_blocking=True)
-        hst.copy_(st, non_blocking=True)
+        start = torch.cuda.Event()
+        start.record(comp)
+        cin.wait_event(start)
+        for b0, b1 in chunks:
+            with torch.cuda.stream(cin):
+                for hd, dd in zip(host, devb):
+                    for k in hd:
+                        if k in ("A", "D"):
+                            dd[k].copy_(hd[k], non_blocking=True)
+                        else:
+                            dd[k][b0:b1].copy_(hd[k][b0:b1], non_blocking=True)
+            ev_in = torch.cuda.Event()
+            ev_in.record(cin)
+            comp.wait_event(ev_in)
+            sub = subs[b1 - b0]
+            bd.allblock(sub, *(rows_of(d, b0, b1) for d in devb), y_clean=yc[b0:b1], y_noisy=yn[b0:b1],
+                        states=st[b0:b1], ws=wss[b1 - b0], stream=comp)
+            ev_done = torch.cuda.Event()
+            ev_done.record(comp)
+            cout.wait_event(ev_done)
+            with torch.cuda.stream(cout):
+                hyc[b0:b1].copy_(yc[b0:b1], non_blocking=True)
+                hyn[b0:b1].copy_(yn[b0:b1], non_blocking=True)
+                hst[b0:b1].copy_(st[b0:b1], non_blocking=True)
+        ev_out = torch.cuda.Event()
+        ev_out.record(cout)
+        comp.wait_event(ev_out)
 
     for _ in range(2):
         step()
     torch.cuda.synchronize(dev)
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    e0.record(comp)
     for _ in range(steps):
         step()
-    e1.record(stream)
+    e1.record(comp)
     torch.cuda.synchronize(dev)
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
-    return {"value": s.batch * s.seqlen * world / (ms * 1e-3), "unit": "tokens/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
-            "steps": steps}
+    out = {"value": s.batch * s.seqlen * world / (ms * 1e-3), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
+           "steps": steps, "chunks": len(chunks)}
+    if ref_y_noisy is not None:
+        # the host copy of the noisy output against the device-resident run's
+        ref = ref_y_noisy.float().cpu()
+        out["check_max_abs_diff_vs_device_run"] = float((hyn - ref).abs().max())
+        out["check_ref_max_abs"] = float(ref.abs().max())
+    return out
 
 
 def _time(fn, dev, reps, warm=3):
