@@ -41,12 +41,14 @@
 //                 h_k = exp(cum_31) h_{k-1} + S; boundary-state stores (one
 //                 128-byte line per warp instruction); h operand (bf16 hi + lo)
 //     warps 12-15 epilogue: thread (p, stream) forms y[t][p] = exp(cum_t) Y_off
-//                 + Y_diag for the block's 32 tokens and stores them; the D x
-//                 terms are small tensor-core products against D I_16 (bf16
-//                 hi + lo) accumulated into Y_diag.  Two blocks ahead, the
-//                 same warps build the masked-decay matrices M and the D I_16
-//                 operands.
-//   S, Y, M and D I_16 are double-buffered; the h operand is single-buffered.
+//                 + Y_diag for the block's 32 tokens and stores them.  Two
+//                 blocks ahead, the same warps build the masked-decay matrices
+//                 M with each direction's D added to the diagonal (so D x is
+//                 part of Y_diag), stored bf16, and the bf16 remainder of
+//                 that diagonal as two 16 x 16 diagonal tiles per direction,
+//                 applied by one more small MMA per 16 tokens.
+//   S, Y, M and the diagonal tiles are double-buffered; the h operand is
+//   single-buffered.
 // Every wait is bounded; on a timeout the CTA raises BDSCAN_ERR_TIMEOUT in the
 // workspace status word, drains its own copies and MMAs, frees TMEM and exits.
 //
@@ -212,7 +214,7 @@ constexpr uint32_t kOffXw = kSlots * kSlot;   // hi [32 t][64 p], lo [32 t][64 p
 constexpr uint32_t kOffH = kOffXw + 2 * kTile;  // {hi, lo} x [128 n][64 p] bf16 (SW128)
 constexpr uint32_t kOffMh = kOffH + 8 * kTile;  // 2 buffers x 4 dirs x [32 t][32 s] interleaved
 constexpr uint32_t kMhBuf = 4 * 2048;
-constexpr uint32_t kOffDg = kOffMh + 2 * kMhBuf;  // 2 items x 4 dirs x {hi, lo} x D I_16 (bf16, 512 B each)
+constexpr uint32_t kOffDg = kOffMh + 2 * kMhBuf;  // 2 steps x 4 dirs x 2 chunks x 16 x 16 diagonal (bf16, 512 B each)
 constexpr uint32_t kDgBuf = 4096;
 // per-step tables, a ring of kTab steps (slot j mod kTab)
 constexpr int kTab = 8;
@@ -230,8 +232,9 @@ constexpr uint32_t kOffItemQ = kOffMisc + 64;             // int4[kItemRing]: pu
 constexpr uint32_t kSmemBytes = kOffItemQ + 16 * kItemRing + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
-// D I_16 operand (B of the D x MMAs): [16 t][16 s] interleaved K-major, 8x8 core
-// matrices, t-groups 128 B apart, s-groups 256 B apart.
+// Diagonal correction tiles (B of the remainder MMAs): [16 t][16 s]
+// interleaved K-major, 8x8 core matrices, t-groups 128 B apart, s-groups 256 B
+// apart; only the diagonal is ever nonzero.
 constexpr uint32_t kDgSbo = 128, kDgLbo = 256;
 
 // masked-decay operand of one direction: [32 t][32 s], interleaved MN-major
@@ -579,7 +582,7 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
   // Y_off^T[p][t] = h C^T over the stacked [C_cf; C_nf] rows (only C_cf without a noisy stream)
   const uint32_t id_yo = p.allblock ? idesc_bf16(64, 64, 1, 0) : idesc_bf16(64, 32, 1, 0);
   const uint32_t id_yd = idesc_bf16(64, 32, 1, 1);  // Y_diag^T[p][t] = X^T M^T, one stream
-  const uint32_t id_dx = idesc_bf16(64, 16, 1, 0);  // (D x)^T[p][t] = X^T (D I_16)
+  const uint32_t id_dx = idesc_bf16(64, 16, 1, 0);  // X^T diag(remainder), 16 tokens
   // descriptor of each operand at its first tile; moving an operand by b bytes adds b >> 4
   const D64 dBcf = split64(sdesc(base + kOffBcf, kTile, 1024, kLayoutSw128));
   const D64 dXw = split64(sdesc(base + kOffXw, 0, 1024, kLayoutSw128));
@@ -595,7 +598,6 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
     Item I;
     if (item_one(p, c, base, m, I) <= 0) break;
     const int nk = I.nk;
-    const uint32_t go = BD_OFF(static_cast<uint32_t>(m & 1) * kDgBuf);  // this item's D I_16 operands
     for (int kk = 0; kk < nk; ++kk, ++j) {
       ok = false;
       const int r = rslot(j), i2 = j & 1;
@@ -645,17 +647,17 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
           umma_bf16(col, dX + so + BD_OFF(i * kTile + ks * 2048), dM + mo + BD_OFF(i * 2048 + ks * 1024), id_yd,
                     (i >= 2 || ks > 0) ? 1u : 0u);
       }
-      // D x of every direction: 16-token diagonal blocks against D I_16 (hi + lo)
+      // the bf16 remainder of M's diagonal (which holds D): one 16-token
+      // diagonal correction tile per chunk and direction
+      const uint32_t lo = BD_OFF(static_cast<uint32_t>(i2) * kDgBuf);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         if (!p.active[i]) continue;
         const uint32_t col = colY + 64 + ((i & 1) ? 32 : 0);
 #pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-          const D64 a = dX + so + BD_OFF(i * kTile + ks * 2048);
-          umma_bf16(col + 16 * ks, a, dDg + go + BD_OFF((2 * i) * 512), id_dx, 1);
-          umma_bf16(col + 16 * ks, a, dDg + go + BD_OFF((2 * i + 1) * 512), id_dx, 1);
-        }
+        for (int ks = 0; ks < 2; ++ks)
+          umma_bf16(col + 16 * ks, dX + so + BD_OFF(i * kTile + ks * 2048), dDg + lo + BD_OFF((2 * i + ks) * 512),
+                    id_dx, 1);
       }
       umma_commit_s(bar_at(c, bYFull0 + i2));
       umma_commit_s(bar_at(c, bEmpty0 + r));
@@ -977,12 +979,11 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
 // (lane < 16) or noisy (lane >= 16) stream's outputs y[t][p], t = 0..31:
 // y = exp(cum_t) Y_off + Y_diag (Y_diag already holds both directions' D x).
 // After the outputs of step j the group builds, two steps ahead, the
-// masked-decay matrices of step j + 2 (warp q: direction slot q, row s = lane
-// of M^T) and, at an item's first step, the D I_16 operands of the item.
+// masked-decay matrices of step j + 2 with D on the diagonal (warp q:
+// direction slot q, row s = lane of M^T) and the diagonal's bf16 remainders.
 __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
   const int lane = threadIdx.x & 31;
   const int q = (threadIdx.x >> 5) & 3;
-  const int gq = threadIdx.x - 384;  // 0..127
   const int pcol = 16 * q + (lane & 15);
   const bool noisy = lane >= 16;
   const int fs = noisy ? kNF : kCF;
@@ -1013,6 +1014,10 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
       const float cs = lds_f32(cq + lane * 4);
       const float ds = lds_f32(base + kOffDt + (ct * 4 + q) * 128 + lane * 4);
       const uint32_t mrow = base + kOffMh + (jm & 1) * kMhBuf + q * 2048;
+      // this direction's D joins the diagonal of M (D x is part of X^T M^T):
+      // M[s][s] + D is stored as bf16 hi in M and its bf16 remainder lo on the
+      // diagonal of the block's 16 x 16 correction tile of chunk s / 16
+      const float Dq = lds_f32(base + kOffDtab + (ct * 4 + q) * 4);
       // (not unrolled: a compact loop keeps the instruction cache footprint down)
 #pragma unroll 1
       for (int jj = 0; jj < 4; ++jj) {
@@ -1029,24 +1034,18 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
           const float e = ex2_approx(cj[i] - cs);
           const float cb = (i & 1) ? bf16_hi_f(r[i >> 1]) : bf16_lo_f(r[i >> 1]);
           mv[i] = valid ? cb * ds * e : 0.f;
+          if (t == lane) {
+            const float v = mv[i] + Dq;
+            const float hi = __bfloat162float(__float2bfloat16_rn(v));
+            const int d = lane & 15;
+            const uint32_t off = static_cast<uint32_t>(jm & 1) * kDgBuf + (d >> 3) * kDgSbo + (d >> 3) * kDgLbo +
+                                 (d & 7) * 16 + (d & 7) * 2;
+            sts_u16(base + kOffDg + (2 * q + (lane >> 4)) * 512 + off, __bfloat16_as_ushort(__float2bfloat16_rn(v - hi)));
+            mv[i] = v;
+          }
         }
         st_shared_v4(mrow + inter_mn_off(8 * jj, lane, kMhSbo, kMhLbo), pack_bf16x2(mv[0], mv[1]),
                      pack_bf16x2(mv[2], mv[3]), pack_bf16x2(mv[4], mv[5]), pack_bf16x2(mv[6], mv[7]));
-      }
-    }
-    if (f > 0 && gq < 64) {
-      // D I_16 operands of the item that starts here: bf16 hi + lo of each
-      // direction's D on the diagonal (the rest of the buffer stays zero).
-      // The MMAs of two items back, the buffer's last readers, are complete.
-      const int i = gq >> 4, d = gq & 15;
-      if (pick4(p.active, i)) {
-        const float Dv = lds_f32(base + kOffDtab + (ct * 4 + i) * 4);
-        const __nv_bfloat16 dh = __float2bfloat16_rn(Dv);
-        const __nv_bfloat16 dl = __float2bfloat16_rn(Dv - __bfloat162float(dh));
-        const uint32_t off =
-            static_cast<uint32_t>(f - 1) * kDgBuf + (d >> 3) * kDgSbo + (d >> 3) * kDgLbo + (d & 7) * 16 + (d & 7) * 2;
-        sts_u16(base + kOffDg + (2 * i) * 512 + off, __bfloat16_as_ushort(dh));
-        sts_u16(base + kOffDg + (2 * i + 1) * 512 + off, __bfloat16_as_ushort(dl));
       }
     }
     fence_proxy_async_smem();
@@ -1131,7 +1130,7 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
     *reinterpret_cast<int **>(sm + kOffMisc + 16) = p.status;
     fence_mbar_init();
   }
-  // Clear the D I_16 buffers (only their diagonals are written).
+  // Clear the diagonal correction tiles (only their diagonals are written).
   if (!p.agg) {
     const uint4 zero = make_uint4(0, 0, 0, 0);
     for (uint32_t o = threadIdx.x * 16; o < 2 * kDgBuf; o += kThreads * 16)
