@@ -64,7 +64,8 @@ __global__ void __launch_bounds__(kNormThreads) bd_norm_kernel(const __grid_cons
   const TY *y = static_cast<const TY *>(p.y) + row * p.C;
   const TZ *z = p.z ? static_cast<const TZ *>(p.z) + row * p.C : nullptr;
 
-  for (int v = threadIdx.x; v < p.nv; v += kNormThreads) {
+  const int nthr = blockDim.x;
+  for (int v = threadIdx.x; v < p.nv; v += nthr) {
     float a[4];
     load4(y + 4 * v, a);
     if (z) {
@@ -79,7 +80,7 @@ __global__ void __launch_bounds__(kNormThreads) bd_norm_kernel(const __grid_cons
   __syncthreads();
   // one warp per group: lanes sum strided vectors, then a fixed shuffle tree
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int g = warp; g < p.groups; g += kNormThreads / 32) {
+  for (int g = warp; g < p.groups; g += nthr / 32) {
     float s = 0.f;
     for (int v = g * p.gsv + lane; v < (g + 1) * p.gsv; v += 32) s += part[v];
 #pragma unroll
@@ -88,7 +89,7 @@ __global__ void __launch_bounds__(kNormThreads) bd_norm_kernel(const __grid_cons
   }
   __syncthreads();
   __nv_bfloat16 *out = p.out + row * p.C;
-  for (int v = threadIdx.x; v < p.nv; v += kNormThreads) {
+  for (int v = threadIdx.x; v < p.nv; v += nthr) {
     const float r = rstd[v / p.gsv];
     const float4 a = vrow[v];
     const float4 w = __ldg(reinterpret_cast<const float4 *>(p.w) + v);
@@ -108,7 +109,9 @@ cudaError_t launch_typed(const NormParams &p, int64_t rows, size_t smem, cudaStr
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3(static_cast<unsigned>(rows));
-  cfg.blockDim = dim3(kNormThreads);
+  // about three 4-channel vectors per thread: whole warps, 64 to 256 threads
+  const int want = (p.nv + 2) / 3;
+  cfg.blockDim = dim3(static_cast<unsigned>(want <= 64 ? 64 : (want <= 128 ? 128 : kNormThreads)));
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
