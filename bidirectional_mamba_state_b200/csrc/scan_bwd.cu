@@ -25,7 +25,7 @@
 // (given) plus dh_s of clean block k+1 plus dh_s of noisy block k+1 (which
 // starts from states[k]); dh_s of clean block 0 and of noisy block 0 is dh0.
 //
-// One CTA of 256 threads per (b, h) walks the blocks from last to first; all
+// One CTA of 512 threads per (b, h) walks the blocks from last to first; all
 // block quantities live in shared memory (with transposed copies where the
 // threads run over tokens), the products are register-tiled (4 x 4 per
 // thread), fp32 arithmetic on CUDA cores.  dB
@@ -43,7 +43,7 @@
 namespace bdscan {
 namespace {
 
-constexpr int kBwdThreads = 256;
+constexpr int kBwdThreads = 512;
 
 struct BwdDir {
   const void *x, *dt, *B, *C;
@@ -97,7 +97,7 @@ __device__ float block_sum(float v, float *red) {
 
 // Register-tiled product over shared-memory operands: for every TM x 4 output
 // tile (m0.., n0..) of an M x Nn result (TM chosen per product so that the
-// 256 threads have a tile each),
+// threads have a tile each),
 //   acc[i][j] = sum_k a1(m0+i, k) B1[k][n0+j]  (+ sum_k a2(m0+i, k) B2[k][n0+j])
 // with a(m, k) = A[m am + k ak] (times ks1[k], resp. ms2[m], when given) and
 // B rows contiguous in n (16-byte loads).  A threads of a warp share m0, so A
