@@ -102,15 +102,17 @@ __device__ __forceinline__ float act(float v, int silu) {
   return silu ? __fdividef(v, 1.0f + __expf(-v)) : v;
 }
 
-// NB consecutive rows (already loaded) of a causal convolution, written to
-// pd[0], pd[step], ...: the window (rows before the batch, oldest first) is
-// extended by the batch and its last W-1 rows kept.
+// NB rows ps[0], ps[step], ... issued back to back (their loads are in flight
+// together).
 template <class Vt, int NB>
 __device__ __forceinline__ void load_rows(typename Vt::Raw (&raw)[NB], const typename Vt::Raw *ps, int64_t step) {
 #pragma unroll
   for (int k = 0; k < NB; ++k) raw[k] = __ldg(ps + k * step);
 }
 
+// NB consecutive rows (already loaded) of a causal convolution, written to
+// pd[0], pd[step], ...: the window (rows before the batch, oldest first) is
+// extended by the batch and its last W-1 rows kept.
 template <class Vt, int W, int NB>
 __device__ __forceinline__ void rows_fwd(const typename Vt::Raw (&raw)[NB], typename Vt::Raw *pd, int64_t step,
                                          const float (&w)[W][Vt::V], const float (&bias)[Vt::V],
