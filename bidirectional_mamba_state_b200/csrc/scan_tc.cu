@@ -44,11 +44,10 @@
 //                 + Y_diag for the block's 32 tokens and stores them.  Two
 //                 blocks ahead, the same warps build the masked-decay matrices
 //                 M with each direction's D added to the diagonal (so D x is
-//                 part of Y_diag), stored bf16, and the bf16 remainder of
-//                 that diagonal as two 16 x 16 diagonal tiles per direction,
-//                 applied by one more small MMA per 16 tokens.
-//   S, Y, M and the diagonal tiles are double-buffered; the h operand is
-//   single-buffered.
+//                 part of Y_diag), stored bf16, next to a diagonal matrix of
+//                 that diagonal's bf16 remainders: one N = 64 MMA per 16
+//                 tokens gives both, summed by the epilogue.
+//   S, Y and M are double-buffered; the h operand is single-buffered.
 // Every wait is bounded; on a timeout the CTA raises BDSCAN_ERR_TIMEOUT in the
 // workspace status word, drains its own copies and MMAs, frees TMEM and exits.
 //
@@ -212,16 +211,14 @@ constexpr uint32_t kOffCB = 10 * kTile;       // 4 dirs x [32 s][32 t] bf16 (SW6
 constexpr uint32_t kSlot = 12 * kTile;        // 48 KB per slot
 constexpr uint32_t kOffXw = kSlots * kSlot;   // hi [32 t][64 p], lo [32 t][64 p] (bf16, SW128)
 constexpr uint32_t kOffH = kOffXw + 2 * kTile;  // {hi, lo} x [128 n][64 p] bf16 (SW128)
-constexpr uint32_t kOffMh = kOffH + 8 * kTile;  // 2 buffers x 4 dirs x [32 t][32 s] interleaved
-constexpr uint32_t kMhBuf = 4 * 2048;
-constexpr uint32_t kOffDg = kOffMh + 2 * kMhBuf;  // 2 steps x 4 dirs x 2 chunks x 16 x 16 diagonal (bf16, 512 B each)
-constexpr uint32_t kDgBuf = 4096;
+constexpr uint32_t kOffMh = kOffH + 8 * kTile;  // 2 buffers x 4 dirs x [64 t'][32 s] interleaved
+constexpr uint32_t kMhDir = 4096;               // one direction: [M^T | diag(remainder)]
+constexpr uint32_t kMhBuf = 4 * kMhDir;
 // per-step tables, a ring of kTab steps (slot j mod kTab)
 constexpr int kTab = 8;
-constexpr uint32_t kOffCum = kOffDg + 2 * kDgBuf;    // [kTab][4 dirs][32] f32: cumulative decay (log2)
+constexpr uint32_t kOffCum = kOffMh + 2 * kMhBuf;    // [kTab][4 dirs][32] f32: cumulative decay (log2)
 constexpr uint32_t kOffDt = kOffCum + kTab * 512;    // [kTab][4][32] f32: dt
-constexpr uint32_t kOffEc = kOffDt + kTab * 512;     // [kTab][2 fwd dirs][32] f32: exp(cum_t)
-constexpr uint32_t kOffDtab = kOffEc + kTab * 256;   // [kTab][4] f32: D of the step's head
+constexpr uint32_t kOffDtab = kOffDt + kTab * 512;  // [kTab][4] f32: D of the step's head
 constexpr uint32_t kOffFtab = kOffDtab + kTab * 16;  // [kTab] s32: 1 + item parity at an item's first step,
                                                      // 0 at its other steps, -1 past the CTA's last step
 constexpr uint32_t kOffBar = kOffFtab + 128;
@@ -232,14 +229,13 @@ constexpr uint32_t kOffItemQ = kOffMisc + 64;             // int4[kItemRing]: pu
 constexpr uint32_t kSmemBytes = kOffItemQ + 16 * kItemRing + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
-// Diagonal correction tiles (B of the remainder MMAs): [16 t][16 s]
-// interleaved K-major, 8x8 core matrices, t-groups 128 B apart, s-groups 256 B
-// apart; only the diagonal is ever nonzero.
-constexpr uint32_t kDgSbo = 128, kDgLbo = 256;
-
-// masked-decay operand of one direction: [32 t][32 s], interleaved MN-major
-// (t contiguous): t-groups 128 B apart, s-groups 512 B apart.
-constexpr uint32_t kMhSbo = 128, kMhLbo = 512;
+// intra-block operand of one direction (B of its Y_diag MMAs): [64 t'][32 s],
+// interleaved MN-major (t' contiguous), t'-groups 128 B apart, s-groups 1024 B
+// apart.  t' < 32: the masked-decay matrix M^T[s][t] with D on the diagonal
+// (bf16); t' = 32 + s: that diagonal's bf16 remainder; zero elsewhere.  One
+// N = 64 MMA per 16 tokens thus yields Y_diag in its first 32 columns and the
+// remainder's X contribution in the next 32.
+constexpr uint32_t kMhSbo = 128, kMhLbo = 1024;
 
 enum : int {
   bFull0 = 0, bFull1, bFull2, bEmpty0, bEmpty1, bEmpty2, bAux0, bAux7 = bAux0 + kTab - 1, bXwFull, bSFull0, bSFull1,
@@ -248,8 +244,9 @@ enum : int {
 };
 static_assert(bCount <= kNumBars, "barrier array");
 
-// TMEM columns: S^T[2] (M=128 x 64), Y^T[2] = {Y_off^T (M=64 x 64), Y_diag^T (M=64 x 64)}
-constexpr uint32_t kColS0 = 0, kColY0 = 128;
+// TMEM columns: S^T[2] (M=128 x 64), Y^T[2] = {Y_off^T (M=64 x 64), clean
+// [Y_diag^T | remainder] (M=64 x 64), noisy [Y_diag^T | remainder] (M=64 x 64)}
+constexpr uint32_t kColS0 = 0, kColY0 = 128, kColYBuf = 192;
 constexpr uint32_t kTmemCols = 512;
 
 struct TcParams {
@@ -581,8 +578,7 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
   const uint32_t id_s = idesc_bf16(128, 64, 1, 1);  // S^T[n][p] = B^T (w o X)
   // Y_off^T[p][t] = h C^T over the stacked [C_cf; C_nf] rows (only C_cf without a noisy stream)
   const uint32_t id_yo = p.allblock ? idesc_bf16(64, 64, 1, 0) : idesc_bf16(64, 32, 1, 0);
-  const uint32_t id_yd = idesc_bf16(64, 32, 1, 1);  // Y_diag^T[p][t] = X^T M^T, one stream
-  const uint32_t id_dx = idesc_bf16(64, 16, 1, 0);  // X^T diag(remainder), 16 tokens
+  const uint32_t id_yd = idesc_bf16(64, 64, 1, 1);  // [Y_diag^T | remainder][p][t'] = X^T [M^T | diag]
   // descriptor of each operand at its first tile; moving an operand by b bytes adds b >> 4
   const D64 dBcf = split64(sdesc(base + kOffBcf, kTile, 1024, kLayoutSw128));
   const D64 dXw = split64(sdesc(base + kOffXw, 0, 1024, kLayoutSw128));
@@ -590,7 +586,6 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
   const D64 dC = split64(sdesc(base + kOffClo, 16, 1024, kLayoutSw128));
   const D64 dX = split64(sdesc(base + kOffX, 0, 1024, kLayoutSw128));
   const D64 dM = split64(sdesc(base + kOffMh, kMhLbo, kMhSbo, kLayoutNone));
-  const D64 dDg = split64(sdesc(base + kOffDg, kDgLbo, kDgSbo, kLayoutNone));
 #define BD_OFF(bytes) (static_cast<uint32_t>((bytes) >> 4))
   int j = 0;
   bool ok = true;
@@ -625,7 +620,7 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
       if (!wait1(c, bHFull, j & 1)) break;
       if (j >= 2 && !wait1(c, bYEmpty0 + i2, par2(j - 2))) break;
       tc_fence_after();
-      const uint32_t colY = tmem + kColY0 + 128 * i2;
+      const uint32_t colY = tmem + kColY0 + kColYBuf * i2;
 #pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
         const D64 bc = dC + so + BD_OFF((ks < 4 ? 0 : 2 * kTile) + (ks & 3) * 32);
@@ -633,31 +628,20 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
         umma_bf16(colY, dH + BD_OFF(4 * kTile + ks * 2048), bc, id_yo, 1);
       }
       umma_commit_s(bar_at(c, bHCons));  // the h operand may now be overwritten
-      // ---- Y_diag^T of each stream = X_fwd^T M_fwd^T + X_rev^T M_rev^T, then
-      //      X^T (D I) of every direction
+      // ---- Y_diag^T of each stream = X_fwd^T M_fwd^T + X_rev^T M_rev^T (M
+      //      with D on its diagonal), and in the next 32 columns the same
+      //      products with the diagonal's bf16 remainders
       if (!wait1(c, bMhFull0 + i2, par2(j))) break;
       tc_fence_after();
       const uint32_t mo = BD_OFF(static_cast<uint32_t>(i2) * kMhBuf);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {  // the forward direction of a stream (i < 2) is always active
         if (!p.active[i]) continue;
-        const uint32_t col = colY + 64 + ((i & 1) ? 32 : 0);
+        const uint32_t col = colY + 64 + ((i & 1) ? 64 : 0);
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks)
-          umma_bf16(col, dX + so + BD_OFF(i * kTile + ks * 2048), dM + mo + BD_OFF(i * 2048 + ks * 1024), id_yd,
+          umma_bf16(col, dX + so + BD_OFF(i * kTile + ks * 2048), dM + mo + BD_OFF(i * kMhDir + ks * 2048), id_yd,
                     (i >= 2 || ks > 0) ? 1u : 0u);
-      }
-      // the bf16 remainder of M's diagonal (which holds D): one 16-token
-      // diagonal correction tile per chunk and direction
-      const uint32_t lo = BD_OFF(static_cast<uint32_t>(i2) * kDgBuf);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (!p.active[i]) continue;
-        const uint32_t col = colY + 64 + ((i & 1) ? 32 : 0);
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks)
-          umma_bf16(col + 16 * ks, dX + so + BD_OFF(i * kTile + ks * 2048), dDg + lo + BD_OFF((2 * i + ks) * 512),
-                    id_dx, 1);
       }
       umma_commit_s(bar_at(c, bYFull0 + i2));
       umma_commit_s(bar_at(c, bEmpty0 + r));
@@ -680,7 +664,7 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
   const int q = wq < 4 ? wq - 2 : wq - 4;
   const int gt = q * 32 + (threadIdx.x & 31);  // 0..127
   const bool act = pick4(p.active, q) != 0;
-  const uint32_t cum = base + kOffCum, dts = base + kOffDt, ecum = base + kOffEc;
+  const uint32_t cum = base + kOffCum, dts = base + kOffDt;
   const int64_t H = p.H, L = p.L;
   const bool rev = q >= 2;
   const float *Ap = pick4(p.A, q);
@@ -755,7 +739,6 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
         if (rev) v = __shfl_sync(0xffffffffu, v, 31) - v + v0;
         sts_f32(cum + ((ct * 4 + q) * 32 + lane) * 4, v);
         sts_f32(dts + ((ct * 4 + q) * 32 + lane) * 4, dt_cur);
-        if (!rev) sts_f32(ecum + ((ct * 2 + q) * 32 + lane) * 4, ex2_approx(v));
       }
       if (dact) sts_f32(base + kOffDtab + (ct * 4 + (gt >> 4)) * 4, Dv);
       if (gt == 0) sts_s32(base + kOffFtab + ct * 4, kk == 0 ? 1 + (m & 1) : 0);
@@ -989,7 +972,7 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
   const int fs = noisy ? kNF : kCF;
   void *yout = noisy ? p.y_noisy : p.y_clean;
   const bool mine = (noisy ? p.allblock != 0 : true) && yout != nullptr;
-  const uint32_t ecum = base + kOffEc;
+  const uint32_t cumt = base + kOffCum;
   const int64_t H = p.H, L = p.L;
   if (p.agg) return;
   const bool act = pick4(p.active, q) != 0;
@@ -1013,7 +996,7 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
       const uint32_t cq = base + kOffCum + (ct * 4 + q) * 128;
       const float cs = lds_f32(cq + lane * 4);
       const float ds = lds_f32(base + kOffDt + (ct * 4 + q) * 128 + lane * 4);
-      const uint32_t mrow = base + kOffMh + (jm & 1) * kMhBuf + q * 2048;
+      const uint32_t mrow = base + kOffMh + (jm & 1) * kMhBuf + q * kMhDir;
       // this direction's D joins the diagonal of M (D x is part of X^T M^T):
       // M[s][s] + D is stored as bf16 hi in M and its bf16 remainder lo on the
       // diagonal of the block's 16 x 16 correction tile of chunk s / 16
@@ -1037,10 +1020,8 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
           if (t == lane) {
             const float v = mv[i] + Dq;
             const float hi = __bfloat162float(__float2bfloat16_rn(v));
-            const int d = lane & 15;
-            const uint32_t off = static_cast<uint32_t>(jm & 1) * kDgBuf + (d >> 3) * kDgSbo + (d >> 3) * kDgLbo +
-                                 (d & 7) * 16 + (d & 7) * 2;
-            sts_u16(base + kOffDg + (2 * q + (lane >> 4)) * 512 + off, __bfloat16_as_ushort(__float2bfloat16_rn(v - hi)));
+            sts_u16(mrow + inter_mn_off(32 + lane, lane, kMhSbo, kMhLbo),
+                    __bfloat16_as_ushort(__float2bfloat16_rn(v - hi)));
             mv[i] = v;
           }
         }
@@ -1065,20 +1046,24 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
       if (!waitw(c, bYFull0 + i2, par2(j))) return;
       tc_fence_after();
       uint32_t yo[32], yd[32];
-      const uint32_t ta = tmem_addr(tmem, 32 * q, kColY0 + 128 * i2);
-      tmem_ld_16x32bx2_x32<32>(ta, yo);
-      tmem_ld_16x32bx2_x32<32>(ta + 64, yd);
+      const uint32_t ta = tmem_addr(tmem, 32 * q, kColY0 + kColYBuf * i2);
+      tmem_ld_16x32bx2_x32<32>(ta, yo);       // Y_off: clean columns 0.., noisy 32..
+      tmem_ld_16x32bx2_x32<64>(ta + 64, yd);  // Y_diag: clean 64.., noisy 128..
       tmem_ld_wait();
-      const uint32_t eq = ecum + (ct * 2 + fs) * 128;
+      const uint32_t eq = cumt + (ct * 4 + fs) * 128;
 #pragma unroll
       for (int jj = 0; jj < 8; ++jj) {
-        float e4[4];
-        ld_shared_v4f(eq + 16 * jj, e4);
+        float c4[4];
+        ld_shared_v4f(eq + 16 * jj, c4);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          yo[4 * jj + i] =
-              __float_as_uint(fmaf(e4[i], __uint_as_float(yo[4 * jj + i]), __uint_as_float(yd[4 * jj + i])));
+          yo[4 * jj + i] = __float_as_uint(
+              fmaf(ex2_approx(c4[i]), __uint_as_float(yo[4 * jj + i]), __uint_as_float(yd[4 * jj + i])));
       }
+      tmem_ld_16x32bx2_x32<64>(ta + 96, yd);  // the diagonal remainders: clean 96.., noisy 160..
+      tmem_ld_wait();
+#pragma unroll
+      for (int t = 0; t < 32; ++t) yo[t] = __float_as_uint(__uint_as_float(yo[t]) + __uint_as_float(yd[t]));
       // the Y buffer may be reused from here on
       tc_fence_before();
       arrive_lane0(c, bYEmpty0 + i2);
@@ -1130,11 +1115,12 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
     *reinterpret_cast<int **>(sm + kOffMisc + 16) = p.status;
     fence_mbar_init();
   }
-  // Clear the diagonal correction tiles (only their diagonals are written).
+  // Clear the intra-block operands: of their remainder halves only the
+  // diagonals are ever written.
   if (!p.agg) {
     const uint4 zero = make_uint4(0, 0, 0, 0);
-    for (uint32_t o = threadIdx.x * 16; o < 2 * kDgBuf; o += kThreads * 16)
-      *reinterpret_cast<uint4 *>(sm + kOffDg + o) = zero;
+    for (uint32_t o = threadIdx.x * 16; o < 2 * kMhBuf; o += kThreads * 16)
+      *reinterpret_cast<uint4 *>(sm + kOffMh + o) = zero;
     fence_proxy_async_smem();
   }
   if (warp == 1) {
