@@ -46,10 +46,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one bd_tc_kernel
 # launch on this workload, from one ncu capture, and the hash of the kernel
 # source it was taken on: reported while the source is unchanged, null after.
-TC_TRAFFIC = {"bytes": 224_177_152 + 547_994_880,
+TC_TRAFFIC = {"bytes": 224_074_240 + 548_320_768,
               "sources": ("bidirectional_mamba_state_b200/csrc/scan_tc.cu",
                           "bidirectional_mamba_state_b200/csrc/sm100.cuh"),
-              "sha256": "2e58528e6a3a59f9c71fb41f15477626766f838c56ee62013734d97b81a81287"}
+              "sha256": "f9701e4af1b27b705f682b3397bf8da8a78bb0b7d6a0de103cedaf3ef1334b49"}
 
 
 def tc_traffic():
@@ -391,6 +391,7 @@ EXTRA = {
     "conv_block_step_700m_b1_24layers": lambda dev, pk: _step_stack(W.WORKLOADS["700m_step"], 24, dev, pk,
                                                                     conv_width=4),
     "gated_rmsnorm_87m": lambda dev, pk: _norm(W.WORKLOADS["87m_allblock"], dev, pk),
+    "step_flatness_700m": lambda dev, pk: _step_flatness(dev, pk),
     "conv_block_step_norm_700m_b1_24layers": lambda dev, pk: _step_stack(W.WORKLOADS["700m_step"], 24, dev,
                                                                          pk, conv_width=4, norm=True),
 }
@@ -554,6 +555,29 @@ def _prefill(s: W.Shape, dev, pk) -> dict:
     b = RL.prefix_bytes(s, block_states=False)
     return {"us_per_layer": ms * 1e3, "tokens_per_s": s.batch * s.seqlen / (ms * 1e-3),
             "algorithmic_bytes": b, "hbm_frac": b / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+
+
+def _step_flatness(dev, pk) -> dict:
+    """Per-step cost against context length: prefill one 700M layer at 8K, 32K
+    and 64K tokens (final state only), then time a denoising step (block_step
+    over the active 32-token block) from each cached state.  The step reads only
+    the fixed-size state, so its time must not grow with the context."""
+    out = {}
+    st = W.WORKLOADS["700m_step"]
+    a, r = W.make_streams(st, 7, device=dev, streams=(W.CLEAN_FWD, W.CLEAN_REV))
+    ws = bd.workspace(st, bd.BDSCAN_OP_BLOCK_STEP, dev)
+    y = torch.empty((st.batch, st.seqlen, st.nheads, st.headdim), device=dev)
+    for name in ("700m_prefill_8k", "700m_prefill_32k", "700m_prefill_64k"):
+        s = W.WORKLOADS[name]
+        f, rr = W.make_streams(s, W.SEEDS[name], device=dev, streams=(W.CLEAN_FWD, W.CLEAN_REV))
+        _, _, fin = bd.prefix(s, f, rr, want_states=False)
+        del f, rr
+        ms = _time(lambda: bd.block_step(st, a, r, fin, y=y, ws=ws), dev, 50, 5)
+        out[f"us_per_step_after_{s.seqlen // 1024}k"] = ms * 1e3
+    v = list(out.values())
+    out["max_over_min"] = max(v) / min(v)
+    out["layers"] = 1
+    return out
 
 
 def run_reference(args):
