@@ -186,15 +186,18 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
     for (int64_t e = tid; e < PN; e += kBwdThreads) s.hs[e] = src[e];
   }
   __syncthreads();
+  // Transposed copies, skewed: consecutive threads take consecutive columns
+  // and rotated rows (i = (j + column) mod T), so that neither the row-major
+  // reads nor the transposed writes of a warp fall into one shared-memory bank.
   for (int e = tid; e < T * P; e += kBwdThreads) {
-    const int pp = e / T, i = e % T;
-    s.xt[e] = s.x[i * P + pp];
-    s.dyt[e] = s.dy[i * P + pp];
+    const int pp = e % P, i = (e / P + pp) % T;
+    s.xt[pp * T + i] = s.x[i * P + pp];
+    s.dyt[pp * T + i] = s.dy[i * P + pp];
   }
   for (int e = tid; e < T * N; e += kBwdThreads) {
-    const int n = e / T, i = e % T;
-    s.Bt[e] = s.Bm[i * N + n];
-    s.Ct[e] = s.Cm[i * N + n];
+    const int n = e % N, i = (e / N + n) % T;
+    s.Bt[n * T + i] = s.Bm[i * N + n];
+    s.Ct[n * T + i] = s.Cm[i * N + n];
   }
   if (tid == 0) {
     float c = 0.f;
