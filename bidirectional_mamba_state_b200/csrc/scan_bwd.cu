@@ -80,7 +80,7 @@ struct BwdSmem {
   float *WCB, *YX, *G2;     // [T][T]: W o (C B^T), dy x^T, W o (dy x^T)
   float *Q;                 // [T][T + 1]: W o (C B^T) o (dy x^T), padded rows
   float *hsCt, *dhBt;       // [P][T]: (h_s C^T)^T, (dh_e B^T)^T
-  float *hs, *carry;        // [P][N]
+  float *hs, *carry;        // [P][N + 4]: rows padded so that rows p, p+1, ... fall into different banks
 };
 
 __device__ float block_sum(float v, float *red) {
@@ -154,6 +154,7 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
                           float &accD) {
   const BwdDir &d = p.dir[kind];
   const int T = p.T, P = p.P, N = p.N, H = p.H, L = p.L, G = p.G, K = p.K;
+  const int NS = N + 4;  // row stride of hs and carry
   const int g = h / (H / G);
   const int tid = threadIdx.x;
   const bool rev = kind == 1 || kind == 3;
@@ -183,7 +184,7 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
   if (has_hs) {
     const float *src = k > 0 ? p.states + ((static_cast<int64_t>(b) * K + (k - 1)) * H + h) * PN
                              : p.h0 + (static_cast<int64_t>(b) * H + h) * PN;
-    for (int64_t e = tid; e < PN; e += kBwdThreads) s.hs[e] = src[e];
+    for (int64_t e = tid; e < PN; e += kBwdThreads) s.hs[(e / N) * NS + e % N] = src[e];
   }
   __syncthreads();
   // Transposed copies, skewed: consecutive threads take consecutive columns
@@ -211,13 +212,13 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
   __syncthreads();
 
   // ---- Gram matrices: C B^T and dy x^T
-  sgemm<1>(T, T, N, s.Cm, N, 1, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+  sgemm<1>(T, T, N, s.Ct, 1, T, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
         [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
           for (int i = 0; i < R; ++i)
             *reinterpret_cast<float4 *>(s.WCB + (m0 + i) * T + n0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
         });
-  sgemm<1>(T, T, P, s.dy, P, 1, nul, s.xt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+  sgemm<1>(T, T, P, s.dyt, 1, T, nul, s.xt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
         [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
           for (int i = 0; i < R; ++i)
@@ -225,14 +226,14 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
         });
   // ---- products with the start state and the end-state gradient
   if (has_hs)
-    sgemm<2>(P, T, N, s.hs, N, 1, nul, s.Ct, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+    sgemm<2>(P, T, N, s.hs, NS, 1, nul, s.Ct, T, 0, nullptr, 0, 0, nul, nullptr, 0,
           [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
             for (int i = 0; i < R; ++i)
               *reinterpret_cast<float4 *>(s.hsCt + (m0 + i) * T + n0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
           });
   if (has_dhe)
-    sgemm<2>(P, T, N, s.carry, N, 1, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+    sgemm<2>(P, T, N, s.carry, NS, 1, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
           [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
             for (int i = 0; i < R; ++i)
@@ -242,7 +243,7 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
   if (has_dhe) {
     const float *he = p.states + ((static_cast<int64_t>(b) * K + k) * H + h) * PN;
     float part = 0.f;
-    for (int64_t e = tid; e < PN; e += kBwdThreads) part += s.carry[e] * he[e];
+    for (int64_t e = tid; e < PN; e += kBwdThreads) part += s.carry[(e / N) * NS + e % N] * he[e];
     he_dot = block_sum(part, s.red);
   }
   __syncthreads();
@@ -275,7 +276,7 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
           }
         });
   // dC_i = sum_u G2[i][u] dt_u B_u (+ Lam_i dy_i^T h_s)
-  sgemm<4>(T, N, T, s.G2, T, 1, s.dt, s.Bm, N, has_hs ? P : 0, has_hs ? s.dy : nullptr, P, 1, s.lam, s.hs, N,
+  sgemm<4>(T, N, T, s.G2, T, 1, s.dt, s.Bm, N, has_hs ? P : 0, has_hs ? s.dy : nullptr, P, 1, s.lam, s.hs, NS,
         [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
           for (int i = 0; i < R; ++i)
@@ -283,7 +284,7 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
                 make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
         });
   // dB_u = dt_u (sum_i G2[i][u] C_i (+ r_u x_u^T dh_e))
-  sgemm<4>(T, N, T, s.G2, 1, T, nul, s.Cm, N, has_dhe ? P : 0, has_dhe ? s.x : nullptr, P, 1, s.r, s.carry, N,
+  sgemm<4>(T, N, T, s.G2, 1, T, nul, s.Cm, N, has_dhe ? P : 0, has_dhe ? s.x : nullptr, P, 1, s.r, s.carry, NS,
         [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
           for (int i = 0; i < R; ++i) {
@@ -335,7 +336,7 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
           [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
             for (int i = 0; i < R; ++i) {
-              float4 *cp = reinterpret_cast<float4 *>(s.carry + (m0 + i) * N + n0);
+              float4 *cp = reinterpret_cast<float4 *>(s.carry + (m0 + i) * NS + n0);
               float4 c = *cp;
               if (kind == 0) {
                 c.x *= lame; c.y *= lame; c.z *= lame; c.w *= lame;
@@ -374,12 +375,14 @@ __global__ void __launch_bounds__(kBwdThreads) bd_bwd_kernel(const __grid_consta
   s.Q = q; q += T * (T + 1);  // (a multiple of 4 floats: the buffers after it stay 16-byte aligned)
   s.hsCt = q; q += P * T;
   s.dhBt = q; q += P * T;
-  s.hs = q; q += PN;
+  const int NS = N + 4;  // padded row stride of hs and carry
+  s.hs = q; q += static_cast<int64_t>(P) * NS;
   s.carry = q;
   const int b = blockIdx.x / H, h = blockIdx.x % H;
   // carry = dL/dstates[K-1] (given part)
   for (int64_t e = threadIdx.x; e < PN; e += kBwdThreads)
-    s.carry[e] = p.dstates ? p.dstates[((static_cast<int64_t>(b) * K + (K - 1)) * H + h) * PN + e] : 0.f;
+    s.carry[(e / N) * NS + e % N] =
+        p.dstates ? p.dstates[((static_cast<int64_t>(b) * K + (K - 1)) * H + h) * PN + e] : 0.f;
   __syncthreads();
   float accA[4] = {0.f, 0.f, 0.f, 0.f}, accD[4] = {0.f, 0.f, 0.f, 0.f};
   for (int k = K - 1; k >= 0; --k) {
@@ -389,13 +392,13 @@ __global__ void __launch_bounds__(kBwdThreads) bd_bwd_kernel(const __grid_consta
     if (p.active[3]) bwd_block(p, s, 3, b, h, k, accA[3], accD[3]);
     if (k > 0 && p.dstates) {
       for (int64_t e = threadIdx.x; e < PN; e += kBwdThreads)
-        s.carry[e] += p.dstates[((static_cast<int64_t>(b) * K + (k - 1)) * H + h) * PN + e];
+        s.carry[(e / N) * NS + e % N] += p.dstates[((static_cast<int64_t>(b) * K + (k - 1)) * H + h) * PN + e];
       __syncthreads();
     }
   }
   if (p.dh0)
     for (int64_t e = threadIdx.x; e < PN; e += kBwdThreads)
-      p.dh0[(static_cast<int64_t>(b) * H + h) * PN + e] = s.carry[e];
+      p.dh0[(static_cast<int64_t>(b) * H + h) * PN + e] = s.carry[(e / N) * NS + e % N];
   if (threadIdx.x == 0)
     for (int di = 0; di < 4; ++di)
       if (p.active[di]) {
@@ -441,7 +444,7 @@ __global__ void bd_bwd_reduce_head_kernel(const float *pA, const float *pD, floa
 
 size_t bwd_smem_bytes(int64_t P, int64_t N, int64_t T) {
   const int64_t floats = 4 * T * P + 4 * T * N + 6 * T + kBwdThreads + 3 * T * T + T * (T + 1) + 2 * P * T +
-                         2 * P * N;
+                         2 * P * (N + 4);
   return static_cast<size_t>(floats) * sizeof(float);
 }
 
