@@ -269,6 +269,7 @@ def run_ours(args):
                      "frac": achieved / pk["hbm_gbs"], "traffic": tc_traffic(),
                      "algorithmic_bytes_per_launch": bytes_step,
                      "peak_source": f"{pk['source']} hbm_gbs",
+                     "frac_of_nominal_8tbs": achieved / 8000.0,
                      "tensor_tflops": flops / (ms_step * 1e-3) / 1e12,
                      "tensor_frac_of_bf16": flops / (ms_step * 1e-3) / 1e12 / pk["bf16_tflops"]},
         "gpu_launches": launches_per_step * args.steps,
