@@ -83,14 +83,16 @@ struct BwdSmem {
   float *hs, *carry;        // [P][N + 4]: rows padded so that rows p, p+1, ... fall into different banks
 };
 
+// Sum over the CTA in a fixed order (a shuffle tree per warp, then the warp
+// sums in warp order): deterministic, two barriers.
 __device__ float block_sum(float v, float *red) {
-  red[threadIdx.x] = v;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
   __syncthreads();
-  for (int s = kBwdThreads / 2; s > 0; s >>= 1) {
-    if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
-    __syncthreads();
-  }
-  const float r = red[0];
+  float r = 0.f;
+#pragma unroll
+  for (int w = 0; w < kBwdThreads / 32; ++w) r += red[w];
   __syncthreads();
   return r;
 }
