@@ -95,6 +95,10 @@ def lib() -> ctypes.CDLL:
             L.bdscan_block_step_noalloc.restype = ctypes.c_int
             L.bdscan_noalloc_scratch.argtypes = []
             L.bdscan_noalloc_scratch.restype = ctypes.c_void_p
+            L.bdscan_set_option.argtypes = [ctypes.c_int, ctypes.c_longlong]
+            L.bdscan_set_option.restype = ctypes.c_longlong
+            L.bdscan_get_option.argtypes = [ctypes.c_int]
+            L.bdscan_get_option.restype = ctypes.c_longlong
             L.bdscan_check_status.argtypes = [vp, vp]
             L.bdscan_status_string.argtypes = [ctypes.c_int]
             L.bdscan_status_string.restype = ctypes.c_char_p
@@ -170,6 +174,34 @@ def bdscan_version() -> int:
     return int(lib().bdscan_version())
 
 
+BDSCAN_OPT_WAIT_TIMEOUT_NS, BDSCAN_OPT_FORCE_GENERIC, BDSCAN_OPT_VERBOSE = 0, 1, 2
+
+
+def bdscan_set_option(option: int, value: int) -> int:
+    return int(lib().bdscan_set_option(int(option), int(value)))
+
+
+def bdscan_get_option(option: int) -> int:
+    return int(lib().bdscan_get_option(int(option)))
+
+
+class option:
+    """Context manager that sets a process-wide option and restores it."""
+
+    def __init__(self, opt: int, value: int):
+        self.opt, self.value = opt, value
+
+    def __enter__(self):
+        old = bdscan_set_option(self.opt, self.value)
+        if old < 0 and self.opt != BDSCAN_OPT_WAIT_TIMEOUT_NS:
+            raise BdscanError("bdscan_set_option", old, "bad option or value")
+        self.old = old
+        return self
+
+    def __exit__(self, *exc):
+        bdscan_set_option(self.opt, self.old)
+
+
 # ----------------------------------------------------------------------------- torch-facing
 _DT = {"bf16": (torch.bfloat16, BDSCAN_BF16), "fp32": (torch.float32, BDSCAN_FP32)}
 
@@ -222,6 +254,18 @@ def _stream(device, stream=None) -> int:
     return s.cuda_stream
 
 
+def _check_ws(ws, s: Shape, op: int, device):
+    """A caller-provided workspace: a contiguous uint8 tensor on ``device``
+    with at least bdscan_workspace_size(shape, op) bytes."""
+    if ws.device != device:
+        raise ValueError(f"ws is on {ws.device}, expected {device}")
+    if ws.dtype != torch.uint8 or ws.dim() != 1 or not ws.is_contiguous():
+        raise ValueError("ws must be a contiguous 1-D uint8 tensor")
+    need = bdscan_workspace_size(ctypes.byref(c_shape(s)), op)
+    if ws.numel() < need:
+        raise ValueError(f"ws holds {ws.numel()} bytes, the call needs {need}")
+
+
 def workspace(s: Shape, op: int, device) -> torch.Tensor:
     n = bdscan_workspace_size(ctypes.byref(c_shape(s)), op)
     if n == 0:
@@ -258,10 +302,21 @@ def prefix(s: Shape, fwd: dict, rev: dict | None = None, h0=None, want_states: b
     cs, cf, cr = c_shape(s), c_dir(s, fwd, dev), c_dir(s, rev, dev)
     if h0 is not None:
         _check_tensor("h0", h0, (s.batch, s.nheads, s.headdim, s.dstate), torch.float32, dev)
-    y = _out(s, dev) if y is None else y
-    states = (_state(s, dev, s.nblocks) if want_states else None) if states is None else states
-    final = (_state(s, dev) if want_final else None) if final is None else final
-    ws = workspace(s, BDSCAN_OP_PREFIX, dev) if ws is None else ws
+    B, L, H, P, N = s.batch, s.seqlen, s.nheads, s.headdim, s.dstate
+    if y is None:
+        y = _out(s, dev)
+    _check_tensor("y", y, (B, L, H, P), _DT[s.out_dtype][0], dev)
+    if states is None:
+        states = _state(s, dev, s.nblocks) if want_states else None
+    else:
+        _check_tensor("states", states, (B, s.nblocks, H, P, N), torch.float32, dev)
+    if final is None:
+        final = _state(s, dev) if want_final else None
+    else:
+        _check_tensor("final", final, (B, H, P, N), torch.float32, dev)
+    if ws is None:
+        ws = workspace(s, BDSCAN_OP_PREFIX, dev)
+    _check_ws(ws, s, BDSCAN_OP_PREFIX, dev)
     rc = bdscan_prefix(ctypes.byref(cs), ctypes.byref(cf), _ref(cr), _ptr(h0), _ptr(y), _ptr(states),
                        _ptr(final), _ptr(ws), ws.numel(), _stream(dev, stream))
     _raise("bdscan_prefix", rc)
@@ -278,8 +333,14 @@ def block_step(s: Shape, fwd: dict, rev: dict | None, state_in, state_out=None, 
     _check_tensor("state_in", state_in, (s.batch, s.nheads, s.headdim, s.dstate), torch.float32, dev)
     if state_out is True:
         state_out = _state(s, dev)
-    y = _out(s, dev) if y is None else y
-    ws = workspace(s, BDSCAN_OP_BLOCK_STEP, dev) if ws is None else ws
+    elif state_out is not None:
+        _check_tensor("state_out", state_out, (s.batch, s.nheads, s.headdim, s.dstate), torch.float32, dev)
+    if y is None:
+        y = _out(s, dev)
+    _check_tensor("y", y, (s.batch, s.seqlen, s.nheads, s.headdim), _DT[s.out_dtype][0], dev)
+    if ws is None:
+        ws = workspace(s, BDSCAN_OP_BLOCK_STEP, dev)
+    _check_ws(ws, s, BDSCAN_OP_BLOCK_STEP, dev)
     rc = bdscan_block_step(ctypes.byref(cs), ctypes.byref(cf), _ref(cr), _ptr(state_in), _ptr(y),
                            _ptr(state_out), _ptr(ws), ws.numel(), _stream(dev, stream))
     _raise("bdscan_block_step", rc)
@@ -296,10 +357,20 @@ def allblock(s: Shape, clean_fwd: dict, clean_rev: dict | None, noisy_fwd: dict,
     nf, nr = c_dir(s, noisy_fwd, dev), c_dir(s, noisy_rev, dev)
     if h0 is not None:
         _check_tensor("h0", h0, (s.batch, s.nheads, s.headdim, s.dstate), torch.float32, dev)
-    y_clean = (_out(s, dev) if want_clean else None) if y_clean is None else y_clean
-    y_noisy = _out(s, dev) if y_noisy is None else y_noisy
-    states = _state(s, dev, s.nblocks) if states is None else states
-    ws = workspace(s, BDSCAN_OP_ALLBLOCK, dev) if ws is None else ws
+    yshape, tout = (s.batch, s.seqlen, s.nheads, s.headdim), _DT[s.out_dtype][0]
+    if y_clean is None:
+        y_clean = _out(s, dev) if want_clean else None
+    else:
+        _check_tensor("y_clean", y_clean, yshape, tout, dev)
+    if y_noisy is None:
+        y_noisy = _out(s, dev)
+    _check_tensor("y_noisy", y_noisy, yshape, tout, dev)
+    if states is None:
+        states = _state(s, dev, s.nblocks)
+    _check_tensor("states", states, (s.batch, s.nblocks, s.nheads, s.headdim, s.dstate), torch.float32, dev)
+    if ws is None:
+        ws = workspace(s, BDSCAN_OP_ALLBLOCK, dev)
+    _check_ws(ws, s, BDSCAN_OP_ALLBLOCK, dev)
     rc = bdscan_allblock(ctypes.byref(cs), ctypes.byref(cf), _ref(cr), ctypes.byref(nf), _ref(nr),
                          _ptr(h0), _ptr(y_clean), _ptr(y_noisy), _ptr(states), _ptr(ws), ws.numel(),
                          _stream(dev, stream))
@@ -337,9 +408,20 @@ def allblock_backward(s: Shape, clean_fwd: dict, clean_rev: dict | None, noisy_f
                  {"x": torch.empty((B, L, H, P), **f), "dt": torch.empty((B, L, H), **f),
                   "B": torch.empty((B, L, G, N), **f), "C": torch.empty((B, L, G, N), **f),
                   "A": torch.empty((H,), **f), "D": torch.empty((H,), **f)} for d in dirs]
-    cg = [None if g is None else bdscan_grad_t(*(_ptr(g[k]) for k in GRAD_KEYS)) for g in grads]
+    gshapes = {"x": (B, L, H, P), "dt": (B, L, H), "B": (B, L, G, N), "C": (B, L, G, N), "A": (H,), "D": (H,)}
+    for i, (d, g) in enumerate(zip(dirs, grads)):
+        if d is None:
+            continue
+        if g is None:
+            raise ValueError(f"grads[{i}] is required for a present direction")
+        for k in GRAD_KEYS:
+            _check_tensor(f"grads[{i}][{k}]", g[k], gshapes[k], torch.float32, dev)
+    cg = [None if g is None or d is None else bdscan_grad_t(*(_ptr(g[k]) for k in GRAD_KEYS))
+          for d, g in zip(dirs, grads)]
     dh0 = _state(s, dev) if want_dh0 else None
-    ws = workspace(s, BDSCAN_OP_ALLBLOCK_BACKWARD, dev) if ws is None else ws
+    if ws is None:
+        ws = workspace(s, BDSCAN_OP_ALLBLOCK_BACKWARD, dev)
+    _check_ws(ws, s, BDSCAN_OP_ALLBLOCK_BACKWARD, dev)
     rc = bdscan_allblock_backward(ctypes.byref(cs), _ref(cd[0]), _ref(cd[1]), _ref(cd[2]), _ref(cd[3]),
                                   _ptr(h0), _ptr(states), _ptr(dy_clean), _ptr(dy_noisy), _ptr(dstates),
                                   _ref(cg[0]), _ref(cg[1]), _ref(cg[2]), _ref(cg[3]), _ptr(dh0), _ptr(ws),

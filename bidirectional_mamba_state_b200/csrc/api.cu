@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
@@ -14,6 +15,36 @@
 #include "bdscan.h"
 #include "bdscan_internal.h"
 #include <nvtx3/nvToolsExt.h>
+
+// ---- process-wide options ------------------------------------------------------
+namespace bdscan {
+namespace {
+
+struct Options {
+  std::atomic<unsigned long long> wait_timeout_ns{2000000000ull};
+  std::atomic<int> force_generic{0};
+  std::atomic<int> verbose{0};
+  Options() {
+    // initial values from the environment, read once
+    if (const char *v = std::getenv("BDSCAN_WAIT_TIMEOUT_NS"); v && *v)
+      wait_timeout_ns = std::strtoull(v, nullptr, 10);
+    if (const char *v = std::getenv("BDSCAN_FORCE_GENERIC"); v && v[0] == '1') force_generic = 1;
+    if (const char *v = std::getenv("BDSCAN_VERBOSE"); v && v[0] == '1') verbose = 1;
+  }
+};
+
+Options &options() {
+  static Options o;
+  return o;
+}
+
+}  // namespace
+
+unsigned long long opt_wait_timeout_ns() { return options().wait_timeout_ns.load(std::memory_order_relaxed); }
+bool opt_force_generic() { return options().force_generic.load(std::memory_order_relaxed) != 0; }
+bool opt_verbose() { return options().verbose.load(std::memory_order_relaxed) != 0; }
+
+}  // namespace bdscan
 
 using bdscan::DirArgs;
 using bdscan::Mode;
@@ -159,8 +190,7 @@ int launch(ScanArgs &a, cudaStream_t stream) {
   }
   cudaError_t e = tc ? bdscan::launch_tc(a, stream) : bdscan::launch_seq(a, stream);
   if (e != cudaSuccess) {
-    const char *v = std::getenv("BDSCAN_VERBOSE");
-    if (v && v[0] == '1') std::fprintf(stderr, "libbdscan: launch failed: %s\n", cudaGetErrorString(e));
+    if (bdscan::opt_verbose()) std::fprintf(stderr, "libbdscan: launch failed: %s\n", cudaGetErrorString(e));
     return BDSCAN_ERR_CUDA;
   }
   return BDSCAN_OK;
@@ -401,8 +431,7 @@ int bdscan_allblock_backward(const bdscan_shape_t *shape, const bdscan_dir_t *cl
   a.ws = static_cast<uint8_t *>(ws) + bdscan::kWsHeader;
   cudaError_t e = bdscan::launch_bwd(a, stream);
   if (e != cudaSuccess) {
-    const char *v = std::getenv("BDSCAN_VERBOSE");
-    if (v && v[0] == '1') std::fprintf(stderr, "libbdscan: launch failed: %s\n", cudaGetErrorString(e));
+    if (bdscan::opt_verbose()) std::fprintf(stderr, "libbdscan: launch failed: %s\n", cudaGetErrorString(e));
     return BDSCAN_ERR_CUDA;
   }
   return BDSCAN_OK;
@@ -439,6 +468,32 @@ const char *bdscan_status_string(int status) {
 
 int bdscan_version(void) { return 100; }
 
+long long bdscan_set_option(int option, long long value) {
+  auto &o = bdscan::options();
+  switch (option) {
+    case BDSCAN_OPT_WAIT_TIMEOUT_NS:
+      if (value < 0) return BDSCAN_ERR_INVALID_ARG;
+      return (long long)o.wait_timeout_ns.exchange((unsigned long long)value);
+    case BDSCAN_OPT_FORCE_GENERIC:
+      if (value != 0 && value != 1) return BDSCAN_ERR_INVALID_ARG;
+      return o.force_generic.exchange((int)value);
+    case BDSCAN_OPT_VERBOSE:
+      if (value != 0 && value != 1) return BDSCAN_ERR_INVALID_ARG;
+      return o.verbose.exchange((int)value);
+    default:
+      return BDSCAN_ERR_INVALID_ARG;
+  }
+}
+
+long long bdscan_get_option(int option) {
+  switch (option) {
+    case BDSCAN_OPT_WAIT_TIMEOUT_NS: return (long long)bdscan::opt_wait_timeout_ns();
+    case BDSCAN_OPT_FORCE_GENERIC: return bdscan::opt_force_generic() ? 1 : 0;
+    case BDSCAN_OPT_VERBOSE: return bdscan::opt_verbose() ? 1 : 0;
+    default: return BDSCAN_ERR_INVALID_ARG;
+  }
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------- no-alloc step
@@ -452,20 +507,53 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
-void *g_noalloc_ptr[kMaxDevices] = {};
+struct ScratchAddr {
+  void *ctx;  // the context the address was looked up in
+  void *ptr;
+};
+ScratchAddr g_noalloc[kMaxDevices] = {};
+
+// The driver's cuCtxGetCurrent, through the runtime's entry-point query (the
+// library links only the runtime).
+using CtxGetCurrentFn = int (*)(void **);
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
 
 // Device address of the scratch buffer on the current device, looked up once per
-// device (with that device current); nullptr if the lookup fails.
+// device and context (with that device current): a device reset or a new primary
+// context reloads the module, and the address is looked up again in the new
+// context.  nullptr if a lookup fails.
 void *noalloc_scratch_ptr() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  CtxGetCurrentFn get = ctx_get_current_fn();
+  void *ctx = nullptr;
+  if (!get || get(&ctx) != 0) return nullptr;
+  if (!ctx) {
+    // no context bound to this thread yet: the symbol lookup makes the
+    // device's primary context current
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || get(&ctx) != 0 || !ctx) return nullptr;
+  }
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  ScratchAddr &e = g_noalloc[dev];
+  if (!e.ptr || e.ctx != ctx) {
     void *ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    g_noalloc_ptr[dev] = ptr;
+    e.ctx = ctx;
+    e.ptr = ptr;
   }
-  return g_noalloc_ptr[dev];
+  return e.ptr;
 }
 
 }  // namespace
@@ -574,8 +662,7 @@ int conv_launch(const bdscan::ConvArgs &a, const ConvSizes &z, cudaStream_t stre
   }
   cudaError_t e = bdscan::launch_conv(a, stream);
   if (e != cudaSuccess) {
-    const char *v = std::getenv("BDSCAN_VERBOSE");
-    if (v && v[0] == '1') std::fprintf(stderr, "libbdscan: conv launch failed: %s\n", cudaGetErrorString(e));
+    if (bdscan::opt_verbose()) std::fprintf(stderr, "libbdscan: conv launch failed: %s\n", cudaGetErrorString(e));
     return BDSCAN_ERR_CUDA;
   }
   return BDSCAN_OK;
@@ -677,8 +764,7 @@ int bdscan_gated_rmsnorm(const bdscan_shape_t *shape, const void *y, const void 
   a.z_bf16 = shape->in_dtype == BDSCAN_BF16;
   cudaError_t e = bdscan::launch_norm(a, static_cast<cudaStream_t>(cuda_stream));
   if (e != cudaSuccess) {
-    const char *v = std::getenv("BDSCAN_VERBOSE");
-    if (v && v[0] == '1') std::fprintf(stderr, "libbdscan: norm launch failed: %s\n", cudaGetErrorString(e));
+    if (bdscan::opt_verbose()) std::fprintf(stderr, "libbdscan: norm launch failed: %s\n", cudaGetErrorString(e));
     return BDSCAN_ERR_CUDA;
   }
   return BDSCAN_OK;

@@ -7,6 +7,12 @@ namespace bdscan {
 
 enum class Mode : int { Prefix = 0, Step = 1, AllBlock = 2 };
 
+// Process-wide options (bdscan_set_option); read from the environment once,
+// at the first use, not per call.
+unsigned long long opt_wait_timeout_ns();
+bool opt_force_generic();
+bool opt_verbose();
+
 struct DirArgs {
   const void *x, *dt, *B, *C, *z;  // z == nullptr: no gate
   const float *A, *D;

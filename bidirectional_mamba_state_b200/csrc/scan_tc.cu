@@ -1253,12 +1253,6 @@ bool device_is_sm100() {
   return cached == 1;
 }
 
-unsigned long long env_ns(const char *name, unsigned long long dflt) {
-  const char *v = std::getenv(name);
-  if (!v || !*v) return dflt;
-  return std::strtoull(v, nullptr, 10);
-}
-
 }  // namespace
 
 bool tc_shape_ok(int64_t P, int64_t N, int64_t T, bool in_bf16) {
@@ -1304,8 +1298,7 @@ bool tc_supported(const ScanArgs &a) {
   if (a.Bsz * a.H > 0x7fffffffLL || a.L > 0x7fffffffLL || 4 * a.Bsz * (a.L / kT) * a.G > 0x7fffffffLL)
     return false;
   if (a.ws_bytes < kWsHeader + tc_workspace_bytes(a.Bsz, a.L, a.G, a.H)) return false;
-  const char *force = std::getenv("BDSCAN_FORCE_GENERIC");
-  if (force && force[0] == '1') return false;
+  if (opt_force_generic()) return false;
   return device_is_sm100();
 }
 
@@ -1314,7 +1307,7 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
   const DirArgs *ds[4] = {&a.cf, all ? &a.nf : nullptr, a.has_cr ? &a.cr : nullptr,
                           (all && a.has_nr) ? &a.nr : nullptr};
   __nv_bfloat16 *cbws = reinterpret_cast<__nv_bfloat16 *>(static_cast<uint8_t *>(a.ws) + kWsHeader);
-  const unsigned long long timeout = env_ns("BDSCAN_WAIT_TIMEOUT_NS", 2000000000ull);
+  const unsigned long long timeout = opt_wait_timeout_ns();
   const int K = static_cast<int>(a.L / kT);
 
   // ---- C B^T of every active direction

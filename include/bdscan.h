@@ -27,10 +27,13 @@
  *              forward state after token (k+1)*T - 1 (end of block k).
  *
  * Ownership: the caller owns every buffer, including the workspace; the
- * library allocates no device memory and keeps no global mutable state, so
- * calls are reentrant.  All device pointers must be device-accessible memory
- * of the current device.  Every call is asynchronous on `cuda_stream` (a
- * cudaStream_t; NULL = the legacy default stream).
+ * library allocates no device memory.  Its only global mutable state is the
+ * process-wide options (bdscan_set_option) and, for
+ * bdscan_block_step_noalloc alone, that entry point's built-in device scratch
+ * buffer; every other entry point works only on the caller's buffers, so
+ * calls with distinct buffers are reentrant.  All device pointers must be
+ * device-accessible memory of the current device.  Every call is asynchronous
+ * on `cuda_stream` (a cudaStream_t; NULL = the legacy default stream).
  *
  * Errors: every entry point validates its arguments synchronously, before any
  * launch, and returns a BDSCAN_* status; nothing aborts the process.  A launch
@@ -304,6 +307,26 @@ void *bdscan_noalloc_scratch(void);
 
 /* Library version (major * 10000 + minor * 100 + patch). */
 int bdscan_version(void);
+
+/* Process-wide options.  Their initial values come from the environment,
+ * read once at the first call that uses them (not per call):
+ *   BDSCAN_OPT_WAIT_TIMEOUT_NS  limit of every bounded device-side wait of
+ *                               the tensor-core kernels, in ns (default 2e9;
+ *                               env BDSCAN_WAIT_TIMEOUT_NS).  A wait that runs
+ *                               out sets BDSCAN_ERR_TIMEOUT in the status word.
+ *   BDSCAN_OPT_FORCE_GENERIC    1: every scan runs on the CUDA-core kernel
+ *                               (default 0; env BDSCAN_FORCE_GENERIC=1)
+ *   BDSCAN_OPT_VERBOSE          1: launch failures are printed to stderr
+ *                               (default 0; env BDSCAN_VERBOSE=1)
+ * bdscan_set_option returns the previous value, or BDSCAN_ERR_INVALID_ARG for
+ * an unknown option or a value out of range; a change applies to calls made
+ * after it returns.  bdscan_get_option returns the current value (or
+ * BDSCAN_ERR_INVALID_ARG). */
+#define BDSCAN_OPT_WAIT_TIMEOUT_NS 0
+#define BDSCAN_OPT_FORCE_GENERIC 1
+#define BDSCAN_OPT_VERBOSE 2
+long long bdscan_set_option(int option, long long value);
+long long bdscan_get_option(int option);
 
 #ifdef __cplusplus
 }

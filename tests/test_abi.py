@@ -253,3 +253,45 @@ def test_gated_rmsnorm_validation():
     assert call(out=y) == -1               # in place needs a bf16 y
     assert call(out=y + 0x40) == -1       # partial overlap with y
     assert call(out=z) == -1 and call(out=w) == -1
+
+
+def test_binding_checks_caller_outputs():
+    """The torch-facing helpers reject caller-provided outputs and workspaces of
+    the wrong shape, dtype or device before anything reaches the C ABI (the C
+    side trusts the sizes its pointers imply)."""
+    import torch
+    from bidirectional_mamba_state_b200 import workload as W
+    s = W.Shape(1, 64, 2, 64, 128, 1, 32, 32, "bf16")
+    f, r = W.make_streams(s, 0, streams=(W.CLEAN_FWD, W.CLEAN_REV))
+    good_y = torch.empty((1, 64, 2, 64))
+    bad = {
+        "y short": dict(y=torch.empty((1, 32, 2, 64))),
+        "y dtype": dict(y=torch.empty((1, 64, 2, 64), dtype=torch.bfloat16)),
+        "states shape": dict(y=good_y, states=torch.empty((1, 1, 2, 64, 128))),
+        "final dtype": dict(y=good_y, final=torch.empty((1, 2, 64, 128), dtype=torch.float64)),
+        "ws dtype": dict(y=good_y, ws=torch.empty(1 << 20, dtype=torch.float32)),
+        "ws small": dict(y=good_y, ws=torch.empty(16, dtype=torch.uint8)),
+        "y strided": dict(y=torch.empty((1, 64, 2, 128))[..., ::2]),
+    }
+    for what, kw in bad.items():
+        with pytest.raises(ValueError):
+            bd.prefix(s, f, r, **kw)
+    st = s.with_(seqlen=32)
+    sf, sr = W.make_streams(st, 0, streams=(W.CLEAN_FWD, W.CLEAN_REV))
+    state = torch.zeros((1, 2, 64, 128))
+    for kw in (dict(state_out=torch.empty((1, 2, 64, 64))), dict(y=torch.empty((1, 64, 2, 64))),
+               dict(ws=torch.empty(8, dtype=torch.uint8))):
+        with pytest.raises(ValueError):
+            bd.block_step(st, sf, sr, state, **kw)
+    cf, cr, nf, nr = W.make_streams(s, 0)
+    for kw in (dict(y_noisy=torch.empty((1, 64, 2, 32))), dict(y_clean=torch.empty((2, 64, 2, 64))),
+               dict(states=torch.empty((1, 2, 2, 64, 128), dtype=torch.bfloat16))):
+        with pytest.raises(ValueError):
+            bd.allblock(s, cf, cr, nf, nr, **kw)
+    yn = torch.empty((1, 64, 2, 64))
+    sts = torch.empty((1, 2, 2, 64, 128))
+    grads = [{"x": torch.empty((1, 64, 2, 64)), "dt": torch.empty((1, 64, 2)), "B": torch.empty((1, 64, 1, 128)),
+              "C": torch.empty((1, 64, 1, 128)), "A": torch.empty(2), "D": torch.empty(2)} for _ in range(4)]
+    grads[2]["B"] = torch.empty((1, 64, 1, 64))
+    with pytest.raises(ValueError):
+        bd.allblock_backward(s, cf, cr, nf, nr, sts, yn, grads=grads)

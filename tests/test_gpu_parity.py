@@ -1,7 +1,6 @@
 """GPU parity: the CUDA path through the C ABI against the fp64 oracle on the
 same seeded inputs, plus the invariants that must hold bit-exactly on the
 device (boundary-state independence, state_in untouched, determinism)."""
-import os
 
 import pytest
 import torch
@@ -175,87 +174,7 @@ def test_workload_87m_allblock_full():
     check_states(st, rst)
 
 
-def test_workload_350m_allblock_sampled_heads():
-    """350M all-block layer (B4 x 8192, 32 heads) on the device at full size;
-    the oracle recomputes 3 heads of 2 batch rows (every block)."""
-    s = W.WORKLOADS["350m_allblock"]
-    cf, cr, nf, nr = W.make_streams(s, W.SEEDS["350m_allblock"], device=DEV)
-    yc, yn, st = bd.allblock(s, cf, cr, nf, nr)
-    hs = [0, 13, 31]
-    bs = [0, 3]
-    sub = s.with_(batch=len(bs), nheads=len(hs))
-    pick = lambda d: {k: (v[bs] if k not in ("A", "D") else v) for k, v in heads(d, hs).items()}
-    ryc, ryn, rst = oracle.allblock(sub.as_dict(), pick(cf), pick(cr), pick(nf), pick(nr))
-    check_y(yc[bs][:, :, hs], ryc, what="y_clean")
-    check_y(yn[bs][:, :, hs], ryn, what="y_noisy")
-    check_states(st[bs][:, :, hs], rst)
-
-
-@pytest.mark.parametrize("L", [8192, 32768])
-def test_workload_700m_prefill_then_steps(L):
-    """700M inference: prefill of L tokens (final state only) on the device over
-    all 48 heads, then two denoising steps and a commit; the oracle follows 4
-    heads through prefill, steps and commit."""
-    s = W.WORKLOADS["700m_prefill_8k"].with_(seqlen=L)
-    f, r = W.make_streams(s, W.SEEDS["700m_prefill_8k"], streams=(W.CLEAN_FWD, W.CLEAN_REV), device=DEV)
-    y, _, fin = bd.prefix(s, f, r, want_states=False)
-    hs = [0, 7, 30, 47]
-    sub = s.with_(nheads=len(hs))
-    ry, _, rfin = oracle.prefix(sub.as_dict(), heads(f, hs), heads(r, hs), want_states=False)
-    check_y(y[:, :, hs], ry)
-    check_states(fin[:, hs], rfin, "prefill final")
-    st = W.WORKLOADS["700m_step"]
-    for step in range(2):
-        af, ar = W.make_streams(st, 100 + step, streams=(W.CLEAN_FWD, W.CLEAN_REV), device=DEV)
-        yb, _ = bd.block_step(st, af, ar, fin)
-        ryb, _ = oracle.block_step(st.with_(nheads=len(hs)).as_dict(), heads(af, hs), heads(ar, hs),
-                                   rfin)
-        check_y(yb[:, :, hs], ryb, what=f"step {step}")
-    yb, so = bd.block_step(st, af, ar, fin, state_out=True)
-    _, rso = oracle.block_step(st.with_(nheads=len(hs)).as_dict(), heads(af, hs), heads(ar, hs), rfin,
-                               want_state_out=True)
-    check_states(so[:, hs], rso, "commit")
-
-
-def test_workload_3b_256k_prefill_and_batch64_step():
-    """3B: 262,144-token prefill on the device (all 80 heads, final state only),
-    oracle on 2 heads; then a batch-64 step (all heads on the device, oracle on
-    4 sequences x 4 heads)."""
-    s = W.WORKLOADS["3b_prefill_256k"]
-    f, r = W.make_streams(s, W.SEEDS["3b_prefill_256k"], streams=(W.CLEAN_FWD, W.CLEAN_REV), device=DEV)
-    y, _, fin = bd.prefix(s, f, r, want_states=False)
-    hs = [0, 79]
-    ry, _, rfin = oracle.prefix(s.with_(nheads=2).as_dict(), heads(f, hs), heads(r, hs),
-                                want_states=False)
-    check_y(y[:, -4096:, hs], ry[:, -4096:], what="last 4096 tokens")
-    check_y(y[:, :, hs], ry)
-    check_states(fin[:, hs], rfin, "final")
-    del y, f, r
-    st = W.WORKLOADS["3b_step_b64"]
-    af, ar = W.make_streams(st, 4, streams=(W.CLEAN_FWD, W.CLEAN_REV), device=DEV)
-    state = W.make_state(st, 4, device=DEV, scale=1.0)
-    yb, so = bd.block_step(st, af, ar, state, state_out=True)
-    bs, hs = [0, 21, 42, 63], [1, 40, 41, 78]
-    pick = lambda d: {k: (v[bs] if k not in ("A", "D") else v) for k, v in heads(d, hs).items()}
-    sub = st.with_(batch=4, nheads=4)
-    ryb, rso = oracle.block_step(sub.as_dict(), pick(af), pick(ar), state[bs][:, hs], want_state_out=True)
-    check_y(yb[bs][:, :, hs], ryb)
-    check_states(so[bs][:, hs], rso, "commit")
-
-
 # ---------------------------------------------------------------- both device paths
-def _with_env(name, value, fn):
-    old = os.environ.get(name)
-    os.environ[name] = value
-    try:
-        return fn()
-    finally:
-        if old is None:
-            del os.environ[name]
-        else:
-            os.environ[name] = old
-
-
 def test_tensor_core_path_matches_generic_path():
     """The tcgen05 kernel and the CUDA-core kernel agree on the same inputs
     (both are also checked against the oracle above)."""
@@ -263,7 +182,8 @@ def test_tensor_core_path_matches_generic_path():
     cf, cr, nf, nr = W.make_streams(s, 10, device=DEV)
     h0 = W.make_state(s, 10, device=DEV)
     tc = bd.allblock(s, cf, cr, nf, nr, h0=h0)
-    gen = _with_env("BDSCAN_FORCE_GENERIC", "1", lambda: bd.allblock(s, cf, cr, nf, nr, h0=h0))
+    with bd.option(bd.BDSCAN_OPT_FORCE_GENERIC, 1):
+        gen = bd.allblock(s, cf, cr, nf, nr, h0=h0)
     # same bounds as against the oracle (the generic path is within 1e-6 of it)
     check_y(tc[0], gen[0].double().cpu().numpy(), what="y_clean tc vs generic")
     check_y(tc[1], gen[1].double().cpu().numpy(), what="y_noisy tc vs generic")
@@ -278,7 +198,8 @@ def test_bounded_wait_timeout_reports_status():
     cf, cr, nf, nr = W.make_streams(s, 11, device=DEV)
     ws = bd.workspace(s, bd.BDSCAN_OP_ALLBLOCK, DEV)
     stream = torch.cuda.current_stream().cuda_stream
-    _with_env("BDSCAN_WAIT_TIMEOUT_NS", "0", lambda: bd.allblock(s, cf, cr, nf, nr, ws=ws))
+    with bd.option(bd.BDSCAN_OPT_WAIT_TIMEOUT_NS, 0):
+        bd.allblock(s, cf, cr, nf, nr, ws=ws)
     assert bd.bdscan_check_status(ws.data_ptr(), stream) == -6
     yc, yn, st = bd.allblock(s, cf, cr, nf, nr, ws=ws)
     assert bd.bdscan_check_status(ws.data_ptr(), stream) == 0
