@@ -386,7 +386,12 @@ EXTRA = {
     "block_step_700m_b1_24layers": lambda dev, pk: _step_stack(W.WORKLOADS["700m_step"], 24, dev, pk),
     "block_step_3b_b1_40layers": lambda dev, pk: _step_stack(W.WORKLOADS["3b_step_b1"], 40, dev, pk),
     "block_step_3b_b64_40layers": lambda dev, pk: _step_stack(W.WORKLOADS["3b_step_b64"], 40, dev, pk),
-    "prefill_700m_8k_per_layer": lambda dev, pk: _prefill(W.WORKLOADS["700m_prefill_8k"], dev, pk),
+    "tiny_allblock": lambda dev, pk: _allblock_line("tiny", dev, pk, reps=50),
+    "allblock_350m": lambda dev, pk: _allblock_line("350m_allblock", dev, pk),
+    "prefill_700m_8k": lambda dev, pk: _prefill_line("700m_prefill_8k", 24, dev, pk),
+    "prefill_700m_32k": lambda dev, pk: _prefill_line("700m_prefill_32k", 24, dev, pk),
+    "prefill_700m_64k": lambda dev, pk: _prefill_line("700m_prefill_64k", 24, dev, pk),
+    "prefill_3b_256k_40layers": lambda dev, pk: _prefill_3b(dev, pk),
     "allblock_backward_87m": lambda dev, pk: _backward(W.WORKLOADS["87m_allblock"], dev, pk),
     "conv_allblock_87m": lambda dev, pk: _conv_allblock(W.WORKLOADS["87m_allblock"], 4, dev, pk),
     "conv_block_step_700m_b1_24layers": lambda dev, pk: _step_stack(W.WORKLOADS["700m_step"], 24, dev, pk,
@@ -484,6 +489,13 @@ def _step_stack(s: W.Shape, layers: int, dev, pk, conv_width: int = 0, norm: boo
     out = {"us_per_step": ms * 1e3, "tokens_per_s": s.batch * s.seqlen / (ms * 1e-3),
            "algorithmic_bytes": b, "hbm_frac": b / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
            "layers": layers, "batch": s.batch, "graph": True}
+    if not conv_width and not norm:
+        import oracle
+        hf, hr, hst = _host(ins[0][0]), _host(ins[0][1]), states[0].to("cpu")
+        out["cpu_baseline"] = _oracle_rate(
+            lambda: oracle.block_step(s.as_dict(), hf, hr, hst), s.batch * s.seqlen * s.nheads,
+            "token-heads/s", f"oracle block_step of layer 0 (all {s.batch} x {s.nheads} sequences, "
+            f"forward from the cached state + block-local reverse)", target_s=1.0)
     if conv_width:
         out["conv_width"] = conv_width
     if norm:
@@ -547,36 +559,151 @@ def _backward(s: W.Shape, dev, pk) -> dict:
                          "hbm_frac": bytes_ / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}}
 
 
-def _prefill(s: W.Shape, dev, pk) -> dict:
-    f, r = W.make_streams(s, W.SEEDS["700m_prefill_8k"], device=dev, streams=(W.CLEAN_FWD, W.CLEAN_REV))
+def _oracle_rate(call, units: float, unit: str, sample: str, target_s: float = 3.0) -> dict:
+    """The fp64 oracle, as it stands, timed on the host's cores: ``call`` is run
+    until about ``target_s`` seconds have passed; ``units`` of work per run."""
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    oracle.set_threads(cores)
+    reps = 0
+    t0 = time.perf_counter()
+    while True:
+        call()
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= target_s or dt / reps * (reps + 1) > 2 * target_s:
+            break
+    return {"value": units * reps / dt, "unit": unit, "cores": cores, "kind": "oracle",
+            "sample": f"{sample}; {reps} run(s) in {dt:.1f} s"}
+
+
+def _host(d: dict) -> dict:
+    return {k: v.to("cpu") for k, v in d.items()}
+
+
+def _heads_host(d: dict, hs: list) -> dict:
+    """Host copy of one direction's inputs restricted to the heads ``hs`` (one
+    B/C group: B and C are shared by all heads)."""
+    return {k: (v[hs] if k in ("A", "D") else v if k in ("B", "C") else v[:, :, hs]).to("cpu")
+            for k, v in d.items()}
+
+
+def _allblock_line(name: str, dev, pk, reps: int = 10) -> dict:
+    """One bdscan_allblock call on a whole workload (CUDA events), with the
+    oracle's rate on one batch row (all heads, full length)."""
+    import oracle
+    s = W.WORKLOADS[name]
+    cf, cr, nf, nr = W.make_streams(s, W.SEEDS[name], device=dev)
+    yc, yn, st = bd.allblock(s, cf, cr, nf, nr)
+    ws = bd.workspace(s, bd.BDSCAN_OP_ALLBLOCK, dev)
+    ms = _time(lambda: bd.allblock(s, cf, cr, nf, nr, y_clean=yc, y_noisy=yn, states=st, ws=ws), dev, reps)
+    b = RL.allblock_bytes(s)
+    del yc, yn, st
+    one = s.with_(batch=1)
+    hs = [_host({k: (v if k in ("A", "D") else v[:1]) for k, v in d.items()}) for d in (cf, cr, nf, nr)]
+    cpu = _oracle_rate(lambda: oracle.allblock(one.as_dict(), *hs), one.seqlen, "tokens/s",
+                       f"oracle allblock on 1 of {s.batch} batch rows, all {s.nheads} heads, "
+                       f"all {s.seqlen} tokens")
+    return {"us_per_call": ms * 1e3, "tokens_per_s": s.batch * s.seqlen / (ms * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": b / (ms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": b / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                         "algorithmic_bytes": b},
+            "cpu_baseline": cpu}
+
+
+def _prefill_line(name: str, layers: int, dev, pk, oracle_heads=None) -> dict:
+    """Prefill (bdscan_prefix, final state only, block-local reverse) of one
+    layer and of a stack of ``layers`` layers with independent weights, each
+    layer's inputs resident (the stack's calls back to back, CUDA events);
+    with the oracle's rate per token-head on one layer."""
+    import oracle
+    s = W.WORKLOADS[name]
+    seed = W.SEEDS[name]
+    ins = [W.make_streams(s, seed, l, device=dev, streams=(W.CLEAN_FWD, W.CLEAN_REV)) for l in range(layers)]
+    y = torch.empty((s.batch, s.seqlen, s.nheads, s.headdim), device=dev)
+    fins = [torch.empty((s.batch, s.nheads, s.headdim, s.dstate), device=dev) for _ in range(layers)]
+    ws = bd.workspace(s, bd.BDSCAN_OP_PREFIX, dev)
+    one = lambda l: bd.prefix(s, ins[l][0], ins[l][1], want_states=False, y=y, final=fins[l], ws=ws)
+    ms1 = _time(lambda: one(0), dev, 20, 5)
+
+    def stack():
+        for l in range(layers):
+            one(l)
+    ms = _time(stack, dev, 3, 1)
+    b = RL.prefix_bytes(s, block_states=False)
+    out = {"us_per_layer": ms1 * 1e3, "tokens_per_s_per_layer": s.batch * s.seqlen / (ms1 * 1e-3),
+           "algorithmic_bytes_per_layer": b, "hbm_frac": b / (ms1 * 1e-3) / 1e9 / pk["hbm_gbs"],
+           f"ms_{layers}_layers": ms, f"hbm_frac_{layers}_layers": b * layers / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+           "layers": layers}
+    hs = list(range(s.nheads)) if oracle_heads is None else list(range(oracle_heads))
+    f, r = _heads_host(ins[0][0], hs), _heads_host(ins[0][1], hs)
+    del ins
+    sub = s.with_(nheads=len(hs))
+    out["cpu_baseline"] = _oracle_rate(
+        lambda: oracle.prefix(sub.as_dict(), f, r, want_states=False), s.batch * s.seqlen * len(hs),
+        "token-heads/s", f"oracle prefix of layer 0, {len(hs)} of {s.nheads} heads, all {s.seqlen} tokens, "
+        f"forward + block-local reverse")
+    return out
+
+
+def _prefill_3b(dev, pk, layers: int = 40) -> dict:
+    """The 3B layer's 262,144-token prefill (final state only): ``layers`` layers
+    with independent weights, each layer's inputs drawn just before its call
+    (untimed; 40 layers' inputs would not fit the device at once), every call
+    timed with CUDA events; per layer (median) and the 40-layer sum."""
+    import oracle
+    s = W.WORKLOADS["3b_prefill_256k"]
+    seed = W.SEEDS["3b_prefill_256k"]
     y = torch.empty((s.batch, s.seqlen, s.nheads, s.headdim), device=dev)
     fin = torch.empty((s.batch, s.nheads, s.headdim, s.dstate), device=dev)
     ws = bd.workspace(s, bd.BDSCAN_OP_PREFIX, dev)
-    ms = _time(lambda: bd.prefix(s, f, r, want_states=False, y=y, final=fin, ws=ws), dev, 20, 5)
+    times = []
+    for l in range(layers):
+        f, r = W.make_streams(s, seed, l, device=dev, streams=(W.CLEAN_FWD, W.CLEAN_REV))
+        if l == 0:
+            bd.prefix(s, f, r, want_states=False, y=y, final=fin, ws=ws)
+        times.append(_time(lambda: bd.prefix(s, f, r, want_states=False, y=y, final=fin, ws=ws), dev, 1, 0))
+        if l == 0:
+            hf, hr = _heads_host(f, list(range(16))), _heads_host(r, list(range(16)))
+        del f, r
+    ms = statistics.median(times)
     b = RL.prefix_bytes(s, block_states=False)
-    return {"us_per_layer": ms * 1e3, "tokens_per_s": s.batch * s.seqlen / (ms * 1e-3),
-            "algorithmic_bytes": b, "hbm_frac": b / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+    sub = s.with_(nheads=16)
+    cpu = _oracle_rate(lambda: oracle.prefix(sub.as_dict(), hf, hr, want_states=False),
+                       s.seqlen * 16, "token-heads/s",
+                       "oracle prefix of layer 0, 16 of 80 heads, all 262144 tokens, forward + block-local "
+                       "reverse", target_s=1.0)
+    return {"us_per_layer_median": ms * 1e3, "ms_40_layers_sum": sum(times),
+            "tokens_per_s_per_layer": s.seqlen / (ms * 1e-3), "algorithmic_bytes_per_layer": b,
+            "hbm_frac": b / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], "layers": layers,
+            "timing": "each layer's call timed alone (CUDA events), inputs drawn before it",
+            "cpu_baseline": cpu}
 
 
 def _step_flatness(dev, pk) -> dict:
-    """Per-step cost against context length: prefill one 700M layer at 8K, 32K
-    and 64K tokens (final state only), then time a denoising step (block_step
-    over the active 32-token block) from each cached state.  The step reads only
-    the fixed-size state, so its time must not grow with the context."""
+    """Per-step cost against context length: prefill one layer (final state
+    only) at several lengths, then time a denoising step (block_step over the
+    active 32-token block) from each cached state.  The step reads only the
+    fixed-size state, so its time must not grow with the context: 700M at
+    8K/32K/64K, 3B at 8K/64K/256K."""
     out = {}
-    st = W.WORKLOADS["700m_step"]
-    a, r = W.make_streams(st, 7, device=dev, streams=(W.CLEAN_FWD, W.CLEAN_REV))
-    ws = bd.workspace(st, bd.BDSCAN_OP_BLOCK_STEP, dev)
-    y = torch.empty((st.batch, st.seqlen, st.nheads, st.headdim), device=dev)
-    for name in ("700m_prefill_8k", "700m_prefill_32k", "700m_prefill_64k"):
-        s = W.WORKLOADS[name]
-        f, rr = W.make_streams(s, W.SEEDS[name], device=dev, streams=(W.CLEAN_FWD, W.CLEAN_REV))
-        _, _, fin = bd.prefix(s, f, rr, want_states=False)
-        del f, rr
-        ms = _time(lambda: bd.block_step(st, a, r, fin, y=y, ws=ws), dev, 50, 5)
-        out[f"us_per_step_after_{s.seqlen // 1024}k"] = ms * 1e3
-    v = list(out.values())
-    out["max_over_min"] = max(v) / min(v)
+    for model, step_name, lens in (("700m", "700m_step", (8192, 32768, 65536)),
+                                   ("3b", "3b_step_b1", (8192, 65536, 262144))):
+        st = W.WORKLOADS[step_name]
+        a, r = W.make_streams(st, 7, device=dev, streams=(W.CLEAN_FWD, W.CLEAN_REV))
+        ws = bd.workspace(st, bd.BDSCAN_OP_BLOCK_STEP, dev)
+        y = torch.empty((st.batch, st.seqlen, st.nheads, st.headdim), device=dev)
+        row = {}
+        for L in lens:
+            s = st.with_(seqlen=L, chunk_len=128)
+            f, rr = W.make_streams(s, W.SEEDS[step_name], device=dev, streams=(W.CLEAN_FWD, W.CLEAN_REV))
+            _, _, fin = bd.prefix(s, f, rr, want_states=False)
+            del f, rr
+            ms = _time(lambda: bd.block_step(st, a, r, fin, y=y, ws=ws), dev, 50, 5)
+            row[f"us_per_step_after_{L // 1024}k"] = ms * 1e3
+        v = list(row.values())
+        row["max_over_min"] = max(v) / min(v)
+        out[model] = row
     out["layers"] = 1
     return out
 
