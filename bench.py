@@ -46,10 +46,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one bd_tc_kernel
 # launch on this workload, from one ncu capture, and the hash of the kernel
 # source it was taken on: reported while the source is unchanged, null after.
-TC_TRAFFIC = {"bytes": 224_074_240 + 548_320_768,
+TC_TRAFFIC = {"bytes": 224_265_728 + 548_283_648,
               "sources": ("bidirectional_mamba_state_b200/csrc/scan_tc.cu",
                           "bidirectional_mamba_state_b200/csrc/sm100.cuh"),
-              "sha256": "f9701e4af1b27b705f682b3397bf8da8a78bb0b7d6a0de103cedaf3ef1334b49"}
+              "sha256": "e067612d76127c853da6dd5a06f3a31e78b88b73e875072b269c4f8249da597f"}
 
 
 def tc_traffic():
@@ -382,6 +382,32 @@ def _time(fn, dev, reps, warm=3):
     return e0.elapsed_time(e1) / reps
 
 
+def _profile_case(name: str, dev, pk) -> dict:
+    """One small case of a kernel for ncu (inputs of one layer, a few hundred MB
+    on the device): three warm-up calls, then one call.  step_3b_b64: one 3B
+    layer's denoising step at batch 64; prefill_700m_8k: one 700M layer's 8K
+    prefill (final state only)."""
+    if name == "step_3b_b64":
+        s = W.WORKLOADS["3b_step_b64"]
+        f, r = W.make_streams(s, W.SEEDS["3b_step_b64"], device=dev, streams=(W.CLEAN_FWD, W.CLEAN_REV))
+        state = W.make_state(s, W.SEEDS["3b_step_b64"], device=dev)
+        y = torch.empty((s.batch, s.seqlen, s.nheads, s.headdim), device=dev)
+        ws = bd.workspace(s, bd.BDSCAN_OP_BLOCK_STEP, dev)
+        call = lambda: bd.block_step(s, f, r, state, y=y, ws=ws)
+        b = RL.block_step_bytes(s)
+    else:
+        s = W.WORKLOADS["700m_prefill_8k"]
+        f, r = W.make_streams(s, W.SEEDS["700m_prefill_8k"], device=dev, streams=(W.CLEAN_FWD, W.CLEAN_REV))
+        y = torch.empty((s.batch, s.seqlen, s.nheads, s.headdim), device=dev)
+        fin = torch.empty((s.batch, s.nheads, s.headdim, s.dstate), device=dev)
+        ws = bd.workspace(s, bd.BDSCAN_OP_PREFIX, dev)
+        call = lambda: bd.prefix(s, f, r, want_states=False, y=y, final=fin, ws=ws)
+        b = RL.prefix_bytes(s, block_states=False)
+    ms = _time(call, dev, 1, 3)
+    return {"us": ms * 1e3, "algorithmic_bytes": b, "launches_per_call": bd.kernel_launches(
+        s, bd.BDSCAN_OP_BLOCK_STEP if name == "step_3b_b64" else bd.BDSCAN_OP_PREFIX)}
+
+
 EXTRA = {
     "block_step_700m_b1_24layers": lambda dev, pk: _step_stack(W.WORKLOADS["700m_step"], 24, dev, pk),
     "block_step_3b_b1_40layers": lambda dev, pk: _step_stack(W.WORKLOADS["3b_step_b1"], 40, dev, pk),
@@ -392,6 +418,8 @@ EXTRA = {
     "prefill_700m_32k": lambda dev, pk: _prefill_line("700m_prefill_32k", 24, dev, pk),
     "prefill_700m_64k": lambda dev, pk: _prefill_line("700m_prefill_64k", 24, dev, pk),
     "prefill_3b_256k_40layers": lambda dev, pk: _prefill_3b(dev, pk),
+    "profile_step_3b_b64": lambda dev, pk: _profile_case("step_3b_b64", dev, pk),
+    "profile_prefill_700m_8k": lambda dev, pk: _profile_case("prefill_700m_8k", dev, pk),
     "allblock_backward_87m": lambda dev, pk: _backward(W.WORKLOADS["87m_allblock"], dev, pk),
     "conv_allblock_87m": lambda dev, pk: _conv_allblock(W.WORKLOADS["87m_allblock"], 4, dev, pk),
     "conv_block_step_700m_b1_24layers": lambda dev, pk: _step_stack(W.WORKLOADS["700m_step"], 24, dev, pk,
@@ -411,7 +439,7 @@ def run_extra(dev, pk, only=None) -> dict:
     out = {}
     try:
         for name, fn in EXTRA.items():
-            if only is None or name == only:
+            if (only is None and not name.startswith("profile_")) or name == only:
                 out[name] = fn(dev, pk)
     except Exception as e:  # report, never hide
         out["error"] = repr(e)

@@ -11,6 +11,7 @@ library is an error.
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 import re
 import threading
@@ -254,6 +255,11 @@ def _stream(device, stream=None) -> int:
     return s.cuda_stream
 
 
+@functools.lru_cache(maxsize=256)
+def _ws_bytes(s: Shape, op: int) -> int:
+    return bdscan_workspace_size(ctypes.byref(c_shape(s)), op)
+
+
 def _check_ws(ws, s: Shape, op: int, device):
     """A caller-provided workspace: a contiguous uint8 tensor on ``device``
     with at least bdscan_workspace_size(shape, op) bytes."""
@@ -261,7 +267,7 @@ def _check_ws(ws, s: Shape, op: int, device):
         raise ValueError(f"ws is on {ws.device}, expected {device}")
     if ws.dtype != torch.uint8 or ws.dim() != 1 or not ws.is_contiguous():
         raise ValueError("ws must be a contiguous 1-D uint8 tensor")
-    need = bdscan_workspace_size(ctypes.byref(c_shape(s)), op)
+    need = _ws_bytes(s, op)
     if ws.numel() < need:
         raise ValueError(f"ws holds {ws.numel()} bytes, the call needs {need}")
 

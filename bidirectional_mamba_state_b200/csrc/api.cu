@@ -209,7 +209,8 @@ size_t bdscan_workspace_size(const bdscan_shape_t *shape, int op) {
   // in the workspace; shapes it cannot take need only the status word.
   if (bdscan::tc_shape_ok(shape->headdim, shape->dstate, shape->block_len, shape->in_dtype == BDSCAN_BF16))
     return bdscan::kWsHeader +
-           bdscan::tc_workspace_bytes(shape->batch, shape->seqlen, shape->ngroups, shape->nheads);
+           bdscan::tc_workspace_bytes(shape->batch, shape->seqlen, shape->ngroups, shape->nheads,
+                                      op == BDSCAN_OP_ALLBLOCK);
   return kStatusBytes;
 }
 

@@ -46,7 +46,7 @@ constexpr size_t kWsHeader = 1024;
 
 // Tensor-core path (sm_100a): bf16 inputs, P = 64, N = 128, T = 32, no gate.
 bool tc_shape_ok(int64_t P, int64_t N, int64_t T, bool in_bf16);
-size_t tc_workspace_bytes(int64_t Bsz, int64_t L, int64_t G, int64_t H);
+size_t tc_workspace_bytes(int64_t Bsz, int64_t L, int64_t G, int64_t H, bool allblock);
 int tc_plan_segments(int64_t Bsz, int64_t H, int64_t K);
 bool tc_supported(const ScanArgs &a);
 cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream);

@@ -1,5 +1,5 @@
 // scan_tc.cu -- tensor-core block-diffusion scan for sm_100a
-// (bf16 inputs, headdim P = 64, d_state N = 128, block T = 32, no gate).
+// (bf16 inputs, headdim P = 64, d_state N = 128, block T = 32; gated or not).
 //
 // Chunked (state-space-duality) form, one 32-token block at a time, of the
 // recurrence of "Training Hybrid Block Diffusion Language Models with Partial
@@ -46,8 +46,12 @@
 //                 M with each direction's D added to the diagonal (so D x is
 //                 part of Y_diag), stored bf16, next to a diagonal matrix of
 //                 that diagonal's bf16 remainders: one N = 64 MMA per 16
-//                 tokens gives both, summed by the epilogue.
-//   S, Y and M are double-buffered; the h operand is single-buffered.
+//                 tokens gives both, summed by the epilogue.  With a gate
+//                 (y_dir * silu(z_dir) before the sum) each direction keeps its
+//                 own Y_diag accumulator and the epilogue loads z; that
+//                 epilogue lives only in the gated instance of the kernel.
+//   S, Y and M are double-buffered (Y single-buffered with a gate: its five
+//   accumulators fill the TMEM); the h operand is single-buffered.
 // Every wait is bounded; on a timeout the CTA raises BDSCAN_ERR_TIMEOUT in the
 // workspace status word, drains its own copies and MMAs, frees TMEM and exits.
 //
@@ -92,7 +96,7 @@ constexpr uint32_t kCbSmem = kCbOffBar + 64 + 1024;
 struct CbParams {
   CUtensorMap tb[4];
   CUtensorMap tc[4];
-  int slot[4];  // blockIdx.z -> stacking slot
+  int slot[4];  // blockIdx.z -> the direction's C B^T tile set (see cb_set)
   int Bsz, K, G;
   __nv_bfloat16 *cb;  // [4][B][K][G][32 s][32 t]
   int *item_counters;  // the scan passes' work-item counters, zeroed here
@@ -171,7 +175,8 @@ __global__ void __launch_bounds__(kCbThreads) bd_cb_kernel(const __grid_constant
     umma_commit(&bars[1]);
   }
   bool ok = mbar_wait(&bars[1], 0, p.timeout_ns, abort_flag);
-  ok = __all_sync(0xffffffffu, ok) && !*abort_flag;
+  // one outcome for the whole warp: the TMEM load below is a warp-wide instruction
+  ok = __all_sync(0xffffffffu, ok && !*abort_flag);
   if (ok) {
     tc_fence_after();
     uint32_t r[32];
@@ -238,15 +243,19 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 constexpr uint32_t kMhSbo = 128, kMhLbo = 1024;
 
 enum : int {
-  bFull0 = 0, bFull1, bFull2, bEmpty0, bEmpty1, bEmpty2, bAux0, bAux7 = bAux0 + kTab - 1, bXwFull, bSFull0, bSFull1,
+  bFull0 = 0, bFull1, bFull2, bEmpty0, bEmpty1, bEmpty2, bAux0, bAux7 = bAux0 + kTab - 1, bXwFull0, bXwFull1, bSFull0,
+  bSFull1,
   bSEmpty0, bSEmpty1, bMhFull0, bMhFull1, bHFull, bHCons, bYFull0, bYFull1, bYEmpty0, bYEmpty1, bDrain,
   bItem0, bCount = bItem0 + kItemRing
 };
 static_assert(bCount <= kNumBars, "barrier array");
 
 // TMEM columns: S^T[2] (M=128 x 64), Y^T[2] = {Y_off^T (M=64 x 64), clean
-// [Y_diag^T | remainder] (M=64 x 64), noisy [Y_diag^T | remainder] (M=64 x 64)}
-constexpr uint32_t kColS0 = 0, kColY0 = 128, kColYBuf = 192;
+// [Y_diag^T | remainder] (M=64 x 64), noisy [Y_diag^T | remainder] (M=64 x 64)}.
+// With a gate the two directions of a stream are gated separately, so each
+// direction keeps its own [Y_diag^T | remainder]: one Y buffer of
+// {Y_off^T, clean fwd, noisy fwd, clean rev, noisy rev} (320 columns).
+constexpr uint32_t kColS0 = 0, kColY0 = 128, kColYBuf = 192, kColRevGated = 128;
 constexpr uint32_t kTmemCols = 512;
 
 struct TcParams {
@@ -258,7 +267,9 @@ struct TcParams {
   const __nv_bfloat16 *dt[4];
   const float *A[4];
   const float *D[4];
+  const __nv_bfloat16 *z[4];  // gate of each direction, or null
   int active[4];
+  int gated;                   // some direction has a gate: single Y buffer, per-direction Y_diag
   int Bsz, L, H, G, K;
   int nseg, seg_blocks;  // each (b, h) sequence is walked as nseg segments of seg_blocks blocks
   int items;             // Bsz * H * nseg work items, handed out one at a time
@@ -286,7 +297,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 __device__ __forceinline__ float bf16_lo_f(uint32_t v) { return __uint_as_float(v << 16); }
+// v * sigmoid(v) with the hardware exponential and divide
+__device__ __forceinline__ float silu_approx(float v) { return __fdividef(v, 1.0f + ex2_approx(-v * 1.4426950408889634f)); }
 __device__ __forceinline__ float bf16_hi_f(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// C B^T tile set of direction slot i in the workspace: the all-block pass keeps
+// four (one per direction), prefix and block step two (the clean forward and
+// reverse directions, slots 0 and 2).
+__host__ __device__ __forceinline__ int cb_set(int allblock, int i) { return allblock ? i : (i >> 1); }
+__host__ __device__ __forceinline__ int cb_sets(bool allblock) { return allblock ? 4 : 2; }
 
 // Element i of a 4-entry kernel-parameter array without dynamic indexing (which
 // would copy the array to local memory).
@@ -302,6 +321,11 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
 }
 __device__ __forceinline__ void sts_f32(uint32_t addr, float v) {
   asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ unsigned short lds_u16(uint32_t addr) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr) : "memory");
+  return v;
 }
 __device__ __forceinline__ void sts_u16(uint32_t addr, unsigned short v) {
   asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
@@ -392,6 +416,12 @@ __device__ __forceinline__ void arrive_lane0(const Ctl &c, int bar) {
 
 // parity of the completion of a double-buffered barrier that block k uses
 __device__ __forceinline__ uint32_t par2(int k) { return (static_cast<uint32_t>(k) >> 1) & 1u; }
+// Y accumulators of step j: buffer, parity of its "full" phase, and the step
+// whose read must precede this step's writes (double-buffered, or single-
+// buffered with a gate)
+__device__ __forceinline__ int ybuf(int gated, int j) { return gated ? 0 : (j & 1); }
+__device__ __forceinline__ uint32_t ypar(int gated, int j) { return gated ? (static_cast<uint32_t>(j) & 1u) : par2(j); }
+__device__ __forceinline__ int yprev(int gated, int j) { return gated ? j - 1 : j - 2; }
 // TMA ring: slot and parity of block k
 __device__ __forceinline__ int rslot(int k) { return k % kSlots; }
 __device__ __forceinline__ uint32_t parr(int k) { return static_cast<uint32_t>(k / kSlots) & 1u; }
@@ -494,7 +524,10 @@ __device__ __forceinline__ int item_warp(const TcParams &p, const Ctl &c, uint32
 // ---------------------------------------------------------------- producer
 __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
   const int nact = p.active[0] + p.active[1] + p.active[2] + p.active[3];
-  const uint32_t bytes = p.agg ? 3 * kTile : nact * (kTile + 2048) + (2 + (p.allblock ? 4 : 2)) * kTile;
+  // x of each active direction, C B^T tiles, B of the clean forward direction
+  // (only when S is formed), C of the clean (and noisy) forward direction
+  const uint32_t bytes = p.agg ? 3 * kTile
+                               : nact * (kTile + 2048) + (2 + (p.allblock ? 4 : 2)) * kTile;
 #pragma unroll
   for (int i = 0; i < 4; ++i)
     if (p.active[i]) tma_prefetch_desc(&p.tx[i]);
@@ -549,7 +582,7 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           if (!p.active[i]) continue;
-          const int idx = ((i * p.Bsz + I.b) * p.K + k) * p.G + I.g;
+          const int idx = ((cb_set(p.allblock, i) * p.Bsz + I.b) * p.K + k) * p.G + I.g;
           tma_load_3d_s(st + kOffCB + i * 2048, &p.tcb, full, 0, 0, idx);
         }
       }
@@ -574,6 +607,7 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
 // Issue order per step: S; Y_off (then commit "h consumed" so the state group
 // may overwrite the h operand at once); Y_diag and the D x products.
 // Descriptors are built once; per step only their start addresses move.
+template <bool kGated>
 __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
   const uint32_t id_s = idesc_bf16(128, 64, 1, 1);  // S^T[n][p] = B^T (w o X)
   // Y_off^T[p][t] = h C^T over the stacked [C_cf; C_nf] rows (only C_cf without a noisy stream)
@@ -600,14 +634,15 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
       if (!wait1(c, bFull0 + r, parr(j))) break;
       // ---- S^T = B_cf^T (w o X): A MN-major (n; halves 4 KB apart), B MN-major (p)
       if (p.need_s) {
-        if (!wait1(c, bXwFull, j & 1)) break;
+        if (!wait1(c, bXwFull0 + i2, par2(j))) break;
         if (j >= 2 && !wait1(c, bSEmpty0 + i2, par2(j - 2))) break;
         tc_fence_after();
         const uint32_t colS = tmem + kColS0 + 64 * i2;
+        const D64 dxw = dXw;
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks) {
-          umma_bf16(colS, dBcf + so + BD_OFF(ks * 2048), dXw + BD_OFF(ks * 2048), id_s, ks > 0);
-          umma_bf16(colS, dBcf + so + BD_OFF(ks * 2048), dXw + BD_OFF(kTile + ks * 2048), id_s, 1);
+          umma_bf16(colS, dBcf + so + BD_OFF(ks * 2048), dxw + BD_OFF(ks * 2048), id_s, ks > 0);
+          umma_bf16(colS, dBcf + so + BD_OFF(ks * 2048), dxw + BD_OFF(kTile + ks * 2048), id_s, 1);
         }
         umma_commit_s(bar_at(c, bSFull0 + i2));
       }
@@ -618,9 +653,10 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
       }
       // ---- Y_off^T = h [C_cf; C_nf]^T, h = the state before this block
       if (!wait1(c, bHFull, j & 1)) break;
-      if (j >= 2 && !wait1(c, bYEmpty0 + i2, par2(j - 2))) break;
+      const int yb = ybuf(kGated, j), jp = yprev(kGated, j);
+      if (jp >= 0 && !wait1(c, bYEmpty0 + yb, ypar(kGated, jp))) break;
       tc_fence_after();
-      const uint32_t colY = tmem + kColY0 + kColYBuf * i2;
+      const uint32_t colY = tmem + kColY0 + kColYBuf * yb;
 #pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
         const D64 bc = dC + so + BD_OFF((ks < 4 ? 0 : 2 * kTile) + (ks & 3) * 32);
@@ -637,13 +673,15 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
 #pragma unroll
       for (int i = 0; i < 4; ++i) {  // the forward direction of a stream (i < 2) is always active
         if (!p.active[i]) continue;
-        const uint32_t col = colY + 64 + ((i & 1) ? 64 : 0);
+        // ungated: a stream's directions share one accumulator; gated: each its own
+        const bool own = kGated && i >= 2;
+        const uint32_t col = colY + 64 + ((i & 1) ? 64 : 0) + (own ? kColRevGated : 0);
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks)
           umma_bf16(col, dX + so + BD_OFF(i * kTile + ks * 2048), dM + mo + BD_OFF(i * kMhDir + ks * 2048), id_yd,
-                    (i >= 2 || ks > 0) ? 1u : 0u);
+                    ((i >= 2 && !own) || ks > 0) ? 1u : 0u);
       }
-      umma_commit_s(bar_at(c, bYFull0 + i2));
+      umma_commit_s(bar_at(c, bYFull0 + yb));
       umma_commit_s(bar_at(c, bEmpty0 + r));
       ok = true;
     }
@@ -651,6 +689,57 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
 #undef BD_OFF
   umma_commit_s(bar_at(c, bDrain));
   (void)mbar_wait_s(bar_at(c, bDrain), 0, p.drain_ns, 0);
+}
+
+// The intra-block operand of direction slot q for step jm (see kMhSbo): the
+// masked-decay matrix M^T[s][t] of the block with the direction's D added to
+// its diagonal, stored bf16, and that diagonal's bf16 remainders; one warp,
+// row s = lane.  Reads the step's C B^T tile (ring slot) and decay tables.
+__device__ __forceinline__ void build_masked_decay(uint32_t base, int q, int lane, int jm, bool act, bool rev) {
+  const int ct = jm % kTab;
+  if (act) {
+    const uint32_t cbrow = base + rslot(jm) * kSlot + kOffCB + q * 2048;
+    const uint32_t cq = base + kOffCum + (ct * 4 + q) * 128;
+    const float cs = lds_f32(cq + lane * 4);
+    const float ds = lds_f32(base + kOffDt + (ct * 4 + q) * 128 + lane * 4);
+    const uint32_t mrow = base + kOffMh + (jm & 1) * kMhBuf + q * kMhDir;
+    // this direction's D joins the diagonal of M (D x is part of X^T M^T):
+    // M[s][s] + D is stored as bf16 hi in M and its bf16 remainder lo on the
+    // diagonal of the block's 16 x 16 correction tile of chunk s / 16
+    const float Dq = lds_f32(base + kOffDtab + (ct * 4 + q) * 4);
+    // off the diagonal in the loop (no divergent branch), the diagonal below
+#pragma unroll 1
+    for (int jj = 0; jj < 4; ++jj) {
+      uint32_t r[4];
+      ld_shared_v4(cbrow + sw64_chunk(lane, jj), r[0], r[1], r[2], r[3]);  // C B^T[s = lane][8 jj ..]
+      float cj[8];
+      ld_shared_v4f(cq + 32 * jj, *reinterpret_cast<float(*)[4]>(&cj[0]));
+      ld_shared_v4f(cq + 32 * jj + 16, *reinterpret_cast<float(*)[4]>(&cj[4]));
+      float mv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int t = 8 * jj + i;
+        const bool valid = rev ? (t <= lane) : (t >= lane);
+        const float e = ex2_approx(cj[i] - cs);
+        const float cb = (i & 1) ? bf16_hi_f(r[i >> 1]) : bf16_lo_f(r[i >> 1]);
+        mv[i] = valid ? cb * ds * e : 0.f;
+      }
+      st_shared_v4(mrow + inter_mn_off(8 * jj, lane, kMhSbo, kMhLbo), pack_bf16x2(mv[0], mv[1]),
+                   pack_bf16x2(mv[2], mv[3]), pack_bf16x2(mv[4], mv[5]), pack_bf16x2(mv[6], mv[7]));
+    }
+    {
+      // M[s][s] + D (the decay factor is exactly 1 there) as bf16, its remainder
+      // on the diagonal of the correction half
+      const float cb = __uint_as_float(static_cast<uint32_t>(lds_u16(cbrow + sw64_chunk(lane, lane >> 3) +
+                                                                     2u * static_cast<uint32_t>(lane & 7)))
+                                       << 16);
+      const float v = cb * ds + Dq;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+      sts_u16(mrow + inter_mn_off(lane, lane, kMhSbo, kMhLbo), __bfloat16_as_ushort(hi));
+      sts_u16(mrow + inter_mn_off(32 + lane, lane, kMhSbo, kMhLbo),
+              __bfloat16_as_ushort(__float2bfloat16_rn(v - __bfloat162float(hi))));
+    }
+  }
 }
 
 // ---------------------------------------------------------------- operand group
@@ -747,7 +836,10 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
       if (!waitw(c, bFull0 + rslot(j), parr(j))) return;
       // ---- (w o X) of the clean forward direction, bf16 hi + lo
       if (p.need_s) {
-        if (j >= 1 && !waitw(c, bSFull0 + ((j + 1) & 1), par2(j - 1))) return;  // S(j-1) read Xw
+        // the S MMA of the previous step has read the w o X buffer
+        const int jr = j - 1;
+        if (jr >= 0 && !waitw(c, bSFull0 + (jr & 1), par2(jr))) return;
+        const uint32_t xw = base + kOffXw;
         const uint32_t cf = cum + (ct * 4 + kCF) * 128, df = dts + (ct * 4 + kCF) * 128;
         const float c31 = lds_f32(cf + 31 * 4);
 #pragma unroll
@@ -760,10 +852,10 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
           const float w = lds_f32(df + t * 4) * ex2_approx(c31 - lds_f32(cf + t * 4));
           float vv[8] = {bf16_lo_f(r0) * w, bf16_hi_f(r0) * w, bf16_lo_f(r1) * w, bf16_hi_f(r1) * w,
                          bf16_lo_f(r2) * w, bf16_hi_f(r2) * w, bf16_lo_f(r3) * w, bf16_hi_f(r3) * w};
-          store_split8(base + kOffXw + off, base + kOffXw + kTile + off, vv);
+          store_split8(xw + off, xw + kTile + off, vv);
         }
         fence_proxy_async_smem();
-        arrive_lane0(c, bXwFull);
+        arrive_lane0(c, bXwFull0 + (j & 1));
       }
       arrive_lane0(c, bEmpty0 + rslot(j));
     }
@@ -806,6 +898,9 @@ __device__ void state_group_staged(const TcParams &p, const Ctl &c, uint32_t bas
     }
     tmem_st_wait();
   };
+  // The loads of item m + 2 are issued as soon as item m + 1 is staged, so
+  // they are in flight through a whole item (the h operand hand-over of item
+  // m + 1 included) before item m + 2 is staged.
   Item I;
   if (item_warp(p, c, base, 0, I) <= 0) return;
   load_h(I);
@@ -964,6 +1059,7 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
 // After the outputs of step j the group builds, two steps ahead, the
 // masked-decay matrices of step j + 2 with D on the diagonal (warp q:
 // direction slot q, row s = lane of M^T) and the diagonal's bf16 remainders.
+template <bool kGated>
 __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
   const int lane = threadIdx.x & 31;
   const int q = (threadIdx.x >> 5) & 3;
@@ -991,44 +1087,7 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
       return true;
     }
     if (!waitw(c, bFull0 + rslot(jm), parr(jm))) return false;  // C B^T tiles
-    if (act) {
-      const uint32_t cbrow = base + rslot(jm) * kSlot + kOffCB + q * 2048;
-      const uint32_t cq = base + kOffCum + (ct * 4 + q) * 128;
-      const float cs = lds_f32(cq + lane * 4);
-      const float ds = lds_f32(base + kOffDt + (ct * 4 + q) * 128 + lane * 4);
-      const uint32_t mrow = base + kOffMh + (jm & 1) * kMhBuf + q * kMhDir;
-      // this direction's D joins the diagonal of M (D x is part of X^T M^T):
-      // M[s][s] + D is stored as bf16 hi in M and its bf16 remainder lo on the
-      // diagonal of the block's 16 x 16 correction tile of chunk s / 16
-      const float Dq = lds_f32(base + kOffDtab + (ct * 4 + q) * 4);
-      // (not unrolled: a compact loop keeps the instruction cache footprint down)
-#pragma unroll 1
-      for (int jj = 0; jj < 4; ++jj) {
-        uint32_t r[4];
-        ld_shared_v4(cbrow + sw64_chunk(lane, jj), r[0], r[1], r[2], r[3]);  // C B^T[s = lane][8 jj ..]
-        float cj[8];
-        ld_shared_v4f(cq + 32 * jj, *reinterpret_cast<float(*)[4]>(&cj[0]));
-        ld_shared_v4f(cq + 32 * jj + 16, *reinterpret_cast<float(*)[4]>(&cj[4]));
-        float mv[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int t = 8 * jj + i;
-          const bool valid = rev ? (t <= lane) : (t >= lane);
-          const float e = ex2_approx(cj[i] - cs);
-          const float cb = (i & 1) ? bf16_hi_f(r[i >> 1]) : bf16_lo_f(r[i >> 1]);
-          mv[i] = valid ? cb * ds * e : 0.f;
-          if (t == lane) {
-            const float v = mv[i] + Dq;
-            const float hi = __bfloat162float(__float2bfloat16_rn(v));
-            sts_u16(mrow + inter_mn_off(32 + lane, lane, kMhSbo, kMhLbo),
-                    __bfloat16_as_ushort(__float2bfloat16_rn(v - hi)));
-            mv[i] = v;
-          }
-        }
-        st_shared_v4(mrow + inter_mn_off(8 * jj, lane, kMhSbo, kMhLbo), pack_bf16x2(mv[0], mv[1]),
-                     pack_bf16x2(mv[2], mv[3]), pack_bf16x2(mv[4], mv[5]), pack_bf16x2(mv[6], mv[7]));
-      }
-    }
+    build_masked_decay(base, q, lane, jm, act, rev);
     fence_proxy_async_smem();
     arrive_lane0(c, bMhFull0 + (jm & 1));
     ++mla;
@@ -1041,12 +1100,12 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
     if (item_warp(p, c, base, m, I) <= 0) return;
     for (int kk = 0; kk < I.nk; ++kk, ++j) {
       const int k = I.k0 + kk;  // block index in the sequence
-      const int i2 = j & 1, ct = j % kTab;
+      const int yb = ybuf(kGated, j), ct = j % kTab;
       if (!waitw(c, bAux0 + ct, part(j))) return;
-      if (!waitw(c, bYFull0 + i2, par2(j))) return;
+      if (!waitw(c, bYFull0 + yb, ypar(kGated, j))) return;
       tc_fence_after();
       uint32_t yo[32], yd[32];
-      const uint32_t ta = tmem_addr(tmem, 32 * q, kColY0 + kColYBuf * i2);
+      const uint32_t ta = tmem_addr(tmem, 32 * q, kColY0 + kColYBuf * yb);
       tmem_ld_16x32bx2_x32<32>(ta, yo);       // Y_off: clean columns 0.., noisy 32..
       tmem_ld_16x32bx2_x32<64>(ta + 64, yd);  // Y_diag: clean 64.., noisy 128..
       tmem_ld_wait();
@@ -1064,9 +1123,43 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
       tmem_ld_wait();
 #pragma unroll
       for (int t = 0; t < 32; ++t) yo[t] = __float_as_uint(__uint_as_float(yo[t]) + __uint_as_float(yd[t]));
+      // gated: yo is the forward direction's output; the reverse direction's
+      // own [Y_diag | remainder] goes to yd.  The TMEM loads are warp-wide
+      // (.sync.aligned), so they run whenever either stream has a reverse
+      // direction (uniform across the warp); a lane uses them only if its own
+      // stream has one.
+      const bool rev_act = kGated && pick4(p.active, fs | 2);
+      if (kGated && (p.active[kCR] || p.active[kNR])) {
+        tmem_ld_16x32bx2_x32<64>(ta + 64 + kColRevGated, yd);
+        tmem_ld_wait();
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t r16[16];
+          tmem_ld_16x32bx2_x16i<64>(ta + 96 + kColRevGated + 16 * hh, r16);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            yd[16 * hh + i] = __float_as_uint(__uint_as_float(yd[16 * hh + i]) + __uint_as_float(r16[i]));
+        }
+      }
       // the Y buffer may be reused from here on
       tc_fence_before();
-      arrive_lane0(c, bYEmpty0 + i2);
+      arrive_lane0(c, bYEmpty0 + yb);
+      if (kGated && mine) {
+        // y = y_fwd silu(z_fwd) + y_rev silu(z_rev) (a direction without z is not gated)
+        const int64_t zi = ((static_cast<int64_t>(I.b) * L + k * kT) * H + I.h) * kP + pcol;
+        const __nv_bfloat16 *zf = pick4(p.z, fs), *zr = rev_act ? pick4(p.z, fs | 2) : nullptr;
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+          float v = __uint_as_float(yo[t]);
+          if (zf) v *= silu_approx(__bfloat162float(zf[zi + t * H * kP]));
+          if (rev_act) {
+            const float u = __uint_as_float(yd[t]);
+            v += zr ? u * silu_approx(__bfloat162float(zr[zi + t * H * kP])) : u;
+          }
+          yo[t] = __float_as_uint(v);
+        }
+      }
       if (mine) {
         const int64_t yi = ((static_cast<int64_t>(I.b) * L + k * kT) * H + I.h) * kP + pcol;
         const int64_t tstride = H * kP;
@@ -1085,6 +1178,10 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
   }
 }
 
+// Instantiated without and with a gate: the gated epilogue (per-direction
+// accumulators, z loads) is compiled only into the gated kernel, so that it adds
+// nothing to the instruction footprint of the ungated one.
+template <bool kGated>
 __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -1141,7 +1238,7 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
   if (warp == 0) {
     if ((threadIdx.x & 31) == 0) producer(p, c, base);
   } else if (warp == 1) {
-    if ((threadIdx.x & 31) == 0) mma_issuer(p, c, base, tmem);
+    if ((threadIdx.x & 31) == 0) mma_issuer<kGated>(p, c, base, tmem);
   } else if (warp == 2 || warp == 3 || warp == 6 || warp == 7) {
     operand_group(p, c, base);
   } else if (warp == 4 || warp == 5) {
@@ -1149,7 +1246,7 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
   } else if (warp < 12) {
     state_group(p, c, base, tmem);
   } else {
-    epilogue_group(p, c, base, tmem);
+    epilogue_group<kGated>(p, c, base, tmem);
   }
   tc_fence_before();
   __syncthreads();
@@ -1234,7 +1331,8 @@ cudaError_t launch_scan(unsigned grid, cudaStream_t stream, const TcParams &p) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, bd_tc_kernel, p);
+  cudaError_t e = p.gated ? cudaLaunchKernelEx(&cfg, bd_tc_kernel<true>, p)
+                          : cudaLaunchKernelEx(&cfg, bd_tc_kernel<false>, p);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
@@ -1278,9 +1376,9 @@ static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 // C B^T tiles (bf16 [32][32] per direction, b, block, group), then for a
 // segmented plan the segments' local end states, their initial states and
 // their decays.
-size_t tc_workspace_bytes(int64_t Bsz, int64_t L, int64_t G, int64_t H) {
+size_t tc_workspace_bytes(int64_t Bsz, int64_t L, int64_t G, int64_t H, bool allblock) {
   const int64_t K = L / kT;
-  size_t bytes = align256(static_cast<size_t>(4) * Bsz * K * G * 2048);
+  size_t bytes = align256(static_cast<size_t>(cb_sets(allblock)) * Bsz * K * G * 2048);
   const int nseg = tc_plan_segments(Bsz, H, K);
   if (nseg > 1) {
     const size_t states = static_cast<size_t>(Bsz) * H * nseg * kP * kN * sizeof(float);
@@ -1292,12 +1390,9 @@ size_t tc_workspace_bytes(int64_t Bsz, int64_t L, int64_t G, int64_t H) {
 bool tc_supported(const ScanArgs &a) {
   if (!tc_shape_ok(a.P, a.N, a.T, a.in_bf16)) return false;
   if (a.Bsz <= 0 || a.L <= 0) return false;
-  const DirArgs *ds[4] = {&a.cf, &a.nf, &a.cr, &a.nr};
-  for (const DirArgs *d : ds)
-    if (d->z) return false;
   if (a.Bsz * a.H > 0x7fffffffLL || a.L > 0x7fffffffLL || 4 * a.Bsz * (a.L / kT) * a.G > 0x7fffffffLL)
     return false;
-  if (a.ws_bytes < kWsHeader + tc_workspace_bytes(a.Bsz, a.L, a.G, a.H)) return false;
+  if (a.ws_bytes < kWsHeader + tc_workspace_bytes(a.Bsz, a.L, a.G, a.H, a.mode == Mode::AllBlock)) return false;
   if (opt_force_generic()) return false;
   return device_is_sm100();
 }
@@ -1319,7 +1414,7 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
     if (!make_map_bf16(&cp.tb[nz], ds[i]->B, kN, a.G, a.L, a.Bsz) ||
         !make_map_bf16(&cp.tc[nz], ds[i]->C, kN, a.G, a.L, a.Bsz))
       return cudaErrorInvalidValue;
-    cp.slot[nz++] = i;
+    cp.slot[nz++] = cb_set(all, i);
   }
   cp.Bsz = static_cast<int>(a.Bsz);
   cp.K = K;
@@ -1361,12 +1456,14 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
     if (!ds[i]) continue;
     if (!make_map_bf16(&p.tx[i], ds[i]->x, kP, a.H, a.L, a.Bsz)) return cudaErrorInvalidValue;
     p.dt[i] = reinterpret_cast<const __nv_bfloat16 *>(ds[i]->dt);
+    p.z[i] = reinterpret_cast<const __nv_bfloat16 *>(ds[i]->z);
+    if (ds[i]->z) p.gated = 1;
     p.A[i] = ds[i]->A;
     p.D[i] = ds[i]->D;
   }
   if (!make_map_bf16(&p.tbcf, a.cf.B, kN, a.G, a.L, a.Bsz) ||
       !make_map_bf16(&p.tccf, a.cf.C, kN, a.G, a.L, a.Bsz) ||
-      !make_map_cb(&p.tcb, cbws, static_cast<uint64_t>(4) * a.Bsz * K * a.G))
+      !make_map_cb(&p.tcb, cbws, static_cast<uint64_t>(cb_sets(all)) * a.Bsz * K * a.G))
     return cudaErrorInvalidValue;
   if (all && !make_map_bf16(&p.tcnf, a.nf.C, kN, a.G, a.L, a.Bsz)) return cudaErrorInvalidValue;
   p.Bsz = static_cast<int>(a.Bsz);
@@ -1390,7 +1487,10 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
   p.status = a.status;
   p.timeout_ns = timeout;
   p.drain_ns = 1000000000ull;
-  e = cudaFuncSetAttribute(bd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(bd_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(bd_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
   // persistent CTAs, one per SM, each walking its share of the work items
@@ -1403,7 +1503,7 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
     // aggregate pass (clean forward state of every segment from zero), then
     // the chain of segment states
     uint8_t *wsb = static_cast<uint8_t *>(a.ws) + kWsHeader;
-    const size_t cb_bytes = align256(static_cast<size_t>(4) * a.Bsz * K * a.G * 2048);
+    const size_t cb_bytes = align256(static_cast<size_t>(cb_sets(all)) * a.Bsz * K * a.G * 2048);
     const size_t st_bytes = align256(static_cast<size_t>(a.Bsz) * a.H * nseg * kP * kN * sizeof(float));
     float *seg_local = reinterpret_cast<float *>(wsb + cb_bytes);
     float *seg_init = reinterpret_cast<float *>(wsb + cb_bytes + st_bytes);

@@ -280,6 +280,20 @@ __device__ __forceinline__ void tmem_ld_16x32bx2_x16(uint32_t taddr, uint32_t (&
       : "r"(taddr));
 }
 
+// 16 lanes x 2 x 16 columns of 32 bit: thread i < 16 receives lane
+// (lane(taddr) + i), columns col .. col + 15; thread i >= 16 receives lane
+// (lane(taddr) + i - 16), columns col + IMM .. col + IMM + 15.
+template <int IMM>
+__device__ __forceinline__ void tmem_ld_16x32bx2_x16i(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15}, [%16], %17;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15])
+      : "r"(taddr), "n"(IMM));
+}
+
 // 16 lanes x 2 x 32 columns of 32 bit: thread i < 16 receives lane
 // (lane(taddr) + i), columns col .. col + 31; thread i >= 16 receives lane
 // (lane(taddr) + i - 16), columns col + IMM .. col + IMM + 31.

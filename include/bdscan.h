@@ -290,7 +290,7 @@ const char *bdscan_status_string(int status);
  * process exits.  It calls no cudaMalloc or cudaFree.
  *   - Shapes whose workspace (bdscan_workspace_size(shape, BLOCK_STEP)) exceeds
  *     BDSCAN_NOALLOC_SCRATCH_BYTES are rejected with BDSCAN_ERR_SCRATCH_LIMIT
- *     (for the tensor-core shapes: batch * ngroups <= 512).
+ *     (for the tensor-core shapes: batch * ngroups <= 1024).
  *   - The first call on a device looks up the buffer's device address on that
  *     device (the device current at the call); make that first call before any
  *     stream capture begins.

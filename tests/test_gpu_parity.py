@@ -97,6 +97,55 @@ def test_no_reverse_and_gated():
         check_states(st, rst)
 
 
+@pytest.mark.parametrize("which", ["all", "fwd_only", "rev_only"])
+def test_gated_allblock(which):
+    """Gate per direction, y_dir * silu(z_dir) before the sum, on the
+    tensor-core path (bf16, P = 64, N = 128, T = 32): every direction gated,
+    or only the forward / only the reverse directions."""
+    s = _shape(batch=2, seqlen=192)
+    gate = {"all": (True, True), "fwd_only": (True, False), "rev_only": (False, True)}[which]
+    dirs = [W.make_dir(s, 12, 0, k, DEV, gated=gate[k in (W.CLEAN_REV, W.NOISY_REV)])
+            for k in (W.CLEAN_FWD, W.CLEAN_REV, W.NOISY_FWD, W.NOISY_REV)]
+    h0 = W.make_state(s, 12, device=DEV)
+    yc, yn, st = bd.allblock(s, *dirs, h0=h0)
+    ryc, ryn, rst = oracle.allblock(s.as_dict(), *dirs, h0=h0)
+    check_y(yc, ryc, what="y_clean")
+    check_y(yn, ryn, what="y_noisy")
+    check_states(st, rst)
+
+
+@pytest.mark.parametrize("commit", [False, True])
+def test_gated_block_step_and_prefix(commit):
+    s = _shape(batch=3, seqlen=32, chunk_len=32)
+    f = W.make_dir(s, 13, 0, W.CLEAN_FWD, DEV, gated=True)
+    r = W.make_dir(s, 13, 0, W.CLEAN_REV, DEV, gated=True)
+    state = W.make_state(s, 13, device=DEV)
+    y, so = bd.block_step(s, f, r, state, state_out=True if commit else None)
+    ry, rso = oracle.block_step(s.as_dict(), f, r, state, want_state_out=commit)
+    check_y(y, ry)
+    if commit:
+        check_states(so, rso, "state_out")
+    sp = _shape(batch=1, nheads=4, ngroups=1, seqlen=1280)  # segmented plan
+    f = W.make_dir(sp, 14, 0, W.CLEAN_FWD, DEV, gated=True)
+    r = W.make_dir(sp, 14, 0, W.CLEAN_REV, DEV, gated=True)
+    y, st, fin = bd.prefix(sp, f, r)
+    ry, rst, rfin = oracle.prefix(sp.as_dict(), f, r)
+    check_y(y, ry)
+    check_states(st, rst)
+    check_states(fin, rfin, "final")
+
+
+def test_gated_87m_allblock_full():
+    """The 87M all-block layer with every direction gated, at full size."""
+    s = W.WORKLOADS["87m_allblock"]
+    cf, cr, nf, nr = W.make_streams(s, W.SEEDS["87m_allblock"], device=DEV, gated=True)
+    yc, yn, st = bd.allblock(s, cf, cr, nf, nr)
+    ryc, ryn, rst = oracle.allblock(s.as_dict(), cf, cr, nf, nr)
+    check_y(yc, ryc, what="y_clean")
+    check_y(yn, ryn, what="y_noisy")
+    check_states(st, rst)
+
+
 def test_cache_independent_of_active_block_bitwise():
     """Boundary states do not depend on the noisy stream or the reverse
     direction (bit-exact), and a perturbation of clean x at token j leaves

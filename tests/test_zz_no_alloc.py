@@ -59,9 +59,9 @@ def test_noalloc_step_matches_block_step(name):
 
 @pytest.mark.gpu
 def test_noalloc_step_rejects_shapes_beyond_its_scratch():
-    # batch * ngroups = 520 > 512 tensor-core tiles' worth of scratch; rejected
+    # batch * ngroups = 1040 > 1024 tensor-core tiles' worth of scratch; rejected
     # on the host before anything is launched
-    s = W.Shape(batch=520, seqlen=32, nheads=1, headdim=64, dstate=128, ngroups=1, block_len=32,
+    s = W.Shape(batch=1040, seqlen=32, nheads=1, headdim=64, dstate=128, ngroups=1, block_len=32,
                 chunk_len=32, in_dtype="bf16")
     f, r = W.make_streams(s, 50, streams=(W.CLEAN_FWD, W.CLEAN_REV), device=DEV)
     state = W.make_state(s, 50, device=DEV)
