@@ -465,6 +465,10 @@ __device__ __forceinline__ Item item_at(const TcParams &p, int it) {
 // barrier ring of the per-step tables: phase parity of step j
 __device__ __forceinline__ uint32_t part(int j) { return (static_cast<uint32_t>(j) / kTab) & 1u; }
 
+// Kernel instances: the call's mode is a template parameter (bits kModeAgg,
+// kModeAll, kModeNeedS), so each instance carries only the code its mode runs.
+enum : int { kModeAgg = 1, kModeAll = 2, kModeNeedS = 4 };
+
 __device__ __forceinline__ int lds_s32(uint32_t addr) {
   int v;
   asm volatile("ld.shared.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
@@ -522,18 +526,19 @@ __device__ __forceinline__ int item_warp(const TcParams &p, const Ctl &c, uint32
 }
 
 // ---------------------------------------------------------------- producer
+template <int kM>
 __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
+  constexpr bool kAgg = kM & kModeAgg, kAll = kM & kModeAll;
   const int nact = p.active[0] + p.active[1] + p.active[2] + p.active[3];
   // x of each active direction, C B^T tiles, B of the clean forward direction
   // (only when S is formed), C of the clean (and noisy) forward direction
-  const uint32_t bytes = p.agg ? 3 * kTile
-                               : nact * (kTile + 2048) + (2 + (p.allblock ? 4 : 2)) * kTile;
+  const uint32_t bytes = kAgg ? 3 * kTile : nact * (kTile + 2048) + (2 + (kAll ? 4 : 2)) * kTile;
 #pragma unroll
   for (int i = 0; i < 4; ++i)
     if (p.active[i]) tma_prefetch_desc(&p.tx[i]);
   tma_prefetch_desc(&p.tbcf);
   tma_prefetch_desc(&p.tccf);
-  if (p.allblock) tma_prefetch_desc(&p.tcnf);
+  if (kAll) tma_prefetch_desc(&p.tcnf);
   tma_prefetch_desc(&p.tcb);
   int last[kSlots] = {-1, -1, -1};
   int j = 0;
@@ -567,10 +572,10 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
         if (p.active[i]) tma_load_4d_s(st + kOffX + i * kTile, &p.tx[i], full, 0, I.h, t0, I.b);
       tma_load_4d_s(st + kOffBcf, &p.tbcf, full, 0, I.g, t0, I.b);
       tma_load_4d_s(st + kOffBcf + kTile, &p.tbcf, full, 64, I.g, t0, I.b);
-      if (!p.agg) {
+      if (!kAgg) {
         tma_load_4d_s(st + kOffClo, &p.tccf, full, 0, I.g, t0, I.b);
         tma_load_4d_s(st + kOffChi, &p.tccf, full, 64, I.g, t0, I.b);
-        if (p.allblock) {
+        if (kAll) {
           tma_load_4d_s(st + kOffClo + kTile, &p.tcnf, full, 0, I.g, t0, I.b);
           tma_load_4d_s(st + kOffChi + kTile, &p.tcnf, full, 64, I.g, t0, I.b);
         }
@@ -582,7 +587,7 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           if (!p.active[i]) continue;
-          const int idx = ((cb_set(p.allblock, i) * p.Bsz + I.b) * p.K + k) * p.G + I.g;
+          const int idx = ((cb_set(kAll, i) * p.Bsz + I.b) * p.K + k) * p.G + I.g;
           tma_load_3d_s(st + kOffCB + i * 2048, &p.tcb, full, 0, 0, idx);
         }
       }
@@ -607,11 +612,12 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
 // Issue order per step: S; Y_off (then commit "h consumed" so the state group
 // may overwrite the h operand at once); Y_diag and the D x products.
 // Descriptors are built once; per step only their start addresses move.
-template <bool kGated>
+template <int kM, bool kGated>
 __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
+  constexpr bool kAgg = kM & kModeAgg, kAll = kM & kModeAll, kNeedS = kM & kModeNeedS;
   const uint32_t id_s = idesc_bf16(128, 64, 1, 1);  // S^T[n][p] = B^T (w o X)
   // Y_off^T[p][t] = h C^T over the stacked [C_cf; C_nf] rows (only C_cf without a noisy stream)
-  const uint32_t id_yo = p.allblock ? idesc_bf16(64, 64, 1, 0) : idesc_bf16(64, 32, 1, 0);
+  const uint32_t id_yo = kAll ? idesc_bf16(64, 64, 1, 0) : idesc_bf16(64, 32, 1, 0);
   const uint32_t id_yd = idesc_bf16(64, 64, 1, 1);  // [Y_diag^T | remainder][p][t'] = X^T [M^T | diag]
   // descriptor of each operand at its first tile; moving an operand by b bytes adds b >> 4
   const D64 dBcf = split64(sdesc(base + kOffBcf, kTile, 1024, kLayoutSw128));
@@ -633,7 +639,7 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
       const uint32_t so = BD_OFF(static_cast<uint32_t>(r) * kSlot);  // this step's ring slot
       if (!wait1(c, bFull0 + r, parr(j))) break;
       // ---- S^T = B_cf^T (w o X): A MN-major (n; halves 4 KB apart), B MN-major (p)
-      if (p.need_s) {
+      if (kNeedS) {
         if (!wait1(c, bXwFull0 + i2, par2(j))) break;
         if (j >= 2 && !wait1(c, bSEmpty0 + i2, par2(j - 2))) break;
         tc_fence_after();
@@ -646,7 +652,7 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
         }
         umma_commit_s(bar_at(c, bSFull0 + i2));
       }
-      if (p.agg) {  // aggregate pass: the forward state is all it needs
+      if (kAgg) {  // aggregate pass: the forward state is all it needs
         umma_commit_s(bar_at(c, bEmpty0 + r));
         ok = true;
         continue;
@@ -747,7 +753,9 @@ __device__ __forceinline__ void build_masked_decay(uint32_t base, int q, int lan
 // Per step: the per-step tables (cumulative decays, dt, exp(cum) of the
 // forward directions, D of the step's head, item-start flag) and w o X.
 // The masked-decay matrices are built by the epilogue warps.
+template <int kM>
 __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
+  constexpr bool kNeedS = kM & kModeNeedS;
   const int lane = threadIdx.x & 31;
   const int wq = threadIdx.x >> 5;
   const int q = wq < 4 ? wq - 2 : wq - 4;
@@ -835,7 +843,7 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
       if (!waitw(c, bAux0 + ct, part(j))) return;
       if (!waitw(c, bFull0 + rslot(j), parr(j))) return;
       // ---- (w o X) of the clean forward direction, bf16 hi + lo
-      if (p.need_s) {
+      if (kNeedS) {
         // the S MMA of the previous step has read the w o X buffer
         const int jr = j - 1;
         if (jr >= 0 && !waitw(c, bSFull0 + (jr & 1), par2(jr))) return;
@@ -940,12 +948,14 @@ __device__ void state_group_staged(const TcParams &p, const Ctl &c, uint32_t bas
 
 // warps 8..11: thread owns column n = 32 q + lane of the state, h^T[n][0..63].
 // A failed (timed-out) wait ends the group at once: nothing else is stored.
+template <int kM>
 __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
+  constexpr bool kAgg = kM & kModeAgg, kNeedS = kM & kModeNeedS;
   const int lane = threadIdx.x & 31;
   const int q = (threadIdx.x >> 5) & 3;
   const int n = 32 * q + lane;
   const uint32_t cum = base + kOffCum;
-  if (!p.need_s) {
+  if constexpr (!kNeedS) {
     state_group_staged(p, c, base, tmem);
     return;
   }
@@ -985,7 +995,7 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
       // initial state of this item: h0 (first segment), the chained state the
       // aggregate and combine passes left in the workspace (later segments),
       // or zero (aggregate pass)
-      const float *src = p.agg ? nullptr
+      const float *src = kAgg ? nullptr
                          : I.seg == 0 ? (p.h0 ? p.h0 + bh * PN + n : nullptr)
                                       : p.seg_init + (bh * p.nseg + I.seg) * PN + n;
       if (src && I.seg > 0) wait_prior_grid();  // segment states: written by the combine kernel
@@ -994,7 +1004,7 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
     }
     float decay_log2 = 0.f;  // total decay over the item (aggregate pass)
     for (int kk = 0;; ++kk) {
-      if (kk < nk && !p.agg) {
+      if (kk < nk && !kAgg) {
         // Y_off of the previous step has read the h operand; the state
         // entering this block replaces it
         if (j >= 1 && !waitw(c, bHCons, (j - 1) & 1)) return;
@@ -1010,7 +1020,7 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
               Item E;  // (re-read from the ring: its entry is not reused before every role moved on)
               (void)item_read(p, base, m, E);
               const int64_t ebh = static_cast<int64_t>(E.b) * H + E.h;
-              if (p.agg) {
+              if (kAgg) {
                 const int64_t ebhs = ebh * p.nseg + E.seg;
                 dst = p.seg_local + ebhs * PN + n;
                 if (n == 0) p.seg_decay[ebhs] = decay_log2;
@@ -1059,18 +1069,19 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
 // After the outputs of step j the group builds, two steps ahead, the
 // masked-decay matrices of step j + 2 with D on the diagonal (warp q:
 // direction slot q, row s = lane of M^T) and the diagonal's bf16 remainders.
-template <bool kGated>
+template <int kM, bool kGated>
 __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
+  constexpr bool kAgg = kM & kModeAgg, kAll = kM & kModeAll;
   const int lane = threadIdx.x & 31;
   const int q = (threadIdx.x >> 5) & 3;
   const int pcol = 16 * q + (lane & 15);
   const bool noisy = lane >= 16;
   const int fs = noisy ? kNF : kCF;
   void *yout = noisy ? p.y_noisy : p.y_clean;
-  const bool mine = (noisy ? p.allblock != 0 : true) && yout != nullptr;
+  const bool mine = (noisy ? kAll : true) && yout != nullptr;
   const uint32_t cumt = base + kOffCum;
   const int64_t H = p.H, L = p.L;
-  if (p.agg) return;
+  if constexpr (kAgg) return;
   const bool act = pick4(p.active, q) != 0;
   const bool rev = q >= 2;
   int mla = 0;        // next step whose masked-decay matrices this group builds
@@ -1181,8 +1192,9 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
 // Instantiated without and with a gate: the gated epilogue (per-direction
 // accumulators, z loads) is compiled only into the gated kernel, so that it adds
 // nothing to the instruction footprint of the ungated one.
-template <bool kGated>
+template <int kM, bool kGated>
 __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constant__ TcParams p) {
+  constexpr bool kAgg = kM & kModeAgg;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -1214,7 +1226,7 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
   }
   // Clear the intra-block operands: of their remainder halves only the
   // diagonals are ever written.
-  if (!p.agg) {
+  if (!kAgg) {
     const uint4 zero = make_uint4(0, 0, 0, 0);
     for (uint32_t o = threadIdx.x * 16; o < 2 * kMhBuf; o += kThreads * 16)
       *reinterpret_cast<uint4 *>(sm + kOffMh + o) = zero;
@@ -1236,17 +1248,17 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
   // just before those reads; everything else overlaps its tail.
 
   if (warp == 0) {
-    if ((threadIdx.x & 31) == 0) producer(p, c, base);
+    if ((threadIdx.x & 31) == 0) producer<kM>(p, c, base);
   } else if (warp == 1) {
-    if ((threadIdx.x & 31) == 0) mma_issuer<kGated>(p, c, base, tmem);
+    if ((threadIdx.x & 31) == 0) mma_issuer<kM, kGated>(p, c, base, tmem);
   } else if (warp == 2 || warp == 3 || warp == 6 || warp == 7) {
-    operand_group(p, c, base);
+    operand_group<kM>(p, c, base);
   } else if (warp == 4 || warp == 5) {
     // idle: keeps the operand warps off the MMA issuer's SM sub-partition
   } else if (warp < 12) {
-    state_group(p, c, base, tmem);
+    state_group<kM>(p, c, base, tmem);
   } else {
-    epilogue_group<kGated>(p, c, base, tmem);
+    epilogue_group<kM, kGated>(p, c, base, tmem);
   }
   tc_fence_before();
   __syncthreads();
@@ -1317,8 +1329,19 @@ bool make_map_cb(CUtensorMap *m, const void *ptr, uint64_t ntiles) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <int kM, bool kGated>
+cudaError_t launch_instance(const cudaLaunchConfig_t &cfg, const TcParams &p) {
+  cudaError_t e = cudaFuncSetAttribute(bd_tc_kernel<kM, kGated>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  return cudaLaunchKernelEx(&cfg, bd_tc_kernel<kM, kGated>, p);
+}
+
 // The scan kernel as a programmatic dependent launch (its prologue may overlap
-// the previous kernel in the stream; it waits for that kernel before reading).
+// the previous kernel in the stream; it waits for that kernel before reading),
+// in the instance of the call's mode: the aggregate pass, the all-block pass,
+// a scan with a state chain (per-block or final state), or one-block items
+// without one; each but the first with or without a gate.
 cudaError_t launch_scan(unsigned grid, cudaStream_t stream, const TcParams &p) {
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
@@ -1331,8 +1354,16 @@ cudaError_t launch_scan(unsigned grid, cudaStream_t stream, const TcParams &p) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = p.gated ? cudaLaunchKernelEx(&cfg, bd_tc_kernel<true>, p)
-                          : cudaLaunchKernelEx(&cfg, bd_tc_kernel<false>, p);
+  cudaError_t e;
+  if (p.agg)
+    e = launch_instance<kModeAgg | kModeNeedS, false>(cfg, p);
+  else if (p.allblock)
+    e = p.gated ? launch_instance<kModeAll | kModeNeedS, true>(cfg, p)
+                : launch_instance<kModeAll | kModeNeedS, false>(cfg, p);
+  else if (p.need_s)
+    e = p.gated ? launch_instance<kModeNeedS, true>(cfg, p) : launch_instance<kModeNeedS, false>(cfg, p);
+  else
+    e = p.gated ? launch_instance<0, true>(cfg, p) : launch_instance<0, false>(cfg, p);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
@@ -1487,12 +1518,6 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
   p.status = a.status;
   p.timeout_ns = timeout;
   p.drain_ns = 1000000000ull;
-  e = cudaFuncSetAttribute(bd_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(kSmemBytes));
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(bd_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(kSmemBytes));
-  if (e != cudaSuccess) return e;
   // persistent CTAs, one per SM, each walking its share of the work items
   int dev = 0, nsm = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
