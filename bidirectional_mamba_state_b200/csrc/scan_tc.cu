@@ -462,6 +462,15 @@ __device__ __forceinline__ Item item_at(const TcParams &p, int it) {
   return r;
 }
 
+// Block of the sequence that step kk of an item covers: in order, or, in the
+// aggregate pass, from the item's last block to its first (the segment's
+// state is accumulated with weights relative to the segment's end, which are
+// known block by block in that order).
+template <bool kAgg>
+__device__ __forceinline__ int item_block(int k0, int nk, int kk) {
+  return kAgg ? k0 + nk - 1 - kk : k0 + kk;
+}
+
 // barrier ring of the per-step tables: phase parity of step j
 __device__ __forceinline__ uint32_t part(int j) { return (static_cast<uint32_t>(j) / kTab) & 1u; }
 
@@ -557,7 +566,7 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
   for (int m = 0; ok && cur >= 0; ++m) {
     const Item I = item_at(p, cur);
     for (int kk = 0; kk < I.nk; ++kk, ++j) {
-      const int k = I.k0 + kk;  // block index in the sequence
+      const int k = item_block<kAgg>(I.k0, I.nk, kk);  // block index in the sequence
       const int r = rslot(j);
       if (!wait1(c, bEmpty0 + r, parr(j) ^ 1)) {
         ok = false;
@@ -638,6 +647,26 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
       const int r = rslot(j), i2 = j & 1;
       const uint32_t so = BD_OFF(static_cast<uint32_t>(r) * kSlot);  // this step's ring slot
       if (!wait1(c, bFull0 + r, parr(j))) break;
+      if constexpr (kAgg) {
+        // ---- aggregate pass: S^T of the item accumulates over its blocks
+        //      (walked last to first, w o X weighted to the item's end) in the
+        //      item's buffer; the state group reads it once, at the item's end
+        if (!wait1(c, bXwFull0 + i2, par2(j))) break;
+        const int sb = m & 1;
+        if (kk == 0 && m >= 2 && !wait1(c, bSEmpty0 + sb, ((m - 2) >> 1) & 1)) break;
+        tc_fence_after();
+        const uint32_t colS = tmem + kColS0 + 64 * sb;
+        const D64 dxw = dXw + (i2 ? BD_OFF(kOffH - kOffXw) : 0u);
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+          umma_bf16(colS, dBcf + so + BD_OFF(ks * 2048), dxw + BD_OFF(ks * 2048), id_s, (kk > 0 || ks > 0) ? 1u : 0u);
+          umma_bf16(colS, dBcf + so + BD_OFF(ks * 2048), dxw + BD_OFF(kTile + ks * 2048), id_s, 1);
+        }
+        umma_commit_s(bar_at(c, bEmpty0 + r));
+        if (kk + 1 == nk) umma_commit_s(bar_at(c, bSFull0 + sb));
+        ok = true;
+        continue;
+      }
       // ---- S^T = B_cf^T (w o X): A MN-major (n; halves 4 KB apart), B MN-major (p)
       if (kNeedS) {
         if (!wait1(c, bXwFull0 + i2, par2(j))) break;
@@ -651,11 +680,6 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
           umma_bf16(colS, dBcf + so + BD_OFF(ks * 2048), dxw + BD_OFF(kTile + ks * 2048), id_s, 1);
         }
         umma_commit_s(bar_at(c, bSFull0 + i2));
-      }
-      if (kAgg) {  // aggregate pass: the forward state is all it needs
-        umma_commit_s(bar_at(c, bEmpty0 + r));
-        ok = true;
-        continue;
       }
       // ---- Y_off^T = h [C_cf; C_nf]^T, h = the state before this block
       if (!wait1(c, bHFull, j & 1)) break;
@@ -755,7 +779,7 @@ __device__ __forceinline__ void build_masked_decay(uint32_t base, int q, int lan
 // The masked-decay matrices are built by the epilogue warps.
 template <int kM>
 __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
-  constexpr bool kNeedS = kM & kModeNeedS;
+  constexpr bool kAgg = kM & kModeAgg, kNeedS = kM & kModeNeedS;
   const int lane = threadIdx.x & 31;
   const int wq = threadIdx.x >> 5;
   const int q = wq < 4 ? wq - 2 : wq - 4;
@@ -786,7 +810,8 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
     qd[e] = 0.f;
     if (!cv) return;
     if (act) {
-      qdt[e] = __bfloat162float(dtp[(static_cast<int64_t>(CI.b) * L + (CI.k0 + ckk) * kT + lane) * H + CI.h]);
+      qdt[e] = __bfloat162float(
+          dtp[(static_cast<int64_t>(CI.b) * L + item_block<kAgg>(CI.k0, CI.nk, ckk) * kT + lane) * H + CI.h]);
       qa[e] = Ap[CI.h] * kLog2e;
     }
     if (dact) qd[e] = Dp[CI.h];
@@ -806,6 +831,7 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
   cursor_load(1);
   if (!cursor_next()) return;
   int j = 0;
+  float rdec = 0.f;  // aggregate pass: decay (log2) of the item's blocks after this one
   for (int m = 0;; ++m) {
     bool has_next = false;
     Item In = I;
@@ -844,12 +870,23 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
       if (!waitw(c, bFull0 + rslot(j), parr(j))) return;
       // ---- (w o X) of the clean forward direction, bf16 hi + lo
       if (kNeedS) {
-        // the S MMA of the previous step has read the w o X buffer
-        const int jr = j - 1;
-        if (jr >= 0 && !waitw(c, bSFull0 + (jr & 1), par2(jr))) return;
-        const uint32_t xw = base + kOffXw;
+        uint32_t xw = base + kOffXw;
+        float rw = 0.f;  // log2 weight of the block's end relative to the item's end
+        if constexpr (kAgg) {
+          // two w o X buffers (the h operand's space is free in this pass):
+          // the S MMAs of step j - 2 have read this one once their commit
+          // completed the ring slot's empty phase of that step
+          if (kk == 0) rdec = 0.f;
+          rw = rdec;
+          if (j & 1) xw = base + kOffH;
+          if (j >= 2 && !waitw(c, bEmpty0 + rslot(j - 2), parr(j - 2))) return;
+        } else {
+          // the S MMA of the previous step has read the w o X buffer
+          if (j >= 1 && !waitw(c, bSFull0 + ((j - 1) & 1), par2(j - 1))) return;
+        }
         const uint32_t cf = cum + (ct * 4 + kCF) * 128, df = dts + (ct * 4 + kCF) * 128;
         const float c31 = lds_f32(cf + 31 * 4);
+        if constexpr (kAgg) rdec += c31;
 #pragma unroll
         for (int rep = 0; rep < 2; ++rep) {
           const int i = gt + 128 * rep;
@@ -857,7 +894,7 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
           const uint32_t off = sw128_chunk(t, ch);
           uint32_t r0, r1, r2, r3;
           ld_shared_v4(st + kOffX + off, r0, r1, r2, r3);
-          const float w = lds_f32(df + t * 4) * ex2_approx(c31 - lds_f32(cf + t * 4));
+          const float w = lds_f32(df + t * 4) * ex2_approx(c31 - lds_f32(cf + t * 4) + rw);
           float vv[8] = {bf16_lo_f(r0) * w, bf16_hi_f(r0) * w, bf16_lo_f(r1) * w, bf16_hi_f(r1) * w,
                          bf16_lo_f(r2) * w, bf16_hi_f(r2) * w, bf16_lo_f(r3) * w, bf16_hi_f(r3) * w};
           store_split8(xw + off, xw + kTile + off, vv);
@@ -946,6 +983,47 @@ __device__ void state_group_staged(const TcParams &p, const Ctl &c, uint32_t bas
   }
 }
 
+// Aggregate pass: an item's S^T accumulates over all its blocks in TMEM (the
+// issuer walks them last to first with weights relative to the item's end), so
+// the group only adds up the item's total decay from the per-step tables and,
+// after its last block, stores the accumulated state (the segment's end state
+// from a zero start) and that decay.
+__device__ void state_group_agg(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
+  const int lane = threadIdx.x & 31;
+  const int q = (threadIdx.x >> 5) & 3;
+  const int n = 32 * q + lane;
+  const uint32_t cum = base + kOffCum;
+  const int64_t PN = kP * kN;
+  int j = 0;
+  for (int m = 0;; ++m) {
+    Item I;
+    if (item_warp(p, c, base, m, I) <= 0) return;
+    float decay_log2 = 0.f;
+    for (int kk = 0; kk < I.nk; ++kk, ++j) {
+      const int ct = j % kTab;
+      if (!waitw(c, bAux0 + ct, part(j))) return;
+      decay_log2 += lds_f32(cum + ((ct * 4 + kCF) * 32 + 31) * 4);
+    }
+    const int sb = m & 1;
+    if (!waitw(c, bSFull0 + sb, (m >> 1) & 1)) return;
+    tc_fence_after();
+    const int64_t ebhs = (static_cast<int64_t>(I.b) * p.H + I.h) * p.nseg + I.seg;
+    float *dst = p.seg_local + ebhs * PN + n;
+    const uint32_t ta = tmem_addr(tmem, 32 * q, kColS0 + 64 * sb);
+#pragma unroll
+    for (int cq = 0; cq < 4; ++cq) {
+      uint32_t sv[16];
+      tmem_ld_32x32b_x16(ta + 16 * cq, sv);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) dst[(16 * cq + i) * kN] = __uint_as_float(sv[i]);
+    }
+    if (n == 0) p.seg_decay[ebhs] = decay_log2;
+    tc_fence_before();
+    arrive_lane0(c, bSEmpty0 + sb);
+  }
+}
+
 // warps 8..11: thread owns column n = 32 q + lane of the state, h^T[n][0..63].
 // A failed (timed-out) wait ends the group at once: nothing else is stored.
 template <int kM>
@@ -957,6 +1035,9 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
   const uint32_t cum = base + kOffCum;
   if constexpr (!kNeedS) {
     state_group_staged(p, c, base, tmem);
+    return;
+  } else if constexpr (kAgg) {
+    state_group_agg(p, c, base, tmem);
     return;
   }
   const int64_t H = p.H;
@@ -1062,6 +1143,14 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
   }
 }
 
+// bf16 outputs of one thread (32 tokens of column p), out of line in the
+// instances with a state chain (their epilogue loop runs faster without the
+// inline copy; the one-block-item instance measured the other way).
+__device__ __noinline__ void store_y_bf16(__nv_bfloat16 *dst, int64_t tstride, const uint32_t (&yo)[32]) {
+#pragma unroll
+  for (int t = 0; t < 32; ++t) dst[t * tstride] = __float2bfloat16_rn(__uint_as_float(yo[t]));
+}
+
 // ---------------------------------------------------------------- epilogue
 // warps 12..15: thread owns column p = 16 q + (lane & 15) of the clean
 // (lane < 16) or noisy (lane >= 16) stream's outputs y[t][p], t = 0..31:
@@ -1071,7 +1160,7 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
 // direction slot q, row s = lane of M^T) and the diagonal's bf16 remainders.
 template <int kM, bool kGated>
 __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
-  constexpr bool kAgg = kM & kModeAgg, kAll = kM & kModeAll;
+  constexpr bool kAgg = kM & kModeAgg, kAll = kM & kModeAll, kNeedS = kM & kModeNeedS;
   const int lane = threadIdx.x & 31;
   const int q = (threadIdx.x >> 5) & 3;
   const int pcol = 16 * q + (lane & 15);
@@ -1176,8 +1265,12 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
         const int64_t tstride = H * kP;
         if (p.out_bf16) {
           __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(yout) + yi;
+          if constexpr (kNeedS) {
+            store_y_bf16(dst, tstride, yo);
+          } else {
 #pragma unroll
-          for (int t = 0; t < 32; ++t) dst[t * tstride] = __float2bfloat16_rn(__uint_as_float(yo[t]));
+            for (int t = 0; t < 32; ++t) dst[t * tstride] = __float2bfloat16_rn(__uint_as_float(yo[t]));
+          }
         } else {
           float *dst = reinterpret_cast<float *>(yout) + yi;
 #pragma unroll
@@ -1315,6 +1408,7 @@ bool make_map_bf16(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, ui
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
 
 // bf16 C B^T tiles [n][32][32], box (32, 32, 1), 64-byte swizzle.
 bool make_map_cb(CUtensorMap *m, const void *ptr, uint64_t ntiles) {
