@@ -175,7 +175,7 @@ def bdscan_version() -> int:
     return int(lib().bdscan_version())
 
 
-BDSCAN_OPT_WAIT_TIMEOUT_NS, BDSCAN_OPT_FORCE_GENERIC, BDSCAN_OPT_VERBOSE = 0, 1, 2
+BDSCAN_OPT_WAIT_TIMEOUT_NS, BDSCAN_OPT_FORCE_GENERIC, BDSCAN_OPT_VERBOSE, BDSCAN_OPT_CB_PREPASS = 0, 1, 2, 3
 
 
 def bdscan_set_option(option: int, value: int) -> int:

@@ -24,12 +24,14 @@ struct Options {
   std::atomic<unsigned long long> wait_timeout_ns{2000000000ull};
   std::atomic<int> force_generic{0};
   std::atomic<int> verbose{0};
+  std::atomic<int> cb_prepass{0};
   Options() {
     // initial values from the environment, read once
     if (const char *v = std::getenv("BDSCAN_WAIT_TIMEOUT_NS"); v && *v)
       wait_timeout_ns = std::strtoull(v, nullptr, 10);
     if (const char *v = std::getenv("BDSCAN_FORCE_GENERIC"); v && v[0] == '1') force_generic = 1;
     if (const char *v = std::getenv("BDSCAN_VERBOSE"); v && v[0] == '1') verbose = 1;
+    if (const char *v = std::getenv("BDSCAN_CB_PREPASS"); v && v[0] == '1') cb_prepass = 1;
   }
 };
 
@@ -43,6 +45,7 @@ Options &options() {
 unsigned long long opt_wait_timeout_ns() { return options().wait_timeout_ns.load(std::memory_order_relaxed); }
 bool opt_force_generic() { return options().force_generic.load(std::memory_order_relaxed) != 0; }
 bool opt_verbose() { return options().verbose.load(std::memory_order_relaxed) != 0; }
+bool opt_cb_prepass() { return options().cb_prepass.load(std::memory_order_relaxed) != 0; }
 
 }  // namespace bdscan
 
@@ -481,6 +484,9 @@ long long bdscan_set_option(int option, long long value) {
     case BDSCAN_OPT_VERBOSE:
       if (value != 0 && value != 1) return BDSCAN_ERR_INVALID_ARG;
       return o.verbose.exchange((int)value);
+    case BDSCAN_OPT_CB_PREPASS:
+      if (value != 0 && value != 1) return BDSCAN_ERR_INVALID_ARG;
+      return o.cb_prepass.exchange((int)value);
     default:
       return BDSCAN_ERR_INVALID_ARG;
   }
@@ -491,6 +497,7 @@ long long bdscan_get_option(int option) {
     case BDSCAN_OPT_WAIT_TIMEOUT_NS: return (long long)bdscan::opt_wait_timeout_ns();
     case BDSCAN_OPT_FORCE_GENERIC: return bdscan::opt_force_generic() ? 1 : 0;
     case BDSCAN_OPT_VERBOSE: return bdscan::opt_verbose() ? 1 : 0;
+    case BDSCAN_OPT_CB_PREPASS: return bdscan::opt_cb_prepass() ? 1 : 0;
     default: return BDSCAN_ERR_INVALID_ARG;
   }
 }

@@ -12,6 +12,7 @@ enum class Mode : int { Prefix = 0, Step = 1, AllBlock = 2 };
 unsigned long long opt_wait_timeout_ns();
 bool opt_force_generic();
 bool opt_verbose();
+bool opt_cb_prepass();
 
 struct DirArgs {
   const void *x, *dt, *B, *C, *z;  // z == nullptr: no gate

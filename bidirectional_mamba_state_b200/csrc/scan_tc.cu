@@ -246,6 +246,7 @@ enum : int {
   bFull0 = 0, bFull1, bFull2, bEmpty0, bEmpty1, bEmpty2, bAux0, bAux7 = bAux0 + kTab - 1, bXwFull0, bXwFull1, bSFull0,
   bSFull1,
   bSEmpty0, bSEmpty1, bMhFull0, bMhFull1, bHFull, bHCons, bYFull0, bYFull1, bYEmpty0, bYEmpty1, bDrain,
+  bCbFull,
   bItem0, bCount = bItem0 + kItemRing
 };
 static_assert(bCount <= kNumBars, "barrier array");
@@ -256,7 +257,32 @@ static_assert(bCount <= kNumBars, "barrier array");
 // direction keeps its own [Y_diag^T | remainder]: one Y buffer of
 // {Y_off^T, clean fwd, noisy fwd, clean rev, noisy rev} (320 columns).
 constexpr uint32_t kColS0 = 0, kColY0 = 128, kColYBuf = 192, kColRevGated = 128;
+// C B^T accumulator of the fused-C B^T instance (M = 64 rows [s_cf; s_cr], N = 64
+// columns [t_cf | t_cr]): the second staging buffer of the initial state, which
+// a CTA that takes a single one-block item never uses
+constexpr uint32_t kColCb = kColS0 + 64;
 constexpr uint32_t kTmemCols = 512;
+
+// Division of n (0 <= n < 2^31) by a divisor d fixed per launch (1 <= d < 2^31)
+// as a multiply and a shift (round-up reciprocal): with s = ceil(log2 d) and
+// m = ceil(2^(31+s) / d), floor(n m / 2^(31+s)) = floor(n / d) for every such
+// n, because the error m d - 2^(31+s) is below d <= 2^s.  A work item's
+// coordinates come from three such divisions; five integer divisions (a long
+// dependent instruction sequence each) delayed the first load by about 0.6 us.
+struct DivU {
+  unsigned long long m;
+  int sh;
+  int pad;
+};
+inline DivU make_divu(int d) {
+  int s = 0;
+  while ((1ll << s) < d) ++s;
+  const unsigned long long num = 1ull << (31 + s);
+  return DivU{(num + static_cast<unsigned long long>(d) - 1) / static_cast<unsigned long long>(d), 31 + s, 0};
+}
+__device__ __forceinline__ int divu(int n, const DivU &v) {
+  return static_cast<int>((static_cast<unsigned long long>(n) * v.m) >> v.sh);
+}
 
 struct TcParams {
   CUtensorMap tx[4];
@@ -264,15 +290,18 @@ struct TcParams {
   CUtensorMap tccf;
   CUtensorMap tcnf;
   CUtensorMap tcb;
+  CUtensorMap tbcr, tccr;  // B and C of the clean reverse direction (kModeCbFused)
   const __nv_bfloat16 *dt[4];
   const float *A[4];
   const float *D[4];
   const __nv_bfloat16 *z[4];  // gate of each direction, or null
   int active[4];
   int gated;                   // some direction has a gate: single Y buffer, per-direction Y_diag
+  int cbfused;                 // C B^T computed in the scan kernel (kModeCbFused)
   int Bsz, L, H, G, K;
   int nseg, seg_blocks;  // each (b, h) sequence is walked as nseg segments of seg_blocks blocks
   int items;             // Bsz * H * nseg work items, handed out one at a time
+  DivU dv_nseg, dv_h, dv_hpg;  // division by nseg, H and H / G
   int *item_counter;     // next unclaimed work item (zeroed by the C B^T kernel)
   int agg;               // aggregate pass: forward state of each segment from zero, nothing else
   int need_s;            // the state after a block is used (outputs, next block, aggregate); if not
@@ -452,11 +481,11 @@ __device__ __forceinline__ Item item_unpack(const TcParams &p, int b, int h, int
 
 __device__ __forceinline__ Item item_at(const TcParams &p, int it) {
   Item r;
-  r.seg = it % p.nseg;
-  const int bh = it / p.nseg;
-  r.b = bh / p.H;
-  r.h = bh % p.H;
-  r.g = r.h / (p.H / p.G);
+  const int bh = divu(it, p.dv_nseg);
+  r.seg = it - bh * p.nseg;
+  r.b = divu(bh, p.dv_h);
+  r.h = bh - r.b * p.H;
+  r.g = divu(r.h, p.dv_hpg);
   r.k0 = r.seg * p.seg_blocks;
   r.nk = min(p.K - r.k0, p.seg_blocks);
   return r;
@@ -476,7 +505,11 @@ __device__ __forceinline__ uint32_t part(int j) { return (static_cast<uint32_t>(
 
 // Kernel instances: the call's mode is a template parameter (bits kModeAgg,
 // kModeAll, kModeNeedS), so each instance carries only the code its mode runs.
-enum : int { kModeAgg = 1, kModeAll = 2, kModeNeedS = 4 };
+enum : int { kModeAgg = 1, kModeAll = 2, kModeNeedS = 4, kModeCbFused = 8 };
+// kModeCbFused (one-block items without a state chain, no more items than
+// SMs: the batch-1 denoising step): no C B^T pre-pass; each step loads B and C
+// of both directions and computes its own C B^T tiles (one M = 64 MMA chain
+// over [B_cf; B_cr] x [C_cf; C_cr]), so a layer's step is one launch.
 
 __device__ __forceinline__ int lds_s32(uint32_t addr) {
   int v;
@@ -503,11 +536,10 @@ __device__ __forceinline__ int claim_item(const TcParams &p, int nth, bool &wait
 }
 // Publish item `it` (-1: none) as this CTA's m-th, as its coordinates
 // {b, h, g, seg} (the barrier arrival releases the write).
-__device__ __forceinline__ void publish_item(const TcParams &p, const Ctl &c, uint32_t base, int m, int it) {
+__device__ __forceinline__ void publish_item(const Ctl &c, uint32_t base, int m, int it, const Item &I) {
   const int e = m & (kItemRing - 1);
   const uint32_t a = base + kOffItemQ + 16 * e;
   if (it >= 0) {
-    const Item I = item_at(p, it);
     asm volatile("st.shared.v4.s32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(I.b), "r"(I.h), "r"(I.g), "r"(I.seg)
                  : "memory");
   } else {
@@ -537,34 +569,45 @@ __device__ __forceinline__ int item_warp(const TcParams &p, const Ctl &c, uint32
 // ---------------------------------------------------------------- producer
 template <int kM>
 __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
-  constexpr bool kAgg = kM & kModeAgg, kAll = kM & kModeAll;
+  constexpr bool kAgg = kM & kModeAgg, kAll = kM & kModeAll, kCbF = kM & kModeCbFused;
   const int nact = p.active[0] + p.active[1] + p.active[2] + p.active[3];
   // x of each active direction, C B^T tiles, B of the clean forward direction
-  // (only when S is formed), C of the clean (and noisy) forward direction
-  const uint32_t bytes = kAgg ? 3 * kTile : nact * (kTile + 2048) + (2 + (kAll ? 4 : 2)) * kTile;
+  // (only when S is formed), C of the clean (and noisy) forward direction;
+  // with the C B^T tiles computed here: x of both directions, B and C of both
+  const uint32_t bytes = kCbF ? 10 * kTile
+                              : kAgg ? 3 * kTile : nact * (kTile + 2048) + (2 + (kAll ? 4 : 2)) * kTile;
 #pragma unroll
   for (int i = 0; i < 4; ++i)
     if (p.active[i]) tma_prefetch_desc(&p.tx[i]);
   tma_prefetch_desc(&p.tbcf);
   tma_prefetch_desc(&p.tccf);
   if (kAll) tma_prefetch_desc(&p.tcnf);
-  tma_prefetch_desc(&p.tcb);
+  if (kCbF) {
+    tma_prefetch_desc(&p.tbcr);
+    tma_prefetch_desc(&p.tccr);
+  } else {
+    tma_prefetch_desc(&p.tcb);
+  }
   int last[kSlots] = {-1, -1, -1};
   int j = 0;
   bool ok = true;
   // items m and m + 1 are published when item m starts (nothing after a -1);
   // claiming further ahead would hold items back from CTAs that run dry at
   // the end of the pass
-  bool waited = false;  // past the wait for the preceding grid
+  bool waited = kCbF;  // past the wait for the preceding grid (done by every thread in that instance)
   int nclaim = 0;
+  // each claimed item is decomposed once, when it is published
   int cur = claim_item(p, nclaim++, waited), nxt = -1;
-  publish_item(p, c, base, 0, cur);
+  Item Icur{}, Inxt{};
+  if (cur >= 0) Icur = item_at(p, cur);
+  publish_item(c, base, 0, cur, Icur);
   if (cur >= 0) {
     nxt = claim_item(p, nclaim++, waited);
-    publish_item(p, c, base, 1, nxt);
+    if (nxt >= 0) Inxt = item_at(p, nxt);
+    publish_item(c, base, 1, nxt, Inxt);
   }
   for (int m = 0; ok && cur >= 0; ++m) {
-    const Item I = item_at(p, cur);
+    const Item I = Icur;
     for (int kk = 0; kk < I.nk; ++kk, ++j) {
       const int k = item_block<kAgg>(I.k0, I.nk, kk);  // block index in the sequence
       const int r = rslot(j);
@@ -576,28 +619,43 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
       mbar_arrive_expect_tx_s(full, bytes);
       const uint32_t st = base + r * kSlot;
       const int t0 = k * kT;
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (p.active[i]) tma_load_4d_s(st + kOffX + i * kTile, &p.tx[i], full, 0, I.h, t0, I.b);
-      tma_load_4d_s(st + kOffBcf, &p.tbcf, full, 0, I.g, t0, I.b);
-      tma_load_4d_s(st + kOffBcf + kTile, &p.tbcf, full, 64, I.g, t0, I.b);
-      if (!kAgg) {
+      if constexpr (kCbF) {
+        // x_cf, x_cr; [B_cf; B_cr] as the A operand of C B^T (n 0..63 at kOffBcf,
+        // n 64..127 at kOffCB, 64 rows each); [C_cf; C_cr] at kOffClo / kOffChi
+        tma_load_4d_s(st + kOffX, &p.tx[kCF], full, 0, I.h, t0, I.b);
+        tma_load_4d_s(st + kOffX + kCR * kTile, &p.tx[kCR], full, 0, I.h, t0, I.b);
+        tma_load_4d_s(st + kOffBcf, &p.tbcf, full, 0, I.g, t0, I.b);
+        tma_load_4d_s(st + kOffBcf + kTile, &p.tbcr, full, 0, I.g, t0, I.b);
+        tma_load_4d_s(st + kOffCB, &p.tbcf, full, 64, I.g, t0, I.b);
+        tma_load_4d_s(st + kOffCB + kTile, &p.tbcr, full, 64, I.g, t0, I.b);
         tma_load_4d_s(st + kOffClo, &p.tccf, full, 0, I.g, t0, I.b);
+        tma_load_4d_s(st + kOffClo + kTile, &p.tccr, full, 0, I.g, t0, I.b);
         tma_load_4d_s(st + kOffChi, &p.tccf, full, 64, I.g, t0, I.b);
-        if (kAll) {
-          tma_load_4d_s(st + kOffClo + kTile, &p.tcnf, full, 0, I.g, t0, I.b);
-          tma_load_4d_s(st + kOffChi + kTile, &p.tcnf, full, 64, I.g, t0, I.b);
-        }
-        // C B^T tiles: written by the pre-pass this kernel may overlap
-        if (!waited) {
-          wait_prior_grid();
-          waited = true;
-        }
+        tma_load_4d_s(st + kOffChi + kTile, &p.tccr, full, 64, I.g, t0, I.b);
+      } else {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          if (!p.active[i]) continue;
-          const int idx = ((cb_set(kAll, i) * p.Bsz + I.b) * p.K + k) * p.G + I.g;
-          tma_load_3d_s(st + kOffCB + i * 2048, &p.tcb, full, 0, 0, idx);
+        for (int i = 0; i < 4; ++i)
+          if (p.active[i]) tma_load_4d_s(st + kOffX + i * kTile, &p.tx[i], full, 0, I.h, t0, I.b);
+        tma_load_4d_s(st + kOffBcf, &p.tbcf, full, 0, I.g, t0, I.b);
+        tma_load_4d_s(st + kOffBcf + kTile, &p.tbcf, full, 64, I.g, t0, I.b);
+        if (!kAgg) {
+          tma_load_4d_s(st + kOffClo, &p.tccf, full, 0, I.g, t0, I.b);
+          tma_load_4d_s(st + kOffChi, &p.tccf, full, 64, I.g, t0, I.b);
+          if (kAll) {
+            tma_load_4d_s(st + kOffClo + kTile, &p.tcnf, full, 0, I.g, t0, I.b);
+            tma_load_4d_s(st + kOffChi + kTile, &p.tcnf, full, 64, I.g, t0, I.b);
+          }
+          // C B^T tiles: written by the pre-pass this kernel may overlap
+          if (!waited) {
+            wait_prior_grid();
+            waited = true;
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (!p.active[i]) continue;
+            const int idx = ((cb_set(kAll, i) * p.Bsz + I.b) * p.K + k) * p.G + I.g;
+            tma_load_3d_s(st + kOffCB + i * 2048, &p.tcb, full, 0, 0, idx);
+          }
         }
       }
 #pragma unroll
@@ -605,10 +663,12 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
         if (s == r) last[s] = j;
     }
     cur = nxt;
+    Icur = Inxt;
     nxt = -1;
     if (ok && cur >= 0) {
       nxt = claim_item(p, nclaim++, waited);
-      publish_item(p, c, base, m + 2, nxt);
+      if (nxt >= 0) Inxt = item_at(p, nxt);
+      publish_item(c, base, m + 2, nxt, Inxt);
     }
   }
   // no copy into this CTA's shared memory may still be in flight at exit
@@ -623,7 +683,7 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
 // Descriptors are built once; per step only their start addresses move.
 template <int kM, bool kGated>
 __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
-  constexpr bool kAgg = kM & kModeAgg, kAll = kM & kModeAll, kNeedS = kM & kModeNeedS;
+  constexpr bool kAgg = kM & kModeAgg, kAll = kM & kModeAll, kNeedS = kM & kModeNeedS, kCbF = kM & kModeCbFused;
   const uint32_t id_s = idesc_bf16(128, 64, 1, 1);  // S^T[n][p] = B^T (w o X)
   // Y_off^T[p][t] = h C^T over the stacked [C_cf; C_nf] rows (only C_cf without a noisy stream)
   const uint32_t id_yo = kAll ? idesc_bf16(64, 64, 1, 0) : idesc_bf16(64, 32, 1, 0);
@@ -635,6 +695,9 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
   const D64 dC = split64(sdesc(base + kOffClo, 16, 1024, kLayoutSw128));
   const D64 dX = split64(sdesc(base + kOffX, 0, 1024, kLayoutSw128));
   const D64 dM = split64(sdesc(base + kOffMh, kMhLbo, kMhSbo, kLayoutNone));
+  // fused C B^T: [B_cf; B_cr] K-major (64 rows s; n 0..63 at kOffBcf, 64..127 at kOffCB)
+  const D64 dBk = split64(sdesc(base + kOffBcf, 16, 1024, kLayoutSw128));
+  const uint32_t id_cb = idesc_bf16(64, 64, 0, 0);
 #define BD_OFF(bytes) (static_cast<uint32_t>((bytes) >> 4))
   int j = 0;
   bool ok = true;
@@ -647,6 +710,20 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
       const int r = rslot(j), i2 = j & 1;
       const uint32_t so = BD_OFF(static_cast<uint32_t>(r) * kSlot);  // this step's ring slot
       if (!wait1(c, bFull0 + r, parr(j))) break;
+      if constexpr (kCbF) {
+        // ---- [C B^T]: rows s of [B_cf; B_cr] against columns t of [C_cf; C_cr];
+        //      the two diagonal 32 x 32 blocks are the directions' tiles.  The
+        //      accumulator is free: its previous reader arrived on MhFull of the
+        //      previous step, which this warp waited for before that step's Y_diag.
+        tc_fence_after();
+#pragma unroll 1
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t ko = BD_OFF((ks & 3) * 32);
+          umma_bf16(tmem + kColCb, dBk + so + ko + (ks < 4 ? 0u : BD_OFF(kOffCB - kOffBcf)),
+                    dC + so + ko + (ks < 4 ? 0u : BD_OFF(2 * kTile)), id_cb, ks > 0);
+        }
+        umma_commit_s(bar_at(c, bCbFull));
+      }
       if constexpr (kAgg) {
         // ---- aggregate pass: S^T of the item accumulates over its blocks
         //      (walked last to first, w o X weighted to the item's end) in the
@@ -770,6 +847,55 @@ __device__ __forceinline__ void build_masked_decay(uint32_t base, int q, int lan
               __bfloat16_as_ushort(__float2bfloat16_rn(v - __bfloat162float(hi))));
     }
   }
+}
+
+// The same matrices in the fused-C B^T instance, from the fp32 C B^T
+// accumulator in TMEM (M = 64 layout: rows 16 q' .. 16 q' + 15 in TMEM lanes
+// 32 q' .. 32 q' + 15).  Epilogue warp q reads its own lanes: rows
+// s = 16 (q & 1) + (lane & 15) of direction slot kCF (q < 2) or kCR (q >= 2),
+// lanes 0..15 the columns t = 0..15, lanes 16..31 t = 16..31.  Warp-wide
+// (the TMEM load is .sync.aligned): every lane of every epilogue warp calls it.
+__device__ __forceinline__ void build_masked_decay_tm(uint32_t base, uint32_t tmem, int q, int lane, int jm) {
+  const int ct = jm % kTab;
+  const bool rev = q >= 2;
+  const int dq = rev ? kCR : kCF;
+  const int s = 16 * (q & 1) + (lane & 15);
+  const int th = lane & 16;
+  uint32_t r[16];
+  tmem_ld_16x32bx2_x16i<16>(tmem_addr(tmem, 32 * q, kColCb + (rev ? 32 : 0)), r);
+  const uint32_t cq = base + kOffCum + (ct * 4 + dq) * 128;
+  const float cs = lds_f32(cq + s * 4);
+  const float ds = lds_f32(base + kOffDt + (ct * 4 + dq) * 128 + s * 4);
+  const float Dq = lds_f32(base + kOffDtab + (ct * 4 + dq) * 4);
+  const uint32_t mrow = base + kOffMh + (jm & 1) * kMhBuf + dq * kMhDir;
+  float cj[16];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) ld_shared_v4f(cq + th * 4 + 16 * u, *reinterpret_cast<float(*)[4]>(&cj[4 * u]));
+  tmem_ld_wait();
+  // M^T[s][t] = C B^T[s][t] dt_s exp(cum_t - cum_s) inside the direction's
+  // causal half, and M[s][s] + D on the diagonal (the decay factor is 1 there)
+  float mv[16], dv = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int t = th + i;
+    const float cb = __uint_as_float(r[i]) * ds;
+    const bool valid = rev ? (t <= s) : (t >= s);
+    float v = cb * ex2_approx(cj[i] - cs);
+    if (t == s) {
+      v = cb + Dq;
+      dv = v;
+    }
+    mv[i] = valid ? v : 0.f;
+  }
+#pragma unroll
+  for (int h2 = 0; h2 < 2; ++h2)
+    st_shared_v4(mrow + inter_mn_off(th + 8 * h2, s, kMhSbo, kMhLbo), pack_bf16x2(mv[8 * h2], mv[8 * h2 + 1]),
+                 pack_bf16x2(mv[8 * h2 + 2], mv[8 * h2 + 3]), pack_bf16x2(mv[8 * h2 + 4], mv[8 * h2 + 5]),
+                 pack_bf16x2(mv[8 * h2 + 6], mv[8 * h2 + 7]));
+  // the diagonal's bf16 remainder, from the lane whose columns hold t = s
+  if ((lane >> 4) == (q & 1))
+    sts_u16(mrow + inter_mn_off(32 + s, s, kMhSbo, kMhLbo),
+            __bfloat16_as_ushort(__float2bfloat16_rn(dv - __bfloat162float(__float2bfloat16_rn(dv)))));
 }
 
 // ---------------------------------------------------------------- operand group
@@ -943,12 +1069,32 @@ __device__ void state_group_staged(const TcParams &p, const Ctl &c, uint32_t bas
     }
     tmem_st_wait();
   };
-  // The loads of item m + 2 are issued as soon as item m + 1 is staged, so
-  // they are in flight through a whole item (the h operand hand-over of item
-  // m + 1 included) before item m + 2 is staged.
+  // h operand rows of this thread: row n, the eight 16-byte chunks of its 64 p
+  // in the 128-byte swizzle (row address made opaque so that the chunk
+  // addresses are formed at the stores)
+  auto h_row = [&]() {
+    uint32_t row = base + kOffH + 128u * static_cast<uint32_t>(n);
+    asm volatile("" : "+r"(row));
+    return row;
+  };
   Item I;
   if (item_warp(p, c, base, 0, I) <= 0) return;
   load_h(I);
+  if (p.items <= static_cast<int>(gridDim.x)) {
+    // a single item per CTA: the state goes straight from registers to the operand
+    const uint32_t row = h_row(), sw = (row >> 7) & 7u;
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
+      const uint32_t a = row + ((static_cast<uint32_t>(cc) ^ sw) << 4);
+      store_split8(a, a + 4 * kTile, hreg + 8 * cc);
+    }
+    fence_proxy_async_smem();
+    arrive_lane0(c, bHFull);
+    return;
+  }
+  // The loads of item m + 2 are issued as soon as item m + 1 is staged, so
+  // they are in flight through a whole item (the h operand hand-over of item
+  // m + 1 included) before item m + 2 is staged.
   stage(0);
   for (int m = 0;; ++m) {
     const int rn = item_warp(p, c, base, m + 1, I);
@@ -957,9 +1103,7 @@ __device__ void state_group_staged(const TcParams &p, const Ctl &c, uint32_t bas
     // Y_off of the previous item has read the h operand
     if (m >= 1 && !waitw(c, bHCons, (m - 1) & 1)) return;
     {
-      uint32_t row = base + kOffH + 128u * static_cast<uint32_t>(n);
-      asm volatile("" : "+r"(row));
-      const uint32_t sw = (row >> 7) & 7u;
+      const uint32_t row = h_row(), sw = (row >> 7) & 7u;
       const uint32_t ta = tmem_addr(tmem, 32 * q, kColS0 + 64 * (m & 1));
 #pragma unroll
       for (int cq = 0; cq < 4; ++cq) {
@@ -1153,14 +1297,16 @@ __device__ __noinline__ void store_y_bf16(__nv_bfloat16 *dst, int64_t tstride, c
 
 // ---------------------------------------------------------------- epilogue
 // warps 12..15: thread owns column p = 16 q + (lane & 15) of the clean
-// (lane < 16) or noisy (lane >= 16) stream's outputs y[t][p], t = 0..31:
+// (lane < 16) or noisy (lane >= 16) stream's outputs y[t][p], t = 0..31
+// (all-block pass; with a single stream, lanes < 16 own tokens 0..15 and
+// lanes >= 16 tokens 16..31 of the clean stream's column p):
 // y = exp(cum_t) Y_off + Y_diag (Y_diag already holds both directions' D x).
 // After the outputs of step j the group builds, two steps ahead, the
 // masked-decay matrices of step j + 2 with D on the diagonal (warp q:
 // direction slot q, row s = lane of M^T) and the diagonal's bf16 remainders.
 template <int kM, bool kGated>
 __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
-  constexpr bool kAgg = kM & kModeAgg, kAll = kM & kModeAll, kNeedS = kM & kModeNeedS;
+  constexpr bool kAgg = kM & kModeAgg, kAll = kM & kModeAll, kNeedS = kM & kModeNeedS, kCbF = kM & kModeCbFused;
   const int lane = threadIdx.x & 31;
   const int q = (threadIdx.x >> 5) & 3;
   const int pcol = 16 * q + (lane & 15);
@@ -1186,8 +1332,15 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
       mend = true;
       return true;
     }
-    if (!waitw(c, bFull0 + rslot(jm), parr(jm))) return false;  // C B^T tiles
-    build_masked_decay(base, q, lane, jm, act, rev);
+    if constexpr (kCbF) {
+      if (!waitw(c, bCbFull, static_cast<uint32_t>(jm) & 1u)) return false;  // C B^T in TMEM
+      tc_fence_after();
+      build_masked_decay_tm(base, tmem, q, lane, jm);
+      tc_fence_before();  // the accumulator's next writer waits for this warp's arrival
+    } else {
+      if (!waitw(c, bFull0 + rslot(jm), parr(jm))) return false;  // C B^T tiles
+      build_masked_decay(base, q, lane, jm, act, rev);
+    }
     fence_proxy_async_smem();
     arrive_lane0(c, bMhFull0 + (jm & 1));
     ++mla;
@@ -1204,77 +1357,141 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
       if (!waitw(c, bAux0 + ct, part(j))) return;
       if (!waitw(c, bYFull0 + yb, ypar(kGated, j))) return;
       tc_fence_after();
-      uint32_t yo[32], yd[32];
-      const uint32_t ta = tmem_addr(tmem, 32 * q, kColY0 + kColYBuf * yb);
-      tmem_ld_16x32bx2_x32<32>(ta, yo);       // Y_off: clean columns 0.., noisy 32..
-      tmem_ld_16x32bx2_x32<64>(ta + 64, yd);  // Y_diag: clean 64.., noisy 128..
-      tmem_ld_wait();
-      const uint32_t eq = cumt + (ct * 4 + fs) * 128;
+      if constexpr (!kAll) {
+        // one stream: lanes 0..15 take tokens 0..15 of column p, lanes 16..31
+        // tokens 16..31 (16x32bx2 loads, the second half 16 columns on)
+        const int th = lane & 16;
+        uint32_t yo[16], yd[16];
+        const uint32_t ta = tmem_addr(tmem, 32 * q, kColY0 + kColYBuf * yb);
+        tmem_ld_16x32bx2_x16i<16>(ta, yo);       // Y_off
+        tmem_ld_16x32bx2_x16i<16>(ta + 64, yd);  // Y_diag
+        tmem_ld_wait();
+        const uint32_t eq = cumt + (ct * 4 + kCF) * 128 + 4 * th;
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
-        float c4[4];
-        ld_shared_v4f(eq + 16 * jj, c4);
+        for (int jj = 0; jj < 4; ++jj) {
+          float c4[4];
+          ld_shared_v4f(eq + 16 * jj, c4);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          yo[4 * jj + i] = __float_as_uint(
-              fmaf(ex2_approx(c4[i]), __uint_as_float(yo[4 * jj + i]), __uint_as_float(yd[4 * jj + i])));
-      }
-      tmem_ld_16x32bx2_x32<64>(ta + 96, yd);  // the diagonal remainders: clean 96.., noisy 160..
-      tmem_ld_wait();
-#pragma unroll
-      for (int t = 0; t < 32; ++t) yo[t] = __float_as_uint(__uint_as_float(yo[t]) + __uint_as_float(yd[t]));
-      // gated: yo is the forward direction's output; the reverse direction's
-      // own [Y_diag | remainder] goes to yd.  The TMEM loads are warp-wide
-      // (.sync.aligned), so they run whenever either stream has a reverse
-      // direction (uniform across the warp); a lane uses them only if its own
-      // stream has one.
-      const bool rev_act = kGated && pick4(p.active, fs | 2);
-      if (kGated && (p.active[kCR] || p.active[kNR])) {
-        tmem_ld_16x32bx2_x32<64>(ta + 64 + kColRevGated, yd);
+          for (int i = 0; i < 4; ++i)
+            yo[4 * jj + i] = __float_as_uint(
+                fmaf(ex2_approx(c4[i]), __uint_as_float(yo[4 * jj + i]), __uint_as_float(yd[4 * jj + i])));
+        }
+        tmem_ld_16x32bx2_x16i<16>(ta + 96, yd);  // the diagonal remainders
         tmem_ld_wait();
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
+        for (int t = 0; t < 16; ++t) yo[t] = __float_as_uint(__uint_as_float(yo[t]) + __uint_as_float(yd[t]));
+        // gated: the reverse direction's own [Y_diag | remainder] (warp-uniform condition)
+        const bool rev_act = kGated && p.active[kCR];
+        if (rev_act) {
+          tmem_ld_16x32bx2_x16i<16>(ta + 64 + kColRevGated, yd);
           uint32_t r16[16];
-          tmem_ld_16x32bx2_x16i<64>(ta + 96 + kColRevGated + 16 * hh, r16);
+          tmem_ld_16x32bx2_x16i<16>(ta + 96 + kColRevGated, r16);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            yd[16 * hh + i] = __float_as_uint(__uint_as_float(yd[16 * hh + i]) + __uint_as_float(r16[i]));
+          for (int i = 0; i < 16; ++i) yd[i] = __float_as_uint(__uint_as_float(yd[i]) + __uint_as_float(r16[i]));
         }
-      }
-      // the Y buffer may be reused from here on
-      tc_fence_before();
-      arrive_lane0(c, bYEmpty0 + yb);
-      if (kGated && mine) {
-        // y = y_fwd silu(z_fwd) + y_rev silu(z_rev) (a direction without z is not gated)
-        const int64_t zi = ((static_cast<int64_t>(I.b) * L + k * kT) * H + I.h) * kP + pcol;
-        const __nv_bfloat16 *zf = pick4(p.z, fs), *zr = rev_act ? pick4(p.z, fs | 2) : nullptr;
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          float v = __uint_as_float(yo[t]);
-          if (zf) v *= silu_approx(__bfloat162float(zf[zi + t * H * kP]));
-          if (rev_act) {
-            const float u = __uint_as_float(yd[t]);
-            v += zr ? u * silu_approx(__bfloat162float(zr[zi + t * H * kP])) : u;
-          }
-          yo[t] = __float_as_uint(v);
-        }
-      }
-      if (mine) {
-        const int64_t yi = ((static_cast<int64_t>(I.b) * L + k * kT) * H + I.h) * kP + pcol;
+        // the Y buffer may be reused from here on
+        tc_fence_before();
+        arrive_lane0(c, bYEmpty0 + yb);
         const int64_t tstride = H * kP;
-        if (p.out_bf16) {
-          __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(yout) + yi;
-          if constexpr (kNeedS) {
-            store_y_bf16(dst, tstride, yo);
-          } else {
+        const int64_t yi = ((static_cast<int64_t>(I.b) * L + k * kT + th) * H + I.h) * kP + pcol;
+        if (kGated) {
+          const __nv_bfloat16 *zf = p.z[kCF], *zr = rev_act ? p.z[kCR] : nullptr;
 #pragma unroll
-            for (int t = 0; t < 32; ++t) dst[t * tstride] = __float2bfloat16_rn(__uint_as_float(yo[t]));
+          for (int t = 0; t < 16; ++t) {
+            float v = __uint_as_float(yo[t]);
+            if (zf) v *= silu_approx(__bfloat162float(zf[yi + t * tstride]));
+            if (rev_act) {
+              const float u = __uint_as_float(yd[t]);
+              v += zr ? u * silu_approx(__bfloat162float(zr[yi + t * tstride])) : u;
+            }
+            yo[t] = __float_as_uint(v);
           }
-        } else {
-          float *dst = reinterpret_cast<float *>(yout) + yi;
+        }
+        if (p.y_clean) {
+          if (p.out_bf16) {
+            __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(p.y_clean) + yi;
 #pragma unroll
-          for (int t = 0; t < 32; ++t) dst[t * tstride] = __uint_as_float(yo[t]);
+            for (int t = 0; t < 16; ++t) dst[t * tstride] = __float2bfloat16_rn(__uint_as_float(yo[t]));
+          } else {
+            float *dst = reinterpret_cast<float *>(p.y_clean) + yi;
+#pragma unroll
+            for (int t = 0; t < 16; ++t) dst[t * tstride] = __uint_as_float(yo[t]);
+          }
+        }
+      } else {
+        uint32_t yo[32], yd[32];
+        const uint32_t ta = tmem_addr(tmem, 32 * q, kColY0 + kColYBuf * yb);
+        tmem_ld_16x32bx2_x32<32>(ta, yo);       // Y_off: clean columns 0.., noisy 32..
+        tmem_ld_16x32bx2_x32<64>(ta + 64, yd);  // Y_diag: clean 64.., noisy 128..
+        tmem_ld_wait();
+        const uint32_t eq = cumt + (ct * 4 + fs) * 128;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          float c4[4];
+          ld_shared_v4f(eq + 16 * jj, c4);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            yo[4 * jj + i] = __float_as_uint(
+                fmaf(ex2_approx(c4[i]), __uint_as_float(yo[4 * jj + i]), __uint_as_float(yd[4 * jj + i])));
+        }
+        tmem_ld_16x32bx2_x32<64>(ta + 96, yd);  // the diagonal remainders: clean 96.., noisy 160..
+        tmem_ld_wait();
+#pragma unroll
+        for (int t = 0; t < 32; ++t) yo[t] = __float_as_uint(__uint_as_float(yo[t]) + __uint_as_float(yd[t]));
+        // gated: yo is the forward direction's output; the reverse direction's
+        // own [Y_diag | remainder] goes to yd.  The TMEM loads are warp-wide
+        // (.sync.aligned), so they run whenever either stream has a reverse
+        // direction (uniform across the warp); a lane uses them only if its own
+        // stream has one.
+        const bool rev_act = kGated && pick4(p.active, fs | 2);
+        if (kGated && (p.active[kCR] || p.active[kNR])) {
+          tmem_ld_16x32bx2_x32<64>(ta + 64 + kColRevGated, yd);
+          tmem_ld_wait();
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t r16[16];
+            tmem_ld_16x32bx2_x16i<64>(ta + 96 + kColRevGated + 16 * hh, r16);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              yd[16 * hh + i] = __float_as_uint(__uint_as_float(yd[16 * hh + i]) + __uint_as_float(r16[i]));
+          }
+        }
+        // the Y buffer may be reused from here on
+        tc_fence_before();
+        arrive_lane0(c, bYEmpty0 + yb);
+        if (kGated && mine) {
+          // y = y_fwd silu(z_fwd) + y_rev silu(z_rev) (a direction without z is not gated)
+          const int64_t zi = ((static_cast<int64_t>(I.b) * L + k * kT) * H + I.h) * kP + pcol;
+          const __nv_bfloat16 *zf = pick4(p.z, fs), *zr = rev_act ? pick4(p.z, fs | 2) : nullptr;
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            float v = __uint_as_float(yo[t]);
+            if (zf) v *= silu_approx(__bfloat162float(zf[zi + t * H * kP]));
+            if (rev_act) {
+              const float u = __uint_as_float(yd[t]);
+              v += zr ? u * silu_approx(__bfloat162float(zr[zi + t * H * kP])) : u;
+            }
+            yo[t] = __float_as_uint(v);
+          }
+        }
+        if (mine) {
+          const int64_t yi = ((static_cast<int64_t>(I.b) * L + k * kT) * H + I.h) * kP + pcol;
+          const int64_t tstride = H * kP;
+          if (p.out_bf16) {
+            __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(yout) + yi;
+            if constexpr (kNeedS) {
+              store_y_bf16(dst, tstride, yo);
+            } else {
+#pragma unroll
+              for (int t = 0; t < 32; ++t) dst[t * tstride] = __float2bfloat16_rn(__uint_as_float(yo[t]));
+            }
+          } else {
+            float *dst = reinterpret_cast<float *>(yout) + yi;
+#pragma unroll
+            for (int t = 0; t < 32; ++t) dst[t * tstride] = __uint_as_float(yo[t]);
+          }
         }
       }
       if (!build_m()) return;  // step j + 2
@@ -1306,7 +1523,7 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
     for (int i = 0; i < bCount; ++i) {
       uint32_t cnt = 4;
       if (i == bFull0 || i == bFull1 || i == bFull2 || i == bSFull0 || i == bSFull1 || i == bYFull0 ||
-          i == bYFull1 || i == bHCons || i == bDrain || i >= bItem0)
+          i == bYFull1 || i == bHCons || i == bDrain || i == bCbFull || i >= bItem0)
         cnt = 1;
       else if (i == bEmpty0 || i == bEmpty1 || i == bEmpty2)
         cnt = 5;
@@ -1334,11 +1551,29 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   Ctl c{smem_u32(bars), base + kOffMisc};
+  if constexpr ((kM & kModeCbFused) != 0) {
+    // No pre-pass precedes this instance: every thread waits for the previous
+    // kernel on the stream before its first read, and one thread clears the
+    // status word (a CTA can raise it only after a wait that ran out its limit).
+    // The tensor maps are kernel parameters, not the previous kernel's output:
+    // their fetch overlaps the wait.
+    if (threadIdx.x == 0) {
+      tma_prefetch_desc(&p.tx[kCF]);
+      tma_prefetch_desc(&p.tx[kCR]);
+      tma_prefetch_desc(&p.tbcf);
+      tma_prefetch_desc(&p.tbcr);
+      tma_prefetch_desc(&p.tccf);
+      tma_prefetch_desc(&p.tccr);
+    }
+    wait_prior_grid();
+    if (blockIdx.x == 0 && threadIdx.x == 0) *p.status = 0;
+  }
   // Launched as a programmatic dependent of the previous kernel on the stream
   // (the C B^T pre-pass, or the segment combine): the threads that read what it
   // wrote -- the producer (work counter, C B^T tiles) and the state warps
   // (segment initial states) -- wait for its completion (griddepcontrol.wait)
-  // just before those reads; everything else overlaps its tail.
+  // just before those reads; everything else overlaps its tail.  The
+  // fused-C B^T instance waited above, before any role starts.
 
   if (warp == 0) {
     if ((threadIdx.x & 31) == 0) producer<kM>(p, c, base);
@@ -1435,7 +1670,8 @@ cudaError_t launch_instance(const cudaLaunchConfig_t &cfg, const TcParams &p) {
 // the previous kernel in the stream; it waits for that kernel before reading),
 // in the instance of the call's mode: the aggregate pass, the all-block pass,
 // a scan with a state chain (per-block or final state), or one-block items
-// without one; each but the first with or without a gate.
+// without one (with the C B^T tiles from the pre-pass or computed in the
+// kernel); each but the first with or without a gate.
 cudaError_t launch_scan(unsigned grid, cudaStream_t stream, const TcParams &p) {
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
@@ -1456,6 +1692,8 @@ cudaError_t launch_scan(unsigned grid, cudaStream_t stream, const TcParams &p) {
                 : launch_instance<kModeAll | kModeNeedS, false>(cfg, p);
   else if (p.need_s)
     e = p.gated ? launch_instance<kModeNeedS, true>(cfg, p) : launch_instance<kModeNeedS, false>(cfg, p);
+  else if (p.cbfused)
+    e = p.gated ? launch_instance<kModeCbFused, true>(cfg, p) : launch_instance<kModeCbFused, false>(cfg, p);
   else
     e = p.gated ? launch_instance<0, true>(cfg, p) : launch_instance<0, false>(cfg, p);
   return e != cudaSuccess ? e : cudaGetLastError();
@@ -1529,6 +1767,16 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
   __nv_bfloat16 *cbws = reinterpret_cast<__nv_bfloat16 *>(static_cast<uint8_t *>(a.ws) + kWsHeader);
   const unsigned long long timeout = opt_wait_timeout_ns();
   const int K = static_cast<int>(a.L / kT);
+  int dev = 0, nsm = 0;
+  cudaError_t e;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  // One-block items without a state chain, both clean directions, no more
+  // items than SMs (small-batch denoising steps): the scan kernel computes
+  // the C B^T tiles itself and the call is one launch.
+  const bool cbfused = !all && a.has_cr && K == 1 && !a.states && !a.final_state && a.Bsz * a.H <= nsm &&
+                       tc_plan_segments(a.Bsz, a.H, K) == 1 && !opt_cb_prepass();
 
   // ---- C B^T of every active direction
   CbParams cp;
@@ -1551,11 +1799,11 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
   cp.item_counters = counters;
   cp.status = a.status;
   cp.timeout_ns = timeout;
-  cudaError_t e = cudaFuncSetAttribute(bd_cb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kCbSmem));
-  if (e != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(bd_cb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kCbSmem))) != cudaSuccess)
+    return e;
   dim3 cgrid((K + 3) / 4, static_cast<unsigned>(a.Bsz * a.G), nz);
-  {
+  if (!cbfused) {
     // programmatic dependent launch: its CTAs may be scheduled while the
     // previous kernel finishes; they wait for it before touching memory
     cudaLaunchConfig_t cfg;
@@ -1591,6 +1839,10 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
       !make_map_cb(&p.tcb, cbws, static_cast<uint64_t>(cb_sets(all)) * a.Bsz * K * a.G))
     return cudaErrorInvalidValue;
   if (all && !make_map_bf16(&p.tcnf, a.nf.C, kN, a.G, a.L, a.Bsz)) return cudaErrorInvalidValue;
+  if (cbfused && (!make_map_bf16(&p.tbcr, a.cr.B, kN, a.G, a.L, a.Bsz) ||
+                  !make_map_bf16(&p.tccr, a.cr.C, kN, a.G, a.L, a.Bsz)))
+    return cudaErrorInvalidValue;
+  p.cbfused = cbfused ? 1 : 0;
   p.Bsz = static_cast<int>(a.Bsz);
   p.L = static_cast<int>(a.L);
   p.H = static_cast<int>(a.H);
@@ -1600,6 +1852,9 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
   p.nseg = nseg;
   p.seg_blocks = (K + nseg - 1) / nseg;
   p.items = static_cast<int>(a.Bsz * a.H * nseg);
+  p.dv_nseg = make_divu(nseg);
+  p.dv_h = make_divu(static_cast<int>(a.H));
+  p.dv_hpg = make_divu(static_cast<int>(a.H / a.G));
   p.item_counter = counters + 1;
   p.allblock = all ? 1 : 0;
   p.need_s = (a.states || a.final_state || p.seg_blocks > 1 || nseg > 1) ? 1 : 0;
@@ -1613,10 +1868,6 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
   p.timeout_ns = timeout;
   p.drain_ns = 1000000000ull;
   // persistent CTAs, one per SM, each walking its share of the work items
-  int dev = 0, nsm = 0;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
-      (e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-    return e;
   const unsigned grid = static_cast<unsigned>(p.items < nsm ? p.items : nsm);
   if (nseg > 1) {
     // aggregate pass (clean forward state of every segment from zero), then

@@ -318,6 +318,12 @@ int bdscan_version(void);
  *                               (default 0; env BDSCAN_FORCE_GENERIC=1)
  *   BDSCAN_OPT_VERBOSE          1: launch failures are printed to stderr
  *                               (default 0; env BDSCAN_VERBOSE=1)
+ *   BDSCAN_OPT_CB_PREPASS       1: small-batch block steps (no state out, at
+ *                               most one (sequence, head) per SM) also take the
+ *                               separate C B^T pre-pass instead of computing
+ *                               C B^T inside the scan kernel (default 0; env
+ *                               BDSCAN_CB_PREPASS=1).  Same results up to the
+ *                               bf16 rounding of the C B^T tiles.
  * bdscan_set_option returns the previous value, or BDSCAN_ERR_INVALID_ARG for
  * an unknown option or a value out of range; a change applies to calls made
  * after it returns.  bdscan_get_option returns the current value (or
@@ -325,6 +331,7 @@ int bdscan_version(void);
 #define BDSCAN_OPT_WAIT_TIMEOUT_NS 0
 #define BDSCAN_OPT_FORCE_GENERIC 1
 #define BDSCAN_OPT_VERBOSE 2
+#define BDSCAN_OPT_CB_PREPASS 3
 long long bdscan_set_option(int option, long long value);
 long long bdscan_get_option(int option);
 

@@ -295,3 +295,27 @@ def test_binding_checks_caller_outputs():
     grads[2]["B"] = torch.empty((1, 64, 1, 64))
     with pytest.raises(ValueError):
         bd.allblock_backward(s, cf, cr, nf, nr, sts, yn, grads=grads)
+
+
+def test_options_set_get_restore():
+    """Process-wide options: set returns the previous value, get the current
+    one, out-of-range values and unknown options are rejected, the context
+    manager restores the old value (host-side only: no GPU needed)."""
+    for opt in (bd.BDSCAN_OPT_FORCE_GENERIC, bd.BDSCAN_OPT_VERBOSE, bd.BDSCAN_OPT_CB_PREPASS):
+        old = bd.bdscan_get_option(opt)
+        assert old in (0, 1)
+        assert bd.bdscan_set_option(opt, 1) == old
+        assert bd.bdscan_get_option(opt) == 1
+        assert bd.bdscan_set_option(opt, 2) == -1  # BDSCAN_ERR_INVALID_ARG, value unchanged
+        assert bd.bdscan_get_option(opt) == 1
+        assert bd.bdscan_set_option(opt, old) == 1
+        with bd.option(opt, 1 - old):
+            assert bd.bdscan_get_option(opt) == 1 - old
+        assert bd.bdscan_get_option(opt) == old
+    t0 = bd.bdscan_get_option(bd.BDSCAN_OPT_WAIT_TIMEOUT_NS)
+    assert t0 > 0
+    with bd.option(bd.BDSCAN_OPT_WAIT_TIMEOUT_NS, 12345):
+        assert bd.bdscan_get_option(bd.BDSCAN_OPT_WAIT_TIMEOUT_NS) == 12345
+    assert bd.bdscan_get_option(bd.BDSCAN_OPT_WAIT_TIMEOUT_NS) == t0
+    assert bd.bdscan_get_option(99) == -1
+    assert bd.bdscan_set_option(99, 0) == -1

@@ -86,6 +86,44 @@ def test_block_step_parity(name, commit):
         check_states(so, rso, "state_out")
 
 
+@pytest.mark.parametrize("name", ["bf16_multi", "bf16_out_bf16", "g1_h8"])
+def test_block_step_cb_in_kernel_and_prepass(name):
+    """Small-batch steps without a state out compute C B^T inside the scan
+    kernel (one launch); with BDSCAN_OPT_CB_PREPASS they take the pre-pass.
+    Both against the oracle, and against each other within the bf16 rounding
+    of the pre-pass's C B^T tiles."""
+    s = SMALL[name].with_(seqlen=32, chunk_len=32)
+    f, r = W.make_streams(s, 15, streams=(W.CLEAN_FWD, W.CLEAN_REV), device=DEV)
+    state = W.make_state(s, 15, device=DEV, scale=2.0)
+    ry, _ = oracle.block_step(s.as_dict(), f, r, state)
+    y, _ = bd.block_step(s, f, r, state)
+    with bd.option(bd.BDSCAN_OPT_CB_PREPASS, 1):
+        y2, _ = bd.block_step(s, f, r, state)
+    torch.cuda.synchronize()
+    bf = s.out_dtype == "bf16"
+    check_y(y, ry, bf16_out=bf, what="C B^T in the scan kernel")
+    check_y(y2, ry, bf16_out=bf, what="C B^T pre-pass")
+    if not bf:  # two bf16-rounded results may sit a whole bf16 ulp apart
+        check_y(y, y2.double().cpu().numpy(), what="in-kernel vs pre-pass")
+
+
+def test_block_step_cb_in_kernel_timeout_reports_status():
+    """The one-launch step (no pre-pass clears the status word there) reports
+    a run-out wait through the status word too, and the next call is clean."""
+    s = _shape(batch=1, seqlen=32, chunk_len=32)
+    f, r = W.make_streams(s, 16, streams=(W.CLEAN_FWD, W.CLEAN_REV), device=DEV)
+    state = W.make_state(s, 16, device=DEV)
+    ws = bd.workspace(s, bd.BDSCAN_OP_BLOCK_STEP, DEV)
+    stream = torch.cuda.current_stream().cuda_stream
+    with bd.option(bd.BDSCAN_OPT_WAIT_TIMEOUT_NS, 0):
+        bd.block_step(s, f, r, state, ws=ws)
+    assert bd.bdscan_check_status(ws.data_ptr(), stream) == -6
+    y, _ = bd.block_step(s, f, r, state, ws=ws)
+    assert bd.bdscan_check_status(ws.data_ptr(), stream) == 0
+    ry, _ = oracle.block_step(s.as_dict(), f, r, state)
+    check_y(y, ry)
+
+
 def test_no_reverse_and_gated():
     s = _shape()
     f = W.make_dir(s, 4, 0, W.CLEAN_FWD, DEV, gated=True)
