@@ -849,20 +849,16 @@ __device__ __forceinline__ void build_masked_decay(uint32_t base, int q, int lan
   }
 }
 
-// The same matrices in the fused-C B^T instance, from the fp32 C B^T
-// accumulator in TMEM (M = 64 layout: rows 16 q' .. 16 q' + 15 in TMEM lanes
-// 32 q' .. 32 q' + 15).  Epilogue warp q reads its own lanes: rows
-// s = 16 (q & 1) + (lane & 15) of direction slot kCF (q < 2) or kCR (q >= 2),
-// lanes 0..15 the columns t = 0..15, lanes 16..31 t = 16..31.  Warp-wide
-// (the TMEM load is .sync.aligned): every lane of every epilogue warp calls it.
-__device__ __forceinline__ void build_masked_decay_tm(uint32_t base, uint32_t tmem, int q, int lane, int jm) {
+// The same matrices split over the four epilogue warps for one-block items
+// of one stream (fused-C B^T and pre-pass step instances): warp q builds rows s = 16 (q & 1) + (lane & 15) of direction slot
+// kCF (q < 2) or kCR (q >= 2); lanes 0..15 the columns t = 0..15, lanes 16..31
+// t = 16..31.  cbv holds C B^T[s][t] of the thread's 16 columns.
+__device__ __forceinline__ void build_rows16(uint32_t base, int q, int lane, int jm, const float (&cbv)[16]) {
   const int ct = jm % kTab;
   const bool rev = q >= 2;
   const int dq = rev ? kCR : kCF;
   const int s = 16 * (q & 1) + (lane & 15);
   const int th = lane & 16;
-  uint32_t r[16];
-  tmem_ld_16x32bx2_x16i<16>(tmem_addr(tmem, 32 * q, kColCb + (rev ? 32 : 0)), r);
   const uint32_t cq = base + kOffCum + (ct * 4 + dq) * 128;
   const float cs = lds_f32(cq + s * 4);
   const float ds = lds_f32(base + kOffDt + (ct * 4 + dq) * 128 + s * 4);
@@ -871,14 +867,13 @@ __device__ __forceinline__ void build_masked_decay_tm(uint32_t base, uint32_t tm
   float cj[16];
 #pragma unroll
   for (int u = 0; u < 4; ++u) ld_shared_v4f(cq + th * 4 + 16 * u, *reinterpret_cast<float(*)[4]>(&cj[4 * u]));
-  tmem_ld_wait();
   // M^T[s][t] = C B^T[s][t] dt_s exp(cum_t - cum_s) inside the direction's
   // causal half, and M[s][s] + D on the diagonal (the decay factor is 1 there)
   float mv[16], dv = 0.f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const int t = th + i;
-    const float cb = __uint_as_float(r[i]) * ds;
+    const float cb = cbv[i] * ds;
     const bool valid = rev ? (t <= s) : (t >= s);
     float v = cb * ex2_approx(cj[i] - cs);
     if (t == s) {
@@ -896,6 +891,33 @@ __device__ __forceinline__ void build_masked_decay_tm(uint32_t base, uint32_t tm
   if ((lane >> 4) == (q & 1))
     sts_u16(mrow + inter_mn_off(32 + s, s, kMhSbo, kMhLbo),
             __bfloat16_as_ushort(__float2bfloat16_rn(dv - __bfloat162float(__float2bfloat16_rn(dv)))));
+}
+
+// From the step's bf16 C B^T tile in its ring slot (pre-pass instances).
+__device__ __forceinline__ void build_masked_decay_split(uint32_t base, int q, int lane, int jm) {
+  const int s = 16 * (q & 1) + (lane & 15);
+  const int th = lane & 16;
+  const uint32_t cbrow = base + rslot(jm) * kSlot + kOffCB + (q >= 2 ? kCR : kCF) * 2048;
+  uint32_t r[8];
+  ld_shared_v4(cbrow + sw64_chunk(s, th >> 3), r[0], r[1], r[2], r[3]);
+  ld_shared_v4(cbrow + sw64_chunk(s, (th >> 3) + 1), r[4], r[5], r[6], r[7]);
+  float cbv[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) cbv[i] = (i & 1) ? bf16_hi_f(r[i >> 1]) : bf16_lo_f(r[i >> 1]);
+  build_rows16(base, q, lane, jm, cbv);
+}
+
+// From the fp32 C B^T accumulator in TMEM (fused-C B^T instance; M = 64
+// layout: rows 16 q' .. 16 q' + 15 in TMEM lanes 32 q' .. 32 q' + 15, so warp q
+// reads exactly its rows).  Warp-wide: every lane of every epilogue warp calls it.
+__device__ __forceinline__ void build_masked_decay_tm(uint32_t base, uint32_t tmem, int q, int lane, int jm) {
+  uint32_t r[16];
+  tmem_ld_16x32bx2_x16i<16>(tmem_addr(tmem, 32 * q, kColCb + (q >= 2 ? 32 : 0)), r);
+  tmem_ld_wait();
+  float cbv[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) cbv[i] = __uint_as_float(r[i]);
+  build_rows16(base, q, lane, jm, cbv);
 }
 
 // ---------------------------------------------------------------- operand group
@@ -1339,7 +1361,14 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
       tc_fence_before();  // the accumulator's next writer waits for this warp's arrival
     } else {
       if (!waitw(c, bFull0 + rslot(jm), parr(jm))) return false;  // C B^T tiles
-      build_masked_decay(base, q, lane, jm, act, rev);
+      // one-block items without a state chain: the four-warp split (the
+      // epilogue is that pipeline's co-bottleneck); otherwise one warp per
+      // direction, which keeps warp 13 (the MMA issuer's sub-partition) idle
+      // in the issue-bound state-chain instances
+      if constexpr (kAll || kNeedS)
+        build_masked_decay(base, q, lane, jm, act, rev);
+      else if (q < 2 || p.active[kCR])
+        build_masked_decay_split(base, q, lane, jm);
     }
     fence_proxy_async_smem();
     arrive_lane0(c, bMhFull0 + (jm & 1));
