@@ -454,11 +454,14 @@ def run_only(args):
     print(json.dumps({"extra": run_extra(dev, peaks(), only=args.only)}), flush=True)
 
 
-def _step_stack(s: W.Shape, layers: int, dev, pk, conv_width: int = 0, norm: bool = False) -> dict:
-    """With ``conv_width``, every layer first runs the short convolution of both
-    directions from its cached conv state (writing the scan's x, B, C), then the
-    scan step; with ``norm``, the gated RMSNorm of the summed output follows
-    (bf16): the selective-scan core of a Mamba layer's denoising step."""
+def _step_stack(s: W.Shape, layers: int, dev, pk, conv_width: int = 0, norm: bool = False,
+                two_calls: bool = False) -> dict:
+    """With ``conv_width``, every layer's step starts with the short convolution
+    of both directions from its cached conv state: one bdscan_conv_block_step
+    call (convolution and scan step in one launch where the shape allows), or
+    with ``two_calls`` bdscan_conv_prefix into the scan's x, B, C and then
+    bdscan_block_step; with ``norm``, the gated RMSNorm of the summed output
+    follows (bf16): the selective-scan core of a Mamba layer's denoising step."""
     seed = W.SEEDS["700m_step" if s.nheads == 48 else "3b_step_b1"]
     ins = [W.make_streams(s, seed, layer, device=dev, streams=(W.CLEAN_FWD, W.CLEAN_REV))
            for layer in range(layers)]
@@ -471,6 +474,7 @@ def _step_stack(s: W.Shape, layers: int, dev, pk, conv_width: int = 0, norm: boo
         cstates = [W.make_conv_state(s, conv_width, seed, layer, device=dev) for layer in range(layers)]
         # the convolution writes straight into the scan's x, B, C
         couts = [[{k: ins[l][i][k] for k in bd.CONV_KEYS} for i in range(2)] for l in range(layers)]
+        cws = [bd.workspace(s, bd.BDSCAN_OP_CONV_BLOCK_STEP, dev) for _ in range(layers)]
     if norm:
         gz = torch.Generator(device=dev).manual_seed(11)
         zs = [torch.randn(ys[0].shape, generator=gz, device=dev).to(torch.bfloat16) for _ in range(layers)]
@@ -480,11 +484,15 @@ def _step_stack(s: W.Shape, layers: int, dev, pk, conv_width: int = 0, norm: boo
 
     def stack():
         for l in range(layers):
-            if conv_width:
-                bd.conv_prefix(s, conv_width, True, convs[l][0], convs[l][1], cstates[l],
-                               out_fwd=couts[l][0], out_rev=couts[l][1], stream=torch.cuda.current_stream(dev))
-            bd.block_step(s, ins[l][0], ins[l][1], states[l], y=ys[l], ws=wss[l],
-                          stream=torch.cuda.current_stream(dev))
+            if conv_width and not two_calls:
+                bd.conv_block_step(s, conv_width, True, convs[l][0], convs[l][1], cstates[l], ins[l][0], ins[l][1],
+                                   states[l], y=ys[l], ws=cws[l], stream=torch.cuda.current_stream(dev))
+            else:
+                if conv_width:
+                    bd.conv_prefix(s, conv_width, True, convs[l][0], convs[l][1], cstates[l],
+                                   out_fwd=couts[l][0], out_rev=couts[l][1], stream=torch.cuda.current_stream(dev))
+                bd.block_step(s, ins[l][0], ins[l][1], states[l], y=ys[l], ws=wss[l],
+                              stream=torch.cuda.current_stream(dev))
             if norm:
                 bd.gated_rmsnorm(s, ys[l], zs[l], nws[l], 1, 1e-5, out=nouts[l],
                                  stream=torch.cuda.current_stream(dev))

@@ -27,6 +27,7 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "bdscan.h")
 BDSCAN_BF16, BDSCAN_FP32 = 0, 1
 BDSCAN_OP_PREFIX, BDSCAN_OP_BLOCK_STEP, BDSCAN_OP_ALLBLOCK, BDSCAN_OP_ALLBLOCK_BACKWARD = 0, 1, 2, 3
 BDSCAN_OP_CONV_PREFIX, BDSCAN_OP_CONV_ALLBLOCK, BDSCAN_OP_GATED_RMSNORM = 4, 5, 6
+BDSCAN_OP_CONV_BLOCK_STEP = 7
 STATUS = {0: "BDSCAN_OK", -1: "BDSCAN_ERR_INVALID_ARG", -2: "BDSCAN_ERR_UNSUPPORTED_SHAPE",
           -3: "BDSCAN_ERR_MISALIGNED", -4: "BDSCAN_ERR_WORKSPACE", -5: "BDSCAN_ERR_CUDA",
           -6: "BDSCAN_ERR_TIMEOUT", -7: "BDSCAN_ERR_SCRATCH_LIMIT"}
@@ -83,9 +84,11 @@ def lib() -> ctypes.CDLL:
             cp, ci = ctypes.POINTER(bdscan_conv_t), ctypes.c_int
             L.bdscan_conv_prefix.argtypes = [sp, ci, ci, cp, cp, vp, vp, vp]
             L.bdscan_conv_allblock.argtypes = [sp, ci, ci, cp, cp, cp, cp, vp, vp]
+            L.bdscan_conv_block_step.argtypes = [sp, ci, ci, cp, cp, vp, dp, dp, vp, vp, vp, sz, vp]
             L.bdscan_gated_rmsnorm.argtypes = [sp, vp, vp, vp, ctypes.c_int64, ctypes.c_float, vp, vp]
             for fn in ("bdscan_prefix", "bdscan_block_step", "bdscan_allblock", "bdscan_allblock_backward",
-                       "bdscan_conv_prefix", "bdscan_conv_allblock", "bdscan_gated_rmsnorm",
+                       "bdscan_conv_prefix", "bdscan_conv_allblock", "bdscan_conv_block_step",
+                       "bdscan_gated_rmsnorm",
                        "bdscan_check_status", "bdscan_version"):
                 getattr(L, fn).restype = ctypes.c_int
             L.bdscan_workspace_size.argtypes = [sp, ctypes.c_int]
@@ -133,6 +136,12 @@ def bdscan_allblock_backward(shape, cf, cr, nf, nr, h0, block_states, dy_clean, 
                              g_cf, g_cr, g_nf, g_nr, dh0, ws, ws_bytes, stream) -> int:
     return lib().bdscan_allblock_backward(shape, cf, cr, nf, nr, h0, block_states, dy_clean, dy_noisy,
                                           dstates, g_cf, g_cr, g_nf, g_nr, dh0, ws, ws_bytes, stream)
+
+
+def bdscan_conv_block_step(shape, width, silu, conv_fwd, conv_rev, conv_state_in, fwd, rev, state_in, y, ws,
+                           ws_bytes, stream) -> int:
+    return lib().bdscan_conv_block_step(shape, width, silu, conv_fwd, conv_rev, conv_state_in, fwd, rev, state_in,
+                                        y, ws, ws_bytes, stream)
 
 
 def bdscan_conv_prefix(shape, width, silu, fwd, rev, conv_state_in, conv_state_out, stream) -> int:
@@ -467,6 +476,19 @@ def c_conv(s: Shape, d: dict | None, width: int, device, out: dict | None = None
     return st, out
 
 
+def c_dir_scan(s: Shape, d: dict, device) -> bdscan_dir_t:
+    """ctypes struct of a scan direction whose x, B, C come from elsewhere (the
+    convolution of bdscan_conv_block_step): dt, A, D and the optional z only."""
+    tin = _DT[s.in_dtype][0]
+    B, L, H, P = s.batch, s.seqlen, s.nheads, s.headdim
+    _check_tensor("dt", d["dt"], (B, L, H), tin, device)
+    if d.get("z") is not None:
+        _check_tensor("z", d["z"], (B, L, H, P), tin, device)
+    _check_tensor("A", d["A"], (H,), torch.float32, device)
+    _check_tensor("D", d["D"], (H,), torch.float32, device)
+    return bdscan_dir_t(None, _ptr(d["dt"]), None, None, _ptr(d.get("z")), _ptr(d["A"]), _ptr(d["D"]))
+
+
 def _check_conv_state(name, t, s: Shape, width: int, device):
     if t is not None:
         _check_tensor(name, t, (s.batch, width - 1, conv_channels(s)), _DT[s.in_dtype][0], device)
@@ -509,6 +531,33 @@ def conv_allblock(s: Shape, width: int, silu: bool, clean_fwd: dict, clean_rev: 
                               _ref(cd[2]), _ref(cd[3]), _ptr(state_in), _stream(dev, stream))
     _raise("bdscan_conv_allblock", rc)
     return [b[1] for b in built]
+
+
+def conv_block_step(s: Shape, width: int, silu: bool, conv_fwd: dict, conv_rev: dict, conv_state_in, fwd: dict,
+                    rev: dict, state_in, y=None, ws=None, stream=None):
+    """One denoising step of a layer's selective-scan core without commit: the
+    short convolution of both directions' x, B, C (``conv_fwd``/``conv_rev``:
+    pre-convolution inputs, weight, bias) from ``conv_state_in``, then the scan
+    step from ``state_in`` with ``fwd``/``rev``'s dt, A, D and z.  One launch
+    when the tensor-core step takes the shape.  Returns y."""
+    dev = conv_fwd["x"].device
+    cs = c_shape(s)
+    cf, _ = c_conv(s, conv_fwd, width, dev, {k: None for k in CONV_KEYS})
+    cr, _ = c_conv(s, conv_rev, width, dev, {k: None for k in CONV_KEYS})
+    _check_conv_state("conv_state_in", conv_state_in, s, width, dev)
+    sf, sr = c_dir_scan(s, fwd, dev), c_dir_scan(s, rev, dev)
+    _check_tensor("state_in", state_in, (s.batch, s.nheads, s.headdim, s.dstate), torch.float32, dev)
+    if y is None:
+        y = _out(s, dev)
+    _check_tensor("y", y, (s.batch, s.seqlen, s.nheads, s.headdim), _DT[s.out_dtype][0], dev)
+    if ws is None:
+        ws = workspace(s, BDSCAN_OP_CONV_BLOCK_STEP, dev)
+    _check_ws(ws, s, BDSCAN_OP_CONV_BLOCK_STEP, dev)
+    rc = bdscan_conv_block_step(ctypes.byref(cs), int(width), 1 if silu else 0, ctypes.byref(cf), ctypes.byref(cr),
+                                _ptr(conv_state_in), ctypes.byref(sf), ctypes.byref(sr), _ptr(state_in), _ptr(y),
+                                _ptr(ws), ws.numel(), _stream(dev, stream))
+    _raise("bdscan_conv_block_step", rc)
+    return y
 
 
 # ----------------------------------------------------------------------------- gated RMSNorm

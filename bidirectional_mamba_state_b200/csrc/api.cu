@@ -148,6 +148,15 @@ DirArgs to_args(const bdscan_dir_t *d) {
   return a;
 }
 
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// One direction's convolved x, B and C (the scan's inputs), each 256-aligned.
+size_t conv_scratch_bytes(const bdscan_shape_t *s) {
+  const size_t in = s->in_dtype == BDSCAN_BF16 ? 2 : 4;
+  const size_t BL = (size_t)s->batch * (size_t)s->seqlen;
+  return align256(BL * (size_t)(s->nheads * s->headdim) * in) + 2 * align256(BL * (size_t)(s->ngroups * s->dstate) * in);
+}
+
 ScanArgs base_args(const bdscan_shape_t *s) {
   ScanArgs a{};
   a.Bsz = s->batch; a.L = s->seqlen; a.H = s->nheads; a.P = s->headdim; a.N = s->dstate;
@@ -205,6 +214,12 @@ extern "C" {
 
 size_t bdscan_workspace_size(const bdscan_shape_t *shape, int op) {
   if (check_shape(shape) != BDSCAN_OK) return 0;
+  if (op == BDSCAN_OP_CONV_BLOCK_STEP) {
+    // the step's workspace, then the convolved x, B, C of both directions (the
+    // two-call path writes them there)
+    if (shape->seqlen != shape->block_len) return 0;
+    return align256(bdscan_workspace_size(shape, BDSCAN_OP_BLOCK_STEP)) + 2 * conv_scratch_bytes(shape);
+  }
   if (op == BDSCAN_OP_ALLBLOCK_BACKWARD)
     return bdscan::kWsHeader + bdscan::bwd_workspace_bytes(shape->batch, shape->seqlen, shape->nheads, shape->dstate);
   if (op != BDSCAN_OP_PREFIX && op != BDSCAN_OP_BLOCK_STEP && op != BDSCAN_OP_ALLBLOCK) return 0;
@@ -222,6 +237,22 @@ int bdscan_kernel_launches(const bdscan_shape_t *shape, int op) {
   if (op == BDSCAN_OP_GATED_RMSNORM) return (shape->batch == 0 || shape->seqlen == 0) ? 0 : 1;
   if (op == BDSCAN_OP_CONV_PREFIX || op == BDSCAN_OP_CONV_ALLBLOCK)
     return (shape->batch == 0 || shape->seqlen == 0) ? 0 : 1;
+  if (op == BDSCAN_OP_BLOCK_STEP || op == BDSCAN_OP_CONV_BLOCK_STEP) {
+    if (shape->seqlen != shape->block_len) return -1;
+    if (shape->batch == 0 || shape->seqlen == 0) return 0;
+    // tensor-core path: one launch for a small-batch step without state_out
+    // (C B^T in the scan kernel), else pre-pass + scan; the convolution of
+    // BDSCAN_OP_CONV_BLOCK_STEP adds its own kernel
+    const int conv = op == BDSCAN_OP_CONV_BLOCK_STEP ? 1 : 0;
+    if (bdscan::tc_shape_ok(shape->headdim, shape->dstate, shape->block_len, shape->in_dtype == BDSCAN_BF16) &&
+        !bdscan::opt_force_generic()) {
+      bdscan::ScanArgs a = base_args(shape);
+      a.mode = bdscan::Mode::Step;
+      a.has_cr = true;
+      return (bdscan::tc_one_launch_step(a) ? 1 : 2) + conv;
+    }
+    return 1 + conv;
+  }
   if (op == BDSCAN_OP_ALLBLOCK_BACKWARD) {
     // backward kernel + a dB/dC and a dA/dD reduction per present direction
     // (2 or 4 directions; counted here for all four)
@@ -734,6 +765,91 @@ int bdscan_conv_allblock(const bdscan_shape_t *shape, int width, int silu,
   a.dir[3] = to_conv_args(noisy_rev);
   a.state_in = conv_state_in;
   return conv_launch(a, z, static_cast<cudaStream_t>(cuda_stream));
+}
+
+int bdscan_conv_block_step(const bdscan_shape_t *shape, int width, int silu, const bdscan_conv_t *conv_fwd,
+                           const bdscan_conv_t *conv_rev, const void *conv_state_in, const bdscan_dir_t *fwd,
+                           const bdscan_dir_t *rev, const float *state_in, void *y, void *ws, size_t ws_bytes,
+                           void *cuda_stream) {
+  NvtxScope nvtx("bdscan_conv_block_step");
+  int rc = check_conv_shape(shape, width);
+  if (rc) return rc;
+  if (shape->seqlen != shape->block_len) return BDSCAN_ERR_UNSUPPORTED_SHAPE;
+  if (!conv_fwd || !conv_rev || !fwd || !rev) return BDSCAN_ERR_INVALID_ARG;
+  const ConvSizes cz = conv_sizes(shape, width);
+  const Sizes z = sizes_of(shape);
+  std::vector<Range> ins, outs;
+  // convolution inputs (its outputs are not used by this call)
+  for (const bdscan_conv_t *d : {conv_fwd, conv_rev}) {
+    if (!d->weight) return BDSCAN_ERR_INVALID_ARG;
+    if (cz.x && (!d->x || !d->B || !d->C)) return BDSCAN_ERR_INVALID_ARG;
+    const void *ptrs[] = {d->x, d->B, d->C, d->weight, d->bias};
+    for (const void *p : ptrs)
+      if (p && !aligned16(p)) return BDSCAN_ERR_MISALIGNED;
+    ins.push_back(range_of(d->x, cz.x));
+    ins.push_back(range_of(d->B, cz.bc));
+    ins.push_back(range_of(d->C, cz.bc));
+    ins.push_back(range_of(d->weight, cz.w));
+    if (d->bias) ins.push_back(range_of(d->bias, cz.bias));
+  }
+  // scan directions: dt, A, D, z (their x, B, C are not used)
+  for (const bdscan_dir_t *d : {fwd, rev}) {
+    if (!d->A || !d->D || (z.dt && !d->dt)) return BDSCAN_ERR_INVALID_ARG;
+    const void *ptrs[] = {d->dt, d->z, d->A, d->D};
+    for (const void *p : ptrs)
+      if (p && !aligned16(p)) return BDSCAN_ERR_MISALIGNED;
+    ins.push_back(range_of(d->dt, z.dt));
+    if (d->z) ins.push_back(range_of(d->z, z.x));
+    ins.push_back(range_of(d->A, z.ad));
+    ins.push_back(range_of(d->D, z.ad));
+  }
+  if ((!y && z.y) || (!state_in && z.state)) return BDSCAN_ERR_INVALID_ARG;
+  const void *ptrs[] = {conv_state_in, state_in, y};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return BDSCAN_ERR_MISALIGNED;
+  if (conv_state_in) ins.push_back(range_of(conv_state_in, cz.state));
+  ins.push_back(range_of(state_in, z.state));
+  outs.push_back(range_of(y, z.y));
+  if ((rc = check_outputs(ins, outs))) return rc;
+  if ((rc = check_ws(ws, ws_bytes, bdscan_workspace_size(shape, BDSCAN_OP_CONV_BLOCK_STEP)))) return rc;
+  // the convolved inputs live in the workspace past the step's own part
+  const size_t step_ws = align256(bdscan_workspace_size(shape, BDSCAN_OP_BLOCK_STEP));
+  const size_t in = shape->in_dtype == BDSCAN_BF16 ? 2 : 4;
+  const size_t BL = (size_t)shape->batch * (size_t)shape->seqlen;
+  const size_t xb = align256(BL * (size_t)(shape->nheads * shape->headdim) * in);
+  const size_t bcb = align256(BL * (size_t)(shape->ngroups * shape->dstate) * in);
+  uint8_t *scratch = static_cast<uint8_t *>(ws) + step_ws;
+  bdscan::ConvArgs ca = conv_base(shape, width, silu);
+  bdscan::ScanArgs a = base_args(shape);
+  a.mode = bdscan::Mode::Step;
+  a.has_cr = true;
+  a.h0 = state_in;
+  a.y_clean = y;
+  a.ws = ws;
+  a.ws_bytes = step_ws;
+  const bdscan_conv_t *cd[2] = {conv_fwd, conv_rev};
+  const bdscan_dir_t *sd[2] = {fwd, rev};
+  for (int d = 0; d < 2; ++d) {
+    uint8_t *base = scratch + d * (xb + 2 * bcb);
+    ca.dir[d] = to_conv_args(cd[d]);
+    ca.dir[d].x_out = base;
+    ca.dir[d].B_out = base + xb;
+    ca.dir[d].C_out = base + xb + bcb;
+    bdscan::DirArgs &da = d == 0 ? a.cf : a.cr;
+    da = to_args(sd[d]);
+    da.x = ca.dir[d].x_out;
+    da.B = ca.dir[d].B_out;
+    da.C = ca.dir[d].C_out;
+  }
+  ca.state_in = conv_state_in;
+  ca.state_out = nullptr;
+  // The convolution into the workspace, then the step (the step's kernel is a
+  // programmatic dependent of the convolution's: its prologue overlaps it).
+  // Convolving inside the one-launch step kernel was measured slower: every
+  // (sequence, head) CTA would recompute its group's B and C convolution.
+  const cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  if ((rc = conv_launch(ca, cz, stream))) return rc;
+  return launch(a, stream);
 }
 
 }  // extern "C"

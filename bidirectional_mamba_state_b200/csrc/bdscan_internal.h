@@ -50,6 +50,9 @@ bool tc_shape_ok(int64_t P, int64_t N, int64_t T, bool in_bf16);
 size_t tc_workspace_bytes(int64_t Bsz, int64_t L, int64_t G, int64_t H, bool allblock);
 int tc_plan_segments(int64_t Bsz, int64_t H, int64_t K);
 bool tc_supported(const ScanArgs &a);
+// Small-batch step without a state chain: C B^T computed in the scan kernel,
+// one launch (see scan_tc.cu).
+bool tc_one_launch_step(const ScanArgs &a);
 cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream);
 
 // Backward of the all-block pass (generic kernel, any accepted ungated shape

@@ -1789,6 +1789,19 @@ bool tc_supported(const ScanArgs &a) {
   return device_is_sm100();
 }
 
+// One-block items without a state chain, both clean directions, no more
+// items than SMs (small-batch denoising steps): the scan kernel computes the
+// C B^T tiles itself and the call is one launch.
+bool tc_one_launch_step(const ScanArgs &a) {
+  if (a.mode == Mode::AllBlock || !a.has_cr || a.L != kT || a.states || a.final_state || opt_cb_prepass())
+    return false;
+  int dev = 0, nsm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return false;
+  return a.Bsz * a.H <= nsm && tc_plan_segments(a.Bsz, a.H, 1) == 1;
+}
+
 cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
   const bool all = a.mode == Mode::AllBlock;
   const DirArgs *ds[4] = {&a.cf, all ? &a.nf : nullptr, a.has_cr ? &a.cr : nullptr,
@@ -1801,11 +1814,7 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
   if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
       (e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return e;
-  // One-block items without a state chain, both clean directions, no more
-  // items than SMs (small-batch denoising steps): the scan kernel computes
-  // the C B^T tiles itself and the call is one launch.
-  const bool cbfused = !all && a.has_cr && K == 1 && !a.states && !a.final_state && a.Bsz * a.H <= nsm &&
-                       tc_plan_segments(a.Bsz, a.H, K) == 1 && !opt_cb_prepass();
+  const bool cbfused = tc_one_launch_step(a);
 
   // ---- C B^T of every active direction
   CbParams cp;

@@ -72,6 +72,7 @@ extern "C" {
 #define BDSCAN_OP_CONV_PREFIX 4   /* no workspace (bdscan_workspace_size returns 0) */
 #define BDSCAN_OP_CONV_ALLBLOCK 5 /* no workspace */
 #define BDSCAN_OP_GATED_RMSNORM 6 /* no workspace */
+#define BDSCAN_OP_CONV_BLOCK_STEP 7
 
 /* Problem shape.  Supported: batch >= 0, seqlen >= 0, seqlen % block_len == 0,
  * 1 <= block_len <= 32 or block_len % 32 == 0 (<= 256), chunk_len % block_len
@@ -239,6 +240,34 @@ int bdscan_conv_allblock(const bdscan_shape_t *shape, int width, int silu,
                          const bdscan_conv_t *noisy_fwd, const bdscan_conv_t *noisy_rev,
                          const void *conv_state_in, void *cuda_stream);
 
+/* bdscan_conv_block_step -- one denoising step of a Mamba layer's
+ * selective-scan core from its cache, without commit: the short convolution
+ * (+SiLU) of both directions' x, B and C over the active block, the forward
+ * direction continuing from the conv state (exactly bdscan_conv_prefix with
+ * seqlen == block_len), then the scan step on the convolved inputs from the
+ * cached scan state (exactly bdscan_block_step with state_out NULL).  The two
+ * halves are the same operations as those calls ("Training Hybrid Block
+ * Diffusion Language Models with Partial Bidirectionality", the paragraph after
+ * eq. (14): a Mamba layer's cache holds its conv state beside its scan state).
+ *   conv_fwd, conv_rev  pre-convolution inputs, weights and bias of the two
+ *                       directions (both required); x_out, B_out and C_out
+ *                       are ignored: the convolved inputs are not returned
+ *   conv_state_in       [B][W-1][Cx] or NULL (zeros), as bdscan_conv_prefix
+ *   fwd, rev            the scan directions' dt, A, D and z (both required);
+ *                       their x, B and C are ignored (the convolution's
+ *                       outputs take their place)
+ *   state_in            [B][H][P][N] cached scan state (read only)
+ *   y                   [B][T][H][P] output (shape->out_dtype)
+ *   ws, ws_bytes        at least bdscan_workspace_size(shape, CONV_BLOCK_STEP)
+ * shape->seqlen must equal shape->block_len.  The convolution kernel writes
+ * the convolved inputs into the workspace and the step's kernels follow as
+ * programmatic dependents (two launches for a small batch on the tensor-core
+ * path: bdscan_kernel_launches).  y must not overlap any input. */
+int bdscan_conv_block_step(const bdscan_shape_t *shape, int width, int silu, const bdscan_conv_t *conv_fwd,
+                           const bdscan_conv_t *conv_rev, const void *conv_state_in, const bdscan_dir_t *fwd,
+                           const bdscan_dir_t *rev, const float *state_in, void *y, void *ws, size_t ws_bytes,
+                           void *cuda_stream);
+
 /* bdscan_gated_rmsnorm -- the normalisation of the summed output before the
  * layer's projection ("Breaking the Bottleneck with DiffuApriel", section 3.2
  * after eq. (6)), read as the Mamba-2 layer's gated RMSNorm with the gate
@@ -265,7 +294,10 @@ size_t bdscan_workspace_size(const bdscan_shape_t *shape, int op);
 
 /* Number of kernels one call of `op` launches for this shape (0 for an empty
  * problem, -1 for an invalid shape/op).  Lets a caller size CUDA graphs and
- * count launches; it does not launch anything. */
+ * count launches; it does not launch anything.  BDSCAN_OP_BLOCK_STEP counts a
+ * step without state_out; a committing step launches the C B^T pre-pass too
+ * (2 on the tensor-core path).  Options in force at the call are assumed
+ * (BDSCAN_OPT_CB_PREPASS, BDSCAN_OPT_FORCE_GENERIC). */
 int bdscan_kernel_launches(const bdscan_shape_t *shape, int op);
 
 /* Reads the device status word in ws after the work queued on cuda_stream

@@ -319,3 +319,39 @@ def test_options_set_get_restore():
     assert bd.bdscan_get_option(bd.BDSCAN_OPT_WAIT_TIMEOUT_NS) == t0
     assert bd.bdscan_get_option(99) == -1
     assert bd.bdscan_set_option(99, 0) == -1
+
+
+def _conv_step(s_kw=None, width=4, cf=None, cr=None, f=None, r=None, st=0x70000000, y=0x71000000,
+               cst=None, ws=0xA0000000, ws_bytes=1 << 24):
+    s = bd.c_shape(Shape(**_base(**dict(dict(seqlen=16, chunk_len=16), **(s_kw or {})))))
+    cf = _fake_conv(0x10000000) if cf is None else cf
+    cr = _fake_conv(0x20000000) if cr is None else cr
+    f = _fake_dir(0x30000000) if f is None else f
+    r = _fake_dir(0x40000000) if r is None else r
+    ref = lambda v: None if v == "null" else ctypes.byref(v)
+    return bd.bdscan_conv_block_step(ctypes.byref(s), width, 1, ref(cf), ref(cr), cst, ref(f), ref(r), st, y,
+                                     ws, ws_bytes, None)
+
+
+def test_conv_block_step_validation():
+    """Every call fails validation before any launch (fake addresses)."""
+    s = bd.c_shape(Shape(**_base(seqlen=16, chunk_len=16)))
+    need = bd.bdscan_workspace_size(ctypes.byref(s), bd.BDSCAN_OP_CONV_BLOCK_STEP)
+    assert need > bd.bdscan_workspace_size(ctypes.byref(s), bd.BDSCAN_OP_BLOCK_STEP)
+    s64 = bd.c_shape(Shape(**_base()))
+    assert bd.bdscan_workspace_size(ctypes.byref(s64), bd.BDSCAN_OP_CONV_BLOCK_STEP) == 0  # seqlen != block_len
+    assert _conv_step(s_kw=dict(seqlen=32, chunk_len=32)) == -2
+    assert _conv_step(width=5) == -2
+    assert _conv_step(cr="null") == -1 and _conv_step(r="null") == -1  # both directions required
+    d = _fake_conv(0x10000000)
+    d.weight = None
+    assert _conv_step(cf=d) == -1
+    d = _fake_dir(0x30000000)
+    d.dt = None
+    assert _conv_step(f=d) == -1
+    assert _conv_step(y=0x71000004) == -3                              # misaligned output
+    assert _conv_step(y=0x10000000) == -1                              # output over the conv input
+    assert _conv_step(cst=0x80000008) == -3                            # misaligned conv state
+    assert _conv_step(st=None) == -1                                   # scan state required
+    assert _conv_step(ws_bytes=need - 16) == -4                        # workspace too small
+    assert _conv_step(ws=None) == -4
