@@ -46,10 +46,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one bd_tc_kernel
 # launch on this workload, from one ncu capture, and the hash of the kernel
 # source it was taken on: reported while the source is unchanged, null after.
-TC_TRAFFIC = {"bytes": 223_820_544 + 550_532_608,
+TC_TRAFFIC = {"bytes": 223_811_584 + 550_921_984,
               "sources": ("bidirectional_mamba_state_b200/csrc/scan_tc.cu",
                           "bidirectional_mamba_state_b200/csrc/sm100.cuh"),
-              "sha256": "b0476c44aa3d7715c8d4485f14dc29e7922b0afd64ee76d5eca54d270dfea31a"}
+              "sha256": "8395df8315e151ffca676d0bfdb94aa45b5ca2f71bf118999a0fcd32b0b154f7"}
 
 
 def tc_traffic():
@@ -385,9 +385,18 @@ def _time(fn, dev, reps, warm=3):
 def _profile_case(name: str, dev, pk) -> dict:
     """One small case of a kernel for ncu (inputs of one layer, a few hundred MB
     on the device): three warm-up calls, then one call.  step_3b_b64: one 3B
-    layer's denoising step at batch 64; prefill_700m_8k: one 700M layer's 8K
+    layer's denoising step at batch 64; step_700m_b1: one 700M layer's batch-1
+    step (the one-launch instance); prefill_700m_8k: one 700M layer's 8K
     prefill (final state only)."""
-    if name == "step_3b_b64":
+    if name == "step_700m_b1":
+        s = W.WORKLOADS["700m_step"]
+        f, r = W.make_streams(s, W.SEEDS["700m_step"], device=dev, streams=(W.CLEAN_FWD, W.CLEAN_REV))
+        state = W.make_state(s, W.SEEDS["700m_step"], device=dev)
+        y = torch.empty((s.batch, s.seqlen, s.nheads, s.headdim), device=dev)
+        ws = bd.workspace(s, bd.BDSCAN_OP_BLOCK_STEP, dev)
+        call = lambda: bd.block_step(s, f, r, state, y=y, ws=ws)
+        b = RL.block_step_bytes(s)
+    elif name == "step_3b_b64":
         s = W.WORKLOADS["3b_step_b64"]
         f, r = W.make_streams(s, W.SEEDS["3b_step_b64"], device=dev, streams=(W.CLEAN_FWD, W.CLEAN_REV))
         state = W.make_state(s, W.SEEDS["3b_step_b64"], device=dev)
@@ -405,7 +414,7 @@ def _profile_case(name: str, dev, pk) -> dict:
         b = RL.prefix_bytes(s, block_states=False)
     ms = _time(call, dev, 1, 3)
     return {"us": ms * 1e3, "algorithmic_bytes": b, "launches_per_call": bd.kernel_launches(
-        s, bd.BDSCAN_OP_BLOCK_STEP if name == "step_3b_b64" else bd.BDSCAN_OP_PREFIX)}
+        s, bd.BDSCAN_OP_PREFIX if name.startswith("prefill") else bd.BDSCAN_OP_BLOCK_STEP)}
 
 
 EXTRA = {
@@ -419,6 +428,7 @@ EXTRA = {
     "prefill_700m_64k": lambda dev, pk: _prefill_line("700m_prefill_64k", 24, dev, pk),
     "prefill_3b_256k_40layers": lambda dev, pk: _prefill_3b(dev, pk),
     "profile_step_3b_b64": lambda dev, pk: _profile_case("step_3b_b64", dev, pk),
+    "profile_step_700m_b1": lambda dev, pk: _profile_case("step_700m_b1", dev, pk),
     "profile_prefill_700m_8k": lambda dev, pk: _profile_case("prefill_700m_8k", dev, pk),
     "allblock_backward_87m": lambda dev, pk: _backward(W.WORKLOADS["87m_allblock"], dev, pk),
     "conv_allblock_87m": lambda dev, pk: _conv_allblock(W.WORKLOADS["87m_allblock"], 4, dev, pk),
