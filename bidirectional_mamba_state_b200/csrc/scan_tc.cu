@@ -206,14 +206,13 @@ __global__ void __launch_bounds__(kCbThreads) bd_cb_kernel(const __grid_constant
 constexpr int kThreads = 512;
 
 // shared memory map (bytes from a 1024-aligned base)
-//   TMA ring, 3 slots (two blocks of lookahead); slot r holds block k = r mod 3:
+//   TMA ring: 144 KB, three 48 KB slots or five 28 KB slots per instance (the
+//   tile offsets inside a slot are Lay's, below the mode enum): x tiles [32 t]
+//   [64 p] bf16 (SW128), B_cf [32 s][n 0..63] then [32 s][n 64..127] (SW128), C
+//   rows x n 0..63 and x n 64..127 (SW128), C B^T tiles [32 s][32 t] bf16
+//   (SW64), 2 KB each; step j uses slot j mod (slots)
 constexpr int kSlots = 3;
-constexpr uint32_t kOffX = 0;                 // 4 dirs x [32 t][64 p] bf16 (SW128)
-constexpr uint32_t kOffBcf = 4 * kTile;       // clean-forward B: [32 s][n 0..63], [32 s][n 64..127] (SW128)
-constexpr uint32_t kOffClo = 6 * kTile;       // [C_cf; C_nf] rows x n 0..63 (SW128)
-constexpr uint32_t kOffChi = 8 * kTile;       // [C_cf; C_nf] rows x n 64..127
-constexpr uint32_t kOffCB = 10 * kTile;       // 4 dirs x [32 s][32 t] bf16 (SW64), 2 KB each
-constexpr uint32_t kSlot = 12 * kTile;        // 48 KB per slot
+constexpr uint32_t kSlot = 12 * kTile;        // 48 KB per slot of the three-slot layout
 constexpr uint32_t kOffXw = kSlots * kSlot;   // hi [32 t][64 p], lo [32 t][64 p] (bf16, SW128)
 constexpr uint32_t kOffH = kOffXw + 2 * kTile;  // {hi, lo} x [128 n][64 p] bf16 (SW128)
 constexpr uint32_t kOffMh = kOffH + 8 * kTile;  // 2 buffers x 4 dirs x [64 t'][32 s] interleaved
@@ -227,7 +226,8 @@ constexpr uint32_t kOffDtab = kOffDt + kTab * 512;  // [kTab][4] f32: D of the s
 constexpr uint32_t kOffFtab = kOffDtab + kTab * 16;  // [kTab] s32: 1 + item parity at an item's first step,
                                                      // 0 at its other steps, -1 past the CTA's last step
 constexpr uint32_t kOffBar = kOffFtab + 128;
-constexpr int kNumBars = 48;
+constexpr int kNumBars = 50;
+constexpr int kMaxSlots = 5;  // ring slots of the compact layout (see Lay)
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // TMEM base, abort flag
 constexpr int kItemRing = 16;
 constexpr uint32_t kOffItemQ = kOffMisc + 64;             // int4[kItemRing]: published work items
@@ -243,7 +243,7 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 constexpr uint32_t kMhSbo = 128, kMhLbo = 1024;
 
 enum : int {
-  bFull0 = 0, bFull1, bFull2, bEmpty0, bEmpty1, bEmpty2, bAux0, bAux7 = bAux0 + kTab - 1, bXwFull0, bXwFull1, bSFull0,
+  bFull0 = 0, bEmpty0 = bFull0 + kMaxSlots, bAux0 = bEmpty0 + kMaxSlots, bAux7 = bAux0 + kTab - 1, bXwFull0, bXwFull1, bSFull0,
   bSFull1,
   bSEmpty0, bSEmpty1, bMhFull0, bMhFull1, bHFull, bHCons, bYFull0, bYFull1, bYEmpty0, bYEmpty1, bDrain,
   bCbFull,
@@ -452,8 +452,7 @@ __device__ __forceinline__ int ybuf(int gated, int j) { return gated ? 0 : (j & 
 __device__ __forceinline__ uint32_t ypar(int gated, int j) { return gated ? (static_cast<uint32_t>(j) & 1u) : par2(j); }
 __device__ __forceinline__ int yprev(int gated, int j) { return gated ? j - 1 : j - 2; }
 // TMA ring: slot and parity of block k
-__device__ __forceinline__ int rslot(int k) { return k % kSlots; }
-__device__ __forceinline__ uint32_t parr(int k) { return static_cast<uint32_t>(k / kSlots) & 1u; }
+
 
 // ---------------------------------------------------------------- work items
 // A work item is one (batch row b, head h, segment seg) sequence of nk blocks
@@ -506,6 +505,32 @@ __device__ __forceinline__ uint32_t part(int j) { return (static_cast<uint32_t>(
 // Kernel instances: the call's mode is a template parameter (bits kModeAgg,
 // kModeAll, kModeNeedS), so each instance carries only the code its mode runs.
 enum : int { kModeAgg = 1, kModeAll = 2, kModeNeedS = 4, kModeCbFused = 8 };
+
+// Ring-slot layout of an instance.  The all-block pass, the aggregate pass and
+// the fused-C B^T step keep three 48 KB slots (x of four directions, B_cf, the
+// C tiles of two streams, four C B^T tiles; or B and C of both clean
+// directions); the one-stream scan and step instances use five 28 KB slots in
+// the same space (x of the two clean directions, B_cf, C_cf, two C B^T tiles),
+// so that the producer runs further ahead of the masked-decay build, which
+// waits for the tiles of the step two ahead.
+template <int kM>
+struct Lay {
+  static constexpr bool kCompact = (kM & (kModeAll | kModeAgg | kModeCbFused)) == 0;
+  static constexpr int kN = kCompact ? kMaxSlots : 3;
+  static constexpr uint32_t kBytes = kCompact ? 7 * kTile : 12 * kTile;
+  static constexpr uint32_t kBcf = kCompact ? 2 * kTile : 4 * kTile;  // B_cf, n 0..63 then 64..127
+  static constexpr uint32_t kClo = kCompact ? 4 * kTile : 6 * kTile;  // C rows x n 0..63
+  static constexpr uint32_t kChi = kCompact ? 5 * kTile : 8 * kTile;  // C rows x n 64..127
+  static constexpr uint32_t kCbBase = kCompact ? 6 * kTile : 10 * kTile;
+  // x tile of direction slot i, C B^T tile of direction slot i
+  __host__ __device__ static constexpr uint32_t x(int i) { return static_cast<uint32_t>(kCompact ? (i >> 1) : i) * kTile; }
+  __host__ __device__ static constexpr uint32_t cb(int i) {
+    return kCbBase + static_cast<uint32_t>(kCompact ? (i >> 1) : i) * 2048u;
+  }
+  __device__ static int slot(int j) { return j % kN; }
+  __device__ static uint32_t par(int j) { return static_cast<uint32_t>(j / kN) & 1u; }
+};
+static_assert(kMaxSlots * 7 * kTile <= kSlots * kSlot, "compact ring within the ring's space");
 // kModeCbFused (one-block items without a state chain, no more items than
 // SMs: the batch-1 denoising step): no C B^T pre-pass; each step loads B and C
 // of both directions and computes its own C B^T tiles (one M = 64 MMA chain
@@ -588,7 +613,10 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
   } else {
     tma_prefetch_desc(&p.tcb);
   }
-  int last[kSlots] = {-1, -1, -1};
+  using Ly = Lay<kM>;
+  int last[Ly::kN];
+#pragma unroll
+  for (int s = 0; s < Ly::kN; ++s) last[s] = -1;
   int j = 0;
   bool ok = true;
   // items m and m + 1 are published when item m starts (nothing after a -1);
@@ -610,40 +638,40 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
     const Item I = Icur;
     for (int kk = 0; kk < I.nk; ++kk, ++j) {
       const int k = item_block<kAgg>(I.k0, I.nk, kk);  // block index in the sequence
-      const int r = rslot(j);
-      if (!wait1(c, bEmpty0 + r, parr(j) ^ 1)) {
+      const int r = Ly::slot(j);
+      if (!wait1(c, bEmpty0 + r, Ly::par(j) ^ 1)) {
         ok = false;
         break;
       }
       const uint32_t full = bar_at(c, bFull0 + r);
       mbar_arrive_expect_tx_s(full, bytes);
-      const uint32_t st = base + r * kSlot;
+      const uint32_t st = base + r * Ly::kBytes;
       const int t0 = k * kT;
       if constexpr (kCbF) {
-        // x_cf, x_cr; [B_cf; B_cr] as the A operand of C B^T (n 0..63 at kOffBcf,
-        // n 64..127 at kOffCB, 64 rows each); [C_cf; C_cr] at kOffClo / kOffChi
-        tma_load_4d_s(st + kOffX, &p.tx[kCF], full, 0, I.h, t0, I.b);
-        tma_load_4d_s(st + kOffX + kCR * kTile, &p.tx[kCR], full, 0, I.h, t0, I.b);
-        tma_load_4d_s(st + kOffBcf, &p.tbcf, full, 0, I.g, t0, I.b);
-        tma_load_4d_s(st + kOffBcf + kTile, &p.tbcr, full, 0, I.g, t0, I.b);
-        tma_load_4d_s(st + kOffCB, &p.tbcf, full, 64, I.g, t0, I.b);
-        tma_load_4d_s(st + kOffCB + kTile, &p.tbcr, full, 64, I.g, t0, I.b);
-        tma_load_4d_s(st + kOffClo, &p.tccf, full, 0, I.g, t0, I.b);
-        tma_load_4d_s(st + kOffClo + kTile, &p.tccr, full, 0, I.g, t0, I.b);
-        tma_load_4d_s(st + kOffChi, &p.tccf, full, 64, I.g, t0, I.b);
-        tma_load_4d_s(st + kOffChi + kTile, &p.tccr, full, 64, I.g, t0, I.b);
+        // x_cf, x_cr; [B_cf; B_cr] as the A operand of C B^T (n 0..63 at kBcf,
+        // n 64..127 at kCbBase, 64 rows each); [C_cf; C_cr] at kClo / kChi
+        tma_load_4d_s(st + Ly::x(kCF), &p.tx[kCF], full, 0, I.h, t0, I.b);
+        tma_load_4d_s(st + Ly::x(kCR), &p.tx[kCR], full, 0, I.h, t0, I.b);
+        tma_load_4d_s(st + Ly::kBcf, &p.tbcf, full, 0, I.g, t0, I.b);
+        tma_load_4d_s(st + Ly::kBcf + kTile, &p.tbcr, full, 0, I.g, t0, I.b);
+        tma_load_4d_s(st + Ly::kCbBase, &p.tbcf, full, 64, I.g, t0, I.b);
+        tma_load_4d_s(st + Ly::kCbBase + kTile, &p.tbcr, full, 64, I.g, t0, I.b);
+        tma_load_4d_s(st + Ly::kClo, &p.tccf, full, 0, I.g, t0, I.b);
+        tma_load_4d_s(st + Ly::kClo + kTile, &p.tccr, full, 0, I.g, t0, I.b);
+        tma_load_4d_s(st + Ly::kChi, &p.tccf, full, 64, I.g, t0, I.b);
+        tma_load_4d_s(st + Ly::kChi + kTile, &p.tccr, full, 64, I.g, t0, I.b);
       } else {
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          if (p.active[i]) tma_load_4d_s(st + kOffX + i * kTile, &p.tx[i], full, 0, I.h, t0, I.b);
-        tma_load_4d_s(st + kOffBcf, &p.tbcf, full, 0, I.g, t0, I.b);
-        tma_load_4d_s(st + kOffBcf + kTile, &p.tbcf, full, 64, I.g, t0, I.b);
+          if (p.active[i]) tma_load_4d_s(st + Ly::x(i), &p.tx[i], full, 0, I.h, t0, I.b);
+        tma_load_4d_s(st + Ly::kBcf, &p.tbcf, full, 0, I.g, t0, I.b);
+        tma_load_4d_s(st + Ly::kBcf + kTile, &p.tbcf, full, 64, I.g, t0, I.b);
         if (!kAgg) {
-          tma_load_4d_s(st + kOffClo, &p.tccf, full, 0, I.g, t0, I.b);
-          tma_load_4d_s(st + kOffChi, &p.tccf, full, 64, I.g, t0, I.b);
+          tma_load_4d_s(st + Ly::kClo, &p.tccf, full, 0, I.g, t0, I.b);
+          tma_load_4d_s(st + Ly::kChi, &p.tccf, full, 64, I.g, t0, I.b);
           if (kAll) {
-            tma_load_4d_s(st + kOffClo + kTile, &p.tcnf, full, 0, I.g, t0, I.b);
-            tma_load_4d_s(st + kOffChi + kTile, &p.tcnf, full, 64, I.g, t0, I.b);
+            tma_load_4d_s(st + Ly::kClo + kTile, &p.tcnf, full, 0, I.g, t0, I.b);
+            tma_load_4d_s(st + Ly::kChi + kTile, &p.tcnf, full, 64, I.g, t0, I.b);
           }
           // C B^T tiles: written by the pre-pass this kernel may overlap
           if (!waited) {
@@ -654,12 +682,12 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
           for (int i = 0; i < 4; ++i) {
             if (!p.active[i]) continue;
             const int idx = ((cb_set(kAll, i) * p.Bsz + I.b) * p.K + k) * p.G + I.g;
-            tma_load_3d_s(st + kOffCB + i * 2048, &p.tcb, full, 0, 0, idx);
+            tma_load_3d_s(st + Ly::cb(i), &p.tcb, full, 0, 0, idx);
           }
         }
       }
 #pragma unroll
-      for (int s = 0; s < kSlots; ++s)
+      for (int s = 0; s < Ly::kN; ++s)
         if (s == r) last[s] = j;
     }
     cur = nxt;
@@ -673,8 +701,8 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
   }
   // no copy into this CTA's shared memory may still be in flight at exit
 #pragma unroll
-  for (int s = 0; s < kSlots; ++s)
-    if (last[s] >= 0) (void)mbar_wait_s(bar_at(c, bFull0 + s), parr(last[s]), p.drain_ns, 0);
+  for (int s = 0; s < Ly::kN; ++s)
+    if (last[s] >= 0) (void)mbar_wait_s(bar_at(c, bFull0 + s), Ly::par(last[s]), p.drain_ns, 0);
 }
 
 // ---------------------------------------------------------------- MMA issuer
@@ -689,14 +717,15 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
   const uint32_t id_yo = kAll ? idesc_bf16(64, 64, 1, 0) : idesc_bf16(64, 32, 1, 0);
   const uint32_t id_yd = idesc_bf16(64, 64, 1, 1);  // [Y_diag^T | remainder][p][t'] = X^T [M^T | diag]
   // descriptor of each operand at its first tile; moving an operand by b bytes adds b >> 4
-  const D64 dBcf = split64(sdesc(base + kOffBcf, kTile, 1024, kLayoutSw128));
+  using Ly = Lay<kM>;
+  const D64 dBcf = split64(sdesc(base + Ly::kBcf, kTile, 1024, kLayoutSw128));
   const D64 dXw = split64(sdesc(base + kOffXw, 0, 1024, kLayoutSw128));
   const D64 dH = split64(sdesc(base + kOffH, 0, 1024, kLayoutSw128));
-  const D64 dC = split64(sdesc(base + kOffClo, 16, 1024, kLayoutSw128));
-  const D64 dX = split64(sdesc(base + kOffX, 0, 1024, kLayoutSw128));
+  const D64 dC = split64(sdesc(base + Ly::kClo, 16, 1024, kLayoutSw128));
+  const D64 dX = split64(sdesc(base + Ly::x(0), 0, 1024, kLayoutSw128));
   const D64 dM = split64(sdesc(base + kOffMh, kMhLbo, kMhSbo, kLayoutNone));
-  // fused C B^T: [B_cf; B_cr] K-major (64 rows s; n 0..63 at kOffBcf, 64..127 at kOffCB)
-  const D64 dBk = split64(sdesc(base + kOffBcf, 16, 1024, kLayoutSw128));
+  // fused C B^T: [B_cf; B_cr] K-major (64 rows s; n 0..63 at kBcf, 64..127 at kCbBase)
+  const D64 dBk = split64(sdesc(base + Ly::kBcf, 16, 1024, kLayoutSw128));
   const uint32_t id_cb = idesc_bf16(64, 64, 0, 0);
 #define BD_OFF(bytes) (static_cast<uint32_t>((bytes) >> 4))
   int j = 0;
@@ -707,9 +736,9 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
     const int nk = I.nk;
     for (int kk = 0; kk < nk; ++kk, ++j) {
       ok = false;
-      const int r = rslot(j), i2 = j & 1;
-      const uint32_t so = BD_OFF(static_cast<uint32_t>(r) * kSlot);  // this step's ring slot
-      if (!wait1(c, bFull0 + r, parr(j))) break;
+      const int r = Ly::slot(j), i2 = j & 1;
+      const uint32_t so = BD_OFF(static_cast<uint32_t>(r) * Ly::kBytes);  // this step's ring slot
+      if (!wait1(c, bFull0 + r, Ly::par(j))) break;
       if constexpr (kCbF) {
         // ---- [C B^T]: rows s of [B_cf; B_cr] against columns t of [C_cf; C_cr];
         //      the two diagonal 32 x 32 blocks are the directions' tiles.  The
@@ -719,8 +748,8 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
 #pragma unroll 1
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t ko = BD_OFF((ks & 3) * 32);
-          umma_bf16(tmem + kColCb, dBk + so + ko + (ks < 4 ? 0u : BD_OFF(kOffCB - kOffBcf)),
-                    dC + so + ko + (ks < 4 ? 0u : BD_OFF(2 * kTile)), id_cb, ks > 0);
+          umma_bf16(tmem + kColCb, dBk + so + ko + (ks < 4 ? 0u : BD_OFF(Ly::kCbBase - Ly::kBcf)),
+                    dC + so + ko + (ks < 4 ? 0u : BD_OFF(Ly::kChi - Ly::kClo)), id_cb, ks > 0);
         }
         umma_commit_s(bar_at(c, bCbFull));
       }
@@ -766,7 +795,7 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
       const uint32_t colY = tmem + kColY0 + kColYBuf * yb;
 #pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
-        const D64 bc = dC + so + BD_OFF((ks < 4 ? 0 : 2 * kTile) + (ks & 3) * 32);
+        const D64 bc = dC + so + BD_OFF((ks < 4 ? 0u : Ly::kChi - Ly::kClo) + (ks & 3) * 32);
         umma_bf16(colY, dH + BD_OFF(ks * 2048), bc, id_yo, ks > 0);
         umma_bf16(colY, dH + BD_OFF(4 * kTile + ks * 2048), bc, id_yo, 1);
       }
@@ -785,7 +814,7 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
         const uint32_t col = colY + 64 + ((i & 1) ? 64 : 0) + (own ? kColRevGated : 0);
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks)
-          umma_bf16(col, dX + so + BD_OFF(i * kTile + ks * 2048), dM + mo + BD_OFF(i * kMhDir + ks * 2048), id_yd,
+          umma_bf16(col, dX + so + BD_OFF(Ly::x(i) + ks * 2048), dM + mo + BD_OFF(i * kMhDir + ks * 2048), id_yd,
                     ((i >= 2 && !own) || ks > 0) ? 1u : 0u);
       }
       umma_commit_s(bar_at(c, bYFull0 + yb));
@@ -802,10 +831,10 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
 // masked-decay matrix M^T[s][t] of the block with the direction's D added to
 // its diagonal, stored bf16, and that diagonal's bf16 remainders; one warp,
 // row s = lane.  Reads the step's C B^T tile (ring slot) and decay tables.
-__device__ __forceinline__ void build_masked_decay(uint32_t base, int q, int lane, int jm, bool act, bool rev) {
+__device__ __forceinline__ void build_masked_decay(uint32_t base, uint32_t cbrow, int q, int lane, int jm, bool act,
+                                                   bool rev) {
   const int ct = jm % kTab;
   if (act) {
-    const uint32_t cbrow = base + rslot(jm) * kSlot + kOffCB + q * 2048;
     const uint32_t cq = base + kOffCum + (ct * 4 + q) * 128;
     const float cs = lds_f32(cq + lane * 4);
     const float ds = lds_f32(base + kOffDt + (ct * 4 + q) * 128 + lane * 4);
@@ -894,10 +923,9 @@ __device__ __forceinline__ void build_rows16(uint32_t base, int q, int lane, int
 }
 
 // From the step's bf16 C B^T tile in its ring slot (pre-pass instances).
-__device__ __forceinline__ void build_masked_decay_split(uint32_t base, int q, int lane, int jm) {
+__device__ __forceinline__ void build_masked_decay_split(uint32_t base, uint32_t cbrow, int q, int lane, int jm) {
   const int s = 16 * (q & 1) + (lane & 15);
   const int th = lane & 16;
-  const uint32_t cbrow = base + rslot(jm) * kSlot + kOffCB + (q >= 2 ? kCR : kCF) * 2048;
   uint32_t r[8];
   ld_shared_v4(cbrow + sw64_chunk(s, th >> 3), r[0], r[1], r[2], r[3]);
   ld_shared_v4(cbrow + sw64_chunk(s, (th >> 3) + 1), r[4], r[5], r[6], r[7]);
@@ -985,7 +1013,7 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
     Item In = I;
     for (int kk = 0; kk < I.nk; ++kk, ++j) {
       const int ct = j % kTab;
-      const uint32_t st = base + rslot(j) * kSlot;
+      const uint32_t st = base + Lay<kM>::slot(j) * Lay<kM>::kBytes;
       const float dt_cur = qdt[0], A2 = qa[0], Dv = qd[0];
       qdt[0] = qdt[1];
       qa[0] = qa[1];
@@ -1015,7 +1043,7 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
       if (gt == 0) sts_s32(base + kOffFtab + ct * 4, kk == 0 ? 1 + (m & 1) : 0);
       arrive_lane0(c, bAux0 + ct);
       if (!waitw(c, bAux0 + ct, part(j))) return;
-      if (!waitw(c, bFull0 + rslot(j), parr(j))) return;
+      if (!waitw(c, bFull0 + Lay<kM>::slot(j), Lay<kM>::par(j))) return;
       // ---- (w o X) of the clean forward direction, bf16 hi + lo
       if (kNeedS) {
         uint32_t xw = base + kOffXw;
@@ -1027,7 +1055,7 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
           if (kk == 0) rdec = 0.f;
           rw = rdec;
           if (j & 1) xw = base + kOffH;
-          if (j >= 2 && !waitw(c, bEmpty0 + rslot(j - 2), parr(j - 2))) return;
+          if (j >= 2 && !waitw(c, bEmpty0 + Lay<kM>::slot(j - 2), Lay<kM>::par(j - 2))) return;
         } else {
           // the S MMA of the previous step has read the w o X buffer
           if (j >= 1 && !waitw(c, bSFull0 + ((j - 1) & 1), par2(j - 1))) return;
@@ -1041,7 +1069,7 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
           const int t = i >> 3, ch = i & 7;
           const uint32_t off = sw128_chunk(t, ch);
           uint32_t r0, r1, r2, r3;
-          ld_shared_v4(st + kOffX + off, r0, r1, r2, r3);
+          ld_shared_v4(st + Lay<kM>::x(kCF) + off, r0, r1, r2, r3);
           const float w = lds_f32(df + t * 4) * ex2_approx(c31 - lds_f32(cf + t * 4) + rw);
           float vv[8] = {bf16_lo_f(r0) * w, bf16_hi_f(r0) * w, bf16_lo_f(r1) * w, bf16_hi_f(r1) * w,
                          bf16_lo_f(r2) * w, bf16_hi_f(r2) * w, bf16_lo_f(r3) * w, bf16_hi_f(r3) * w};
@@ -1050,7 +1078,7 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
         fence_proxy_async_smem();
         arrive_lane0(c, bXwFull0 + (j & 1));
       }
-      arrive_lane0(c, bEmpty0 + rslot(j));
+      arrive_lane0(c, bEmpty0 + Lay<kM>::slot(j));
     }
     if (!has_next) break;
     I = In;
@@ -1360,15 +1388,17 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
       build_masked_decay_tm(base, tmem, q, lane, jm);
       tc_fence_before();  // the accumulator's next writer waits for this warp's arrival
     } else {
-      if (!waitw(c, bFull0 + rslot(jm), parr(jm))) return false;  // C B^T tiles
+      using Ly = Lay<kM>;
+      if (!waitw(c, bFull0 + Ly::slot(jm), Ly::par(jm))) return false;  // C B^T tiles
+      const uint32_t sl = base + static_cast<uint32_t>(Ly::slot(jm)) * Ly::kBytes;
       // one-block items without a state chain: the four-warp split (the
       // epilogue is that pipeline's co-bottleneck); otherwise one warp per
       // direction, which keeps warp 13 (the MMA issuer's sub-partition) idle
       // in the issue-bound state-chain instances
       if constexpr (kAll || kNeedS)
-        build_masked_decay(base, q, lane, jm, act, rev);
+        build_masked_decay(base, sl + Ly::cb(q), q, lane, jm, act, rev);
       else if (q < 2 || p.active[kCR])
-        build_masked_decay_split(base, q, lane, jm);
+        build_masked_decay_split(base, sl + Ly::cb(q >= 2 ? kCR : kCF), q, lane, jm);
     }
     fence_proxy_async_smem();
     arrive_lane0(c, bMhFull0 + (jm & 1));
@@ -1551,10 +1581,10 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
     // operand warps; commits of the MMA warp count 1; the rest 4 warps each
     for (int i = 0; i < bCount; ++i) {
       uint32_t cnt = 4;
-      if (i == bFull0 || i == bFull1 || i == bFull2 || i == bSFull0 || i == bSFull1 || i == bYFull0 ||
+      if ((i >= bFull0 && i < bFull0 + kMaxSlots) || i == bSFull0 || i == bSFull1 || i == bYFull0 ||
           i == bYFull1 || i == bHCons || i == bDrain || i == bCbFull || i >= bItem0)
         cnt = 1;
-      else if (i == bEmpty0 || i == bEmpty1 || i == bEmpty2)
+      else if (i >= bEmpty0 && i < bEmpty0 + kMaxSlots)
         cnt = 5;
       mbar_init(&bars[i], cnt);
     }
