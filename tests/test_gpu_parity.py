@@ -293,3 +293,36 @@ def test_bounded_wait_timeout_reports_status():
     ryc, ryn, rst = oracle.allblock(s.as_dict(), cf, cr, nf, nr)
     check_y(yn, ryn)
     check_states(st, rst)
+
+
+@pytest.mark.parametrize("case", ["pairs_eq_sms", "pairs_over_sms", "fwd_only", "gated_g2", "bf16_out_g2"])
+def test_block_step_one_launch_edges(case):
+    """Edges of the one-launch small-batch step (C B^T in the scan kernel):
+    exactly as many (sequence, head) pairs as SMs, one sequence more (pre-pass path),
+    a forward-only step (pre-pass path), gated directions with two groups, bf16
+    output; each against the oracle, and the pair-count edges also against the
+    pre-pass path."""
+    nsm = torch.cuda.get_device_properties(0).multi_processor_count
+    kw = dict(batch=2, seqlen=32, chunk_len=32, nheads=6, ngroups=2)
+    if case in ("pairs_eq_sms", "pairs_over_sms"):
+        assert nsm % 4 == 0
+        kw.update(batch=nsm // 4, nheads=4, ngroups=1)
+    elif case == "bf16_out_g2":
+        kw.update(out_dtype="bf16")
+    s = _shape(**kw)
+    if case == "pairs_over_sms":  # one more sequence than fills the SMs
+        s = s.with_(batch=s.batch + 1)
+    gated = case == "gated_g2"
+    f = W.make_dir(s, 17, 0, W.CLEAN_FWD, DEV, gated=gated)
+    r = None if case == "fwd_only" else W.make_dir(s, 17, 0, W.CLEAN_REV, DEV, gated=gated)
+    state = W.make_state(s, 17, device=DEV, scale=2.0)
+    y, _ = bd.block_step(s, f, r, state)
+    with bd.option(bd.BDSCAN_OPT_CB_PREPASS, 1):
+        y2, _ = bd.block_step(s, f, r, state)
+    torch.cuda.synchronize()
+    ry, _ = oracle.block_step(s.as_dict(), f, r, state)
+    bf = s.out_dtype == "bf16"
+    check_y(y, ry, bf16_out=bf, what=case)
+    check_y(y2, ry, bf16_out=bf, what=case + " (pre-pass)")
+    if r is not None:  # the launch count assumes both directions
+        assert bd.kernel_launches(s, bd.BDSCAN_OP_BLOCK_STEP) == (1 if s.batch * s.nheads <= nsm else 2)
