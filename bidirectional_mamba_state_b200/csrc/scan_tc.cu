@@ -226,8 +226,8 @@ constexpr uint32_t kOffDtab = kOffDt + kTab * 512;  // [kTab][4] f32: D of the s
 constexpr uint32_t kOffFtab = kOffDtab + kTab * 16;  // [kTab] s32: 1 + item parity at an item's first step,
                                                      // 0 at its other steps, -1 past the CTA's last step
 constexpr uint32_t kOffBar = kOffFtab + 128;
-constexpr int kNumBars = 50;
-constexpr int kMaxSlots = 5;  // ring slots of the compact layout (see Lay)
+constexpr int kNumBars = 56;
+constexpr int kMaxSlots = 8;  // ring slots of the compact layouts (see Lay)
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // TMEM base, abort flag
 constexpr int kItemRing = 16;
 constexpr uint32_t kOffItemQ = kOffMisc + 64;             // int4[kItemRing]: published work items
@@ -506,31 +506,35 @@ __device__ __forceinline__ uint32_t part(int j) { return (static_cast<uint32_t>(
 // kModeAll, kModeNeedS), so each instance carries only the code its mode runs.
 enum : int { kModeAgg = 1, kModeAll = 2, kModeNeedS = 4, kModeCbFused = 8 };
 
-// Ring-slot layout of an instance.  The all-block pass, the aggregate pass and
-// the fused-C B^T step keep three 48 KB slots (x of four directions, B_cf, the
-// C tiles of two streams, four C B^T tiles; or B and C of both clean
-// directions); the one-stream scan and step instances use five 28 KB slots in
-// the same space (x of the two clean directions, B_cf, C_cf, two C B^T tiles),
-// so that the producer runs further ahead of the masked-decay build, which
-// waits for the tiles of the step two ahead.
+// Ring-slot layout of an instance.  The all-block pass and the fused-C B^T
+// step keep three 48 KB slots (x of four directions, B_cf, the C tiles of two
+// streams, four C B^T tiles; or B and C of both clean directions); the
+// one-stream scan and step instances use five 28 KB slots in the same space
+// (x of the two clean directions, B_cf, C_cf, two C B^T tiles), so that the
+// producer runs further ahead of the masked-decay build, which waits for the
+// tiles of the step two ahead; the aggregate pass, which reads only x_cf and
+// B_cf, eight 12 KB slots.
 template <int kM>
 struct Lay {
+  static constexpr bool kAggL = (kM & kModeAgg) != 0;
   static constexpr bool kCompact = (kM & (kModeAll | kModeAgg | kModeCbFused)) == 0;
-  static constexpr int kN = kCompact ? kMaxSlots : 3;
-  static constexpr uint32_t kBytes = kCompact ? 7 * kTile : 12 * kTile;
-  static constexpr uint32_t kBcf = kCompact ? 2 * kTile : 4 * kTile;  // B_cf, n 0..63 then 64..127
+  static constexpr int kN = kAggL ? 8 : (kCompact ? 5 : 3);
+  static constexpr uint32_t kBytes = kAggL ? 3 * kTile : (kCompact ? 7 * kTile : 12 * kTile);
+  static constexpr uint32_t kBcf = kAggL ? kTile : (kCompact ? 2 * kTile : 4 * kTile);  // B_cf, n 0..63 then 64..127
   static constexpr uint32_t kClo = kCompact ? 4 * kTile : 6 * kTile;  // C rows x n 0..63
   static constexpr uint32_t kChi = kCompact ? 5 * kTile : 8 * kTile;  // C rows x n 64..127
   static constexpr uint32_t kCbBase = kCompact ? 6 * kTile : 10 * kTile;
   // x tile of direction slot i, C B^T tile of direction slot i
-  __host__ __device__ static constexpr uint32_t x(int i) { return static_cast<uint32_t>(kCompact ? (i >> 1) : i) * kTile; }
+  __host__ __device__ static constexpr uint32_t x(int i) {
+    return kAggL ? 0u : static_cast<uint32_t>(kCompact ? (i >> 1) : i) * kTile;  // the aggregate pass: x_cf only
+  }
   __host__ __device__ static constexpr uint32_t cb(int i) {
     return kCbBase + static_cast<uint32_t>(kCompact ? (i >> 1) : i) * 2048u;
   }
   __device__ static int slot(int j) { return j % kN; }
   __device__ static uint32_t par(int j) { return static_cast<uint32_t>(j / kN) & 1u; }
 };
-static_assert(kMaxSlots * 7 * kTile <= kSlots * kSlot, "compact ring within the ring's space");
+static_assert(5 * 7 * kTile <= kSlots * kSlot && 8 * 3 * kTile <= kSlots * kSlot, "compact rings within the ring's space");
 // kModeCbFused (one-block items without a state chain, no more items than
 // SMs: the batch-1 denoising step): no C B^T pre-pass; each step loads B and C
 // of both directions and computes its own C B^T tiles (one M = 64 MMA chain
