@@ -202,14 +202,27 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
     s.Bt[n * T + i] = s.Bm[i * N + n];
     s.Ct[n * T + i] = s.Cm[i * N + n];
   }
-  if (tid == 0) {
-    float c = 0.f;
-    for (int i = 0; i < T; ++i) {
-      c += s.dt[i] * A;
-      s.cum[i] = c;
-      s.lam[i] = expf(c);
+  // cumulative decays: a warp prefix scan over 32-token chunks (lane order
+  // within a chunk, chunks in order), then Lam and r in parallel
+  if (tid < 32) {
+    float carry = 0.f;
+    for (int i0 = 0; i0 < T; i0 += 32) {
+      const int i = i0 + tid;
+      float v = i < T ? s.dt[i] * A : 0.f;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, v, o);
+        if (tid >= o) v += u;
+      }
+      v += carry;
+      if (i < T) {
+        s.cum[i] = v;
+        s.lam[i] = expf(v);
+      }
+      carry = __shfl_sync(0xffffffffu, v, 31);  // = cum of the chunk's last token (padding adds 0)
     }
-    for (int i = 0; i < T; ++i) s.r[i] = expf(c - s.cum[i]);
+    __syncwarp();
+    for (int i = tid; i < T; i += 32) s.r[i] = expf(carry - s.cum[i]);
   }
   __syncthreads();
 
@@ -318,13 +331,29 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
   }
   __syncthreads();
   float pa = 0.f, pd = 0.f;
-  if (tid == 0) {
-    float suffix = 0.f;
-    for (int v = T - 1; v >= 0; --v) {
-      suffix += s.S[v];
-      d.ddt[(static_cast<int64_t>(b) * L + tok(v)) * H + h] = s.expl[v] + A * suffix;
-      pa += s.dt[v] * suffix;
+  // suffix sums of dL/dcum: a warp scan over 32-token chunks from the block's
+  // end (lane 0 = the chunk's last token); the dA partial is summed in a fixed
+  // shuffle order
+  if (tid < 32) {
+    float carry = 0.f, pacc = 0.f;
+    for (int i1 = T; i1 > 0; i1 -= 32) {
+      const int v = i1 - 1 - tid;
+      float x = v >= 0 ? s.S[v] : 0.f;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, x, o);
+        if (tid >= o) x += u;
+      }
+      x += carry;
+      if (v >= 0) {
+        d.ddt[(static_cast<int64_t>(b) * L + tok(v)) * H + h] = s.expl[v] + A * x;
+        pacc = fmaf(s.dt[v], x, pacc);
+      }
+      carry = __shfl_sync(0xffffffffu, x, 31);
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) pacc += __shfl_xor_sync(0xffffffffu, pacc, o);
+    pa = pacc;
   }
   for (int e = tid; e < T * P; e += kBwdThreads) pd += s.dy[e] * s.x[e];
   pd = block_sum(pd, s.red);
