@@ -131,3 +131,44 @@ def test_nan_stays_in_its_sequence(kw):
                             ("states", st0, st1, mask_s)):
         assert torch.equal(a0[m], a1[m]), f"{name}: the NaN leaked into another sequence"
     assert torch.isnan(yc1[b, :, h]).any() and torch.isnan(st1[b, :, h]).any()
+
+
+@pytest.mark.parametrize("gated", [False, True])
+def test_one_launch_step_guards_and_nan(gated):
+    """The one-launch small-batch step (C B^T computed in the scan kernel): its
+    output stays inside its buffer, the state is not written, and a NaN in one
+    (b, h)'s x reaches only that sequence (a NaN in B or C of a group reaches
+    exactly the heads of that group)."""
+    s = _shape(seqlen=32, chunk_len=32, nheads=6, ngroups=2, batch=2)
+    f = W.make_dir(s, 6, 0, W.CLEAN_FWD, DEV, gated=gated)
+    r = W.make_dir(s, 6, 0, W.CLEAN_REV, DEV, gated=gated)
+    state = W.make_state(s, 6, device=DEV)
+    keep = state.clone()
+    tout = torch.float32
+    y = Guarded((s.batch, s.seqlen, s.nheads, s.headdim), tout)
+    bd.block_step(s, f, r, state, y=y.t)
+    torch.cuda.synchronize()
+    assert y.intact(), "step y: a guard region was overwritten"
+    assert torch.equal(state, keep), "the cached state was written by a non-committing step"
+    y0 = y.t.clone()
+    b, h = 1, 4
+    bad = dict(f)
+    bad["x"] = f["x"].clone()
+    bad["x"][b, 7, h, 3] = float("nan")
+    y1, _ = bd.block_step(s, bad, r, state)
+    torch.cuda.synchronize()
+    m = torch.ones(y0.shape, dtype=torch.bool, device=DEV)
+    m[b, :, h] = False
+    assert torch.equal(y0[m], y1[m]), "the NaN leaked into another sequence"
+    assert torch.isnan(y1[b, :, h]).any()
+    # a NaN in B of group 0 of row b reaches the heads of that group only
+    badb = dict(f)
+    badb["B"] = f["B"].clone()
+    badb["B"][b, 5, 0, 11] = float("nan")
+    y2, _ = bd.block_step(s, badb, r, state)
+    torch.cuda.synchronize()
+    hpg = s.nheads // s.ngroups
+    m2 = torch.ones(y0.shape, dtype=torch.bool, device=DEV)
+    m2[b, :, :hpg] = False
+    assert torch.equal(y0[m2], y2[m2]), "a NaN in B leaked beyond its group"
+    assert torch.isnan(y2[b, :, :hpg]).any()
