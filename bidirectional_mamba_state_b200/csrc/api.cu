@@ -265,7 +265,10 @@ int bdscan_kernel_launches(const bdscan_shape_t *shape, int op) {
   // tensor-core path: C B^T pre-pass + scan, plus an aggregate pass and a
   // segment combine when sequences are cut into segments; generic path: one kernel
   if (bdscan::tc_shape_ok(shape->headdim, shape->dstate, shape->block_len, shape->in_dtype == BDSCAN_BF16))
-    return bdscan::tc_plan_segments(shape->batch, shape->nheads, shape->seqlen / shape->block_len) > 1 ? 4 : 2;
+    return bdscan::tc_plan_segments(shape->batch, shape->nheads, shape->seqlen / shape->block_len,
+                                    op == BDSCAN_OP_ALLBLOCK) > 1
+               ? 4
+               : 2;
   return 1;
 }
 

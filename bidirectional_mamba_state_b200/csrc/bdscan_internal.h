@@ -48,7 +48,7 @@ constexpr size_t kWsHeader = 1024;
 // Tensor-core path (sm_100a): bf16 inputs, P = 64, N = 128, T = 32, no gate.
 bool tc_shape_ok(int64_t P, int64_t N, int64_t T, bool in_bf16);
 size_t tc_workspace_bytes(int64_t Bsz, int64_t L, int64_t G, int64_t H, bool allblock);
-int tc_plan_segments(int64_t Bsz, int64_t H, int64_t K);
+int tc_plan_segments(int64_t Bsz, int64_t H, int64_t K, bool allblock);
 bool tc_supported(const ScanArgs &a);
 // Small-batch step without a state chain: C B^T computed in the scan kernel,
 // one launch (see scan_tc.cu).

@@ -1783,18 +1783,33 @@ bool tc_shape_ok(int64_t P, int64_t N, int64_t T, bool in_bf16) {
   return in_bf16 && P == kP && N == kN && T == kT;
 }
 
-// Number of segments each (b, h) sequence is cut into: enough CTAs to fill the
-// machine several times over when there are few sequences (long prefill at
-// batch 1), at least 4 blocks per segment; one segment otherwise.
-int tc_plan_segments(int64_t Bsz, int64_t H, int64_t K) {
+// Number of segments each (b, h) sequence is cut into.  Segments let few long
+// sequences (prefill at batch 1) fill the machine, at the price of an
+// aggregate pass over the clean forward stream (each segment's state from
+// zero), a segment combine and per-item start-up.  The plan minimises a cost
+// in units of one main-pass block step: the main pass's makespan (items run
+// in waves of one per SM; a wave lasts its longest segment), the aggregate
+// pass's (the same waves at kAggCost of a main step), the combine's chain
+// and the two extra launches; one segment when that is cheapest.
+int tc_plan_segments(int64_t Bsz, int64_t H, int64_t K, bool allblock) {
   constexpr int64_t kSms = 148;
+  const double kAggCost = allblock ? 0.45 : 0.6;  // aggregate step / main step, measured
   const int64_t chains = Bsz * H;
-  if (K < 8 || chains >= 2 * kSms) return 1;
-  int64_t nseg = (4 * kSms + chains - 1) / chains;
-  if (nseg > K / 4) nseg = K / 4;
-  if (nseg < 1) nseg = 1;
-  const int64_t seg_blocks = (K + nseg - 1) / nseg;
-  return static_cast<int>((K + seg_blocks - 1) / seg_blocks);
+  if (K < 8 || chains <= 0) return 1;
+  int64_t best = 1;
+  double best_cost = static_cast<double>((chains + kSms - 1) / kSms) * static_cast<double>(K);
+  for (int64_t s = 2; s <= K / 4; ++s) {
+    const int64_t seg_blocks = (K + s - 1) / s;
+    const int64_t nseg = (K + seg_blocks - 1) / seg_blocks;
+    const int64_t waves = (chains * nseg + kSms - 1) / kSms;
+    const double cost = static_cast<double>(waves) * (static_cast<double>(seg_blocks) * (1.0 + kAggCost) + 2.0) +
+                        0.5 * static_cast<double>(nseg) + 4.0;
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = nseg;
+    }
+  }
+  return static_cast<int>(best);
 }
 
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -1805,7 +1820,7 @@ static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 size_t tc_workspace_bytes(int64_t Bsz, int64_t L, int64_t G, int64_t H, bool allblock) {
   const int64_t K = L / kT;
   size_t bytes = align256(static_cast<size_t>(cb_sets(allblock)) * Bsz * K * G * 2048);
-  const int nseg = tc_plan_segments(Bsz, H, K);
+  const int nseg = tc_plan_segments(Bsz, H, K, allblock);
   if (nseg > 1) {
     const size_t states = static_cast<size_t>(Bsz) * H * nseg * kP * kN * sizeof(float);
     bytes += 2 * align256(states) + align256(static_cast<size_t>(Bsz) * H * nseg * sizeof(float));
@@ -1833,7 +1848,7 @@ bool tc_one_launch_step(const ScanArgs &a) {
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return false;
-  return a.Bsz * a.H <= nsm && tc_plan_segments(a.Bsz, a.H, 1) == 1;
+  return a.Bsz * a.H <= nsm && tc_plan_segments(a.Bsz, a.H, 1, false) == 1;
 }
 
 cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
@@ -1920,7 +1935,7 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
   p.H = static_cast<int>(a.H);
   p.G = static_cast<int>(a.G);
   p.K = K;
-  const int nseg = tc_plan_segments(a.Bsz, a.H, K);
+  const int nseg = tc_plan_segments(a.Bsz, a.H, K, all);
   p.nseg = nseg;
   p.seg_blocks = (K + nseg - 1) / nseg;
   p.items = static_cast<int>(a.Bsz * a.H * nseg);

@@ -38,8 +38,9 @@ SMALL = {
     "bf16_segmented": _shape(batch=1, nheads=2, ngroups=1, seqlen=1280),
     # more work items than SMs: each persistent CTA walks several (b, h)
     # sequences, resp. several segments, with the pipeline running across them
+    # (40 sequences of 80 blocks: 7 segments each, 280 items in two waves)
     "bf16_many_items": _shape(batch=5, nheads=64, ngroups=4, seqlen=96),
-    "bf16_segmented_many_items": _shape(batch=1, nheads=40, ngroups=2, seqlen=1280),
+    "bf16_segmented_many_items": _shape(batch=1, nheads=40, ngroups=2, seqlen=2560),
 }
 
 
