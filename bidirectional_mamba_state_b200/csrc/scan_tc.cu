@@ -21,7 +21,7 @@
 // from the same h_{k-1} (the clean boundary state before block k), its
 // reverse part is block-local.
 //
-// Two kernels:
+// Kernels:
 //   bd_cb_kernel  C B^T of every (direction, batch, block, group) -- shared by
 //                 all heads of a group -- with one M=128 tcgen05 MMA chain per
 //                 four blocks, into the workspace (bf16, 2 KB per block; the
@@ -52,6 +52,11 @@
 //                 epilogue lives only in the gated instance of the kernel.
 //   S, Y and M are double-buffered (Y single-buffered with a gate: its five
 //   accumulators fill the TMEM); the h operand is single-buffered.
+//   bd_agg_kernel and bd_seg_combine_kernel  (segmented plans: few long
+//                 sequences cut into segments) each segment's state from a
+//                 zero start as one contraction over its tokens, then the
+//                 chain of segment states; the scan kernel then starts each
+//                 segment from its true initial state.
 // Every wait is bounded; on a timeout the CTA raises BDSCAN_ERR_TIMEOUT in the
 // workspace status word, drains its own copies and MMAs, frees TMEM and exits.
 //
@@ -227,7 +232,7 @@ constexpr uint32_t kOffFtab = kOffDtab + kTab * 16;  // [kTab] s32: 1 + item par
                                                      // 0 at its other steps, -1 past the CTA's last step
 constexpr uint32_t kOffBar = kOffFtab + 128;
 constexpr int kNumBars = 56;
-constexpr int kMaxSlots = 8;  // ring slots of the compact layouts (see Lay)
+constexpr int kMaxSlots = 5;  // ring slots of the compact layout (see Lay)
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // TMEM base, abort flag
 constexpr int kItemRing = 16;
 constexpr uint32_t kOffItemQ = kOffMisc + 64;             // int4[kItemRing]: published work items
@@ -303,14 +308,13 @@ struct TcParams {
   int items;             // Bsz * H * nseg work items, handed out one at a time
   DivU dv_nseg, dv_h, dv_hpg;  // division by nseg, H and H / G
   int *item_counter;     // next unclaimed work item (zeroed by the C B^T kernel)
-  int agg;               // aggregate pass: forward state of each segment from zero, nothing else
-  int need_s;            // the state after a block is used (outputs, next block, aggregate); if not
+  int need_s;            // the state after a block is used (outputs, next block); if not
                          // (one-block items, no state outputs), S, w o X and the state update are skipped
   int allblock;
   int out_bf16;
   const float *seg_init;  // [B][H][nseg][P][N] initial state of every segment (nseg > 1)
-  float *seg_local;       // [B][H][nseg][P][N] aggregate pass: end state from a zero start
-  float *seg_decay;       // [B][H][nseg] aggregate pass: total decay (log2 units)
+  float *seg_local;       // [B][H][nseg][P][N] aggregate kernel: end state from a zero start
+  float *seg_decay;       // [B][H][nseg] aggregate kernel: total decay (log2 units)
   const float *h0;
   float *states;
   float *final_state;
@@ -490,21 +494,13 @@ __device__ __forceinline__ Item item_at(const TcParams &p, int it) {
   return r;
 }
 
-// Block of the sequence that step kk of an item covers: in order, or, in the
-// aggregate pass, from the item's last block to its first (the segment's
-// state is accumulated with weights relative to the segment's end, which are
-// known block by block in that order).
-template <bool kAgg>
-__device__ __forceinline__ int item_block(int k0, int nk, int kk) {
-  return kAgg ? k0 + nk - 1 - kk : k0 + kk;
-}
-
 // barrier ring of the per-step tables: phase parity of step j
 __device__ __forceinline__ uint32_t part(int j) { return (static_cast<uint32_t>(j) / kTab) & 1u; }
 
-// Kernel instances: the call's mode is a template parameter (bits kModeAgg,
-// kModeAll, kModeNeedS), so each instance carries only the code its mode runs.
-enum : int { kModeAgg = 1, kModeAll = 2, kModeNeedS = 4, kModeCbFused = 8 };
+// Kernel instances: the call's mode is a template parameter (bits kModeAll,
+// kModeNeedS, kModeCbFused), so each instance carries only the code its mode
+// runs.  (The aggregate pass of segmented plans is a kernel of its own.)
+enum : int { kModeAll = 2, kModeNeedS = 4, kModeCbFused = 8 };
 
 // Ring-slot layout of an instance.  The all-block pass and the fused-C B^T
 // step keep three 48 KB slots (x of four directions, B_cf, the C tiles of two
@@ -512,21 +508,19 @@ enum : int { kModeAgg = 1, kModeAll = 2, kModeNeedS = 4, kModeCbFused = 8 };
 // one-stream scan and step instances use five 28 KB slots in the same space
 // (x of the two clean directions, B_cf, C_cf, two C B^T tiles), so that the
 // producer runs further ahead of the masked-decay build, which waits for the
-// tiles of the step two ahead; the aggregate pass, which reads only x_cf and
-// B_cf, eight 12 KB slots.
+// tiles of the step two ahead.
 template <int kM>
 struct Lay {
-  static constexpr bool kAggL = (kM & kModeAgg) != 0;
-  static constexpr bool kCompact = (kM & (kModeAll | kModeAgg | kModeCbFused)) == 0;
-  static constexpr int kN = kAggL ? 8 : (kCompact ? 5 : 3);
-  static constexpr uint32_t kBytes = kAggL ? 3 * kTile : (kCompact ? 7 * kTile : 12 * kTile);
-  static constexpr uint32_t kBcf = kAggL ? kTile : (kCompact ? 2 * kTile : 4 * kTile);  // B_cf, n 0..63 then 64..127
+  static constexpr bool kCompact = (kM & (kModeAll | kModeCbFused)) == 0;
+  static constexpr int kN = kCompact ? 5 : 3;
+  static constexpr uint32_t kBytes = kCompact ? 7 * kTile : 12 * kTile;
+  static constexpr uint32_t kBcf = kCompact ? 2 * kTile : 4 * kTile;  // B_cf, n 0..63 then 64..127
   static constexpr uint32_t kClo = kCompact ? 4 * kTile : 6 * kTile;  // C rows x n 0..63
   static constexpr uint32_t kChi = kCompact ? 5 * kTile : 8 * kTile;  // C rows x n 64..127
   static constexpr uint32_t kCbBase = kCompact ? 6 * kTile : 10 * kTile;
   // x tile of direction slot i, C B^T tile of direction slot i
   __host__ __device__ static constexpr uint32_t x(int i) {
-    return kAggL ? 0u : static_cast<uint32_t>(kCompact ? (i >> 1) : i) * kTile;  // the aggregate pass: x_cf only
+    return static_cast<uint32_t>(kCompact ? (i >> 1) : i) * kTile;
   }
   __host__ __device__ static constexpr uint32_t cb(int i) {
     return kCbBase + static_cast<uint32_t>(kCompact ? (i >> 1) : i) * 2048u;
@@ -534,7 +528,7 @@ struct Lay {
   __device__ static int slot(int j) { return j % kN; }
   __device__ static uint32_t par(int j) { return static_cast<uint32_t>(j / kN) & 1u; }
 };
-static_assert(5 * 7 * kTile <= kSlots * kSlot && 8 * 3 * kTile <= kSlots * kSlot, "compact rings within the ring's space");
+static_assert(5 * 7 * kTile <= kSlots * kSlot, "compact ring within the ring's space");
 // kModeCbFused (one-block items without a state chain, no more items than
 // SMs: the batch-1 denoising step): no C B^T pre-pass; each step loads B and C
 // of both directions and computes its own C B^T tiles (one M = 64 MMA chain
@@ -598,13 +592,12 @@ __device__ __forceinline__ int item_warp(const TcParams &p, const Ctl &c, uint32
 // ---------------------------------------------------------------- producer
 template <int kM>
 __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
-  constexpr bool kAgg = kM & kModeAgg, kAll = kM & kModeAll, kCbF = kM & kModeCbFused;
+  constexpr bool kAll = kM & kModeAll, kCbF = kM & kModeCbFused;
   const int nact = p.active[0] + p.active[1] + p.active[2] + p.active[3];
   // x of each active direction, C B^T tiles, B of the clean forward direction
   // (only when S is formed), C of the clean (and noisy) forward direction;
   // with the C B^T tiles computed here: x of both directions, B and C of both
-  const uint32_t bytes = kCbF ? 10 * kTile
-                              : kAgg ? 3 * kTile : nact * (kTile + 2048) + (2 + (kAll ? 4 : 2)) * kTile;
+  const uint32_t bytes = kCbF ? 10 * kTile : nact * (kTile + 2048) + (2 + (kAll ? 4 : 2)) * kTile;
 #pragma unroll
   for (int i = 0; i < 4; ++i)
     if (p.active[i]) tma_prefetch_desc(&p.tx[i]);
@@ -641,7 +634,7 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
   for (int m = 0; ok && cur >= 0; ++m) {
     const Item I = Icur;
     for (int kk = 0; kk < I.nk; ++kk, ++j) {
-      const int k = item_block<kAgg>(I.k0, I.nk, kk);  // block index in the sequence
+      const int k = I.k0 + kk;  // block index in the sequence
       const int r = Ly::slot(j);
       if (!wait1(c, bEmpty0 + r, Ly::par(j) ^ 1)) {
         ok = false;
@@ -670,24 +663,22 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
           if (p.active[i]) tma_load_4d_s(st + Ly::x(i), &p.tx[i], full, 0, I.h, t0, I.b);
         tma_load_4d_s(st + Ly::kBcf, &p.tbcf, full, 0, I.g, t0, I.b);
         tma_load_4d_s(st + Ly::kBcf + kTile, &p.tbcf, full, 64, I.g, t0, I.b);
-        if (!kAgg) {
-          tma_load_4d_s(st + Ly::kClo, &p.tccf, full, 0, I.g, t0, I.b);
-          tma_load_4d_s(st + Ly::kChi, &p.tccf, full, 64, I.g, t0, I.b);
-          if (kAll) {
-            tma_load_4d_s(st + Ly::kClo + kTile, &p.tcnf, full, 0, I.g, t0, I.b);
-            tma_load_4d_s(st + Ly::kChi + kTile, &p.tcnf, full, 64, I.g, t0, I.b);
-          }
-          // C B^T tiles: written by the pre-pass this kernel may overlap
-          if (!waited) {
-            wait_prior_grid();
-            waited = true;
-          }
+        tma_load_4d_s(st + Ly::kClo, &p.tccf, full, 0, I.g, t0, I.b);
+        tma_load_4d_s(st + Ly::kChi, &p.tccf, full, 64, I.g, t0, I.b);
+        if (kAll) {
+          tma_load_4d_s(st + Ly::kClo + kTile, &p.tcnf, full, 0, I.g, t0, I.b);
+          tma_load_4d_s(st + Ly::kChi + kTile, &p.tcnf, full, 64, I.g, t0, I.b);
+        }
+        // C B^T tiles: written by the pre-pass this kernel may overlap
+        if (!waited) {
+          wait_prior_grid();
+          waited = true;
+        }
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            if (!p.active[i]) continue;
-            const int idx = ((cb_set(kAll, i) * p.Bsz + I.b) * p.K + k) * p.G + I.g;
-            tma_load_3d_s(st + Ly::cb(i), &p.tcb, full, 0, 0, idx);
-          }
+        for (int i = 0; i < 4; ++i) {
+          if (!p.active[i]) continue;
+          const int idx = ((cb_set(kAll, i) * p.Bsz + I.b) * p.K + k) * p.G + I.g;
+          tma_load_3d_s(st + Ly::cb(i), &p.tcb, full, 0, 0, idx);
         }
       }
 #pragma unroll
@@ -715,7 +706,7 @@ __device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
 // Descriptors are built once; per step only their start addresses move.
 template <int kM, bool kGated>
 __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
-  constexpr bool kAgg = kM & kModeAgg, kAll = kM & kModeAll, kNeedS = kM & kModeNeedS, kCbF = kM & kModeCbFused;
+  constexpr bool kAll = kM & kModeAll, kNeedS = kM & kModeNeedS, kCbF = kM & kModeCbFused;
   const uint32_t id_s = idesc_bf16(128, 64, 1, 1);  // S^T[n][p] = B^T (w o X)
   // Y_off^T[p][t] = h C^T over the stacked [C_cf; C_nf] rows (only C_cf without a noisy stream)
   const uint32_t id_yo = kAll ? idesc_bf16(64, 64, 1, 0) : idesc_bf16(64, 32, 1, 0);
@@ -756,26 +747,6 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
                     dC + so + ko + (ks < 4 ? 0u : BD_OFF(Ly::kChi - Ly::kClo)), id_cb, ks > 0);
         }
         umma_commit_s(bar_at(c, bCbFull));
-      }
-      if constexpr (kAgg) {
-        // ---- aggregate pass: S^T of the item accumulates over its blocks
-        //      (walked last to first, w o X weighted to the item's end) in the
-        //      item's buffer; the state group reads it once, at the item's end
-        if (!wait1(c, bXwFull0 + i2, par2(j))) break;
-        const int sb = m & 1;
-        if (kk == 0 && m >= 2 && !wait1(c, bSEmpty0 + sb, ((m - 2) >> 1) & 1)) break;
-        tc_fence_after();
-        const uint32_t colS = tmem + kColS0 + 64 * sb;
-        const D64 dxw = dXw + (i2 ? BD_OFF(kOffH - kOffXw) : 0u);
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-          umma_bf16(colS, dBcf + so + BD_OFF(ks * 2048), dxw + BD_OFF(ks * 2048), id_s, (kk > 0 || ks > 0) ? 1u : 0u);
-          umma_bf16(colS, dBcf + so + BD_OFF(ks * 2048), dxw + BD_OFF(kTile + ks * 2048), id_s, 1);
-        }
-        umma_commit_s(bar_at(c, bEmpty0 + r));
-        if (kk + 1 == nk) umma_commit_s(bar_at(c, bSFull0 + sb));
-        ok = true;
-        continue;
       }
       // ---- S^T = B_cf^T (w o X): A MN-major (n; halves 4 KB apart), B MN-major (p)
       if (kNeedS) {
@@ -959,7 +930,7 @@ __device__ __forceinline__ void build_masked_decay_tm(uint32_t base, uint32_t tm
 // The masked-decay matrices are built by the epilogue warps.
 template <int kM>
 __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
-  constexpr bool kAgg = kM & kModeAgg, kNeedS = kM & kModeNeedS;
+  constexpr bool kNeedS = kM & kModeNeedS;
   const int lane = threadIdx.x & 31;
   const int wq = threadIdx.x >> 5;
   const int q = wq < 4 ? wq - 2 : wq - 4;
@@ -991,7 +962,7 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
     if (!cv) return;
     if (act) {
       qdt[e] = __bfloat162float(
-          dtp[(static_cast<int64_t>(CI.b) * L + item_block<kAgg>(CI.k0, CI.nk, ckk) * kT + lane) * H + CI.h]);
+          dtp[(static_cast<int64_t>(CI.b) * L + (CI.k0 + ckk) * kT + lane) * H + CI.h]);
       qa[e] = Ap[CI.h] * kLog2e;
     }
     if (dact) qd[e] = Dp[CI.h];
@@ -1011,7 +982,6 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
   cursor_load(1);
   if (!cursor_next()) return;
   int j = 0;
-  float rdec = 0.f;  // aggregate pass: decay (log2) of the item's blocks after this one
   for (int m = 0;; ++m) {
     bool has_next = false;
     Item In = I;
@@ -1050,23 +1020,11 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
       if (!waitw(c, bFull0 + Lay<kM>::slot(j), Lay<kM>::par(j))) return;
       // ---- (w o X) of the clean forward direction, bf16 hi + lo
       if (kNeedS) {
-        uint32_t xw = base + kOffXw;
-        float rw = 0.f;  // log2 weight of the block's end relative to the item's end
-        if constexpr (kAgg) {
-          // two w o X buffers (the h operand's space is free in this pass):
-          // the S MMAs of step j - 2 have read this one once their commit
-          // completed the ring slot's empty phase of that step
-          if (kk == 0) rdec = 0.f;
-          rw = rdec;
-          if (j & 1) xw = base + kOffH;
-          if (j >= 2 && !waitw(c, bEmpty0 + Lay<kM>::slot(j - 2), Lay<kM>::par(j - 2))) return;
-        } else {
-          // the S MMA of the previous step has read the w o X buffer
-          if (j >= 1 && !waitw(c, bSFull0 + ((j - 1) & 1), par2(j - 1))) return;
-        }
+        const uint32_t xw = base + kOffXw;
+        // the S MMA of the previous step has read the w o X buffer
+        if (j >= 1 && !waitw(c, bSFull0 + ((j - 1) & 1), par2(j - 1))) return;
         const uint32_t cf = cum + (ct * 4 + kCF) * 128, df = dts + (ct * 4 + kCF) * 128;
         const float c31 = lds_f32(cf + 31 * 4);
-        if constexpr (kAgg) rdec += c31;
 #pragma unroll
         for (int rep = 0; rep < 2; ++rep) {
           const int i = gt + 128 * rep;
@@ -1074,7 +1032,7 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
           const uint32_t off = sw128_chunk(t, ch);
           uint32_t r0, r1, r2, r3;
           ld_shared_v4(st + Lay<kM>::x(kCF) + off, r0, r1, r2, r3);
-          const float w = lds_f32(df + t * 4) * ex2_approx(c31 - lds_f32(cf + t * 4) + rw);
+          const float w = lds_f32(df + t * 4) * ex2_approx(c31 - lds_f32(cf + t * 4));
           float vv[8] = {bf16_lo_f(r0) * w, bf16_hi_f(r0) * w, bf16_lo_f(r1) * w, bf16_hi_f(r1) * w,
                          bf16_lo_f(r2) * w, bf16_hi_f(r2) * w, bf16_lo_f(r3) * w, bf16_hi_f(r3) * w};
           store_split8(xw + off, xw + kTile + off, vv);
@@ -1181,61 +1139,17 @@ __device__ void state_group_staged(const TcParams &p, const Ctl &c, uint32_t bas
   }
 }
 
-// Aggregate pass: an item's S^T accumulates over all its blocks in TMEM (the
-// issuer walks them last to first with weights relative to the item's end), so
-// the group only adds up the item's total decay from the per-step tables and,
-// after its last block, stores the accumulated state (the segment's end state
-// from a zero start) and that decay.
-__device__ void state_group_agg(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
-  const int lane = threadIdx.x & 31;
-  const int q = (threadIdx.x >> 5) & 3;
-  const int n = 32 * q + lane;
-  const uint32_t cum = base + kOffCum;
-  const int64_t PN = kP * kN;
-  int j = 0;
-  for (int m = 0;; ++m) {
-    Item I;
-    if (item_warp(p, c, base, m, I) <= 0) return;
-    float decay_log2 = 0.f;
-    for (int kk = 0; kk < I.nk; ++kk, ++j) {
-      const int ct = j % kTab;
-      if (!waitw(c, bAux0 + ct, part(j))) return;
-      decay_log2 += lds_f32(cum + ((ct * 4 + kCF) * 32 + 31) * 4);
-    }
-    const int sb = m & 1;
-    if (!waitw(c, bSFull0 + sb, (m >> 1) & 1)) return;
-    tc_fence_after();
-    const int64_t ebhs = (static_cast<int64_t>(I.b) * p.H + I.h) * p.nseg + I.seg;
-    float *dst = p.seg_local + ebhs * PN + n;
-    const uint32_t ta = tmem_addr(tmem, 32 * q, kColS0 + 64 * sb);
-#pragma unroll
-    for (int cq = 0; cq < 4; ++cq) {
-      uint32_t sv[16];
-      tmem_ld_32x32b_x16(ta + 16 * cq, sv);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 16; ++i) dst[(16 * cq + i) * kN] = __uint_as_float(sv[i]);
-    }
-    if (n == 0) p.seg_decay[ebhs] = decay_log2;
-    tc_fence_before();
-    arrive_lane0(c, bSEmpty0 + sb);
-  }
-}
-
 // warps 8..11: thread owns column n = 32 q + lane of the state, h^T[n][0..63].
 // A failed (timed-out) wait ends the group at once: nothing else is stored.
 template <int kM>
 __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
-  constexpr bool kAgg = kM & kModeAgg, kNeedS = kM & kModeNeedS;
+  constexpr bool kNeedS = kM & kModeNeedS;
   const int lane = threadIdx.x & 31;
   const int q = (threadIdx.x >> 5) & 3;
   const int n = 32 * q + lane;
   const uint32_t cum = base + kOffCum;
   if constexpr (!kNeedS) {
     state_group_staged(p, c, base, tmem);
-    return;
-  } else if constexpr (kAgg) {
-    state_group_agg(p, c, base, tmem);
     return;
   }
   const int64_t H = p.H;
@@ -1271,19 +1185,16 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
       nk = I.nk;
       const int64_t bh = static_cast<int64_t>(I.b) * H + I.h;
       sdst = p.states ? p.states + ((static_cast<int64_t>(I.b) * p.K + I.k0) * H + I.h) * PN + n : nullptr;
-      // initial state of this item: h0 (first segment), the chained state the
-      // aggregate and combine passes left in the workspace (later segments),
-      // or zero (aggregate pass)
-      const float *src = kAgg ? nullptr
-                         : I.seg == 0 ? (p.h0 ? p.h0 + bh * PN + n : nullptr)
-                                      : p.seg_init + (bh * p.nseg + I.seg) * PN + n;
+      // initial state of this item: h0 (first segment) or the chained state
+      // the aggregate and combine kernels left in the workspace (later segments)
+      const float *src = I.seg == 0 ? (p.h0 ? p.h0 + bh * PN + n : nullptr)
+                                    : p.seg_init + (bh * p.nseg + I.seg) * PN + n;
       if (src && I.seg > 0) wait_prior_grid();  // segment states: written by the combine kernel
 #pragma unroll
       for (int pp = 0; pp < kP; ++pp) hreg[pp] = src ? src[pp * kN] : 0.f;
     }
-    float decay_log2 = 0.f;  // total decay over the item (aggregate pass)
     for (int kk = 0;; ++kk) {
-      if (kk < nk && !kAgg) {
+      if (kk < nk) {
         // Y_off of the previous step has read the h operand; the state
         // entering this block replaces it
         if (j >= 1 && !waitw(c, bHCons, (j - 1) & 1)) return;
@@ -1293,19 +1204,13 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
 #pragma unroll 1
         for (int d = 0; d < 2; ++d) {
           float *dst = sdst;
-          if (d == 1) {  // after the item's last block: final or segment state
+          if (d == 1) {  // after the item's last block: the final state
             dst = nullptr;
             if (kk == nk && !aborted(c)) {
               Item E;  // (re-read from the ring: its entry is not reused before every role moved on)
               (void)item_read(p, base, m, E);
               const int64_t ebh = static_cast<int64_t>(E.b) * H + E.h;
-              if (kAgg) {
-                const int64_t ebhs = ebh * p.nseg + E.seg;
-                dst = p.seg_local + ebhs * PN + n;
-                if (n == 0) p.seg_decay[ebhs] = decay_log2;
-              } else if (p.final_state && E.k0 + E.nk == p.K) {
-                dst = p.final_state + ebh * PN + n;
-              }
+              if (p.final_state && E.k0 + E.nk == p.K) dst = p.final_state + ebh * PN + n;
             }
           }
           if (dst) {  // each warp instruction stores one contiguous 128-byte row segment
@@ -1320,7 +1225,6 @@ __device__ void state_group(const TcParams &p, const Ctl &c, uint32_t base, uint
       if (!waitw(c, bAux0 + ct, part(j))) return;
       const float c31 = lds_f32(cum + ((ct * 4 + kCF) * 32 + 31) * 4);
       const float atot = ex2_approx(c31);
-      decay_log2 += c31;
       if (!waitw(c, bSFull0 + i2, par2(j))) return;
       tc_fence_after();
       {
@@ -1360,7 +1264,7 @@ __device__ __noinline__ void store_y_bf16(__nv_bfloat16 *dst, int64_t tstride, c
 // direction slot q, row s = lane of M^T) and the diagonal's bf16 remainders.
 template <int kM, bool kGated>
 __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
-  constexpr bool kAgg = kM & kModeAgg, kAll = kM & kModeAll, kNeedS = kM & kModeNeedS, kCbF = kM & kModeCbFused;
+  constexpr bool kAll = kM & kModeAll, kNeedS = kM & kModeNeedS, kCbF = kM & kModeCbFused;
   const int lane = threadIdx.x & 31;
   const int q = (threadIdx.x >> 5) & 3;
   const int pcol = 16 * q + (lane & 15);
@@ -1370,7 +1274,6 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
   const bool mine = (noisy ? kAll : true) && yout != nullptr;
   const uint32_t cumt = base + kOffCum;
   const int64_t H = p.H, L = p.L;
-  if constexpr (kAgg) return;
   const bool act = pick4(p.active, q) != 0;
   const bool rev = q >= 2;
   int mla = 0;        // next step whose masked-decay matrices this group builds
@@ -1567,7 +1470,6 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
 // nothing to the instruction footprint of the ungated one.
 template <int kM, bool kGated>
 __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constant__ TcParams p) {
-  constexpr bool kAgg = kM & kModeAgg;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -1599,7 +1501,7 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
   }
   // Clear the intra-block operands: of their remainder halves only the
   // diagonals are ever written.
-  if (!kAgg) {
+  {
     const uint4 zero = make_uint4(0, 0, 0, 0);
     for (uint32_t o = threadIdx.x * 16; o < 2 * kMhBuf; o += kThreads * 16)
       *reinterpret_cast<uint4 *>(sm + kOffMh + o) = zero;
@@ -1657,6 +1559,327 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
   if (warp == 1) {
     __syncwarp();
     tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ aggregate pass
+// Each segment's forward state from a zero start and its total decay, the
+// input of the segment combine.  Unrolling [BDLM-PR] eq. (1) over a segment,
+//   S_seg = sum_t w_t x_t B_t^T,   w_t = dt_t exp(sum_{u > t in seg} dt_u A),
+// one dense contraction per segment, S^T[n][p] = B^T (w o X) over the
+// segment's tokens, with no per-block state chain.  It is taken 128 tokens
+// (four blocks) per pipeline step, from the segment's last step to its first,
+// so that the weights relative to the segment's end are known step by step
+// (a running sum of the later steps' decays).  w o X is split into bf16
+// hi + lo (two MMAs per 16 tokens); S^T accumulates in TMEM (lane n, 64
+// columns p), two buffers so that a segment's readout overlaps the next
+// segment's MMAs.  Warps: 0 the TMA producer (x and B tiles, a three-step
+// ring), 1 the MMA issuer and TMEM owner, 2..5 the operands (warp 2 + w
+// builds block w of a step) and, at a segment's end, the readout (TMEM lanes
+// 32 (warp % 4) ..).  Work items (b, h, segment) go round-robin: item
+// blockIdx.x + m gridDim.x.
+namespace agg {
+constexpr int kBlocks = 4;                          // blocks per pipeline step
+constexpr int kStages = 3;                          // TMA ring depth
+constexpr uint32_t kStB = kBlocks * kTile;          // B tiles within a stage (x tiles first)
+constexpr uint32_t kStage = 3 * kBlocks * kTile;    // x: one tile per block; B: two per block
+constexpr uint32_t kXwBuf = 2 * kBlocks * kTile;    // w o X {hi, lo} per block
+constexpr uint32_t kOffXw = kStages * kStage;       // two w o X buffers
+constexpr uint32_t kOffBar = kOffXw + 2 * kXwBuf;
+enum : int {
+  bFull = 0,
+  bEmpty = bFull + kStages,
+  bXwFull = bEmpty + kStages,
+  bXwEmpty = bXwFull + 2,
+  bSFull = bXwEmpty + 2,
+  bSEmpty = bSFull + 2,
+  bDrain = bSEmpty + 2,
+  bCount
+};
+constexpr uint32_t kOffMisc = kOffBar + 8 * bCount;  // control block (layout of Ctl)
+constexpr uint32_t kSmem = kOffMisc + 32 + 1024;     // + alignment of the base to 1 KB
+constexpr int kThreadsAgg = 192;
+constexpr uint32_t kCols = 128;  // two S^T buffers of 64 columns
+static_assert(kSmem <= 227 * 1024, "aggregate kernel shared memory");
+
+struct Seg {
+  int b, h, g, seg, k0, nk;
+};
+// This CTA's m-th item; false past the last.
+__device__ __forceinline__ bool item(const TcParams &p, int m, Seg &I) {
+  const int it = static_cast<int>(blockIdx.x) + m * static_cast<int>(gridDim.x);
+  if (it >= p.items) return false;
+  const int bh = it / p.nseg;
+  I.seg = it - bh * p.nseg;
+  I.b = bh / p.H;
+  I.h = bh - I.b * p.H;
+  I.g = I.h / (p.H / p.G);
+  I.k0 = I.seg * p.seg_blocks;
+  I.nk = min(p.K - I.k0, p.seg_blocks);
+  return true;
+}
+__device__ __forceinline__ int steps(const Seg &I) { return (I.nk + kBlocks - 1) / kBlocks; }
+// Step ci of an item (0: its last four blocks): first block kb, nb blocks.
+__device__ __forceinline__ void step_blocks(const Seg &I, int ci, int &kb, int &nb) {
+  const int hi = I.k0 + I.nk - kBlocks * ci;
+  kb = max(I.k0, hi - kBlocks);
+  nb = hi - kb;
+}
+__device__ __forceinline__ uint32_t doff(uint32_t bytes) { return bytes >> 4; }
+
+__device__ void producer(const TcParams &p, const Ctl &c, uint32_t base) {
+  tma_prefetch_desc(&p.tx[kCF]);
+  tma_prefetch_desc(&p.tbcf);
+  int last[kStages] = {-1, -1, -1};
+  int j = 0;
+  Seg I;
+  for (int m = 0; item(p, m, I); ++m) {
+    const int nc = steps(I);
+    for (int ci = 0; ci < nc; ++ci, ++j) {
+      const int s = j % kStages;
+      const uint32_t par = static_cast<uint32_t>(j / kStages) & 1u;
+      if (!wait1(c, bEmpty + s, par ^ 1u)) goto drain;
+      int kb, nb;
+      step_blocks(I, ci, kb, nb);
+      const uint32_t full = bar_at(c, bFull + s);
+      mbar_arrive_expect_tx_s(full, static_cast<uint32_t>(nb) * 3u * kTile);
+      const uint32_t st = base + static_cast<uint32_t>(s) * kStage;
+      for (int bi = 0; bi < nb; ++bi) {
+        const int t0 = (kb + bi) * kT;
+        tma_load_4d_s(st + bi * kTile, &p.tx[kCF], full, 0, I.h, t0, I.b);
+        tma_load_4d_s(st + kStB + bi * 2 * kTile, &p.tbcf, full, 0, I.g, t0, I.b);
+        tma_load_4d_s(st + kStB + bi * 2 * kTile + kTile, &p.tbcf, full, 64, I.g, t0, I.b);
+      }
+#pragma unroll
+      for (int r = 0; r < kStages; ++r)
+        if (r == s) last[r] = j;
+    }
+  }
+drain:
+  // no copy into this CTA's shared memory may still be in flight at exit
+#pragma unroll
+  for (int s = 0; s < kStages; ++s)
+    if (last[s] >= 0)
+      (void)mbar_wait_s(bar_at(c, bFull + s), static_cast<uint32_t>(last[s] / kStages) & 1u, p.drain_ns, 0);
+}
+
+// ---- MMA issuer
+__device__ void issuer(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
+  const uint32_t id_s = idesc_bf16(128, 64, 1, 1);  // S^T[n][p] = B^T (w o X): both MN-major
+  const D64 dB = split64(sdesc(base + kStB, kTile, 1024, kLayoutSw128));  // n 0..63, 64..127 one tile apart
+  const D64 dXw = split64(sdesc(base + kOffXw, 0, 1024, kLayoutSw128));
+  int j = 0;
+  Seg I;
+  for (int m = 0; item(p, m, I); ++m) {
+    const int nc = steps(I), sb = m & 1;
+    const uint32_t colS = tmem + 64u * static_cast<uint32_t>(sb);
+    // the readout of item m - 2 has emptied this accumulator
+    if (!wait1(c, bSEmpty + sb, (static_cast<uint32_t>(m >> 1) & 1u) ^ 1u)) break;
+    bool ok = true;
+    for (int ci = 0; ci < nc; ++ci, ++j) {
+      const int s = j % kStages, xb = j & 1;
+      if (!wait1(c, bFull + s, static_cast<uint32_t>(j / kStages) & 1u) ||
+          !wait1(c, bXwFull + xb, static_cast<uint32_t>(j >> 1) & 1u)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      int kb, nb;
+      step_blocks(I, ci, kb, nb);
+      const uint32_t so = doff(static_cast<uint32_t>(s) * kStage), xo = doff(static_cast<uint32_t>(xb) * kXwBuf);
+#pragma unroll 1
+      for (int bi = 0; bi < nb; ++bi) {
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+          const uint32_t ob = doff(static_cast<uint32_t>(bi) * 2u * kTile + static_cast<uint32_t>(ks) * 2048u);
+          umma_bf16(colS, dB + so + ob, dXw + xo + ob, id_s, (ci > 0 || bi > 0 || ks > 0) ? 1u : 0u);
+          umma_bf16(colS, dB + so + ob, dXw + xo + ob + doff(kTile), id_s, 1u);
+        }
+      }
+      umma_commit_s(bar_at(c, bEmpty + s));
+      umma_commit_s(bar_at(c, bXwEmpty + xb));
+      if (ci + 1 == nc) umma_commit_s(bar_at(c, bSFull + sb));
+    }
+    if (!ok) break;
+  }
+  // every MMA issued has completed before TMEM is released
+  umma_commit_s(bar_at(c, bDrain));
+  (void)mbar_wait_s(bar_at(c, bDrain), 0, p.drain_ns, 0);
+}
+
+// ---- operand warps 2..5 (w = warp - 2 builds block w of each step)
+// Every lane loads dt of its token in all four blocks of a step (two steps
+// ahead), so that each warp forms the four blocks' decay sums itself and
+// the group needs no exchange: per step, with v_k = dt A (log2 units) of
+// block k, the warp's own suffix sums give sum_{u > t} over its block, the
+// later blocks' totals and the running sum of the later steps the rest.
+__device__ void operands(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
+  const int lane = threadIdx.x & 31, w = (threadIdx.x >> 5) - 2;
+  const int q = (threadIdx.x >> 5) & 3;  // TMEM lane quadrant of this warp
+  const int64_t H = p.H, L = p.L, PN = kP * kN;
+  const __nv_bfloat16 *dtp = p.dt[kCF];
+  const float *Ap = p.A[kCF];
+  // cursor over (item, step) for the loads two steps ahead
+  int cm = 0, cci = 0;
+  Seg CI;
+  bool cv = item(p, 0, CI);
+  float qdt[2][kBlocks], qa[2];
+  auto load = [&](int e) {
+    qa[e] = 0.f;
+#pragma unroll
+    for (int k = 0; k < kBlocks; ++k) qdt[e][k] = 0.f;
+    if (!cv) return;
+    int kb, nb;
+    step_blocks(CI, cci, kb, nb);
+    qa[e] = Ap[CI.h] * kLog2e;
+    const __nv_bfloat16 *src = dtp + (static_cast<int64_t>(CI.b) * L + static_cast<int64_t>(kb) * kT + lane) * H + CI.h;
+#pragma unroll
+    for (int k = 0; k < kBlocks; ++k)
+      if (k < nb) qdt[e][k] = __bfloat162float(src[static_cast<int64_t>(k) * kT * H]);
+  };
+  auto advance = [&]() {
+    if (!cv) return;
+    if (++cci < steps(CI)) return;
+    cci = 0;
+    cv = item(p, ++cm, CI);
+  };
+  load(0);
+  advance();
+  load(1);
+  advance();
+  int j = 0;
+  Seg I;
+  for (int m = 0; item(p, m, I); ++m) {
+    const int nc = steps(I);
+    float later_steps = 0.f;  // decay (log2) of the item's steps after this one
+    for (int ci = 0; ci < nc; ++ci, ++j) {
+      const int s = j % kStages, xb = j & 1;
+      float dtk[kBlocks];
+#pragma unroll
+      for (int k = 0; k < kBlocks; ++k) {
+        dtk[k] = qdt[0][k];
+        qdt[0][k] = qdt[1][k];
+      }
+      const float A2 = qa[0];
+      qa[0] = qa[1];
+      load(1);
+      advance();
+      // decays: totals of the four blocks (every lane) and this warp's block's
+      // inclusive suffix sums
+      float tot[kBlocks], own = 0.f, dt_own = 0.f;
+#pragma unroll
+      for (int k = 0; k < kBlocks; ++k) {
+        const float v = dtk[k] * A2;
+        float r = v;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+        tot[k] = r;
+        if (k == w) {
+          own = v;
+          dt_own = dtk[k];
+        }
+      }
+      float suf = own;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_down_sync(0xffffffffu, suf, o);
+        if (lane + o < 32) suf += u;
+      }
+      float later = later_steps + (suf - own);
+#pragma unroll
+      for (int k = 0; k < kBlocks; ++k)
+        if (k > w) later += tot[k];
+      const float wt = dt_own * ex2_approx(later);
+      later_steps += (tot[0] + tot[1]) + (tot[2] + tot[3]);
+      // x of this step has landed; the MMAs of step j - 2 have read this buffer
+      if (!waitw(c, bFull + s, static_cast<uint32_t>(j / kStages) & 1u)) return;
+      if (!waitw(c, bXwEmpty + xb, (static_cast<uint32_t>(j >> 1) & 1u) ^ 1u)) return;
+      int kb, nb;
+      step_blocks(I, ci, kb, nb);
+      if (w < nb) {
+        // row `lane` of block w: 64 values of x, scaled by w_t, as bf16 hi + lo
+        const uint32_t xs = base + static_cast<uint32_t>(s) * kStage + static_cast<uint32_t>(w) * kTile;
+        const uint32_t xh = base + kOffXw + static_cast<uint32_t>(xb) * kXwBuf + static_cast<uint32_t>(w) * 2u * kTile;
+#pragma unroll 2
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint32_t off = sw128_chunk(static_cast<uint32_t>(lane), static_cast<uint32_t>(ch));
+          uint32_t r0, r1, r2, r3;
+          ld_shared_v4(xs + off, r0, r1, r2, r3);
+          float vv[8] = {bf16_lo_f(r0) * wt, bf16_hi_f(r0) * wt, bf16_lo_f(r1) * wt, bf16_hi_f(r1) * wt,
+                         bf16_lo_f(r2) * wt, bf16_hi_f(r2) * wt, bf16_lo_f(r3) * wt, bf16_hi_f(r3) * wt};
+          store_split8(xh + off, xh + kTile + off, vv);
+        }
+        fence_proxy_async_smem();
+      }
+      arrive_lane0(c, bXwFull + xb);
+    }
+    // ---- readout: S^T (lane n = 32 q + lane, columns p) and the decay
+    const int sb = m & 1;
+    if (!waitw(c, bSFull + sb, static_cast<uint32_t>(m >> 1) & 1u)) return;
+    tc_fence_after();
+    const int64_t ebhs = (static_cast<int64_t>(I.b) * p.H + I.h) * p.nseg + I.seg;
+    float *dst = p.seg_local + ebhs * PN + 32 * q + lane;
+    const uint32_t ta = tmem_addr(tmem, 32u * static_cast<uint32_t>(q), 64u * static_cast<uint32_t>(sb));
+#pragma unroll 1
+    for (int cq = 0; cq < 4; ++cq) {
+      uint32_t sv[16];
+      tmem_ld_32x32b_x16(ta + 16u * static_cast<uint32_t>(cq), sv);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) dst[(16 * cq + i) * kN] = __uint_as_float(sv[i]);
+    }
+    if (w == 0 && lane == 0) p.seg_decay[ebhs] = later_steps;
+    tc_fence_before();
+    arrive_lane0(c, bSEmpty + sb);
+  }
+}
+}  // namespace agg
+
+__global__ void __launch_bounds__(agg::kThreadsAgg, 1) bd_agg_kernel(const __grid_constant__ TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t *sm = smem_raw + (base - raw);
+  const int warp = threadIdx.x >> 5;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + agg::kOffBar);
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(sm + agg::kOffMisc);
+  if (threadIdx.x == 0) {
+    // full: producer + TMA bytes; empty, xw-empty, S-full, drain: one MMA
+    // commit; xw-full, S-empty: the four operand warps
+    for (int i = 0; i < agg::bCount; ++i)
+      mbar_init(&bars[i], (i >= agg::bXwFull && i < agg::bXwFull + 2) || (i >= agg::bSEmpty && i < agg::bSEmpty + 2) ? 4u : 1u);
+    *reinterpret_cast<volatile int *>(sm + agg::kOffMisc + 4) = 0;
+    *reinterpret_cast<unsigned long long *>(sm + agg::kOffMisc + 8) = p.timeout_ns;
+    *reinterpret_cast<int **>(sm + agg::kOffMisc + 16) = p.status;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, agg::kCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const Ctl c{smem_u32(bars), base + agg::kOffMisc};
+  // Launched as a programmatic dependent of the C B^T pre-pass, whose CTAs
+  // trigger only after every earlier kernel on the stream has completed: the
+  // inputs are ready; the pre-pass's own output is not read here.
+  if (warp == 0) {
+    if ((threadIdx.x & 31) == 0) agg::producer(p, c, base);
+  } else if (warp == 1) {
+    if ((threadIdx.x & 31) == 0) agg::issuer(p, c, base, tmem);
+  } else {
+    agg::operands(p, c, base, tmem);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // this grid completes after the pre-pass, as a plain launch would
+  wait_prior_grid();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, agg::kCols);
   }
 }
 
@@ -1731,10 +1954,10 @@ cudaError_t launch_instance(const cudaLaunchConfig_t &cfg, const TcParams &p) {
 
 // The scan kernel as a programmatic dependent launch (its prologue may overlap
 // the previous kernel in the stream; it waits for that kernel before reading),
-// in the instance of the call's mode: the aggregate pass, the all-block pass,
-// a scan with a state chain (per-block or final state), or one-block items
-// without one (with the C B^T tiles from the pre-pass or computed in the
-// kernel); each but the first with or without a gate.
+// in the instance of the call's mode: the all-block pass, a scan with a state
+// chain (per-block or final state), or one-block items without one (with the
+// C B^T tiles from the pre-pass or computed in the kernel); each with or
+// without a gate.
 cudaError_t launch_scan(unsigned grid, cudaStream_t stream, const TcParams &p) {
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
@@ -1748,9 +1971,7 @@ cudaError_t launch_scan(unsigned grid, cudaStream_t stream, const TcParams &p) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e;
-  if (p.agg)
-    e = launch_instance<kModeAgg | kModeNeedS, false>(cfg, p);
-  else if (p.allblock)
+  if (p.allblock)
     e = p.gated ? launch_instance<kModeAll | kModeNeedS, true>(cfg, p)
                 : launch_instance<kModeAll | kModeNeedS, false>(cfg, p);
   else if (p.need_s)
@@ -1759,6 +1980,27 @@ cudaError_t launch_scan(unsigned grid, cudaStream_t stream, const TcParams &p) {
     e = p.gated ? launch_instance<kModeCbFused, true>(cfg, p) : launch_instance<kModeCbFused, false>(cfg, p);
   else
     e = p.gated ? launch_instance<0, true>(cfg, p) : launch_instance<0, false>(cfg, p);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+// The aggregate pass as a programmatic dependent of the C B^T pre-pass (its
+// prologue overlaps the pre-pass's tail), one CTA per SM at most.
+cudaError_t launch_agg(unsigned grid, cudaStream_t stream, const TcParams &p) {
+  cudaError_t e = cudaFuncSetAttribute(bd_agg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(agg::kSmem));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(agg::kThreadsAgg);
+  cfg.dynamicSmemBytes = agg::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, bd_agg_kernel, p);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
@@ -1793,7 +2035,7 @@ bool tc_shape_ok(int64_t P, int64_t N, int64_t T, bool in_bf16) {
 // and the two extra launches; one segment when that is cheapest.
 int tc_plan_segments(int64_t Bsz, int64_t H, int64_t K, bool allblock) {
   constexpr int64_t kSms = 148;
-  const double kAggCost = allblock ? 0.45 : 0.6;  // aggregate step / main step, measured
+  const double kAggCost = allblock ? 0.13 : 0.2;  // aggregate / main pass time per block, measured
   const int64_t chains = Bsz * H;
   if (K < 8 || chains <= 0) return 1;
   int64_t best = 1;
@@ -1880,8 +2122,8 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
   cp.K = K;
   cp.G = static_cast<int>(a.G);
   cp.cb = cbws;
-  // work-item counters of the aggregate [0] and main [1] scan passes, in the
-  // workspace header next to the status word
+  // work-item counters ([1]: the scan kernel's), in the workspace header next
+  // to the status word; the pre-pass zeroes both
   int *counters = reinterpret_cast<int *>(static_cast<uint8_t *>(a.ws) + kCounterOffset);
   cp.item_counters = counters;
   cp.status = a.status;
@@ -1957,8 +2199,8 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
   // persistent CTAs, one per SM, each walking its share of the work items
   const unsigned grid = static_cast<unsigned>(p.items < nsm ? p.items : nsm);
   if (nseg > 1) {
-    // aggregate pass (clean forward state of every segment from zero), then
-    // the chain of segment states
+    // aggregate kernel (clean forward state of every segment from zero, items
+    // round-robin over the CTAs), then the chain of segment states
     uint8_t *wsb = static_cast<uint8_t *>(a.ws) + kWsHeader;
     const size_t cb_bytes = align256(static_cast<size_t>(cb_sets(all)) * a.Bsz * K * a.G * 2048);
     const size_t st_bytes = align256(static_cast<size_t>(a.Bsz) * a.H * nseg * kP * kN * sizeof(float));
@@ -1966,7 +2208,6 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
     float *seg_init = reinterpret_cast<float *>(wsb + cb_bytes + st_bytes);
     float *seg_decay = reinterpret_cast<float *>(wsb + cb_bytes + 2 * st_bytes);
     TcParams q = p;
-    q.agg = 1;
     q.need_s = 1;
     q.allblock = 0;
     for (int i = 1; i < 4; ++i) q.active[i] = 0;
@@ -1974,9 +2215,9 @@ cudaError_t launch_tc(const ScanArgs &a, cudaStream_t stream) {
     q.final_state = nullptr;
     q.y_clean = q.y_noisy = nullptr;
     q.seg_local = seg_local;
-    q.item_counter = counters;
+    q.item_counter = nullptr;
     q.seg_decay = seg_decay;
-    if ((e = launch_scan(grid, stream, q)) != cudaSuccess) return e;
+    if ((e = launch_agg(grid, stream, q)) != cudaSuccess) return e;
     bd_seg_combine_kernel<<<dim3(static_cast<unsigned>(a.Bsz * a.H), (kP * kN) / 256), 256, 0, stream>>>(
         a.h0, seg_local, seg_decay, seg_init, nseg);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

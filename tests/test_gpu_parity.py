@@ -38,9 +38,9 @@ SMALL = {
     "bf16_segmented": _shape(batch=1, nheads=2, ngroups=1, seqlen=1280),
     # more work items than SMs: each persistent CTA walks several (b, h)
     # sequences, resp. several segments, with the pipeline running across them
-    # (40 sequences of 80 blocks: 7 segments each, 280 items in two waves)
+    # (80 sequences of 64 blocks: 5 segments each, 400 items in three waves)
     "bf16_many_items": _shape(batch=5, nheads=64, ngroups=4, seqlen=96),
-    "bf16_segmented_many_items": _shape(batch=1, nheads=40, ngroups=2, seqlen=2560),
+    "bf16_segmented_many_items": _shape(batch=1, nheads=80, ngroups=2, seqlen=2048),
 }
 
 
@@ -294,6 +294,25 @@ def test_bounded_wait_timeout_reports_status():
     ryc, ryn, rst = oracle.allblock(s.as_dict(), cf, cr, nf, nr)
     check_y(yn, ryn)
     check_states(st, rst)
+
+
+def test_bounded_wait_timeout_segmented_prefix():
+    """The same for a segmented prefix (the aggregate pass, the segment combine
+    and the main pass): a zero wait limit gives BDSCAN_ERR_TIMEOUT, the next
+    call is clean and matches the oracle."""
+    s = _shape(batch=1, nheads=2, ngroups=1, seqlen=1280)
+    assert bd.kernel_launches(s, bd.BDSCAN_OP_PREFIX) == 4  # segmented plan
+    f, r = W.make_streams(s, 12, streams=(W.CLEAN_FWD, W.CLEAN_REV), device=DEV)
+    ws = bd.workspace(s, bd.BDSCAN_OP_PREFIX, DEV)
+    stream = torch.cuda.current_stream().cuda_stream
+    with bd.option(bd.BDSCAN_OPT_WAIT_TIMEOUT_NS, 0):
+        bd.prefix(s, f, r, want_states=False, ws=ws)
+    assert bd.bdscan_check_status(ws.data_ptr(), stream) == -6
+    y, _, fin = bd.prefix(s, f, r, want_states=False, ws=ws)
+    assert bd.bdscan_check_status(ws.data_ptr(), stream) == 0
+    ry, _, rfin = oracle.prefix(s.as_dict(), f, r)
+    check_y(y, ry)
+    check_states(fin, rfin)
 
 
 @pytest.mark.parametrize("case", ["pairs_eq_sms", "pairs_over_sms", "fwd_only", "gated_g2", "bf16_out_g2"])
