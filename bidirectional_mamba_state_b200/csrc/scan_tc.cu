@@ -1713,109 +1713,104 @@ __device__ void issuer(const TcParams &p, const Ctl &c, uint32_t base, uint32_t 
 // the group needs no exchange: per step, with v_k = dt A (log2 units) of
 // block k, the warp's own suffix sums give sum_{u > t} over its block, the
 // later blocks' totals and the running sum of the later steps the rest.
+// A step's loads stay in their registers, as loaded, until that step is
+// processed: the steps go in pairs with one register set each, so nothing
+// reads (or converts) a load's destination before its latency has passed.
+struct Raw {
+  unsigned short dt[kBlocks];  // bf16 bits of dt of this lane's token in each block
+  float A;
+};
+
 __device__ void operands(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
   const int lane = threadIdx.x & 31, w = (threadIdx.x >> 5) - 2;
   const int q = (threadIdx.x >> 5) & 3;  // TMEM lane quadrant of this warp
   const int64_t H = p.H, L = p.L, PN = kP * kN;
-  const __nv_bfloat16 *dtp = p.dt[kCF];
+  const unsigned short *dtp = reinterpret_cast<const unsigned short *>(p.dt[kCF]);
   const float *Ap = p.A[kCF];
-  // cursor over (item, step) for the loads two steps ahead
+  // cursor over (item, step) of the loads
   int cm = 0, cci = 0;
   Seg CI;
   bool cv = item(p, 0, CI);
-  float qdt[2][kBlocks], qa[2];
-  auto load = [&](int e) {
-    qa[e] = 0.f;
+  auto load = [&](Raw &r) {
+    r.A = 0.f;
 #pragma unroll
-    for (int k = 0; k < kBlocks; ++k) qdt[e][k] = 0.f;
+    for (int k = 0; k < kBlocks; ++k) r.dt[k] = 0;
     if (!cv) return;
     int kb, nb;
     step_blocks(CI, cci, kb, nb);
-    qa[e] = Ap[CI.h] * kLog2e;
-    const __nv_bfloat16 *src = dtp + (static_cast<int64_t>(CI.b) * L + static_cast<int64_t>(kb) * kT + lane) * H + CI.h;
+    r.A = Ap[CI.h];
+    const unsigned short *src = dtp + (static_cast<int64_t>(CI.b) * L + static_cast<int64_t>(kb) * kT + lane) * H + CI.h;
 #pragma unroll
     for (int k = 0; k < kBlocks; ++k)
-      if (k < nb) qdt[e][k] = __bfloat162float(src[static_cast<int64_t>(k) * kT * H]);
-  };
-  auto advance = [&]() {
-    if (!cv) return;
-    if (++cci < steps(CI)) return;
-    cci = 0;
-    cv = item(p, ++cm, CI);
-  };
-  load(0);
-  advance();
-  load(1);
-  advance();
-  int j = 0;
-  Seg I;
-  for (int m = 0; item(p, m, I); ++m) {
-    const int nc = steps(I);
-    float later_steps = 0.f;  // decay (log2) of the item's steps after this one
-    for (int ci = 0; ci < nc; ++ci, ++j) {
-      const int s = j % kStages, xb = j & 1;
-      float dtk[kBlocks];
-#pragma unroll
-      for (int k = 0; k < kBlocks; ++k) {
-        dtk[k] = qdt[0][k];
-        qdt[0][k] = qdt[1][k];
-      }
-      const float A2 = qa[0];
-      qa[0] = qa[1];
-      load(1);
-      advance();
-      // decays: totals of the four blocks (every lane) and this warp's block's
-      // inclusive suffix sums
-      float tot[kBlocks], own = 0.f, dt_own = 0.f;
-#pragma unroll
-      for (int k = 0; k < kBlocks; ++k) {
-        const float v = dtk[k] * A2;
-        float r = v;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
-        tot[k] = r;
-        if (k == w) {
-          own = v;
-          dt_own = dtk[k];
-        }
-      }
-      float suf = own;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float u = __shfl_down_sync(0xffffffffu, suf, o);
-        if (lane + o < 32) suf += u;
-      }
-      float later = later_steps + (suf - own);
-#pragma unroll
-      for (int k = 0; k < kBlocks; ++k)
-        if (k > w) later += tot[k];
-      const float wt = dt_own * ex2_approx(later);
-      later_steps += (tot[0] + tot[1]) + (tot[2] + tot[3]);
-      // x of this step has landed; the MMAs of step j - 2 have read this buffer
-      if (!waitw(c, bFull + s, static_cast<uint32_t>(j / kStages) & 1u)) return;
-      if (!waitw(c, bXwEmpty + xb, (static_cast<uint32_t>(j >> 1) & 1u) ^ 1u)) return;
-      int kb, nb;
-      step_blocks(I, ci, kb, nb);
-      if (w < nb) {
-        // row `lane` of block w: 64 values of x, scaled by w_t, as bf16 hi + lo
-        const uint32_t xs = base + static_cast<uint32_t>(s) * kStage + static_cast<uint32_t>(w) * kTile;
-        const uint32_t xh = base + kOffXw + static_cast<uint32_t>(xb) * kXwBuf + static_cast<uint32_t>(w) * 2u * kTile;
-#pragma unroll 2
-        for (int ch = 0; ch < 8; ++ch) {
-          const uint32_t off = sw128_chunk(static_cast<uint32_t>(lane), static_cast<uint32_t>(ch));
-          uint32_t r0, r1, r2, r3;
-          ld_shared_v4(xs + off, r0, r1, r2, r3);
-          float vv[8] = {bf16_lo_f(r0) * wt, bf16_hi_f(r0) * wt, bf16_lo_f(r1) * wt, bf16_hi_f(r1) * wt,
-                         bf16_lo_f(r2) * wt, bf16_hi_f(r2) * wt, bf16_lo_f(r3) * wt, bf16_hi_f(r3) * wt};
-          store_split8(xh + off, xh + kTile + off, vv);
-        }
-        fence_proxy_async_smem();
-      }
-      arrive_lane0(c, bXwFull + xb);
+      if (k < nb) r.dt[k] = src[static_cast<int64_t>(k) * kT * H];
+    if (++cci == steps(CI)) {
+      cci = 0;
+      cv = item(p, ++cm, CI);
     }
+  };
+  int j = 0, m = 0, ci = 0;
+  Seg I;
+  bool have = item(p, 0, I);
+  float later_steps = 0.f;  // decay (log2) of the item's steps after this one
+  // one step of item m; after its last step, the item's readout. false: a
+  // wait ran out
+  auto process = [&](const Raw &r) -> bool {
+    const int s = j % kStages, xb = j & 1;
+    const float A2 = r.A * kLog2e;
+    // decays: totals of the four blocks (every lane) and this warp's block's
+    // inclusive suffix sums
+    float tot[kBlocks], own = 0.f, dt_own = 0.f;
+#pragma unroll
+    for (int k = 0; k < kBlocks; ++k) {
+      const float dtk = __uint_as_float(static_cast<uint32_t>(r.dt[k]) << 16);
+      const float v = dtk * A2;
+      float rr = v;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) rr += __shfl_xor_sync(0xffffffffu, rr, o);
+      tot[k] = rr;
+      if (k == w) {
+        own = v;
+        dt_own = dtk;
+      }
+    }
+    float suf = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float u = __shfl_down_sync(0xffffffffu, suf, o);
+      if (lane + o < 32) suf += u;
+    }
+    float later = later_steps + (suf - own);
+#pragma unroll
+    for (int k = 0; k < kBlocks; ++k)
+      if (k > w) later += tot[k];
+    const float wt = dt_own * ex2_approx(later);
+    later_steps += (tot[0] + tot[1]) + (tot[2] + tot[3]);
+    // x of this step has landed; the MMAs of step j - 2 have read this buffer
+    if (!waitw(c, bFull + s, static_cast<uint32_t>(j / kStages) & 1u)) return false;
+    if (!waitw(c, bXwEmpty + xb, (static_cast<uint32_t>(j >> 1) & 1u) ^ 1u)) return false;
+    int kb, nb;
+    step_blocks(I, ci, kb, nb);
+    if (w < nb) {
+      // row `lane` of block w: 64 values of x, scaled by w_t, as bf16 hi + lo
+      const uint32_t xs = base + static_cast<uint32_t>(s) * kStage + static_cast<uint32_t>(w) * kTile;
+      const uint32_t xh = base + kOffXw + static_cast<uint32_t>(xb) * kXwBuf + static_cast<uint32_t>(w) * 2u * kTile;
+#pragma unroll 2
+      for (int ch = 0; ch < 8; ++ch) {
+        const uint32_t off = sw128_chunk(static_cast<uint32_t>(lane), static_cast<uint32_t>(ch));
+        uint32_t r0, r1, r2, r3;
+        ld_shared_v4(xs + off, r0, r1, r2, r3);
+        float vv[8] = {bf16_lo_f(r0) * wt, bf16_hi_f(r0) * wt, bf16_lo_f(r1) * wt, bf16_hi_f(r1) * wt,
+                       bf16_lo_f(r2) * wt, bf16_hi_f(r2) * wt, bf16_lo_f(r3) * wt, bf16_hi_f(r3) * wt};
+        store_split8(xh + off, xh + kTile + off, vv);
+      }
+      fence_proxy_async_smem();
+    }
+    arrive_lane0(c, bXwFull + xb);
+    ++j;
+    if (++ci < steps(I)) return true;
     // ---- readout: S^T (lane n = 32 q + lane, columns p) and the decay
     const int sb = m & 1;
-    if (!waitw(c, bSFull + sb, static_cast<uint32_t>(m >> 1) & 1u)) return;
+    if (!waitw(c, bSFull + sb, static_cast<uint32_t>(m >> 1) & 1u)) return false;
     tc_fence_after();
     const int64_t ebhs = (static_cast<int64_t>(I.b) * p.H + I.h) * p.nseg + I.seg;
     float *dst = p.seg_local + ebhs * PN + 32 * q + lane;
@@ -1831,6 +1826,21 @@ __device__ void operands(const TcParams &p, const Ctl &c, uint32_t base, uint32_
     if (w == 0 && lane == 0) p.seg_decay[ebhs] = later_steps;
     tc_fence_before();
     arrive_lane0(c, bSEmpty + sb);
+    ++m;
+    ci = 0;
+    later_steps = 0.f;
+    have = item(p, m, I);
+    return true;
+  };
+  Raw ra, rb;
+  load(ra);
+  load(rb);
+  while (have) {
+    if (!process(ra)) return;
+    load(ra);
+    if (!have) break;
+    if (!process(rb)) return;
+    load(rb);
   }
 }
 }  // namespace agg
