@@ -954,16 +954,19 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
   int cm = 0, ckk = 0;
   bool cv = true;  // the cursor is on an item
   Item CI = I;
-  float qdt[2], qa[2], qd[2];
+  // (kept as loaded -- dt as its bf16 bits -- and converted at use: an
+  // arithmetic use here would wait for the load)
+  uint32_t qdt[2];
+  float qa[2], qd[2];
   auto cursor_load = [&](int e) {
-    qdt[e] = 0.f;
+    qdt[e] = 0u;
     qa[e] = 0.f;
     qd[e] = 0.f;
     if (!cv) return;
     if (act) {
-      qdt[e] = __bfloat162float(
-          dtp[(static_cast<int64_t>(CI.b) * L + (CI.k0 + ckk) * kT + lane) * H + CI.h]);
-      qa[e] = Ap[CI.h] * kLog2e;
+      qdt[e] = reinterpret_cast<const unsigned short *>(
+          dtp)[(static_cast<int64_t>(CI.b) * L + (CI.k0 + ckk) * kT + lane) * H + CI.h];
+      qa[e] = Ap[CI.h];
     }
     if (dact) qd[e] = Dp[CI.h];
   };
@@ -988,7 +991,7 @@ __device__ void operand_group(const TcParams &p, const Ctl &c, uint32_t base) {
     for (int kk = 0; kk < I.nk; ++kk, ++j) {
       const int ct = j % kTab;
       const uint32_t st = base + Lay<kM>::slot(j) * Lay<kM>::kBytes;
-      const float dt_cur = qdt[0], A2 = qa[0], Dv = qd[0];
+      const float dt_cur = __uint_as_float(qdt[0] << 16), A2 = qa[0] * kLog2e, Dv = qd[0];
       qdt[0] = qdt[1];
       qa[0] = qa[1];
       qd[0] = qd[1];
