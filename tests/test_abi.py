@@ -34,6 +34,46 @@ def test_workspace_size_valid(name):
         assert bd.bdscan_workspace_size(ctypes.byref(s), bd.BDSCAN_OP_BLOCK_STEP) >= 256
 
 
+def _plan_segments(shape, op) -> int:
+    """The segment count the library planned for a tensor-core call, read back
+    from the workspace it asks for: header, C B^T tiles, then (when cut into
+    segments) two [B][H][nseg][P][N] fp32 state arrays and [B][H][nseg] decays,
+    each rounded up to 256 bytes."""
+    al = lambda x: (x + 255) // 256 * 256
+    K = shape.seqlen // shape.block_len
+    sets = 4 if op == bd.BDSCAN_OP_ALLBLOCK else 2
+    base = 1024 + al(sets * shape.batch * K * shape.ngroups * 2048)
+    ws = bd.bdscan_workspace_size(ctypes.byref(bd.c_shape(shape)), op)
+    if ws == base:
+        return 1
+    for nseg in range(2, K + 1):
+        bh = shape.batch * shape.nheads
+        if ws == base + 2 * al(bh * nseg * shape.headdim * shape.dstate * 4) + al(bh * nseg * 4):
+            return nseg
+    raise AssertionError(f"workspace {ws} matches no plan")
+
+
+@pytest.mark.parametrize("name,op,nseg,launches", [
+    # 48 sequences of 256 blocks: 3 segments (144 items, one wave on 148 SMs)
+    ("700m_prefill_8k", "prefix", 3, 4),
+    ("700m_prefill_64k", "prefix", 3, 4),
+    # 80 sequences of 8192 blocks: segments enough for 13 waves of 148 items
+    ("3b_prefill_256k", "prefix", 24, 4),
+    # 128 sequences (one wave) and 384 sequences: not cut
+    ("350m_allblock", "allblock", 1, 2),
+    ("87m_allblock", "allblock", 1, 2),
+    ("3b_step_b64", "prefix", 1, 2),
+])
+def test_segment_plan(name, op, nseg, launches):
+    """The planner's choices for the stated workloads (host logic: a cost model
+    of the waves of work items on 148 SMs), seen through the workspace size and
+    the launch count."""
+    s = WORKLOADS[name]
+    o = bd.BDSCAN_OP_PREFIX if op == "prefix" else bd.BDSCAN_OP_ALLBLOCK
+    assert _plan_segments(s, o) == nseg
+    assert bd.bdscan_kernel_launches(ctypes.byref(bd.c_shape(s)), o) == launches
+
+
 BAD_SHAPES = [
     (dict(seqlen=100), -2),        # not a multiple of block_len
     (dict(chunk_len=40), -2),      # chunk not a multiple of block
