@@ -79,7 +79,8 @@ struct BwdSmem {
   float *S, *expl, *red;    // [T], [T], [kBwdThreads]
   float *WCB, *YX, *G2;     // [T][T]: W o (C B^T), dy x^T, W o (dy x^T)
   float *Q;                 // [T][T + 1]: W o (C B^T) o (dy x^T), padded rows
-  float *hsCt, *dhBt;       // [P][T]: (h_s C^T)^T, (dh_e B^T)^T
+  float *hsCt, *dhBt;       // [P][T + 1]: (h_s C^T)^T, (dh_e B^T)^T, rows padded so that a
+                            // warp reading one column over 32 rows meets 32 banks
   float *hs, *carry;        // [P][N + 4]: rows padded so that rows p, p+1, ... fall into different banks
 };
 
@@ -168,13 +169,17 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
   auto tok = [&](int i) { return k * T + (rev ? T - 1 - i : i); };
   const float *nul = nullptr;
 
-  // ---- inputs of the block in processing order (row-major and transposed copies)
+  // ---- inputs of the block in processing order (row-major and transposed copies);
+  //      the loops are unrolled so that each thread has several loads in flight
+  //      before their stores wait for them
+#pragma unroll 4
   for (int e = tid; e < T * P; e += kBwdThreads) {
     const int i = e / P, pp = e % P;
     const int64_t xi = ((static_cast<int64_t>(b) * L + tok(i)) * H + h) * P + pp;
     s.x[e] = ldv(d.x, xi, p.in_bf16);
     s.dy[e] = dy ? ldv(dy, xi, p.dy_bf16) : 0.f;
   }
+#pragma unroll 8
   for (int e = tid; e < T * N; e += kBwdThreads) {
     const int i = e / N, n = e % N;
     const int64_t bi = ((static_cast<int64_t>(b) * L + tok(i)) * G + g) * N + n;
@@ -186,6 +191,7 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
   if (has_hs) {
     const float *src = k > 0 ? p.states + ((static_cast<int64_t>(b) * K + (k - 1)) * H + h) * PN
                              : p.h0 + (static_cast<int64_t>(b) * H + h) * PN;
+#pragma unroll 8
     for (int64_t e = tid; e < PN; e += kBwdThreads) s.hs[(e / N) * NS + e % N] = src[e];
   }
   __syncthreads();
@@ -245,19 +251,20 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
           [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
             for (int i = 0; i < R; ++i)
-              *reinterpret_cast<float4 *>(s.hsCt + (m0 + i) * T + n0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+              for (int jj = 0; jj < 4; ++jj) s.hsCt[(m0 + i) * (T + 1) + n0 + jj] = acc[i][jj];
           });
   if (has_dhe)
     sgemm<2>(P, T, N, s.carry, NS, 1, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
           [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
             for (int i = 0; i < R; ++i)
-              *reinterpret_cast<float4 *>(s.dhBt + (m0 + i) * T + n0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+              for (int jj = 0; jj < 4; ++jj) s.dhBt[(m0 + i) * (T + 1) + n0 + jj] = acc[i][jj];
           });
   float he_dot = 0.f;
   if (has_dhe) {
     const float *he = p.states + ((static_cast<int64_t>(b) * K + k) * H + h) * PN;
     float part = 0.f;
+#pragma unroll 8
     for (int64_t e = tid; e < PN; e += kBwdThreads) part += s.carry[(e / N) * NS + e % N] * he[e];
     he_dot = block_sum(part, s.red);
   }
@@ -284,7 +291,7 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
             float v[4];
             for (int j = 0; j < 4; ++j) {
               v[j] = Dh * s.dy[u * P + n0 + j] + s.dt[u] * acc[i][j];
-              if (has_dhe) v[j] += s.dt[u] * s.r[u] * s.dhBt[(n0 + j) * T + u];
+              if (has_dhe) v[j] += s.dt[u] * s.r[u] * s.dhBt[(n0 + j) * (T + 1) + u];
             }
             *reinterpret_cast<float4 *>(d.dx + ((static_cast<int64_t>(b) * L + tok(u)) * H + h) * P + n0) =
                 make_float4(v[0], v[1], v[2], v[3]);
@@ -308,26 +315,37 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
                 make_float4(du * acc[i][0], du * acc[i][1], du * acc[i][2], du * acc[i][3]);
           }
         });
-  // dL/dcum and the explicit dt terms
-  for (int i = tid; i < T; i += kBwdThreads) {
-    float sa = 0.f;
-    if (has_hs)
-      for (int q = 0; q < P; ++q) sa += s.dyt[q * T + i] * s.hsCt[q * T + i];
-    sa *= s.lam[i];
-    float num = 0.f, den = 0.f;
-    for (int u = 0; u <= i; ++u) num += s.Q[i * (T + 1) + u] * s.dt[u];
-    for (int i2 = i; i2 < T; ++i2) den += s.Q[i2 * (T + 1) + i];
-    float Si = sa + num - s.dt[i] * den;
-    float ex = den;
-    if (has_dhe) {
-      float xd = 0.f;
-      for (int q = 0; q < P; ++q) xd += s.xt[q * T + i] * s.dhBt[q * T + i];
-      Si -= s.dt[i] * s.r[i] * xd;
-      ex += s.r[i] * xd;
-      if (i == T - 1) Si += he_dot;
+  // dL/dcum and the explicit dt terms: one warp per token, its lanes over
+  // the sums' terms, the lanes' parts added in a fixed shuffle order
+  {
+    const int warp = tid >> 5, lane = tid & 31;
+    for (int i = warp; i < T; i += kBwdThreads / 32) {
+      float sa = 0.f, xd = 0.f, num = 0.f, den = 0.f;
+      for (int q = lane; q < P; q += 32) {
+        if (has_hs) sa += s.dy[i * P + q] * s.hsCt[q * (T + 1) + i];
+        if (has_dhe) xd += s.x[i * P + q] * s.dhBt[q * (T + 1) + i];
+      }
+      for (int u = lane; u <= i; u += 32) num += s.Q[i * (T + 1) + u] * s.dt[u];
+      for (int i2 = i + lane; i2 < T; i2 += 32) den += s.Q[i2 * (T + 1) + i];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        sa += __shfl_xor_sync(0xffffffffu, sa, o);
+        xd += __shfl_xor_sync(0xffffffffu, xd, o);
+        num += __shfl_xor_sync(0xffffffffu, num, o);
+        den += __shfl_xor_sync(0xffffffffu, den, o);
+      }
+      if (lane == 0) {
+        float Si = sa * s.lam[i] + num - s.dt[i] * den;
+        float ex = den;
+        if (has_dhe) {
+          Si -= s.dt[i] * s.r[i] * xd;
+          ex += s.r[i] * xd;
+          if (i == T - 1) Si += he_dot;
+        }
+        s.S[i] = Si;
+        s.expl[i] = ex;
+      }
     }
-    s.S[i] = Si;
-    s.expl[i] = ex;
   }
   __syncthreads();
   float pa = 0.f, pd = 0.f;
@@ -404,8 +422,9 @@ __global__ void __launch_bounds__(kBwdThreads) bd_bwd_kernel(const __grid_consta
   s.YX = q; q += T * T;
   s.G2 = q; q += T * T;
   s.Q = q; q += T * (T + 1);  // (a multiple of 4 floats: the buffers after it stay 16-byte aligned)
-  s.hsCt = q; q += P * T;
-  s.dhBt = q; q += P * T;
+  const int PTS = (P * (T + 1) + 3) & ~3;  // padded [P][T + 1], a multiple of 4 floats
+  s.hsCt = q; q += PTS;
+  s.dhBt = q; q += PTS;
   const int NS = N + 4;  // padded row stride of hs and carry
   s.hs = q; q += static_cast<int64_t>(P) * NS;
   s.carry = q;
@@ -422,6 +441,7 @@ __global__ void __launch_bounds__(kBwdThreads) bd_bwd_kernel(const __grid_consta
     if (p.active[1]) bwd_block(p, s, 1, b, h, k, accA[1], accD[1]);
     if (p.active[3]) bwd_block(p, s, 3, b, h, k, accA[3], accD[3]);
     if (k > 0 && p.dstates) {
+#pragma unroll 8
       for (int64_t e = threadIdx.x; e < PN; e += kBwdThreads)
         s.carry[(e / N) * NS + e % N] += p.dstates[((static_cast<int64_t>(b) * K + (k - 1)) * H + h) * PN + e];
       __syncthreads();
@@ -474,8 +494,8 @@ __global__ void bd_bwd_reduce_head_kernel(const float *pA, const float *pD, floa
 }  // namespace
 
 size_t bwd_smem_bytes(int64_t P, int64_t N, int64_t T) {
-  const int64_t floats = 4 * T * P + 4 * T * N + 6 * T + kBwdThreads + 3 * T * T + T * (T + 1) + 2 * P * T +
-                         2 * P * (N + 4);
+  const int64_t floats = 4 * T * P + 4 * T * N + 6 * T + kBwdThreads + 3 * T * T + T * (T + 1) +
+                         2 * ((P * (T + 1) + 3) & ~3) + 2 * P * (N + 4);
   return static_cast<size_t>(floats) * sizeof(float);
 }
 
