@@ -1577,9 +1577,10 @@ __global__ void __launch_bounds__(kThreads, 1) bd_tc_kernel(const __grid_constan
 // hi + lo (two MMAs per 16 tokens); S^T accumulates in TMEM (lane n, 64
 // columns p), two buffers so that a segment's readout overlaps the next
 // segment's MMAs.  Warps: 0 the TMA producer (x and B tiles, a three-step
-// ring), 1 the MMA issuer and TMEM owner, 2..5 the operands (warp 2 + w
-// builds block w of a step) and, at a segment's end, the readout (TMEM lanes
-// 32 (warp % 4) ..).  Work items (b, h, segment) go round-robin: item
+// ring), 1 the MMA issuer and TMEM owner, 2..9 the operands (warps 2 + w and
+// 6 + w build block w of a step, columns p 0..31 and 32..63) and, at a
+// segment's end, the readout (TMEM lanes 32 (warp % 4) .., the same halves of
+// the columns).  Work items (b, h, segment) go round-robin: item
 // blockIdx.x + m gridDim.x.
 namespace agg {
 constexpr int kBlocks = 4;                          // blocks per pipeline step
@@ -1601,7 +1602,7 @@ enum : int {
 };
 constexpr uint32_t kOffMisc = kOffBar + 8 * bCount;  // control block (layout of Ctl)
 constexpr uint32_t kSmem = kOffMisc + 32 + 1024;     // + alignment of the base to 1 KB
-constexpr int kThreadsAgg = 192;
+constexpr int kThreadsAgg = 320;  // producer, issuer, eight operand warps
 constexpr uint32_t kCols = 128;  // two S^T buffers of 64 columns
 static_assert(kSmem <= 227 * 1024, "aggregate kernel shared memory");
 
@@ -1710,7 +1711,8 @@ __device__ void issuer(const TcParams &p, const Ctl &c, uint32_t base, uint32_t 
   (void)mbar_wait_s(bar_at(c, bDrain), 0, p.drain_ns, 0);
 }
 
-// ---- operand warps 2..5 (w = warp - 2 builds block w of each step)
+// ---- operand warps 2..9 (w = (warp - 2) % 4 builds block w of each step,
+// half = (warp - 2) / 4 its columns p 32 half .. 32 half + 31)
 // Every lane loads dt of its token in all four blocks of a step (two steps
 // ahead), so that each warp forms the four blocks' decay sums itself and
 // the group needs no exchange: per step, with v_k = dt A (log2 units) of
@@ -1725,7 +1727,7 @@ struct Raw {
 };
 
 __device__ void operands(const TcParams &p, const Ctl &c, uint32_t base, uint32_t tmem) {
-  const int lane = threadIdx.x & 31, w = (threadIdx.x >> 5) - 2;
+  const int lane = threadIdx.x & 31, w = ((threadIdx.x >> 5) - 2) & 3, half = ((threadIdx.x >> 5) - 2) >> 2;
   const int q = (threadIdx.x >> 5) & 3;  // TMEM lane quadrant of this warp
   const int64_t H = p.H, L = p.L, PN = kP * kN;
   const unsigned short *dtp = reinterpret_cast<const unsigned short *>(p.dt[kCF]);
@@ -1794,11 +1796,11 @@ __device__ void operands(const TcParams &p, const Ctl &c, uint32_t base, uint32_
     int kb, nb;
     step_blocks(I, ci, kb, nb);
     if (w < nb) {
-      // row `lane` of block w: 64 values of x, scaled by w_t, as bf16 hi + lo
+      // row `lane` of block w: this half's 32 values of x, scaled by w_t, as bf16 hi + lo
       const uint32_t xs = base + static_cast<uint32_t>(s) * kStage + static_cast<uint32_t>(w) * kTile;
       const uint32_t xh = base + kOffXw + static_cast<uint32_t>(xb) * kXwBuf + static_cast<uint32_t>(w) * 2u * kTile;
 #pragma unroll 2
-      for (int ch = 0; ch < 8; ++ch) {
+      for (int ch = 4 * half; ch < 4 * half + 4; ++ch) {
         const uint32_t off = sw128_chunk(static_cast<uint32_t>(lane), static_cast<uint32_t>(ch));
         uint32_t r0, r1, r2, r3;
         ld_shared_v4(xs + off, r0, r1, r2, r3);
@@ -1819,14 +1821,14 @@ __device__ void operands(const TcParams &p, const Ctl &c, uint32_t base, uint32_
     float *dst = p.seg_local + ebhs * PN + 32 * q + lane;
     const uint32_t ta = tmem_addr(tmem, 32u * static_cast<uint32_t>(q), 64u * static_cast<uint32_t>(sb));
 #pragma unroll 1
-    for (int cq = 0; cq < 4; ++cq) {
+    for (int cq = 2 * half; cq < 2 * half + 2; ++cq) {
       uint32_t sv[16];
       tmem_ld_32x32b_x16(ta + 16u * static_cast<uint32_t>(cq), sv);
       tmem_ld_wait();
 #pragma unroll
       for (int i = 0; i < 16; ++i) dst[(16 * cq + i) * kN] = __uint_as_float(sv[i]);
     }
-    if (w == 0 && lane == 0) p.seg_decay[ebhs] = later_steps;
+    if (threadIdx.x == 64) p.seg_decay[ebhs] = later_steps;
     tc_fence_before();
     arrive_lane0(c, bSEmpty + sb);
     ++m;
@@ -1858,9 +1860,9 @@ __global__ void __launch_bounds__(agg::kThreadsAgg, 1) bd_agg_kernel(const __gri
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(sm + agg::kOffMisc);
   if (threadIdx.x == 0) {
     // full: producer + TMA bytes; empty, xw-empty, S-full, drain: one MMA
-    // commit; xw-full, S-empty: the four operand warps
+    // commit; xw-full, S-empty: the eight operand warps
     for (int i = 0; i < agg::bCount; ++i)
-      mbar_init(&bars[i], (i >= agg::bXwFull && i < agg::bXwFull + 2) || (i >= agg::bSEmpty && i < agg::bSEmpty + 2) ? 4u : 1u);
+      mbar_init(&bars[i], (i >= agg::bXwFull && i < agg::bXwFull + 2) || (i >= agg::bSEmpty && i < agg::bSEmpty + 2) ? 8u : 1u);
     *reinterpret_cast<volatile int *>(sm + agg::kOffMisc + 4) = 0;
     *reinterpret_cast<unsigned long long *>(sm + agg::kOffMisc + 8) = p.timeout_ns;
     *reinterpret_cast<int **>(sm + agg::kOffMisc + 16) = p.status;
