@@ -423,6 +423,7 @@ EXTRA = {
     "block_step_3b_b64_40layers": lambda dev, pk: _step_stack(W.WORKLOADS["3b_step_b64"], 40, dev, pk),
     "tiny_allblock": lambda dev, pk: _allblock_line("tiny", dev, pk, reps=50),
     "allblock_350m": lambda dev, pk: _allblock_line("350m_allblock", dev, pk),
+    "allblock_87m_gated": lambda dev, pk: _allblock_line("87m_allblock", dev, pk, gated=True),
     "prefill_700m_8k": lambda dev, pk: _prefill_line("700m_prefill_8k", 24, dev, pk),
     "prefill_700m_32k": lambda dev, pk: _prefill_line("700m_prefill_32k", 24, dev, pk),
     "prefill_700m_64k": lambda dev, pk: _prefill_line("700m_prefill_64k", 24, dev, pk),
@@ -634,16 +635,18 @@ def _heads_host(d: dict, hs: list) -> dict:
             for k, v in d.items()}
 
 
-def _allblock_line(name: str, dev, pk, reps: int = 10) -> dict:
+def _allblock_line(name: str, dev, pk, reps: int = 10, gated: bool = False) -> dict:
     """One bdscan_allblock call on a whole workload (CUDA events), with the
-    oracle's rate on one batch row (all heads, full length)."""
+    oracle's rate on one batch row (all heads, full length); gated: every
+    direction with its gate z (y_dir silu(z_dir) before the sum, fused in the
+    scan kernel's epilogue)."""
     import oracle
     s = W.WORKLOADS[name]
-    cf, cr, nf, nr = W.make_streams(s, W.SEEDS[name], device=dev)
+    cf, cr, nf, nr = W.make_streams(s, W.SEEDS[name], device=dev, gated=gated)
     yc, yn, st = bd.allblock(s, cf, cr, nf, nr)
     ws = bd.workspace(s, bd.BDSCAN_OP_ALLBLOCK, dev)
     ms = _time(lambda: bd.allblock(s, cf, cr, nf, nr, y_clean=yc, y_noisy=yn, states=st, ws=ws), dev, reps)
-    b = RL.allblock_bytes(s)
+    b = RL.allblock_bytes(s, gated=gated)
     del yc, yn, st
     one = s.with_(batch=1)
     hs = [_host({k: (v if k in ("A", "D") else v[:1]) for k, v in d.items()}) for d in (cf, cr, nf, nr)]

@@ -334,6 +334,23 @@ __device__ __forceinline__ float bf16_lo_f(uint32_t v) { return __uint_as_float(
 __device__ __forceinline__ float silu_approx(float v) { return __fdividef(v, 1.0f + ex2_approx(-v * 1.4426950408889634f)); }
 __device__ __forceinline__ float bf16_hi_f(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
+// silu(z) of 16 gate values z[base + i stride] (1 where there is no gate).
+// The 16 loads are issued before any of them is used, so that their latencies
+// overlap (a load consumed at once would wait for it before the next is issued).
+__device__ __forceinline__ void gates16(const __nv_bfloat16 *z, int64_t base, int64_t stride, float (&g)[16]) {
+  if (!z) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) g[i] = 1.f;
+    return;
+  }
+  const unsigned short *z16 = reinterpret_cast<const unsigned short *>(z) + base;
+  unsigned short r[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) r[i] = z16[i * stride];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) g[i] = silu_approx(__uint_as_float(static_cast<uint32_t>(r[i]) << 16));
+}
+
 // C B^T tile set of direction slot i in the workspace: the all-block pass keeps
 // four (one per direction), prefix and block step two (the clean forward and
 // reverse directions, slots 0 and 2).
@@ -544,6 +561,11 @@ __device__ __forceinline__ void sts_s32(uint32_t addr, int v) {
 }
 
 __device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Fire-and-forget fetch of a line into this SM's L1 (the next block's gates:
+// their loads then wait for L1, not for HBM).
+__device__ __forceinline__ void prefetch_l1(const void *ptr) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(ptr));
+}
 
 // Claim the next work item (-1: none left).  With no more items than CTAs,
 // CTA c takes item c and nothing else (no counter, no wait for the pre-pass);
@@ -1366,14 +1388,13 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
         const int64_t yi = ((static_cast<int64_t>(I.b) * L + k * kT + th) * H + I.h) * kP + pcol;
         if (kGated) {
           const __nv_bfloat16 *zf = p.z[kCF], *zr = rev_act ? p.z[kCR] : nullptr;
+          float gf[16], gr[16];
+          gates16(zf, yi, tstride, gf);
+          gates16(zr, yi, tstride, gr);
 #pragma unroll
           for (int t = 0; t < 16; ++t) {
-            float v = __uint_as_float(yo[t]);
-            if (zf) v *= silu_approx(__bfloat162float(zf[yi + t * tstride]));
-            if (rev_act) {
-              const float u = __uint_as_float(yd[t]);
-              v += zr ? u * silu_approx(__bfloat162float(zr[yi + t * tstride])) : u;
-            }
+            float v = __uint_as_float(yo[t]) * gf[t];
+            if (rev_act) v = fmaf(__uint_as_float(yd[t]), gr[t], v);
             yo[t] = __float_as_uint(v);
           }
         }
@@ -1435,14 +1456,24 @@ __device__ void epilogue_group(const TcParams &p, const Ctl &c, uint32_t base, u
           const int64_t zi = ((static_cast<int64_t>(I.b) * L + k * kT) * H + I.h) * kP + pcol;
           const __nv_bfloat16 *zf = pick4(p.z, fs), *zr = rev_act ? pick4(p.z, fs | 2) : nullptr;
 #pragma unroll
-          for (int t = 0; t < 32; ++t) {
-            float v = __uint_as_float(yo[t]);
-            if (zf) v *= silu_approx(__bfloat162float(zf[zi + t * H * kP]));
-            if (rev_act) {
-              const float u = __uint_as_float(yd[t]);
-              v += zr ? u * silu_approx(__bfloat162float(zr[zi + t * H * kP])) : u;
+          for (int t0 = 0; t0 < 32; t0 += 16) {
+            float gf[16], gr[16];
+            gates16(zf, zi + t0 * H * kP, H * kP, gf);
+            gates16(zr, zi + t0 * H * kP, H * kP, gr);
+#pragma unroll
+            for (int t = 0; t < 16; ++t) {
+              float v = __uint_as_float(yo[t0 + t]) * gf[t];
+              if (rev_act) v = fmaf(__uint_as_float(yd[t0 + t]), gr[t], v);
+              yo[t0 + t] = __float_as_uint(v);
             }
-            yo[t] = __float_as_uint(v);
+          }
+          if (kk + 1 < I.nk) {  // the next block's gates
+            const int64_t zn = zi + static_cast<int64_t>(kT) * H * kP;
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+              if (zf) prefetch_l1(zf + zn + t * H * kP);
+              if (zr) prefetch_l1(zr + zn + t * H * kP);
+            }
           }
         }
         if (mine) {

@@ -34,9 +34,11 @@ def state_bytes(s: Shape) -> int:
     return 4 * s.batch * s.nheads * s.headdim * s.dstate
 
 
-def allblock_bytes(s: Shape, with_clean_y: bool = True, with_rev: bool = True) -> int:
+def allblock_bytes(s: Shape, with_clean_y: bool = True, with_rev: bool = True, gated: bool = False) -> int:
+    """gated: every direction also reads its gate z (the input dtype, like x)."""
     ndir = 4 if with_rev else 2
-    return ndir * dir_bytes(s) + (2 if with_clean_y else 1) * y_bytes(s) + \
+    z = ndir * _elt(s.in_dtype) * s.batch * s.seqlen * s.nheads * s.headdim if gated else 0
+    return ndir * dir_bytes(s) + z + (2 if with_clean_y else 1) * y_bytes(s) + \
         s.nblocks * state_bytes(s)
 
 
