@@ -104,14 +104,18 @@ __device__ float block_sum(float v, float *red) {
 //   acc[i][j] = sum_k a1(m0+i, k) B1[k][n0+j]  (+ sum_k a2(m0+i, k) B2[k][n0+j])
 // with a(m, k) = A[m am + k ak] (times ks1[k], resp. ms2[m], when given) and
 // B rows contiguous in n (16-byte loads).  A threads of a warp share m0, so A
-// loads are broadcasts.  epi(m0, n0, acc) consumes the tile.
+// loads are broadcasts.  epi(m0, n0, acc) consumes the tile.  Threads lo ..
+// lo + cnt - 1 take the tiles (two products of a phase run side by side on
+// the two halves of the CTA).
 template <int TM, class Epi>
-__device__ __forceinline__ void sgemm(int M, int Nn, int K1, const float *A1, int am1, int ak1, const float *ks1,
-                                      const float *B1, int ldb1, int K2, const float *A2, int am2, int ak2,
-                                      const float *ms2, const float *B2, int ldb2, Epi epi) {
+__device__ __forceinline__ void sgemm(int lo, int cnt, int M, int Nn, int K1, const float *A1, int am1, int ak1,
+                                      const float *ks1, const float *B1, int ldb1, int K2, const float *A2,
+                                      int am2, int ak2, const float *ms2, const float *B2, int ldb2, Epi epi) {
   const int nt = Nn >> 2;
   const int tiles = (M / TM) * nt;
-  for (int t = threadIdx.x; t < tiles; t += kBwdThreads) {
+  const int me = static_cast<int>(threadIdx.x) - lo;
+  if (me < 0 || me >= cnt) return;
+  for (int t = me; t < tiles; t += cnt) {
     const int m0 = (t / nt) * TM, n0 = (t % nt) << 2;
     float acc[TM][4];
 #pragma unroll
@@ -232,29 +236,31 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
   }
   __syncthreads();
 
-  // ---- Gram matrices: C B^T and dy x^T
-  sgemm<1>(T, T, N, s.Ct, 1, T, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+  // ---- Gram matrices: C B^T and dy x^T; then the products with the start
+  //      state and the end-state gradient (each half of the CTA takes one
+  //      product of each pair)
+  constexpr int kHalf = kBwdThreads / 2;
+  sgemm<1>(0, kHalf, T, T, N, s.Ct, 1, T, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
         [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
           for (int i = 0; i < R; ++i)
             *reinterpret_cast<float4 *>(s.WCB + (m0 + i) * T + n0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
         });
-  sgemm<1>(T, T, P, s.dyt, 1, T, nul, s.xt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+  sgemm<1>(kHalf, kHalf, T, T, P, s.dyt, 1, T, nul, s.xt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
         [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
           for (int i = 0; i < R; ++i)
             *reinterpret_cast<float4 *>(s.YX + (m0 + i) * T + n0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
         });
-  // ---- products with the start state and the end-state gradient
   if (has_hs)
-    sgemm<2>(P, T, N, s.hs, NS, 1, nul, s.Ct, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+    sgemm<2>(0, kHalf, P, T, N, s.hs, NS, 1, nul, s.Ct, T, 0, nullptr, 0, 0, nul, nullptr, 0,
           [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
             for (int i = 0; i < R; ++i)
               for (int jj = 0; jj < 4; ++jj) s.hsCt[(m0 + i) * (T + 1) + n0 + jj] = acc[i][jj];
           });
   if (has_dhe)
-    sgemm<2>(P, T, N, s.carry, NS, 1, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+    sgemm<2>(kHalf, kHalf, P, T, N, s.carry, NS, 1, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
           [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
             for (int i = 0; i < R; ++i)
@@ -283,7 +289,7 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
 
   // ---- token gradients
   // dx_u = D dy_u + dt_u sum_i WCB[i][u] dy_i (+ dt_u r_u dh_e B_u)
-  sgemm<2>(T, P, T, s.WCB, 1, T, nul, s.dy, P, 0, nullptr, 0, 0, nul, nullptr, 0,
+  sgemm<2>(0, kHalf, T, P, T, s.WCB, 1, T, nul, s.dy, P, 0, nullptr, 0, 0, nul, nullptr, 0,
         [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
           for (int i = 0; i < R; ++i) {
@@ -298,7 +304,7 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
           }
         });
   // dC_i = sum_u G2[i][u] dt_u B_u (+ Lam_i dy_i^T h_s)
-  sgemm<4>(T, N, T, s.G2, T, 1, s.dt, s.Bm, N, has_hs ? P : 0, has_hs ? s.dy : nullptr, P, 1, s.lam, s.hs, NS,
+  sgemm<4>(0, kHalf, T, N, T, s.G2, T, 1, s.dt, s.Bm, N, has_hs ? P : 0, has_hs ? s.dy : nullptr, P, 1, s.lam, s.hs, NS,
         [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
           for (int i = 0; i < R; ++i)
@@ -306,7 +312,7 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
                 make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
         });
   // dB_u = dt_u (sum_i G2[i][u] C_i (+ r_u x_u^T dh_e))
-  sgemm<4>(T, N, T, s.G2, 1, T, nul, s.Cm, N, has_dhe ? P : 0, has_dhe ? s.x : nullptr, P, 1, s.r, s.carry, NS,
+  sgemm<4>(kHalf, kHalf, T, N, T, s.G2, 1, T, nul, s.Cm, N, has_dhe ? P : 0, has_dhe ? s.x : nullptr, P, 1, s.r, s.carry, NS,
         [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
           for (int i = 0; i < R; ++i) {
@@ -315,11 +321,12 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
                 make_float4(du * acc[i][0], du * acc[i][1], du * acc[i][2], du * acc[i][3]);
           }
         });
-  // dL/dcum and the explicit dt terms: one warp per token, its lanes over
-  // the sums' terms, the lanes' parts added in a fixed shuffle order
-  {
-    const int warp = tid >> 5, lane = tid & 31;
-    for (int i = warp; i < T; i += kBwdThreads / 32) {
+  // dL/dcum and the explicit dt terms (the second half of the CTA, after dB):
+  // one warp per token, its lanes over the sums' terms, the lanes' parts
+  // added in a fixed shuffle order
+  if (tid >= kHalf) {
+    const int warp = (tid - kHalf) >> 5, lane = tid & 31;
+    for (int i = warp; i < T; i += kHalf / 32) {
       float sa = 0.f, xd = 0.f, num = 0.f, den = 0.f;
       for (int q = lane; q < P; q += 32) {
         if (has_hs) sa += s.dy[i * P + q] * s.hsCt[q * (T + 1) + i];
@@ -381,7 +388,7 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
   }
   // ---- gradient of the start state: dh_s = Lam_e dh_e + sum_i Lam_i dy_i C_i^T
   if (!rev)
-    sgemm<4>(P, N, T, s.dy, 1, P, s.lam, s.Cm, N, 0, nullptr, 0, 0, nul, nullptr, 0,
+    sgemm<4>(0, kBwdThreads, P, N, T, s.dy, 1, P, s.lam, s.Cm, N, 0, nullptr, 0, 0, nul, nullptr, 0,
           [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
             for (int i = 0; i < R; ++i) {
