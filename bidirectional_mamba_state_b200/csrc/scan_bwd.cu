@@ -84,6 +84,16 @@ struct BwdSmem {
   float *hs, *carry;        // [P][N + 4]: rows padded so that rows p, p+1, ... fall into different banks
 };
 
+// Eight bf16 values (one 16-byte load) as floats.
+__device__ __forceinline__ void unpack8(const uint4 &v, float *o) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    o[2 * i] = __uint_as_float(w[i] << 16);
+    o[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
 // Sum over the CTA in a fixed order (a shuffle tree per warp, then the warp
 // sums in warp order): deterministic, two barriers.
 __device__ float block_sum(float v, float *red) {
@@ -175,28 +185,69 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
 
   // ---- inputs of the block in processing order (row-major and transposed copies);
   //      the loops are unrolled so that each thread has several loads in flight
-  //      before their stores wait for them
+  //      before their stores wait for them; bf16 rows whose lengths are
+  //      multiples of 8 are read 16 bytes at a time
+  if (p.in_bf16 && (P & 7) == 0 && (N & 7) == 0) {
+    const int cx = P >> 3, cn = N >> 3;
+    const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(d.x);
+#pragma unroll 2
+    for (int e = tid; e < T * cx; e += kBwdThreads) {
+      const int i = e / cx, c8 = (e - i * cx) << 3;
+      const int64_t xi = ((static_cast<int64_t>(b) * L + tok(i)) * H + h) * P + c8;
+      unpack8(*reinterpret_cast<const uint4 *>(xb + xi), s.x + i * P + c8);
+      if (!dy) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s.dy[i * P + c8 + j] = 0.f;
+      } else if (p.dy_bf16) {
+        unpack8(*reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(dy) + xi), s.dy + i * P + c8);
+      } else {
+        const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(dy) + xi);
+        const float4 v0 = src[0], v1 = src[1];
+        *reinterpret_cast<float4 *>(s.dy + i * P + c8) = v0;
+        *reinterpret_cast<float4 *>(s.dy + i * P + c8 + 4) = v1;
+      }
+    }
+    const __nv_bfloat16 *Bb = static_cast<const __nv_bfloat16 *>(d.B), *Cb = static_cast<const __nv_bfloat16 *>(d.C);
+#pragma unroll 2
+    for (int e = tid; e < T * cn; e += kBwdThreads) {
+      const int i = e / cn, c8 = (e - i * cn) << 3;
+      const int64_t bi = ((static_cast<int64_t>(b) * L + tok(i)) * G + g) * N + c8;
+      const uint4 vb = *reinterpret_cast<const uint4 *>(Bb + bi), vc = *reinterpret_cast<const uint4 *>(Cb + bi);
+      unpack8(vb, s.Bm + i * N + c8);
+      unpack8(vc, s.Cm + i * N + c8);
+    }
+  } else {
 #pragma unroll 4
-  for (int e = tid; e < T * P; e += kBwdThreads) {
-    const int i = e / P, pp = e % P;
-    const int64_t xi = ((static_cast<int64_t>(b) * L + tok(i)) * H + h) * P + pp;
-    s.x[e] = ldv(d.x, xi, p.in_bf16);
-    s.dy[e] = dy ? ldv(dy, xi, p.dy_bf16) : 0.f;
-  }
+    for (int e = tid; e < T * P; e += kBwdThreads) {
+      const int i = e / P, pp = e % P;
+      const int64_t xi = ((static_cast<int64_t>(b) * L + tok(i)) * H + h) * P + pp;
+      s.x[e] = ldv(d.x, xi, p.in_bf16);
+      s.dy[e] = dy ? ldv(dy, xi, p.dy_bf16) : 0.f;
+    }
 #pragma unroll 8
-  for (int e = tid; e < T * N; e += kBwdThreads) {
-    const int i = e / N, n = e % N;
-    const int64_t bi = ((static_cast<int64_t>(b) * L + tok(i)) * G + g) * N + n;
-    s.Bm[e] = ldv(d.B, bi, p.in_bf16);
-    s.Cm[e] = ldv(d.C, bi, p.in_bf16);
+    for (int e = tid; e < T * N; e += kBwdThreads) {
+      const int i = e / N, n = e % N;
+      const int64_t bi = ((static_cast<int64_t>(b) * L + tok(i)) * G + g) * N + n;
+      s.Bm[e] = ldv(d.B, bi, p.in_bf16);
+      s.Cm[e] = ldv(d.C, bi, p.in_bf16);
+    }
   }
   for (int i = tid; i < T; i += kBwdThreads)
     s.dt[i] = ldv(d.dt, (static_cast<int64_t>(b) * L + tok(i)) * H + h, p.in_bf16);
   if (has_hs) {
     const float *src = k > 0 ? p.states + ((static_cast<int64_t>(b) * K + (k - 1)) * H + h) * PN
                              : p.h0 + (static_cast<int64_t>(b) * H + h) * PN;
+    if ((N & 3) == 0) {
+      const int cn4 = N >> 2;
+#pragma unroll 4
+      for (int e = tid; e < static_cast<int>(PN >> 2); e += kBwdThreads) {
+        const int row = e / cn4, c4 = (e - row * cn4) << 2;
+        *reinterpret_cast<float4 *>(s.hs + row * NS + c4) = reinterpret_cast<const float4 *>(src)[e];
+      }
+    } else {
 #pragma unroll 8
-    for (int64_t e = tid; e < PN; e += kBwdThreads) s.hs[(e / N) * NS + e % N] = src[e];
+      for (int64_t e = tid; e < PN; e += kBwdThreads) s.hs[(e / N) * NS + e % N] = src[e];
+    }
   }
   __syncthreads();
   // Transposed copies, skewed: consecutive threads take consecutive columns

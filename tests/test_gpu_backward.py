@@ -62,6 +62,7 @@ def _run(s, with_rev=True, with_h0=True, with_dyc=True, with_dst=True, seed=5):
 SHAPES = {
     "bf16_g2": _shape(),
     "fp32_in_bf16_out": _shape(in_dtype="fp32", out_dtype="bf16", seqlen=64),
+    "bf16_in_bf16_out": _shape(out_dtype="bf16", seqlen=64),  # bf16 dy through the 16-byte loads
     "p16_n48_t16": _shape(headdim=16, dstate=48, block_len=16, chunk_len=16, seqlen=80, nheads=6, ngroups=3),
     "one_block": _shape(seqlen=32, batch=3),
 }
