@@ -249,6 +249,26 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
       for (int64_t e = tid; e < PN; e += kBwdThreads) s.hs[(e / N) * NS + e % N] = src[e];
     }
   }
+  // this thread's part of <dh_e, h_e> (the clean forward stream): the end
+  // state's loads go out with the inputs' (the carried gradient dh_e is
+  // already in shared memory)
+  float he_part = 0.f;
+  if (has_dhe) {
+    const float *he = p.states + ((static_cast<int64_t>(b) * K + k) * H + h) * PN;
+    if ((N & 3) == 0) {
+      const int cn4 = N >> 2;
+#pragma unroll 4
+      for (int e = tid; e < static_cast<int>(PN >> 2); e += kBwdThreads) {
+        const int row = e / cn4, c4 = (e - row * cn4) << 2;
+        const float4 hv = reinterpret_cast<const float4 *>(he)[e];
+        const float4 cv = *reinterpret_cast<const float4 *>(s.carry + row * NS + c4);
+        he_part += hv.x * cv.x + hv.y * cv.y + hv.z * cv.z + hv.w * cv.w;
+      }
+    } else {
+#pragma unroll 8
+      for (int64_t e = tid; e < PN; e += kBwdThreads) he_part += s.carry[(e / N) * NS + e % N] * he[e];
+    }
+  }
   __syncthreads();
   // Transposed copies, skewed: consecutive threads take consecutive columns
   // and rotated rows (i = (j + column) mod T), so that neither the row-major
@@ -318,13 +338,7 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
               for (int jj = 0; jj < 4; ++jj) s.dhBt[(m0 + i) * (T + 1) + n0 + jj] = acc[i][jj];
           });
   float he_dot = 0.f;
-  if (has_dhe) {
-    const float *he = p.states + ((static_cast<int64_t>(b) * K + k) * H + h) * PN;
-    float part = 0.f;
-#pragma unroll 8
-    for (int64_t e = tid; e < PN; e += kBwdThreads) part += s.carry[(e / N) * NS + e % N] * he[e];
-    he_dot = block_sum(part, s.red);
-  }
+  if (has_dhe) he_dot = block_sum(he_part, s.red);
   __syncthreads();
   // ---- decay-weighted matrices (W_iu = exp(cum_i - cum_u), u <= i)
   for (int e = tid; e < T * T; e += kBwdThreads) {
