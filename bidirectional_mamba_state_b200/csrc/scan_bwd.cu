@@ -187,25 +187,35 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
   //      the loops are unrolled so that each thread has several loads in flight
   //      before their stores wait for them; bf16 rows whose lengths are
   //      multiples of 8 are read 16 bytes at a time
-  if (p.in_bf16 && (P & 7) == 0 && (N & 7) == 0) {
+  // (the 16-byte path also forms this thread's part of sum dy . x, the dD term)
+  float pd_part = 0.f;
+  const bool vec = p.in_bf16 && (P & 7) == 0 && (N & 7) == 0;
+  if (vec) {
     const int cx = P >> 3, cn = N >> 3;
     const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(d.x);
 #pragma unroll 2
     for (int e = tid; e < T * cx; e += kBwdThreads) {
       const int i = e / cx, c8 = (e - i * cx) << 3;
       const int64_t xi = ((static_cast<int64_t>(b) * L + tok(i)) * H + h) * P + c8;
-      unpack8(*reinterpret_cast<const uint4 *>(xb + xi), s.x + i * P + c8);
+      float xv[8], dv[8];
+      unpack8(*reinterpret_cast<const uint4 *>(xb + xi), xv);
       if (!dy) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) s.dy[i * P + c8 + j] = 0.f;
+        for (int j = 0; j < 8; ++j) dv[j] = 0.f;
       } else if (p.dy_bf16) {
-        unpack8(*reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(dy) + xi), s.dy + i * P + c8);
+        unpack8(*reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(dy) + xi), dv);
       } else {
         const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(dy) + xi);
         const float4 v0 = src[0], v1 = src[1];
-        *reinterpret_cast<float4 *>(s.dy + i * P + c8) = v0;
-        *reinterpret_cast<float4 *>(s.dy + i * P + c8 + 4) = v1;
+        dv[0] = v0.x; dv[1] = v0.y; dv[2] = v0.z; dv[3] = v0.w;
+        dv[4] = v1.x; dv[5] = v1.y; dv[6] = v1.z; dv[7] = v1.w;
       }
+      *reinterpret_cast<float4 *>(s.x + i * P + c8) = make_float4(xv[0], xv[1], xv[2], xv[3]);
+      *reinterpret_cast<float4 *>(s.x + i * P + c8 + 4) = make_float4(xv[4], xv[5], xv[6], xv[7]);
+      *reinterpret_cast<float4 *>(s.dy + i * P + c8) = make_float4(dv[0], dv[1], dv[2], dv[3]);
+      *reinterpret_cast<float4 *>(s.dy + i * P + c8 + 4) = make_float4(dv[4], dv[5], dv[6], dv[7]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) pd_part = fmaf(dv[j], xv[j], pd_part);
     }
     const __nv_bfloat16 *Bb = static_cast<const __nv_bfloat16 *>(d.B), *Cb = static_cast<const __nv_bfloat16 *>(d.C);
 #pragma unroll 2
@@ -272,16 +282,33 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
   __syncthreads();
   // Transposed copies, skewed: consecutive threads take consecutive columns
   // and rotated rows (i = (j + column) mod T), so that neither the row-major
-  // reads nor the transposed writes of a warp fall into one shared-memory bank.
-  for (int e = tid; e < T * P; e += kBwdThreads) {
-    const int pp = e % P, i = (e / P + pp) % T;
-    s.xt[pp * T + i] = s.x[i * P + pp];
-    s.dyt[pp * T + i] = s.dy[i * P + pp];
-  }
-  for (int e = tid; e < T * N; e += kBwdThreads) {
-    const int n = e % N, i = (e / N + n) % T;
-    s.Bt[n * T + i] = s.Bm[i * N + n];
-    s.Ct[n * T + i] = s.Cm[i * N + n];
+  // reads nor the transposed writes of a warp fall into one shared-memory bank
+  // (with power-of-two sizes the index arithmetic is shifts and masks).
+  if (((P & (P - 1)) | (N & (N - 1)) | (T & (T - 1))) == 0) {
+    const int lp = __ffs(P) - 1, ln = __ffs(N) - 1;
+#pragma unroll 4
+    for (int e = tid; e < T * P; e += kBwdThreads) {
+      const int pp = e & (P - 1), i = ((e >> lp) + pp) & (T - 1);
+      s.xt[pp * T + i] = s.x[i * P + pp];
+      s.dyt[pp * T + i] = s.dy[i * P + pp];
+    }
+#pragma unroll 4
+    for (int e = tid; e < T * N; e += kBwdThreads) {
+      const int n = e & (N - 1), i = ((e >> ln) + n) & (T - 1);
+      s.Bt[n * T + i] = s.Bm[i * N + n];
+      s.Ct[n * T + i] = s.Cm[i * N + n];
+    }
+  } else {
+    for (int e = tid; e < T * P; e += kBwdThreads) {
+      const int pp = e % P, i = (e / P + pp) % T;
+      s.xt[pp * T + i] = s.x[i * P + pp];
+      s.dyt[pp * T + i] = s.dy[i * P + pp];
+    }
+    for (int e = tid; e < T * N; e += kBwdThreads) {
+      const int n = e % N, i = (e / N + n) % T;
+      s.Bt[n * T + i] = s.Bm[i * N + n];
+      s.Ct[n * T + i] = s.Cm[i * N + n];
+    }
   }
   // cumulative decays: a warp prefix scan over 32-token chunks (lane order
   // within a chunk, chunks in order), then Lam and r in parallel
@@ -445,7 +472,10 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
     for (int o = 16; o > 0; o >>= 1) pacc += __shfl_xor_sync(0xffffffffu, pacc, o);
     pa = pacc;
   }
-  for (int e = tid; e < T * P; e += kBwdThreads) pd += s.dy[e] * s.x[e];
+  if (vec)
+    pd = pd_part;
+  else
+    for (int e = tid; e < T * P; e += kBwdThreads) pd += s.dy[e] * s.x[e];
   pd = block_sum(pd, s.red);
   if (tid == 0) {
     accA += pa;
