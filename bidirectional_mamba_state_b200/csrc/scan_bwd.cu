@@ -244,7 +244,9 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
   }
   for (int i = tid; i < T; i += kBwdThreads)
     s.dt[i] = ldv(d.dt, (static_cast<int64_t>(b) * L + tok(i)) * H + h, p.in_bf16);
-  if (has_hs) {
+  // (the noisy block starts from the clean stream's state before it, which
+  // the clean block of the same k, processed just before, left in place)
+  if (has_hs && kind != 2) {
     const float *src = k > 0 ? p.states + ((static_cast<int64_t>(b) * K + (k - 1)) * H + h) * PN
                              : p.h0 + (static_cast<int64_t>(b) * H + h) * PN;
     if ((N & 3) == 0) {
