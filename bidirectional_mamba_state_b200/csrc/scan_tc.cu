@@ -787,7 +787,16 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
       // ---- Y_off^T = h [C_cf; C_nf]^T, h = the state before this block
       if (!wait1(c, bHFull, j & 1)) break;
       const int yb = ybuf(kGated, j), jp = yprev(kGated, j);
-      if (jp >= 0 && !wait1(c, bYEmpty0 + yb, ypar(kGated, jp))) break;
+      // Double-buffered Y with the masked-decay operands built two steps ahead
+      // (ungated, C B^T from the pre-pass): each epilogue warp frees Y of step
+      // j - 2 before it builds the operands of step j, so their completion
+      // implies the buffer is free -- one wait instead of two.
+      constexpr bool kMhFirst = !kGated && !kCbF;
+      if constexpr (kMhFirst) {
+        if (!wait1(c, bMhFull0 + i2, par2(j))) break;
+      } else {
+        if (jp >= 0 && !wait1(c, bYEmpty0 + yb, ypar(kGated, jp))) break;
+      }
       tc_fence_after();
       const uint32_t colY = tmem + kColY0 + kColYBuf * yb;
 #pragma unroll 1
@@ -800,7 +809,7 @@ __device__ void mma_issuer(const TcParams &p, const Ctl &c, uint32_t base, uint3
       // ---- Y_diag^T of each stream = X_fwd^T M_fwd^T + X_rev^T M_rev^T (M
       //      with D on its diagonal), and in the next 32 columns the same
       //      products with the diagonal's bf16 remainders
-      if (!wait1(c, bMhFull0 + i2, par2(j))) break;
+      if (!kMhFirst && !wait1(c, bMhFull0 + i2, par2(j))) break;
       tc_fence_after();
       const uint32_t mo = BD_OFF(static_cast<uint32_t>(i2) * kMhBuf);
 #pragma unroll
