@@ -340,13 +340,13 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
   //      state and the end-state gradient (each half of the CTA takes one
   //      product of each pair)
   constexpr int kHalf = kBwdThreads / 2;
-  sgemm<1>(0, kHalf, T, T, N, s.Ct, 1, T, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+  sgemm<2>(0, kHalf, T, T, N, s.Ct, 1, T, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
         [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
           for (int i = 0; i < R; ++i)
             *reinterpret_cast<float4 *>(s.WCB + (m0 + i) * T + n0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
         });
-  sgemm<1>(kHalf, kHalf, T, T, P, s.dyt, 1, T, nul, s.xt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+  sgemm<2>(kHalf, kHalf, T, T, P, s.dyt, 1, T, nul, s.xt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
         [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
           for (int i = 0; i < R; ++i)
