@@ -37,6 +37,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <type_traits>
 
 #include "bdscan_internal.h"
 
@@ -108,6 +109,21 @@ __device__ float block_sum(float v, float *red) {
   return r;
 }
 
+// TM consecutive floats from an address aligned to TM floats (TM = 2 or 4)
+template <int TM>
+__device__ __forceinline__ void load_row(const float *p, float (&a)[TM]) {
+  if constexpr (TM == 4) {
+    const float4 v = *reinterpret_cast<const float4 *>(p);
+    a[0] = v.x; a[1] = v.y; a[2] = v.z; a[3] = v.w;
+  } else if constexpr (TM == 2) {
+    const float2 v = *reinterpret_cast<const float2 *>(p);
+    a[0] = v.x; a[1] = v.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < TM; ++i) a[i] = p[i];
+  }
+}
+
 // Register-tiled product over shared-memory operands: for every TM x 4 output
 // tile (m0.., n0..) of an M x Nn result (TM chosen per product so that the
 // threads have a tile each),
@@ -132,18 +148,36 @@ __device__ __forceinline__ void sgemm(int lo, int cnt, int M, int Nn, int K1, co
     for (int i = 0; i < TM; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-    for (int k = 0; k < K1; ++k) {
-      const float4 bv = *reinterpret_cast<const float4 *>(B1 + k * ldb1 + n0);
-      const float sk = ks1 ? ks1[k] : 1.f;
+    // the TM values a1(m0.., k) are contiguous when am1 = 1: one vector load
+    // per k where the addresses allow it
+    const bool avec = (TM == 2 || TM == 4) && am1 == 1 &&
+                      ((reinterpret_cast<uintptr_t>(A1 + m0) | static_cast<uintptr_t>(ak1) * sizeof(float)) &
+                       (TM * sizeof(float) - 1)) == 0;
+    auto k1_loop = [&](auto vec) {
+      for (int k = 0; k < K1; ++k) {
+        const float4 bv = *reinterpret_cast<const float4 *>(B1 + k * ldb1 + n0);
+        const float sk = ks1 ? ks1[k] : 1.f;
+        float a[TM];
+        if constexpr (decltype(vec)::value) {
+          load_row<TM>(A1 + m0 + k * ak1, a);
+        } else {
 #pragma unroll
-      for (int i = 0; i < TM; ++i) {
-        const float a = A1[(m0 + i) * am1 + k * ak1] * sk;
-        acc[i][0] = fmaf(a, bv.x, acc[i][0]);
-        acc[i][1] = fmaf(a, bv.y, acc[i][1]);
-        acc[i][2] = fmaf(a, bv.z, acc[i][2]);
-        acc[i][3] = fmaf(a, bv.w, acc[i][3]);
+          for (int i = 0; i < TM; ++i) a[i] = A1[(m0 + i) * am1 + k * ak1];
+        }
+#pragma unroll
+        for (int i = 0; i < TM; ++i) {
+          const float ai = a[i] * sk;
+          acc[i][0] = fmaf(ai, bv.x, acc[i][0]);
+          acc[i][1] = fmaf(ai, bv.y, acc[i][1]);
+          acc[i][2] = fmaf(ai, bv.z, acc[i][2]);
+          acc[i][3] = fmaf(ai, bv.w, acc[i][3]);
+        }
       }
-    }
+    };
+    if (avec)
+      k1_loop(std::true_type{});
+    else
+      k1_loop(std::false_type{});
     if (A2) {
       float sm2[TM];
 #pragma unroll
