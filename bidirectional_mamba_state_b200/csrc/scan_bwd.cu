@@ -109,24 +109,24 @@ __device__ float block_sum(float v, float *red) {
   return r;
 }
 
-// TM consecutive floats from an address aligned to TM floats (TM = 2 or 4)
-template <int TM>
-__device__ __forceinline__ void load_row(const float *p, float (&a)[TM]) {
-  if constexpr (TM == 4) {
+// W consecutive floats from an address aligned to W floats (W = 2 or 4)
+template <int W>
+__device__ __forceinline__ void load_row(const float *p, float *a) {
+  if constexpr (W == 4) {
     const float4 v = *reinterpret_cast<const float4 *>(p);
     a[0] = v.x; a[1] = v.y; a[2] = v.z; a[3] = v.w;
-  } else if constexpr (TM == 2) {
+  } else if constexpr (W == 2) {
     const float2 v = *reinterpret_cast<const float2 *>(p);
     a[0] = v.x; a[1] = v.y;
   } else {
 #pragma unroll
-    for (int i = 0; i < TM; ++i) a[i] = p[i];
+    for (int i = 0; i < W; ++i) a[i] = p[i];
   }
 }
 
 // Register-tiled product over shared-memory operands: for every TM x 4 output
-// tile (m0.., n0..) of an M x Nn result (TM chosen per product so that the
-// threads have a tile each),
+// tile (m0.., n0..) of an M x Nn result (TM chosen per product by timing:
+// taller tiles need fewer shared-memory loads per FMA but leave threads idle),
 //   acc[i][j] = sum_k a1(m0+i, k) B1[k][n0+j]  (+ sum_k a2(m0+i, k) B2[k][n0+j])
 // with a(m, k) = A[m am + k ak] (times ks1[k], resp. ms2[m], when given) and
 // B rows contiguous in n (16-byte loads).  A threads of a warp share m0, so A
@@ -148,36 +148,67 @@ __device__ __forceinline__ void sgemm(int lo, int cnt, int M, int Nn, int K1, co
     for (int i = 0; i < TM; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-    // the TM values a1(m0.., k) are contiguous when am1 = 1: one vector load
-    // per k where the addresses allow it
-    const bool avec = (TM == 2 || TM == 4) && am1 == 1 &&
-                      ((reinterpret_cast<uintptr_t>(A1 + m0) | static_cast<uintptr_t>(ak1) * sizeof(float)) &
-                       (TM * sizeof(float) - 1)) == 0;
-    auto k1_loop = [&](auto vec) {
-      for (int k = 0; k < K1; ++k) {
-        const float4 bv = *reinterpret_cast<const float4 *>(B1 + k * ldb1 + n0);
-        const float sk = ks1 ? ks1[k] : 1.f;
-        float a[TM];
-        if constexpr (decltype(vec)::value) {
-          load_row<TM>(A1 + m0 + k * ak1, a);
-        } else {
+    // a1(m0.., k) is contiguous in m when am1 = 1 (one vector load per k) and
+    // contiguous in k when ak1 = 1 (one 16-byte load per row and four k)
+    constexpr int VW = TM >= 4 ? 4 : TM;
+    const uintptr_t a_at = reinterpret_cast<uintptr_t>(A1);  // m0 is a multiple of TM
+    const int mode = (TM % VW == 0 && VW > 1 && am1 == 1 &&
+                      ((a_at | static_cast<uintptr_t>(ak1) * sizeof(float)) & (VW * sizeof(float) - 1)) == 0)
+                         ? 1
+                     : (ak1 == 1 && (K1 & 3) == 0 &&
+                        ((a_at | static_cast<uintptr_t>(am1) * sizeof(float)) & (4 * sizeof(float) - 1)) == 0)
+                         ? 2
+                         : 0;
+    auto k1_loop = [&](auto md) {
+      constexpr int kMode = decltype(md)::value;
+      if constexpr (kMode == 2) {
+        for (int k = 0; k < K1; k += 4) {
+          float4 a4[TM];
 #pragma unroll
-          for (int i = 0; i < TM; ++i) a[i] = A1[(m0 + i) * am1 + k * ak1];
+          for (int i = 0; i < TM; ++i) a4[i] = *reinterpret_cast<const float4 *>(A1 + (m0 + i) * am1 + k);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const float4 bv = *reinterpret_cast<const float4 *>(B1 + (k + kk) * ldb1 + n0);
+            const float sk = ks1 ? ks1[k + kk] : 1.f;
+#pragma unroll
+            for (int i = 0; i < TM; ++i) {
+              const float ai = (kk == 0 ? a4[i].x : kk == 1 ? a4[i].y : kk == 2 ? a4[i].z : a4[i].w) * sk;
+              acc[i][0] = fmaf(ai, bv.x, acc[i][0]);
+              acc[i][1] = fmaf(ai, bv.y, acc[i][1]);
+              acc[i][2] = fmaf(ai, bv.z, acc[i][2]);
+              acc[i][3] = fmaf(ai, bv.w, acc[i][3]);
+            }
+          }
         }
+      } else {
+        for (int k = 0; k < K1; ++k) {
+          const float4 bv = *reinterpret_cast<const float4 *>(B1 + k * ldb1 + n0);
+          const float sk = ks1 ? ks1[k] : 1.f;
+          float a[TM];
+          if constexpr (kMode == 1) {
 #pragma unroll
-        for (int i = 0; i < TM; ++i) {
-          const float ai = a[i] * sk;
-          acc[i][0] = fmaf(ai, bv.x, acc[i][0]);
-          acc[i][1] = fmaf(ai, bv.y, acc[i][1]);
-          acc[i][2] = fmaf(ai, bv.z, acc[i][2]);
-          acc[i][3] = fmaf(ai, bv.w, acc[i][3]);
+            for (int i = 0; i < TM; i += VW) load_row<VW>(A1 + m0 + i + k * ak1, a + i);
+          } else {
+#pragma unroll
+            for (int i = 0; i < TM; ++i) a[i] = A1[(m0 + i) * am1 + k * ak1];
+          }
+#pragma unroll
+          for (int i = 0; i < TM; ++i) {
+            const float ai = a[i] * sk;
+            acc[i][0] = fmaf(ai, bv.x, acc[i][0]);
+            acc[i][1] = fmaf(ai, bv.y, acc[i][1]);
+            acc[i][2] = fmaf(ai, bv.z, acc[i][2]);
+            acc[i][3] = fmaf(ai, bv.w, acc[i][3]);
+          }
         }
       }
     };
-    if (avec)
-      k1_loop(std::true_type{});
+    if (mode == 1)
+      k1_loop(std::integral_constant<int, 1>{});
+    else if (mode == 2)
+      k1_loop(std::integral_constant<int, 2>{});
     else
-      k1_loop(std::false_type{});
+      k1_loop(std::integral_constant<int, 0>{});
     if (A2) {
       float sm2[TM];
 #pragma unroll
@@ -387,14 +418,14 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
             *reinterpret_cast<float4 *>(s.YX + (m0 + i) * T + n0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
         });
   if (has_hs)
-    sgemm<2>(0, kHalf, P, T, N, s.hs, NS, 1, nul, s.Ct, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+    sgemm<4>(0, kHalf, P, T, N, s.hs, NS, 1, nul, s.Ct, T, 0, nullptr, 0, 0, nul, nullptr, 0,
           [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
             for (int i = 0; i < R; ++i)
               for (int jj = 0; jj < 4; ++jj) s.hsCt[(m0 + i) * (T + 1) + n0 + jj] = acc[i][jj];
           });
   if (has_dhe)
-    sgemm<2>(kHalf, kHalf, P, T, N, s.carry, NS, 1, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+    sgemm<4>(kHalf, kHalf, P, T, N, s.carry, NS, 1, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
           [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
             for (int i = 0; i < R; ++i)
