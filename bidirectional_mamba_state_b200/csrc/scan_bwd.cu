@@ -213,7 +213,29 @@ __device__ __forceinline__ void sgemm(int lo, int cnt, int M, int Nn, int K1, co
       float sm2[TM];
 #pragma unroll
       for (int i = 0; i < TM; ++i) sm2[i] = ms2 ? ms2[m0 + i] : 1.f;
-      for (int k = 0; k < K2; ++k) {
+      int k = 0;
+      // rows contiguous in k: 16-byte loads, four k at a time
+      if (ak2 == 1 && ((reinterpret_cast<uintptr_t>(A2) | static_cast<uintptr_t>(am2) * sizeof(float)) &
+                       (4 * sizeof(float) - 1)) == 0) {
+        for (; k + 4 <= K2; k += 4) {
+          float4 a4[TM];
+#pragma unroll
+          for (int i = 0; i < TM; ++i) a4[i] = *reinterpret_cast<const float4 *>(A2 + (m0 + i) * am2 + k);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const float4 bv = *reinterpret_cast<const float4 *>(B2 + (k + kk) * ldb2 + n0);
+#pragma unroll
+            for (int i = 0; i < TM; ++i) {
+              const float a = (kk == 0 ? a4[i].x : kk == 1 ? a4[i].y : kk == 2 ? a4[i].z : a4[i].w) * sm2[i];
+              acc[i][0] = fmaf(a, bv.x, acc[i][0]);
+              acc[i][1] = fmaf(a, bv.y, acc[i][1]);
+              acc[i][2] = fmaf(a, bv.z, acc[i][2]);
+              acc[i][3] = fmaf(a, bv.w, acc[i][3]);
+            }
+          }
+        }
+      }
+      for (; k < K2; ++k) {
         const float4 bv = *reinterpret_cast<const float4 *>(B2 + k * ldb2 + n0);
 #pragma unroll
         for (int i = 0; i < TM; ++i) {
