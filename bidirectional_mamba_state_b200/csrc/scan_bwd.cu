@@ -45,6 +45,12 @@ namespace bdscan {
 namespace {
 
 constexpr int kBwdThreads = 512;
+// The reverse directions start every block from a zero state and take no
+// end-state gradient, so their blocks depend on nothing carried: they run in
+// CTAs of their own, kRevSplit per (b, h), each over a contiguous range of
+// blocks, after the (b, h) CTAs of the forward chain.  The short pieces fill
+// the SMs that the forward chains' last wave leaves idle.
+constexpr int kRevSplit = 8;
 
 struct BwdDir {
   const void *x, *dt, *B, *C;
@@ -59,6 +65,7 @@ struct BwdParams {
   int active[4];
   int Bsz, L, H, P, N, G, T, K;
   int in_bf16, dy_bf16;
+  int rev_split;         // reverse-direction CTAs per (b, h) (0: the chain CTA runs them)
   const float *h0;       // [B][H][P][N] or null
   const float *states;   // [B][K][H][P][N] (forward output)
   const void *dy_clean;  // [B][L][H][P] or null
@@ -619,6 +626,26 @@ __global__ void __launch_bounds__(kBwdThreads) bd_bwd_kernel(const __grid_consta
   const int NS = N + 4;  // padded row stride of hs and carry
   s.hs = q; q += static_cast<int64_t>(P) * NS;
   s.carry = q;
+  const int BH = p.Bsz * H;
+  if (static_cast<int>(blockIdx.x) >= BH) {
+    // a piece of the reverse directions: blocks k0 .. k1 - 1 of one (b, h);
+    // its dA, dD partials go to row r of the direction's [rev_split][B][H]
+    const int idx = static_cast<int>(blockIdx.x) - BH, r = idx / BH, bh = idx % BH;
+    const int b = bh / H, h = bh % H;
+    const int k0 = r * K / p.rev_split, k1 = (r + 1) * K / p.rev_split;
+    float accA[4] = {0.f, 0.f, 0.f, 0.f}, accD[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int k = k1 - 1; k >= k0; --k) {
+      if (p.active[1]) bwd_block(p, s, 1, b, h, k, accA[1], accD[1]);
+      if (p.active[3]) bwd_block(p, s, 3, b, h, k, accA[3], accD[3]);
+    }
+    if (threadIdx.x == 0)
+      for (int di = 1; di < 4; di += 2)
+        if (p.active[di]) {
+          p.dir[di].pA[static_cast<int64_t>(r) * BH + bh] = accA[di];
+          p.dir[di].pD[static_cast<int64_t>(r) * BH + bh] = accD[di];
+        }
+    return;
+  }
   const int b = blockIdx.x / H, h = blockIdx.x % H;
   // carry = dL/dstates[K-1] (given part)
   for (int64_t e = threadIdx.x; e < PN; e += kBwdThreads)
@@ -629,8 +656,8 @@ __global__ void __launch_bounds__(kBwdThreads) bd_bwd_kernel(const __grid_consta
   for (int k = K - 1; k >= 0; --k) {
     bwd_block(p, s, 0, b, h, k, accA[0], accD[0]);
     bwd_block(p, s, 2, b, h, k, accA[2], accD[2]);
-    if (p.active[1]) bwd_block(p, s, 1, b, h, k, accA[1], accD[1]);
-    if (p.active[3]) bwd_block(p, s, 3, b, h, k, accA[3], accD[3]);
+    if (!p.rev_split && p.active[1]) bwd_block(p, s, 1, b, h, k, accA[1], accD[1]);
+    if (!p.rev_split && p.active[3]) bwd_block(p, s, 3, b, h, k, accA[3], accD[3]);
     if (k > 0 && p.dstates) {
 #pragma unroll 8
       for (int64_t e = threadIdx.x; e < PN; e += kBwdThreads)
@@ -643,7 +670,7 @@ __global__ void __launch_bounds__(kBwdThreads) bd_bwd_kernel(const __grid_consta
       p.dh0[(static_cast<int64_t>(b) * H + h) * PN + e] = s.carry[(e / N) * NS + e % N];
   if (threadIdx.x == 0)
     for (int di = 0; di < 4; ++di)
-      if (p.active[di]) {
+      if (p.active[di] && !(p.rev_split && (di & 1))) {
         p.dir[di].pA[static_cast<int64_t>(b) * H + h] = accA[di];
         p.dir[di].pD[static_cast<int64_t>(b) * H + h] = accD[di];
       }
@@ -691,15 +718,17 @@ size_t bwd_smem_bytes(int64_t P, int64_t N, int64_t T) {
 }
 
 size_t bwd_workspace_bytes(int64_t Bsz, int64_t L, int64_t H, int64_t N) {
-  // per direction: dB, dC partials [B][L][H][N] and dA, dD partials [B][H]
-  const size_t per = (2 * static_cast<size_t>(Bsz) * L * H * N + 2 * static_cast<size_t>(Bsz) * H) * sizeof(float);
+  // per direction: dB, dC partials [B][L][H][N] and dA, dD partials
+  // [kRevSplit][B][H] (a forward direction uses the first B x H)
+  const size_t per =
+      (2 * static_cast<size_t>(Bsz) * L * H * N + 2 * static_cast<size_t>(kRevSplit) * Bsz * H) * sizeof(float);
   return 4 * ((per + 255) & ~static_cast<size_t>(255));
 }
 
 cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream) {
   BwdParams p;
   std::memset(&p, 0, sizeof(p));
-  const int64_t per_floats = 2 * a.Bsz * a.L * a.H * a.N + 2 * a.Bsz * a.H;
+  const int64_t per_floats = 2 * a.Bsz * a.L * a.H * a.N + 2 * kRevSplit * a.Bsz * a.H;
   const size_t per = ((static_cast<size_t>(per_floats) * sizeof(float)) + 255) & ~static_cast<size_t>(255);
   for (int i = 0; i < 4; ++i) {
     p.active[i] = a.dir[i].x != nullptr;
@@ -717,7 +746,7 @@ cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream) {
     d.pB = base;
     d.pC = base + a.Bsz * a.L * a.H * a.N;
     d.pA = base + 2 * a.Bsz * a.L * a.H * a.N;
-    d.pD = d.pA + a.Bsz * a.H;
+    d.pD = d.pA + kRevSplit * a.Bsz * a.H;
   }
   p.Bsz = static_cast<int>(a.Bsz);
   p.L = static_cast<int>(a.L);
@@ -735,11 +764,12 @@ cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream) {
   p.dy_noisy = a.dy_noisy;
   p.dstates = a.dstates;
   p.dh0 = a.dh0;
+  p.rev_split = (p.active[1] || p.active[3]) ? kRevSplit : 0;
   const size_t smem = bwd_smem_bytes(a.P, a.N, a.T);
   cudaError_t e = cudaFuncSetAttribute(bd_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  bd_bwd_kernel<<<static_cast<unsigned>(a.Bsz * a.H), kBwdThreads, smem, stream>>>(p);
+  bd_bwd_kernel<<<static_cast<unsigned>(a.Bsz * a.H * (1 + p.rev_split)), kBwdThreads, smem, stream>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int64_t rows = a.Bsz * a.L;
   const int64_t cnt = rows * a.G * a.N;
@@ -749,7 +779,7 @@ cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream) {
     bd_bwd_reduce_kernel<<<static_cast<unsigned>((cnt + 255) / 256), 256, 0, stream>>>(
         d.pB, d.pC, a.grad[i].dB, a.grad[i].dC, rows, p.H, p.G, p.N);
     bd_bwd_reduce_head_kernel<<<static_cast<unsigned>((a.H + 127) / 128), 128, 0, stream>>>(
-        d.pA, d.pD, a.grad[i].dA, a.grad[i].dD, p.Bsz, p.H);
+        d.pA, d.pD, a.grad[i].dA, a.grad[i].dD, (i & 1) && p.rev_split ? p.Bsz * p.rev_split : p.Bsz, p.H);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;
