@@ -430,31 +430,31 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
   }
   __syncthreads();
 
-  // ---- Gram matrices: C B^T and dy x^T; then the products with the start
-  //      state and the end-state gradient (each half of the CTA takes one
-  //      product of each pair)
-  constexpr int kHalf = kBwdThreads / 2;
-  sgemm<2>(0, kHalf, T, T, N, s.Ct, 1, T, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+  // ---- Gram matrices C B^T and dy x^T and the products with the start state
+  //      and the end-state gradient, side by side on the four quarters of the
+  //      CTA (each has a tile per thread of its quarter)
+  constexpr int kHalf = kBwdThreads / 2, kQuarter = kBwdThreads / 4;
+  sgemm<2>(0, kQuarter, T, T, N, s.Ct, 1, T, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
         [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
           for (int i = 0; i < R; ++i)
             *reinterpret_cast<float4 *>(s.WCB + (m0 + i) * T + n0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
         });
-  sgemm<2>(kHalf, kHalf, T, T, P, s.dyt, 1, T, nul, s.xt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+  sgemm<2>(kQuarter, kQuarter, T, T, P, s.dyt, 1, T, nul, s.xt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
         [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
           for (int i = 0; i < R; ++i)
             *reinterpret_cast<float4 *>(s.YX + (m0 + i) * T + n0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
         });
   if (has_hs)
-    sgemm<4>(0, kHalf, P, T, N, s.hs, NS, 1, nul, s.Ct, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+    sgemm<4>(2 * kQuarter, kQuarter, P, T, N, s.hs, NS, 1, nul, s.Ct, T, 0, nullptr, 0, 0, nul, nullptr, 0,
           [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
             for (int i = 0; i < R; ++i)
               for (int jj = 0; jj < 4; ++jj) s.hsCt[(m0 + i) * (T + 1) + n0 + jj] = acc[i][jj];
           });
   if (has_dhe)
-    sgemm<4>(kHalf, kHalf, P, T, N, s.carry, NS, 1, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
+    sgemm<4>(3 * kQuarter, kQuarter, P, T, N, s.carry, NS, 1, nul, s.Bt, T, 0, nullptr, 0, 0, nul, nullptr, 0,
           [&](int m0, int n0, auto &acc) {
           constexpr int R = sizeof(acc) / sizeof(acc[0]);
             for (int i = 0; i < R; ++i)
