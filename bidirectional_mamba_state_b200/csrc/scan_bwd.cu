@@ -35,6 +35,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <type_traits>
@@ -676,37 +677,62 @@ __global__ void __launch_bounds__(kBwdThreads) bd_bwd_kernel(const __grid_consta
       }
 }
 
-// Fixed-order sums of the partials: dB, dC over the heads of a group, dA, dD
-// over the batch rows.
-__global__ void bd_bwd_reduce_kernel(const float *pB, const float *pC, float *dB, float *dC, int64_t rows,
-                                     int H, int G, int N) {
-  const int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // over rows * G * N
-  if (e >= rows * G * N) return;
-  const int n = static_cast<int>(e % N);
-  const int g = static_cast<int>((e / N) % G);
-  const int64_t r = e / (static_cast<int64_t>(N) * G);  // (b, t)
-  const int hpg = H / G;
-  float sb = 0.f, sc = 0.f;
-  for (int j = 0; j < hpg; ++j) {
-    const int64_t o = (r * H + g * hpg + j) * N + n;
-    sb += pB[o];
-    sc += pC[o];
-  }
-  dB[e] = sb;
-  dC[e] = sc;
-}
+// Fixed-order sums of the partials, all directions in one launch (grid row y =
+// the y-th present direction): dB, dC over the heads of a group (16-byte loads
+// and stores when N is a multiple of 4 and the outputs are 16-byte aligned),
+// and, in the row's first CTA, dA, dD over the batch rows (and reverse ranges).
+struct BwdSums {
+  const float *pB[4], *pC[4], *pA[4], *pD[4];
+  float *dB[4], *dC[4], *dA[4], *dD[4];
+  int dir[4];    // direction of grid row y
+  int arows[4];  // rows of the dA, dD partials of each direction
+  int vec;       // 16-byte path
+};
 
-__global__ void bd_bwd_reduce_head_kernel(const float *pA, const float *pD, float *dA, float *dD, int Bsz,
-                                          int H) {
-  const int h = blockIdx.x * blockDim.x + threadIdx.x;
-  if (h >= H) return;
-  float sa = 0.f, sd = 0.f;
-  for (int b = 0; b < Bsz; ++b) {
-    sa += pA[static_cast<int64_t>(b) * H + h];
-    sd += pD[static_cast<int64_t>(b) * H + h];
+__global__ void bd_bwd_reduce_kernel(const __grid_constant__ BwdSums a, int64_t rows, int H, int G, int N) {
+  const int di = a.dir[blockIdx.y];
+  if (blockIdx.x == 0)
+    for (int h = threadIdx.x; h < H; h += blockDim.x) {
+      float sa = 0.f, sd = 0.f;
+      for (int b = 0; b < a.arows[di]; ++b) {
+        sa += a.pA[di][static_cast<int64_t>(b) * H + h];
+        sd += a.pD[di][static_cast<int64_t>(b) * H + h];
+      }
+      a.dA[di][h] = sa;
+      a.dD[di][h] = sd;
+    }
+  const float *pB = a.pB[di], *pC = a.pC[di];
+  const int hpg = H / G;
+  const int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (a.vec) {  // e over rows * G * N / 4
+    const int n4 = N >> 2;
+    if (e >= rows * G * n4) return;
+    const int n = static_cast<int>(e % n4) << 2;
+    const int g = static_cast<int>((e / n4) % G);
+    const int64_t r = e / (static_cast<int64_t>(n4) * G);  // (b, t)
+    float4 sb = make_float4(0.f, 0.f, 0.f, 0.f), sc = sb;
+    for (int j = 0; j < hpg; ++j) {
+      const int64_t o = (r * H + g * hpg + j) * N + n;
+      const float4 vb = *reinterpret_cast<const float4 *>(pB + o), vc = *reinterpret_cast<const float4 *>(pC + o);
+      sb.x += vb.x; sb.y += vb.y; sb.z += vb.z; sb.w += vb.w;
+      sc.x += vc.x; sc.y += vc.y; sc.z += vc.z; sc.w += vc.w;
+    }
+    reinterpret_cast<float4 *>(a.dB[di])[e] = sb;
+    reinterpret_cast<float4 *>(a.dC[di])[e] = sc;
+  } else {  // e over rows * G * N
+    if (e >= rows * G * N) return;
+    const int n = static_cast<int>(e % N);
+    const int g = static_cast<int>((e / N) % G);
+    const int64_t r = e / (static_cast<int64_t>(N) * G);
+    float sb = 0.f, sc = 0.f;
+    for (int j = 0; j < hpg; ++j) {
+      const int64_t o = (r * H + g * hpg + j) * N + n;
+      sb += pB[o];
+      sc += pC[o];
+    }
+    a.dB[di][e] = sb;
+    a.dC[di][e] = sc;
   }
-  dA[h] = sa;
-  dD[h] = sd;
 }
 
 }  // namespace
@@ -772,14 +798,30 @@ cudaError_t launch_bwd(const BwdArgs &a, cudaStream_t stream) {
   bd_bwd_kernel<<<static_cast<unsigned>(a.Bsz * a.H * (1 + p.rev_split)), kBwdThreads, smem, stream>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int64_t rows = a.Bsz * a.L;
-  const int64_t cnt = rows * a.G * a.N;
+  BwdSums sums;
+  std::memset(&sums, 0, sizeof(sums));
+  int ndir = 0;
+  bool aligned = (a.N & 3) == 0;
   for (int i = 0; i < 4; ++i) {
     if (!p.active[i]) continue;
     const BwdDir &d = p.dir[i];
-    bd_bwd_reduce_kernel<<<static_cast<unsigned>((cnt + 255) / 256), 256, 0, stream>>>(
-        d.pB, d.pC, a.grad[i].dB, a.grad[i].dC, rows, p.H, p.G, p.N);
-    bd_bwd_reduce_head_kernel<<<static_cast<unsigned>((a.H + 127) / 128), 128, 0, stream>>>(
-        d.pA, d.pD, a.grad[i].dA, a.grad[i].dD, (i & 1) && p.rev_split ? p.Bsz * p.rev_split : p.Bsz, p.H);
+    sums.pB[i] = d.pB;
+    sums.pC[i] = d.pC;
+    sums.pA[i] = d.pA;
+    sums.pD[i] = d.pD;
+    sums.dB[i] = a.grad[i].dB;
+    sums.dC[i] = a.grad[i].dC;
+    sums.dA[i] = a.grad[i].dA;
+    sums.dD[i] = a.grad[i].dD;
+    sums.arows[i] = (i & 1) && p.rev_split ? p.Bsz * p.rev_split : p.Bsz;
+    sums.dir[ndir++] = i;
+    aligned = aligned && ((reinterpret_cast<uintptr_t>(a.grad[i].dB) | reinterpret_cast<uintptr_t>(a.grad[i].dC)) & 15) == 0;
+  }
+  sums.vec = aligned ? 1 : 0;
+  const int64_t cnt = rows * a.G * (aligned ? a.N / 4 : a.N);
+  if (ndir > 0) {
+    const dim3 grid(static_cast<unsigned>(std::max<int64_t>(1, (cnt + 255) / 256)), static_cast<unsigned>(ndir));
+    bd_bwd_reduce_kernel<<<grid, 256, 0, stream>>>(sums, rows, p.H, p.G, p.N);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;
