@@ -357,23 +357,35 @@ __device__ void bwd_block(const BwdParams &p, const BwdSmem &s, int kind, int b,
     }
   }
   // this thread's part of <dh_e, h_e> (the clean forward stream): the end
-  // state's loads go out with the inputs' (the carried gradient dh_e is
-  // already in shared memory)
+  // state's loads go out with the inputs', and so do those of the given
+  // dL/dstates[k], which completes the carried gradient dh_e in shared memory
+  // (below the last block; the last block's was the carry's initial value)
   float he_part = 0.f;
   if (has_dhe) {
     const float *he = p.states + ((static_cast<int64_t>(b) * K + k) * H + h) * PN;
+    const float *ds = p.dstates && k + 1 < K ? p.dstates + ((static_cast<int64_t>(b) * K + k) * H + h) * PN : nullptr;
     if ((N & 3) == 0) {
       const int cn4 = N >> 2;
 #pragma unroll 4
       for (int e = tid; e < static_cast<int>(PN >> 2); e += kBwdThreads) {
         const int row = e / cn4, c4 = (e - row * cn4) << 2;
         const float4 hv = reinterpret_cast<const float4 *>(he)[e];
-        const float4 cv = *reinterpret_cast<const float4 *>(s.carry + row * NS + c4);
+        float4 *cp = reinterpret_cast<float4 *>(s.carry + row * NS + c4);
+        float4 cv = *cp;
+        if (ds) {
+          const float4 dv = reinterpret_cast<const float4 *>(ds)[e];
+          cv.x += dv.x; cv.y += dv.y; cv.z += dv.z; cv.w += dv.w;
+          *cp = cv;
+        }
         he_part += hv.x * cv.x + hv.y * cv.y + hv.z * cv.z + hv.w * cv.w;
       }
     } else {
 #pragma unroll 8
-      for (int64_t e = tid; e < PN; e += kBwdThreads) he_part += s.carry[(e / N) * NS + e % N] * he[e];
+      for (int64_t e = tid; e < PN; e += kBwdThreads) {
+        float &c = s.carry[(e / N) * NS + e % N];
+        if (ds) c += ds[e];
+        he_part += c * he[e];
+      }
     }
   }
   __syncthreads();
@@ -659,12 +671,7 @@ __global__ void __launch_bounds__(kBwdThreads) bd_bwd_kernel(const __grid_consta
     bwd_block(p, s, 2, b, h, k, accA[2], accD[2]);
     if (!p.rev_split && p.active[1]) bwd_block(p, s, 1, b, h, k, accA[1], accD[1]);
     if (!p.rev_split && p.active[3]) bwd_block(p, s, 3, b, h, k, accA[3], accD[3]);
-    if (k > 0 && p.dstates) {
-#pragma unroll 8
-      for (int64_t e = threadIdx.x; e < PN; e += kBwdThreads)
-        s.carry[(e / N) * NS + e % N] += p.dstates[((static_cast<int64_t>(b) * K + (k - 1)) * H + h) * PN + e];
-      __syncthreads();
-    }
+    // (dL/dstates[k - 1] joins the carried gradient in the next clean block's loads)
   }
   if (p.dh0)
     for (int64_t e = threadIdx.x; e < PN; e += kBwdThreads)
