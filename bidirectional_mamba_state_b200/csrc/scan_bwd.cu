@@ -25,13 +25,15 @@
 // (given) plus dh_s of clean block k+1 plus dh_s of noisy block k+1 (which
 // starts from states[k]); dh_s of clean block 0 and of noisy block 0 is dh0.
 //
-// One CTA of 512 threads per (b, h) walks the blocks from last to first; all
+// One CTA of 512 threads per (b, h) walks the forward chain's blocks (clean
+// and noisy) from last to first; the reverse directions' blocks, which carry
+// nothing, run in CTAs of their own after those, a range of blocks each.  All
 // block quantities live in shared memory (with transposed copies where the
-// threads run over tokens), the products are register-tiled (4 x 4 per
-// thread), fp32 arithmetic on CUDA cores.  dB
-// and dC of a group and dA, dD of a head are sums over heads / batch rows:
-// each CTA writes its own partials to the workspace and a second kernel sums
-// them in a fixed order, so the result is deterministic.
+// threads run over tokens), the products are register-tiled (TM x 4 per
+// thread), fp32 arithmetic on CUDA cores.  dB and dC of a group and dA, dD of
+// a head are sums over heads / batch rows (and reverse ranges): each CTA
+// writes its own partials to the workspace and a second kernel sums them in a
+// fixed order, so the result is deterministic.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
