@@ -603,7 +603,21 @@ def _backward(s: W.Shape, dev, pk) -> dict:
             "roofline": {"bound": "alu", "achieved": tf, "peak": alu_peak, "unit": "TFLOP/s",
                          "frac": tf / alu_peak, "algorithmic_flops": flops,
                          "algorithmic_bytes": bytes_,
-                         "hbm_frac": bytes_ / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}}
+                         "hbm_frac": bytes_ / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]},
+            "cpu_baseline": _backward_oracle_rate(s, (cf, cr, nf, nr), dyn, dyc)}
+
+
+def _backward_oracle_rate(s: W.Shape, dirs, dyn, dyc) -> dict:
+    """The oracle's backward on the first batch row of the same inputs and output
+    gradients (all heads, all tokens, four directions), timed on the host cores."""
+    import oracle
+    one = s.with_(batch=1)
+    hs = [_host({k: (v if k in ("A", "D") else v[:1]) for k, v in d.items()}) for d in dirs]
+    hdyn, hdyc = dyn[:1].to("cpu"), dyc[:1].to("cpu")
+    return _oracle_rate(lambda: oracle.allblock_backward(one.as_dict(), *hs, dy_clean=hdyc, dy_noisy=hdyn),
+                        one.seqlen, "tokens/s",
+                        f"oracle allblock_backward on 1 of {s.batch} batch rows, all {s.nheads} heads, "
+                        f"all {s.seqlen} tokens, loss on y_clean and y_noisy")
 
 
 def _oracle_rate(call, units: float, unit: str, sample: str, target_s: float = 3.0) -> dict:
