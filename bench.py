@@ -564,7 +564,17 @@ def _norm(s: W.Shape, dev, pk) -> dict:
     achieved = b / (ms * 1e-3) / 1e9
     return {"us_per_call": ms * 1e3, "tokens_per_s": s.batch * s.seqlen / (ms * 1e-3),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / pk["hbm_gbs"], "algorithmic_bytes": b}}
+                         "frac": achieved / pk["hbm_gbs"], "algorithmic_bytes": b},
+            "cpu_baseline": _norm_oracle_rate(s, yn, z, w)}
+
+
+def _norm_oracle_rate(s: W.Shape, yn, z, w) -> dict:
+    """The oracle's gated RMSNorm on the first batch row, timed on the host cores."""
+    import oracle
+    hy, hz, hw = yn[:1].to("cpu"), z[:1].to("cpu"), w.to("cpu")
+    return _oracle_rate(lambda: oracle.gated_rmsnorm(hy, hz, hw, 1, 1e-5), s.seqlen, "tokens/s",
+                        f"oracle gated_rmsnorm on 1 of {s.batch} batch rows ({s.seqlen} tokens x "
+                        f"{s.nheads * s.headdim} channels)")
 
 
 def _conv_allblock(s: W.Shape, width: int, dev, pk) -> dict:
@@ -578,7 +588,19 @@ def _conv_allblock(s: W.Shape, width: int, dev, pk) -> dict:
     return {"us_per_call": ms * 1e3, "tokens_per_s": s.batch * s.seqlen / (ms * 1e-3), "width": width,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "algorithmic_bytes": b,
-                         "algorithmic_flops": RL.conv_flops(s, width, 4)}}
+                         "algorithmic_flops": RL.conv_flops(s, width, 4)},
+            "cpu_baseline": _conv_oracle_rate(s, width, dirs)}
+
+
+def _conv_oracle_rate(s: W.Shape, width: int, dirs) -> dict:
+    """The oracle's all-block convolution (four directions) on the first batch
+    row, timed on the host cores."""
+    import oracle
+    one = s.with_(batch=1)
+    hd = [_host({k: (v if k in ("weight", "bias") else v[:1]) for k, v in d.items()}) for d in dirs]
+    return _oracle_rate(lambda: oracle.conv_allblock(one.as_dict(), width, True, *hd), one.seqlen, "tokens/s",
+                        f"oracle conv_allblock (width {width}, four directions) on 1 of {s.batch} batch rows, "
+                        f"all {s.seqlen} tokens")
 
 
 def _backward(s: W.Shape, dev, pk) -> dict:
