@@ -565,7 +565,16 @@ def _norm(s: W.Shape, dev, pk) -> dict:
     return {"us_per_call": ms * 1e3, "tokens_per_s": s.batch * s.seqlen / (ms * 1e-3),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "algorithmic_bytes": b},
-            "cpu_baseline": _norm_oracle_rate(s, yn, z, w)}
+            "cpu_baseline": _guarded(_norm_oracle_rate, s, yn, z, w)}
+
+
+def _guarded(fn, *args) -> dict:
+    """A secondary line's oracle rate; a failure there is reported in the line
+    instead of ending the remaining lines."""
+    try:
+        return fn(*args)
+    except Exception as e:  # report, never hide
+        return {"kind": "oracle", "error": repr(e)}
 
 
 def _norm_oracle_rate(s: W.Shape, yn, z, w) -> dict:
@@ -589,7 +598,7 @@ def _conv_allblock(s: W.Shape, width: int, dev, pk) -> dict:
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "algorithmic_bytes": b,
                          "algorithmic_flops": RL.conv_flops(s, width, 4)},
-            "cpu_baseline": _conv_oracle_rate(s, width, dirs)}
+            "cpu_baseline": _guarded(_conv_oracle_rate, s, width, dirs)}
 
 
 def _conv_oracle_rate(s: W.Shape, width: int, dirs) -> dict:
@@ -626,7 +635,7 @@ def _backward(s: W.Shape, dev, pk) -> dict:
                          "frac": tf / alu_peak, "algorithmic_flops": flops,
                          "algorithmic_bytes": bytes_,
                          "hbm_frac": bytes_ / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]},
-            "cpu_baseline": _backward_oracle_rate(s, (cf, cr, nf, nr), dyn, dyc)}
+            "cpu_baseline": _guarded(_backward_oracle_rate, s, (cf, cr, nf, nr), dyn, dyc)}
 
 
 def _backward_oracle_rate(s: W.Shape, dirs, dyn, dyc) -> dict:
